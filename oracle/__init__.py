@@ -1,0 +1,146 @@
+"""CPU oracle for C = ReLU(A . B) (fp16 in, fp32 accumulate, fp16 out).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
+CPU-baseline leg import this package.  The product library never loads it and
+has no fallback to it.  It shares no code with the CUDA path.
+
+The arithmetic lives in ``oracle.c`` (plain C, compiled with gcc at -O2 and
+no fast-math, fp contraction off).  This module only builds that file and
+marshals numpy arrays through ctypes.
+
+What it follows: the quick-start ``matmul_relu`` kernel on the "TileLang"
+wiki page, section "Programming model": fp16 A (M x K) and B (K x N), an fp32
+accumulator cleared to zero, a K loop of tile products, ``max(C_local, 0)`` on
+the fp32 values and a copy into the fp16 output C (M x N).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+
+_lib = None
+_lock = threading.Lock()
+
+CFLAGS = ["-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC",
+          "-shared", "-std=c11", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``_build/liboracle.so`` (if stale) and return its path."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def compile_variant(src_text: str, out_path: str) -> str:
+    """Compile an alternative oracle source (used by the pin-strength tests)."""
+    src_path = out_path + ".c"
+    with open(src_path, "w") as f:
+        f.write(src_text)
+    subprocess.run(["gcc", *CFLAGS, src_path, "-o", out_path, "-lm"], check=True)
+    return out_path
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _bind(lib):
+    u16p = ctypes.POINTER(ctypes.c_uint16)
+    f32p = ctypes.POINTER(ctypes.c_float)
+    i64 = ctypes.c_int64
+    lib.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
+    lib.oracle_f16_to_f32.restype = ctypes.c_float
+    lib.oracle_f32_to_f16_rne.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_f16_rne.restype = ctypes.c_uint16
+    lib.oracle_f16_to_f32_array.argtypes = [u16p, f32p, i64]
+    lib.oracle_f16_to_f32_array.restype = None
+    lib.oracle_f32_to_f16_rne_array.argtypes = [f32p, u16p, i64]
+    lib.oracle_f32_to_f16_rne_array.restype = None
+    lib.oracle_gemm_relu_f16.argtypes = [u16p, u16p, u16p, i64, i64, i64, ctypes.c_int]
+    lib.oracle_gemm_relu_f16.restype = ctypes.c_int
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
+def load_library(path: str | None = None):
+    """Load (building first if needed) the oracle library; ``path`` loads a variant."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _u16(a: np.ndarray) -> np.ndarray:
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected float16 or uint16 bit patterns, got {a.dtype}")
+    return np.ascontiguousarray(a)
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def f16_bits_to_f32(h: np.ndarray, lib=None) -> np.ndarray:
+    lib = lib or load_library()
+    h = _u16(np.asarray(h))
+    out = np.empty(h.shape, dtype=np.float32)
+    lib.oracle_f16_to_f32_array(_ptr(h, ctypes.c_uint16), _ptr(out, ctypes.c_float), h.size)
+    return out
+
+
+def f32_to_f16_bits(x: np.ndarray, lib=None) -> np.ndarray:
+    lib = lib or load_library()
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib.oracle_f32_to_f16_rne_array(_ptr(x, ctypes.c_float), _ptr(out, ctypes.c_uint16), x.size)
+    return out
+
+
+def gemm_relu_f16(A: np.ndarray, B: np.ndarray, nthreads: int = 0, lib=None) -> np.ndarray:
+    """C = f16_rne(relu(A . B)) with sequential fp32 accumulation; returns float16 (M, N)."""
+    lib = lib or load_library()
+    A = _u16(np.asarray(A))
+    B = _u16(np.asarray(B))
+    if A.ndim != 2 or B.ndim != 2 or A.shape[1] != B.shape[0]:
+        raise ValueError(f"shape mismatch: A{A.shape} B{B.shape}")
+    M, K = A.shape
+    N = B.shape[1]
+    C = np.empty((M, N), dtype=np.uint16)
+    rc = lib.oracle_gemm_relu_f16(_ptr(A, ctypes.c_uint16), _ptr(B, ctypes.c_uint16),
+                                  _ptr(C, ctypes.c_uint16), M, N, K, int(nthreads))
+    if rc != 0:
+        raise MemoryError("oracle could not allocate its work buffers")
+    return C.view(np.float16)
+
+
+def gemm_relu_f16_rows(A: np.ndarray, B: np.ndarray, rows, nthreads: int = 0, lib=None) -> np.ndarray:
+    """Rows ``rows`` of the oracle result: the same definition applied to A[rows, :]."""
+    rows = np.asarray(rows, dtype=np.int64)
+    return gemm_relu_f16(np.ascontiguousarray(A[rows, :]), B, nthreads=nthreads, lib=lib)
+
+
+def max_threads(lib=None) -> int:
+    lib = lib or load_library()
+    return int(lib.oracle_max_threads())

@@ -1,0 +1,210 @@
+/*
+ * oracle.c -- CPU oracle for C = ReLU(A . B) with fp16 operands, fp32
+ * accumulation and an fp16 result.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, includes
+ * or calls this file.  Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark load it.  It shares no code, header, table or
+ * helper with the CUDA path.
+ *
+ * What it computes (the quick-start matmul_relu kernel, "TileLang" wiki page,
+ * section "Programming model"):
+ *   - A is an M x K fp16 tensor and B is a K x N fp16 tensor; C is a fresh
+ *     M x N fp16 tensor (the kernel's tensor declarations).  All three are
+ *     dense and row-major: element (r, c) of an R x S matrix sits at r*S + c.
+ *   - The accumulator is an fp32 fragment (alloc_fragment of float32) that is
+ *     cleared to zero (T.clear) before the K loop.
+ *   - The K loop walks ceildiv(K, block_K) tiles and accumulates the tile
+ *     products (T.gemm).  Tiling only partitions the sum, so the plain
+ *     definition is the full sum over k = 0 .. K-1.
+ *   - The epilogue takes max(C_local, 0) on the fp32 values, then T.copy
+ *     writes them into the fp16 output, which converts fp32 -> fp16.
+ *
+ * Readings where the page is silent (each one is listed in the design notes):
+ *   - Accumulation is IEEE fp32, sequential in k = 0, 1, ..., K-1, with
+ *     round-to-nearest-even at every add.  Every fp16 x fp16 product is exact
+ *     in fp32 (11-bit x 11-bit significands need at most 22 bits), so the
+ *     only rounding in the loop is in the adds, and a fused multiply-add would
+ *     give the same bits.
+ *   - The fp32 -> fp16 conversion is IEEE 754 round-to-nearest, ties to even,
+ *     with gradual underflow and overflow to +inf.
+ *   - ReLU maps every value that is not > 0 (negative values, -0 and NaN) to
+ *     +0, so the output never carries the bit pattern 0x8000.
+ *
+ * Parity pins: every function here is pinned by tests that do not run this
+ * code's arithmetic a second time (numpy's independent float16 conversion on
+ * all 65536 halves and on random and edge fp32 values, hand-derived IEEE 754
+ * edge values, exact integer matrix products, exact rational sums with the
+ * standard fp32 summation error bound, and closed forms such as identity and
+ * all-ones matrices).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/*
+ * binary16 -> binary32, from the IEEE 754 binary16 definition:
+ *   exponent field 0      : value = (-1)^s * frac * 2^-24   (zero, subnormal)
+ *   exponent field 1..30  : value = (-1)^s * (1024 + frac) * 2^(e - 25)
+ *   exponent field 31     : +-inf (frac == 0) or NaN
+ * ldexpf of an integer below 2^11 is exact.
+ */
+float oracle_f16_to_f32(uint16_t h)
+{
+    const int sign = (h >> 15) & 1;
+    const int expo = (h >> 10) & 0x1f;
+    const int frac = h & 0x3ff;
+    float mag;
+    if (expo == 0)
+        mag = ldexpf((float)frac, -24);
+    else if (expo == 31)
+        mag = frac ? NAN : INFINITY;
+    else
+        mag = ldexpf((float)(1024 + frac), expo - 25);
+    return sign ? -mag : mag;
+}
+
+/*
+ * binary32 -> binary16, round to nearest, ties to even.
+ * The value's fp16 quantum is 2^(e-10) for |x| in [2^e, 2^(e+1)), e >= -14,
+ * and 2^-24 below 2^-14.  |x| / quantum is computed exactly in double (a
+ * float has 24 significant bits), rounded to an integer q with ties to even,
+ * and q * quantum is encoded.  A value that rounds to 2^16 or above is out of
+ * range and becomes inf.
+ */
+uint16_t oracle_f32_to_f16_rne(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, sizeof u);
+    const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    if (isnan(x))
+        return (uint16_t)(sign | 0x7e00u);
+    const double a = fabs((double)x);
+    if (isinf(x))
+        return (uint16_t)(sign | 0x7c00u);
+    if (a == 0.0)
+        return sign;
+
+    int e2;
+    (void)frexp(a, &e2); /* a = m * 2^e2 with m in [0.5, 1): 2^(e2-1) <= a */
+    int e = e2 - 1;      /* a in [2^e, 2^(e+1)) */
+    const int subnormal = e < -14;
+    const int qexp = subnormal ? -24 : e - 10; /* quantum = 2^qexp */
+
+    const double q = ldexp(a, -qexp); /* exact */
+    double qi = floor(q);
+    const double r = q - qi; /* exact */
+    if (r > 0.5 || (r == 0.5 && fmod(qi, 2.0) != 0.0))
+        qi += 1.0;
+    long qn = (long)qi;
+
+    if (subnormal) {
+        /* qn in [0, 1024]; 1024 is the smallest normal, 2^-14. */
+        if (qn == 1024)
+            return (uint16_t)(sign | (1u << 10));
+        return (uint16_t)(sign | (uint16_t)qn);
+    }
+    /* qn in [1024, 2048]; 2048 carries into the next binade. */
+    if (qn == 2048) {
+        qn = 1024;
+        e += 1;
+    }
+    if (e > 15)
+        return (uint16_t)(sign | 0x7c00u);
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)(qn - 1024));
+}
+
+/* Element-wise helpers over arrays, for the tests. */
+void oracle_f16_to_f32_array(const uint16_t *h, float *f, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        f[i] = oracle_f16_to_f32(h[i]);
+}
+
+void oracle_f32_to_f16_rne_array(const float *f, uint16_t *h, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        h[i] = oracle_f32_to_f16_rne(f[i]);
+}
+
+/*
+ * C[i, j] = f16_rne( relu( sum_{k=0}^{K-1} f32(A[i, k]) * f32(B[k, j]) ) )
+ *
+ * A: M x K, B: K x N, C: M x N, all row-major fp16 bit patterns.
+ * The sum for each (i, j) runs in k order with an fp32 accumulator.  The
+ * loop nest is i, k, j: a row of accumulators acc[0..N) is cleared, then for
+ * each k the row acc += A[i,k] * B[k, :] is added; the order of the adds into
+ * any one acc[j] is still k = 0, 1, ..., K-1.  Rows i are independent, so
+ * splitting them over threads changes no rounding.
+ *
+ * nthreads <= 0 means "whatever OpenMP picks".  Returns 0 on success and -1
+ * if a work buffer cannot be allocated.
+ */
+int oracle_gemm_relu_f16(const uint16_t *A, const uint16_t *B, uint16_t *C,
+                         int64_t M, int64_t N, int64_t K, int nthreads)
+{
+    if (M <= 0 || N <= 0)
+        return 0;
+
+    /* Widen B once: B[k, j] -> Bf[k*N + j]. */
+    float *Bf = NULL;
+    if (K > 0) {
+        Bf = (float *)malloc((size_t)K * (size_t)N * sizeof(float));
+        if (!Bf)
+            return -1;
+        oracle_f16_to_f32_array(B, Bf, K * N);
+    }
+
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        float *acc = (float *)malloc((size_t)N * sizeof(float));
+        if (!acc) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            failed = 1;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int64_t i = 0; i < M; ++i) {
+            if (!acc)
+                continue;
+            for (int64_t j = 0; j < N; ++j)
+                acc[j] = 0.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                const float a = oracle_f16_to_f32(A[i * K + k]);
+                const float *brow = Bf + k * N;
+                for (int64_t j = 0; j < N; ++j)
+                    acc[j] = acc[j] + a * brow[j];
+            }
+            for (int64_t j = 0; j < N; ++j) {
+                const float v = acc[j] > 0.0f ? acc[j] : 0.0f;
+                C[i * N + j] = oracle_f32_to_f16_rne(v);
+            }
+        }
+        free(acc);
+    }
+    free(Bf);
+    return failed ? -1 : 0;
+}
+
+/* Number of threads OpenMP would use by default (1 without OpenMP). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

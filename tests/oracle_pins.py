@@ -1,0 +1,298 @@
+"""Pins for the CPU oracle: checks against facts that do not come from the oracle.
+
+Each ``check_*`` function takes a loaded oracle library (the real one, or a
+deliberately broken variant in ``test_oracle_pin_strength.py``) and raises
+AssertionError when the oracle disagrees with:
+  * numpy's own float16 conversion (an independent implementation),
+  * IEEE 754 binary16 values derived by hand (``tests/golden/``),
+  * exact integer matrix products,
+  * exact rational sums and the standard error bound of recursive fp32
+    summation,
+  * closed forms (identity, all-ones, zero operands, overflow),
+  * the hand-worked examples of the matmul_relu quick-start kernel
+    ("TileLang" wiki page, "Programming model").
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import oracle
+from tiled_dense_gemm_fp16_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bits(a):
+    return np.asarray(a).view(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# fp16 <-> fp32 conversions
+# --------------------------------------------------------------------------
+
+def check_f16_to_f32_all_patterns(lib):
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.f16_bits_to_f32(h, lib=lib)
+    ref = h.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def load_f16_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "f16_rne_edges.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            tok = line.split()
+            x = float(tok[0]) if tok[0] in ("inf", "-inf") else float.fromhex(tok[0])
+            rows.append((x, int(tok[1], 16), " ".join(tok[2:])))
+    return rows
+
+
+def check_f32_to_f16_golden(lib):
+    rows = load_f16_golden()
+    assert len(rows) >= 20
+    x = np.array([r[0] for r in rows], dtype=np.float32)
+    # Every golden input is exactly representable in fp32.
+    assert all(float(xi) == r[0] for xi, r in zip(x, rows))
+    got = oracle.f32_to_f16_bits(x, lib=lib)
+    for g, (xv, want, why) in zip(got, rows):
+        assert int(g) == want, f"{xv!r}: got 0x{int(g):04x}, want 0x{want:04x} ({why})"
+
+
+def check_f32_to_f16_vs_numpy(lib, n=1 << 20, seed=123):
+    rng = np.random.default_rng(seed)
+    # Uniform random bit patterns: every exponent, NaNs and infinities.
+    u = rng.integers(0, 1 << 32, size=n, dtype=np.uint64).astype(np.uint32)
+    # Values concentrated on the fp16 range, subnormals included.
+    e = rng.integers(-30, 18, size=n)
+    v = (rng.uniform(1.0, 2.0, size=n) * np.exp2(e)) * rng.choice([-1.0, 1.0], size=n)
+    x = np.concatenate([u.view(np.float32), v.astype(np.float32)])
+    got = oracle.f32_to_f16_bits(x, lib=lib)
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16).view(np.uint16)
+    nan = np.isnan(x)
+    assert np.array_equal(got[~nan], ref[~nan])
+    gh = got[nan]
+    assert np.all((gh & 0x7C00) == 0x7C00) and np.all((gh & 0x03FF) != 0)
+
+
+def check_f32_to_f16_ties(lib):
+    """Midpoints of every pair of adjacent positive halves round to the even pattern.
+
+    For positive finite halves the bit pattern order is the value order, so the
+    two neighbours of the midpoint of patterns p and p+1 are p and p+1 and the
+    even one is whichever has a clear low bit.  The midpoint above 65504 is
+    65520 and ties to the even pattern 0x7c00, which is +inf.
+    """
+    p = np.arange(0, 0x7BFF, dtype=np.uint16)          # p and p+1 both finite
+    lo = p.view(np.float16).astype(np.float64)
+    hi = (p + 1).astype(np.uint16).view(np.float16).astype(np.float64)
+    mid = ((lo + hi) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (lo + hi) / 2)  # exact in fp32
+    want = np.where(p % 2 == 0, p, p + 1).astype(np.uint16)
+    got = oracle.f32_to_f16_bits(mid, lib=lib)
+    assert np.array_equal(got, want)
+    got_neg = oracle.f32_to_f16_bits(-mid, lib=lib)
+    assert np.array_equal(got_neg, want | 0x8000)
+    assert int(oracle.f32_to_f16_bits(np.array([65520.0], np.float32), lib=lib)[0]) == 0x7C00
+
+
+# --------------------------------------------------------------------------
+# GEMM + ReLU
+# --------------------------------------------------------------------------
+
+def load_worked_examples():
+    examples = []
+    cur = None
+    with open(os.path.join(GOLDEN, "gemm_worked_examples.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            tok = line.split()
+            if tok[0] == "example":
+                cur = {"id": int(tok[1])}
+                examples.append(cur)
+            elif tok[0] == "M":
+                cur["M"], cur["N"], cur["K"] = (int(t) for t in tok[3:6])
+            else:
+                cur[tok[0]] = [float(t) for t in tok[1:]]
+    return examples
+
+
+def check_worked_examples(lib):
+    ex = load_worked_examples()
+    assert len(ex) == 3
+    for e in ex:
+        M, N, K = e["M"], e["N"], e["K"]
+        A = np.array(e["A"], dtype=np.float16).reshape(M, K)
+        B = np.array(e["B"], dtype=np.float16).reshape(K, N)
+        want = np.array(e["C"], dtype=np.float16).reshape(M, N)
+        got = oracle.gemm_relu_f16(A, B, lib=lib)
+        assert np.array_equal(_bits(got), _bits(want)), f"example {e['id']}: {got} != {want}"
+
+
+def _exact_int_reference(A, B):
+    """ReLU of the exact integer product, rounded to fp16 by numpy."""
+    S = A.astype(np.int64) @ B.astype(np.int64)
+    R = np.maximum(S, 0).astype(np.float64)
+    with np.errstate(over="ignore"):
+        return R.astype(np.float16)
+
+
+def check_integer_exact(lib):
+    """Integer operands: every partial sum is an integer below 2^24, so fp32 is exact."""
+    rng = np.random.default_rng(7)
+    for (M, N, K) in [(7, 5, 13), (33, 17, 65), (64, 48, 300), (3, 129, 2500), (1, 1, 1)]:
+        A = rng.integers(-2, 3, size=(M, K)).astype(np.float16)
+        B = rng.integers(-2, 3, size=(K, N)).astype(np.float16)
+        got = oracle.gemm_relu_f16(A, B, lib=lib)
+        assert np.array_equal(_bits(got), _bits(_exact_int_reference(A, B))), (M, N, K)
+
+
+def check_all_ones(lib):
+    """All-ones operands: C = fp16(K); exactly K up to 2048, its nearest even half above."""
+    for K in (1, 2, 17, 255, 2048, 2049, 2051, 4097, 6001):
+        A = np.ones((3, K), np.float16)
+        B = np.ones((K, 5), np.float16)
+        got = oracle.gemm_relu_f16(A, B, lib=lib)
+        if K <= 2048:
+            want = float(K)
+        else:
+            # quantum 2 in [2048, 4096), 4 in [4096, 8192); ties to even patterns
+            q = 2 if K < 4096 else 4
+            lo = (K // q) * q
+            r = K - lo
+            up = r * 2 > q or (r * 2 == q and (lo // q) % 2 == 1)
+            want = float(lo + q if up else lo)
+        assert np.all(got.astype(np.float64) == want), (K, got[0, 0], want)
+
+
+def check_overflow(lib):
+    """Products of 2 * 2 summed K times: 4K; 65504 is finite, 65520 and above is +inf."""
+    for K, want in [(16376, 0x7BFF), (16379, 0x7BFF), (16380, 0x7C00), (20000, 0x7C00)]:
+        A = np.full((1, K), 2.0, np.float16)
+        B = np.full((K, 2), 2.0, np.float16)
+        got = oracle.gemm_relu_f16(A, B, lib=lib)
+        assert np.all(_bits(got) == want), (K, hex(int(_bits(got)[0, 0])))
+
+
+def check_identity(lib):
+    """A = I gives ReLU(B) bit for bit, with +0 for every non-positive entry."""
+    rng = np.random.default_rng(11)
+    K, N = 96, 70
+    B = rng.uniform(-3, 3, size=(K, N)).astype(np.float16)
+    B[0, :8] = np.array([0.0, -0.0, 6e-8, -6e-8, 1e-5, 65504, -65504, 2.0**-24], np.float16)
+    A = np.eye(K, dtype=np.float16)
+    got = oracle.gemm_relu_f16(A, B, lib=lib)
+    want = np.where(B.astype(np.float32) > 0, B, np.float16(0.0)).astype(np.float16)
+    assert np.array_equal(_bits(got), _bits(want))
+    # Transposed roles on a non-square right operand: B = I gives ReLU(A).
+    A2 = rng.uniform(-3, 3, size=(40, K)).astype(np.float16)
+    got2 = oracle.gemm_relu_f16(A2, np.eye(K, dtype=np.float16), lib=lib)
+    want2 = np.where(A2.astype(np.float32) > 0, A2, np.float16(0.0)).astype(np.float16)
+    assert np.array_equal(_bits(got2), _bits(want2))
+
+
+def check_zero_operands(lib):
+    rng = np.random.default_rng(5)
+    A = rng.uniform(-1, 1, size=(9, 31)).astype(np.float16)
+    B = rng.uniform(-1, 1, size=(31, 12)).astype(np.float16)
+    for a, b in [(np.zeros_like(A), B), (A, np.zeros_like(B)), (-np.zeros_like(A), B)]:
+        got = oracle.gemm_relu_f16(a, b, lib=lib)
+        assert np.all(_bits(got) == 0)
+    # K = 0: the empty sum is +0.
+    got = oracle.gemm_relu_f16(np.zeros((4, 0), np.float16), np.zeros((0, 6), np.float16), lib=lib)
+    assert got.shape == (4, 6) and np.all(_bits(got) == 0)
+
+
+def check_nonnegative(lib):
+    for dist in inputs.DISTRIBUTIONS:
+        A, B = inputs.operands(37, 53, 211, dist, seed=3)
+        got = oracle.gemm_relu_f16(A, B, lib=lib)
+        assert np.all((_bits(got) & 0x8000) == 0)
+        assert np.all(got.astype(np.float32) >= 0)
+
+
+def _f16_of_real(x: float, toward: str) -> float:
+    """fp16(x) of a real x, with x first pushed one double ulp outward."""
+    y = float(x)
+    y = math.nextafter(y, -math.inf) if toward == "down" else math.nextafter(y, math.inf)
+    with np.errstate(over="ignore"):
+        return float(np.float16(max(y, 0.0)))
+
+
+def check_exact_rational_bound(lib):
+    """|fp32 recursive sum - exact sum| <= gamma_{K-1} * sum |a_k b_k| (products exact).
+
+    The oracle's fp16 output must then lie between fp16(relu(S - E)) and
+    fp16(relu(S + E)), because ReLU and rounding to nearest are monotone.
+    """
+    u = Fraction(1, 1 << 24)
+    for (M, N, K), dist, seed in [((8, 8, 8), "uniform", 0), ((5, 3, 17), "normal01", 1),
+                                  ((4, 6, 257), "uniform", 2)]:
+        A, B = inputs.operands(M, N, K, dist, seed=seed)
+        got = oracle.gemm_relu_f16(A, B, lib=lib).astype(np.float64)
+        Af = [[Fraction(float(v)) for v in row] for row in A.astype(np.float64)]
+        Bf = [[Fraction(float(v)) for v in row] for row in B.astype(np.float64)]
+        gamma = (K - 1) * u / (1 - (K - 1) * u)
+        for i in range(M):
+            for j in range(N):
+                prods = [Af[i][k] * Bf[k][j] for k in range(K)]
+                S = sum(prods, Fraction(0))
+                E = gamma * sum(abs(p) for p in prods)
+                lo = _f16_of_real(S - E, "down")
+                hi = _f16_of_real(S + E, "up")
+                assert lo <= got[i, j] <= hi, (i, j, float(S), got[i, j], lo, hi)
+
+
+def check_sequential_fp32_tiny(lib):
+    """An independent fp32 scalar loop (numpy.float32 arithmetic) in k order agrees bit for bit."""
+    for (M, N, K), dist, seed in [((8, 8, 8), "uniform", 0), ((5, 3, 17), "normal01", 4),
+                                  ((2, 7, 64), "uniform", 9)]:
+        A, B = inputs.operands(M, N, K, dist, seed=seed)
+        got = oracle.gemm_relu_f16(A, B, lib=lib)
+        want = np.empty((M, N), np.float16)
+        for i in range(M):
+            for j in range(N):
+                s = np.float32(0.0)
+                for k in range(K):
+                    s = np.float32(s + np.float32(A[i, k]) * np.float32(B[k, j]))
+                want[i, j] = np.float16(s) if s > 0 else np.float16(0.0)
+        assert np.array_equal(_bits(got), _bits(want)), (M, N, K)
+
+
+def check_rows_and_threads(lib):
+    A, B = inputs.operands(67, 45, 129, "uniform", seed=8)
+    full = oracle.gemm_relu_f16(A, B, nthreads=1, lib=lib)
+    par = oracle.gemm_relu_f16(A, B, nthreads=4, lib=lib)
+    assert np.array_equal(_bits(full), _bits(par))
+    rows = [0, 5, 66, 31]
+    sub = oracle.gemm_relu_f16_rows(A, B, rows, lib=lib)
+    assert np.array_equal(_bits(sub), _bits(full[rows]))
+
+
+ALL_CHECKS = [
+    check_f16_to_f32_all_patterns,
+    check_f32_to_f16_golden,
+    check_f32_to_f16_vs_numpy,
+    check_f32_to_f16_ties,
+    check_worked_examples,
+    check_integer_exact,
+    check_all_ones,
+    check_overflow,
+    check_identity,
+    check_zero_operands,
+    check_nonnegative,
+    check_exact_rational_bound,
+    check_sequential_fp32_tiny,
+    check_rows_and_threads,
+]

@@ -1,0 +1,41 @@
+"""The pins are strong enough: plausible mistakes planted in a copy of the
+oracle (compiled on the CPU, never run on a GPU) each fail at least one pin."""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_CHECKS
+
+# (name, text in oracle.c, replacement): each is a mistake someone could make.
+# "ReLU keeps -0" (">= 0" in place of "> 0") is not listed: a sum that starts
+# at +0 and rounds to nearest can never be -0 (x + (-x) is +0), so that change
+# computes the same function.
+MUTANTS = [
+    ("transposed_B", "acc[j] = acc[j] + a * brow[j];", "acc[j] = acc[j] + a * Bf[j * K + k];"),
+    ("transposed_A", "oracle_f16_to_f32(A[i * K + k])", "oracle_f16_to_f32(A[k * M + i])"),
+    ("dropped_last_k", "for (int64_t k = 0; k < K; ++k) {", "for (int64_t k = 0; k + 1 < K; ++k) {"),
+    ("relu_missing", "acc[j] > 0.0f ? acc[j] : 0.0f", "acc[j]"),
+    ("truncate_not_round", "if (r > 0.5 || (r == 0.5 && fmod(qi, 2.0) != 0.0))", "if (0)"),
+    ("ties_away_from_zero", "(r == 0.5 && fmod(qi, 2.0) != 0.0)", "(r == 0.5)"),
+    ("wrong_subnormal_quantum", "subnormal ? -24 : e - 10", "subnormal ? -25 : e - 10"),
+    ("wrong_f16_bias", "ldexpf((float)(1024 + frac), expo - 25)", "ldexpf((float)(1024 + frac), expo - 24)"),
+    ("no_overflow_to_inf", "if (e > 15)", "if (e > 16)"),
+    ("fp64_accumulator", "float *acc = (float *)malloc((size_t)N * sizeof(float));",
+     "double *acc = (double *)malloc((size_t)N * sizeof(double));"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(tmp_path, name, old, new):
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    lib = oracle.load_library(oracle.compile_variant(src.replace(old, new),
+                                                     os.path.join(tmp_path, f"lib{name}.so")))
+    failed = []
+    for check in ALL_CHECKS:
+        try:
+            check(lib)
+        except AssertionError:
+            failed.append(check.__name__)
+    assert failed, f"no pin catches the planted mistake {name}"
