@@ -1,0 +1,410 @@
+#!/usr/bin/env python3
+"""Benchmark of C = ReLU(A . B) (fp16 in, fp32 accumulate, fp16 out) on B200.
+
+One step = one full GEMM+ReLU over one problem whose operands are already
+resident in HBM.  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload square8192]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own
+independent problem (weak scaling, no data-path collective); the timed region
+is bracketed by barriers and the slowest rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from tiled_dense_gemm_fp16_b200 import inputs  # noqa: E402
+
+METRIC = "GEMM+ReLU TFLOP/s at 8192³ fp16 (1×B200) and % of dense FP16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Sources of the dominant kernel; the committed ncu traffic figure is only
+# reported while these are unchanged.
+KERNEL_SOURCES = ["tiled_dense_gemm_fp16_b200/csrc/gemm_tc.cuh", "tiled_dense_gemm_fp16_b200/csrc/ptx.cuh"]
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "gemm_relu_tc_square8192.md")
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="square8192",
+                    help="square8192 (the metric's workload), square4096, square256, skinny:<M>, ragged:<i>")
+    ap.add_argument("--path", default="auto", help="force a kernel path: auto, tc, tc_edge, skinny, gemv")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# Workload
+# ---------------------------------------------------------------------------
+
+def workload_problem(spec: str, rank: int = 0):
+    """(name, M, N, K, A, B) for a workload spec; ranks > 0 draw their own problem."""
+    name, _, sub = spec.partition(":")
+    wl = inputs.WORKLOADS[name]
+    problems = list(wl.shapes)
+    idx = 0
+    if name == "skinny":
+        ms = [s[0] for s in problems]
+        idx = ms.index(int(sub)) if sub else len(ms) - 1
+    elif name == "ragged":
+        idx = int(sub) if sub else 0
+    M, N, K = problems[idx]
+    if rank == 0:
+        # Exactly the workload's own draw (the generator is advanced over earlier shapes).
+        for i, ((m, n, k), A, B) in enumerate(wl.problems()):
+            if i == idx:
+                return f"{name}" + (f":{sub}" if sub else ""), m, n, k, A, B
+    A, B = inputs.operands(M, N, K, wl.dist, seed=wl.seed * 1000 + rank)
+    return f"{name}" + (f":{sub}" if sub else ""), M, N, K, A, B
+
+
+def describe(name, M, N, K):
+    wl = inputs.WORKLOADS[name.partition(":")[0]]
+    return {"workload": name, "M": M, "N": N, "K": K, "dtype_in": "fp16", "accumulate": "fp32",
+            "dtype_out": "fp16", "layout": "row-major A, B, C", "values": wl.dist, "seed": wl.seed}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling (NVML) during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.nvml = None
+            self.error = str(e)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# ncu traffic figure (committed summary), valid only for unchanged sources
+# ---------------------------------------------------------------------------
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    if not os.path.exists(TRAFFIC_SUMMARY):
+        return None
+    text = open(TRAFFIC_SUMMARY).read()
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    m_wl = re.search(r"traffic_workload:\s*(\S+)", text)
+    m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_b and m_wl) or m_sha.group(1) != kernel_source_sha() or m_wl.group(1) != workload:
+        return None
+    return float(m_b.group(1))
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample of rows
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(A, B, target_s: float):
+    import oracle
+    cores = os.cpu_count() or 1
+    M, K = A.shape
+    N = B.shape[1]
+    # Calibrate on a few rows, then size the sample to about target_s seconds.
+    probe = max(1, min(M, cores))
+    t0 = time.perf_counter()
+    oracle.gemm_relu_f16_rows(A, B, np.arange(probe), nthreads=cores)
+    t_probe = time.perf_counter() - t0
+    rows = int(max(probe, min(M, probe * target_s / max(t_probe, 1e-3))))
+    rows = max(cores, (rows // cores) * cores) if rows >= cores else rows
+    rows = min(rows, M)
+    sel = np.arange(rows)
+    t0 = time.perf_counter()
+    oracle.gemm_relu_f16_rows(A, B, sel, nthreads=cores)
+    dt = time.perf_counter() - t0
+    flops = inputs.flops(rows, N, K)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(oracle.max_threads() if cores <= 0 else cores),
+            "kind": "oracle", "sample": f"rows 0..{rows - 1} of C ({rows} x {N} x {K}); {dt:.1f} s on {cores} threads",
+            "seconds": dt}
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the oracle on host cores, per step a bounded row sample
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    name, M, N, K, A, B = workload_problem(args.workload)
+    cores = os.cpu_count() or 1
+    # Each step computes `rows` rows of C; sized so that warmup + steps fit a few minutes.
+    probe = max(1, min(M, cores))
+    t0 = time.perf_counter()
+    oracle.gemm_relu_f16_rows(A, B, np.arange(probe), nthreads=cores)
+    t_probe = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(M, probe * budget / max(t_probe, 1e-3))))
+    sel = np.arange(rows)
+    for _ in range(args.warmup):
+        oracle.gemm_relu_f16_rows(A, B, sel, nthreads=cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.gemm_relu_f16_rows(A, B, sel, nthreads=cores)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = inputs.flops(rows, N, K) * args.steps / total / 1e12
+    sample = f"each step computes rows 0..{rows - 1} of C ({rows} x {N} x {K}) with the CPU oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32-accumulate f16",
+        "data": "synthetic", "config": describe(name, M, N, K),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    path = {"auto": tg.Path.AUTO, "tc": tg.Path.TC, "tc_edge": tg.Path.TC_EDGE, "skinny": tg.Path.SKINNY,
+            "gemv": tg.Path.GEMV}[args.path]
+    name, M, N, K, A, B = workload_problem(args.workload, rank)
+    flops = inputs.flops(M, N, K)
+
+    Ad = torch.from_numpy(A).to(dev)
+    Bd = torch.from_numpy(B).to(dev)
+    Cd = torch.empty((M, N), dtype=torch.float16, device=dev)
+    stream = torch.cuda.Stream(dev)
+    sh = stream.cuda_stream
+    chosen = tg.select_path(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K) if path == tg.Path.AUTO else path
+    ws = 2 * (M * K + K * N + M * N)
+    # Inputs smaller than L2 get an L2 flush (a write larger than L2) between timed steps.
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if ws <= L2_BYTES else None
+
+    def step():
+        st = tg.gemm_relu_f16_raw(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, sh, path)
+        if st != tg.Status.OK:
+            raise tg.TGError(st, "tg_gemm_relu_f16")
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            if flush is not None:
+                flush.fill_(1)
+            step()
+    torch.cuda.synchronize(dev)
+    st, word = tg.device_status()
+    if st != tg.Status.OK:
+        raise SystemExit(f"device error after warm-up: {tg.status_string(st)} 0x{word:x}")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    region0 = torch.cuda.Event(enable_timing=True)
+    region1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        region0.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(1)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        region1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    region_ms = region0.elapsed_time(region1)
+    kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kern_avg_ms = sum(kern_ms) / len(kern_ms)
+    # The step time excludes the L2 flush writes when there are any.
+    step_ms = kern_avg_ms if flush is not None else region_ms / args.steps
+    if dist is not None:
+        t = torch.tensor([step_ms, kern_avg_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, kern_avg_ms = float(t[0]), float(t[1])
+    st, word = tg.device_status()
+    if st != tg.Status.OK:
+        raise SystemExit(f"device error in timed region: {tg.status_string(st)} 0x{word:x}")
+
+    value = world * flops / (step_ms * 1e-3) / 1e12
+
+    # End to end through the C ABI from pinned host buffers: H2D of A and B,
+    # the call, D2H of C, every step.
+    Ah = torch.from_numpy(A).pin_memory()
+    Bh = torch.from_numpy(B).pin_memory()
+    Ch = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(args.e2e_steps + 1):
+            if i == 1:
+                e0.record(stream)
+            Ad.copy_(Ah, non_blocking=True)
+            Bd.copy_(Bh, non_blocking=True)
+            step()
+            Ch.copy_(Cd, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    if chosen in (tg.Path.TC, tg.Path.TC_EDGE) and name.startswith("square"):
+        bound, unit_r = "tensor", "TFLOP/s"
+        achieved = flops / (kern_avg_ms * 1e-3) / 1e12
+        peak = float(peaks["bf16_tflops"])
+        peak_note = f"{peak_src} cuBLAS bf16 burst peak (fp16 kind::f16 runs at the bf16 rate)"
+    else:
+        bound, unit_r = "hbm", "GB/s"
+        achieved = inputs.min_bytes(M, N, K) / (kern_avg_ms * 1e-3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        peak_note = f"{peak_src} STREAM-copy HBM bandwidth"
+    traffic = committed_traffic(name) if rank == 0 else None
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 (fp32 accumulate)", "data": "synthetic",
+        "config": {**describe(name, M, N, K), "path": tg.path_name(chosen),
+                   "l2": "inputs larger than L2" if flush is None else "L2 flushed between timed steps",
+                   "parallelism": f"dp{world} independent problems" if world > 1 else "1 GPU"},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit_r,
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
+                     "kernel_ms": kern_avg_ms},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * (M * K + K * N),
+                "d2h_bytes_per_step": 2 * M * N, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(A, B, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,136 @@
+/*
+ * tg_gemm.h -- C ABI of the B200 (sm_100a) tiled fp16 GEMM + ReLU library.
+ *
+ * The operation (the matmul_relu quick-start kernel, "TileLang" wiki page,
+ * section "Programming model"):
+ *
+ *     C[i, j] = fp16( max( sum_k fp32(A[i, k]) * fp32(B[k, j]), 0 ) )
+ *
+ * with A an M x K fp16 matrix, B a K x N fp16 matrix, an fp32 accumulator
+ * that starts at zero, ReLU applied to the fp32 value, and the result rounded
+ * to fp16 (round to nearest, ties to even; values >= 65520 become +inf).
+ * ReLU maps every value that is not > 0 (including -0 and NaN) to +0.  The
+ * order in which the tensor cores add the K products is not specified, so
+ * for non-integer inputs results agree with a sequential fp32 sum up to
+ * rounding; integer-valued inputs whose partial sums stay below 2^24 give
+ * bit-identical results.
+ *
+ * Layout: A, B and C are dense and row-major (leading dimensions K, N and N
+ * elements), fp16 (IEEE binary16), in device memory of the current CUDA
+ * device.  The caller owns all three buffers; the library never allocates,
+ * frees or retains device memory and keeps no pointer after a call returns.
+ *
+ * Threading and streams: calls are asynchronous on `stream` (a cudaStream_t
+ * passed as void*; NULL is the legacy default stream).  On TG_OK the work is
+ * enqueued; on any error nothing was enqueued.  The functions are
+ * thread-safe.
+ *
+ * Device: NVIDIA B200 class GPU, compute capability 10.0 (sm_100a).
+ */
+#ifndef TG_GEMM_H
+#define TG_GEMM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TG_API __attribute__((visibility("default")))
+#else
+#define TG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tg_status {
+    TG_OK = 0,
+    TG_ERR_INVALID_ARG = 1,        /* bad pointer, size, alignment or overlap    */
+    TG_ERR_UNSUPPORTED_DEVICE = 2, /* no device, or not compute capability 10.0 */
+    TG_ERR_LAUNCH = 3,             /* a kernel launch or CUDA call failed         */
+    TG_ERR_TIMEOUT = 4,            /* a bounded device-side wait ran out          */
+    TG_ERR_INTERNAL = 5            /* invariant broken inside the library         */
+} tg_status;
+
+/* Kernel paths.  TG_PATH_AUTO lets the dispatcher choose (see
+ * tg_select_path); the others force one kernel, for tests and tuning. */
+typedef enum tg_path {
+    TG_PATH_NONE = -1,   /* nothing to launch: M == 0 or N == 0            */
+    TG_PATH_AUTO = 0,
+    TG_PATH_TC = 1,      /* TMA + tcgen05 persistent kernel, 128x256 tiles;
+                            needs K % 8 == 0, N % 8 == 0 and 16-byte
+                            aligned A, B, C                                 */
+    TG_PATH_TC_EDGE = 2, /* same kernel, operands staged by predicated
+                            loads: any K, N and 2-byte alignment            */
+    TG_PATH_SKINNY = 3,  /* small-M split-K tcgen05 kernel (computes
+                            C^T = B^T A^T); same alignment needs as TC       */
+    TG_PATH_GEMV = 4,    /* CUDA-core kernel for M <= 8; same alignment
+                            needs as TC                                     */
+    TG_PATH_ZERO = 5     /* K == 0: C is filled with +0 (empty sum)         */
+} tg_path;
+
+/*
+ * C = ReLU(A . B).
+ *   A      device pointer, M x K fp16, row-major (may be NULL if M*K == 0)
+ *   B      device pointer, K x N fp16, row-major (may be NULL if K*N == 0)
+ *   C      device pointer, M x N fp16, row-major, written in full; must not
+ *          overlap A or B (may be NULL if M*N == 0)
+ *   M,N,K  sizes, each in [0, 2^31 - 1]
+ *   stream cudaStream_t as void*
+ * Returns TG_OK, or TG_ERR_INVALID_ARG (negative or too large size, NULL
+ * pointer with a non-empty matrix, pointer not 2-byte aligned, C overlapping
+ * A or B), TG_ERR_UNSUPPORTED_DEVICE or TG_ERR_LAUNCH.  M == 0 or N == 0 is
+ * TG_OK with nothing enqueued; K == 0 fills C with +0.
+ */
+TG_API tg_status tg_gemm_relu_f16(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                           void *stream);
+
+/*
+ * As tg_gemm_relu_f16, with the kernel path forced (a tg_path value).
+ * Forcing a path whose requirements the arguments do not meet returns
+ * TG_ERR_INVALID_ARG.  TG_PATH_AUTO behaves like tg_gemm_relu_f16.
+ */
+TG_API tg_status tg_gemm_relu_f16_path(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                                void *stream, int path);
+
+/*
+ * The path tg_gemm_relu_f16 would take for these arguments (a tg_path value;
+ * TG_PATH_NONE for an empty C), or -2 when the arguments are invalid.  Host
+ * logic only: makes no CUDA call and needs no GPU.
+ */
+TG_API int tg_select_path(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Whether `path` can run these arguments (1) or not (0).  Host logic only.
+ */
+TG_API int tg_path_supports(int path, const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Synchronizes the current device, then reads and clears the library's
+ * device-side error word.  Returns TG_OK, TG_ERR_TIMEOUT if a bounded wait
+ * inside a kernel gave up since the last call (the kernel then stopped early
+ * and its output is incomplete), or TG_ERR_LAUNCH if the device reported an
+ * error.  `detail` (may be NULL) receives the raw error word.
+ */
+TG_API tg_status tg_device_status(uint32_t *detail);
+
+/*
+ * Failure-detection self-test: launches one CTA on `stream` that waits on an
+ * mbarrier nothing will ever arrive on, with a budget of `budget_ns`
+ * nanoseconds (clamped to [1e3, 1e10]).  The wait gives up, records
+ * TG_ERR_TIMEOUT in the device error word and the kernel returns normally;
+ * tg_device_status() then reports it.  No trap, no fault, no hang.
+ */
+TG_API tg_status tg_wait_timeout_selftest(int64_t budget_ns, void *stream);
+
+/* Static description of a status or path value. */
+TG_API const char *tg_status_string(int status);
+TG_API const char *tg_path_name(int path);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+TG_API int tg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TG_GEMM_H */

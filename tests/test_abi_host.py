@@ -1,0 +1,105 @@
+"""C-ABI library: it loads, exports every function the headers declare, and its
+host-side argument logic (validation, path choice) behaves as documented.
+No kernel is launched: these run without a GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import tiled_dense_gemm_fp16_b200 as tg
+from tiled_dense_gemm_fp16_b200 import Path, Status
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# Well-separated fake device addresses (never dereferenced by host logic).
+A0, B0, C0 = 0x10_0000_0000, 0x20_0000_0000, 0x30_0000_0000
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"TG_API\s+[^;(]*?\b(tg_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = tg.lib()
+    names = declared_functions()
+    assert "tg_gemm_relu_f16" in names and len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+        assert isinstance(getattr(lib, n), ctypes._CFuncPtr)
+    assert set(tg.EXPORTS) <= set(names)
+
+
+def test_version_and_strings():
+    assert tg.version() >= 100
+    assert tg.status_string(Status.OK) == "ok"
+    assert "invalid" in tg.status_string(Status.INVALID_ARG)
+    assert tg.path_name(Path.TC) == "tc" and tg.path_name(Path.TC_EDGE) == "tc_edge"
+    assert tg.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("M,N,K", [(-1, 4, 4), (4, -1, 4), (4, 4, -1), (2**31, 8, 8), (8, 2**31, 8), (8, 8, 2**31)])
+def test_invalid_sizes(M, N, K):
+    assert tg.select_path(A0, B0, C0, M, N, K) == Path.INVALID
+    assert tg.gemm_relu_f16_raw(A0, B0, C0, M, N, K) == Status.INVALID_ARG
+
+
+def test_null_pointers():
+    assert tg.gemm_relu_f16_raw(0, B0, C0, 8, 8, 8) == Status.INVALID_ARG
+    assert tg.gemm_relu_f16_raw(A0, 0, C0, 8, 8, 8) == Status.INVALID_ARG
+    assert tg.gemm_relu_f16_raw(A0, B0, 0, 8, 8, 8) == Status.INVALID_ARG
+    # Empty C: nothing to do, pointers may be NULL, no CUDA call is made.
+    assert tg.gemm_relu_f16_raw(0, 0, 0, 0, 8, 8) == Status.OK
+    assert tg.gemm_relu_f16_raw(0, 0, 0, 8, 0, 8) == Status.OK
+    assert tg.select_path(0, 0, 0, 0, 0, 0) == Path.NONE
+
+
+def test_odd_pointer_rejected():
+    assert tg.gemm_relu_f16_raw(A0 + 1, B0, C0, 8, 8, 8) == Status.INVALID_ARG
+    assert tg.gemm_relu_f16_raw(A0, B0, C0 + 1, 8, 8, 8) == Status.INVALID_ARG
+
+
+def test_overlap_rejected():
+    M, N, K = 64, 64, 64
+    # C overlapping the last byte of A, or starting inside B.
+    assert tg.gemm_relu_f16_raw(A0, B0, A0 + 2 * M * K - 2, M, N, K) == Status.INVALID_ARG
+    assert tg.gemm_relu_f16_raw(A0, B0, B0 + 128, M, N, K) == Status.INVALID_ARG
+    # Adjacent but not overlapping is fine for the host logic.
+    assert tg.select_path(A0, B0, A0 + 2 * M * K, M, N, K) == Path.TC
+
+
+def test_path_selection():
+    assert tg.select_path(A0, B0, C0, 128, 128, 0) == Path.ZERO
+    assert tg.select_path(A0, B0, C0, 4096, 4096, 4096) == Path.TC
+    assert tg.select_path(A0, B0, C0, 8192, 8192, 8192) == Path.TC
+    # Row strides that are not 16-byte multiples, or misaligned bases, need the edge mode.
+    assert tg.select_path(A0, B0, C0, 3001, 5003, 1021) == Path.TC_EDGE
+    assert tg.select_path(A0, B0, C0, 777, 12289, 4095) == Path.TC_EDGE
+    assert tg.select_path(A0, B0, C0, 8191, 129, 8193) == Path.TC_EDGE
+    assert tg.select_path(A0 + 2, B0, C0, 256, 256, 256) == Path.TC_EDGE
+
+
+def test_forced_path_requirements():
+    assert tg.path_supports(Path.TC, A0, B0, C0, 256, 256, 256)
+    assert not tg.path_supports(Path.TC, A0, B0, C0, 256, 250, 256)
+    assert not tg.path_supports(Path.TC, A0, B0, C0, 256, 256, 250)
+    assert tg.path_supports(Path.TC_EDGE, A0, B0, C0, 256, 250, 250)
+    assert not tg.path_supports(Path.ZERO, A0, B0, C0, 256, 256, 256)
+    assert tg.path_supports(Path.ZERO, A0, B0, C0, 256, 256, 0)
+    assert not tg.path_supports(42, A0, B0, C0, 256, 256, 256)
+    assert tg.gemm_relu_f16_raw(A0, B0, C0, 256, 250, 256, 0, Path.TC) == Status.INVALID_ARG
+
+
+def test_no_device_is_reported_not_faked():
+    """Without a GPU a valid call reports the missing device; it never computes on the CPU."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert tg.gemm_relu_f16_raw(A0, B0, C0, 64, 64, 64) == Status.UNSUPPORTED_DEVICE
+    st, _ = tg.device_status()
+    assert st == Status.UNSUPPORTED_DEVICE

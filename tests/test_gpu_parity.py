@@ -1,0 +1,222 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bar: bit-exact on integer-valued inputs (values in {-2..2}: every partial sum
+is an integer below 2^24, so any summation order is exact), and
+|gpu - oracle| <= 1e-3 + 4e-3 * |oracle| elementwise on float inputs.
+Guard bands around C check that nothing outside C is written.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from gpu_util import assert_bitexact, assert_close, run_gpu, sample_rows
+from tiled_dense_gemm_fp16_b200 import inputs
+from tiled_dense_gemm_fp16_b200._binding import Path
+
+pytestmark = pytest.mark.gpu
+
+TC, EDGE = Path.TC, Path.TC_EDGE
+
+
+def _paths_for(M, N, K):
+    paths = [None, EDGE]
+    if N % 8 == 0 and K % 8 == 0:
+        paths.append(TC)
+    return paths
+
+
+# ---------------------------------------------------------------------------
+# Small square workload (256^3): integer variant bit-exact, uniform within tolerance
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("path", [None, TC, EDGE], ids=["auto", "tc", "edge"])
+def test_square256_integer_bitexact(path):
+    A, B = inputs.operands(256, 256, 256, "int", seed=0)
+    got, guards = run_gpu(A, B, path)
+    assert guards
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), "square256 int")
+
+
+@pytest.mark.parametrize("path", [None, TC, EDGE], ids=["auto", "tc", "edge"])
+def test_square256_uniform(path):
+    (shape, A, B), = inputs.WORKLOADS["square256"].problems()
+    got, guards = run_gpu(A, B, path)
+    assert guards
+    assert_close(got, oracle.gemm_relu_f16(A, B), "square256 uniform")
+
+
+# ---------------------------------------------------------------------------
+# Tile edges: sizes around the 128 x 256 x 64 tile, bit-exact on integer inputs
+# ---------------------------------------------------------------------------
+
+EDGE_SHAPES = [
+    (1, 1, 1), (1, 8, 8), (15, 17, 9), (16, 16, 16), (17, 33, 65), (127, 255, 63),
+    (128, 256, 64), (129, 257, 65), (255, 129, 127), (257, 513, 200), (300, 264, 136),
+    (128, 8, 1000), (8, 1000, 24), (640, 520, 72), (1000, 1000, 1000),
+]
+
+
+@pytest.mark.parametrize("M,N,K", EDGE_SHAPES)
+def test_tile_edges_integer_bitexact(M, N, K):
+    A, B = inputs.operands(M, N, K, "int", seed=M * 7 + N * 3 + K)
+    ref = oracle.gemm_relu_f16(A, B)
+    for path in _paths_for(M, N, K):
+        got, guards = run_gpu(A, B, path)
+        assert guards, (M, N, K, path)
+        assert_bitexact(got, ref, f"{(M, N, K)} path={path}")
+
+
+@pytest.mark.parametrize("M,N,K", [(129, 257, 65), (300, 264, 136), (1000, 1000, 1000)])
+def test_tile_edges_uniform(M, N, K):
+    A, B = inputs.operands(M, N, K, "uniform", seed=5)
+    ref = oracle.gemm_relu_f16(A, B)
+    for path in _paths_for(M, N, K):
+        got, guards = run_gpu(A, B, path)
+        assert guards
+        assert_close(got, ref, f"{(M, N, K)} path={path}")
+
+
+def test_misaligned_base_pointers_use_edge_mode():
+    """Bases 2 bytes off a 16-byte boundary: TMA cannot take them; the edge mode can."""
+    A, B = inputs.operands(200, 136, 72, "int", seed=2)
+    ref = oracle.gemm_relu_f16(A, B)
+    got, guards = run_gpu(A, B, None, offset_elems=1)
+    assert guards
+    assert_bitexact(got, ref, "offset 1")
+
+
+# ---------------------------------------------------------------------------
+# Degenerate sizes
+# ---------------------------------------------------------------------------
+
+def test_k_zero_fills_positive_zero():
+    A = np.zeros((37, 0), np.float16)
+    B = np.zeros((0, 53), np.float16)
+    got, guards = run_gpu(A, B)
+    assert guards
+    assert np.all(got.view(np.uint16) == 0)
+
+
+def test_empty_outputs_are_noops():
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    A = torch.zeros((0, 16), dtype=torch.float16, device="cuda")
+    B = torch.zeros((16, 8), dtype=torch.float16, device="cuda")
+    assert tg.gemm_relu(A, B).shape == (0, 8)
+    A = torch.zeros((8, 16), dtype=torch.float16, device="cuda")
+    B = torch.zeros((16, 0), dtype=torch.float16, device="cuda")
+    assert tg.gemm_relu(A, B).shape == (8, 0)
+
+
+def test_special_values():
+    """Overflow to +inf past 65504, and ReLU of all-negative tiles to +0."""
+    K = 16384
+    A = np.full((130, K), 2.0, np.float16)
+    B = np.full((K, 264), 2.0, np.float16)       # 4K = 65536 -> +inf
+    B[:, 8:16] = -2.0                             # -65536 -> ReLU -> +0
+    B[:4095, 16:24] = 0.0                         # 4 * 12289 = 49156 -> 49152 (nearest even half)
+    ref = oracle.gemm_relu_f16(A, B)
+    for path in (TC, EDGE):
+        got, _ = run_gpu(A, B, path)
+        assert_bitexact(got, ref, f"special path={path}")
+    assert np.all(np.isinf(ref[:, :8].astype(np.float32))) and np.all(ref[:, 8:16].view(np.uint16) == 0)
+
+
+def test_deterministic():
+    A, B = inputs.operands(513, 777, 300, "uniform", seed=9)
+    a, _ = run_gpu(A, B)
+    b, _ = run_gpu(A, B)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+def test_non_default_stream():
+    import torch
+    A, B = inputs.operands(256, 512, 128, "int", seed=3)
+    s = torch.cuda.Stream()
+    got, _ = run_gpu(A, B, stream=s)
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), "side stream")
+
+
+# ---------------------------------------------------------------------------
+# The five workloads at full size (sampled rows where the full oracle is slow)
+# ---------------------------------------------------------------------------
+
+def _check_workload(name, dist=None, exact=False, full_oracle_max_macs=5e9, paths=(None,)):
+    for (M, N, K), A, B in inputs.WORKLOADS[name].problems(dist):
+        full = M * N * K <= full_oracle_max_macs
+        rows = list(range(M)) if full else sample_rows(M, seed=M + N + K)
+        ref = oracle.gemm_relu_f16_rows(A, B, rows)
+        for path in paths:
+            got, guards = run_gpu(A, B, path)
+            assert guards, (name, M, N, K, path)
+            sub = got[rows]
+            what = f"{name} {(M, N, K)} path={path} dist={dist or inputs.WORKLOADS[name].dist}"
+            if exact:
+                assert_bitexact(sub, ref, what)
+            else:
+                assert_close(sub, ref, what)
+
+
+def test_workload_square4096():
+    _check_workload("square4096", paths=(None, EDGE))
+
+
+def test_workload_square4096_integer():
+    _check_workload("square4096", dist="int", exact=True)
+
+
+def test_workload_square8192():
+    _check_workload("square8192")
+
+
+def test_workload_square8192_integer():
+    _check_workload("square8192", dist="int", exact=True)
+
+
+def test_workload_skinny():
+    _check_workload("skinny", paths=(None, TC, EDGE))
+
+
+def test_workload_skinny_integer():
+    _check_workload("skinny", dist="int", exact=True, paths=(None, TC, EDGE))
+
+
+def test_workload_ragged():
+    _check_workload("ragged")
+
+
+def test_workload_ragged_integer():
+    _check_workload("ragged", dist="int", exact=True)
+
+
+# ---------------------------------------------------------------------------
+# Large indices: more than 2^31 elements in A (64-bit address arithmetic)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K", [32776, 32775], ids=["aligned", "odd_K"])
+def test_more_than_2_31_elements(K):
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    M, N = 65544, 136
+    assert M * K > 2**31
+    rng = np.random.default_rng(K)
+    dev = torch.device("cuda", 0)
+    # Only the checked rows carry seeded random values; every other row of A
+    # is all ones, and one of those rows is checked too.
+    rows = [0, 1, 127, 128, M // 2, M - 129, M - 2, M - 1]
+    A_rows = rng.integers(-2, 3, size=(len(rows), K)).astype(np.float16)
+    B = rng.integers(-2, 3, size=(K, N)).astype(np.float16)
+    Ad = torch.ones((M, K), dtype=torch.float16, device=dev)
+    for r, a in zip(rows, A_rows):
+        Ad[r].copy_(torch.from_numpy(a))
+    Bd = torch.from_numpy(B).to(dev)
+    C = tg.gemm_relu(Ad, Bd)
+    torch.cuda.synchronize()
+    got = C[rows].cpu().numpy()
+    assert_bitexact(got, oracle.gemm_relu_f16(A_rows, B), f"M*K > 2^31, K={K}")
+    # An all-ones row: C = ReLU(column sums of B).
+    ones_row = C[2].cpu().numpy()
+    ref_ones = oracle.gemm_relu_f16(np.ones((1, K), np.float16), B)[0]
+    assert_bitexact(ones_row, ref_ones, "all-ones row")
+    del Ad, Bd, C
+    torch.cuda.empty_cache()

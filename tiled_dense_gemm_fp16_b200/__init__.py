@@ -1,0 +1,24 @@
+"""B200 (sm_100a) tiled fp16 GEMM with fused ReLU: C = ReLU(A . B).
+
+The compute path is the C-ABI library ``libtg_gemm.so`` (hand-written CUDA
+kernels: TMA, tcgen05.mma into tensor memory, fused ReLU + fp16 epilogue).
+This package only marshals arguments to it; the library is loaded on first
+use and every call raises if it is missing.
+"""
+from ._binding import (  # noqa: F401
+    EXPORTS,
+    LIB_PATH,
+    Path,
+    Status,
+    TGError,
+    device_status,
+    gemm_relu,
+    gemm_relu_f16_raw,
+    lib,
+    path_name,
+    path_supports,
+    select_path,
+    status_string,
+    version,
+    wait_timeout_selftest,
+)

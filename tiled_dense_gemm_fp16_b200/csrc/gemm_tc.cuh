@@ -1,0 +1,347 @@
+// gemm_tc.cuh -- persistent, warp-specialised tcgen05 kernel for
+// C = ReLU(A . B), A (M x K) and B (K x N) row-major fp16, fp32 accumulation
+// in tensor memory, fp16 C (M x N) row-major.
+//
+// The tile model follows the matmul_relu quick-start kernel ("TileLang" wiki
+// page, "Programming model"): one output tile per (block_M x block_N) block
+// of C over a ceildiv grid, A and B tiles staged in shared memory through a
+// multi-stage pipelined K loop, a cleared fp32 accumulator, tile MMAs, then
+// max(acc, 0) and a copy into the fp16 output.  On sm_100a:
+//   * tiles are 128 x 256 x 64 (BM x BN x BK); a persistent grid of one CTA
+//     per SM walks the tiles in grouped (L2-friendly) order;
+//   * role warps: producer(s), one MMA-issuing warp that also owns TMEM, and
+//     four epilogue warps;
+//   * the fp32 accumulator lives in TMEM, double-buffered (2 x 256 columns),
+//     so the epilogue of tile i overlaps the main loop of tile i+1;
+//   * the first MMA of each tile runs with accumulate disabled, which is the
+//     accumulator clear.
+// Two operand-staging modes share the rest:
+//   * TMA mode: one producer thread issues 2-D TMA loads with 128-byte
+//     swizzle (needs 16-byte aligned bases and row strides); the hardware
+//     zero-fills out-of-bounds boxes.
+//   * EDGE mode: four producer warps load A and B with predicated 2-byte
+//     loads (zero outside the matrix) and write the same swizzled layout, for
+//     row strides that TMA cannot describe.
+// The epilogue reads TMEM with tcgen05.ld, applies ReLU on fp32 (every value
+// that is not > 0 becomes +0), rounds to fp16 (round to nearest even) and
+// stores the rows that lie inside C.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace tg {
+
+struct TcParams {
+  const __half* A;
+  const __half* B;
+  __half* C;
+  int M, N, K;
+  int m_tiles, n_tiles, num_tiles, k_blocks;
+  int group_m;           // tile rows per raster group
+  uint64_t wait_budget_ns;
+};
+
+template <bool EDGE>
+struct TcCfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = 256;
+  static constexpr int BK = 64;
+  static constexpr int STAGES = 4;
+  static constexpr int PRODUCER_WARPS = EDGE ? 4 : 1;
+  static constexpr int MMA_WARP = PRODUCER_WARPS;
+  static constexpr int EPI_WARP0 = MMA_WARP + 1;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
+  static constexpr int A_BYTES = BM * BK * 2;          // 16 KiB
+  static constexpr int B_BYTES = BK * BN * 2;          // 32 KiB
+  static constexpr int B_CHUNK_BYTES = BK * 64 * 2;    // one 64-column swizzle panel: 8 KiB
+  static constexpr int NUM_ACC = 2;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + BAR_BYTES;
+  static constexpr uint32_t FULL_COUNT = EDGE ? PRODUCER_WARPS * 32 : 1;
+  // A: K-major, B: MN-major (row-major K x N), M = 128, N = 256.
+  static constexpr uint32_t IDESC = make_idesc_f16_f32(BM, BN, false, true);
+};
+
+__device__ __forceinline__ void tile_coords(const TcParams& p, int t, int& m_blk, int& n_blk) {
+  const int group_tiles = p.group_m * p.n_tiles;
+  const int g = t / group_tiles;
+  const int first_m = g * p.group_m;
+  const int gm = min(p.m_tiles - first_m, p.group_m);
+  const int local = t - g * group_tiles;
+  m_blk = first_m + local % gm;
+  n_blk = local / gm;
+}
+
+// Swizzled byte offset of the 16-byte chunk `chunk` (0..7) of row `row` in a
+// tile whose rows are 128 bytes: chunk index XOR (row mod 8).
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
+  return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// EDGE mode: one 16-byte chunk of 8 consecutive fp16 values from a row-major
+// matrix, zero where (row >= rows) or (col >= cols).
+__device__ __forceinline__ uint4 load_chunk_pred(const __half* base, int64_t ld, int row, int rows, int col,
+                                                 int cols) {
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  if (row < rows) {
+    const unsigned short* p = reinterpret_cast<const unsigned short*>(base) + static_cast<int64_t>(row) * ld;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = col + e;
+      const uint32_t v = (c < cols) ? static_cast<uint32_t>(__ldg(p + c)) : 0u;
+      w[e >> 1] |= v << ((e & 1) * 16);
+    }
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <bool EDGE>
+__global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
+    gemm_relu_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                        const TcParams p) {
+  using Cfg = TcCfg<EDGE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_smem = smem;
+  uint8_t* b_smem = smem + Cfg::STAGES * Cfg::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES));
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + Cfg::STAGES;
+  uint64_t* acc_full_bar = bars + 2 * Cfg::STAGES;
+  uint64_t* acc_empty_bar = acc_full_bar + Cfg::NUM_ACC;
+  uint64_t* mma_done_bar = acc_empty_bar + Cfg::NUM_ACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&full_bar[s], Cfg::FULL_COUNT);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < Cfg::NUM_ACC; ++b) {
+      mbar_init(&acc_full_bar[b], 1);
+      mbar_init(&acc_empty_bar[b], Cfg::EPI_WARPS);
+    }
+    mbar_init(mma_done_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    if (!EDGE) {
+      tma_prefetch_desc(&tmap_a);
+      tma_prefetch_desc(&tmap_b);
+    }
+  }
+  if (warp == Cfg::MMA_WARP) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_alloc_permit();
+  }
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  tcgen05_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp < Cfg::PRODUCER_WARPS) {
+    // ------------------------------------------------------------------
+    // Producer: stage A (BM x BK) and B (BK x BN) tiles into the ring.
+    // ------------------------------------------------------------------
+    if (!EDGE) {
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int last_parity[Cfg::STAGES];
+#pragma unroll
+        for (int s = 0; s < Cfg::STAGES; ++s) last_parity[s] = -1;
+        bool ok = true;
+        for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+          int m_blk, n_blk;
+          tile_coords(p, t, m_blk, n_blk);
+          const int m0 = m_blk * Cfg::BM;
+          const int n0 = n_blk * Cfg::BN;
+          for (int kb = 0; kb < p.k_blocks; ++kb) {
+            if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full_bar[stage], Cfg::A_BYTES + Cfg::B_BYTES);
+            const int k0 = kb * Cfg::BK;
+            tma_load_2d(a_smem + stage * Cfg::A_BYTES, &tmap_a, &full_bar[stage], k0, m0);
+            uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
+#pragma unroll
+            for (int j = 0; j < Cfg::BN / 64; ++j)
+              tma_load_2d(bdst + j * Cfg::B_CHUNK_BYTES, &tmap_b, &full_bar[stage], n0 + j * 64, k0);
+            last_parity[stage] = static_cast<int>(phase);
+            if (++stage == Cfg::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        // Every load issued has landed before the CTA may exit (a no-op on
+        // the normal path, where the MMA warp consumed them all).
+#pragma unroll 1
+        for (int s = 0; s < Cfg::STAGES; ++s) {
+          if (last_parity[s] >= 0) {
+            volatile int no_abort = 0;
+            mbar_wait(&full_bar[s], static_cast<uint32_t>(last_parity[s]), &no_abort, p.wait_budget_ns, 2);
+          }
+        }
+      }
+    } else {
+      const int ptid = threadIdx.x;  // 0 .. 127
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      const int64_t lda = p.K, ldb = p.N;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int m_blk, n_blk;
+        tile_coords(p, t, m_blk, n_blk);
+        const int m0 = m_blk * Cfg::BM;
+        const int n0 = n_blk * Cfg::BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          const bool free_slot = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 3);
+          if (!__all_sync(0xffffffffu, free_slot)) {
+            ok = false;
+            break;
+          }
+          const int k0 = kb * Cfg::BK;
+          uint8_t* adst = a_smem + stage * Cfg::A_BYTES;
+          uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
+          // A tile: 128 rows x 8 chunks.
+#pragma unroll 4
+          for (int i = 0; i < (Cfg::BM * 8) / 128; ++i) {
+            const int c = ptid + i * 128;
+            const int r = c >> 3, kc = c & 7;
+            const uint4 v = load_chunk_pred(p.A, lda, m0 + r, p.M, k0 + kc * 8, p.K);
+            *reinterpret_cast<uint4*>(adst + sw128_offset(r, kc)) = v;
+          }
+          // B tile: 64 k-rows x 32 chunks, in 4 panels of 64 columns.
+#pragma unroll 4
+          for (int i = 0; i < (Cfg::BK * 32) / 128; ++i) {
+            const int c = ptid + i * 128;
+            const int kr = c >> 5, nc = c & 31;
+            const uint4 v = load_chunk_pred(p.B, ldb, k0 + kr, p.K, n0 + nc * 8, p.N);
+            *reinterpret_cast<uint4*>(bdst + (nc >> 3) * Cfg::B_CHUNK_BYTES + sw128_offset(kr, nc & 7)) = v;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&full_bar[stage]);
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == Cfg::MMA_WARP) {
+    // ------------------------------------------------------------------
+    // MMA issuer: one thread drives the tensor core.
+    // ------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, abort_flag, p.wait_budget_ns, 4)) break;
+        tcgen05_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + acc * Cfg::BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 5)) {
+            ok = false;
+            break;
+          }
+          tcgen05_fence_after_sync();
+          const uint32_t a_addr = smem_u32(a_smem + stage * Cfg::A_BYTES);
+          const uint32_t b_addr = smem_u32(b_smem + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < Cfg::BK / 16; ++k) {
+            // A: advance 16 elements (32 bytes) inside the swizzled row.
+            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+            // B: advance 16 k-rows (2048 bytes); 64-column panels 8 KiB apart.
+            const uint64_t bdesc = make_sw128_desc(b_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
+            umma_f16_ss(d_tmem, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[stage]);  // frees the stage when these MMAs finish
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full_bar[acc]);  // accumulator ready for the epilogue
+      }
+      // All MMAs issued by this thread are complete before TMEM is released.
+      umma_commit(mma_done_bar);
+      volatile int no_abort = 0;
+      mbar_wait(mma_done_bar, 0, &no_abort, p.wait_budget_ns, 6);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------
+    // Epilogue: TMEM -> registers -> ReLU -> fp16 -> C.
+    // ------------------------------------------------------------------
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      int m_blk, n_blk;
+      tile_coords(p, t, m_blk, n_blk);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      // The TMEM loads below are warp-collective: leave only as a whole warp.
+      const bool ready = mbar_wait(&acc_full_bar[acc], acc_phase, abort_flag, p.wait_budget_ns, 7);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tcgen05_fence_after_sync();
+      const int row = m_blk * Cfg::BM + quad * 32 + lane;
+      const bool row_ok = row < p.M;
+      __half* crow = p.C + static_cast<int64_t>(row) * p.N;
+#pragma unroll 1
+      for (int c = 0; c < Cfg::BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + c * 32, r);
+        tmem_ld_wait();
+        const int col0 = n_blk * Cfg::BN + c * 32;
+        if (row_ok && col0 < p.N) {
+          uint32_t h[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = __uint_as_float(r[2 * e]);
+            const float x1 = __uint_as_float(r[2 * e + 1]);
+            const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
+            h[e] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          if (!EDGE) {
+            // N % 8 == 0 and C is 16-byte aligned: whole 8-column pieces.
+            uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+          } else {
+            unsigned short* dst = reinterpret_cast<unsigned short*>(crow + col0);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (col0 + e < p.N) dst[e] = static_cast<unsigned short>((h[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+          }
+        }
+      }
+      tcgen05_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty_bar[acc]);
+    }
+  }
+
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  if (warp == Cfg::MMA_WARP) {
+    tcgen05_fence_after_sync();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace tg

@@ -1,0 +1,320 @@
+// tg_gemm.cu -- C ABI, argument checks, path choice, TMA descriptor encoding
+// and kernel launches for C = ReLU(A . B) on sm_100a.
+//
+// The whole device side is one translation unit: the kernels live in the
+// headers included below and share the device error word of ptx.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tg_gemm.h"
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace tg {
+namespace {
+
+constexpr uint64_t kWaitBudgetNs = 4000000000ull;  // 4 s per pipeline wait
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  bool tc_attr = false;
+  bool tc_edge_attr = false;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+bool g_encode_probed = false;
+
+// ---------------------------------------------------------------------------
+// Host-side argument logic (no CUDA calls)
+// ---------------------------------------------------------------------------
+bool ranges_overlap(const void* a, int64_t a_bytes, const void* b, int64_t b_bytes) {
+  if (a_bytes <= 0 || b_bytes <= 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + static_cast<uintptr_t>(b_bytes) && b0 < a0 + static_cast<uintptr_t>(a_bytes);
+}
+
+bool args_valid(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return false;
+  if (M > INT_MAX || N > INT_MAX || K > INT_MAX) return false;
+  if (M == 0 || N == 0) return true;
+  if (C == nullptr) return false;
+  if (K > 0 && (A == nullptr || B == nullptr)) return false;
+  const uintptr_t bits = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+                         reinterpret_cast<uintptr_t>(C);
+  if (bits & 1u) return false;
+  const int64_t c_bytes = 2 * M * N;
+  if (K > 0 && (ranges_overlap(C, c_bytes, A, 2 * M * K) || ranges_overlap(C, c_bytes, B, 2 * K * N)))
+    return false;
+  // Tile counts must fit the kernels' 32-bit tile indices.
+  const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
+  if (tiles > INT_MAX) return false;
+  return true;
+}
+
+bool aligned16(const void* A, const void* B, const void* C, int64_t N, int64_t K) {
+  const uintptr_t bits = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
+                         reinterpret_cast<uintptr_t>(C);
+  return (bits & 15u) == 0 && (N % 8) == 0 && (K % 8) == 0;
+}
+
+bool path_supports(int path, const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
+  if (!args_valid(A, B, C, M, N, K)) return false;
+  if (M == 0 || N == 0) return path == TG_PATH_NONE || path == TG_PATH_AUTO;
+  if (K == 0) return path == TG_PATH_ZERO || path == TG_PATH_AUTO;
+  switch (path) {
+    case TG_PATH_AUTO:
+    case TG_PATH_TC_EDGE:
+      return true;
+    case TG_PATH_TC:
+      return aligned16(A, B, C, N, K);
+    default:
+      return false;
+  }
+}
+
+int select_path(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
+  if (!args_valid(A, B, C, M, N, K)) return -2;
+  if (M == 0 || N == 0) return TG_PATH_NONE;
+  if (K == 0) return TG_PATH_ZERO;
+  if (aligned16(A, B, C, N, K)) return TG_PATH_TC;
+  return TG_PATH_TC_EDGE;
+}
+
+// ---------------------------------------------------------------------------
+// Device probing and TMA descriptors
+// ---------------------------------------------------------------------------
+tg_status current_device(int& dev, DeviceInfo*& info) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return TG_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return TG_ERR_UNSUPPORTED_DEVICE;
+    }
+    d.probed = true;
+    d.supported = (major == 10 && minor == 0);
+    d.sm_count = sms;
+  }
+  info = &d;
+  return d.supported ? TG_OK : TG_ERR_UNSUPPORTED_DEVICE;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_encode_probed) {
+    g_encode_probed = true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    cudaGetLastError();
+  }
+  return g_encode_tiled;
+}
+
+// Row-major (rows x cols) fp16 matrix; box = box_cols x box_rows, 128-byte
+// swizzle (box_cols * 2 must be 128).
+bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+template <bool EDGE>
+tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, cudaStream_t stream,
+                    DeviceInfo* info) {
+  using Cfg = TcCfg<EDGE>;
+  auto kernel = gemm_relu_tc_kernel<EDGE>;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    bool& attr = EDGE ? info->tc_edge_attr : info->tc_attr;
+    if (!attr) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      attr = true;
+    }
+  }
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof ta);
+  std::memset(&tb, 0, sizeof tb);
+  if (!EDGE) {
+    if (!encode_2d(&ta, A, M, K, 64, Cfg::BM)) return TG_ERR_LAUNCH;
+    if (!encode_2d(&tb, B, K, N, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+  }
+  TcParams p;
+  p.A = static_cast<const __half*>(A);
+  p.B = static_cast<const __half*>(B);
+  p.C = static_cast<__half*>(C);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.m_tiles = static_cast<int>((M + Cfg::BM - 1) / Cfg::BM);
+  p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
+  p.group_m = 16;
+  p.wait_budget_ns = kWaitBudgetNs;
+  const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
+  kernel<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+}
+
+__global__ void wait_timeout_selftest_kernel(uint64_t budget_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on `bar`: this wait must give up by itself.
+    mbar_wait(&bar, 0, &abort_flag, budget_ns, 0xEE);
+  }
+  __syncthreads();
+}
+
+tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream_ptr,
+              int path) {
+  if (!args_valid(A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
+  if (path == TG_PATH_AUTO) path = select_path(A, B, C, M, N, K);
+  if (!path_supports(path, A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
+  if (path == TG_PATH_NONE) return TG_OK;
+  int dev = 0;
+  DeviceInfo* info = nullptr;
+  tg_status st = current_device(dev, info);
+  if (st != TG_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  switch (path) {
+    case TG_PATH_ZERO:
+      if (cudaMemsetAsync(C, 0, static_cast<size_t>(2 * M * N), stream) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      return TG_OK;
+    case TG_PATH_TC:
+      return launch_tc<false>(A, B, C, M, N, K, stream, info);
+    case TG_PATH_TC_EDGE:
+      return launch_tc<true>(A, B, C, M, N, K, stream, info);
+    default:
+      return TG_ERR_INTERNAL;
+  }
+}
+
+}  // namespace
+}  // namespace tg
+
+extern "C" {
+
+tg_status tg_gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream) {
+  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO);
+}
+
+tg_status tg_gemm_relu_f16_path(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                                void* stream, int path) {
+  return tg::run(A, B, C, M, N, K, stream, path);
+}
+
+int tg_select_path(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
+  return tg::select_path(A, B, C, M, N, K);
+}
+
+int tg_path_supports(int path, const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
+  return tg::path_supports(path, A, B, C, M, N, K) ? 1 : 0;
+}
+
+tg_status tg_device_status(uint32_t* detail) {
+  int dev = 0;
+  tg::DeviceInfo* info = nullptr;
+  tg_status st = tg::current_device(dev, info);
+  if (st != TG_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, tg::g_device_error, sizeof word) != cudaSuccess ||
+      cudaMemcpyToSymbol(tg::g_device_error, &zero, sizeof zero) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  if (detail) *detail = word;
+  if (word == 0) return TG_OK;
+  if ((word & 0xff00u) == tg::kDevErrWaitTimeout) return TG_ERR_TIMEOUT;
+  return TG_ERR_INTERNAL;
+}
+
+tg_status tg_wait_timeout_selftest(int64_t budget_ns, void* stream) {
+  int dev = 0;
+  tg::DeviceInfo* info = nullptr;
+  tg_status st = tg::current_device(dev, info);
+  if (st != TG_OK) return st;
+  if (budget_ns < 1000) budget_ns = 1000;
+  if (budget_ns > 10000000000ll) budget_ns = 10000000000ll;
+  tg::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(budget_ns));
+  return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+}
+
+const char* tg_status_string(int status) {
+  switch (status) {
+    case TG_OK: return "ok";
+    case TG_ERR_INVALID_ARG: return "invalid argument";
+    case TG_ERR_UNSUPPORTED_DEVICE: return "unsupported or missing device (needs compute capability 10.0)";
+    case TG_ERR_LAUNCH: return "kernel launch or CUDA call failed";
+    case TG_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case TG_ERR_INTERNAL: return "internal error";
+    default: return "unknown status";
+  }
+}
+
+const char* tg_path_name(int path) {
+  switch (path) {
+    case TG_PATH_NONE: return "none";
+    case TG_PATH_AUTO: return "auto";
+    case TG_PATH_TC: return "tc";
+    case TG_PATH_TC_EDGE: return "tc_edge";
+    case TG_PATH_SKINNY: return "skinny";
+    case TG_PATH_GEMV: return "gemv";
+    case TG_PATH_ZERO: return "zero";
+    default: return "invalid";
+  }
+}
+
+int tg_version(void) { return 100; }
+
+}  // extern "C"
