@@ -70,13 +70,18 @@ def test_overlap_rejected():
     assert tg.gemm_relu_f16_raw(A0, B0, A0 + 2 * M * K - 2, M, N, K) == Status.INVALID_ARG
     assert tg.gemm_relu_f16_raw(A0, B0, B0 + 128, M, N, K) == Status.INVALID_ARG
     # Adjacent but not overlapping is fine for the host logic.
-    assert tg.select_path(A0, B0, A0 + 2 * M * K, M, N, K) == Path.TC
+    assert tg.select_path(A0, B0, A0 + 2 * M * K, M, N, K) == Path.SKINNY
 
 
 def test_path_selection():
     assert tg.select_path(A0, B0, C0, 128, 128, 0) == Path.ZERO
     assert tg.select_path(A0, B0, C0, 4096, 4096, 4096) == Path.TC
     assert tg.select_path(A0, B0, C0, 8192, 8192, 8192) == Path.TC
+    # Small M with aligned rows: the split-K small-M kernel.
+    for M in (1, 16, 64, 256):
+        assert tg.select_path(A0, B0, C0, M, 8192, 8192) == Path.SKINNY
+    assert tg.select_path(A0, B0, C0, 257, 8192, 8192) == Path.TC
+    assert tg.select_path(A0, B0, C0, 64, 8191, 8192) == Path.TC_EDGE
     # Row strides that are not 16-byte multiples, or misaligned bases, need the edge mode.
     assert tg.select_path(A0, B0, C0, 3001, 5003, 1021) == Path.TC_EDGE
     assert tg.select_path(A0, B0, C0, 777, 12289, 4095) == Path.TC_EDGE
@@ -92,6 +97,9 @@ def test_forced_path_requirements():
     assert not tg.path_supports(Path.ZERO, A0, B0, C0, 256, 256, 256)
     assert tg.path_supports(Path.ZERO, A0, B0, C0, 256, 256, 0)
     assert not tg.path_supports(42, A0, B0, C0, 256, 256, 256)
+    assert tg.path_supports(Path.SKINNY, A0, B0, C0, 256, 256, 256)
+    assert not tg.path_supports(Path.SKINNY, A0, B0, C0, 257, 256, 256)
+    assert not tg.path_supports(Path.SKINNY, A0, B0, C0, 16, 250, 256)
     assert tg.gemm_relu_f16_raw(A0, B0, C0, 256, 250, 256, 0, Path.TC) == Status.INVALID_ARG
 
 

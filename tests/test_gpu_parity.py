@@ -15,13 +15,15 @@ from tiled_dense_gemm_fp16_b200._binding import Path
 
 pytestmark = pytest.mark.gpu
 
-TC, EDGE = Path.TC, Path.TC_EDGE
+TC, EDGE, SKINNY = Path.TC, Path.TC_EDGE, Path.SKINNY
 
 
 def _paths_for(M, N, K):
     paths = [None, EDGE]
     if N % 8 == 0 and K % 8 == 0:
         paths.append(TC)
+        if M <= 256:
+            paths.append(SKINNY)
     return paths
 
 
@@ -74,6 +76,32 @@ def test_tile_edges_uniform(M, N, K):
         got, guards = run_gpu(A, B, path)
         assert guards
         assert_close(got, ref, f"{(M, N, K)} path={path}")
+
+
+SKINNY_SHAPES = [
+    (1, 8, 8), (1, 136, 72), (2, 1024, 1000), (7, 520, 4096), (8, 128, 64), (15, 264, 136),
+    (16, 8192, 512), (17, 1000, 200), (31, 128, 8), (64, 520, 1000), (100, 2048, 2048),
+    (128, 136, 4104), (129, 256, 64), (200, 1024, 312), (255, 392, 1000), (256, 8192, 256),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SKINNY_SHAPES)
+def test_skinny_integer_bitexact(M, N, K):
+    """Small M: panels of 128 columns, split K, cluster reduction; partial panels and short K."""
+    A, B = inputs.operands(M, N, K, "int", seed=M + 11 * N + K)
+    ref = oracle.gemm_relu_f16(A, B)
+    got, guards = run_gpu(A, B, SKINNY)
+    assert guards, (M, N, K)
+    assert_bitexact(got, ref, f"skinny {(M, N, K)}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8192, 8192), (16, 1024, 4096), (64, 8192, 1024), (256, 520, 2048)])
+def test_skinny_uniform(M, N, K):
+    A, B = inputs.operands(M, N, K, "uniform", seed=M + N + K)
+    ref = oracle.gemm_relu_f16(A, B)
+    got, guards = run_gpu(A, B, SKINNY)
+    assert guards
+    assert_close(got, ref, f"skinny {(M, N, K)}")
 
 
 def test_misaligned_base_pointers_use_edge_mode():
@@ -174,11 +202,11 @@ def test_workload_square8192_integer():
 
 
 def test_workload_skinny():
-    _check_workload("skinny", paths=(None, TC, EDGE))
+    _check_workload("skinny", paths=(None, SKINNY, TC, EDGE))
 
 
 def test_workload_skinny_integer():
-    _check_workload("skinny", dist="int", exact=True, paths=(None, TC, EDGE))
+    _check_workload("skinny", dist="int", exact=True, paths=(None, SKINNY, TC, EDGE))
 
 
 def test_workload_ragged():

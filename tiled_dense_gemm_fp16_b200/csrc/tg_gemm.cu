@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "../../include/tg_gemm.h"
+#include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 
@@ -21,6 +22,7 @@ namespace {
 
 constexpr uint64_t kWaitBudgetNs = 4000000000ull;  // 4 s per pipeline wait
 constexpr int kMaxDevices = 64;
+constexpr int64_t kSkinnyMaxM = 256;               // largest M the small-M path takes
 
 struct DeviceInfo {
   bool probed = false;
@@ -28,6 +30,7 @@ struct DeviceInfo {
   int sm_count = 0;
   bool tc_attr = false;
   bool tc_edge_attr = false;
+  bool skinny_attr = false;
 };
 
 std::mutex g_mutex;
@@ -78,6 +81,8 @@ bool path_supports(int path, const void* A, const void* B, const void* C, int64_
       return true;
     case TG_PATH_TC:
       return aligned16(A, B, C, N, K);
+    case TG_PATH_SKINNY:
+      return aligned16(A, B, C, N, K) && M <= kSkinnyMaxM;
     default:
       return false;
   }
@@ -87,7 +92,7 @@ int select_path(const void* A, const void* B, const void* C, int64_t M, int64_t 
   if (!args_valid(A, B, C, M, N, K)) return -2;
   if (M == 0 || N == 0) return TG_PATH_NONE;
   if (K == 0) return TG_PATH_ZERO;
-  if (aligned16(A, B, C, N, K)) return TG_PATH_TC;
+  if (aligned16(A, B, C, N, K)) return M <= kSkinnyMaxM ? TG_PATH_SKINNY : TG_PATH_TC;
   return TG_PATH_TC_EDGE;
 }
 
@@ -192,6 +197,78 @@ tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N,
   return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
 }
 
+// Small-M path: grid (S, P) with clusters of S CTAs along K.
+tg_status launch_skinny(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                        cudaStream_t stream, DeviceInfo* info) {
+  using Cfg = SkinnyCfg;
+  constexpr int kMaxSmem = 1024 + 220 * 1024 + Cfg::BAR_BYTES;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!info->skinny_attr) {
+      if (cudaFuncSetAttribute(gemm_relu_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      info->skinny_attr = true;
+    }
+  }
+  SkinnyParams p;
+  std::memset(&p, 0, sizeof p);
+  p.C = static_cast<__half*>(C);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.m_pad = static_cast<int>((M + 15) / 16 * 16);
+  p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
+  // Two CTAs per SM fit while the ring stays within ~112 KiB (M_pad <= 128).
+  const bool two_per_sm = p.m_pad <= 128;
+  const int budget = (two_per_sm ? 112 : 220) * 1024;
+  const int stage_bytes = Cfg::stage_bytes(p.m_pad);
+  int stages = budget / stage_bytes;
+  stages = stages > 8 ? 8 : stages;
+  if (stages < 2) return TG_ERR_INTERNAL;
+  // The fp32 partial [M_pad][128] reuses the ring after the main loop.
+  if (stages * stage_bytes < p.m_pad * Cfg::PANEL * 4) return TG_ERR_INTERNAL;
+  p.stages = stages;
+  p.a_stage_bytes = static_cast<uint32_t>(p.m_pad * 128);
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(p.m_pad)) cols <<= 1;
+  p.tmem_cols = cols;
+  p.idesc = make_idesc_f16_f32(Cfg::PANEL, p.m_pad, true, false);
+  p.wait_budget_ns = kWaitBudgetNs;
+  const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);
+  const int slots = (two_per_sm ? 2 : 1) * info->sm_count;
+  int splits = slots / panels;
+  splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
+  if (splits > p.k_blocks) splits = p.k_blocks;
+  p.splits = splits;
+  if (panels > 65535) return TG_ERR_INVALID_ARG;
+
+  CUtensorMap ta, tb;
+  if (!encode_2d(&ta, A, M, K, 64, p.m_pad)) return TG_ERR_LAUNCH;
+  if (!encode_2d(&tb, B, K, N, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(panels), 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::smem_bytes(p.m_pad, stages));
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_relu_skinny_kernel, ta, tb, p) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
+}
+
 __global__ void wait_timeout_selftest_kernel(uint64_t budget_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -230,6 +307,8 @@ tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64
       return launch_tc<false>(A, B, C, M, N, K, stream, info);
     case TG_PATH_TC_EDGE:
       return launch_tc<true>(A, B, C, M, N, K, stream, info);
+    case TG_PATH_SKINNY:
+      return launch_skinny(A, B, C, M, N, K, stream, info);
     default:
       return TG_ERR_INTERNAL;
   }
