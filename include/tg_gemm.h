@@ -65,7 +65,10 @@ typedef enum tg_path {
                             C^T = B^T A^T); same alignment needs as TC       */
     TG_PATH_GEMV = 4,    /* CUDA-core kernel for M <= 8; same alignment
                             needs as TC                                     */
-    TG_PATH_ZERO = 5     /* K == 0: C is filled with +0 (empty sum)         */
+    TG_PATH_ZERO = 5,    /* K == 0: C is filled with +0 (empty sum)         */
+    TG_PATH_TC_PAIR = 6  /* the TMA + tcgen05 kernel on SM pairs
+                            (cta_group::2), 256x256 tiles; same alignment
+                            needs as TC                                     */
 } tg_path;
 
 /*

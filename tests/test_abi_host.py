@@ -40,6 +40,7 @@ def test_version_and_strings():
     assert tg.status_string(Status.OK) == "ok"
     assert "invalid" in tg.status_string(Status.INVALID_ARG)
     assert tg.path_name(Path.TC) == "tc" and tg.path_name(Path.TC_EDGE) == "tc_edge"
+    assert tg.path_name(Path.TC_PAIR) == "tc_pair" and tg.path_name(Path.SKINNY) == "skinny"
     assert tg.status_string(99) == "unknown status"
 
 
@@ -75,12 +76,12 @@ def test_overlap_rejected():
 
 def test_path_selection():
     assert tg.select_path(A0, B0, C0, 128, 128, 0) == Path.ZERO
-    assert tg.select_path(A0, B0, C0, 4096, 4096, 4096) == Path.TC
-    assert tg.select_path(A0, B0, C0, 8192, 8192, 8192) == Path.TC
+    assert tg.select_path(A0, B0, C0, 4096, 4096, 4096) == Path.TC_PAIR
+    assert tg.select_path(A0, B0, C0, 8192, 8192, 8192) == Path.TC_PAIR
     # Small M with aligned rows: the split-K small-M kernel.
     for M in (1, 16, 64, 256):
         assert tg.select_path(A0, B0, C0, M, 8192, 8192) == Path.SKINNY
-    assert tg.select_path(A0, B0, C0, 257, 8192, 8192) == Path.TC
+    assert tg.select_path(A0, B0, C0, 257, 8192, 8192) == Path.TC_PAIR
     assert tg.select_path(A0, B0, C0, 64, 8191, 8192) == Path.TC_EDGE
     # Row strides that are not 16-byte multiples, or misaligned bases, need the edge mode.
     assert tg.select_path(A0, B0, C0, 3001, 5003, 1021) == Path.TC_EDGE
@@ -91,6 +92,8 @@ def test_path_selection():
 
 def test_forced_path_requirements():
     assert tg.path_supports(Path.TC, A0, B0, C0, 256, 256, 256)
+    assert tg.path_supports(Path.TC_PAIR, A0, B0, C0, 256, 256, 256)
+    assert not tg.path_supports(Path.TC_PAIR, A0, B0, C0, 256, 250, 256)
     assert not tg.path_supports(Path.TC, A0, B0, C0, 256, 250, 256)
     assert not tg.path_supports(Path.TC, A0, B0, C0, 256, 256, 250)
     assert tg.path_supports(Path.TC_EDGE, A0, B0, C0, 256, 250, 250)

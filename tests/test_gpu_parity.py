@@ -15,23 +15,31 @@ from tiled_dense_gemm_fp16_b200._binding import Path
 
 pytestmark = pytest.mark.gpu
 
-TC, EDGE, SKINNY = Path.TC, Path.TC_EDGE, Path.SKINNY
+TC, EDGE, SKINNY, PAIR = Path.TC, Path.TC_EDGE, Path.SKINNY, Path.TC_PAIR
 
 
 def _paths_for(M, N, K):
     paths = [None, EDGE]
     if N % 8 == 0 and K % 8 == 0:
-        paths.append(TC)
+        paths += [TC, PAIR]
         if M <= 256:
             paths.append(SKINNY)
     return paths
+
+
+def test_pair_kernel_single_tile():
+    """One 256 x 256 tile on one SM pair, one 64-deep k-block: the smallest cta_group::2 case."""
+    A, B = inputs.operands(256, 256, 64, "int", seed=12)
+    got, guards = run_gpu(A, B, PAIR)
+    assert guards
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), "pair 256x256x64")
 
 
 # ---------------------------------------------------------------------------
 # Small square workload (256^3): integer variant bit-exact, uniform within tolerance
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("path", [None, TC, EDGE], ids=["auto", "tc", "edge"])
+@pytest.mark.parametrize("path", [None, TC, EDGE, PAIR], ids=["auto", "tc", "edge", "pair"])
 def test_square256_integer_bitexact(path):
     A, B = inputs.operands(256, 256, 256, "int", seed=0)
     got, guards = run_gpu(A, B, path)
@@ -39,7 +47,7 @@ def test_square256_integer_bitexact(path):
     assert_bitexact(got, oracle.gemm_relu_f16(A, B), "square256 int")
 
 
-@pytest.mark.parametrize("path", [None, TC, EDGE], ids=["auto", "tc", "edge"])
+@pytest.mark.parametrize("path", [None, TC, EDGE, PAIR], ids=["auto", "tc", "edge", "pair"])
 def test_square256_uniform(path):
     (shape, A, B), = inputs.WORKLOADS["square256"].problems()
     got, guards = run_gpu(A, B, path)
@@ -144,7 +152,7 @@ def test_special_values():
     B[:, 8:16] = -2.0                             # -65536 -> ReLU -> +0
     B[:4095, 16:24] = 0.0                         # 4 * 12289 = 49156 -> 49152 (nearest even half)
     ref = oracle.gemm_relu_f16(A, B)
-    for path in (TC, EDGE):
+    for path in (TC, EDGE, PAIR):
         got, _ = run_gpu(A, B, path)
         assert_bitexact(got, ref, f"special path={path}")
     assert np.all(np.isinf(ref[:, :8].astype(np.float32))) and np.all(ref[:, 8:16].view(np.uint16) == 0)
@@ -186,19 +194,19 @@ def _check_workload(name, dist=None, exact=False, full_oracle_max_macs=5e9, path
 
 
 def test_workload_square4096():
-    _check_workload("square4096", paths=(None, EDGE))
+    _check_workload("square4096", paths=(None, TC, EDGE))
 
 
 def test_workload_square4096_integer():
-    _check_workload("square4096", dist="int", exact=True)
+    _check_workload("square4096", dist="int", exact=True, paths=(None, TC))
 
 
 def test_workload_square8192():
-    _check_workload("square8192")
+    _check_workload("square8192", paths=(None, TC))
 
 
 def test_workload_square8192_integer():
-    _check_workload("square8192", dist="int", exact=True)
+    _check_workload("square8192", dist="int", exact=True, paths=(None, TC))
 
 
 def test_workload_skinny():

@@ -34,6 +34,7 @@ class Path(enum.IntEnum):
     SKINNY = 3
     GEMV = 4
     ZERO = 5
+    TC_PAIR = 6
 
 
 class TGError(RuntimeError):

@@ -1,0 +1,246 @@
+// gemm_tc_pair.cuh -- the persistent tcgen05 GEMM + ReLU kernel on CTA pairs
+// (cta_group::2): 256 x 256 output tiles, each computed by the two SMs of a
+// 2-CTA cluster.
+//
+// Same tile model as gemm_tc.cuh (the matmul_relu quick-start kernel: tiles
+// staged through a pipelined K loop, cleared fp32 accumulator, tile MMAs,
+// max(acc, 0), fp16 output), with the MMA spread over an SM pair:
+//   * CTA r of the pair (r = 0, 1) loads rows [128 r, 128 r + 128) of the
+//     A tile and columns [128 r, 128 r + 128) of the B tile into its own
+//     shared memory (TMA, 128-byte swizzle, no multicast), 32 KiB per stage,
+//     6 stages;
+//   * both CTAs' loads count their bytes on the even CTA's "full" barrier;
+//     the even CTA's single MMA thread issues 256 x 256 x 16 pair MMAs that
+//     read both CTAs' shared memory and write both CTAs' TMEM (rows
+//     [128 r, 128 r + 128) of the tile land in CTA r);
+//   * the MMA commits multicast to both CTAs' "empty" barriers (each CTA then
+//     refills its own stage) and, per tile, to both CTAs' "accumulator full"
+//     barriers; the eight epilogue warps of the pair release the accumulator
+//     on the even CTA's "accumulator empty" barrier;
+//   * per SM, each 64-deep k-block moves 32 KiB from L2 for 128 x 256 x 64
+//     MACs, two thirds of the 48 KiB the single-CTA 128 x 256 tile needs.
+// Every wait is bounded; a cluster barrier brackets the kernel so that no
+// CTA exits while its peer may still touch its shared memory or barriers.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace tg {
+
+struct TcPairCfg {
+  static constexpr int BM = 128;        // rows per CTA (the pair tile is 256)
+  static constexpr int PAIR_M = 256;
+  static constexpr int BN = 256;        // columns per pair tile
+  static constexpr int BN_HALF = 128;   // columns of B each CTA loads
+  static constexpr int BK = 64;
+  static constexpr int STAGES = 6;
+  static constexpr int THREADS = 192;   // producer, MMA, 4 epilogue warps
+  static constexpr int MMA_WARP = 1;
+  static constexpr int EPI_WARP0 = 2;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int A_BYTES = BM * BK * 2;        // 16 KiB
+  static constexpr int B_BYTES = BK * BN_HALF * 2;   // 16 KiB
+  static constexpr int B_CHUNK_BYTES = BK * 64 * 2;  // 8 KiB panel of 64 columns
+  static constexpr int NUM_ACC = 2;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + BAR_BYTES;
+  static constexpr uint32_t IDESC = make_idesc_f16_f32(PAIR_M, BN, false, true);
+};
+
+__global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
+    gemm_relu_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                             const TcParams p) {
+  using Cfg = TcPairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_smem = smem;
+  uint8_t* b_smem = smem + Cfg::STAGES * Cfg::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES));
+  uint64_t* full_bar = bars;                         // used in the even CTA
+  uint64_t* empty_bar = bars + Cfg::STAGES;          // per CTA
+  uint64_t* acc_full_bar = bars + 2 * Cfg::STAGES;   // per CTA
+  uint64_t* acc_empty_bar = acc_full_bar + Cfg::NUM_ACC;  // used in the even CTA
+  uint64_t* mma_done_bar = acc_empty_bar + Cfg::NUM_ACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = even CTA (issues the MMAs), 1 = odd CTA
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x >> 1;
+  const int num_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < Cfg::NUM_ACC; ++b) {
+      mbar_init(&acc_full_bar[b], 1);
+      mbar_init(&acc_empty_bar[b], 2 * Cfg::EPI_WARPS);
+    }
+    mbar_init(mma_done_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+  }
+  if (warp == Cfg::MMA_WARP) {
+    tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_alloc_permit_pair();
+  }
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote use
+  tcgen05_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------
+    // Producer (both CTAs): this CTA's half of the A and B tiles.
+    // ------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[Cfg::STAGES];
+#pragma unroll
+      for (int s = 0; s < Cfg::STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters) {
+        int m_blk, n_blk;
+        tile_coords(p, t, m_blk, n_blk);
+        const int m0 = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM;
+        const int nb = n_blk * Cfg::BN + static_cast<int>(rank) * Cfg::BN_HALF;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 0x41)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_even = mapa_shared(smem_u32(&full_bar[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
+          const int k0 = kb * Cfg::BK;
+          uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
+          tma_load_2d_pair(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, k0, m0);
+          tma_load_2d_pair(bdst, &tmap_b, full_even, nb, k0);
+          tma_load_2d_pair(bdst + Cfg::B_CHUNK_BYTES, &tmap_b, full_even, nb + 64, k0);
+          last_parity[stage] = static_cast<int>(phase);
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // The even CTA's full barriers count both CTAs' bytes: once they have
+      // completed, every load of the pair has landed.
+      if (leader) {
+#pragma unroll 1
+        for (int s = 0; s < Cfg::STAGES; ++s) {
+          if (last_parity[s] >= 0) {
+            volatile int no_abort = 0;
+            mbar_wait(&full_bar[s], static_cast<uint32_t>(last_parity[s]), &no_abort, p.wait_budget_ns, 0x42);
+          }
+        }
+      }
+    }
+  } else if (warp == Cfg::MMA_WARP) {
+    // ------------------------------------------------------------------
+    // MMA issuer (even CTA only).
+    // ------------------------------------------------------------------
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, abort_flag, p.wait_budget_ns, 0x43)) break;
+        tcgen05_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + acc * Cfg::BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 0x44)) {
+            ok = false;
+            break;
+          }
+          tcgen05_fence_after_sync();
+          const uint32_t a_addr = smem_u32(a_smem + stage * Cfg::A_BYTES);
+          const uint32_t b_addr = smem_u32(b_smem + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < Cfg::BK / 16; ++k) {
+            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+            const uint64_t bdesc = make_sw128_desc(b_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
+            umma_f16_ss_pair(d_tmem, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair_mc(&empty_bar[stage], 0x3);  // both CTAs may refill this stage
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(&acc_full_bar[acc], 0x3);  // both halves of the accumulator are ready
+      }
+      umma_commit_pair_mc(mma_done_bar, 0x1);
+      volatile int no_abort = 0;
+      mbar_wait(mma_done_bar, 0, &no_abort, p.wait_budget_ns, 0x45);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------
+    // Epilogue (both CTAs): this CTA's 128 rows of the 256 x 256 tile.
+    // ------------------------------------------------------------------
+    const int quad = warp & 3;
+    int local = 0;
+    for (int t = cluster_id; t < p.num_tiles; t += num_clusters, ++local) {
+      int m_blk, n_blk;
+      tile_coords(p, t, m_blk, n_blk);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      const bool ready = mbar_wait(&acc_full_bar[acc], acc_phase, abort_flag, p.wait_budget_ns, 0x46);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tcgen05_fence_after_sync();
+      const int row = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM + quad * 32 + lane;
+      const bool row_ok = row < p.M;
+      __half* crow = p.C + static_cast<int64_t>(row) * p.N;
+#pragma unroll 1
+      for (int c = 0; c < Cfg::BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + c * 32, r);
+        tmem_ld_wait();
+        const int col0 = n_blk * Cfg::BN + c * 32;
+        if (row_ok && col0 < p.N) {
+          uint32_t h[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = __uint_as_float(r[2 * e]);
+            const float x1 = __uint_as_float(r[2 * e + 1]);
+            const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
+            h[e] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        }
+      }
+      tcgen05_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
+    }
+  }
+
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // the pair is done with each other's shared memory and barriers
+  if (warp == Cfg::MMA_WARP) {
+    tcgen05_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace tg

@@ -15,6 +15,7 @@
 #include "../../include/tg_gemm.h"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc_pair.cuh"
 #include "ptx.cuh"
 
 namespace tg {
@@ -31,6 +32,7 @@ struct DeviceInfo {
   bool tc_attr = false;
   bool tc_edge_attr = false;
   bool skinny_attr = false;
+  bool tc_pair_attr = false;
 };
 
 std::mutex g_mutex;
@@ -80,6 +82,7 @@ bool path_supports(int path, const void* A, const void* B, const void* C, int64_
     case TG_PATH_TC_EDGE:
       return true;
     case TG_PATH_TC:
+    case TG_PATH_TC_PAIR:
       return aligned16(A, B, C, N, K);
     case TG_PATH_SKINNY:
       return aligned16(A, B, C, N, K) && M <= kSkinnyMaxM;
@@ -92,7 +95,7 @@ int select_path(const void* A, const void* B, const void* C, int64_t M, int64_t 
   if (!args_valid(A, B, C, M, N, K)) return -2;
   if (M == 0 || N == 0) return TG_PATH_NONE;
   if (K == 0) return TG_PATH_ZERO;
-  if (aligned16(A, B, C, N, K)) return M <= kSkinnyMaxM ? TG_PATH_SKINNY : TG_PATH_TC;
+  if (aligned16(A, B, C, N, K)) return M <= kSkinnyMaxM ? TG_PATH_SKINNY : TG_PATH_TC_PAIR;
   return TG_PATH_TC_EDGE;
 }
 
@@ -195,6 +198,61 @@ tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N,
   const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
   kernel<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
   return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+}
+
+// 2-CTA path: 256 x 256 tiles on SM pairs, clusters of 2 along x.
+tg_status launch_tc_pair(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                         cudaStream_t stream, DeviceInfo* info) {
+  using Cfg = TcPairCfg;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!info->tc_pair_attr) {
+      if (cudaFuncSetAttribute(gemm_relu_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::SMEM_BYTES) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      info->tc_pair_attr = true;
+    }
+  }
+  CUtensorMap ta, tb;
+  if (!encode_2d(&ta, A, M, K, 64, Cfg::BM)) return TG_ERR_LAUNCH;
+  if (!encode_2d(&tb, B, K, N, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+  TcParams p;
+  std::memset(&p, 0, sizeof p);
+  p.A = static_cast<const __half*>(A);
+  p.B = static_cast<const __half*>(B);
+  p.C = static_cast<__half*>(C);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.m_tiles = static_cast<int>((M + Cfg::PAIR_M - 1) / Cfg::PAIR_M);
+  p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
+  p.group_m = 8;
+  p.wait_budget_ns = kWaitBudgetNs;
+  const int pairs = info->sm_count / 2;
+  const int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::SMEM_BYTES);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_relu_tc_pair_kernel, ta, tb, p) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
 }
 
 // Small-M path: grid (S, P) with clusters of S CTAs along K.
@@ -309,6 +367,8 @@ tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64
       return launch_tc<true>(A, B, C, M, N, K, stream, info);
     case TG_PATH_SKINNY:
       return launch_skinny(A, B, C, M, N, K, stream, info);
+    case TG_PATH_TC_PAIR:
+      return launch_tc_pair(A, B, C, M, N, K, stream, info);
     default:
       return TG_ERR_INTERNAL;
   }
@@ -390,6 +450,7 @@ const char* tg_path_name(int path) {
     case TG_PATH_SKINNY: return "skinny";
     case TG_PATH_GEMV: return "gemv";
     case TG_PATH_ZERO: return "zero";
+    case TG_PATH_TC_PAIR: return "tc_pair";
     default: return "invalid";
   }
 }
