@@ -34,11 +34,17 @@ from tiled_dense_gemm_fp16_b200 import inputs  # noqa: E402
 METRIC = "GEMM+ReLU TFLOP/s at 8192³ fp16 (1×B200) and % of dense FP16 tensor peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Sources of the dominant kernel; the committed ncu traffic figure is only
+# Sources of each kernel path; a committed ncu traffic figure is only
 # reported while these are unchanged.
-KERNEL_SOURCES = ["tiled_dense_gemm_fp16_b200/csrc/gemm_tc.cuh", "tiled_dense_gemm_fp16_b200/csrc/ptx.cuh"]
-KERNEL_SOURCES_BY_PATH = {"tc_pair": KERNEL_SOURCES + ["tiled_dense_gemm_fp16_b200/csrc/gemm_tc_pair.cuh"]}
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "gemm_relu_tc_square8192.md")
+_CSRC = "tiled_dense_gemm_fp16_b200/csrc/"
+KERNEL_SOURCES = {
+    "tc": [_CSRC + "gemm_tc.cuh", _CSRC + "ptx.cuh"],
+    "tc_edge": [_CSRC + "gemm_tc.cuh", _CSRC + "ptx.cuh"],
+    "tc_pair": [_CSRC + "gemm_tc.cuh", _CSRC + "gemm_tc_pair.cuh", _CSRC + "ptx.cuh"],
+    "tc_pair512": [_CSRC + "gemm_tc.cuh", _CSRC + "gemm_tc_pair.cuh", _CSRC + "ptx.cuh"],
+    "skinny": [_CSRC + "gemm_skinny.cuh", _CSRC + "ptx.cuh"],
+}
+PROFILES = os.path.join(ROOT, "profiles")
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -157,22 +163,24 @@ class ClockSampler:
 # ncu traffic figure (committed summary), valid only for unchanged sources
 # ---------------------------------------------------------------------------
 
-def kernel_source_sha():
+def kernel_source_sha(path_name: str):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES.get(path_name, []):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload: str):
-    if not os.path.exists(TRAFFIC_SUMMARY):
+def committed_traffic(path_name: str, workload: str):
+    """DRAM bytes per launch from profiles/gemm_relu_<path>_<workload>.md, if still valid."""
+    summary = os.path.join(PROFILES, f"gemm_relu_{path_name}_{workload.replace(':', '_m')}.md")
+    if not os.path.exists(summary) or path_name not in KERNEL_SOURCES:
         return None
-    text = open(TRAFFIC_SUMMARY).read()
+    text = open(summary).read()
     m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
     m_wl = re.search(r"traffic_workload:\s*(\S+)", text)
     m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not (m_sha and m_b and m_wl) or m_sha.group(1) != kernel_source_sha() or m_wl.group(1) != workload:
+    if not (m_sha and m_b and m_wl) or m_sha.group(1) != kernel_source_sha(path_name) or m_wl.group(1) != workload:
         return None
     return float(m_b.group(1))
 
@@ -280,7 +288,7 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     path = {"auto": tg.Path.AUTO, "tc": tg.Path.TC, "tc_edge": tg.Path.TC_EDGE, "skinny": tg.Path.SKINNY,
-            "gemv": tg.Path.GEMV, "tc_pair": tg.Path.TC_PAIR}[args.path]
+            "gemv": tg.Path.GEMV, "tc_pair": tg.Path.TC_PAIR, "tc_pair512": tg.Path.TC_PAIR512}[args.path]
     name, M, N, K, A, B = workload_problem(args.workload, rank)
     flops = inputs.flops(M, N, K)
 
@@ -391,7 +399,7 @@ def run_ours(args):
     e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
-    if chosen in (tg.Path.TC, tg.Path.TC_EDGE, tg.Path.TC_PAIR) and name.startswith("square"):
+    if chosen in (tg.Path.TC, tg.Path.TC_EDGE, tg.Path.TC_PAIR, tg.Path.TC_PAIR512) and name.startswith("square"):
         bound, unit_r = "tensor", "TFLOP/s"
         achieved = flops / (kern_avg_ms * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
@@ -401,7 +409,7 @@ def run_ours(args):
         achieved = inputs.min_bytes(M, N, K) / (kern_avg_ms * 1e-3) / 1e9
         peak = float(peaks["hbm_gbs"])
         peak_note = f"{peak_src} STREAM-copy HBM bandwidth"
-    traffic = committed_traffic(name) if rank == 0 else None
+    traffic = committed_traffic(tg.path_name(chosen), name) if rank == 0 else None
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -66,9 +66,10 @@ typedef enum tg_path {
     TG_PATH_GEMV = 4,    /* CUDA-core kernel for M <= 8; same alignment
                             needs as TC                                     */
     TG_PATH_ZERO = 5,    /* K == 0: C is filled with +0 (empty sum)         */
-    TG_PATH_TC_PAIR = 6  /* the TMA + tcgen05 kernel on SM pairs
+    TG_PATH_TC_PAIR = 6, /* the TMA + tcgen05 kernel on SM pairs
                             (cta_group::2), 256x256 tiles; same alignment
                             needs as TC                                     */
+    TG_PATH_TC_PAIR512 = 7 /* as TC_PAIR with 256x512 tiles                 */
 } tg_path;
 
 /*
@@ -98,7 +99,10 @@ TG_API tg_status tg_gemm_relu_f16_path(const void *A, const void *B, void *C, in
 /*
  * The path tg_gemm_relu_f16 would take for these arguments (a tg_path value;
  * TG_PATH_NONE for an empty C), or -2 when the arguments are invalid.  Host
- * logic only: makes no CUDA call and needs no GPU.
+ * logic only: makes no CUDA call and needs no GPU.  Rules: K == 0 -> ZERO;
+ * rows not 16-byte aligned -> TC_EDGE; M <= 256 -> SKINNY; otherwise the
+ * tensor-core kernel (TC, TC_PAIR or TC_PAIR512) with the least estimated
+ * time from its tile count in waves of a 148-SM device.
  */
 TG_API int tg_select_path(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K);
 

@@ -41,6 +41,7 @@ def test_version_and_strings():
     assert "invalid" in tg.status_string(Status.INVALID_ARG)
     assert tg.path_name(Path.TC) == "tc" and tg.path_name(Path.TC_EDGE) == "tc_edge"
     assert tg.path_name(Path.TC_PAIR) == "tc_pair" and tg.path_name(Path.SKINNY) == "skinny"
+    assert tg.path_name(Path.TC_PAIR512) == "tc_pair512"
     assert tg.status_string(99) == "unknown status"
 
 
@@ -76,8 +77,12 @@ def test_overlap_rejected():
 
 def test_path_selection():
     assert tg.select_path(A0, B0, C0, 128, 128, 0) == Path.ZERO
-    assert tg.select_path(A0, B0, C0, 4096, 4096, 4096) == Path.TC_PAIR
-    assert tg.select_path(A0, B0, C0, 8192, 8192, 8192) == Path.TC_PAIR
+    # Large aligned shapes: the tensor-core kernel whose tile waves cost least.
+    assert tg.select_path(A0, B0, C0, 4096, 4096, 4096) == Path.TC_PAIR512
+    assert tg.select_path(A0, B0, C0, 8192, 8192, 8192) == Path.TC_PAIR512
+    assert tg.select_path(A0, B0, C0, 300, 264, 64) == Path.TC_PAIR       # 4 pair tiles vs 2 wide ones
+    assert tg.select_path(A0, B0, C0, 20000, 256, 64) == Path.TC_PAIR
+    assert tg.select_path(A0, B0, C0, 384, 10240, 64) == Path.TC          # 120 CTA tiles fit one wave
     # Small M with aligned rows: the split-K small-M kernel.
     for M in (1, 16, 64, 256):
         assert tg.select_path(A0, B0, C0, M, 8192, 8192) == Path.SKINNY
@@ -94,6 +99,8 @@ def test_forced_path_requirements():
     assert tg.path_supports(Path.TC, A0, B0, C0, 256, 256, 256)
     assert tg.path_supports(Path.TC_PAIR, A0, B0, C0, 256, 256, 256)
     assert not tg.path_supports(Path.TC_PAIR, A0, B0, C0, 256, 250, 256)
+    assert tg.path_supports(Path.TC_PAIR512, A0, B0, C0, 256, 256, 256)
+    assert not tg.path_supports(Path.TC_PAIR512, A0, B0, C0, 256, 256, 252)
     assert not tg.path_supports(Path.TC, A0, B0, C0, 256, 250, 256)
     assert not tg.path_supports(Path.TC, A0, B0, C0, 256, 256, 250)
     assert tg.path_supports(Path.TC_EDGE, A0, B0, C0, 256, 250, 250)

@@ -15,31 +15,32 @@ from tiled_dense_gemm_fp16_b200._binding import Path
 
 pytestmark = pytest.mark.gpu
 
-TC, EDGE, SKINNY, PAIR = Path.TC, Path.TC_EDGE, Path.SKINNY, Path.TC_PAIR
+TC, EDGE, SKINNY, PAIR, WIDE = Path.TC, Path.TC_EDGE, Path.SKINNY, Path.TC_PAIR, Path.TC_PAIR512
 
 
 def _paths_for(M, N, K):
     paths = [None, EDGE]
     if N % 8 == 0 and K % 8 == 0:
-        paths += [TC, PAIR]
+        paths += [TC, PAIR, WIDE]
         if M <= 256:
             paths.append(SKINNY)
     return paths
 
 
-def test_pair_kernel_single_tile():
-    """One 256 x 256 tile on one SM pair, one 64-deep k-block: the smallest cta_group::2 case."""
-    A, B = inputs.operands(256, 256, 64, "int", seed=12)
-    got, guards = run_gpu(A, B, PAIR)
+@pytest.mark.parametrize("path,N", [(PAIR, 256), (WIDE, 512)], ids=["pair256", "pair512"])
+def test_pair_kernel_single_tile(path, N):
+    """One tile on one SM pair, one 64-deep k-block: the smallest cta_group::2 case."""
+    A, B = inputs.operands(256, N, 64, "int", seed=12)
+    got, guards = run_gpu(A, B, path)
     assert guards
-    assert_bitexact(got, oracle.gemm_relu_f16(A, B), "pair 256x256x64")
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"pair 256x{N}x64")
 
 
 # ---------------------------------------------------------------------------
 # Small square workload (256^3): integer variant bit-exact, uniform within tolerance
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("path", [None, TC, EDGE, PAIR], ids=["auto", "tc", "edge", "pair"])
+@pytest.mark.parametrize("path", [None, TC, EDGE, PAIR, WIDE], ids=["auto", "tc", "edge", "pair", "wide"])
 def test_square256_integer_bitexact(path):
     A, B = inputs.operands(256, 256, 256, "int", seed=0)
     got, guards = run_gpu(A, B, path)
@@ -47,7 +48,7 @@ def test_square256_integer_bitexact(path):
     assert_bitexact(got, oracle.gemm_relu_f16(A, B), "square256 int")
 
 
-@pytest.mark.parametrize("path", [None, TC, EDGE, PAIR], ids=["auto", "tc", "edge", "pair"])
+@pytest.mark.parametrize("path", [None, TC, EDGE, PAIR, WIDE], ids=["auto", "tc", "edge", "pair", "wide"])
 def test_square256_uniform(path):
     (shape, A, B), = inputs.WORKLOADS["square256"].problems()
     got, guards = run_gpu(A, B, path)
@@ -112,13 +113,16 @@ def test_skinny_uniform(M, N, K):
     assert_close(got, ref, f"skinny {(M, N, K)}")
 
 
-def test_misaligned_base_pointers_use_edge_mode():
-    """Bases 2 bytes off a 16-byte boundary: TMA cannot take them; the edge mode can."""
-    A, B = inputs.operands(200, 136, 72, "int", seed=2)
+@pytest.mark.parametrize("offset", [1, 2, 3, 5, 7])
+@pytest.mark.parametrize("M,N,K", [(200, 136, 72), (131, 257, 199)])
+def test_misaligned_base_pointers_use_edge_mode(offset, M, N, K):
+    """Bases 2*offset bytes off a 16-byte boundary: TMA cannot take them; the
+    edge mode realigns rows from aligned 16-byte loads (every shift 2..14 B)."""
+    A, B = inputs.operands(M, N, K, "int", seed=2 + offset)
     ref = oracle.gemm_relu_f16(A, B)
-    got, guards = run_gpu(A, B, None, offset_elems=1)
+    got, guards = run_gpu(A, B, None, offset_elems=offset)
     assert guards
-    assert_bitexact(got, ref, "offset 1")
+    assert_bitexact(got, ref, f"offset {offset}")
 
 
 # ---------------------------------------------------------------------------
@@ -152,7 +156,7 @@ def test_special_values():
     B[:, 8:16] = -2.0                             # -65536 -> ReLU -> +0
     B[:4095, 16:24] = 0.0                         # 4 * 12289 = 49156 -> 49152 (nearest even half)
     ref = oracle.gemm_relu_f16(A, B)
-    for path in (TC, EDGE, PAIR):
+    for path in (TC, EDGE, PAIR, WIDE):
         got, _ = run_gpu(A, B, path)
         assert_bitexact(got, ref, f"special path={path}")
     assert np.all(np.isinf(ref[:, :8].astype(np.float32))) and np.all(ref[:, 8:16].view(np.uint16) == 0)
@@ -194,19 +198,19 @@ def _check_workload(name, dist=None, exact=False, full_oracle_max_macs=5e9, path
 
 
 def test_workload_square4096():
-    _check_workload("square4096", paths=(None, TC, EDGE))
+    _check_workload("square4096", paths=(None, TC, PAIR, EDGE))
 
 
 def test_workload_square4096_integer():
-    _check_workload("square4096", dist="int", exact=True, paths=(None, TC))
+    _check_workload("square4096", dist="int", exact=True, paths=(None, TC, PAIR))
 
 
 def test_workload_square8192():
-    _check_workload("square8192", paths=(None, TC))
+    _check_workload("square8192", paths=(None, TC, PAIR))
 
 
 def test_workload_square8192_integer():
-    _check_workload("square8192", dist="int", exact=True, paths=(None, TC))
+    _check_workload("square8192", dist="int", exact=True, paths=(None, TC, PAIR))
 
 
 def test_workload_skinny():

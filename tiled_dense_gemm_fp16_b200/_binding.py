@@ -35,6 +35,7 @@ class Path(enum.IntEnum):
     GEMV = 4
     ZERO = 5
     TC_PAIR = 6
+    TC_PAIR512 = 7
 
 
 class TGError(RuntimeError):

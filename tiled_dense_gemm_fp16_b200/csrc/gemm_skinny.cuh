@@ -36,6 +36,7 @@ struct SkinnyParams {
   uint32_t a_stage_bytes; // m_pad * 128
   uint32_t tmem_cols;     // power of two >= max(32, m_pad)
   uint32_t idesc;
+  int prefetch_kb;        // > 0: also prefetch into L2 the B boxes this many k-blocks ahead
   uint64_t wait_budget_ns;
 };
 
@@ -117,6 +118,11 @@ __global__ void __launch_bounds__(SkinnyCfg::THREADS, 1)
         tma_load_2d(bdst, &tmap_b, &full_bar[stage], n0, k0);
         tma_load_2d(bdst + Cfg::B_BOX_BYTES, &tmap_b, &full_bar[stage], n0 + 64, k0);
         tma_load_2d(a_smem + stage * p.a_stage_bytes, &tmap_a, &full_bar[stage], k0, 0);
+        if (p.prefetch_kb > 0 && kb + p.prefetch_kb < kb_hi) {
+          const int kp = (kb + p.prefetch_kb) * Cfg::BK;
+          tma_prefetch_l2_2d(&tmap_b, n0, kp);
+          tma_prefetch_l2_2d(&tmap_b, n0 + 64, kp);
+        }
         last_parity[stage] = static_cast<int>(phase);
         if (++stage == p.stages) {
           stage = 0;

@@ -40,6 +40,9 @@ struct TcParams {
   int M, N, K;
   int m_tiles, n_tiles, num_tiles, k_blocks;
   int group_m;           // tile rows per raster group
+  int store_streaming;   // 1: C stores with the streaming (evict-first) cache hint
+  int l2_hints;          // bit 0: A loads evict-last; bit 1: B loads evict-last; bit 2: B loads evict-first
+  int prefetch_kb;       // > 0: also prefetch into L2 the boxes this many k-blocks ahead
   uint64_t wait_budget_ns;
 };
 
@@ -49,7 +52,7 @@ struct TcCfg {
   static constexpr int BN = 256;
   static constexpr int BK = 64;
   static constexpr int STAGES = 4;
-  static constexpr int PRODUCER_WARPS = EDGE ? 4 : 1;
+  static constexpr int PRODUCER_WARPS = EDGE ? 8 : 1;
   static constexpr int MMA_WARP = PRODUCER_WARPS;
   static constexpr int EPI_WARP0 = MMA_WARP + 1;
   static constexpr int EPI_WARPS = 4;
@@ -83,7 +86,7 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
 }
 
 // EDGE mode: one 16-byte chunk of 8 consecutive fp16 values from a row-major
-// matrix, zero where (row >= rows) or (col >= cols).
+// matrix, zero where (row >= rows) or (col >= cols).  Scalar reference form.
 __device__ __forceinline__ uint4 load_chunk_pred(const __half* base, int64_t ld, int row, int rows, int col,
                                                  int cols) {
   uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -97,6 +100,50 @@ __device__ __forceinline__ uint4 load_chunk_pred(const __half* base, int64_t ld,
     }
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// EDGE mode, fast form of load_chunk_pred for rows whose start is only
+// 2-byte aligned, split so that a thread can issue the loads of several
+// chunks before it uses any of them.  When the 8 values lie inside the row
+// and the two 16-byte aligned blocks that cover them lie inside
+// [base, end), the chunk is read with two aligned 16-byte loads and shifted
+// into place; otherwise the caller falls back to the scalar form.  No byte
+// outside [base, end) is ever read.
+struct EdgeChunk {
+  const uint4* src;  // first aligned block (valid when fast)
+  uint32_t shift;    // byte offset of the chunk in the 32 loaded bytes: 0, 2, ..., 14
+  bool fast;
+};
+
+__device__ __forceinline__ EdgeChunk edge_chunk_plan(const __half* base, const __half* end, int64_t ld, int row,
+                                                     int rows, int col, int cols) {
+  EdgeChunk c;
+  c.fast = false;
+  c.shift = 0;
+  c.src = reinterpret_cast<const uint4*>(base);
+  if (row < rows && col + 8 <= cols) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(base + static_cast<int64_t>(row) * ld + col);
+    const uintptr_t a0 = a & ~uintptr_t(15);
+    if (a0 >= reinterpret_cast<uintptr_t>(base) && a0 + 32 <= reinterpret_cast<uintptr_t>(end)) {
+      c.fast = true;
+      c.src = reinterpret_cast<const uint4*>(a0);
+      c.shift = static_cast<uint32_t>(a - a0);
+    }
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint4 edge_realign(const uint4& lo, const uint4& hi, uint32_t sh) {
+  uint32_t w0 = lo.x, w1 = lo.y, w2 = lo.z, w3 = lo.w, w4 = hi.x, w5 = hi.y, w6 = hi.z, w7 = hi.w;
+  if (sh & 8u) {
+    w0 = w2; w1 = w3; w2 = w4; w3 = w5; w4 = w6; w5 = w7;
+  }
+  if (sh & 4u) {
+    w0 = w1; w1 = w2; w2 = w3; w3 = w4; w4 = w5;
+  }
+  const uint32_t bits = (sh & 2u) * 8u;  // 0 or 16
+  return make_uint4(__funnelshift_r(w0, w1, bits), __funnelshift_r(w1, w2, bits), __funnelshift_r(w2, w3, bits),
+                    __funnelshift_r(w3, w4, bits));
 }
 
 template <bool EDGE>
@@ -193,11 +240,14 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
         }
       }
     } else {
-      const int ptid = threadIdx.x;  // 0 .. 127
+      const int ptid = threadIdx.x;  // 0 .. PRODUCER_THREADS - 1
+      constexpr int kThreads = Cfg::PRODUCER_WARPS * 32;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       const int64_t lda = p.K, ldb = p.N;
+      const __half* a_end = p.A + static_cast<int64_t>(p.M) * p.K;
+      const __half* b_end = p.B + static_cast<int64_t>(p.K) * p.N;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         int m_blk, n_blk;
         tile_coords(p, t, m_blk, n_blk);
@@ -210,23 +260,60 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
             break;
           }
           const int k0 = kb * Cfg::BK;
-          uint8_t* adst = a_smem + stage * Cfg::A_BYTES;
-          uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
-          // A tile: 128 rows x 8 chunks.
-#pragma unroll 4
-          for (int i = 0; i < (Cfg::BM * 8) / 128; ++i) {
-            const int c = ptid + i * 128;
-            const int r = c >> 3, kc = c & 7;
-            const uint4 v = load_chunk_pred(p.A, lda, m0 + r, p.M, k0 + kc * 8, p.K);
-            *reinterpret_cast<uint4*>(adst + sw128_offset(r, kc)) = v;
-          }
-          // B tile: 64 k-rows x 32 chunks, in 4 panels of 64 columns.
-#pragma unroll 4
-          for (int i = 0; i < (Cfg::BK * 32) / 128; ++i) {
-            const int c = ptid + i * 128;
-            const int kr = c >> 5, nc = c & 31;
-            const uint4 v = load_chunk_pred(p.B, ldb, k0 + kr, p.K, n0 + nc * 8, p.N);
-            *reinterpret_cast<uint4*>(bdst + (nc >> 3) * Cfg::B_CHUNK_BYTES + sw128_offset(kr, nc & 7)) = v;
+          // Each producer thread stages 4 chunks of the A tile (128 rows x 8
+          // chunks, 8 consecutive threads per row) and 8 of the B tile (64
+          // k-rows x 32 chunks, one warp per k-row), in batches whose loads
+          // are all in flight before any is used.
+          constexpr int kA = (Cfg::BM * 8) / kThreads;
+          constexpr int kB = (Cfg::BK * 32) / kThreads;
+          constexpr int kBatch = 6;
+          static_assert((kA + kB) % kBatch == 0, "batching");
+#pragma unroll
+          for (int b0 = 0; b0 < kA + kB; b0 += kBatch) {
+            EdgeChunk plan[kBatch];
+            uint32_t dst_off[kBatch];
+            int row_of[kBatch], col_of[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int j = b0 + u;
+              if (j < kA) {
+                const int c = ptid + j * kThreads;
+                const int r = c >> 3, kc = c & 7;
+                row_of[u] = m0 + r;
+                col_of[u] = k0 + kc * 8;
+                dst_off[u] = static_cast<uint32_t>(stage * Cfg::A_BYTES) + sw128_offset(r, kc);
+                plan[u] = edge_chunk_plan(p.A, a_end, lda, row_of[u], p.M, col_of[u], p.K);
+              } else {
+                const int c = ptid + (j - kA) * kThreads;
+                const int kr = c >> 5, nc = c & 31;
+                row_of[u] = k0 + kr;
+                col_of[u] = n0 + nc * 8;
+                dst_off[u] = static_cast<uint32_t>(stage * Cfg::B_BYTES + (nc >> 3) * Cfg::B_CHUNK_BYTES) +
+                             sw128_offset(kr, nc & 7);
+                plan[u] = edge_chunk_plan(p.B, b_end, ldb, row_of[u], p.K, col_of[u], p.N);
+              }
+            }
+            uint4 lo[kBatch], hi[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              lo[u] = make_uint4(0u, 0u, 0u, 0u);
+              hi[u] = lo[u];
+              ld_nc_v4_pred(lo[u], plan[u].src, plan[u].fast);
+              ld_nc_v4_pred(hi[u], plan[u].src + 1, plan[u].fast);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+              const int j = b0 + u;
+              uint4 v;
+              if (plan[u].fast) {
+                v = edge_realign(lo[u], hi[u], plan[u].shift);
+              } else if (j < kA) {
+                v = load_chunk_pred(p.A, lda, row_of[u], p.M, col_of[u], p.K);
+              } else {
+                v = load_chunk_pred(p.B, ldb, row_of[u], p.K, col_of[u], p.N);
+              }
+              *reinterpret_cast<uint4*>((j < kA ? a_smem : b_smem) + dst_off[u]) = v;
+            }
           }
           fence_proxy_async_smem();
           mbar_arrive(&full_bar[stage]);
@@ -323,10 +410,25 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
             for (int q = 0; q < 4; ++q)
               if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
           } else {
+            // Rows are only 2-byte aligned: 4-byte stores of aligned pairs,
+            // 2-byte stores at a misaligned start and at the end of C.
             unsigned short* dst = reinterpret_cast<unsigned short*>(crow + col0);
+            const int n_here = min(32, p.N - col0);
+            if ((reinterpret_cast<uintptr_t>(dst) & 2u) == 0) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (col0 + e < p.N) dst[e] = static_cast<unsigned short>((h[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+              for (int q = 0; q < 16; ++q)
+                if (2 * q + 1 < n_here) reinterpret_cast<uint32_t*>(dst)[q] = h[q];
+              if (n_here & 1)
+                dst[n_here - 1] = static_cast<unsigned short>(h[(n_here - 1) >> 1] & 0xffffu);
+            } else {
+              dst[0] = static_cast<unsigned short>(h[0] & 0xffffu);
+              uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + 1);
+#pragma unroll
+              for (int q = 0; q < 15; ++q)
+                if (2 * q + 2 < n_here) d32[q] = __funnelshift_r(h[q], h[q + 1], 16);
+              if (n_here >= 2 && (n_here & 1) == 0)
+                dst[n_here - 1] = static_cast<unsigned short>(h[(n_here - 1) >> 1] >> 16);
+            }
           }
         }
       }

@@ -1,24 +1,28 @@
 // gemm_tc_pair.cuh -- the persistent tcgen05 GEMM + ReLU kernel on CTA pairs
-// (cta_group::2): 256 x 256 output tiles, each computed by the two SMs of a
-// 2-CTA cluster.
+// (cta_group::2): 256 x BN output tiles (BN = 256 or 512), each computed by
+// the two SMs of a 2-CTA cluster.
 //
 // Same tile model as gemm_tc.cuh (the matmul_relu quick-start kernel: tiles
 // staged through a pipelined K loop, cleared fp32 accumulator, tile MMAs,
 // max(acc, 0), fp16 output), with the MMA spread over an SM pair:
 //   * CTA r of the pair (r = 0, 1) loads rows [128 r, 128 r + 128) of the
-//     A tile and columns [128 r, 128 r + 128) of the B tile into its own
-//     shared memory (TMA, 128-byte swizzle, no multicast), 32 KiB per stage,
-//     6 stages;
+//     A tile and, of every 256-column slab of the B tile, the columns
+//     [128 r, 128 r + 128) into its own shared memory (TMA, 128-byte swizzle,
+//     no multicast): 32 KiB per stage and 6 stages for BN = 256, 48 KiB per
+//     stage and 4 stages for BN = 512;
 //   * both CTAs' loads count their bytes on the even CTA's "full" barrier;
-//     the even CTA's single MMA thread issues 256 x 256 x 16 pair MMAs that
-//     read both CTAs' shared memory and write both CTAs' TMEM (rows
-//     [128 r, 128 r + 128) of the tile land in CTA r);
+//     the even CTA's single MMA thread issues BN / 256 pair MMAs of
+//     256 x 256 x 16 per k-step that read both CTAs' shared memory and write
+//     both CTAs' TMEM (rows [128 r, 128 r + 128) of the tile land in CTA r);
+//     BN = 256 double-buffers the accumulator (2 x 256 columns), BN = 512
+//     uses all 512 columns for one accumulator;
 //   * the MMA commits multicast to both CTAs' "empty" barriers (each CTA then
 //     refills its own stage) and, per tile, to both CTAs' "accumulator full"
 //     barriers; the eight epilogue warps of the pair release the accumulator
 //     on the even CTA's "accumulator empty" barrier;
 //   * per SM, each 64-deep k-block moves 32 KiB from L2 for 128 x 256 x 64
-//     MACs, two thirds of the 48 KiB the single-CTA 128 x 256 tile needs.
+//     MACs at BN = 256 (two thirds of what the single-CTA 128 x 256 tile
+//     needs) and 48 KiB for 128 x 512 x 64 MACs at BN = 512 (one half).
 // Every wait is bounded; a cluster barrier brackets the kernel so that no
 // CTA exits while its peer may still touch its shared memory or barriers.
 #pragma once
@@ -30,31 +34,37 @@
 
 namespace tg {
 
+template <int STAGES_, int BN_>
 struct TcPairCfg {
   static constexpr int BM = 128;        // rows per CTA (the pair tile is 256)
   static constexpr int PAIR_M = 256;
-  static constexpr int BN = 256;        // columns per pair tile
-  static constexpr int BN_HALF = 128;   // columns of B each CTA loads
+  static constexpr int BN = BN_;        // columns per pair tile: 256 or 512
+  static constexpr int SLABS = BN / 256;          // pair MMAs per k-step
+  static constexpr int BN_HALF = BN / 2;          // columns of B each CTA loads
   static constexpr int BK = 64;
-  static constexpr int STAGES = 6;
-  static constexpr int THREADS = 192;   // producer, MMA, 4 epilogue warps
+  static constexpr int STAGES = STAGES_;
   static constexpr int MMA_WARP = 1;
   static constexpr int EPI_WARP0 = 2;
-  static constexpr int EPI_WARPS = 4;
+  static constexpr int EPI_WARPS = 4 * SLABS;     // 4 per 256-column slab
+  static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
   static constexpr int A_BYTES = BM * BK * 2;        // 16 KiB
-  static constexpr int B_BYTES = BK * BN_HALF * 2;   // 16 KiB
+  static constexpr int B_BYTES = BK * BN_HALF * 2;   // 16 or 32 KiB
   static constexpr int B_CHUNK_BYTES = BK * 64 * 2;  // 8 KiB panel of 64 columns
-  static constexpr int NUM_ACC = 2;
+  static constexpr int B_SLAB_BYTES = 2 * B_CHUNK_BYTES;  // this CTA's 128 columns of one slab
+  static constexpr int NUM_ACC = (BN == 256) ? 2 : 1;
   static constexpr int TMEM_COLS = 512;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + BAR_BYTES;
-  static constexpr uint32_t IDESC = make_idesc_f16_f32(PAIR_M, BN, false, true);
+  static constexpr uint32_t IDESC = make_idesc_f16_f32(PAIR_M, 256, false, true);
+  static_assert(BN == 256 || BN == 512, "pair tile width");
+  static_assert(NUM_ACC * BN <= TMEM_COLS, "TMEM columns");
 };
 
-__global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
+template <int STAGES, int BN>
+__global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
     gemm_relu_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                              const TcParams p) {
-  using Cfg = TcPairCfg;
+  using Cfg = TcPairCfg<STAGES, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_smem = smem;
@@ -111,11 +121,16 @@ __global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
 #pragma unroll
       for (int s = 0; s < Cfg::STAGES; ++s) last_parity[s] = -1;
       bool ok = true;
+      const uint64_t pol_a = (p.l2_hints & 1) ? l2_policy_evict_last() : l2_policy_evict_normal();
+      const uint64_t pol_b = (p.l2_hints & 2)   ? l2_policy_evict_last()
+                             : (p.l2_hints & 4) ? l2_policy_evict_first()
+                                                : l2_policy_evict_normal();
       for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters) {
         int m_blk, n_blk;
         tile_coords(p, t, m_blk, n_blk);
         const int m0 = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM;
-        const int nb = n_blk * Cfg::BN + static_cast<int>(rank) * Cfg::BN_HALF;
+        // This CTA's 128 columns of slab j start at n0 + 256 j + 128 r.
+        const int nb = n_blk * Cfg::BN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 0x41)) {
             ok = false;
@@ -125,9 +140,24 @@ __global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
           const int k0 = kb * Cfg::BK;
           uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
-          tma_load_2d_pair(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, k0, m0);
-          tma_load_2d_pair(bdst, &tmap_b, full_even, nb, k0);
-          tma_load_2d_pair(bdst + Cfg::B_CHUNK_BYTES, &tmap_b, full_even, nb + 64, k0);
+          tma_load_2d_pair_hint(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, k0, m0, pol_a);
+#pragma unroll
+          for (int j = 0; j < Cfg::SLABS; ++j) {
+            tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, nb + 256 * j, k0, pol_b);
+            tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES + Cfg::B_CHUNK_BYTES, &tmap_b, full_even,
+                                  nb + 256 * j + 64, k0, pol_b);
+          }
+          if (p.prefetch_kb > 0 && kb + p.prefetch_kb < p.k_blocks) {
+            // Warm L2 with the boxes a few k-blocks ahead, so the ring's
+            // loads find them there instead of waiting on HBM.
+            const int kp = (kb + p.prefetch_kb) * Cfg::BK;
+            tma_prefetch_l2_2d(&tmap_a, kp, m0);
+#pragma unroll
+            for (int j = 0; j < Cfg::SLABS; ++j) {
+              tma_prefetch_l2_2d(&tmap_b, nb + 256 * j, kp);
+              tma_prefetch_l2_2d(&tmap_b, nb + 256 * j + 64, kp);
+            }
+          }
           last_parity[stage] = static_cast<int>(phase);
           if (++stage == Cfg::STAGES) {
             stage = 0;
@@ -157,8 +187,8 @@ __global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
       int local = 0;
       bool ok = true;
       for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters, ++local) {
-        const int acc = local & 1;
-        const uint32_t acc_phase = (local >> 1) & 1;
+        const int acc = local % Cfg::NUM_ACC;
+        const uint32_t acc_phase = (local / Cfg::NUM_ACC) & 1;
         if (!mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, abort_flag, p.wait_budget_ns, 0x43)) break;
         tcgen05_fence_after_sync();
         const uint32_t d_tmem = tmem_base + acc * Cfg::BN;
@@ -173,8 +203,13 @@ __global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < Cfg::BK / 16; ++k) {
             const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
-            const uint64_t bdesc = make_sw128_desc(b_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
-            umma_f16_ss_pair(d_tmem, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int j = 0; j < Cfg::SLABS; ++j) {
+              // Slab j: this CTA's two 64-column panels, 8 KiB apart.
+              const uint64_t bdesc =
+                  make_sw128_desc(b_addr + j * Cfg::B_SLAB_BYTES + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
+              umma_f16_ss_pair(d_tmem + 256 * j, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
+            }
           }
           umma_commit_pair_mc(&empty_bar[stage], 0x3);  // both CTAs may refill this stage
           if (++stage == Cfg::STAGES) {
@@ -192,15 +227,17 @@ __global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------
-    // Epilogue (both CTAs): this CTA's 128 rows of the 256 x 256 tile.
+    // Epilogue (both CTAs): this CTA's 128 rows of the 256 x BN tile; warp
+    // w reads TMEM lanes 32 (w mod 4) .. + 31 of slab (w - 2) / 4.
     // ------------------------------------------------------------------
     const int quad = warp & 3;
+    const int slab = (warp - Cfg::EPI_WARP0) >> 2;
     int local = 0;
     for (int t = cluster_id; t < p.num_tiles; t += num_clusters, ++local) {
       int m_blk, n_blk;
       tile_coords(p, t, m_blk, n_blk);
-      const int acc = local & 1;
-      const uint32_t acc_phase = (local >> 1) & 1;
+      const int acc = local % Cfg::NUM_ACC;
+      const uint32_t acc_phase = (local / Cfg::NUM_ACC) & 1;
       const bool ready = mbar_wait(&acc_full_bar[acc], acc_phase, abort_flag, p.wait_budget_ns, 0x46);
       if (!__all_sync(0xffffffffu, ready)) break;
       tcgen05_fence_after_sync();
@@ -208,11 +245,12 @@ __global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
       const bool row_ok = row < p.M;
       __half* crow = p.C + static_cast<int64_t>(row) * p.N;
 #pragma unroll 1
-      for (int c = 0; c < Cfg::BN / 32; ++c) {
+      for (int c = 0; c < 256 / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + c * 32, r);
+        const int tcol = slab * 256 + c * 32;  // column within this CTA's accumulator
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + tcol, r);
         tmem_ld_wait();
-        const int col0 = n_blk * Cfg::BN + c * 32;
+        const int col0 = n_blk * Cfg::BN + tcol;
         if (row_ok && col0 < p.N) {
           uint32_t h[16];
 #pragma unroll
@@ -223,9 +261,16 @@ __global__ void __launch_bounds__(TcPairCfg::THREADS, 1)
             h[e] = *reinterpret_cast<const uint32_t*>(&v);
           }
           uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+          if (p.store_streaming) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+              if (col0 + q * 8 < p.N)
+                __stcs(reinterpret_cast<int4*>(dst + q), make_int4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+          }
         }
       }
       tcgen05_fence_before_sync();

@@ -9,10 +9,11 @@
 
 #include <climits>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
-#include "../../include/tg_gemm.h"
+#include "tg_gemm.h"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc_pair.cuh"
@@ -32,11 +33,18 @@ struct DeviceInfo {
   bool tc_attr = false;
   bool tc_edge_attr = false;
   bool skinny_attr = false;
-  bool tc_pair_attr = false;
+  unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
 };
 
 std::mutex g_mutex;
 DeviceInfo g_devices[kMaxDevices];
+
+// Tuning knobs for experiments (environment, read on each launch); the
+// defaults are the tuned values.
+int tune_int(const char* name, int dflt) {
+  const char* v = std::getenv(name);
+  return (v && *v) ? std::atoi(v) : dflt;
+}
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 bool g_encode_probed = false;
 
@@ -83,6 +91,7 @@ bool path_supports(int path, const void* A, const void* B, const void* C, int64_
       return true;
     case TG_PATH_TC:
     case TG_PATH_TC_PAIR:
+    case TG_PATH_TC_PAIR512:
       return aligned16(A, B, C, N, K);
     case TG_PATH_SKINNY:
       return aligned16(A, B, C, N, K) && M <= kSkinnyMaxM;
@@ -91,12 +100,27 @@ bool path_supports(int path, const void* A, const void* B, const void* C, int64_
   }
 }
 
+// Estimated relative time of the three tensor-core kernels for an M x N
+// output on a 148-SM device: waves of tiles x per-SM work of one tile /
+// measured relative efficiency (single CTA 0.90, pair 256x256 0.95,
+// pair 256x512 1.0 at 8192^3).  K scales all three alike.
+int pick_tc_kernel(int64_t M, int64_t N) {
+  constexpr int64_t kSms = 148, kPairs = 74;
+  auto waves = [](int64_t tiles, int64_t units) { return (tiles + units - 1) / units; };
+  const double t1 = waves(((M + 127) / 128) * ((N + 255) / 256), kSms) * (128.0 * 256.0) / 0.90;
+  const double t2 = waves(((M + 255) / 256) * ((N + 255) / 256), kPairs) * (128.0 * 256.0) / 0.95;
+  const double t3 = waves(((M + 255) / 256) * ((N + 511) / 512), kPairs) * (128.0 * 512.0) / 1.0;
+  if (t3 <= t2 && t3 <= t1) return TG_PATH_TC_PAIR512;
+  return t2 <= t1 ? TG_PATH_TC_PAIR : TG_PATH_TC;
+}
+
 int select_path(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
   if (!args_valid(A, B, C, M, N, K)) return -2;
   if (M == 0 || N == 0) return TG_PATH_NONE;
   if (K == 0) return TG_PATH_ZERO;
-  if (aligned16(A, B, C, N, K)) return M <= kSkinnyMaxM ? TG_PATH_SKINNY : TG_PATH_TC_PAIR;
-  return TG_PATH_TC_EDGE;
+  if (!aligned16(A, B, C, N, K)) return TG_PATH_TC_EDGE;
+  if (M <= kSkinnyMaxM) return TG_PATH_SKINNY;
+  return pick_tc_kernel(M, N);
 }
 
 // ---------------------------------------------------------------------------
@@ -193,7 +217,11 @@ tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N,
   p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
-  p.group_m = 16;
+  p.group_m = tune_int("TG_TUNE_GROUP_M", 16);
+  if (p.group_m < 1) p.group_m = 1;
+  p.store_streaming = 0;
+  p.l2_hints = 0;
+  p.prefetch_kb = 0;
   p.wait_budget_ns = kWaitBudgetNs;
   const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
   kernel<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
@@ -201,18 +229,21 @@ tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N,
 }
 
 // 2-CTA path: 256 x 256 tiles on SM pairs, clusters of 2 along x.
-tg_status launch_tc_pair(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
-                         cudaStream_t stream, DeviceInfo* info) {
-  using Cfg = TcPairCfg;
+template <int STAGES, int BN>
+tg_status launch_tc_pair_cfg(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                             cudaStream_t stream, DeviceInfo* info) {
+  using Cfg = TcPairCfg<STAGES, BN>;
+  auto kernel = gemm_relu_tc_pair_kernel<STAGES, BN>;
+  constexpr unsigned kAttrBit = 1u << (STAGES + (BN == 512 ? 16 : 0));
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!info->tc_pair_attr) {
-      if (cudaFuncSetAttribute(gemm_relu_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg::SMEM_BYTES) != cudaSuccess) {
+    if (!(info->tc_pair_attr & kAttrBit)) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
+          cudaSuccess) {
         cudaGetLastError();
         return TG_ERR_LAUNCH;
       }
-      info->tc_pair_attr = true;
+      info->tc_pair_attr |= kAttrBit;
     }
   }
   CUtensorMap ta, tb;
@@ -230,7 +261,11 @@ tg_status launch_tc_pair(const void* A, const void* B, void* C, int64_t M, int64
   p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
-  p.group_m = 8;
+  p.group_m = tune_int("TG_TUNE_GROUP_M", BN == 512 ? 16 : 12);
+  if (p.group_m < 1) p.group_m = 1;
+  p.store_streaming = tune_int("TG_TUNE_STORE_CS", 1);
+  p.l2_hints = tune_int("TG_TUNE_L2_HINTS", BN == 512 ? 0 : 5);
+  p.prefetch_kb = tune_int("TG_TUNE_PREFETCH_KB", 0);
   p.wait_budget_ns = kWaitBudgetNs;
   const int pairs = info->sm_count / 2;
   const int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
@@ -248,11 +283,26 @@ tg_status launch_tc_pair(const void* A, const void* B, void* C, int64_t M, int64
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gemm_relu_tc_pair_kernel, ta, tb, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
     cudaGetLastError();
     return TG_ERR_LAUNCH;
   }
   return TG_OK;
+}
+
+tg_status launch_tc_pair(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                         cudaStream_t stream, DeviceInfo* info, int bn) {
+  if (bn == 512) {
+    switch (tune_int("TG_TUNE_PAIR_STAGES", 4)) {
+      case 3: return launch_tc_pair_cfg<3, 512>(A, B, C, M, N, K, stream, info);
+      default: return launch_tc_pair_cfg<4, 512>(A, B, C, M, N, K, stream, info);
+    }
+  }
+  switch (tune_int("TG_TUNE_PAIR_STAGES", 6)) {
+    case 5: return launch_tc_pair_cfg<5, 256>(A, B, C, M, N, K, stream, info);
+    case 7: return launch_tc_pair_cfg<7, 256>(A, B, C, M, N, K, stream, info);
+    default: return launch_tc_pair_cfg<6, 256>(A, B, C, M, N, K, stream, info);
+  }
 }
 
 // Small-M path: grid (S, P) with clusters of S CTAs along K.
@@ -281,7 +331,11 @@ tg_status launch_skinny(const void* A, const void* B, void* C, int64_t M, int64_
   p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
   // Two CTAs per SM fit while the ring stays within ~112 KiB (M_pad <= 128).
   const bool two_per_sm = p.m_pad <= 128;
-  const int budget = (two_per_sm ? 112 : 220) * 1024;
+  // Measured: M_pad <= 32 streams best with a 3-stage ring, larger M_pad
+  // with ~112 KiB (4 stages at M_pad = 64).
+  int budget_kb = tune_int("TG_TUNE_SKINNY_SMEM_KB", p.m_pad <= 32 ? 64 : (two_per_sm ? 112 : 220));
+  budget_kb = budget_kb < 32 ? 32 : (budget_kb > 220 ? 220 : budget_kb);
+  const int budget = budget_kb * 1024;
   const int stage_bytes = Cfg::stage_bytes(p.m_pad);
   int stages = budget / stage_bytes;
   stages = stages > 8 ? 8 : stages;
@@ -294,10 +348,11 @@ tg_status launch_skinny(const void* A, const void* B, void* C, int64_t M, int64_
   while (cols < static_cast<uint32_t>(p.m_pad)) cols <<= 1;
   p.tmem_cols = cols;
   p.idesc = make_idesc_f16_f32(Cfg::PANEL, p.m_pad, true, false);
+  p.prefetch_kb = tune_int("TG_TUNE_SKINNY_PREFETCH_KB", 0);
   p.wait_budget_ns = kWaitBudgetNs;
   const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);
   const int slots = (two_per_sm ? 2 : 1) * info->sm_count;
-  int splits = slots / panels;
+  int splits = tune_int("TG_TUNE_SKINNY_SPLITS", slots / panels);
   splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
   if (splits > p.k_blocks) splits = p.k_blocks;
   p.splits = splits;
@@ -368,7 +423,9 @@ tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64
     case TG_PATH_SKINNY:
       return launch_skinny(A, B, C, M, N, K, stream, info);
     case TG_PATH_TC_PAIR:
-      return launch_tc_pair(A, B, C, M, N, K, stream, info);
+      return launch_tc_pair(A, B, C, M, N, K, stream, info, 256);
+    case TG_PATH_TC_PAIR512:
+      return launch_tc_pair(A, B, C, M, N, K, stream, info, 512);
     default:
       return TG_ERR_INTERNAL;
   }
@@ -451,6 +508,7 @@ const char* tg_path_name(int path) {
     case TG_PATH_GEMV: return "gemv";
     case TG_PATH_ZERO: return "zero";
     case TG_PATH_TC_PAIR: return "tc_pair";
+    case TG_PATH_TC_PAIR512: return "tc_pair512";
     default: return "invalid";
   }
 }
