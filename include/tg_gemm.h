@@ -18,7 +18,9 @@
  * Layout: A, B and C are dense and row-major (leading dimensions K, N and N
  * elements), fp16 (IEEE binary16), in device memory of the current CUDA
  * device.  The caller owns all three buffers; the library never allocates,
- * frees or retains device memory and keeps no pointer after a call returns.
+ * frees or retains device memory and keeps no pointer after a call returns;
+ * the one call that uses scratch memory (tg_gemm_relu_f16_ws) takes it from
+ * the caller.
  *
  * Threading and streams: calls are asynchronous on `stream` (a cudaStream_t
  * passed as void*; NULL is the legacy default stream).  On TG_OK the work is
@@ -58,7 +60,7 @@ typedef enum tg_path {
     TG_PATH_AUTO = 0,
     TG_PATH_TC = 1,      /* TMA + tcgen05 persistent kernel, 128x256 tiles;
                             needs K % 8 == 0, N % 8 == 0 and 16-byte
-                            aligned A, B, C                                 */
+                            aligned A and B (any 2-byte aligned C)          */
     TG_PATH_TC_EDGE = 2, /* same kernel, operands staged by predicated
                             loads: any K, N and 2-byte alignment            */
     TG_PATH_SKINNY = 3,  /* small-M split-K tcgen05 kernel (computes
@@ -69,7 +71,10 @@ typedef enum tg_path {
     TG_PATH_TC_PAIR = 6, /* the TMA + tcgen05 kernel on SM pairs
                             (cta_group::2), 256x256 tiles; same alignment
                             needs as TC                                     */
-    TG_PATH_TC_PAIR512 = 7 /* as TC_PAIR with 256x512 tiles                 */
+    TG_PATH_TC_PAIR512 = 7, /* as TC_PAIR with 256x512 tiles                */
+    TG_PATH_REPACK = 8   /* operands TMA cannot describe are first copied
+                            into zero-padded rows in the caller's workspace,
+                            then a TMA kernel runs (tg_gemm_relu_f16_ws)    */
 } tg_path;
 
 /*
@@ -91,16 +96,47 @@ TG_API tg_status tg_gemm_relu_f16(const void *A, const void *B, void *C, int64_t
 /*
  * As tg_gemm_relu_f16, with the kernel path forced (a tg_path value).
  * Forcing a path whose requirements the arguments do not meet returns
- * TG_ERR_INVALID_ARG.  TG_PATH_AUTO behaves like tg_gemm_relu_f16.
+ * TG_ERR_INVALID_ARG, and so does TG_PATH_REPACK (it needs a workspace: use
+ * tg_gemm_relu_f16_ws).  TG_PATH_AUTO behaves like tg_gemm_relu_f16.
  */
 TG_API tg_status tg_gemm_relu_f16_path(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
                                 void *stream, int path);
 
 /*
+ * C = ReLU(A . B) with a caller-provided device workspace.  Identical to
+ * tg_gemm_relu_f16 except when TMA cannot describe A or B (a row stride that
+ * is not a multiple of 16 bytes, or a base that is not 16-byte aligned): then,
+ * if `workspace_bytes` >= tg_workspace_size(...), those operands are first
+ * copied into zero-padded rows in the workspace (path TG_PATH_REPACK) and a
+ * TMA kernel runs on the copies, which is several times faster than the edge
+ * mode.  With less workspace the call behaves like tg_gemm_relu_f16.
+ *   workspace        device pointer, 256-byte aligned, not overlapping A, B
+ *                    or C; owned by the caller and free to reuse once the
+ *                    call's work on `stream` has finished (may be NULL if
+ *                    workspace_bytes == 0)
+ *   workspace_bytes  size of the workspace in bytes
+ * Errors as tg_gemm_relu_f16, plus TG_ERR_INVALID_ARG for a misaligned or
+ * overlapping workspace, or a negative size.
+ */
+TG_API tg_status tg_gemm_relu_f16_ws(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                                     void *stream, void *workspace, int64_t workspace_bytes);
+
+/*
+ * Workspace bytes tg_gemm_relu_f16_ws needs to take the repack path for these
+ * arguments: 0 when no repacking is needed, -1 for invalid arguments.  Host
+ * logic only.
+ */
+TG_API int64_t tg_workspace_size(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K);
+
+/* The path tg_gemm_relu_f16_ws would take with `workspace_bytes` of workspace. */
+TG_API int tg_select_path_ws(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K,
+                             int64_t workspace_bytes);
+
+/*
  * The path tg_gemm_relu_f16 would take for these arguments (a tg_path value;
  * TG_PATH_NONE for an empty C), or -2 when the arguments are invalid.  Host
  * logic only: makes no CUDA call and needs no GPU.  Rules: K == 0 -> ZERO;
- * rows not 16-byte aligned -> TC_EDGE; M <= 256 -> SKINNY; otherwise the
+ * A or B rows not 16-byte aligned -> TC_EDGE; M <= 256 -> SKINNY; otherwise the
  * tensor-core kernel (TC, TC_PAIR or TC_PAIR512) with the least estimated
  * time from its tile count in waves of a 148-SM device.
  */

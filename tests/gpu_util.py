@@ -9,11 +9,14 @@ GUARD_BITS = 0x7E55        # a NaN pattern the kernels never write
 ATOL, RTOL = 1e-3, 4e-3    # |gpu - ref| <= ATOL + RTOL * |ref|
 
 
-def run_gpu(A: np.ndarray, B: np.ndarray, path=None, stream=None, offset_elems: int = 0):
+def run_gpu(A: np.ndarray, B: np.ndarray, path=None, stream=None, offset_elems: int = 0, offsets=None,
+            workspace: bool = False):
     """C = ReLU(A . B) through the C ABI; returns (C as float16 numpy, guards intact?).
 
     ``offset_elems`` shifts A, B and C by that many fp16 elements from a
-    16-byte boundary, to exercise base-pointer alignment handling.
+    16-byte boundary (``offsets`` = (a, b, c) shifts them separately), to
+    exercise base-pointer alignment handling.  ``workspace`` calls
+    tg_gemm_relu_f16_ws with exactly tg_workspace_size bytes of workspace.
     """
     import torch
     import tiled_dense_gemm_fp16_b200 as tg
@@ -21,31 +24,37 @@ def run_gpu(A: np.ndarray, B: np.ndarray, path=None, stream=None, offset_elems: 
     M, K = A.shape
     N = B.shape[1]
     dev = torch.device("cuda", 0)
+    oa, ob, oc = offsets if offsets is not None else (offset_elems,) * 3
 
-    def put(x):
+    def put(x, off):
         buf = torch.empty(x.size + 8, dtype=torch.float16, device=dev)
-        view = buf[offset_elems:offset_elems + x.size].view(x.shape)
+        view = buf[off:off + x.size].view(x.shape)
         view.copy_(torch.from_numpy(np.ascontiguousarray(x)).to(dev))
         return buf, view
 
-    _, Ad = put(A)
-    _, Bd = put(B)
+    _, Ad = put(A, oa)
+    _, Bd = put(B, ob)
     cbuf = torch.full((M * N + 2 * GUARD + 8,), GUARD_BITS, dtype=torch.int16, device=dev)
     cbuf = cbuf.view(torch.float16)
-    C = cbuf[GUARD + offset_elems:GUARD + offset_elems + M * N].view(M, N)
-    st = tg.gemm_relu_f16_raw(Ad.data_ptr(), Bd.data_ptr(), C.data_ptr(), M, N, K,
-                              (stream or torch.cuda.current_stream(dev)).cuda_stream,
-                              tg.Path.AUTO if path is None else path)
+    C = cbuf[GUARD + oc:GUARD + oc + M * N].view(M, N)
+    sh = (stream or torch.cuda.current_stream(dev)).cuda_stream
+    if workspace:
+        need = tg.workspace_size(Ad.data_ptr(), Bd.data_ptr(), C.data_ptr(), M, N, K)
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        st = tg.gemm_relu_f16_ws_raw(Ad.data_ptr(), Bd.data_ptr(), C.data_ptr(), M, N, K, sh, ws.data_ptr(), need)
+    else:
+        st = tg.gemm_relu_f16_raw(Ad.data_ptr(), Bd.data_ptr(), C.data_ptr(), M, N, K, sh,
+                                  tg.Path.AUTO if path is None else path)
     if st != tg.Status.OK:
         raise tg.TGError(st, "tg_gemm_relu_f16")
     torch.cuda.synchronize(dev)
     dst, word = tg.device_status()
     assert dst == tg.Status.OK, f"device error word 0x{word:x}"
     host = cbuf.view(torch.int16).cpu().numpy().view(np.uint16)
-    lo = host[:GUARD + offset_elems]
-    hi = host[GUARD + offset_elems + M * N:]
+    lo = host[:GUARD + oc]
+    hi = host[GUARD + oc + M * N:]
     guards_ok = bool(np.all(lo == GUARD_BITS) and np.all(hi == GUARD_BITS))
-    out = host[GUARD + offset_elems:GUARD + offset_elems + M * N].reshape(M, N).view(np.float16)
+    out = host[GUARD + oc:GUARD + oc + M * N].reshape(M, N).view(np.float16)
     return out, guards_ok
 
 

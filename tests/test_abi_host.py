@@ -121,3 +121,33 @@ def test_no_device_is_reported_not_faked():
     assert tg.gemm_relu_f16_raw(A0, B0, C0, 64, 64, 64) == Status.UNSUPPORTED_DEVICE
     st, _ = tg.device_status()
     assert st == Status.UNSUPPORTED_DEVICE
+
+
+def test_workspace_size_and_repack_choice():
+    # TMA-describable operands need no workspace, whatever C's alignment.
+    assert tg.workspace_size(A0, B0, C0, 8192, 8192, 8192) == 0
+    assert tg.workspace_size(A0, B0, C0 + 2, 512, 512, 512) == 0
+    assert tg.select_path(A0, B0, C0 + 2, 512, 512, 512) != Path.TC_EDGE
+    # Odd K pads A to K rounded up to 8; odd N pads B; each copy 256-byte aligned.
+    up = lambda x: (x + 255) // 256 * 256
+    M, N, K = 3001, 5003, 1021
+    assert tg.workspace_size(A0, B0, C0, M, N, K) == up(2 * M * 1024) + up(2 * K * 5008)
+    assert tg.workspace_size(A0, B0, C0, 8191, 129, 8193) == up(2 * 8191 * 8200) + up(2 * 8193 * 136)
+    assert tg.workspace_size(A0, B0, C0, 64, 64, 100) == up(2 * 64 * 104)          # only A
+    assert tg.workspace_size(A0 + 2, B0, C0, 64, 64, 64) == up(2 * 64 * 64)        # misaligned A base
+    assert tg.workspace_size(A0, B0, C0, -1, 4, 4) == -1
+    need = tg.workspace_size(A0, B0, C0, M, N, K)
+    assert tg.select_path_ws(A0, B0, C0, M, N, K, need) == Path.REPACK
+    assert tg.select_path_ws(A0, B0, C0, M, N, K, need - 1) == Path.TC_EDGE
+    assert tg.select_path_ws(A0, B0, C0, 4096, 4096, 4096, need) == Path.TC_PAIR512
+
+
+def test_workspace_argument_checks():
+    M, N, K = 300, 301, 299
+    need = tg.workspace_size(A0, B0, C0, M, N, K)
+    W0 = 0x40_0000_0000
+    assert tg.gemm_relu_f16_ws_raw(A0, B0, C0, M, N, K, 0, W0 + 16, need) == Status.INVALID_ARG   # not 256-aligned
+    assert tg.gemm_relu_f16_ws_raw(A0, B0, C0, M, N, K, 0, A0, need) == Status.INVALID_ARG        # overlaps A
+    assert tg.gemm_relu_f16_ws_raw(A0, B0, C0, M, N, K, 0, 0, 64) == Status.INVALID_ARG           # NULL with bytes
+    assert tg.gemm_relu_f16_ws_raw(A0, B0, C0, M, N, K, 0, W0, -5) == Status.INVALID_ARG
+    assert tg.gemm_relu_f16_raw(A0, B0, C0, M, N, K, 0, Path.REPACK) == Status.INVALID_ARG        # needs _ws

@@ -126,6 +126,56 @@ def test_misaligned_base_pointers_use_edge_mode(offset, M, N, K):
 
 
 # ---------------------------------------------------------------------------
+# Repack path (caller workspace) and unaligned C on the TMA kernels
+# ---------------------------------------------------------------------------
+
+REPACK_SHAPES = [(1, 9, 7), (15, 17, 9), (129, 257, 65), (255, 129, 127), (300, 301, 299),
+                 (640, 520, 75), (1000, 1001, 1003), (16, 8191, 517), (257, 777, 1021)]
+
+
+@pytest.mark.parametrize("M,N,K", REPACK_SHAPES)
+def test_repack_integer_bitexact(M, N, K):
+    """Odd row lengths: A and/or B copied into zero-padded rows, then a TMA kernel; C stored unaligned."""
+    A, B = inputs.operands(M, N, K, "int", seed=M + 3 * N + 5 * K)
+    got, guards = run_gpu(A, B, workspace=True)
+    assert guards, (M, N, K)
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"repack {(M, N, K)}")
+
+
+@pytest.mark.parametrize("offsets", [(1, 0, 0), (0, 3, 0), (0, 0, 5), (7, 2, 1), (0, 0, 4)])
+def test_unaligned_bases(offsets):
+    """Misaligned A or B go through the repack path; a misaligned C alone keeps the TMA kernels."""
+    for (M, N, K) in [(300, 264, 136), (64, 520, 72)]:
+        A, B = inputs.operands(M, N, K, "int", seed=sum(offsets) + M)
+        ref = oracle.gemm_relu_f16(A, B)
+        for ws in (False, True):
+            got, guards = run_gpu(A, B, offsets=offsets, workspace=ws)
+            assert guards, (offsets, M, N, K, ws)
+            assert_bitexact(got, ref, f"offsets {offsets} {(M, N, K)} ws={ws}")
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 301, 299), (1000, 1001, 1003)])
+def test_repack_uniform(M, N, K):
+    A, B = inputs.operands(M, N, K, "uniform", seed=17)
+    got, guards = run_gpu(A, B, workspace=True)
+    assert guards
+    assert_close(got, oracle.gemm_relu_f16(A, B), f"repack uniform {(M, N, K)}")
+
+
+def test_torch_api_allocates_workspace_itself():
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    A, B = inputs.operands(257, 259, 261, "int", seed=4)
+    Ad, Bd = torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda()
+    C1 = tg.gemm_relu(Ad, Bd)                  # repack path, torch-allocated workspace
+    C2 = tg.gemm_relu(Ad, Bd, workspace=None)  # edge mode
+    torch.cuda.synchronize()
+    ref = oracle.gemm_relu_f16(A, B)
+    assert_bitexact(C1.cpu().numpy(), ref, "torch api repack")
+    assert_bitexact(C2.cpu().numpy(), ref, "torch api edge")
+
+
+# ---------------------------------------------------------------------------
 # Degenerate sizes
 # ---------------------------------------------------------------------------
 
@@ -187,7 +237,10 @@ def _check_workload(name, dist=None, exact=False, full_oracle_max_macs=5e9, path
         rows = list(range(M)) if full else sample_rows(M, seed=M + N + K)
         ref = oracle.gemm_relu_f16_rows(A, B, rows)
         for path in paths:
-            got, guards = run_gpu(A, B, path)
+            if path == "ws":
+                got, guards = run_gpu(A, B, workspace=True)
+            else:
+                got, guards = run_gpu(A, B, path)
             assert guards, (name, M, N, K, path)
             sub = got[rows]
             what = f"{name} {(M, N, K)} path={path} dist={dist or inputs.WORKLOADS[name].dist}"
@@ -222,11 +275,11 @@ def test_workload_skinny_integer():
 
 
 def test_workload_ragged():
-    _check_workload("ragged")
+    _check_workload("ragged", paths=(None, "ws"))
 
 
 def test_workload_ragged_integer():
-    _check_workload("ragged", dist="int", exact=True)
+    _check_workload("ragged", dist="int", exact=True, paths=(None, "ws"))
 
 
 # ---------------------------------------------------------------------------

@@ -14,11 +14,14 @@ from ._binding import (  # noqa: F401
     device_status,
     gemm_relu,
     gemm_relu_f16_raw,
+    gemm_relu_f16_ws_raw,
     lib,
     path_name,
     path_supports,
     select_path,
+    select_path_ws,
     status_string,
     version,
     wait_timeout_selftest,
+    workspace_size,
 )

@@ -36,6 +36,7 @@ class Path(enum.IntEnum):
     ZERO = 5
     TC_PAIR = 6
     TC_PAIR512 = 7
+    REPACK = 8
 
 
 class TGError(RuntimeError):
@@ -47,6 +48,9 @@ class TGError(RuntimeError):
 EXPORTS = (
     "tg_gemm_relu_f16",
     "tg_gemm_relu_f16_path",
+    "tg_gemm_relu_f16_ws",
+    "tg_workspace_size",
+    "tg_select_path_ws",
     "tg_select_path",
     "tg_path_supports",
     "tg_device_status",
@@ -68,6 +72,12 @@ def _bind(lib):
     lib.tg_gemm_relu_f16_path.restype = i32
     lib.tg_select_path.argtypes = [vp, vp, vp, i64, i64, i64]
     lib.tg_select_path.restype = i32
+    lib.tg_gemm_relu_f16_ws.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp, i64]
+    lib.tg_gemm_relu_f16_ws.restype = i32
+    lib.tg_workspace_size.argtypes = [vp, vp, vp, i64, i64, i64]
+    lib.tg_workspace_size.restype = i64
+    lib.tg_select_path_ws.argtypes = [vp, vp, vp, i64, i64, i64, i64]
+    lib.tg_select_path_ws.restype = i32
     lib.tg_path_supports.argtypes = [i32, vp, vp, vp, i64, i64, i64]
     lib.tg_path_supports.restype = i32
     lib.tg_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -125,8 +135,21 @@ def gemm_relu_f16_raw(A: int, B: int, C: int, M: int, N: int, K: int, stream: in
     return int(lib().tg_gemm_relu_f16_path(A, B, C, M, N, K, stream, int(path)))
 
 
+def gemm_relu_f16_ws_raw(A: int, B: int, C: int, M: int, N: int, K: int, stream: int, ws: int, ws_bytes: int) -> int:
+    """tg_gemm_relu_f16_ws on raw device pointers; returns the tg_status value."""
+    return int(lib().tg_gemm_relu_f16_ws(A, B, C, M, N, K, stream, ws, ws_bytes))
+
+
+def workspace_size(A: int, B: int, C: int, M: int, N: int, K: int) -> int:
+    return int(lib().tg_workspace_size(A, B, C, M, N, K))
+
+
 def select_path(A: int, B: int, C: int, M: int, N: int, K: int) -> int:
     return int(lib().tg_select_path(A, B, C, M, N, K))
+
+
+def select_path_ws(A: int, B: int, C: int, M: int, N: int, K: int, ws_bytes: int) -> int:
+    return int(lib().tg_select_path_ws(A, B, C, M, N, K, ws_bytes))
 
 
 def path_supports(path: int, A: int, B: int, C: int, M: int, N: int, K: int) -> bool:
@@ -153,11 +176,15 @@ def _stream_handle(device):
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def gemm_relu(A, B, out=None, path: int = Path.AUTO, stream=None):
+def gemm_relu(A, B, out=None, path: int = Path.AUTO, stream=None, workspace="auto"):
     """C = ReLU(A @ B) for row-major fp16 CUDA tensors A (M, K) and B (K, N).
 
     ``out`` (M, N) fp16 on the same device is written in place if given.
     Runs on ``stream`` (a torch.cuda.Stream) or on the current stream.
+    ``workspace``: "auto" lets torch allocate the scratch bytes the repack path
+    needs when TMA cannot describe A or B (odd row lengths, unaligned bases);
+    None never uses a workspace (edge mode instead); a uint8 CUDA tensor is
+    used as given.  The library itself never allocates.
     """
     import torch
     if A.dtype != torch.float16 or B.dtype != torch.float16:
@@ -176,7 +203,16 @@ def gemm_relu(A, B, out=None, path: int = Path.AUTO, stream=None):
           or out.device != A.device):
         raise ValueError("out must be a contiguous (M, N) float16 tensor on A's device")
     handle = stream.cuda_stream if stream is not None else _stream_handle(A.device)
+    a, b, c = A.data_ptr(), B.data_ptr(), out.data_ptr()
     with torch.cuda.device(A.device):
-        st = gemm_relu_f16_raw(A.data_ptr(), B.data_ptr(), out.data_ptr(), M, N, K, handle, path)
+        if int(path) == Path.AUTO and workspace is not None:
+            need = workspace_size(a, b, c, M, N, K)
+            if need > 0:
+                if isinstance(workspace, str):
+                    workspace = torch.empty(need, dtype=torch.uint8, device=A.device)
+                st = gemm_relu_f16_ws_raw(a, b, c, M, N, K, handle, workspace.data_ptr(), workspace.numel())
+                _check(st, "tg_gemm_relu_f16_ws")
+                return out
+        st = gemm_relu_f16_raw(a, b, c, M, N, K, handle, path)
     _check(st, "tg_gemm_relu_f16")
     return out

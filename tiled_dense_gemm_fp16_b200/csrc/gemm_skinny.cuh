@@ -37,6 +37,7 @@ struct SkinnyParams {
   uint32_t tmem_cols;     // power of two >= max(32, m_pad)
   uint32_t idesc;
   int prefetch_kb;        // > 0: also prefetch into L2 the B boxes this many k-blocks ahead
+  int c_aligned;          // 1: rows of C start on 8-byte boundaries (4-value stores)
   uint64_t wait_budget_ns;
 };
 
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(SkinnyCfg::THREADS, 1)
       const int m = it / (Cfg::PANEL / 4);
       const int j = it - m * (Cfg::PANEL / 4);
       const int n = n0 + 4 * j;
-      if (n >= p.N) continue;  // N % 8 == 0: a group is wholly inside or outside
+      if (n >= p.N) continue;  // with aligned rows (N % 8 == 0) a group is wholly inside or outside
       const uint32_t off = static_cast<uint32_t>((m * Cfg::PANEL + 4 * j) * 4);
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int q = 0; q < p.splits; ++q) {
@@ -226,7 +227,17 @@ __global__ void __launch_bounds__(SkinnyCfg::THREADS, 1)
       uint2 packed;
       packed.x = *reinterpret_cast<const uint32_t*>(&h01);
       packed.y = *reinterpret_cast<const uint32_t*>(&h23);
-      *reinterpret_cast<uint2*>(p.C + static_cast<int64_t>(m) * p.N + n) = packed;
+      __half* dst = p.C + static_cast<int64_t>(m) * p.N + n;
+      if (p.c_aligned) {
+        *reinterpret_cast<uint2*>(dst) = packed;
+      } else {
+        // Unaligned rows of C: 2-byte stores, only of columns inside C.
+        unsigned short* d16 = reinterpret_cast<unsigned short*>(dst);
+        const uint32_t w[2] = {packed.x, packed.y};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (n + e < p.N) d16[e] = static_cast<unsigned short>(w[e >> 1] >> ((e & 1) * 16));
+      }
     }
   }
 

@@ -43,6 +43,7 @@ struct TcParams {
   int store_streaming;   // 1: C stores with the streaming (evict-first) cache hint
   int l2_hints;          // bit 0: A loads evict-last; bit 1: B loads evict-last; bit 2: B loads evict-first
   int prefetch_kb;       // > 0: also prefetch into L2 the boxes this many k-blocks ahead
+  int c_aligned;         // 1: every row of C starts on a 16-byte boundary (C aligned, N % 8 == 0)
   uint64_t wait_budget_ns;
 };
 
@@ -68,6 +69,44 @@ struct TcCfg {
   // A: K-major, B: MN-major (row-major K x N), M = 128, N = 256.
   static constexpr uint32_t IDESC = make_idesc_f16_f32(BM, BN, false, true);
 };
+
+// Store 32 consecutive fp16 values of one row of C, packed two per word in
+// h[0..15] (low half first), to crow[col0 .. col0 + n) with
+// n = min(32, N - col0) >= 1.  With aligned rows: 16-byte stores (streaming
+// cache hint on request).  Otherwise the row start is only 2-byte aligned:
+// 4-byte stores of aligned pairs and 2-byte stores at either end.
+__device__ __forceinline__ void store_row_chunk(__half* crow, int col0, int N, const uint32_t (&h)[16],
+                                                bool aligned16, bool streaming) {
+  if (aligned16) {
+    uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (col0 + q * 8 < N) {
+        const uint4 v = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        if (streaming)
+          __stcs(reinterpret_cast<int4*>(dst + q), *reinterpret_cast<const int4*>(&v));
+        else
+          dst[q] = v;
+      }
+    }
+    return;
+  }
+  unsigned short* dst = reinterpret_cast<unsigned short*>(crow + col0);
+  const int n_here = min(32, N - col0);
+  if ((reinterpret_cast<uintptr_t>(dst) & 2u) == 0) {
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (2 * q + 1 < n_here) reinterpret_cast<uint32_t*>(dst)[q] = h[q];
+    if (n_here & 1) dst[n_here - 1] = static_cast<unsigned short>(h[(n_here - 1) >> 1] & 0xffffu);
+  } else {
+    dst[0] = static_cast<unsigned short>(h[0] & 0xffffu);
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + 1);
+#pragma unroll
+    for (int q = 0; q < 15; ++q)
+      if (2 * q + 2 < n_here) d32[q] = __funnelshift_r(h[q], h[q + 1], 16);
+    if (n_here >= 2 && (n_here & 1) == 0) dst[n_here - 1] = static_cast<unsigned short>(h[(n_here - 1) >> 1] >> 16);
+  }
+}
 
 __device__ __forceinline__ void tile_coords(const TcParams& p, int t, int& m_blk, int& n_blk) {
   const int group_tiles = p.group_m * p.n_tiles;
@@ -403,33 +442,7 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
             const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
             h[e] = *reinterpret_cast<const uint32_t*>(&v);
           }
-          if (!EDGE) {
-            // N % 8 == 0 and C is 16-byte aligned: whole 8-column pieces.
-            uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
-          } else {
-            // Rows are only 2-byte aligned: 4-byte stores of aligned pairs,
-            // 2-byte stores at a misaligned start and at the end of C.
-            unsigned short* dst = reinterpret_cast<unsigned short*>(crow + col0);
-            const int n_here = min(32, p.N - col0);
-            if ((reinterpret_cast<uintptr_t>(dst) & 2u) == 0) {
-#pragma unroll
-              for (int q = 0; q < 16; ++q)
-                if (2 * q + 1 < n_here) reinterpret_cast<uint32_t*>(dst)[q] = h[q];
-              if (n_here & 1)
-                dst[n_here - 1] = static_cast<unsigned short>(h[(n_here - 1) >> 1] & 0xffffu);
-            } else {
-              dst[0] = static_cast<unsigned short>(h[0] & 0xffffu);
-              uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + 1);
-#pragma unroll
-              for (int q = 0; q < 15; ++q)
-                if (2 * q + 2 < n_here) d32[q] = __funnelshift_r(h[q], h[q + 1], 16);
-              if (n_here >= 2 && (n_here & 1) == 0)
-                dst[n_here - 1] = static_cast<unsigned short>(h[(n_here - 1) >> 1] >> 16);
-            }
-          }
+          store_row_chunk(crow, col0, p.N, h, p.c_aligned != 0, false);
         }
       }
       tcgen05_fence_before_sync();

@@ -260,17 +260,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
             const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
             h[e] = *reinterpret_cast<const uint32_t*>(&v);
           }
-          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-          if (p.store_streaming) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (col0 + q * 8 < p.N)
-                __stcs(reinterpret_cast<int4*>(dst + q), make_int4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]));
-          } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
-          }
+          store_row_chunk(crow, col0, p.N, h, p.c_aligned != 0, p.store_streaming != 0);
         }
       }
       tcgen05_fence_before_sync();

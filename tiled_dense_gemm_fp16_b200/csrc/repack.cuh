@@ -1,0 +1,67 @@
+// repack.cuh -- copy a row-major fp16 matrix whose rows are not 16-byte
+// aligned into a row-major copy with rows padded to a multiple of 8 elements
+// (16 bytes), zero in the padding, so that TMA can describe it.
+//
+// Used by the workspace path of C = ReLU(A . B) for operands whose leading
+// dimension (K for A, N for B) is not a multiple of 8 or whose base address
+// is not 16-byte aligned.  Zero padding columns contribute nothing to the K
+// sum (A) and produce output columns that are never stored (B).
+//
+// Bandwidth-bound: every thread writes whole 16-byte chunks of the padded
+// copy; a chunk's 8 source values are read with two aligned 16-byte loads and
+// shifted into place (the loads of several chunks are issued before any is
+// used), with a scalar path at row ends and at the edges of the source.  No
+// byte outside the source matrix is read.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace tg {
+
+struct RepackParams {
+  const __half* src;
+  __half* dst;
+  int rows, cols, cols_pad;  // cols_pad = cols rounded up to a multiple of 8
+  int64_t chunks;            // rows * cols_pad / 8
+};
+
+__global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
+  constexpr int kUnroll = 4;
+  const int chunks_per_row = p.cols_pad >> 3;
+  const __half* src_end = p.src + static_cast<int64_t>(p.rows) * p.cols;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < p.chunks;
+       base += stride * kUnroll) {
+    EdgeChunk plan[kUnroll];
+    int row[kUnroll], col[kUnroll];
+    bool live[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t c = base + u * stride;
+      live[u] = c < p.chunks;
+      row[u] = live[u] ? static_cast<int>(c / chunks_per_row) : 0;
+      col[u] = live[u] ? static_cast<int>(c - static_cast<int64_t>(row[u]) * chunks_per_row) * 8 : 0;
+      plan[u] = edge_chunk_plan(p.src, src_end, p.cols, live[u] ? row[u] : p.rows, p.rows, col[u], p.cols);
+    }
+    uint4 lo[kUnroll], hi[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      lo[u] = make_uint4(0u, 0u, 0u, 0u);
+      hi[u] = lo[u];
+      ld_nc_v4_pred(lo[u], plan[u].src, plan[u].fast);
+      ld_nc_v4_pred(hi[u], plan[u].src + 1, plan[u].fast);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (!live[u]) continue;
+      const uint4 v = plan[u].fast ? edge_realign(lo[u], hi[u], plan[u].shift)
+                                   : load_chunk_pred(p.src, p.cols, row[u], p.rows, col[u], p.cols);
+      *reinterpret_cast<uint4*>(p.dst + static_cast<int64_t>(row[u]) * p.cols_pad + col[u]) = v;
+    }
+  }
+}
+
+}  // namespace tg

@@ -18,6 +18,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_tc_pair.cuh"
 #include "ptx.cuh"
+#include "repack.cuh"
 
 namespace tg {
 namespace {
@@ -48,6 +49,20 @@ int tune_int(const char* name, int dflt) {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 bool g_encode_probed = false;
 
+// One GEMM as the kernels see it: A has rows of `lda` elements (K, or K
+// rounded up to 8 in a zero-padded copy), B has rows of `ldb` elements (N, or
+// N rounded up to 8), C is dense M x N.  c_aligned: every row of C starts on
+// a 16-byte boundary.
+struct Operands {
+  const void* A;
+  int64_t lda;
+  const void* B;
+  int64_t ldb;
+  void* C;
+  int64_t M, N, K;
+  bool c_aligned;
+};
+
 // ---------------------------------------------------------------------------
 // Host-side argument logic (no CUDA calls)
 // ---------------------------------------------------------------------------
@@ -75,10 +90,38 @@ bool args_valid(const void* A, const void* B, const void* C, int64_t M, int64_t 
   return true;
 }
 
-bool aligned16(const void* A, const void* B, const void* C, int64_t N, int64_t K) {
-  const uintptr_t bits = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
-                         reinterpret_cast<uintptr_t>(C);
+// TMA can describe A and B: 16-byte aligned bases and row strides.
+bool tma_ok(const void* A, const void* B, int64_t N, int64_t K) {
+  const uintptr_t bits = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B);
   return (bits & 15u) == 0 && (N % 8) == 0 && (K % 8) == 0;
+}
+
+// Every row of C starts on a 16-byte boundary.
+bool c_rows_aligned(const void* C, int64_t N) {
+  return (reinterpret_cast<uintptr_t>(C) & 15u) == 0 && (N % 8) == 0;
+}
+
+// Workspace of the repack path: zero-padded copies (rows rounded up to 8
+// elements) of whichever of A and B TMA cannot describe, each 256-byte aligned.
+struct RepackPlan {
+  bool pad_a = false, pad_b = false;
+  int64_t kp = 0, np = 0;
+  int64_t off_a = 0, off_b = 0, bytes = 0;
+};
+
+RepackPlan repack_plan(const void* A, const void* B, int64_t M, int64_t N, int64_t K) {
+  RepackPlan r;
+  r.kp = (K + 7) / 8 * 8;
+  r.np = (N + 7) / 8 * 8;
+  r.pad_a = (K % 8) != 0 || (reinterpret_cast<uintptr_t>(A) & 15u) != 0;
+  r.pad_b = (N % 8) != 0 || (reinterpret_cast<uintptr_t>(B) & 15u) != 0;
+  auto up256 = [](int64_t x) { return (x + 255) / 256 * 256; };
+  const int64_t bytes_a = r.pad_a ? up256(2 * M * r.kp) : 0;
+  const int64_t bytes_b = r.pad_b ? up256(2 * K * r.np) : 0;
+  r.off_a = 0;
+  r.off_b = bytes_a;
+  r.bytes = bytes_a + bytes_b;
+  return r;
 }
 
 bool path_supports(int path, const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
@@ -92,9 +135,11 @@ bool path_supports(int path, const void* A, const void* B, const void* C, int64_
     case TG_PATH_TC:
     case TG_PATH_TC_PAIR:
     case TG_PATH_TC_PAIR512:
-      return aligned16(A, B, C, N, K);
+      return tma_ok(A, B, N, K);
     case TG_PATH_SKINNY:
-      return aligned16(A, B, C, N, K) && M <= kSkinnyMaxM;
+      return tma_ok(A, B, N, K) && M <= kSkinnyMaxM;
+    case TG_PATH_REPACK:
+      return !tma_ok(A, B, N, K);
     default:
       return false;
   }
@@ -118,10 +163,22 @@ int select_path(const void* A, const void* B, const void* C, int64_t M, int64_t 
   if (!args_valid(A, B, C, M, N, K)) return -2;
   if (M == 0 || N == 0) return TG_PATH_NONE;
   if (K == 0) return TG_PATH_ZERO;
-  if (!aligned16(A, B, C, N, K)) return TG_PATH_TC_EDGE;
+  if (!tma_ok(A, B, N, K)) return TG_PATH_TC_EDGE;
   if (M <= kSkinnyMaxM) return TG_PATH_SKINNY;
   return pick_tc_kernel(M, N);
 }
+
+// As select_path, for a call that offers `ws_bytes` of workspace: operands
+// TMA cannot describe go through the repack path when the workspace suffices.
+int select_path_ws(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K,
+                   int64_t ws_bytes) {
+  const int path = select_path(A, B, C, M, N, K);
+  if (path == TG_PATH_TC_EDGE && ws_bytes >= repack_plan(A, B, M, N, K).bytes) return TG_PATH_REPACK;
+  return path;
+}
+
+// The tensor-core kernel that runs on TMA-describable (possibly repacked) operands.
+int inner_path(int64_t M, int64_t N) { return M <= kSkinnyMaxM ? TG_PATH_SKINNY : pick_tc_kernel(M, N); }
 
 // ---------------------------------------------------------------------------
 // Device probing and TMA descriptors
@@ -183,9 +240,9 @@ bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, i
 // Launchers
 // ---------------------------------------------------------------------------
 template <bool EDGE>
-tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, cudaStream_t stream,
-                    DeviceInfo* info) {
+tg_status launch_tc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   using Cfg = TcCfg<EDGE>;
+  const int64_t M = o.M, N = o.N, K = o.K;
   auto kernel = gemm_relu_tc_kernel<EDGE>;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -203,13 +260,14 @@ tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N,
   std::memset(&ta, 0, sizeof ta);
   std::memset(&tb, 0, sizeof tb);
   if (!EDGE) {
-    if (!encode_2d(&ta, A, M, K, 64, Cfg::BM)) return TG_ERR_LAUNCH;
-    if (!encode_2d(&tb, B, K, N, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+    if (!encode_2d(&ta, o.A, M, o.lda, 64, Cfg::BM)) return TG_ERR_LAUNCH;
+    if (!encode_2d(&tb, o.B, K, o.ldb, 64, Cfg::BK)) return TG_ERR_LAUNCH;
   }
   TcParams p;
-  p.A = static_cast<const __half*>(A);
-  p.B = static_cast<const __half*>(B);
-  p.C = static_cast<__half*>(C);
+  std::memset(&p, 0, sizeof p);
+  p.A = static_cast<const __half*>(o.A);
+  p.B = static_cast<const __half*>(o.B);
+  p.C = static_cast<__half*>(o.C);
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -222,6 +280,7 @@ tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N,
   p.store_streaming = 0;
   p.l2_hints = 0;
   p.prefetch_kb = 0;
+  p.c_aligned = o.c_aligned ? 1 : 0;
   p.wait_budget_ns = kWaitBudgetNs;
   const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
   kernel<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
@@ -230,9 +289,9 @@ tg_status launch_tc(const void* A, const void* B, void* C, int64_t M, int64_t N,
 
 // 2-CTA path: 256 x 256 tiles on SM pairs, clusters of 2 along x.
 template <int STAGES, int BN>
-tg_status launch_tc_pair_cfg(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
-                             cudaStream_t stream, DeviceInfo* info) {
+tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   using Cfg = TcPairCfg<STAGES, BN>;
+  const int64_t M = o.M, N = o.N, K = o.K;
   auto kernel = gemm_relu_tc_pair_kernel<STAGES, BN>;
   constexpr unsigned kAttrBit = 1u << (STAGES + (BN == 512 ? 16 : 0));
   {
@@ -247,13 +306,13 @@ tg_status launch_tc_pair_cfg(const void* A, const void* B, void* C, int64_t M, i
     }
   }
   CUtensorMap ta, tb;
-  if (!encode_2d(&ta, A, M, K, 64, Cfg::BM)) return TG_ERR_LAUNCH;
-  if (!encode_2d(&tb, B, K, N, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+  if (!encode_2d(&ta, o.A, M, o.lda, 64, Cfg::BM)) return TG_ERR_LAUNCH;
+  if (!encode_2d(&tb, o.B, K, o.ldb, 64, Cfg::BK)) return TG_ERR_LAUNCH;
   TcParams p;
   std::memset(&p, 0, sizeof p);
-  p.A = static_cast<const __half*>(A);
-  p.B = static_cast<const __half*>(B);
-  p.C = static_cast<__half*>(C);
+  p.A = static_cast<const __half*>(o.A);
+  p.B = static_cast<const __half*>(o.B);
+  p.C = static_cast<__half*>(o.C);
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -266,6 +325,7 @@ tg_status launch_tc_pair_cfg(const void* A, const void* B, void* C, int64_t M, i
   p.store_streaming = tune_int("TG_TUNE_STORE_CS", 1);
   p.l2_hints = tune_int("TG_TUNE_L2_HINTS", BN == 512 ? 0 : 5);
   p.prefetch_kb = tune_int("TG_TUNE_PREFETCH_KB", 0);
+  p.c_aligned = o.c_aligned ? 1 : 0;
   p.wait_budget_ns = kWaitBudgetNs;
   const int pairs = info->sm_count / 2;
   const int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
@@ -290,24 +350,23 @@ tg_status launch_tc_pair_cfg(const void* A, const void* B, void* C, int64_t M, i
   return TG_OK;
 }
 
-tg_status launch_tc_pair(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
-                         cudaStream_t stream, DeviceInfo* info, int bn) {
+tg_status launch_tc_pair(const Operands& o, cudaStream_t stream, DeviceInfo* info, int bn) {
   if (bn == 512) {
     switch (tune_int("TG_TUNE_PAIR_STAGES", 4)) {
-      case 3: return launch_tc_pair_cfg<3, 512>(A, B, C, M, N, K, stream, info);
-      default: return launch_tc_pair_cfg<4, 512>(A, B, C, M, N, K, stream, info);
+      case 3: return launch_tc_pair_cfg<3, 512>(o, stream, info);
+      default: return launch_tc_pair_cfg<4, 512>(o, stream, info);
     }
   }
   switch (tune_int("TG_TUNE_PAIR_STAGES", 6)) {
-    case 5: return launch_tc_pair_cfg<5, 256>(A, B, C, M, N, K, stream, info);
-    case 7: return launch_tc_pair_cfg<7, 256>(A, B, C, M, N, K, stream, info);
-    default: return launch_tc_pair_cfg<6, 256>(A, B, C, M, N, K, stream, info);
+    case 5: return launch_tc_pair_cfg<5, 256>(o, stream, info);
+    case 7: return launch_tc_pair_cfg<7, 256>(o, stream, info);
+    default: return launch_tc_pair_cfg<6, 256>(o, stream, info);
   }
 }
 
 // Small-M path: grid (S, P) with clusters of S CTAs along K.
-tg_status launch_skinny(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
-                        cudaStream_t stream, DeviceInfo* info) {
+tg_status launch_skinny(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
+  const int64_t M = o.M, N = o.N, K = o.K;
   using Cfg = SkinnyCfg;
   constexpr int kMaxSmem = 1024 + 220 * 1024 + Cfg::BAR_BYTES;
   {
@@ -323,10 +382,11 @@ tg_status launch_skinny(const void* A, const void* B, void* C, int64_t M, int64_
   }
   SkinnyParams p;
   std::memset(&p, 0, sizeof p);
-  p.C = static_cast<__half*>(C);
+  p.C = static_cast<__half*>(o.C);
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
+  p.c_aligned = (reinterpret_cast<uintptr_t>(o.C) % 8 == 0 && N % 4 == 0) ? 1 : 0;
   p.m_pad = static_cast<int>((M + 15) / 16 * 16);
   p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
   // Two CTAs per SM fit while the ring stays within ~112 KiB (M_pad <= 128).
@@ -350,7 +410,7 @@ tg_status launch_skinny(const void* A, const void* B, void* C, int64_t M, int64_
   p.idesc = make_idesc_f16_f32(Cfg::PANEL, p.m_pad, true, false);
   p.prefetch_kb = tune_int("TG_TUNE_SKINNY_PREFETCH_KB", 0);
   p.wait_budget_ns = kWaitBudgetNs;
-  const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);
+  const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);  // panels past N are not stored
   const int slots = (two_per_sm ? 2 : 1) * info->sm_count;
   int splits = tune_int("TG_TUNE_SKINNY_SPLITS", slots / panels);
   splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
@@ -359,8 +419,8 @@ tg_status launch_skinny(const void* A, const void* B, void* C, int64_t M, int64_
   if (panels > 65535) return TG_ERR_INVALID_ARG;
 
   CUtensorMap ta, tb;
-  if (!encode_2d(&ta, A, M, K, 64, p.m_pad)) return TG_ERR_LAUNCH;
-  if (!encode_2d(&tb, B, K, N, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+  if (!encode_2d(&ta, o.A, M, o.lda, 64, p.m_pad)) return TG_ERR_LAUNCH;
+  if (!encode_2d(&tb, o.B, K, o.ldb, 64, Cfg::BK)) return TG_ERR_LAUNCH;
 
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
@@ -398,37 +458,86 @@ __global__ void wait_timeout_selftest_kernel(uint64_t budget_ns) {
   __syncthreads();
 }
 
-tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream_ptr,
-              int path) {
+tg_status launch_path(int path, const Operands& o, cudaStream_t stream, DeviceInfo* info) {
+  switch (path) {
+    case TG_PATH_TC:
+      return launch_tc<false>(o, stream, info);
+    case TG_PATH_TC_EDGE:
+      return launch_tc<true>(o, stream, info);
+    case TG_PATH_SKINNY:
+      return launch_skinny(o, stream, info);
+    case TG_PATH_TC_PAIR:
+      return launch_tc_pair(o, stream, info, 256);
+    case TG_PATH_TC_PAIR512:
+      return launch_tc_pair(o, stream, info, 512);
+    default:
+      return TG_ERR_INTERNAL;
+  }
+}
+
+tg_status launch_pad(const void* src, void* dst, int64_t rows, int64_t cols, int64_t cols_pad, cudaStream_t stream,
+                     DeviceInfo* info) {
+  RepackParams rp;
+  rp.src = static_cast<const __half*>(src);
+  rp.dst = static_cast<__half*>(dst);
+  rp.rows = static_cast<int>(rows);
+  rp.cols = static_cast<int>(cols);
+  rp.cols_pad = static_cast<int>(cols_pad);
+  rp.chunks = rows * (cols_pad / 8);
+  int64_t blocks = (rp.chunks + 256 * 4 - 1) / (256 * 4);
+  const int64_t cap = static_cast<int64_t>(info->sm_count) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  pad_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(rp);
+  return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+}
+
+tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream_ptr, int path,
+              void* ws, int64_t ws_bytes) {
   if (!args_valid(A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
-  if (path == TG_PATH_AUTO) path = select_path(A, B, C, M, N, K);
+  if (ws_bytes < 0 || (ws_bytes > 0 && ws == nullptr)) return TG_ERR_INVALID_ARG;
+  if (path == TG_PATH_AUTO) path = select_path_ws(A, B, C, M, N, K, ws ? ws_bytes : 0);
   if (!path_supports(path, A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
   if (path == TG_PATH_NONE) return TG_OK;
+  RepackPlan plan;
+  if (path == TG_PATH_REPACK) {
+    plan = repack_plan(A, B, M, N, K);
+    if (ws == nullptr || ws_bytes < plan.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+      return TG_ERR_INVALID_ARG;
+    if (ranges_overlap(ws, plan.bytes, A, 2 * M * K) || ranges_overlap(ws, plan.bytes, B, 2 * K * N) ||
+        ranges_overlap(ws, plan.bytes, C, 2 * M * N))
+      return TG_ERR_INVALID_ARG;
+  }
   int dev = 0;
   DeviceInfo* info = nullptr;
   tg_status st = current_device(dev, info);
   if (st != TG_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  switch (path) {
-    case TG_PATH_ZERO:
-      if (cudaMemsetAsync(C, 0, static_cast<size_t>(2 * M * N), stream) != cudaSuccess) {
-        cudaGetLastError();
-        return TG_ERR_LAUNCH;
-      }
-      return TG_OK;
-    case TG_PATH_TC:
-      return launch_tc<false>(A, B, C, M, N, K, stream, info);
-    case TG_PATH_TC_EDGE:
-      return launch_tc<true>(A, B, C, M, N, K, stream, info);
-    case TG_PATH_SKINNY:
-      return launch_skinny(A, B, C, M, N, K, stream, info);
-    case TG_PATH_TC_PAIR:
-      return launch_tc_pair(A, B, C, M, N, K, stream, info, 256);
-    case TG_PATH_TC_PAIR512:
-      return launch_tc_pair(A, B, C, M, N, K, stream, info, 512);
-    default:
-      return TG_ERR_INTERNAL;
+  Operands o{A, K, B, N, C, M, N, K, c_rows_aligned(C, N)};
+  if (path == TG_PATH_ZERO) {
+    if (cudaMemsetAsync(C, 0, static_cast<size_t>(2 * M * N), stream) != cudaSuccess) {
+      cudaGetLastError();
+      return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
   }
+  if (path == TG_PATH_REPACK) {
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    if (plan.pad_a) {
+      st = launch_pad(A, base + plan.off_a, M, K, plan.kp, stream, info);
+      if (st != TG_OK) return st;
+      o.A = base + plan.off_a;
+      o.lda = plan.kp;
+    }
+    if (plan.pad_b) {
+      st = launch_pad(B, base + plan.off_b, K, N, plan.np, stream, info);
+      if (st != TG_OK) return st;
+      o.B = base + plan.off_b;
+      o.ldb = plan.np;
+    }
+    return launch_path(inner_path(M, N), o, stream, info);
+  }
+  return launch_path(path, o, stream, info);
 }
 
 }  // namespace
@@ -437,12 +546,29 @@ tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64
 extern "C" {
 
 tg_status tg_gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream) {
-  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO);
+  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO, nullptr, 0);
 }
 
 tg_status tg_gemm_relu_f16_path(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
                                 void* stream, int path) {
-  return tg::run(A, B, C, M, N, K, stream, path);
+  if (path == TG_PATH_REPACK) return TG_ERR_INVALID_ARG;  // needs a workspace: tg_gemm_relu_f16_ws
+  return tg::run(A, B, C, M, N, K, stream, path, nullptr, 0);
+}
+
+tg_status tg_gemm_relu_f16_ws(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream,
+                              void* workspace, int64_t workspace_bytes) {
+  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO, workspace, workspace_bytes);
+}
+
+int64_t tg_workspace_size(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
+  if (!tg::args_valid(A, B, C, M, N, K)) return -1;
+  if (M == 0 || N == 0 || K == 0 || tg::tma_ok(A, B, N, K)) return 0;
+  return tg::repack_plan(A, B, M, N, K).bytes;
+}
+
+int tg_select_path_ws(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K,
+                      int64_t workspace_bytes) {
+  return tg::select_path_ws(A, B, C, M, N, K, workspace_bytes);
 }
 
 int tg_select_path(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
@@ -509,6 +635,7 @@ const char* tg_path_name(int path) {
     case TG_PATH_ZERO: return "zero";
     case TG_PATH_TC_PAIR: return "tc_pair";
     case TG_PATH_TC_PAIR512: return "tc_pair512";
+    case TG_PATH_REPACK: return "repack";
     default: return "invalid";
   }
 }
