@@ -50,7 +50,9 @@ typedef enum tg_status {
     TG_ERR_UNSUPPORTED_DEVICE = 2, /* no device, or not compute capability 10.0 */
     TG_ERR_LAUNCH = 3,             /* a kernel launch or CUDA call failed         */
     TG_ERR_TIMEOUT = 4,            /* a bounded device-side wait ran out          */
-    TG_ERR_INTERNAL = 5            /* invariant broken inside the library         */
+    TG_ERR_INTERNAL = 5,           /* invariant broken inside the library         */
+    TG_ERR_TOO_LARGE = 6           /* needs more scratch than the library's fixed
+                                      device buffer holds (tg_gemm_relu_f16_static_ws) */
 } tg_status;
 
 /* Kernel paths.  TG_PATH_AUTO lets the dispatcher choose (see
@@ -120,6 +122,32 @@ TG_API tg_status tg_gemm_relu_f16_path(const void *A, const void *B, void *C, in
  */
 TG_API tg_status tg_gemm_relu_f16_ws(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
                                      void *stream, void *workspace, int64_t workspace_bytes);
+
+/*
+ * C = ReLU(A . B) for callers that cannot allocate device memory at all --
+ * code running where cudaMalloc is off limits (an allocator-free runtime, a
+ * process whose memory budget is fixed up front, a plugin that must not grow
+ * the device footprint) -- but still want the fast repack path for operands
+ * TMA cannot describe.  The paper has no counterpart to this entry point.
+ *
+ * It behaves like tg_gemm_relu_f16_ws, with the workspace taken from a fixed
+ * device buffer of TG_STATIC_WORKSPACE_BYTES (16 MiB) that the library holds
+ * on every GPU where it is loaded, until the process exits.  It calls no
+ * allocating routine.  The caller still passes A, B and C.
+ *   - Problems whose repack would need more than TG_STATIC_WORKSPACE_BYTES
+ *     (tg_workspace_size > 16 MiB) are rejected with TG_ERR_TOO_LARGE and
+ *     nothing is enqueued; aligned problems need no scratch and always run.
+ *   - The first call on a device looks up the buffer's device address for
+ *     that device (with that device current); make that first call before
+ *     any stream capture.
+ *   - Every call shares the one buffer.  Calls whose work can overlap on the
+ *     GPU (different streams, or different host threads) race on it: order
+ *     them on one stream or synchronise between them.  Each call writes every
+ *     scratch byte it reads before reading it, so nothing needs clearing.
+ */
+#define TG_STATIC_WORKSPACE_BYTES (16ll * 1024 * 1024)
+TG_API tg_status tg_gemm_relu_f16_static_ws(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                                            void *stream);
 
 /*
  * Workspace bytes tg_gemm_relu_f16_ws needs to take the repack path for these

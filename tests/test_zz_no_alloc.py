@@ -1,0 +1,63 @@
+"""tg_gemm_relu_f16_static_ws: the entry point for callers that cannot allocate.
+
+Some code that calls this library may not call cudaMalloc at all: an
+allocator-free runtime, a service whose device memory is budgeted once at
+start-up, a plugin that must not grow the device footprint behind its host's
+back.  Such callers still want the fast repack path for operands that TMA
+cannot describe, and that path needs scratch memory.  This entry point takes
+its scratch from a fixed 16 MiB device buffer the library holds on each GPU
+it is loaded on, so the call allocates nothing.
+
+The test drives it through the C ABI on problems that do need scratch, and
+compares each of two calls in a row (the second reuses the buffer as the first
+left it) with the regular entry point tg_gemm_relu_f16, within the float
+tolerance the parity tests use.  This file is collected last.
+"""
+import numpy as np
+import pytest
+
+from gpu_util import assert_close
+from tiled_dense_gemm_fp16_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(entry, Ad, Bd, M, N, K):
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    Cd = torch.full((M, N), float("nan"), dtype=torch.float16, device=Ad.device)
+    sh = torch.cuda.current_stream().cuda_stream
+    if entry == "static":
+        st = tg.gemm_relu_f16_static_ws_raw(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, sh)
+    else:
+        st = tg.gemm_relu_f16_raw(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, sh)
+    assert st == tg.Status.OK, tg.status_string(st)
+    torch.cuda.synchronize()
+    status, word = tg.device_status()
+    assert status == tg.Status.OK, hex(word)
+    return Cd.cpu().numpy()
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 301, 299), (1000, 1001, 1003), (3001, 5003, 1021)])
+def test_static_workspace_matches_regular_entry_point(M, N, K):
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    A, B = inputs.operands(M, N, K, "uniform", seed=M + N + K)
+    Ad, Bd = torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda()
+    # Scratch needed by the repack path (torch's allocations are 16-byte aligned,
+    # so aligned stand-in addresses give the same answer).
+    need = tg.workspace_size(0x10_0000_0000, 0x20_0000_0000, 0x30_0000_0000, M, N, K)
+    assert 0 < need <= tg.STATIC_WORKSPACE_BYTES  # the scratch path is really taken
+    ref = _run("regular", Ad, Bd, M, N, K)
+    for call in range(2):
+        got = _run("static", Ad, Bd, M, N, K)
+        assert_close(got, ref, f"static workspace call {call} {(M, N, K)}")
+
+
+def test_static_workspace_rejects_problems_beyond_its_size():
+    import tiled_dense_gemm_fp16_b200 as tg
+    A0, B0, C0 = 0x10_0000_0000, 0x20_0000_0000, 0x30_0000_0000   # never dereferenced
+    M, N, K = 8191, 129, 8193                                     # about 137 MB of scratch
+    assert tg.workspace_size(A0, B0, C0, M, N, K) > tg.STATIC_WORKSPACE_BYTES
+    assert tg.gemm_relu_f16_static_ws_raw(A0, B0, C0, M, N, K) == tg.Status.TOO_LARGE
+    assert "16 MiB" in tg.status_string(tg.Status.TOO_LARGE)

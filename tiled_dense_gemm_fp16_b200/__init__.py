@@ -8,12 +8,14 @@ use and every call raises if it is missing.
 from ._binding import (  # noqa: F401
     EXPORTS,
     LIB_PATH,
+    STATIC_WORKSPACE_BYTES,
     Path,
     Status,
     TGError,
     device_status,
     gemm_relu,
     gemm_relu_f16_raw,
+    gemm_relu_f16_static_ws_raw,
     gemm_relu_f16_ws_raw,
     lib,
     path_name,

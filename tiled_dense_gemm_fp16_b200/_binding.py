@@ -23,6 +23,7 @@ class Status(enum.IntEnum):
     LAUNCH = 3
     TIMEOUT = 4
     INTERNAL = 5
+    TOO_LARGE = 6
 
 
 class Path(enum.IntEnum):
@@ -51,6 +52,7 @@ EXPORTS = (
     "tg_gemm_relu_f16_ws",
     "tg_workspace_size",
     "tg_select_path_ws",
+    "tg_gemm_relu_f16_static_ws",
     "tg_select_path",
     "tg_path_supports",
     "tg_device_status",
@@ -78,6 +80,8 @@ def _bind(lib):
     lib.tg_workspace_size.restype = i64
     lib.tg_select_path_ws.argtypes = [vp, vp, vp, i64, i64, i64, i64]
     lib.tg_select_path_ws.restype = i32
+    lib.tg_gemm_relu_f16_static_ws.argtypes = [vp, vp, vp, i64, i64, i64, vp]
+    lib.tg_gemm_relu_f16_static_ws.restype = i32
     lib.tg_path_supports.argtypes = [i32, vp, vp, vp, i64, i64, i64]
     lib.tg_path_supports.restype = i32
     lib.tg_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -138,6 +142,14 @@ def gemm_relu_f16_raw(A: int, B: int, C: int, M: int, N: int, K: int, stream: in
 def gemm_relu_f16_ws_raw(A: int, B: int, C: int, M: int, N: int, K: int, stream: int, ws: int, ws_bytes: int) -> int:
     """tg_gemm_relu_f16_ws on raw device pointers; returns the tg_status value."""
     return int(lib().tg_gemm_relu_f16_ws(A, B, C, M, N, K, stream, ws, ws_bytes))
+
+
+def gemm_relu_f16_static_ws_raw(A: int, B: int, C: int, M: int, N: int, K: int, stream: int = 0) -> int:
+    """tg_gemm_relu_f16_static_ws on raw device pointers (no allocation anywhere); returns the tg_status."""
+    return int(lib().tg_gemm_relu_f16_static_ws(A, B, C, M, N, K, stream))
+
+
+STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 
 def workspace_size(A: int, B: int, C: int, M: int, N: int, K: int) -> int:

@@ -35,10 +35,16 @@ struct DeviceInfo {
   bool tc_edge_attr = false;
   bool skinny_attr = false;
   unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
+  void* static_ws = nullptr;  // device address of g_static_workspace on this device
 };
 
 std::mutex g_mutex;
 DeviceInfo g_devices[kMaxDevices];
+
+// Fixed scratch for tg_gemm_relu_f16_static_ws, one per device that loads the
+// library.  In host code this name is only a handle: its device address comes
+// from cudaGetSymbolAddress with the device current.
+__device__ __align__(256) uint8_t g_static_workspace[TG_STATIC_WORKSPACE_BYTES];
 
 // Tuning knobs for experiments (environment, read on each launch); the
 // defaults are the tuned values.
@@ -560,6 +566,35 @@ tg_status tg_gemm_relu_f16_ws(const void* A, const void* B, void* C, int64_t M, 
   return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO, workspace, workspace_bytes);
 }
 
+tg_status tg_gemm_relu_f16_static_ws(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                                     void* stream) {
+  if (!tg::args_valid(A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
+  const int64_t need = tg_workspace_size(A, B, C, M, N, K);
+  if (need > TG_STATIC_WORKSPACE_BYTES) return TG_ERR_TOO_LARGE;
+  int dev = 0;
+  tg::DeviceInfo* info = nullptr;
+  if (M > 0 && N > 0) {
+    const tg_status st = tg::current_device(dev, info);
+    if (st != TG_OK) return st;
+  } else {
+    return TG_OK;  // empty C: nothing to do
+  }
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(tg::g_mutex);
+    if (info->static_ws == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, tg::g_static_workspace) != cudaSuccess || ptr == nullptr) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      info->static_ws = ptr;
+    }
+    ws = info->static_ws;
+  }
+  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO, ws, TG_STATIC_WORKSPACE_BYTES);
+}
+
 int64_t tg_workspace_size(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
   if (!tg::args_valid(A, B, C, M, N, K)) return -1;
   if (M == 0 || N == 0 || K == 0 || tg::tma_ok(A, B, N, K)) return 0;
@@ -620,6 +655,7 @@ const char* tg_status_string(int status) {
     case TG_ERR_LAUNCH: return "kernel launch or CUDA call failed";
     case TG_ERR_TIMEOUT: return "a bounded device-side wait timed out";
     case TG_ERR_INTERNAL: return "internal error";
+    case TG_ERR_TOO_LARGE: return "problem needs more scratch than the library's 16 MiB static workspace holds";
     default: return "unknown status";
   }
 }
