@@ -51,7 +51,7 @@ L2_BYTES = 126 * 1024 * 1024
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="square8192",
@@ -87,7 +87,7 @@ def workload_problem(spec: str, rank: int = 0):
         for i, ((m, n, k), A, B) in enumerate(wl.problems()):
             if i == idx:
                 return f"{name}" + (f":{sub}" if sub else ""), m, n, k, A, B
-    A, B = inputs.operands(M, N, K, wl.dist, seed=wl.seed * 1000 + rank)
+    A, B = inputs.operands(M, N, K, wl.dist, seed=rank_seed(wl.seed, rank))
     return f"{name}" + (f":{sub}" if sub else ""), M, N, K, A, B
 
 
@@ -268,6 +268,28 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank plumbing (also exercised by CPU tests with the gloo backend)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(dist, value: float, device) -> float:
+    """The largest of every rank's `value` (all ranks take part)."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t[0])
+
+
+def aggregate_throughput(world: int, flops_per_rank: int, slowest_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank's independent problem over the slowest rank's step time."""
+    return world * flops_per_rank / (slowest_ms * 1e-3) / 1e12
+
+
+def rank_seed(workload_seed: int, rank: int) -> int:
+    """Seed of rank `rank`'s own problem (rank 0 draws the workload itself)."""
+    return workload_seed * 1000 + rank
+
+
+# ---------------------------------------------------------------------------
 # Our arm
 # ---------------------------------------------------------------------------
 
@@ -356,8 +378,12 @@ def run_ours(args):
     if st != tg.Status.OK:
         raise SystemExit(f"device error after warm-up: {tg.status_string(st)} 0x{word:x}")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # Per-step event pairs only when an L2 flush runs between steps (they
+    # bracket the steps and leave the flushes out); otherwise one pair around
+    # the whole region, so tiny kernels are not charged for event records.
+    per_step = flush is not None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps if per_step else 0)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps if per_step else 0)]
     region0 = torch.cuda.Event(enable_timing=True)
     region1 = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
@@ -368,30 +394,31 @@ def run_ours(args):
     with torch.cuda.stream(stream):
         region0.record(stream)
         for i in range(args.steps):
-            if flush is not None:
+            if per_step:
                 flush.fill_(1)
-            starts[i].record(stream)
+                starts[i].record(stream)
             step()
-            ends[i].record(stream)
+            if per_step:
+                ends[i].record(stream)
         region1.record(stream)
     torch.cuda.synchronize(dev)
     sampler.stop()
     if dist is not None:
         dist.barrier()
     region_ms = region0.elapsed_time(region1)
-    kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    kern_avg_ms = sum(kern_ms) / len(kern_ms)
-    # The step time excludes the L2 flush writes when there are any.
-    step_ms = kern_avg_ms if flush is not None else region_ms / args.steps
+    if per_step:
+        step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
+    else:
+        step_ms = region_ms / args.steps
+    kern_avg_ms = step_ms
     if dist is not None:
-        t = torch.tensor([step_ms, kern_avg_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, kern_avg_ms = float(t[0]), float(t[1])
+        step_ms = max_over_ranks(dist, step_ms, dev)
+        kern_avg_ms = step_ms
     st, word = tg.device_status()
     if st != tg.Status.OK:
         raise SystemExit(f"device error in timed region: {tg.status_string(st)} 0x{word:x}")
 
-    value = world * flops / (step_ms * 1e-3) / 1e12
+    value = aggregate_throughput(world, flops, step_ms)
 
     # End to end through the C ABI from pinned host buffers: H2D of A and B,
     # the call, D2H of C, every step.
@@ -412,10 +439,8 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
     if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+        e2e_ms = max_over_ranks(dist, e2e_ms, dev)
+    e2e_value = aggregate_throughput(world, flops, e2e_ms)
 
     peaks, peak_src = load_peaks()
     if chosen in (tg.Path.TC, tg.Path.TC_EDGE, tg.Path.TC_PAIR, tg.Path.TC_PAIR512) and name.startswith("square"):

@@ -1,0 +1,72 @@
+"""The multi-rank plumbing of bench.py, on CPU with the gloo backend (world size 2).
+
+With N GPUs every rank runs its own independent problem (weak scaling, no
+data-path collective); the only collectives are the barriers around the timed
+region and the max-reduction of the per-rank step times.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+    import sys
+
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        dist.barrier()
+        step_ms = [0.5, 0.8][rank]                      # rank 1 is the slowest
+        slowest = bench.max_over_ranks(dist, step_ms, "cpu")
+        value = bench.aggregate_throughput(world, 2 * 256 ** 3, slowest)
+        dist.barrier()
+        out.put((rank, slowest, value, bench.rank_seed(3, rank)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_time():
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted(out.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, s0, v0, seed0), (r1, s1, v1, seed1) = results
+    assert s0 == s1 == 0.8                              # every rank sees the max
+    assert v0 == v1 == pytest.approx(2 * 2 * 256 ** 3 / 0.8e-3 / 1e12)
+    assert seed0 != seed1                               # independent problems per rank
+
+
+def test_rank_problems_are_independent_and_rank0_is_the_workload():
+    import bench
+    from tiled_dense_gemm_fp16_b200 import inputs
+    name, M, N, K, A0, B0 = bench.workload_problem("square256", rank=0)
+    (shape, A, B), = inputs.WORKLOADS["square256"].problems()
+    assert (M, N, K) == shape and (A0 == A).all() and (B0 == B).all()
+    _, _, _, _, A1, _ = bench.workload_problem("square256", rank=1)
+    assert not (A1 == A0).all()
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    args = type("Args", (), {"workload": "square8192", "steps": 1, "warmup": 3, "gpus": 2})()
+    assert bench.run_reference(args) == 0               # returns at once: no oracle run

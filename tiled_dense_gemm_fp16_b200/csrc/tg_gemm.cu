@@ -151,16 +151,23 @@ bool path_supports(int path, const void* A, const void* B, const void* C, int64_
   }
 }
 
-// Estimated relative time of the three tensor-core kernels for an M x N
-// output on a 148-SM device: waves of tiles x per-SM work of one tile /
-// measured relative efficiency (single CTA 0.90, pair 256x256 0.95,
-// pair 256x512 1.0 at 8192^3).  K scales all three alike.
-int pick_tc_kernel(int64_t M, int64_t N) {
+// Estimated relative time of the three tensor-core kernels on a 148-SM
+// device: waves of tiles x per-SM work of one tile.  The main loop of a tile
+// costs its per-SM MACs over the kernel's measured relative efficiency
+// (single CTA 0.85, pair 256x256 0.88, pair 256x512 1.0 at 8192^3).  The
+// 256x512 tile has one accumulator, so each tile's epilogue (draining TMEM and
+// storing C, worth about 384 k-steps of MMA, twice that when the rows of C are
+// only 2-byte aligned) adds to every tile; the double-buffered kernels hide
+// it behind the next tile and pay it once at the end.
+int pick_tc_kernel(int64_t M, int64_t N, int64_t K, bool c_aligned) {
   constexpr int64_t kSms = 148, kPairs = 74;
-  auto waves = [](int64_t tiles, int64_t units) { return (tiles + units - 1) / units; };
-  const double t1 = waves(((M + 127) / 128) * ((N + 255) / 256), kSms) * (128.0 * 256.0) / 0.90;
-  const double t2 = waves(((M + 255) / 256) * ((N + 255) / 256), kPairs) * (128.0 * 256.0) / 0.95;
-  const double t3 = waves(((M + 255) / 256) * ((N + 511) / 512), kPairs) * (128.0 * 512.0) / 1.0;
+  auto waves = [](int64_t tiles, int64_t units) { return static_cast<double>((tiles + units - 1) / units); };
+  const double kepi = c_aligned ? 384.0 : 768.0;
+  const double k = static_cast<double>(K);
+  const double area1 = 128.0 * 256.0, area3 = 128.0 * 512.0;
+  const double t1 = waves(((M + 127) / 128) * ((N + 255) / 256), kSms) * area1 * k / 0.85 + area1 * kepi;
+  const double t2 = waves(((M + 255) / 256) * ((N + 255) / 256), kPairs) * area1 * k / 0.88 + area1 * kepi;
+  const double t3 = waves(((M + 255) / 256) * ((N + 511) / 512), kPairs) * area3 * (k + kepi);
   if (t3 <= t2 && t3 <= t1) return TG_PATH_TC_PAIR512;
   return t2 <= t1 ? TG_PATH_TC_PAIR : TG_PATH_TC;
 }
@@ -171,7 +178,7 @@ int select_path(const void* A, const void* B, const void* C, int64_t M, int64_t 
   if (K == 0) return TG_PATH_ZERO;
   if (!tma_ok(A, B, N, K)) return TG_PATH_TC_EDGE;
   if (M <= kSkinnyMaxM) return TG_PATH_SKINNY;
-  return pick_tc_kernel(M, N);
+  return pick_tc_kernel(M, N, K, c_rows_aligned(C, N));
 }
 
 // As select_path, for a call that offers `ws_bytes` of workspace: operands
@@ -184,7 +191,9 @@ int select_path_ws(const void* A, const void* B, const void* C, int64_t M, int64
 }
 
 // The tensor-core kernel that runs on TMA-describable (possibly repacked) operands.
-int inner_path(int64_t M, int64_t N) { return M <= kSkinnyMaxM ? TG_PATH_SKINNY : pick_tc_kernel(M, N); }
+int inner_path(int64_t M, int64_t N, int64_t K, bool c_aligned) {
+  return M <= kSkinnyMaxM ? TG_PATH_SKINNY : pick_tc_kernel(M, N, K, c_aligned);
+}
 
 // ---------------------------------------------------------------------------
 // Device probing and TMA descriptors
@@ -541,7 +550,7 @@ tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64
       o.B = base + plan.off_b;
       o.ldb = plan.np;
     }
-    return launch_path(inner_path(M, N), o, stream, info);
+    return launch_path(inner_path(M, N, K, o.c_aligned), o, stream, info);
   }
   return launch_path(path, o, stream, info);
 }
