@@ -175,6 +175,41 @@ def test_torch_api_allocates_workspace_itself():
     assert_bitexact(C2.cpu().numpy(), ref, "torch api edge")
 
 
+def test_random_shapes_fuzz():
+    """Random sizes (aligned and not) through the default path and the workspace path, bit for bit."""
+    rng = np.random.default_rng(2024)
+    for i in range(40):
+        M, N, K = (int(x) for x in rng.integers(1, 1200, size=3))
+        if i % 4 == 0:  # every fourth shape with 16-byte row strides
+            N, K = (N + 7) // 8 * 8, (K + 7) // 8 * 8
+        A, B = inputs.operands(M, N, K, "int", seed=5000 + i)
+        ref = oracle.gemm_relu_f16(A, B)
+        for ws in (False, True):
+            got, guards = run_gpu(A, B, workspace=ws)
+            assert guards, (M, N, K, ws)
+            assert_bitexact(got, ref, f"fuzz {(M, N, K)} ws={ws}")
+
+
+def test_back_to_back_calls_on_one_stream():
+    """Consecutive dependent launches (a call's output feeds the next) stay ordered."""
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    M = 512
+    A, B = inputs.operands(M, M, M, "int", seed=77)
+    Ad, Bd = torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda()
+    ones = torch.ones((M, M), dtype=torch.float16, device="cuda") / 64
+    C1 = tg.gemm_relu(Ad, Bd)
+    C2 = tg.gemm_relu(C1, ones)          # reads C1 right after the kernel that writes it
+    C3 = tg.gemm_relu(C2, ones)
+    torch.cuda.synchronize()
+    r1 = oracle.gemm_relu_f16(A, B)
+    r2 = oracle.gemm_relu_f16(r1, np.full((M, M), 1 / 64, np.float16))
+    r3 = oracle.gemm_relu_f16(r2, np.full((M, M), 1 / 64, np.float16))
+    assert_bitexact(C1.cpu().numpy(), r1, "first")
+    assert_close(C2.cpu().numpy(), r2, "second")
+    assert_close(C3.cpu().numpy(), r3, "third")
+
+
 # ---------------------------------------------------------------------------
 # Degenerate sizes
 # ---------------------------------------------------------------------------

@@ -101,6 +101,10 @@ __global__ void __launch_bounds__(SkinnyCfg::THREADS, 1)
   __syncthreads();
   tcgen05_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touched only shared memory, TMEM and kernel parameters;
+  // global memory is used only after the previous grid on the stream is done.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // Producer: one thread issues the TMA loads of this CTA's K slice.

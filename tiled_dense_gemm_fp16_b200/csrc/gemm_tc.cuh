@@ -70,6 +70,15 @@ struct TcCfg {
   static constexpr uint32_t IDESC = make_idesc_f16_f32(BM, BN, false, true);
 };
 
+// ReLU on two fp32 accumulator values (every value that is not > 0 becomes
+// +0), rounded to fp16 (nearest even) and packed, the first in the low half.
+__device__ __forceinline__ uint32_t relu_pack_f16x2(uint32_t a, uint32_t b) {
+  const float x0 = __uint_as_float(a);
+  const float x1 = __uint_as_float(b);
+  const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 // Store 32 consecutive fp16 values of one row of C, packed two per word in
 // h[0..15] (low half first), to crow[col0 .. col0 + n) with
 // n = min(32, N - col0) >= 1.  With aligned rows: 16-byte stores (streaming
@@ -231,6 +240,10 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
   __syncthreads();
   tcgen05_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touched only shared memory, TMEM and kernel parameters;
+  // global memory is used only after the previous grid on the stream is done.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp < Cfg::PRODUCER_WARPS) {
     // ------------------------------------------------------------------

@@ -45,7 +45,12 @@ struct TcPairCfg {
   static constexpr int STAGES = STAGES_;
   static constexpr int MMA_WARP = 1;
   static constexpr int EPI_WARP0 = 2;
-  static constexpr int EPI_WARPS = 4 * SLABS;     // 4 per 256-column slab
+  // Epilogue warps: 4 per 256-column slab, each taking the slab's columns
+  // for one TMEM lane quadrant (with the single accumulator of BN = 512 a
+  // thread holds its 256 values in registers and releases TMEM before it
+  // stores).
+  static constexpr int EPI_WARPS = 4 * SLABS;
+  static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // accumulator columns per epilogue warp
   static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
   static constexpr int A_BYTES = BM * BK * 2;        // 16 KiB
   static constexpr int B_BYTES = BK * BN_HALF * 2;   // 16 or 32 KiB
@@ -109,6 +114,10 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
   cluster_sync();  // both CTAs' barriers are initialised before any remote use
   tcgen05_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touched only shared memory, TMEM and kernel parameters;
+  // global memory is used only after the previous grid on the stream is done.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------------
@@ -228,10 +237,11 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
   } else {
     // ------------------------------------------------------------------
     // Epilogue (both CTAs): this CTA's 128 rows of the 256 x BN tile; warp
-    // w reads TMEM lanes 32 (w mod 4) .. + 31 of slab (w - 2) / 4.
+    // w reads TMEM lanes 32 (w mod 4) .. + 31, columns
+    // [EPI_COLS * ((w - 2) / 4), + EPI_COLS) of the accumulator.
     // ------------------------------------------------------------------
     const int quad = warp & 3;
-    const int slab = (warp - Cfg::EPI_WARP0) >> 2;
+    const int col_base = ((warp - Cfg::EPI_WARP0) >> 2) * Cfg::EPI_COLS;
     int local = 0;
     for (int t = cluster_id; t < p.num_tiles; t += num_clusters, ++local) {
       int m_blk, n_blk;
@@ -244,28 +254,51 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
       const int row = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM + quad * 32 + lane;
       const bool row_ok = row < p.M;
       __half* crow = p.C + static_cast<int64_t>(row) * p.N;
-#pragma unroll 1
-      for (int c = 0; c < 256 / 32; ++c) {
-        uint32_t r[32];
-        const int tcol = slab * 256 + c * 32;  // column within this CTA's accumulator
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + tcol, r);
-        tmem_ld_wait();
-        const int col0 = n_blk * Cfg::BN + tcol;
-        if (row_ok && col0 < p.N) {
-          uint32_t h[16];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + col_base;
+      if (Cfg::NUM_ACC == 1) {
+        // Single accumulator: read this thread's EPI_COLS columns into
+        // registers as ReLU'd fp16 pairs, release the accumulator to the MMA
+        // warp, and only then store, so the stores overlap the next tile's MMAs.
+        uint32_t h[Cfg::EPI_COLS / 2];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = __uint_as_float(r[2 * e]);
-            const float x1 = __uint_as_float(r[2 * e + 1]);
-            const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
-            h[e] = *reinterpret_cast<const uint32_t*>(&v);
-          }
-          store_row_chunk(crow, col0, p.N, h, p.c_aligned != 0, p.store_streaming != 0);
+        for (int c = 0; c < Cfg::EPI_COLS / 16; ++c) {
+          uint32_t r[16];  // 16 columns at a time keeps the register peak low
+          tmem_ld_32x32b_x16(taddr + c * 16, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) h[c * 8 + e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
         }
+        tcgen05_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
+#pragma unroll
+        for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
+          const int col0 = n_blk * Cfg::BN + col_base + c * 32;
+          uint32_t hc[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) hc[e] = h[c * 16 + e];
+          if (row_ok && col0 < p.N) store_row_chunk(crow, col0, p.N, hc, p.c_aligned != 0, p.store_streaming != 0);
+        }
+      } else {
+        // Double-buffered accumulator: the next tile's MMAs already run in
+        // the other buffer; drain 32 columns at a time.
+#pragma unroll 1
+        for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, r);
+          tmem_ld_wait();
+          const int col0 = n_blk * Cfg::BN + col_base + c * 32;
+          if (row_ok && col0 < p.N) {
+            uint32_t hc[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) hc[e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
+            store_row_chunk(crow, col0, p.N, hc, p.c_aligned != 0, p.store_streaming != 0);
+          }
+        }
+        tcgen05_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
       }
-      tcgen05_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
     }
   }
 

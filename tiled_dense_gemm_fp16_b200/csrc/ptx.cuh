@@ -40,6 +40,20 @@ __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31u) == 0u; }
 
 // ----------------------------------------------------------------------------
+// Programmatic dependent launch
+// ----------------------------------------------------------------------------
+// Wait until the grids this grid depends on (the previous kernel on the stream
+// when launched with programmatic stream serialization) have completed and
+// their memory is visible.  Returns at once when there is no such dependency.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next grid on the stream be scheduled (its own prologue overlaps
+// this grid's tail; it still waits for this grid before touching memory).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------
 // mbarrier
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

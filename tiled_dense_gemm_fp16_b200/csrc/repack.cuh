@@ -30,6 +30,8 @@ struct RepackParams {
 
 __global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
   constexpr int kUnroll = 4;
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int chunks_per_row = p.cols_pad >> 3;
   const __half* src_end = p.src + static_cast<int64_t>(p.rows) * p.cols;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;

@@ -254,6 +254,30 @@ bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, i
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
+// Every kernel is launched with programmatic stream serialization: it may be
+// scheduled while the previous kernel on the stream drains, runs its
+// prologue (barriers, TMEM), and waits for that kernel before touching
+// global memory.  `cluster_x` > 1 adds a cluster dimension.
+struct LaunchAttrs {
+  cudaLaunchAttribute attr[2];
+  unsigned count = 0;
+  void fill(cudaLaunchConfig_t& cfg, unsigned cluster_x) {
+    count = 0;
+    attr[count].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[count].val.programmaticStreamSerializationAllowed = tune_int("TG_TUNE_PDL", 1) ? 1 : 0;
+    ++count;
+    if (cluster_x > 1) {
+      attr[count].id = cudaLaunchAttributeClusterDimension;
+      attr[count].val.clusterDim.x = cluster_x;
+      attr[count].val.clusterDim.y = 1;
+      attr[count].val.clusterDim.z = 1;
+      ++count;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = count;
+  }
+};
+
 template <bool EDGE>
 tg_status launch_tc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   using Cfg = TcCfg<EDGE>;
@@ -298,8 +322,19 @@ tg_status launch_tc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   p.c_aligned = o.c_aligned ? 1 : 0;
   p.wait_budget_ns = kWaitBudgetNs;
   const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
-  kernel<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
-  return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::SMEM_BYTES);
+  cfg.stream = stream;
+  LaunchAttrs la;
+  la.fill(cfg, 1);
+  if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
 }
 
 // 2-CTA path: 256 x 256 tiles on SM pairs, clusters of 2 along x.
@@ -351,13 +386,8 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
   cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::SMEM_BYTES);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  LaunchAttrs la;
+  la.fill(cfg, 2);
   if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
     cudaGetLastError();
     return TG_ERR_LAUNCH;
@@ -443,13 +473,8 @@ tg_status launch_skinny(const Operands& o, cudaStream_t stream, DeviceInfo* info
   cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::smem_bytes(p.m_pad, stages));
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  LaunchAttrs la;
+  la.fill(cfg, static_cast<unsigned>(splits));
   if (cudaLaunchKernelEx(&cfg, gemm_relu_skinny_kernel, ta, tb, p) != cudaSuccess) {
     cudaGetLastError();
     return TG_ERR_LAUNCH;
@@ -503,8 +528,18 @@ tg_status launch_pad(const void* src, void* dst, int64_t rows, int64_t cols, int
   const int64_t cap = static_cast<int64_t>(info->sm_count) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  pad_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(rp);
-  return cudaGetLastError() == cudaSuccess ? TG_OK : TG_ERR_LAUNCH;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  LaunchAttrs la;
+  la.fill(cfg, 1);
+  if (cudaLaunchKernelEx(&cfg, pad_rows_kernel, rp) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
 }
 
 tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream_ptr, int path,
