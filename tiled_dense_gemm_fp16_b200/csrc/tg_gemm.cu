@@ -23,7 +23,15 @@
 namespace tg {
 namespace {
 
-constexpr uint64_t kWaitBudgetNs = 4000000000ull;  // 4 s per pipeline wait
+constexpr uint64_t kWaitBudgetNs = 4000000000ull;  // 4 s per pipeline wait, plus:
+constexpr uint64_t kWaitPerKBlockNs = 4000ull;      // 4 us per k-block (waits that span a tile's K loop)
+
+// Bound of one wait: generous for a single pipeline step, and longer than a
+// whole tile's K loop (about 0.5 us per 64-deep k-block at full speed) for the
+// waits that span one.
+uint64_t wait_budget(int64_t k_blocks) {
+  return kWaitBudgetNs + static_cast<uint64_t>(k_blocks > 0 ? k_blocks : 0) * kWaitPerKBlockNs;
+}
 constexpr int kMaxDevices = 64;
 constexpr int64_t kSkinnyMaxM = 256;               // largest M the small-M path takes
 
@@ -320,7 +328,7 @@ tg_status launch_tc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   p.l2_hints = 0;
   p.prefetch_kb = 0;
   p.c_aligned = o.c_aligned ? 1 : 0;
-  p.wait_budget_ns = kWaitBudgetNs;
+  p.wait_budget_ns = wait_budget(p.k_blocks);
   const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
@@ -373,10 +381,10 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
   p.group_m = tune_int("TG_TUNE_GROUP_M", BN == 512 ? 16 : 12);
   if (p.group_m < 1) p.group_m = 1;
   p.store_streaming = tune_int("TG_TUNE_STORE_CS", 1);
-  p.l2_hints = tune_int("TG_TUNE_L2_HINTS", BN == 512 ? 0 : 5);
+  p.l2_hints = tune_int("TG_TUNE_L2_HINTS", BN == 512 ? 2 : 5);
   p.prefetch_kb = tune_int("TG_TUNE_PREFETCH_KB", 0);
   p.c_aligned = o.c_aligned ? 1 : 0;
-  p.wait_budget_ns = kWaitBudgetNs;
+  p.wait_budget_ns = wait_budget(p.k_blocks);
   const int pairs = info->sm_count / 2;
   const int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
 
@@ -454,7 +462,7 @@ tg_status launch_skinny(const Operands& o, cudaStream_t stream, DeviceInfo* info
   p.tmem_cols = cols;
   p.idesc = make_idesc_f16_f32(Cfg::PANEL, p.m_pad, true, false);
   p.prefetch_kb = tune_int("TG_TUNE_SKINNY_PREFETCH_KB", 0);
-  p.wait_budget_ns = kWaitBudgetNs;
+  p.wait_budget_ns = wait_budget(p.k_blocks);
   const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);  // panels past N are not stored
   const int slots = (two_per_sm ? 2 : 1) * info->sm_count;
   int splits = tune_int("TG_TUNE_SKINNY_SPLITS", slots / panels);
