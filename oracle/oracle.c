@@ -199,6 +199,77 @@ int oracle_gemm_relu_f16(const uint16_t *A, const uint16_t *B, uint16_t *C,
     return failed ? -1 : 0;
 }
 
+/*
+ * General layouts and a per-column bias:
+ *
+ *   C[i*ldc + j] = f16_rne( relu( fp32( sum_k a(i,k) * b(k,j) ) + f32(bias[j]) ) )
+ *
+ * with a(i,k) = A[i*lda + k]; b(k,j) = B[k*ldb + j] when b_nk == 0 (B stored
+ * K x N) and B[j*ldb + k] when b_nk == 1 (B stored N x K, so C = A . B^T);
+ * bias may be NULL (no bias term).  The sum runs in k order with an fp32
+ * accumulator exactly as in oracle_gemm_relu_f16; the bias is added to the
+ * finished sum with one fp32 addition, then ReLU, then the fp16 rounding.
+ * Elements of C outside the M x N block (padding of ldc) are not written.
+ * Returns 0, or -1 if a work buffer cannot be allocated.
+ */
+int oracle_gemm_relu_f16_ex(const uint16_t *A, const uint16_t *B, uint16_t *C, int64_t M, int64_t N,
+                            int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int b_nk, const uint16_t *bias,
+                            int nthreads)
+{
+    if (M <= 0 || N <= 0)
+        return 0;
+
+    /* Widen B once into the K x N order the i-k-j loop walks: Bf[k*N + j]. */
+    float *Bf = NULL;
+    if (K > 0) {
+        Bf = (float *)malloc((size_t)K * (size_t)N * sizeof(float));
+        if (!Bf)
+            return -1;
+        for (int64_t k = 0; k < K; ++k)
+            for (int64_t j = 0; j < N; ++j)
+                Bf[k * N + j] = oracle_f16_to_f32(b_nk ? B[j * ldb + k] : B[k * ldb + j]);
+    }
+
+    int failed = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        float *acc = (float *)malloc((size_t)N * sizeof(float));
+        if (!acc) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            failed = 1;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int64_t i = 0; i < M; ++i) {
+            if (!acc)
+                continue;
+            for (int64_t j = 0; j < N; ++j)
+                acc[j] = 0.0f;
+            for (int64_t k = 0; k < K; ++k) {
+                const float a = oracle_f16_to_f32(A[i * lda + k]);
+                const float *brow = Bf + k * N;
+                for (int64_t j = 0; j < N; ++j)
+                    acc[j] = acc[j] + a * brow[j];
+            }
+            for (int64_t j = 0; j < N; ++j) {
+                const float y = bias ? acc[j] + oracle_f16_to_f32(bias[j]) : acc[j];
+                const float v = y > 0.0f ? y : 0.0f;
+                C[i * ldc + j] = oracle_f32_to_f16_rne(v);
+            }
+        }
+        free(acc);
+    }
+    free(Bf);
+    return failed ? -1 : 0;
+}
+
 /* Number of threads OpenMP would use by default (1 without OpenMP). */
 int oracle_max_threads(void)
 {

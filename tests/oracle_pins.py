@@ -280,6 +280,67 @@ def check_rows_and_threads(lib):
     assert np.array_equal(_bits(sub), _bits(full[rows]))
 
 
+# --------------------------------------------------------------------------
+# General layouts and bias (oracle_gemm_relu_f16_ex)
+# --------------------------------------------------------------------------
+
+def check_ex_dense_equals_base(lib):
+    """Dense strides, B as K x N, no bias: the same bits as the base oracle."""
+    for (M, N, K), dist in [((37, 53, 211), "uniform"), ((8, 8, 8), "normal01"), ((64, 17, 300), "int")]:
+        A, B = inputs.operands(M, N, K, dist, seed=M + N)
+        base = oracle.gemm_relu_f16(A, B, lib=lib)
+        ex = oracle.gemm_relu_f16_ex(A, B, M, N, K, K, N, N, lib=lib).reshape(M, N)
+        assert np.array_equal(_bits(ex), _bits(base)), (M, N, K)
+
+
+def check_ex_weight_layout(lib):
+    """B stored N x K (C = A . B^T) gives the base oracle's bits on the transposed copy."""
+    for (M, N, K) in [(29, 41, 67), (5, 130, 9)]:
+        A, B = inputs.operands(M, N, K, "uniform", seed=K)
+        Bt = np.ascontiguousarray(B.T)                       # N x K storage of the same B
+        ex = oracle.gemm_relu_f16_ex(A, Bt, M, N, K, K, K, N, b_nk=True, lib=lib).reshape(M, N)
+        assert np.array_equal(_bits(ex), _bits(oracle.gemm_relu_f16(A, B, lib=lib))), (M, N, K)
+
+
+def check_ex_strides(lib):
+    """Row strides wider than the rows read the same values; C's padding is left alone."""
+    M, N, K = 23, 31, 45
+    lda, ldb, ldc = K + 7, N + 3, N + 5
+    A, B = inputs.operands(M, N, K, "int", seed=9)
+    rng = np.random.default_rng(10)
+    Ap = rng.uniform(-9, 9, size=(M, lda)).astype(np.float16)
+    Bp = rng.uniform(-9, 9, size=(K, ldb)).astype(np.float16)
+    Ap[:, :K] = A
+    Bp[:, :N] = B
+    Cinit = np.full(M * ldc, 0x7E55, dtype=np.uint16)
+    got = oracle.gemm_relu_f16_ex(Ap, Bp, M, N, K, lda, ldb, ldc, C=Cinit, lib=lib).view(np.uint16).reshape(M, ldc)
+    assert np.array_equal(got[:, :N], _bits(oracle.gemm_relu_f16(A, B, lib=lib)))
+    assert np.all(got[:, N:] == 0x7E55)
+
+
+def check_ex_bias_exact(lib):
+    """Integer operands and bias: relu(A . B + bias) is exact, so fp16 of it is unique."""
+    M, N, K = 19, 40, 133
+    A, B = inputs.operands(M, N, K, "int", seed=21)
+    bias = np.random.default_rng(22).integers(-40, 41, size=N).astype(np.float16)
+    got = oracle.gemm_relu_f16_ex(A, B, M, N, K, K, N, N, bias=bias, lib=lib).reshape(M, N)
+    S = A.astype(np.int64) @ B.astype(np.int64) + bias.astype(np.int64)[None, :]
+    want = np.maximum(S, 0).astype(np.float64).astype(np.float16)
+    assert np.array_equal(_bits(got), _bits(want))
+
+
+def check_ex_bias_closed_form(lib):
+    """A = 0: every row of C is ReLU(bias) (+0 for non-positive entries)."""
+    M, N, K = 6, 33, 17
+    bias = np.random.default_rng(3).uniform(-4, 4, size=N).astype(np.float16)
+    bias[:4] = np.array([0.0, -0.0, 65504, -1e-7], np.float16)
+    A = np.zeros((M, K), np.float16)
+    B = np.random.default_rng(4).uniform(-1, 1, size=(N, K)).astype(np.float16)
+    got = oracle.gemm_relu_f16_ex(A, B, M, N, K, K, K, N, b_nk=True, bias=bias, lib=lib).reshape(M, N)
+    want = np.where(bias.astype(np.float32) > 0, bias, np.float16(0)).astype(np.float16)
+    assert np.array_equal(_bits(got), np.tile(_bits(want), (M, 1)))
+
+
 ALL_CHECKS = [
     check_f16_to_f32_all_patterns,
     check_f32_to_f16_golden,
@@ -295,4 +356,9 @@ ALL_CHECKS = [
     check_exact_rational_bound,
     check_sequential_fp32_tiny,
     check_rows_and_threads,
+    check_ex_dense_equals_base,
+    check_ex_weight_layout,
+    check_ex_strides,
+    check_ex_bias_exact,
+    check_ex_bias_closed_form,
 ]
