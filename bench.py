@@ -56,7 +56,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="square8192",
                     help="square8192 (the metric's workload), square4096, square256, skinny:<M>, ragged:<i>")
-    ap.add_argument("--path", default="auto", help="force a kernel path: auto, tc, tc_edge, skinny, gemv")
+    ap.add_argument("--path", default="auto", help="force a kernel path: auto, tc, tc_edge, skinny, tc_pair, tc_pair512")
     ap.add_argument("--workspace", choices=["auto", "none"], default="auto",
                     help="auto: give the library the scratch bytes it asks for (repack path for "
                          "operands TMA cannot describe), allocated by torch outside the timed region")
@@ -82,6 +82,9 @@ def workload_problem(spec: str, rank: int = 0):
     elif name == "ragged":
         idx = int(sub) if sub else 0
     M, N, K = problems[idx]
+    if name == "linear8192":
+        x, W, b = inputs.linear_operands(M, N, K, seed=wl.seed if rank == 0 else rank_seed(wl.seed, rank))
+        return name, M, N, K, x, (W, b)
     if rank == 0:
         # Exactly the workload's own draw (the generator is advanced over earlier shapes).
         for i, ((m, n, k), A, B) in enumerate(wl.problems()):
@@ -93,8 +96,10 @@ def workload_problem(spec: str, rank: int = 0):
 
 def describe(name, M, N, K):
     wl = inputs.WORKLOADS[name.partition(":")[0]]
+    layout = ("x (M x K) row-major, weight stored N x K, fp16 bias, C row-major" if name == "linear8192"
+              else "row-major A, B, C")
     return {"workload": name, "M": M, "N": N, "K": K, "dtype_in": "fp16", "accumulate": "fp32",
-            "dtype_out": "fp16", "layout": "row-major A, B, C", "values": wl.dist, "seed": wl.seed}
+            "dtype_out": "fp16", "layout": layout, "values": wl.dist, "seed": wl.seed}
 
 
 def load_peaks():
@@ -313,9 +318,14 @@ def run_ours(args):
     torch.cuda.set_device(dev)
 
     path = {"auto": tg.Path.AUTO, "tc": tg.Path.TC, "tc_edge": tg.Path.TC_EDGE, "skinny": tg.Path.SKINNY,
-            "gemv": tg.Path.GEMV, "tc_pair": tg.Path.TC_PAIR, "tc_pair512": tg.Path.TC_PAIR512}[args.path]
+            "tc_pair": tg.Path.TC_PAIR, "tc_pair512": tg.Path.TC_PAIR512}[args.path]
     name, M, N, K, A, B = workload_problem(args.workload, rank)
     flops = inputs.flops(M, N, K)
+    linear = name == "linear8192"
+    bias_d = None
+    if linear:
+        B, bias = B
+        bias_d = torch.from_numpy(bias).to(dev)
 
     Ad = torch.from_numpy(A).to(dev)
     Bd = torch.from_numpy(B).to(dev)
@@ -356,8 +366,14 @@ def run_ours(args):
     if chosen == tg.Path.REPACK:
         launches_per_step += int(K % 8 != 0 or Ad.data_ptr() % 16 != 0) + int(N % 8 != 0 or Bd.data_ptr() % 16 != 0)
 
+    lin_opts = tg.options(b_layout=tg.B_NK, bias=bias_d.data_ptr()) if linear else None
+    if linear:
+        chosen = tg.select_path_ex(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, lin_opts, 0)
+
     def call(a, b, c):
-        if ws_bytes > 0:
+        if linear:
+            st = tg.gemm_relu_f16_ex_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, lin_opts, sh)
+        elif ws_bytes > 0:
             st = tg.gemm_relu_f16_ws_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, sh, ws.data_ptr(), ws_bytes)
         else:
             st = tg.gemm_relu_f16_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, sh, path)
@@ -443,7 +459,8 @@ def run_ours(args):
     e2e_value = aggregate_throughput(world, flops, e2e_ms)
 
     peaks, peak_src = load_peaks()
-    if chosen in (tg.Path.TC, tg.Path.TC_EDGE, tg.Path.TC_PAIR, tg.Path.TC_PAIR512) and name.startswith("square"):
+    if chosen in (tg.Path.TC, tg.Path.TC_EDGE, tg.Path.TC_PAIR, tg.Path.TC_PAIR512) and (
+            name.startswith("square") or linear):
         bound, unit_r = "tensor", "TFLOP/s"
         achieved = flops / (kern_avg_ms * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])

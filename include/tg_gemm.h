@@ -66,9 +66,8 @@ typedef enum tg_path {
     TG_PATH_TC_EDGE = 2, /* same kernel, operands staged by predicated
                             loads: any K, N and 2-byte alignment            */
     TG_PATH_SKINNY = 3,  /* small-M split-K tcgen05 kernel (computes
-                            C^T = B^T A^T); same alignment needs as TC       */
-    TG_PATH_GEMV = 4,    /* CUDA-core kernel for M <= 8; same alignment
-                            needs as TC                                     */
+                            C^T = B^T A^T), M <= 256 (this kernel also
+                            serves M = 1); same alignment needs as TC       */
     TG_PATH_ZERO = 5,    /* K == 0: C is filled with +0 (empty sum)         */
     TG_PATH_TC_PAIR = 6, /* the TMA + tcgen05 kernel on SM pairs
                             (cta_group::2), 256x256 tiles; same alignment
@@ -80,7 +79,8 @@ typedef enum tg_path {
 } tg_path;
 
 /*
- * C = ReLU(A . B).
+ * C = ReLU(A . B).  (tg_gemm_relu_f16_ex below adds strides, the N x K
+ * layout of B, a bias and batches.)
  *   A      device pointer, M x K fp16, row-major (may be NULL if M*K == 0)
  *   B      device pointer, K x N fp16, row-major (may be NULL if K*N == 0)
  *   C      device pointer, M x N fp16, row-major, written in full; must not
@@ -148,6 +148,66 @@ TG_API tg_status tg_gemm_relu_f16_ws(const void *A, const void *B, void *C, int6
 #define TG_STATIC_WORKSPACE_BYTES (16ll * 1024 * 1024)
 TG_API tg_status tg_gemm_relu_f16_static_ws(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
                                             void *stream);
+
+/*
+ * General operand layouts, a fused bias and strided batches.
+ *
+ * For each batch entry e = 0 .. batch-1:
+ *
+ *   C_e[i*ldc + j] = fp16( max( sum_k A_e[i*lda + k] * b_e(k, j) + bias[j], 0 ) )
+ *
+ * with A_e = A + e*stride_a, B_e = B + e*stride_b, C_e = C + e*stride_c
+ * (element offsets) and b_e(k, j) = B_e[k*ldb + j] when B is stored K x N
+ * (TG_B_KN) or B_e[j*ldb + k] when it is stored N x K (TG_B_NK, the layout of
+ * a linear layer's weight: C = A . W^T).  The sum is accumulated in fp32;
+ * the bias (fp16, N values, optional) is added to it in fp32 before ReLU.
+ * This widens the quick-start kernel's dense row-major operands to the
+ * layouts its T.gemm tile operator accepts ("TileLang" wiki page,
+ * "Programming model": layouts inferred per operand; symbolic shapes).
+ *
+ * A zero-initialised tg_gemm_options (or NULL) means: dense row-major A, B
+ * (K x N) and C, no bias, one problem, automatic kernel choice.
+ */
+enum { TG_B_KN = 0, TG_B_NK = 1 };
+
+typedef struct tg_gemm_options {
+    int64_t lda;        /* elements between rows of A; 0 = K; must be >= K        */
+    int64_t ldb;        /* elements between rows of B as stored; 0 = N (TG_B_KN)
+                           or K (TG_B_NK); must be at least that                */
+    int64_t ldc;        /* elements between rows of C; 0 = N; must be >= N        */
+    int32_t b_layout;   /* TG_B_KN or TG_B_NK                                    */
+    int32_t path;       /* TG_PATH_AUTO (0) or a forced kernel path (testing)     */
+    const void *bias;   /* device fp16[N], or NULL                                */
+    int64_t batch;      /* number of problems; 0 = 1                             */
+    int64_t stride_a;   /* elements between consecutive A, B and C entries;     */
+    int64_t stride_b;   /* C entries must not overlap each other                */
+    int64_t stride_c;
+} tg_gemm_options;
+
+/*
+ * C = ReLU(A . B + bias) with the layouts and batching of `options`.
+ * Operands TMA cannot describe (row or batch strides that are not multiples
+ * of 8 elements, bases that are not 16-byte aligned) go through the repack
+ * path when `workspace_bytes` >= tg_workspace_size_ex(...); without enough
+ * workspace, B stored K x N uses the edge mode and B stored N x K is refused
+ * (TG_ERR_INVALID_ARG).  Batch entries run in order on `stream` and share the
+ * workspace.  Errors as tg_gemm_relu_f16_ws, plus TG_ERR_INVALID_ARG for
+ * strides below the row lengths, overlapping C entries, an unknown b_layout
+ * or a forced path that cannot run these operands.
+ */
+TG_API tg_status tg_gemm_relu_f16_ex(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                                     const tg_gemm_options *options, void *stream, void *workspace,
+                                     int64_t workspace_bytes);
+
+/* Workspace bytes tg_gemm_relu_f16_ex needs for its repack path (0: none;
+ * -1: invalid arguments).  Host logic only. */
+TG_API int64_t tg_workspace_size_ex(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K,
+                                    const tg_gemm_options *options);
+
+/* The path tg_gemm_relu_f16_ex takes with `workspace_bytes` of workspace
+ * (-2: invalid arguments).  Host logic only. */
+TG_API int tg_select_path_ex(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K,
+                             const tg_gemm_options *options, int64_t workspace_bytes);
 
 /*
  * Workspace bytes tg_gemm_relu_f16_ws needs to take the repack path for these

@@ -151,3 +151,32 @@ def test_workspace_argument_checks():
     assert tg.gemm_relu_f16_ws_raw(A0, B0, C0, M, N, K, 0, 0, 64) == Status.INVALID_ARG           # NULL with bytes
     assert tg.gemm_relu_f16_ws_raw(A0, B0, C0, M, N, K, 0, W0, -5) == Status.INVALID_ARG
     assert tg.gemm_relu_f16_raw(A0, B0, C0, M, N, K, 0, Path.REPACK) == Status.INVALID_ARG        # needs _ws
+
+
+def test_extended_options_validation_and_paths():
+    o = tg.options(b_layout=tg.B_NK)
+    assert tg.select_path_ex(A0, B0, C0, 8192, 8192, 8192, o) == Path.TC_PAIR512
+    assert tg.select_path_ex(A0, B0, C0, 64, 8192, 8192, o) == Path.SKINNY
+    assert tg.select_path_ex(A0, B0, C0, 64, 8192, 8192, None) == Path.SKINNY
+    # Strides below the row lengths, overlapping C entries, unknown layouts are refused.
+    assert tg.select_path_ex(A0, B0, C0, 64, 128, 64, tg.options(ldc=100)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 64, 128, 64, tg.options(lda=32)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 64, 128, 64, tg.options(b_layout=tg.B_NK, ldb=32)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 64, 128, 64, tg.options(b_layout=7)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 64, 128, 64, tg.options(batch=2, stride_c=64 * 128 - 1)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 64, 128, 64, tg.options(batch=2, stride_a=64 * 64, stride_b=64 * 128,
+                                                                 stride_c=64 * 128)) == Path.SKINNY
+    # Padded strides that are multiples of 8 keep TMA; others need the repack path.
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=520, ldb=528, ldc=536)) == Path.TC_PAIR
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513)) == Path.TC_EDGE
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513), 1 << 30) == Path.REPACK
+    # B stored N x K with an odd K: only the repack path (the edge mode reads K x N).
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 511, tg.options(b_layout=tg.B_NK)) == Path.REPACK
+    up = lambda x: (x + 255) // 256 * 256
+    assert tg.workspace_size_ex(A0, B0, C0, 300, 200, 511, tg.options(b_layout=tg.B_NK)) == up(2 * 300 * 512) + up(2 * 200 * 512)
+    assert tg.workspace_size_ex(A0, B0, C0, 300, 200, 512, tg.options(b_layout=tg.B_NK, ldb=515)) == up(2 * 200 * 512)
+    # A forced path must be able to run the operands.
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(path=Path.TC_EDGE, b_layout=tg.B_NK)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(path=Path.TC)) == Path.TC
+    # A bias that overlaps C is refused.
+    assert tg.gemm_relu_f16_ex_raw(A0, B0, C0, 64, 64, 64, tg.options(bias=C0 + 64)) == Status.INVALID_ARG

@@ -6,24 +6,33 @@ This package only marshals arguments to it; the library is loaded on first
 use and every call raises if it is missing.
 """
 from ._binding import (  # noqa: F401
+    B_KN,
+    B_NK,
     EXPORTS,
+    GemmOptions,
     LIB_PATH,
     STATIC_WORKSPACE_BYTES,
     Path,
     Status,
     TGError,
+    bmm_relu,
     device_status,
     gemm_relu,
+    gemm_relu_f16_ex_raw,
     gemm_relu_f16_raw,
     gemm_relu_f16_static_ws_raw,
     gemm_relu_f16_ws_raw,
+    linear_relu,
     lib,
+    options,
     path_name,
     path_supports,
     select_path,
+    select_path_ex,
     select_path_ws,
     status_string,
     version,
     wait_timeout_selftest,
     workspace_size,
+    workspace_size_ex,
 )

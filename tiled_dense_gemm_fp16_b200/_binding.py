@@ -33,7 +33,6 @@ class Path(enum.IntEnum):
     TC = 1
     TC_EDGE = 2
     SKINNY = 3
-    GEMV = 4
     ZERO = 5
     TC_PAIR = 6
     TC_PAIR512 = 7
@@ -46,7 +45,29 @@ class TGError(RuntimeError):
         super().__init__(f"{what}: {status_string(status)} ({int(status)})" if what else status_string(status))
 
 
+B_KN, B_NK = 0, 1
+
+
+class GemmOptions(ctypes.Structure):
+    """Mirror of tg_gemm_options (include/tg_gemm.h)."""
+    _fields_ = [
+        ("lda", ctypes.c_int64),
+        ("ldb", ctypes.c_int64),
+        ("ldc", ctypes.c_int64),
+        ("b_layout", ctypes.c_int32),
+        ("path", ctypes.c_int32),
+        ("bias", ctypes.c_void_p),
+        ("batch", ctypes.c_int64),
+        ("stride_a", ctypes.c_int64),
+        ("stride_b", ctypes.c_int64),
+        ("stride_c", ctypes.c_int64),
+    ]
+
+
 EXPORTS = (
+    "tg_gemm_relu_f16_ex",
+    "tg_workspace_size_ex",
+    "tg_select_path_ex",
     "tg_gemm_relu_f16",
     "tg_gemm_relu_f16_path",
     "tg_gemm_relu_f16_ws",
@@ -82,6 +103,13 @@ def _bind(lib):
     lib.tg_select_path_ws.restype = i32
     lib.tg_gemm_relu_f16_static_ws.argtypes = [vp, vp, vp, i64, i64, i64, vp]
     lib.tg_gemm_relu_f16_static_ws.restype = i32
+    optp = ctypes.POINTER(GemmOptions)
+    lib.tg_gemm_relu_f16_ex.argtypes = [vp, vp, vp, i64, i64, i64, optp, vp, vp, i64]
+    lib.tg_gemm_relu_f16_ex.restype = i32
+    lib.tg_workspace_size_ex.argtypes = [vp, vp, vp, i64, i64, i64, optp]
+    lib.tg_workspace_size_ex.restype = i64
+    lib.tg_select_path_ex.argtypes = [vp, vp, vp, i64, i64, i64, optp, i64]
+    lib.tg_select_path_ex.restype = i32
     lib.tg_path_supports.argtypes = [i32, vp, vp, vp, i64, i64, i64]
     lib.tg_path_supports.restype = i32
     lib.tg_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
@@ -156,6 +184,28 @@ def workspace_size(A: int, B: int, C: int, M: int, N: int, K: int) -> int:
     return int(lib().tg_workspace_size(A, B, C, M, N, K))
 
 
+def options(lda=0, ldb=0, ldc=0, b_layout=B_KN, bias=0, batch=0, stride_a=0, stride_b=0, stride_c=0,
+            path=Path.AUTO) -> GemmOptions:
+    """A tg_gemm_options value (zeros mean the dense defaults)."""
+    return GemmOptions(lda, ldb, ldc, int(b_layout), int(path), bias or None, batch, stride_a, stride_b, stride_c)
+
+
+def gemm_relu_f16_ex_raw(A: int, B: int, C: int, M: int, N: int, K: int, opts: GemmOptions | None = None,
+                         stream: int = 0, ws: int = 0, ws_bytes: int = 0) -> int:
+    """tg_gemm_relu_f16_ex on raw device pointers; returns the tg_status value."""
+    return int(lib().tg_gemm_relu_f16_ex(A, B, C, M, N, K, ctypes.byref(opts) if opts is not None else None,
+                                         stream, ws, ws_bytes))
+
+
+def workspace_size_ex(A: int, B: int, C: int, M: int, N: int, K: int, opts: GemmOptions | None = None) -> int:
+    return int(lib().tg_workspace_size_ex(A, B, C, M, N, K, ctypes.byref(opts) if opts is not None else None))
+
+
+def select_path_ex(A: int, B: int, C: int, M: int, N: int, K: int, opts: GemmOptions | None = None,
+                   ws_bytes: int = 0) -> int:
+    return int(lib().tg_select_path_ex(A, B, C, M, N, K, ctypes.byref(opts) if opts is not None else None, ws_bytes))
+
+
 def select_path(A: int, B: int, C: int, M: int, N: int, K: int) -> int:
     return int(lib().tg_select_path(A, B, C, M, N, K))
 
@@ -227,4 +277,63 @@ def gemm_relu(A, B, out=None, path: int = Path.AUTO, stream=None, workspace="aut
                 return out
         st = gemm_relu_f16_raw(a, b, c, M, N, K, handle, path)
     _check(st, "tg_gemm_relu_f16")
+    return out
+
+
+def _call_ex(a, b, c, M, N, K, opts, device, stream, workspace):
+    import torch
+    handle = stream.cuda_stream if stream is not None else _stream_handle(device)
+    with torch.cuda.device(device):
+        need = workspace_size_ex(a, b, c, M, N, K, opts)
+        if need < 0:
+            raise TGError(Status.INVALID_ARG, "tg_workspace_size_ex")
+        ws_ptr, ws_bytes = 0, 0
+        if need > 0 and workspace is not None:
+            if isinstance(workspace, str):
+                workspace = torch.empty(need, dtype=torch.uint8, device=device)
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        st = gemm_relu_f16_ex_raw(a, b, c, M, N, K, opts, handle, ws_ptr, ws_bytes)
+    _check(st, "tg_gemm_relu_f16_ex")
+
+
+def linear_relu(x, weight, bias=None, out=None, stream=None, workspace="auto"):
+    """ReLU(x @ weight^T + bias) for fp16 CUDA tensors: x (..., K), weight (N, K) as a
+    linear layer stores it, bias (N,) or None.  Leading dimensions of x are flattened
+    into M rows (x must be contiguous)."""
+    import torch
+    if x.dtype != torch.float16 or weight.dtype != torch.float16:
+        raise TypeError("x and weight must be torch.float16")
+    if weight.dim() != 2 or x.shape[-1] != weight.shape[1]:
+        raise ValueError(f"shape mismatch: x{tuple(x.shape)} weight{tuple(weight.shape)}")
+    if not (x.is_contiguous() and weight.is_contiguous()):
+        raise ValueError("x and weight must be contiguous")
+    K = x.shape[-1]
+    N = weight.shape[0]
+    lead = tuple(x.shape[:-1])
+    M = 1
+    for d in lead:
+        M *= d
+    if bias is not None and (bias.dtype != torch.float16 or bias.numel() != N or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous float16 tensor of N elements")
+    if out is None:
+        out = torch.empty(lead + (N,), dtype=torch.float16, device=x.device)
+    opts = options(b_layout=B_NK, bias=bias.data_ptr() if bias is not None else 0)
+    _call_ex(x.data_ptr(), weight.data_ptr(), out.data_ptr(), M, N, K, opts, x.device, stream, workspace)
+    return out
+
+
+def bmm_relu(A, B, bias=None, out=None, stream=None, workspace="auto"):
+    """ReLU(A[e] @ B[e] + bias) for fp16 CUDA tensors A (b, M, K) and B (b, K, N)."""
+    import torch
+    if A.dim() != 3 or B.dim() != 3 or A.shape[0] != B.shape[0] or A.shape[2] != B.shape[1]:
+        raise ValueError(f"shape mismatch: A{tuple(A.shape)} B{tuple(B.shape)}")
+    if A.dtype != torch.float16 or B.dtype != torch.float16 or not (A.is_contiguous() and B.is_contiguous()):
+        raise ValueError("A and B must be contiguous float16 tensors")
+    nb, M, K = A.shape
+    N = B.shape[2]
+    if out is None:
+        out = torch.empty((nb, M, N), dtype=torch.float16, device=A.device)
+    opts = options(bias=bias.data_ptr() if bias is not None else 0, batch=nb, stride_a=M * K, stride_b=K * N,
+                   stride_c=M * N)
+    _call_ex(A.data_ptr(), B.data_ptr(), out.data_ptr(), M, N, K, opts, A.device, stream, workspace)
     return out

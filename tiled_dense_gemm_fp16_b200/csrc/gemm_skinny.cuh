@@ -28,6 +28,9 @@ namespace tg {
 
 struct SkinnyParams {
   __half* C;
+  const __half* bias;     // optional fp16[N] added before ReLU; nullptr = none
+  int64_t ldc;            // row stride of C (elements)
+  int b_kmajor;           // 1: B stored N x K, so the MMA's A operand is K-major
   int M, N, K;
   int m_pad;              // MMA N: M rounded up to a multiple of 16 (16..256)
   int k_blocks;           // ceil(K / 64)
@@ -120,8 +123,12 @@ __global__ void __launch_bounds__(SkinnyCfg::THREADS, 1)
         mbar_arrive_expect_tx(&full_bar[stage], tx);
         const int k0 = kb * Cfg::BK;
         uint8_t* bdst = b_smem + stage * Cfg::B_STAGE_BYTES;
-        tma_load_2d(bdst, &tmap_b, &full_bar[stage], n0, k0);
-        tma_load_2d(bdst + Cfg::B_BOX_BYTES, &tmap_b, &full_bar[stage], n0 + 64, k0);
+        if (p.b_kmajor) {
+          tma_load_2d(bdst, &tmap_b, &full_bar[stage], k0, n0);  // 128 n-rows x 64 k, K-major
+        } else {
+          tma_load_2d(bdst, &tmap_b, &full_bar[stage], n0, k0);
+          tma_load_2d(bdst + Cfg::B_BOX_BYTES, &tmap_b, &full_bar[stage], n0 + 64, k0);
+        }
         tma_load_2d(a_smem + stage * p.a_stage_bytes, &tmap_a, &full_bar[stage], k0, 0);
         if (p.prefetch_kb > 0 && kb + p.prefetch_kb < kb_hi) {
           const int kp = (kb + p.prefetch_kb) * Cfg::BK;
@@ -157,9 +164,10 @@ __global__ void __launch_bounds__(SkinnyCfg::THREADS, 1)
         const uint32_t a_addr = smem_u32(a_smem + stage * p.a_stage_bytes);
 #pragma unroll
         for (int k = 0; k < Cfg::BK / 16; ++k) {
-          // MMA A operand = B^T panel: MN-major, 64-column boxes 8 KiB apart,
-          // 16 k-rows (2 KiB) per step.
-          const uint64_t adesc = make_sw128_desc(b_addr + k * 2048, Cfg::B_BOX_BYTES, 1024);
+          // MMA A operand = B^T panel.  B as K x N: MN-major, 64-column boxes
+          // 8 KiB apart, 16 k-rows (2 KiB) per step.  B as N x K: K-major.
+          const uint64_t adesc = p.b_kmajor ? make_sw128_desc(b_addr + k * 32, 16, 1024)
+                                            : make_sw128_desc(b_addr + k * 2048, Cfg::B_BOX_BYTES, 1024);
           // MMA B operand = A^T: K-major rows of A, 32 bytes per 16-deep step.
           const uint64_t bdesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
           umma_f16_ss(tmem_base, adesc, bdesc, p.idesc, (i | k) != 0 ? 1u : 0u);
@@ -226,12 +234,22 @@ __global__ void __launch_bounds__(SkinnyCfg::THREADS, 1)
         acc.z += v.z;
         acc.w += v.w;
       }
+      if (p.bias != nullptr) {
+        const unsigned short* b16 = reinterpret_cast<const unsigned short*>(p.bias) + n;
+        float bb[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) bb[e] = (n + e < p.N) ? __half2float(__ushort_as_half(__ldg(b16 + e))) : 0.0f;
+        acc.x += bb[0];
+        acc.y += bb[1];
+        acc.z += bb[2];
+        acc.w += bb[3];
+      }
       const __half2 h01 = __floats2half2_rn(acc.x > 0.f ? acc.x : 0.f, acc.y > 0.f ? acc.y : 0.f);
       const __half2 h23 = __floats2half2_rn(acc.z > 0.f ? acc.z : 0.f, acc.w > 0.f ? acc.w : 0.f);
       uint2 packed;
       packed.x = *reinterpret_cast<const uint32_t*>(&h01);
       packed.y = *reinterpret_cast<const uint32_t*>(&h23);
-      __half* dst = p.C + static_cast<int64_t>(m) * p.N + n;
+      __half* dst = p.C + static_cast<int64_t>(m) * p.ldc + n;
       if (p.c_aligned) {
         *reinterpret_cast<uint2*>(dst) = packed;
       } else {

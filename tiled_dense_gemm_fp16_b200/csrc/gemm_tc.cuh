@@ -37,6 +37,9 @@ struct TcParams {
   const __half* A;
   const __half* B;
   __half* C;
+  const __half* bias;    // optional fp16[N], added to every row before ReLU; nullptr = none
+  int64_t lda, ldb, ldc; // row strides (elements) of A, of B as stored, and of C
+  int b_kmajor;          // 1: B is stored N x K (rows of length K; C = A . B^T)
   int M, N, K;
   int m_tiles, n_tiles, num_tiles, k_blocks;
   int group_m;           // tile rows per raster group
@@ -66,8 +69,6 @@ struct TcCfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + BAR_BYTES;
   static constexpr uint32_t FULL_COUNT = EDGE ? PRODUCER_WARPS * 32 : 1;
-  // A: K-major, B: MN-major (row-major K x N), M = 128, N = 256.
-  static constexpr uint32_t IDESC = make_idesc_f16_f32(BM, BN, false, true);
 };
 
 // ReLU on two fp32 accumulator values (every value that is not > 0 becomes
@@ -77,6 +78,40 @@ __device__ __forceinline__ uint32_t relu_pack_f16x2(uint32_t a, uint32_t b) {
   const float x1 = __uint_as_float(b);
   const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// 16 bias values bias[col .. col + 16) as fp32 (0 past N or without bias).
+// All lanes of a warp ask for the same columns, so each load is a broadcast.
+__device__ __forceinline__ void load_bias16(const __half* bias, int col, int N, float (&b)[16]) {
+  if (bias == nullptr) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) b[e] = 0.0f;
+    return;
+  }
+  const __half* src = bias + col;
+  if (col + 16 <= N && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const __half2 h2 = *reinterpret_cast<const __half2*>(&w[q]);
+      const float2 f = __half22float2(h2);
+      b[2 * q] = f.x;
+      b[2 * q + 1] = f.y;
+    }
+    return;
+  }
+  const unsigned short* s16 = reinterpret_cast<const unsigned short*>(src);
+#pragma unroll
+  for (int e = 0; e < 16; ++e)
+    b[e] = (col + e < N) ? __half2float(__ushort_as_half(__ldg(s16 + e))) : 0.0f;
+}
+
+// relu_pack_f16x2 of (a + bias_a, b + bias_b): the bias is added to the fp32
+// accumulator with one fp32 addition before ReLU.
+__device__ __forceinline__ uint32_t relu_pack_f16x2_bias(uint32_t a, uint32_t b, float ba, float bb) {
+  return relu_pack_f16x2(__float_as_uint(__uint_as_float(a) + ba), __float_as_uint(__uint_as_float(b) + bb));
 }
 
 // Store 32 consecutive fp16 values of one row of C, packed two per word in
@@ -271,9 +306,14 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
             const int k0 = kb * Cfg::BK;
             tma_load_2d(a_smem + stage * Cfg::A_BYTES, &tmap_a, &full_bar[stage], k0, m0);
             uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
+            if (p.b_kmajor) {
+              // B stored N x K: one box of BN rows (n) x 64 k, K-major like A.
+              tma_load_2d(bdst, &tmap_b, &full_bar[stage], k0, n0);
+            } else {
 #pragma unroll
-            for (int j = 0; j < Cfg::BN / 64; ++j)
-              tma_load_2d(bdst + j * Cfg::B_CHUNK_BYTES, &tmap_b, &full_bar[stage], n0 + j * 64, k0);
+              for (int j = 0; j < Cfg::BN / 64; ++j)
+                tma_load_2d(bdst + j * Cfg::B_CHUNK_BYTES, &tmap_b, &full_bar[stage], n0 + j * 64, k0);
+            }
             last_parity[stage] = static_cast<int>(phase);
             if (++stage == Cfg::STAGES) {
               stage = 0;
@@ -297,9 +337,9 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      const int64_t lda = p.K, ldb = p.N;
-      const __half* a_end = p.A + static_cast<int64_t>(p.M) * p.K;
-      const __half* b_end = p.B + static_cast<int64_t>(p.K) * p.N;
+      const int64_t lda = p.lda, ldb = p.ldb;
+      const __half* a_end = p.A + static_cast<int64_t>(p.M - 1) * lda + p.K;
+      const __half* b_end = p.B + static_cast<int64_t>(p.K - 1) * ldb + p.N;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         int m_blk, n_blk;
         tile_coords(p, t, m_blk, n_blk);
@@ -385,6 +425,7 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
+      const uint32_t idesc = make_idesc_f16_f32(Cfg::BM, Cfg::BN, false, p.b_kmajor == 0);
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -403,9 +444,11 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
           for (int k = 0; k < Cfg::BK / 16; ++k) {
             // A: advance 16 elements (32 bytes) inside the swizzled row.
             const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
-            // B: advance 16 k-rows (2048 bytes); 64-column panels 8 KiB apart.
-            const uint64_t bdesc = make_sw128_desc(b_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
-            umma_f16_ss(d_tmem, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
+            // B as K x N: advance 16 k-rows (2048 bytes); 64-column panels 8 KiB
+            // apart.  B as N x K: K-major like A.
+            const uint64_t bdesc = p.b_kmajor ? make_sw128_desc(b_addr + k * 32, 16, 1024)
+                                              : make_sw128_desc(b_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
+            umma_f16_ss(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit(&empty_bar[stage]);  // frees the stage when these MMAs finish
           if (++stage == Cfg::STAGES) {
@@ -439,23 +482,24 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
       tcgen05_fence_after_sync();
       const int row = m_blk * Cfg::BM + quad * 32 + lane;
       const bool row_ok = row < p.M;
-      __half* crow = p.C + static_cast<int64_t>(row) * p.N;
+      __half* crow = p.C + static_cast<int64_t>(row) * p.ldc;
 #pragma unroll 1
       for (int c = 0; c < Cfg::BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + c * 32, r);
         tmem_ld_wait();
         const int col0 = n_blk * Cfg::BN + c * 32;
-        if (row_ok && col0 < p.N) {
+        if (col0 < p.N) {
+          float b0[16], b1[16];
+          load_bias16(p.bias, col0, p.N, b0);
+          load_bias16(p.bias, col0 + 16, p.N, b1);
           uint32_t h[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = __uint_as_float(r[2 * e]);
-            const float x1 = __uint_as_float(r[2 * e + 1]);
-            const __half2 v = __floats2half2_rn(x0 > 0.0f ? x0 : 0.0f, x1 > 0.0f ? x1 : 0.0f);
-            h[e] = *reinterpret_cast<const uint32_t*>(&v);
-          }
-          store_row_chunk(crow, col0, p.N, h, p.c_aligned != 0, false);
+          for (int e = 0; e < 8; ++e) h[e] = relu_pack_f16x2_bias(r[2 * e], r[2 * e + 1], b0[2 * e], b0[2 * e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            h[8 + e] = relu_pack_f16x2_bias(r[16 + 2 * e], r[16 + 2 * e + 1], b1[2 * e], b1[2 * e + 1]);
+          if (row_ok) store_row_chunk(crow, col0, p.N, h, p.c_aligned != 0, false);
         }
       }
       tcgen05_fence_before_sync();

@@ -60,7 +60,6 @@ struct TcPairCfg {
   static constexpr int TMEM_COLS = 512;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + BAR_BYTES;
-  static constexpr uint32_t IDESC = make_idesc_f16_f32(PAIR_M, 256, false, true);
   static_assert(BN == 256 || BN == 512, "pair tile width");
   static_assert(NUM_ACC * BN <= TMEM_COLS, "TMEM columns");
 };
@@ -152,9 +151,14 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           tma_load_2d_pair_hint(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, k0, m0, pol_a);
 #pragma unroll
           for (int j = 0; j < Cfg::SLABS; ++j) {
-            tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, nb + 256 * j, k0, pol_b);
-            tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES + Cfg::B_CHUNK_BYTES, &tmap_b, full_even,
-                                  nb + 256 * j + 64, k0, pol_b);
+            if (p.b_kmajor) {
+              // B stored N x K: this CTA's 128 n-rows x 64 k of slab j, K-major.
+              tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, k0, nb + 256 * j, pol_b);
+            } else {
+              tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, nb + 256 * j, k0, pol_b);
+              tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES + Cfg::B_CHUNK_BYTES, &tmap_b, full_even,
+                                    nb + 256 * j + 64, k0, pol_b);
+            }
           }
           if (p.prefetch_kb > 0 && kb + p.prefetch_kb < p.k_blocks) {
             // Warm L2 with the boxes a few k-blocks ahead, so the ring's
@@ -163,8 +167,12 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
             tma_prefetch_l2_2d(&tmap_a, kp, m0);
 #pragma unroll
             for (int j = 0; j < Cfg::SLABS; ++j) {
-              tma_prefetch_l2_2d(&tmap_b, nb + 256 * j, kp);
-              tma_prefetch_l2_2d(&tmap_b, nb + 256 * j + 64, kp);
+              if (p.b_kmajor) {
+                tma_prefetch_l2_2d(&tmap_b, kp, nb + 256 * j);
+              } else {
+                tma_prefetch_l2_2d(&tmap_b, nb + 256 * j, kp);
+                tma_prefetch_l2_2d(&tmap_b, nb + 256 * j + 64, kp);
+              }
             }
           }
           last_parity[stage] = static_cast<int>(phase);
@@ -195,6 +203,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
+      const uint32_t idesc = make_idesc_f16_f32(Cfg::PAIR_M, 256, false, p.b_kmajor == 0);
       for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters, ++local) {
         const int acc = local % Cfg::NUM_ACC;
         const uint32_t acc_phase = (local / Cfg::NUM_ACC) & 1;
@@ -214,10 +223,12 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
             const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
 #pragma unroll
             for (int j = 0; j < Cfg::SLABS; ++j) {
-              // Slab j: this CTA's two 64-column panels, 8 KiB apart.
-              const uint64_t bdesc =
-                  make_sw128_desc(b_addr + j * Cfg::B_SLAB_BYTES + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
-              umma_f16_ss_pair(d_tmem + 256 * j, adesc, bdesc, Cfg::IDESC, (kb | k) != 0 ? 1u : 0u);
+              // Slab j: as K x N, this CTA's two 64-column panels, 8 KiB apart;
+              // as N x K, 128 K-major rows like A.
+              const uint32_t slab_addr = b_addr + j * Cfg::B_SLAB_BYTES;
+              const uint64_t bdesc = p.b_kmajor ? make_sw128_desc(slab_addr + k * 32, 16, 1024)
+                                                : make_sw128_desc(slab_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
+              umma_f16_ss_pair(d_tmem + 256 * j, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
             }
           }
           umma_commit_pair_mc(&empty_bar[stage], 0x3);  // both CTAs may refill this stage
@@ -253,7 +264,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
       tcgen05_fence_after_sync();
       const int row = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM + quad * 32 + lane;
       const bool row_ok = row < p.M;
-      __half* crow = p.C + static_cast<int64_t>(row) * p.N;
+      __half* crow = p.C + static_cast<int64_t>(row) * p.ldc;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * Cfg::BN + col_base;
       if (Cfg::NUM_ACC == 1) {
         // Single accumulator: read this thread's EPI_COLS columns into
@@ -265,8 +276,15 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           uint32_t r[16];  // 16 columns at a time keeps the register peak low
           tmem_ld_32x32b_x16(taddr + c * 16, r);
           tmem_ld_wait();
+          if (p.bias != nullptr) {
+            float bv[16];
+            load_bias16(p.bias, n_blk * Cfg::BN + col_base + c * 16, p.N, bv);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) h[c * 8 + e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
+            for (int e = 0; e < 8; ++e) h[c * 8 + e] = relu_pack_f16x2_bias(r[2 * e], r[2 * e + 1], bv[2 * e], bv[2 * e + 1]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) h[c * 8 + e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
+          }
         }
         tcgen05_fence_before_sync();
         __syncwarp();
@@ -289,9 +307,15 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           tmem_ld_wait();
           const int col0 = n_blk * Cfg::BN + col_base + c * 32;
           if (row_ok && col0 < p.N) {
+            float b0[16], b1[16];
+            load_bias16(p.bias, col0, p.N, b0);
+            load_bias16(p.bias, col0 + 16, p.N, b1);
             uint32_t hc[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) hc[e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
+            for (int e = 0; e < 8; ++e) hc[e] = relu_pack_f16x2_bias(r[2 * e], r[2 * e + 1], b0[2 * e], b0[2 * e + 1]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              hc[8 + e] = relu_pack_f16x2_bias(r[16 + 2 * e], r[16 + 2 * e + 1], b1[2 * e], b1[2 * e + 1]);
             store_row_chunk(crow, col0, p.N, hc, p.c_aligned != 0, p.store_streaming != 0);
           }
         }

@@ -24,6 +24,7 @@ namespace tg {
 struct RepackParams {
   const __half* src;
   __half* dst;
+  int64_t src_ld;            // row stride of the source (elements, >= cols)
   int rows, cols, cols_pad;  // cols_pad = cols rounded up to a multiple of 8
   int64_t chunks;            // rows * cols_pad / 8
 };
@@ -33,7 +34,7 @@ __global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
   grid_dependency_wait();
   grid_launch_dependents();
   const int chunks_per_row = p.cols_pad >> 3;
-  const __half* src_end = p.src + static_cast<int64_t>(p.rows) * p.cols;
+  const __half* src_end = p.src + static_cast<int64_t>(p.rows - 1) * p.src_ld + p.cols;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < p.chunks;
        base += stride * kUnroll) {
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
       live[u] = c < p.chunks;
       row[u] = live[u] ? static_cast<int>(c / chunks_per_row) : 0;
       col[u] = live[u] ? static_cast<int>(c - static_cast<int64_t>(row[u]) * chunks_per_row) * 8 : 0;
-      plan[u] = edge_chunk_plan(p.src, src_end, p.cols, live[u] ? row[u] : p.rows, p.rows, col[u], p.cols);
+      plan[u] = edge_chunk_plan(p.src, src_end, p.src_ld, live[u] ? row[u] : p.rows, p.rows, col[u], p.cols);
     }
     uint4 lo[kUnroll], hi[kUnroll];
 #pragma unroll
@@ -60,9 +61,35 @@ __global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
     for (int u = 0; u < kUnroll; ++u) {
       if (!live[u]) continue;
       const uint4 v = plan[u].fast ? edge_realign(lo[u], hi[u], plan[u].shift)
-                                   : load_chunk_pred(p.src, p.cols, row[u], p.rows, col[u], p.cols);
+                                   : load_chunk_pred(p.src, p.src_ld, row[u], p.rows, col[u], p.cols);
       *reinterpret_cast<uint4*>(p.dst + static_cast<int64_t>(row[u]) * p.cols_pad + col[u]) = v;
     }
+  }
+}
+
+}  // namespace tg
+
+namespace tg {
+
+// K == 0 with a bias: every row of C is ReLU(bias) rounded to fp16 (the sum
+// over an empty K range is zero).
+struct BiasRowsParams {
+  __half* C;
+  const __half* bias;
+  int64_t ldc;
+  int M, N;
+};
+
+__global__ void __launch_bounds__(256) bias_relu_rows_kernel(const BiasRowsParams p) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t total = static_cast<int64_t>(p.M) * p.N;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int m = static_cast<int>(i / p.N);
+    const int n = static_cast<int>(i - static_cast<int64_t>(m) * p.N);
+    const float b = __half2float(p.bias[n]);
+    p.C[static_cast<int64_t>(m) * p.ldc + n] = __float2half_rn(b > 0.0f ? b : 0.0f);
   }
 }
 

@@ -63,97 +63,149 @@ int tune_int(const char* name, int dflt) {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 bool g_encode_probed = false;
 
-// One GEMM as the kernels see it: A has rows of `lda` elements (K, or K
-// rounded up to 8 in a zero-padded copy), B has rows of `ldb` elements (N, or
-// N rounded up to 8), C is dense M x N.  c_aligned: every row of C starts on
-// a 16-byte boundary.
+// One problem as the caller describes it: batch entries of
+//   C[i*ldc + j] = f16(relu(sum_k A[i*lda + k] * b(k, j) + bias[j]))
+// with b(k, j) = B[k*ldb + j] (B stored K x N) or B[j*ldb + k] (B stored
+// N x K), entry e starting at A + e*sa, B + e*sb, C + e*sc (elements).
+struct Problem {
+  const void* A;
+  const void* B;
+  void* C;
+  int64_t M, N, K;
+  int64_t lda, ldb, ldc;
+  bool b_nk;
+  const void* bias;
+  int64_t batch, sa, sb, sc;
+};
+
+Problem dense_problem(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K) {
+  return Problem{A, B, C, M, N, K, K, N, N, false, nullptr, 1, 0, 0, 0};
+}
+
+// One GEMM as the kernels see it (one batch entry, possibly repacked).
 struct Operands {
   const void* A;
   int64_t lda;
   const void* B;
   int64_t ldb;
+  bool b_nk;
   void* C;
+  int64_t ldc;
+  const void* bias;
   int64_t M, N, K;
-  bool c_aligned;
+  bool c_aligned;  // every row of C starts on a 16-byte boundary
 };
 
 // ---------------------------------------------------------------------------
 // Host-side argument logic (no CUDA calls)
 // ---------------------------------------------------------------------------
+constexpr int64_t kMaxStride = int64_t(1) << 40;  // elements; keeps every byte offset in int64
+
 bool ranges_overlap(const void* a, int64_t a_bytes, const void* b, int64_t b_bytes) {
   if (a_bytes <= 0 || b_bytes <= 0) return false;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
   return a0 < b0 + static_cast<uintptr_t>(b_bytes) && b0 < a0 + static_cast<uintptr_t>(a_bytes);
 }
 
-bool args_valid(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
-  if (M < 0 || N < 0 || K < 0) return false;
-  if (M > INT_MAX || N > INT_MAX || K > INT_MAX) return false;
-  if (M == 0 || N == 0) return true;
-  if (C == nullptr) return false;
-  if (K > 0 && (A == nullptr || B == nullptr)) return false;
-  const uintptr_t bits = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) |
-                         reinterpret_cast<uintptr_t>(C);
-  if (bits & 1u) return false;
-  const int64_t c_bytes = 2 * M * N;
-  if (K > 0 && (ranges_overlap(C, c_bytes, A, 2 * M * K) || ranges_overlap(C, c_bytes, B, 2 * K * N)))
+// Bytes each operand spans over all batch entries.
+int64_t span_a(const Problem& p) {
+  return (p.M > 0 && p.K > 0) ? 2 * ((p.batch - 1) * p.sa + (p.M - 1) * p.lda + p.K) : 0;
+}
+int64_t span_b(const Problem& p) {
+  if (p.K <= 0 || p.N <= 0) return 0;
+  const int64_t one = p.b_nk ? (p.N - 1) * p.ldb + p.K : (p.K - 1) * p.ldb + p.N;
+  return 2 * ((p.batch - 1) * p.sb + one);
+}
+int64_t span_c_one(const Problem& p) { return (p.M > 0 && p.N > 0) ? (p.M - 1) * p.ldc + p.N : 0; }
+int64_t span_c(const Problem& p) { return (p.M > 0 && p.N > 0) ? 2 * ((p.batch - 1) * p.sc + span_c_one(p)) : 0; }
+
+bool problem_valid(const Problem& p) {
+  if (p.M < 0 || p.N < 0 || p.K < 0) return false;
+  if (p.M > INT_MAX || p.N > INT_MAX || p.K > INT_MAX) return false;
+  if (p.batch < 1 || p.batch > INT_MAX) return false;
+  if (p.M == 0 || p.N == 0) return true;
+  if (p.lda < (p.K > 0 ? p.K : 0) || p.ldc < p.N) return false;
+  if (p.ldb < (p.b_nk ? p.K : p.N)) return false;
+  if (p.lda > kMaxStride || p.ldb > kMaxStride || p.ldc > kMaxStride) return false;
+  if (p.sa < 0 || p.sb < 0 || p.sc < 0 || p.sa > kMaxStride || p.sb > kMaxStride || p.sc > kMaxStride)
     return false;
+  if (p.batch > 1 && p.sc < span_c_one(p)) return false;  // C entries must not overlap each other
+  if (p.C == nullptr) return false;
+  if (p.K > 0 && (p.A == nullptr || p.B == nullptr)) return false;
+  const uintptr_t bits = reinterpret_cast<uintptr_t>(p.A) | reinterpret_cast<uintptr_t>(p.B) |
+                         reinterpret_cast<uintptr_t>(p.C) | reinterpret_cast<uintptr_t>(p.bias);
+  if (bits & 1u) return false;
+  const int64_t c_bytes = span_c(p);
+  if (p.K > 0 && (ranges_overlap(p.C, c_bytes, p.A, span_a(p)) || ranges_overlap(p.C, c_bytes, p.B, span_b(p))))
+    return false;
+  if (p.bias && ranges_overlap(p.C, c_bytes, p.bias, 2 * p.N)) return false;
   // Tile counts must fit the kernels' 32-bit tile indices.
-  const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
+  const int64_t tiles = ((p.M + 127) / 128) * ((p.N + 255) / 256);
   if (tiles > INT_MAX) return false;
   return true;
 }
 
-// TMA can describe A and B: 16-byte aligned bases and row strides.
-bool tma_ok(const void* A, const void* B, int64_t N, int64_t K) {
-  const uintptr_t bits = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B);
-  return (bits & 15u) == 0 && (N % 8) == 0 && (K % 8) == 0;
+// TMA can describe A (B) in every batch entry: 16-byte aligned bases, row
+// strides and batch strides.
+bool tma_ok_a(const Problem& p) {
+  return (reinterpret_cast<uintptr_t>(p.A) & 15u) == 0 && p.lda % 8 == 0 && (p.batch == 1 || p.sa % 8 == 0);
 }
+bool tma_ok_b(const Problem& p) {
+  return (reinterpret_cast<uintptr_t>(p.B) & 15u) == 0 && p.ldb % 8 == 0 && (p.batch == 1 || p.sb % 8 == 0);
+}
+bool tma_ok(const Problem& p) { return tma_ok_a(p) && tma_ok_b(p); }
 
-// Every row of C starts on a 16-byte boundary.
-bool c_rows_aligned(const void* C, int64_t N) {
-  return (reinterpret_cast<uintptr_t>(C) & 15u) == 0 && (N % 8) == 0;
+// Every row of C, in every batch entry, starts on a 16-byte boundary.
+bool c_rows_aligned(const Problem& p) {
+  return (reinterpret_cast<uintptr_t>(p.C) & 15u) == 0 && p.ldc % 8 == 0 && (p.batch == 1 || p.sc % 8 == 0);
 }
 
 // Workspace of the repack path: zero-padded copies (rows rounded up to 8
-// elements) of whichever of A and B TMA cannot describe, each 256-byte aligned.
+// elements) of one batch entry of whichever of A and B TMA cannot describe,
+// each 256-byte aligned; batch entries reuse it in stream order.
 struct RepackPlan {
   bool pad_a = false, pad_b = false;
   int64_t kp = 0, np = 0;
   int64_t off_a = 0, off_b = 0, bytes = 0;
 };
 
-RepackPlan repack_plan(const void* A, const void* B, int64_t M, int64_t N, int64_t K) {
+RepackPlan repack_plan(const Problem& p) {
   RepackPlan r;
-  r.kp = (K + 7) / 8 * 8;
-  r.np = (N + 7) / 8 * 8;
-  r.pad_a = (K % 8) != 0 || (reinterpret_cast<uintptr_t>(A) & 15u) != 0;
-  r.pad_b = (N % 8) != 0 || (reinterpret_cast<uintptr_t>(B) & 15u) != 0;
+  r.kp = (p.K + 7) / 8 * 8;
+  r.np = (p.N + 7) / 8 * 8;
+  r.pad_a = !tma_ok_a(p);
+  r.pad_b = !tma_ok_b(p);
   auto up256 = [](int64_t x) { return (x + 255) / 256 * 256; };
-  const int64_t bytes_a = r.pad_a ? up256(2 * M * r.kp) : 0;
-  const int64_t bytes_b = r.pad_b ? up256(2 * K * r.np) : 0;
+  const int64_t bytes_a = r.pad_a ? up256(2 * p.M * r.kp) : 0;
+  const int64_t bytes_b = r.pad_b ? up256(p.b_nk ? 2 * p.N * r.kp : 2 * p.K * r.np) : 0;
   r.off_a = 0;
   r.off_b = bytes_a;
   r.bytes = bytes_a + bytes_b;
   return r;
 }
 
-bool path_supports(int path, const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
-  if (!args_valid(A, B, C, M, N, K)) return false;
-  if (M == 0 || N == 0) return path == TG_PATH_NONE || path == TG_PATH_AUTO;
-  if (K == 0) return path == TG_PATH_ZERO || path == TG_PATH_AUTO;
+int64_t workspace_bytes_needed(const Problem& p) {
+  if (p.M == 0 || p.N == 0 || p.K == 0 || tma_ok(p)) return 0;
+  return repack_plan(p).bytes;
+}
+
+bool path_supports(int path, const Problem& p) {
+  if (!problem_valid(p)) return false;
+  if (p.M == 0 || p.N == 0) return path == TG_PATH_NONE || path == TG_PATH_AUTO;
+  if (p.K == 0) return path == TG_PATH_ZERO || path == TG_PATH_AUTO;
   switch (path) {
     case TG_PATH_AUTO:
-    case TG_PATH_TC_EDGE:
       return true;
+    case TG_PATH_TC_EDGE:
+      return !p.b_nk;  // the realigning producer reads B stored K x N
     case TG_PATH_TC:
     case TG_PATH_TC_PAIR:
     case TG_PATH_TC_PAIR512:
-      return tma_ok(A, B, N, K);
+      return tma_ok(p);
     case TG_PATH_SKINNY:
-      return tma_ok(A, B, N, K) && M <= kSkinnyMaxM;
+      return tma_ok(p) && p.M <= kSkinnyMaxM;
     case TG_PATH_REPACK:
-      return !tma_ok(A, B, N, K);
+      return !tma_ok(p);
     default:
       return false;
   }
@@ -163,10 +215,10 @@ bool path_supports(int path, const void* A, const void* B, const void* C, int64_
 // device: waves of tiles x per-SM work of one tile.  The main loop of a tile
 // costs its per-SM MACs over the kernel's measured relative efficiency
 // (single CTA 0.85, pair 256x256 0.88, pair 256x512 1.0 at 8192^3).  The
-// 256x512 tile has one accumulator, so each tile's epilogue (draining TMEM and
-// storing C, worth about 384 k-steps of MMA, twice that when the rows of C are
-// only 2-byte aligned) adds to every tile; the double-buffered kernels hide
-// it behind the next tile and pay it once at the end.
+// 256x512 tile has one accumulator, so each tile's epilogue (draining TMEM,
+// worth about 384 k-steps of MMA, twice that when the rows of C are only
+// 2-byte aligned) adds to every tile; the double-buffered kernels hide it
+// behind the next tile and pay it once at the end.
 int pick_tc_kernel(int64_t M, int64_t N, int64_t K, bool c_aligned) {
   constexpr int64_t kSms = 148, kPairs = 74;
   auto waves = [](int64_t tiles, int64_t units) { return static_cast<double>((tiles + units - 1) / units); };
@@ -180,27 +232,24 @@ int pick_tc_kernel(int64_t M, int64_t N, int64_t K, bool c_aligned) {
   return t2 <= t1 ? TG_PATH_TC_PAIR : TG_PATH_TC;
 }
 
-int select_path(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
-  if (!args_valid(A, B, C, M, N, K)) return -2;
-  if (M == 0 || N == 0) return TG_PATH_NONE;
-  if (K == 0) return TG_PATH_ZERO;
-  if (!tma_ok(A, B, N, K)) return TG_PATH_TC_EDGE;
-  if (M <= kSkinnyMaxM) return TG_PATH_SKINNY;
-  return pick_tc_kernel(M, N, K, c_rows_aligned(C, N));
-}
-
-// As select_path, for a call that offers `ws_bytes` of workspace: operands
-// TMA cannot describe go through the repack path when the workspace suffices.
-int select_path_ws(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K,
-                   int64_t ws_bytes) {
-  const int path = select_path(A, B, C, M, N, K);
-  if (path == TG_PATH_TC_EDGE && ws_bytes >= repack_plan(A, B, M, N, K).bytes) return TG_PATH_REPACK;
-  return path;
-}
-
 // The tensor-core kernel that runs on TMA-describable (possibly repacked) operands.
-int inner_path(int64_t M, int64_t N, int64_t K, bool c_aligned) {
-  return M <= kSkinnyMaxM ? TG_PATH_SKINNY : pick_tc_kernel(M, N, K, c_aligned);
+int inner_path(const Problem& p) {
+  return p.M <= kSkinnyMaxM ? TG_PATH_SKINNY : pick_tc_kernel(p.M, p.N, p.K, c_rows_aligned(p));
+}
+
+// The path a call takes with `ws_bytes` of workspace (-2: invalid arguments).
+// Operands TMA cannot describe take the repack path when the workspace
+// suffices, else the edge mode (B stored K x N) or, for B stored N x K, the
+// repack path that run() then refuses for want of a workspace.
+int select_path(const Problem& p, int64_t ws_bytes) {
+  if (!problem_valid(p)) return -2;
+  if (p.M == 0 || p.N == 0) return TG_PATH_NONE;
+  if (p.K == 0) return TG_PATH_ZERO;
+  if (!tma_ok(p)) {
+    if (ws_bytes >= repack_plan(p).bytes || p.b_nk) return TG_PATH_REPACK;
+    return TG_PATH_TC_EDGE;
+  }
+  return inner_path(p);
 }
 
 // ---------------------------------------------------------------------------
@@ -244,19 +293,45 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return g_encode_tiled;
 }
 
-// Row-major (rows x cols) fp16 matrix; box = box_cols x box_rows, 128-byte
-// swizzle (box_cols * 2 must be 128).
-bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+// Row-major fp16 matrix of rows x cols with a row stride of `ld` elements
+// (ld * 2 a multiple of 16); box = box_cols x box_rows, 128-byte swizzle
+// (box_cols * 2 must be 128).  Columns past `cols` read as zero.
+bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_cols,
+               int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estride[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estride,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Tensor maps of one GEMM's A (box 64 k x a_rows) and B: stored K x N, boxes
+// of 64 n x 64 k; stored N x K, boxes of 64 k x b_rows.
+bool encode_operands(const Operands& o, CUtensorMap* ta, CUtensorMap* tb, int a_rows, int b_rows) {
+  if (!encode_2d(ta, o.A, o.M, o.K, o.lda, 64, a_rows)) return false;
+  if (o.b_nk) return encode_2d(tb, o.B, o.N, o.K, o.ldb, 64, b_rows);
+  return encode_2d(tb, o.B, o.K, o.N, o.ldb, 64, 64);
+}
+
+void fill_tc_params(TcParams& p, const Operands& o) {
+  std::memset(&p, 0, sizeof p);
+  p.A = static_cast<const __half*>(o.A);
+  p.B = static_cast<const __half*>(o.B);
+  p.C = static_cast<__half*>(o.C);
+  p.bias = static_cast<const __half*>(o.bias);
+  p.lda = o.lda;
+  p.ldb = o.ldb;
+  p.ldc = o.ldc;
+  p.b_kmajor = o.b_nk ? 1 : 0;
+  p.M = static_cast<int>(o.M);
+  p.N = static_cast<int>(o.N);
+  p.K = static_cast<int>(o.K);
+  p.c_aligned = o.c_aligned ? 1 : 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -306,28 +381,15 @@ tg_status launch_tc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   CUtensorMap ta, tb;
   std::memset(&ta, 0, sizeof ta);
   std::memset(&tb, 0, sizeof tb);
-  if (!EDGE) {
-    if (!encode_2d(&ta, o.A, M, o.lda, 64, Cfg::BM)) return TG_ERR_LAUNCH;
-    if (!encode_2d(&tb, o.B, K, o.ldb, 64, Cfg::BK)) return TG_ERR_LAUNCH;
-  }
+  if (!EDGE && !encode_operands(o, &ta, &tb, Cfg::BM, Cfg::BN)) return TG_ERR_LAUNCH;
   TcParams p;
-  std::memset(&p, 0, sizeof p);
-  p.A = static_cast<const __half*>(o.A);
-  p.B = static_cast<const __half*>(o.B);
-  p.C = static_cast<__half*>(o.C);
-  p.M = static_cast<int>(M);
-  p.N = static_cast<int>(N);
-  p.K = static_cast<int>(K);
+  fill_tc_params(p, o);
   p.m_tiles = static_cast<int>((M + Cfg::BM - 1) / Cfg::BM);
   p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
   p.group_m = tune_int("TG_TUNE_GROUP_M", 16);
   if (p.group_m < 1) p.group_m = 1;
-  p.store_streaming = 0;
-  p.l2_hints = 0;
-  p.prefetch_kb = 0;
-  p.c_aligned = o.c_aligned ? 1 : 0;
   p.wait_budget_ns = wait_budget(p.k_blocks);
   const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
   cudaLaunchConfig_t cfg;
@@ -364,16 +426,9 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
     }
   }
   CUtensorMap ta, tb;
-  if (!encode_2d(&ta, o.A, M, o.lda, 64, Cfg::BM)) return TG_ERR_LAUNCH;
-  if (!encode_2d(&tb, o.B, K, o.ldb, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+  if (!encode_operands(o, &ta, &tb, Cfg::BM, 128)) return TG_ERR_LAUNCH;
   TcParams p;
-  std::memset(&p, 0, sizeof p);
-  p.A = static_cast<const __half*>(o.A);
-  p.B = static_cast<const __half*>(o.B);
-  p.C = static_cast<__half*>(o.C);
-  p.M = static_cast<int>(M);
-  p.N = static_cast<int>(N);
-  p.K = static_cast<int>(K);
+  fill_tc_params(p, o);
   p.m_tiles = static_cast<int>((M + Cfg::PAIR_M - 1) / Cfg::PAIR_M);
   p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
   p.num_tiles = p.m_tiles * p.n_tiles;
@@ -383,7 +438,6 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
   p.store_streaming = tune_int("TG_TUNE_STORE_CS", 1);
   p.l2_hints = tune_int("TG_TUNE_L2_HINTS", BN == 512 ? 2 : 5);
   p.prefetch_kb = tune_int("TG_TUNE_PREFETCH_KB", 0);
-  p.c_aligned = o.c_aligned ? 1 : 0;
   p.wait_budget_ns = wait_budget(p.k_blocks);
   const int pairs = info->sm_count / 2;
   const int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
@@ -436,10 +490,13 @@ tg_status launch_skinny(const Operands& o, cudaStream_t stream, DeviceInfo* info
   SkinnyParams p;
   std::memset(&p, 0, sizeof p);
   p.C = static_cast<__half*>(o.C);
+  p.bias = static_cast<const __half*>(o.bias);
+  p.ldc = o.ldc;
+  p.b_kmajor = o.b_nk ? 1 : 0;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.c_aligned = (reinterpret_cast<uintptr_t>(o.C) % 8 == 0 && N % 4 == 0) ? 1 : 0;
+  p.c_aligned = (reinterpret_cast<uintptr_t>(o.C) % 8 == 0 && o.ldc % 4 == 0) ? 1 : 0;
   p.m_pad = static_cast<int>((M + 15) / 16 * 16);
   p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
   // Two CTAs per SM fit while the ring stays within ~112 KiB (M_pad <= 128).
@@ -460,7 +517,7 @@ tg_status launch_skinny(const Operands& o, cudaStream_t stream, DeviceInfo* info
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(p.m_pad)) cols <<= 1;
   p.tmem_cols = cols;
-  p.idesc = make_idesc_f16_f32(Cfg::PANEL, p.m_pad, true, false);
+  p.idesc = make_idesc_f16_f32(Cfg::PANEL, p.m_pad, !o.b_nk, false);
   p.prefetch_kb = tune_int("TG_TUNE_SKINNY_PREFETCH_KB", 0);
   p.wait_budget_ns = wait_budget(p.k_blocks);
   const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);  // panels past N are not stored
@@ -472,8 +529,7 @@ tg_status launch_skinny(const Operands& o, cudaStream_t stream, DeviceInfo* info
   if (panels > 65535) return TG_ERR_INVALID_ARG;
 
   CUtensorMap ta, tb;
-  if (!encode_2d(&ta, o.A, M, o.lda, 64, p.m_pad)) return TG_ERR_LAUNCH;
-  if (!encode_2d(&tb, o.B, K, o.ldb, 64, Cfg::BK)) return TG_ERR_LAUNCH;
+  if (!encode_operands(o, &ta, &tb, p.m_pad, Cfg::PANEL)) return TG_ERR_LAUNCH;
 
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
@@ -523,16 +579,10 @@ tg_status launch_path(int path, const Operands& o, cudaStream_t stream, DeviceIn
   }
 }
 
-tg_status launch_pad(const void* src, void* dst, int64_t rows, int64_t cols, int64_t cols_pad, cudaStream_t stream,
-                     DeviceInfo* info) {
-  RepackParams rp;
-  rp.src = static_cast<const __half*>(src);
-  rp.dst = static_cast<__half*>(dst);
-  rp.rows = static_cast<int>(rows);
-  rp.cols = static_cast<int>(cols);
-  rp.cols_pad = static_cast<int>(cols_pad);
-  rp.chunks = rows * (cols_pad / 8);
-  int64_t blocks = (rp.chunks + 256 * 4 - 1) / (256 * 4);
+template <typename Kernel, typename Params>
+tg_status launch_simple(Kernel kernel, const Params& params, int64_t work_items, int per_thread,
+                        cudaStream_t stream, DeviceInfo* info) {
+  int64_t blocks = (work_items + 256 * per_thread - 1) / (256 * per_thread);
   const int64_t cap = static_cast<int64_t>(info->sm_count) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
@@ -543,27 +593,61 @@ tg_status launch_pad(const void* src, void* dst, int64_t rows, int64_t cols, int
   cfg.stream = stream;
   LaunchAttrs la;
   la.fill(cfg, 1);
-  if (cudaLaunchKernelEx(&cfg, pad_rows_kernel, rp) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel, params) != cudaSuccess) {
     cudaGetLastError();
     return TG_ERR_LAUNCH;
   }
   return TG_OK;
 }
 
-tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream_ptr, int path,
-              void* ws, int64_t ws_bytes) {
-  if (!args_valid(A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
+tg_status launch_pad(const void* src, int64_t src_ld, void* dst, int64_t rows, int64_t cols, int64_t cols_pad,
+                     cudaStream_t stream, DeviceInfo* info) {
+  RepackParams rp;
+  rp.src = static_cast<const __half*>(src);
+  rp.dst = static_cast<__half*>(dst);
+  rp.src_ld = src_ld;
+  rp.rows = static_cast<int>(rows);
+  rp.cols = static_cast<int>(cols);
+  rp.cols_pad = static_cast<int>(cols_pad);
+  rp.chunks = rows * (cols_pad / 8);
+  return launch_simple(pad_rows_kernel, rp, rp.chunks, 4, stream, info);
+}
+
+// K == 0: C = ReLU(bias), or +0 without a bias (the empty sum).
+tg_status launch_k_zero(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
+  if (o.bias == nullptr) {
+    const cudaError_t e = (o.ldc == o.N)
+        ? cudaMemsetAsync(o.C, 0, static_cast<size_t>(2 * o.M * o.N), stream)
+        : cudaMemset2DAsync(o.C, static_cast<size_t>(2 * o.ldc), 0, static_cast<size_t>(2 * o.N),
+                            static_cast<size_t>(o.M), stream);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
+  }
+  BiasRowsParams bp;
+  bp.C = static_cast<__half*>(o.C);
+  bp.bias = static_cast<const __half*>(o.bias);
+  bp.ldc = o.ldc;
+  bp.M = static_cast<int>(o.M);
+  bp.N = static_cast<int>(o.N);
+  return launch_simple(bias_relu_rows_kernel, bp, o.M * o.N, 1, stream, info);
+}
+
+tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws_bytes) {
+  if (!problem_valid(p)) return TG_ERR_INVALID_ARG;
   if (ws_bytes < 0 || (ws_bytes > 0 && ws == nullptr)) return TG_ERR_INVALID_ARG;
-  if (path == TG_PATH_AUTO) path = select_path_ws(A, B, C, M, N, K, ws ? ws_bytes : 0);
-  if (!path_supports(path, A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
+  if (path == TG_PATH_AUTO) path = select_path(p, ws ? ws_bytes : 0);
+  if (!path_supports(path, p)) return TG_ERR_INVALID_ARG;
   if (path == TG_PATH_NONE) return TG_OK;
   RepackPlan plan;
   if (path == TG_PATH_REPACK) {
-    plan = repack_plan(A, B, M, N, K);
+    plan = repack_plan(p);
     if (ws == nullptr || ws_bytes < plan.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
       return TG_ERR_INVALID_ARG;
-    if (ranges_overlap(ws, plan.bytes, A, 2 * M * K) || ranges_overlap(ws, plan.bytes, B, 2 * K * N) ||
-        ranges_overlap(ws, plan.bytes, C, 2 * M * N))
+    if (ranges_overlap(ws, plan.bytes, p.A, span_a(p)) || ranges_overlap(ws, plan.bytes, p.B, span_b(p)) ||
+        ranges_overlap(ws, plan.bytes, p.C, span_c(p)) || (p.bias && ranges_overlap(ws, plan.bytes, p.bias, 2 * p.N)))
       return TG_ERR_INVALID_ARG;
   }
   int dev = 0;
@@ -571,31 +655,65 @@ tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64
   tg_status st = current_device(dev, info);
   if (st != TG_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  Operands o{A, K, B, N, C, M, N, K, c_rows_aligned(C, N)};
-  if (path == TG_PATH_ZERO) {
-    if (cudaMemsetAsync(C, 0, static_cast<size_t>(2 * M * N), stream) != cudaSuccess) {
-      cudaGetLastError();
-      return TG_ERR_LAUNCH;
+  const int inner = (path == TG_PATH_REPACK) ? inner_path(p) : path;
+  for (int64_t e = 0; e < p.batch; ++e) {
+    Operands o{static_cast<const uint8_t*>(p.A) + 2 * e * p.sa,
+               p.lda,
+               static_cast<const uint8_t*>(p.B) + 2 * e * p.sb,
+               p.ldb,
+               p.b_nk,
+               static_cast<uint8_t*>(p.C) + 2 * e * p.sc,
+               p.ldc,
+               p.bias,
+               p.M,
+               p.N,
+               p.K,
+               c_rows_aligned(p)};
+    if (path == TG_PATH_ZERO) {
+      st = launch_k_zero(o, stream, info);
+    } else if (path == TG_PATH_REPACK) {
+      uint8_t* base = static_cast<uint8_t*>(ws);
+      if (plan.pad_a) {
+        st = launch_pad(o.A, o.lda, base + plan.off_a, p.M, p.K, plan.kp, stream, info);
+        if (st != TG_OK) return st;
+        o.A = base + plan.off_a;
+        o.lda = plan.kp;
+      }
+      if (plan.pad_b) {
+        const int64_t rows = p.b_nk ? p.N : p.K, cols = p.b_nk ? p.K : p.N, cols_pad = p.b_nk ? plan.kp : plan.np;
+        st = launch_pad(o.B, o.ldb, base + plan.off_b, rows, cols, cols_pad, stream, info);
+        if (st != TG_OK) return st;
+        o.B = base + plan.off_b;
+        o.ldb = cols_pad;
+      }
+      st = launch_path(inner, o, stream, info);
+    } else {
+      st = launch_path(path, o, stream, info);
     }
-    return TG_OK;
+    if (st != TG_OK) return st;
   }
-  if (path == TG_PATH_REPACK) {
-    uint8_t* base = static_cast<uint8_t*>(ws);
-    if (plan.pad_a) {
-      st = launch_pad(A, base + plan.off_a, M, K, plan.kp, stream, info);
-      if (st != TG_OK) return st;
-      o.A = base + plan.off_a;
-      o.lda = plan.kp;
-    }
-    if (plan.pad_b) {
-      st = launch_pad(B, base + plan.off_b, K, N, plan.np, stream, info);
-      if (st != TG_OK) return st;
-      o.B = base + plan.off_b;
-      o.ldb = plan.np;
-    }
-    return launch_path(inner_path(M, N, K, o.c_aligned), o, stream, info);
-  }
-  return launch_path(path, o, stream, info);
+  return TG_OK;
+}
+
+// Options of tg_gemm_relu_f16_ex as a Problem (NULL options: dense defaults).
+bool problem_from_options(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                          const tg_gemm_options* opt, Problem& p, int& path) {
+  p = dense_problem(A, B, C, M, N, K);
+  path = TG_PATH_AUTO;
+  if (opt == nullptr) return true;
+  if (opt->b_layout != TG_B_KN && opt->b_layout != TG_B_NK) return false;
+  p.b_nk = opt->b_layout == TG_B_NK;
+  p.lda = opt->lda ? opt->lda : K;
+  p.ldb = opt->ldb ? opt->ldb : (p.b_nk ? K : N);
+  p.ldc = opt->ldc ? opt->ldc : N;
+  p.bias = opt->bias;
+  p.batch = opt->batch ? opt->batch : 1;
+  p.sa = opt->stride_a;
+  p.sb = opt->stride_b;
+  p.sc = opt->stride_c;
+  path = opt->path;
+  if (path == TG_PATH_REPACK) return false;  // chosen by the library when a workspace is given
+  return true;
 }
 
 }  // namespace
@@ -604,33 +722,58 @@ tg_status run(const void* A, const void* B, void* C, int64_t M, int64_t N, int64
 extern "C" {
 
 tg_status tg_gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream) {
-  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO, nullptr, 0);
+  return tg::run(tg::dense_problem(A, B, C, M, N, K), stream, TG_PATH_AUTO, nullptr, 0);
 }
 
 tg_status tg_gemm_relu_f16_path(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
                                 void* stream, int path) {
   if (path == TG_PATH_REPACK) return TG_ERR_INVALID_ARG;  // needs a workspace: tg_gemm_relu_f16_ws
-  return tg::run(A, B, C, M, N, K, stream, path, nullptr, 0);
+  return tg::run(tg::dense_problem(A, B, C, M, N, K), stream, path, nullptr, 0);
 }
 
 tg_status tg_gemm_relu_f16_ws(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream,
                               void* workspace, int64_t workspace_bytes) {
-  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO, workspace, workspace_bytes);
+  return tg::run(tg::dense_problem(A, B, C, M, N, K), stream, TG_PATH_AUTO, workspace, workspace_bytes);
+}
+
+tg_status tg_gemm_relu_f16_ex(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
+                              const tg_gemm_options* options, void* stream, void* workspace,
+                              int64_t workspace_bytes) {
+  tg::Problem p;
+  int path = TG_PATH_AUTO;
+  if (!tg::problem_from_options(A, B, C, M, N, K, options, p, path)) return TG_ERR_INVALID_ARG;
+  return tg::run(p, stream, path, workspace, workspace_bytes);
+}
+
+int64_t tg_workspace_size_ex(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K,
+                             const tg_gemm_options* options) {
+  tg::Problem p;
+  int path = TG_PATH_AUTO;
+  if (!tg::problem_from_options(A, B, const_cast<void*>(C), M, N, K, options, p, path) || !tg::problem_valid(p))
+    return -1;
+  return tg::workspace_bytes_needed(p);
+}
+
+int tg_select_path_ex(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K,
+                      const tg_gemm_options* options, int64_t workspace_bytes) {
+  tg::Problem p;
+  int path = TG_PATH_AUTO;
+  if (!tg::problem_from_options(A, B, const_cast<void*>(C), M, N, K, options, p, path)) return -2;
+  if (path != TG_PATH_AUTO) return tg::path_supports(path, p) ? path : -2;
+  return tg::select_path(p, workspace_bytes);
 }
 
 tg_status tg_gemm_relu_f16_static_ws(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K,
                                      void* stream) {
-  if (!tg::args_valid(A, B, C, M, N, K)) return TG_ERR_INVALID_ARG;
-  const int64_t need = tg_workspace_size(A, B, C, M, N, K);
+  const tg::Problem p = tg::dense_problem(A, B, C, M, N, K);
+  if (!tg::problem_valid(p)) return TG_ERR_INVALID_ARG;
+  const int64_t need = tg::workspace_bytes_needed(p);
   if (need > TG_STATIC_WORKSPACE_BYTES) return TG_ERR_TOO_LARGE;
+  if (M == 0 || N == 0) return TG_OK;  // empty C: nothing to do
   int dev = 0;
   tg::DeviceInfo* info = nullptr;
-  if (M > 0 && N > 0) {
-    const tg_status st = tg::current_device(dev, info);
-    if (st != TG_OK) return st;
-  } else {
-    return TG_OK;  // empty C: nothing to do
-  }
+  const tg_status st = tg::current_device(dev, info);
+  if (st != TG_OK) return st;
   void* ws = nullptr;
   {
     std::lock_guard<std::mutex> lock(tg::g_mutex);
@@ -644,26 +787,26 @@ tg_status tg_gemm_relu_f16_static_ws(const void* A, const void* B, void* C, int6
     }
     ws = info->static_ws;
   }
-  return tg::run(A, B, C, M, N, K, stream, TG_PATH_AUTO, ws, TG_STATIC_WORKSPACE_BYTES);
+  return tg::run(p, stream, TG_PATH_AUTO, ws, TG_STATIC_WORKSPACE_BYTES);
 }
 
 int64_t tg_workspace_size(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
-  if (!tg::args_valid(A, B, C, M, N, K)) return -1;
-  if (M == 0 || N == 0 || K == 0 || tg::tma_ok(A, B, N, K)) return 0;
-  return tg::repack_plan(A, B, M, N, K).bytes;
+  const tg::Problem p = tg::dense_problem(A, B, const_cast<void*>(C), M, N, K);
+  if (!tg::problem_valid(p)) return -1;
+  return tg::workspace_bytes_needed(p);
 }
 
 int tg_select_path_ws(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K,
                       int64_t workspace_bytes) {
-  return tg::select_path_ws(A, B, C, M, N, K, workspace_bytes);
+  return tg::select_path(tg::dense_problem(A, B, const_cast<void*>(C), M, N, K), workspace_bytes);
 }
 
 int tg_select_path(const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
-  return tg::select_path(A, B, C, M, N, K);
+  return tg::select_path(tg::dense_problem(A, B, const_cast<void*>(C), M, N, K), 0);
 }
 
 int tg_path_supports(int path, const void* A, const void* B, const void* C, int64_t M, int64_t N, int64_t K) {
-  return tg::path_supports(path, A, B, C, M, N, K) ? 1 : 0;
+  return tg::path_supports(path, tg::dense_problem(A, B, const_cast<void*>(C), M, N, K)) ? 1 : 0;
 }
 
 tg_status tg_device_status(uint32_t* detail) {
@@ -719,7 +862,6 @@ const char* tg_path_name(int path) {
     case TG_PATH_TC: return "tc";
     case TG_PATH_TC_EDGE: return "tc_edge";
     case TG_PATH_SKINNY: return "skinny";
-    case TG_PATH_GEMV: return "gemv";
     case TG_PATH_ZERO: return "zero";
     case TG_PATH_TC_PAIR: return "tc_pair";
     case TG_PATH_TC_PAIR512: return "tc_pair512";

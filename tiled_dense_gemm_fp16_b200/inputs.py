@@ -42,6 +42,18 @@ def operands(M: int, N: int, K: int, dist: str = "uniform", seed: int = 0,
     return A, B
 
 
+def linear_operands(M: int, N: int, K: int, seed: int = 5, dist: str = "uniform"):
+    """A linear layer's operands: x (M x K), the weight W stored N x K, and a bias of N values.
+
+    Drawn in that order from ``default_rng(seed)``.
+    """
+    rng = np.random.default_rng(seed)
+    x = draw(rng, (M, K), dist)
+    W = draw(rng, (N, K), dist)
+    b = draw(rng, (N,), dist)
+    return x, W, b
+
+
 @dataclass(frozen=True)
 class Workload:
     name: str
@@ -71,6 +83,9 @@ WORKLOADS = {
                        "uniform", 3, "decode-like small M, bandwidth-bound"),
     "ragged": Workload("ragged", ((3001, 5003, 1021), (777, 12289, 4095), (8191, 129, 8193)),
                        "uniform", 4, "non-tile-multiple shapes with unaligned row strides"),
+    # Beyond the five: a linear layer relu(x W^T + b) with the weight stored N x K.
+    "linear8192": Workload("linear8192", ((8192, 8192, 8192),), "uniform", 5,
+                           "x (M x K), weight stored N x K, fp16 bias; drawn by linear_operands"),
 }
 
 
