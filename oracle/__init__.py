@@ -74,8 +74,8 @@ def _bind(lib):
     lib.oracle_f32_to_f16_rne_array.restype = None
     lib.oracle_gemm_relu_f16.argtypes = [u16p, u16p, u16p, i64, i64, i64, ctypes.c_int]
     lib.oracle_gemm_relu_f16.restype = ctypes.c_int
-    lib.oracle_gemm_relu_f16_ex.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, i64, ctypes.c_int, u16p,
-                                            ctypes.c_int]
+    lib.oracle_gemm_relu_f16_ex.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, i64, ctypes.c_int,
+                                            ctypes.c_int, u16p, ctypes.c_int]
     lib.oracle_gemm_relu_f16_ex.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
@@ -140,12 +140,12 @@ def gemm_relu_f16(A: np.ndarray, B: np.ndarray, nthreads: int = 0, lib=None) -> 
 
 def gemm_relu_f16_ex(A: np.ndarray, B: np.ndarray, M: int, N: int, K: int, lda: int, ldb: int, ldc: int,
                      b_nk: bool = False, bias: np.ndarray | None = None, C: np.ndarray | None = None,
-                     nthreads: int = 0, lib=None) -> np.ndarray:
+                     nthreads: int = 0, lib=None, a_km: bool = False) -> np.ndarray:
     """General-layout form: A, B and C are flat fp16 buffers read/written with the given row strides.
 
-    B holds K x N (b_nk False) or N x K (b_nk True) with row stride ldb; ``bias`` is an fp16 vector of
-    N or None.  Returns C (a fresh zero buffer of M*ldc elements unless one is given; only the M x N
-    block is written).
+    A holds M x K (a_km False) or K x M (a_km True) with row stride lda; B holds K x N (b_nk False)
+    or N x K (b_nk True) with row stride ldb; ``bias`` is an fp16 vector of N or None.  Returns C (a
+    fresh zero buffer of M*ldc elements unless one is given; only the M x N block is written).
     """
     lib = lib or load_library()
     A = _u16(np.asarray(A).reshape(-1))
@@ -160,12 +160,13 @@ def gemm_relu_f16_ex(A: np.ndarray, B: np.ndarray, M: int, N: int, K: int, lda: 
         if bias.size < N:
             raise ValueError("bias must have N elements")
         bias_p = _ptr(bias, ctypes.c_uint16)
-    need_a = (M - 1) * lda + K if M > 0 and K > 0 else 0
+    need_a = ((K - 1) * lda + M if a_km else (M - 1) * lda + K) if M > 0 and K > 0 else 0
     need_b = ((K - 1) * ldb + N if not b_nk else (N - 1) * ldb + K) if K > 0 and N > 0 else 0
     if A.size < need_a or B.size < need_b or C.size < (M - 1) * ldc + N:
         raise ValueError("buffer too small for the given shape and strides")
     rc = lib.oracle_gemm_relu_f16_ex(_ptr(A, ctypes.c_uint16), _ptr(B, ctypes.c_uint16), _ptr(C, ctypes.c_uint16),
-                                     M, N, K, lda, ldb, ldc, 1 if b_nk else 0, bias_p, int(nthreads))
+                                     M, N, K, lda, ldb, ldc, 1 if a_km else 0, 1 if b_nk else 0, bias_p,
+                                     int(nthreads))
     if rc != 0:
         raise MemoryError("oracle could not allocate its work buffers")
     return C.view(np.float16)

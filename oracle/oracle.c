@@ -204,8 +204,10 @@ int oracle_gemm_relu_f16(const uint16_t *A, const uint16_t *B, uint16_t *C,
  *
  *   C[i*ldc + j] = f16_rne( relu( fp32( sum_k a(i,k) * b(k,j) ) + f32(bias[j]) ) )
  *
- * with a(i,k) = A[i*lda + k]; b(k,j) = B[k*ldb + j] when b_nk == 0 (B stored
- * K x N) and B[j*ldb + k] when b_nk == 1 (B stored N x K, so C = A . B^T);
+ * with a(i,k) = A[i*lda + k] when a_km == 0 (A stored M x K) and A[k*lda + i]
+ * when a_km == 1 (A stored K x M, so C = A^T . B); b(k,j) = B[k*ldb + j] when
+ * b_nk == 0 (B stored K x N) and B[j*ldb + k] when b_nk == 1 (B stored N x K,
+ * so C = A . B^T);
  * bias may be NULL (no bias term).  The sum runs in k order with an fp32
  * accumulator exactly as in oracle_gemm_relu_f16; the bias is added to the
  * finished sum with one fp32 addition, then ReLU, then the fp16 rounding.
@@ -213,8 +215,8 @@ int oracle_gemm_relu_f16(const uint16_t *A, const uint16_t *B, uint16_t *C,
  * Returns 0, or -1 if a work buffer cannot be allocated.
  */
 int oracle_gemm_relu_f16_ex(const uint16_t *A, const uint16_t *B, uint16_t *C, int64_t M, int64_t N,
-                            int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int b_nk, const uint16_t *bias,
-                            int nthreads)
+                            int64_t K, int64_t lda, int64_t ldb, int64_t ldc, int a_km, int b_nk,
+                            const uint16_t *bias, int nthreads)
 {
     if (M <= 0 || N <= 0)
         return 0;
@@ -253,7 +255,7 @@ int oracle_gemm_relu_f16_ex(const uint16_t *A, const uint16_t *B, uint16_t *C, i
             for (int64_t j = 0; j < N; ++j)
                 acc[j] = 0.0f;
             for (int64_t k = 0; k < K; ++k) {
-                const float a = oracle_f16_to_f32(A[i * lda + k]);
+                const float a = oracle_f16_to_f32(a_km ? A[k * lda + i] : A[i * lda + k]);
                 const float *brow = Bf + k * N;
                 for (int64_t j = 0; j < N; ++j)
                     acc[j] = acc[j] + a * brow[j];

@@ -302,6 +302,20 @@ def check_ex_weight_layout(lib):
         assert np.array_equal(_bits(ex), _bits(oracle.gemm_relu_f16(A, B, lib=lib))), (M, N, K)
 
 
+def check_ex_transposed_a(lib):
+    """A stored K x M (C = A^T . B) gives the base oracle's bits on the transposed copy, also with
+    B stored N x K."""
+    for (M, N, K) in [(29, 41, 67), (70, 9, 33)]:
+        A, B = inputs.operands(M, N, K, "uniform", seed=M * K)
+        At = np.ascontiguousarray(A.T)                       # K x M storage of the same A
+        want = _bits(oracle.gemm_relu_f16(A, B, lib=lib))
+        ex = oracle.gemm_relu_f16_ex(At, B, M, N, K, M, N, N, a_km=True, lib=lib).reshape(M, N)
+        assert np.array_equal(_bits(ex), want), (M, N, K)
+        Bt = np.ascontiguousarray(B.T)
+        ex2 = oracle.gemm_relu_f16_ex(At, Bt, M, N, K, M, K, N, a_km=True, b_nk=True, lib=lib).reshape(M, N)
+        assert np.array_equal(_bits(ex2), want), (M, N, K)
+
+
 def check_ex_strides(lib):
     """Row strides wider than the rows read the same values; C's padding is left alone."""
     M, N, K = 23, 31, 45
@@ -358,6 +372,7 @@ ALL_CHECKS = [
     check_rows_and_threads,
     check_ex_dense_equals_base,
     check_ex_weight_layout,
+    check_ex_transposed_a,
     check_ex_strides,
     check_ex_bias_exact,
     check_ex_bias_closed_form,

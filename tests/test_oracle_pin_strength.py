@@ -25,6 +25,7 @@ MUTANTS = [
     ("ex_bias_dropped", "bias ? acc[j] + oracle_f16_to_f32(bias[j]) : acc[j]", "acc[j]"),
     ("ex_bias_after_relu", "const float v = y > 0.0f ? y : 0.0f;",
      "const float v = (acc[j] > 0.0f ? acc[j] : 0.0f) + (bias ? oracle_f16_to_f32(bias[j]) : 0.0f);"),
+    ("ex_transposed_a_ignored", "a_km ? A[k * lda + i] : A[i * lda + k]", "A[i * lda + k]"),
     ("ex_ldc_ignored", "C[i * ldc + j] = oracle_f32_to_f16_rne(v);", "C[i * N + j] = oracle_f32_to_f16_rne(v);"),
     ("fp64_accumulator", "float *acc = (float *)malloc((size_t)N * sizeof(float));",
      "double *acc = (double *)malloc((size_t)N * sizeof(double));"),
