@@ -154,12 +154,14 @@ TG_API tg_status tg_gemm_relu_f16_static_ws(const void *A, const void *B, void *
  *
  * For each batch entry e = 0 .. batch-1:
  *
- *   C_e[i*ldc + j] = fp16( max( sum_k A_e[i*lda + k] * b_e(k, j) + bias[j], 0 ) )
+ *   C_e[i*ldc + j] = fp16( max( sum_k a_e(i, k) * b_e(k, j) + bias[j], 0 ) )
  *
  * with A_e = A + e*stride_a, B_e = B + e*stride_b, C_e = C + e*stride_c
- * (element offsets) and b_e(k, j) = B_e[k*ldb + j] when B is stored K x N
- * (TG_B_KN) or B_e[j*ldb + k] when it is stored N x K (TG_B_NK, the layout of
- * a linear layer's weight: C = A . W^T).  The sum is accumulated in fp32;
+ * (element offsets); a_e(i, k) = A_e[i*lda + k] when A is stored M x K
+ * (TG_A_MK) or A_e[k*lda + i] when it is stored K x M (TG_A_KM: C = A^T . B);
+ * b_e(k, j) = B_e[k*ldb + j] when B is stored K x N (TG_B_KN) or
+ * B_e[j*ldb + k] when it is stored N x K (TG_B_NK, the layout of a linear
+ * layer's weight: C = A . W^T).  The sum is accumulated in fp32;
  * the bias (fp16, N values, optional) is added to it in fp32 before ReLU.
  * This widens the quick-start kernel's dense row-major operands to the
  * layouts its T.gemm tile operator accepts ("TileLang" wiki page,
@@ -168,15 +170,19 @@ TG_API tg_status tg_gemm_relu_f16_static_ws(const void *A, const void *B, void *
  * A zero-initialised tg_gemm_options (or NULL) means: dense row-major A, B
  * (K x N) and C, no bias, one problem, automatic kernel choice.
  */
+enum { TG_A_MK = 0, TG_A_KM = 1 };
 enum { TG_B_KN = 0, TG_B_NK = 1 };
 
 typedef struct tg_gemm_options {
-    int64_t lda;        /* elements between rows of A; 0 = K; must be >= K        */
+    int64_t lda;        /* elements between rows of A as stored; 0 = K (TG_A_MK)
+                           or M (TG_A_KM); must be at least that                */
     int64_t ldb;        /* elements between rows of B as stored; 0 = N (TG_B_KN)
                            or K (TG_B_NK); must be at least that                */
     int64_t ldc;        /* elements between rows of C; 0 = N; must be >= N        */
+    int32_t a_layout;   /* TG_A_MK or TG_A_KM                                    */
     int32_t b_layout;   /* TG_B_KN or TG_B_NK                                    */
     int32_t path;       /* TG_PATH_AUTO (0) or a forced kernel path (testing)     */
+    int32_t reserved;   /* must be 0                                             */
     const void *bias;   /* device fp16[N], or NULL                                */
     int64_t batch;      /* number of problems; 0 = 1                             */
     int64_t stride_a;   /* elements between consecutive A, B and C entries;     */
@@ -189,8 +195,9 @@ typedef struct tg_gemm_options {
  * Operands TMA cannot describe (row or batch strides that are not multiples
  * of 8 elements, bases that are not 16-byte aligned) go through the repack
  * path when `workspace_bytes` >= tg_workspace_size_ex(...); without enough
- * workspace, B stored K x N uses the edge mode and B stored N x K is refused
- * (TG_ERR_INVALID_ARG).  Batch entries run in order on `stream` and share the
+ * workspace, A stored M x K with B stored K x N uses the edge mode and the
+ * other layouts are refused (TG_ERR_INVALID_ARG).  A stored K x M runs on the
+ * 128- and 256-row tensor-core kernels (not the small-M kernel).  Batch entries run in order on `stream` and share the
  * workspace.  Errors as tg_gemm_relu_f16_ws, plus TG_ERR_INVALID_ARG for
  * strides below the row lengths, overlapping C entries, an unknown b_layout
  * or a forced path that cannot run these operands.

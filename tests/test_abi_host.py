@@ -178,5 +178,20 @@ def test_extended_options_validation_and_paths():
     # A forced path must be able to run the operands.
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(path=Path.TC_EDGE, b_layout=tg.B_NK)) == Path.INVALID
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(path=Path.TC)) == Path.TC
+    # A stored K x M: the 128/256-row tensor-core kernels, never the small-M kernel or the edge mode.
+    t = tg.options(a_layout=tg.A_KM)
+    assert tg.select_path_ex(A0, B0, C0, 8192, 8192, 8192, t) == Path.TC_PAIR512
+    assert tg.select_path_ex(A0, B0, C0, 64, 8192, 8192, t) in (Path.TC, Path.TC_PAIR)
+    assert tg.select_path_ex(A0, B0, C0, 64, 8192, 8192, tg.options(a_layout=tg.A_KM, path=Path.SKINNY)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(a_layout=tg.A_KM, path=Path.TC_EDGE)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 300, 128, 64, tg.options(a_layout=tg.A_KM, lda=299)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 300, 128, 64, tg.options(a_layout=2)) == Path.INVALID
+    assert tg.select_path_ex(A0, B0, C0, 64, 128, 64, tg.options(reserved=1)) == Path.INVALID
+    # An M that is not a multiple of 8 leaves K x M rows unaligned: repack into K x roundup(M, 8).
+    assert tg.select_path_ex(A0, B0, C0, 300, 512, 512, t) == Path.REPACK     # the call then needs a workspace
+    assert tg.gemm_relu_f16_ex_raw(A0, B0, C0, 300, 512, 512, t) == Status.INVALID_ARG
+    assert tg.select_path_ex(A0, B0, C0, 304, 512, 512, t) in (Path.TC, Path.TC_PAIR)
+    assert tg.workspace_size_ex(A0, B0, C0, 301, 512, 512, t) == up(2 * 512 * 304)
+    assert tg.workspace_size_ex(A0, B0, C0, 304, 512, 512, t) == 0
     # A bias that overlaps C is refused.
     assert tg.gemm_relu_f16_ex_raw(A0, B0, C0, 64, 64, 64, tg.options(bias=C0 + 64)) == Status.INVALID_ARG

@@ -1,6 +1,6 @@
 """Parity of the general-layout entry point tg_gemm_relu_f16_ex with the oracle:
-row strides, B stored N x K (a linear layer's weight), a fused bias, strided
-batches, and the torch helpers built on it.  Integer-valued inputs (and
+row strides, A stored K x M (C = A^T . B), B stored N x K (a linear layer's
+weight), a fused bias, strided batches, and the torch helpers built on it.  Integer-valued inputs (and
 integer bias) are compared bit for bit; float inputs within the tolerance."""
 import numpy as np
 import pytest
@@ -22,17 +22,17 @@ def _flat(rng, rows, cols, ld, dist):
 
 
 def run_ex(M, N, K, *, lda, ldb, ldc, b_nk, bias, batch=1, gap=0, dist="int", seed=0, path=Path.AUTO,
-           workspace=True, offsets=(0, 0, 0)):
+           workspace=True, offsets=(0, 0, 0), a_km=False):
     """Draw operands, run tg_gemm_relu_f16_ex, and return (gpu C entries, oracle C entries, guards ok)."""
     import torch
     import tiled_dense_gemm_fp16_b200 as tg
     rng = np.random.default_rng(seed)
-    a_rows, a_cols = M, K
+    a_rows, a_cols = (K, M) if a_km else (M, K)
     b_rows, b_cols = (N, K) if b_nk else (K, N)
-    sa = M * lda + gap
+    sa = a_rows * lda + gap
     sb = b_rows * ldb + gap
     sc = (M - 1) * ldc + N + gap if M > 0 else gap
-    A_all = np.zeros(max(1, (batch - 1) * sa + M * lda), np.float16)
+    A_all = np.zeros(max(1, (batch - 1) * sa + a_rows * lda), np.float16)
     B_all = np.zeros(max(1, (batch - 1) * sb + b_rows * ldb), np.float16)
     entries = []
     for e in range(batch):
@@ -58,6 +58,7 @@ def run_ex(M, N, K, *, lda, ldb, ldc, b_nk, bias, batch=1, gap=0, dist="int", se
     Cd = cbuf[G + offsets[2]:]
     bias_d = torch.from_numpy(bias_h).to(dev) if bias_h is not None else None
     opts = tg.options(lda=lda, ldb=ldb, ldc=ldc, b_layout=tg.B_NK if b_nk else tg.B_KN,
+                      a_layout=tg.A_KM if a_km else tg.A_MK,
                       bias=bias_d.data_ptr() if bias_d is not None else 0, batch=batch,
                       stride_a=sa, stride_b=sb, stride_c=sc, path=path)
     need = tg.workspace_size_ex(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, opts)
@@ -76,7 +77,7 @@ def run_ex(M, N, K, *, lda, ldb, ldc, b_nk, bias, batch=1, gap=0, dist="int", se
     got, ref = [], []
     for (oa, ob, oc) in entries:
         want = oracle.gemm_relu_f16_ex(A_all[oa:], B_all[ob:], M, N, K, lda, ldb, ldc, b_nk=b_nk, bias=bias_h,
-                                       C=np.full(M * ldc, GUARD_BITS, np.uint16)).view(np.uint16)
+                                       C=np.full(M * ldc, GUARD_BITS, np.uint16), a_km=a_km).view(np.uint16)
         g = cflat[oc:oc + M * ldc]
         # Padding columns of C between rows are never written.
         pad = np.ones(M * ldc, bool)
@@ -160,6 +161,38 @@ def test_float_inputs_with_bias():
                               seed=19)
     assert guards
     assert_close(got[0], ref[0], "float B_NK + bias")
+
+
+@pytest.mark.parametrize("b_nk", [False, True], ids=["B_KN", "B_NK"])
+@pytest.mark.parametrize("path", [Path.AUTO, Path.TC, Path.TC_PAIR, Path.TC_PAIR512],
+                         ids=["auto", "tc", "pair", "pair512"])
+@pytest.mark.parametrize("M,N,K", [(520, 1032, 264), (64, 520, 72), (301, 777, 333)])
+def test_transposed_a(M, N, K, path, b_nk):
+    """A stored K x M (C = A^T . B) with every tensor-core kernel; ragged M goes through the repack path."""
+    if path != Path.AUTO and M % 8:
+        pytest.skip("a K x M A with M not a multiple of 8 needs the repack path")
+    got, ref, guards = run_ex(M, N, K, lda=M, ldb=K if b_nk else N, ldc=N, b_nk=b_nk, bias=True, path=path,
+                              a_km=True, seed=M + int(path) + 3 * int(b_nk))
+    assert guards
+    assert_bitexact(got[0], ref[0], f"A_KM {(M, N, K)} path {path} b_nk={b_nk}")
+
+
+@pytest.mark.parametrize("strides", ["padded8", "odd"])
+def test_transposed_a_strides_and_batches(strides):
+    M, N, K = 200, 264, 136
+    lda, ldb, ldc = (M + 8, N + 16, N + 24) if strides == "padded8" else (M + 3, N + 1, N + 5)
+    got, ref, guards = run_ex(M, N, K, lda=lda, ldb=ldb, ldc=ldc, b_nk=False, bias=True, batch=2, gap=24,
+                              a_km=True, seed=31)
+    assert guards
+    for e in range(2):
+        assert_bitexact(got[e], ref[e], f"A_KM {strides} entry {e}")
+
+
+def test_transposed_a_float_full_tiles():
+    got, ref, guards = run_ex(1024, 1024, 1024, lda=1024, ldb=1024, ldc=1024, b_nk=False, bias=False,
+                              dist="uniform", a_km=True, seed=41)
+    assert guards
+    assert_close(got[0], ref[0], "A_KM float 1024")
 
 
 def test_torch_helpers():

@@ -6,6 +6,8 @@ This package only marshals arguments to it; the library is loaded on first
 use and every call raises if it is missing.
 """
 from ._binding import (  # noqa: F401
+    A_KM,
+    A_MK,
     B_KN,
     B_NK,
     EXPORTS,

@@ -45,6 +45,7 @@ class TGError(RuntimeError):
         super().__init__(f"{what}: {status_string(status)} ({int(status)})" if what else status_string(status))
 
 
+A_MK, A_KM = 0, 1
 B_KN, B_NK = 0, 1
 
 
@@ -54,8 +55,10 @@ class GemmOptions(ctypes.Structure):
         ("lda", ctypes.c_int64),
         ("ldb", ctypes.c_int64),
         ("ldc", ctypes.c_int64),
+        ("a_layout", ctypes.c_int32),
         ("b_layout", ctypes.c_int32),
         ("path", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
         ("bias", ctypes.c_void_p),
         ("batch", ctypes.c_int64),
         ("stride_a", ctypes.c_int64),
@@ -185,9 +188,10 @@ def workspace_size(A: int, B: int, C: int, M: int, N: int, K: int) -> int:
 
 
 def options(lda=0, ldb=0, ldc=0, b_layout=B_KN, bias=0, batch=0, stride_a=0, stride_b=0, stride_c=0,
-            path=Path.AUTO) -> GemmOptions:
+            path=Path.AUTO, a_layout=A_MK, reserved=0) -> GemmOptions:
     """A tg_gemm_options value (zeros mean the dense defaults)."""
-    return GemmOptions(lda, ldb, ldc, int(b_layout), int(path), bias or None, batch, stride_a, stride_b, stride_c)
+    return GemmOptions(lda, ldb, ldc, int(a_layout), int(b_layout), int(path), int(reserved), bias or None, batch,
+                       stride_a, stride_b, stride_c)
 
 
 def gemm_relu_f16_ex_raw(A: int, B: int, C: int, M: int, N: int, K: int, opts: GemmOptions | None = None,

@@ -40,6 +40,7 @@ struct TcParams {
   const __half* bias;    // optional fp16[N], added to every row before ReLU; nullptr = none
   int64_t lda, ldb, ldc; // row strides (elements) of A, of B as stored, and of C
   int b_kmajor;          // 1: B is stored N x K (rows of length K; C = A . B^T)
+  int a_mnmajor;         // 1: A is stored K x M (rows of length M; C = A^T . B)
   int M, N, K;
   int m_tiles, n_tiles, num_tiles, k_blocks;
   int group_m;           // tile rows per raster group
@@ -304,7 +305,13 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
             }
             mbar_arrive_expect_tx(&full_bar[stage], Cfg::A_BYTES + Cfg::B_BYTES);
             const int k0 = kb * Cfg::BK;
-            tma_load_2d(a_smem + stage * Cfg::A_BYTES, &tmap_a, &full_bar[stage], k0, m0);
+            if (p.a_mnmajor) {
+              // A stored K x M: two 64-row (m) x 64 k boxes, MN-major like B.
+              tma_load_2d(a_smem + stage * Cfg::A_BYTES, &tmap_a, &full_bar[stage], m0, k0);
+              tma_load_2d(a_smem + stage * Cfg::A_BYTES + Cfg::B_CHUNK_BYTES, &tmap_a, &full_bar[stage], m0 + 64, k0);
+            } else {
+              tma_load_2d(a_smem + stage * Cfg::A_BYTES, &tmap_a, &full_bar[stage], k0, m0);
+            }
             uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
             if (p.b_kmajor) {
               // B stored N x K: one box of BN rows (n) x 64 k, K-major like A.
@@ -425,7 +432,7 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      const uint32_t idesc = make_idesc_f16_f32(Cfg::BM, Cfg::BN, false, p.b_kmajor == 0);
+      const uint32_t idesc = make_idesc_f16_f32(Cfg::BM, Cfg::BN, p.a_mnmajor != 0, p.b_kmajor == 0);
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -442,8 +449,10 @@ __global__ void __launch_bounds__(TcCfg<EDGE>::THREADS, 1)
           const uint32_t b_addr = smem_u32(b_smem + stage * Cfg::B_BYTES);
 #pragma unroll
           for (int k = 0; k < Cfg::BK / 16; ++k) {
-            // A: advance 16 elements (32 bytes) inside the swizzled row.
-            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+            // A as M x K: advance 16 elements (32 bytes) inside the swizzled
+            // row.  A as K x M: MN-major, two 64-row panels 8 KiB apart.
+            const uint64_t adesc = p.a_mnmajor ? make_sw128_desc(a_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024)
+                                               : make_sw128_desc(a_addr + k * 32, 16, 1024);
             // B as K x N: advance 16 k-rows (2048 bytes); 64-column panels 8 KiB
             // apart.  B as N x K: K-major like A.
             const uint64_t bdesc = p.b_kmajor ? make_sw128_desc(b_addr + k * 32, 16, 1024)

@@ -148,7 +148,14 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
           const int k0 = kb * Cfg::BK;
           uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
-          tma_load_2d_pair_hint(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, k0, m0, pol_a);
+          if (p.a_mnmajor) {
+            // A stored K x M: this CTA's 128 m-rows as two 64 m x 64 k boxes.
+            tma_load_2d_pair_hint(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, m0, k0, pol_a);
+            tma_load_2d_pair_hint(a_smem + stage * Cfg::A_BYTES + Cfg::B_CHUNK_BYTES, &tmap_a, full_even, m0 + 64,
+                                  k0, pol_a);
+          } else {
+            tma_load_2d_pair_hint(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, k0, m0, pol_a);
+          }
 #pragma unroll
           for (int j = 0; j < Cfg::SLABS; ++j) {
             if (p.b_kmajor) {
@@ -164,7 +171,12 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
             // Warm L2 with the boxes a few k-blocks ahead, so the ring's
             // loads find them there instead of waiting on HBM.
             const int kp = (kb + p.prefetch_kb) * Cfg::BK;
-            tma_prefetch_l2_2d(&tmap_a, kp, m0);
+            if (p.a_mnmajor) {
+              tma_prefetch_l2_2d(&tmap_a, m0, kp);
+              tma_prefetch_l2_2d(&tmap_a, m0 + 64, kp);
+            } else {
+              tma_prefetch_l2_2d(&tmap_a, kp, m0);
+            }
 #pragma unroll
             for (int j = 0; j < Cfg::SLABS; ++j) {
               if (p.b_kmajor) {
@@ -203,7 +215,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      const uint32_t idesc = make_idesc_f16_f32(Cfg::PAIR_M, 256, false, p.b_kmajor == 0);
+      const uint32_t idesc = make_idesc_f16_f32(Cfg::PAIR_M, 256, p.a_mnmajor != 0, p.b_kmajor == 0);
       for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters, ++local) {
         const int acc = local % Cfg::NUM_ACC;
         const uint32_t acc_phase = (local / Cfg::NUM_ACC) & 1;
@@ -220,7 +232,8 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           const uint32_t b_addr = smem_u32(b_smem + stage * Cfg::B_BYTES);
 #pragma unroll
           for (int k = 0; k < Cfg::BK / 16; ++k) {
-            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+            const uint64_t adesc = p.a_mnmajor ? make_sw128_desc(a_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024)
+                                               : make_sw128_desc(a_addr + k * 32, 16, 1024);
 #pragma unroll
             for (int j = 0; j < Cfg::SLABS; ++j) {
               // Slab j: as K x N, this CTA's two 64-column panels, 8 KiB apart;

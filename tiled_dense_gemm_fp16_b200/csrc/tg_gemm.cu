@@ -73,19 +73,21 @@ struct Problem {
   void* C;
   int64_t M, N, K;
   int64_t lda, ldb, ldc;
-  bool b_nk;
+  bool a_km;  // A stored K x M (C = A^T . B)
+  bool b_nk;  // B stored N x K (C = A . B^T)
   const void* bias;
   int64_t batch, sa, sb, sc;
 };
 
 Problem dense_problem(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K) {
-  return Problem{A, B, C, M, N, K, K, N, N, false, nullptr, 1, 0, 0, 0};
+  return Problem{A, B, C, M, N, K, K, N, N, false, false, nullptr, 1, 0, 0, 0};
 }
 
 // One GEMM as the kernels see it (one batch entry, possibly repacked).
 struct Operands {
   const void* A;
   int64_t lda;
+  bool a_km;
   const void* B;
   int64_t ldb;
   bool b_nk;
@@ -109,7 +111,9 @@ bool ranges_overlap(const void* a, int64_t a_bytes, const void* b, int64_t b_byt
 
 // Bytes each operand spans over all batch entries.
 int64_t span_a(const Problem& p) {
-  return (p.M > 0 && p.K > 0) ? 2 * ((p.batch - 1) * p.sa + (p.M - 1) * p.lda + p.K) : 0;
+  if (p.M <= 0 || p.K <= 0) return 0;
+  const int64_t one = p.a_km ? (p.K - 1) * p.lda + p.M : (p.M - 1) * p.lda + p.K;
+  return 2 * ((p.batch - 1) * p.sa + one);
 }
 int64_t span_b(const Problem& p) {
   if (p.K <= 0 || p.N <= 0) return 0;
@@ -124,7 +128,7 @@ bool problem_valid(const Problem& p) {
   if (p.M > INT_MAX || p.N > INT_MAX || p.K > INT_MAX) return false;
   if (p.batch < 1 || p.batch > INT_MAX) return false;
   if (p.M == 0 || p.N == 0) return true;
-  if (p.lda < (p.K > 0 ? p.K : 0) || p.ldc < p.N) return false;
+  if (p.lda < (p.a_km ? p.M : (p.K > 0 ? p.K : 0)) || p.ldc < p.N) return false;
   if (p.ldb < (p.b_nk ? p.K : p.N)) return false;
   if (p.lda > kMaxStride || p.ldb > kMaxStride || p.ldc > kMaxStride) return false;
   if (p.sa < 0 || p.sb < 0 || p.sc < 0 || p.sa > kMaxStride || p.sb > kMaxStride || p.sc > kMaxStride)
@@ -165,7 +169,7 @@ bool c_rows_aligned(const Problem& p) {
 // each 256-byte aligned; batch entries reuse it in stream order.
 struct RepackPlan {
   bool pad_a = false, pad_b = false;
-  int64_t kp = 0, np = 0;
+  int64_t kp = 0, np = 0, mp = 0;
   int64_t off_a = 0, off_b = 0, bytes = 0;
 };
 
@@ -173,10 +177,11 @@ RepackPlan repack_plan(const Problem& p) {
   RepackPlan r;
   r.kp = (p.K + 7) / 8 * 8;
   r.np = (p.N + 7) / 8 * 8;
+  r.mp = (p.M + 7) / 8 * 8;
   r.pad_a = !tma_ok_a(p);
   r.pad_b = !tma_ok_b(p);
   auto up256 = [](int64_t x) { return (x + 255) / 256 * 256; };
-  const int64_t bytes_a = r.pad_a ? up256(2 * p.M * r.kp) : 0;
+  const int64_t bytes_a = r.pad_a ? up256(p.a_km ? 2 * p.K * r.mp : 2 * p.M * r.kp) : 0;
   const int64_t bytes_b = r.pad_b ? up256(p.b_nk ? 2 * p.N * r.kp : 2 * p.K * r.np) : 0;
   r.off_a = 0;
   r.off_b = bytes_a;
@@ -197,13 +202,13 @@ bool path_supports(int path, const Problem& p) {
     case TG_PATH_AUTO:
       return true;
     case TG_PATH_TC_EDGE:
-      return !p.b_nk;  // the realigning producer reads B stored K x N
+      return !p.b_nk && !p.a_km;  // the realigning producer reads A stored M x K, B stored K x N
     case TG_PATH_TC:
     case TG_PATH_TC_PAIR:
     case TG_PATH_TC_PAIR512:
       return tma_ok(p);
     case TG_PATH_SKINNY:
-      return tma_ok(p) && p.M <= kSkinnyMaxM;
+      return tma_ok(p) && p.M <= kSkinnyMaxM && !p.a_km;
     case TG_PATH_REPACK:
       return !tma_ok(p);
     default:
@@ -234,7 +239,7 @@ int pick_tc_kernel(int64_t M, int64_t N, int64_t K, bool c_aligned) {
 
 // The tensor-core kernel that runs on TMA-describable (possibly repacked) operands.
 int inner_path(const Problem& p) {
-  return p.M <= kSkinnyMaxM ? TG_PATH_SKINNY : pick_tc_kernel(p.M, p.N, p.K, c_rows_aligned(p));
+  return (p.M <= kSkinnyMaxM && !p.a_km) ? TG_PATH_SKINNY : pick_tc_kernel(p.M, p.N, p.K, c_rows_aligned(p));
 }
 
 // The path a call takes with `ws_bytes` of workspace (-2: invalid arguments).
@@ -246,7 +251,7 @@ int select_path(const Problem& p, int64_t ws_bytes) {
   if (p.M == 0 || p.N == 0) return TG_PATH_NONE;
   if (p.K == 0) return TG_PATH_ZERO;
   if (!tma_ok(p)) {
-    if (ws_bytes >= repack_plan(p).bytes || p.b_nk) return TG_PATH_REPACK;
+    if (ws_bytes >= repack_plan(p).bytes || p.b_nk || p.a_km) return TG_PATH_REPACK;
     return TG_PATH_TC_EDGE;
   }
   return inner_path(p);
@@ -310,10 +315,15 @@ bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, i
   return r == CUDA_SUCCESS;
 }
 
-// Tensor maps of one GEMM's A (box 64 k x a_rows) and B: stored K x N, boxes
-// of 64 n x 64 k; stored N x K, boxes of 64 k x b_rows.
+// Tensor maps of one GEMM's A (stored M x K: boxes of 64 k x a_rows; stored
+// K x M: boxes of 64 m x 64 k) and B (stored K x N: boxes of 64 n x 64 k;
+// stored N x K: boxes of 64 k x b_rows).
 bool encode_operands(const Operands& o, CUtensorMap* ta, CUtensorMap* tb, int a_rows, int b_rows) {
-  if (!encode_2d(ta, o.A, o.M, o.K, o.lda, 64, a_rows)) return false;
+  if (o.a_km) {
+    if (!encode_2d(ta, o.A, o.K, o.M, o.lda, 64, 64)) return false;
+  } else if (!encode_2d(ta, o.A, o.M, o.K, o.lda, 64, a_rows)) {
+    return false;
+  }
   if (o.b_nk) return encode_2d(tb, o.B, o.N, o.K, o.ldb, 64, b_rows);
   return encode_2d(tb, o.B, o.K, o.N, o.ldb, 64, 64);
 }
@@ -328,6 +338,7 @@ void fill_tc_params(TcParams& p, const Operands& o) {
   p.ldb = o.ldb;
   p.ldc = o.ldc;
   p.b_kmajor = o.b_nk ? 1 : 0;
+  p.a_mnmajor = o.a_km ? 1 : 0;
   p.M = static_cast<int>(o.M);
   p.N = static_cast<int>(o.N);
   p.K = static_cast<int>(o.K);
@@ -659,6 +670,7 @@ tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws
   for (int64_t e = 0; e < p.batch; ++e) {
     Operands o{static_cast<const uint8_t*>(p.A) + 2 * e * p.sa,
                p.lda,
+               p.a_km,
                static_cast<const uint8_t*>(p.B) + 2 * e * p.sb,
                p.ldb,
                p.b_nk,
@@ -674,10 +686,11 @@ tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws
     } else if (path == TG_PATH_REPACK) {
       uint8_t* base = static_cast<uint8_t*>(ws);
       if (plan.pad_a) {
-        st = launch_pad(o.A, o.lda, base + plan.off_a, p.M, p.K, plan.kp, stream, info);
+        const int64_t rows = p.a_km ? p.K : p.M, cols = p.a_km ? p.M : p.K, cols_pad = p.a_km ? plan.mp : plan.kp;
+        st = launch_pad(o.A, o.lda, base + plan.off_a, rows, cols, cols_pad, stream, info);
         if (st != TG_OK) return st;
         o.A = base + plan.off_a;
-        o.lda = plan.kp;
+        o.lda = cols_pad;
       }
       if (plan.pad_b) {
         const int64_t rows = p.b_nk ? p.N : p.K, cols = p.b_nk ? p.K : p.N, cols_pad = p.b_nk ? plan.kp : plan.np;
@@ -702,8 +715,11 @@ bool problem_from_options(const void* A, const void* B, void* C, int64_t M, int6
   path = TG_PATH_AUTO;
   if (opt == nullptr) return true;
   if (opt->b_layout != TG_B_KN && opt->b_layout != TG_B_NK) return false;
+  if (opt->a_layout != TG_A_MK && opt->a_layout != TG_A_KM) return false;
+  if (opt->reserved != 0) return false;
   p.b_nk = opt->b_layout == TG_B_NK;
-  p.lda = opt->lda ? opt->lda : K;
+  p.a_km = opt->a_layout == TG_A_KM;
+  p.lda = opt->lda ? opt->lda : (p.a_km ? M : K);
   p.ldb = opt->ldb ? opt->ldb : (p.b_nk ? K : N);
   p.ldc = opt->ldc ? opt->ldc : N;
   p.bias = opt->bias;
