@@ -77,6 +77,17 @@ def _bind(lib):
     lib.oracle_gemm_relu_f16_ex.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, i64, ctypes.c_int,
                                             ctypes.c_int, u16p, ctypes.c_int]
     lib.oracle_gemm_relu_f16_ex.restype = ctypes.c_int
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    lib.oracle_fp8_to_f64.argtypes = [ctypes.c_uint8, ctypes.c_int]
+    lib.oracle_fp8_to_f64.restype = ctypes.c_double
+    lib.oracle_ue8m0_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_ue8m0_to_f64.restype = ctypes.c_double
+    lib.oracle_f64_to_bf16_rne.argtypes = [ctypes.c_double]
+    lib.oracle_f64_to_bf16_rne.restype = ctypes.c_uint16
+    lib.oracle_gemm_mxf8_grouped.argtypes = [u8p, u8p, u8p, u8p, u16p, i64p, i64p, ctypes.c_int, i64, i64,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    lib.oracle_gemm_mxf8_grouped.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -176,6 +187,58 @@ def gemm_relu_f16_rows(A: np.ndarray, B: np.ndarray, rows, nthreads: int = 0, li
     """Rows ``rows`` of the oracle result: the same definition applied to A[rows, :]."""
     rows = np.asarray(rows, dtype=np.int64)
     return gemm_relu_f16(np.ascontiguousarray(A[rows, :]), B, nthreads=nthreads, lib=lib)
+
+
+E4M3, E5M2 = 0, 1
+
+
+def fp8_to_f64(codes, fmt: int, lib=None) -> np.ndarray:
+    """Values of FP8 codes (format E4M3 = 0 or E5M2 = 1)."""
+    lib = lib or load_library()
+    codes = np.asarray(codes, dtype=np.uint8).reshape(-1)
+    return np.array([lib.oracle_fp8_to_f64(int(c), fmt) for c in codes], dtype=np.float64)
+
+
+def ue8m0_to_f64(codes, lib=None) -> np.ndarray:
+    lib = lib or load_library()
+    codes = np.asarray(codes, dtype=np.uint8).reshape(-1)
+    return np.array([lib.oracle_ue8m0_to_f64(int(c)) for c in codes], dtype=np.float64)
+
+
+def f64_to_bf16_bits(x, lib=None) -> np.ndarray:
+    lib = lib or load_library()
+    x = np.asarray(x, dtype=np.float64).reshape(-1)
+    return np.array([lib.oracle_f64_to_bf16_rne(float(v)) for v in x], dtype=np.uint16)
+
+
+def gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, row_offsets, N: int, K: int, a_format: int = E4M3,
+                      b_format: int = E4M3, relu: bool = False, C=None, nthreads: int = 0, lib=None) -> np.ndarray:
+    """Grouped MXFP8 GEMM: A (rows x K codes), SFA (rows x K/32 UE8M0), B (G x N x K codes),
+    SFB (G x N x K/32); group g covers rows row_offsets[g] .. + m_sizes[g].  Returns bf16 bit patterns
+    (rows x N, uint16); rows outside every group keep C's initial contents (zero by default)."""
+    lib = lib or load_library()
+    A = np.ascontiguousarray(np.asarray(A, dtype=np.uint8))
+    SFA = np.ascontiguousarray(np.asarray(SFA, dtype=np.uint8))
+    B = np.ascontiguousarray(np.asarray(B, dtype=np.uint8))
+    SFB = np.ascontiguousarray(np.asarray(SFB, dtype=np.uint8))
+    m_sizes = np.ascontiguousarray(np.asarray(m_sizes, dtype=np.int64))
+    row_offsets = np.ascontiguousarray(np.asarray(row_offsets, dtype=np.int64))
+    G = int(m_sizes.size)
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    rows = A.size // K if K else 0
+    if row_offsets.size != G or (G and int((row_offsets + m_sizes).max()) > rows):
+        raise ValueError("groups do not fit in A")
+    if B.size < G * N * K or SFB.size < G * N * (K // 32) or SFA.size < rows * (K // 32):
+        raise ValueError("operand too small")
+    C = np.zeros(rows * N, np.uint16) if C is None else np.ascontiguousarray(np.asarray(C, np.uint16)).reshape(-1).copy()
+    rc = lib.oracle_gemm_mxf8_grouped(_ptr(A, ctypes.c_uint8), _ptr(SFA, ctypes.c_uint8), _ptr(B, ctypes.c_uint8),
+                                      _ptr(SFB, ctypes.c_uint8), _ptr(C, ctypes.c_uint16), _ptr(row_offsets, ctypes.c_int64),
+                                      _ptr(m_sizes, ctypes.c_int64), G, N, K, int(a_format), int(b_format),
+                                      1 if relu else 0, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return C.reshape(rows, N) if N else C
 
 
 def max_threads(lib=None) -> int:

@@ -272,6 +272,141 @@ int oracle_gemm_relu_f16_ex(const uint16_t *A, const uint16_t *B, uint16_t *C, i
     return failed ? -1 : 0;
 }
 
+/* ------------------------------------------------------------------------
+ * MXFP8 block-scaled grouped GEMM (the "Blackwell MXFP8 grouped GEMM with
+ * block scaling + transposed B matrix" milestone, page 3, "Key Technical
+ * Milestones").  The page names the operation only; its number formats are
+ * the OCP Microscaling (MX) v1.0 definitions, which is the reading taken:
+ *   - elements are FP8 E4M3 ("fn": no infinities, S.1111.111 is NaN, bias 7)
+ *     or FP8 E5M2 (IEEE-style, bias 15, exponent 31 is inf/NaN);
+ *   - every 32 consecutive elements along K share one UE8M0 scale, the
+ *     power of two 2^(e - 127), with e = 255 meaning NaN;
+ *   - a scaled element is value(code) * scale, so one output is
+ *       sum over k of (a[i,k] * sa[i, k/32]) * (b[j,k] * sb[j, k/32]).
+ * B is "transposed": each group's weight is stored N x K (rows of length K).
+ * Readings where the page is silent: the sum is formed in double precision
+ * (every product of two scaled fp8 values is exact in double; the only
+ * rounding is in the adds, far below the output's precision); an optional
+ * ReLU maps every value not > 0 to +0; the result is rounded once to
+ * bfloat16, round to nearest, ties to even, overflow to +inf.
+ * ------------------------------------------------------------------------ */
+
+/* FP8 code -> value.  format 0: E4M3 (fn), format 1: E5M2. */
+double oracle_fp8_to_f64(uint8_t code, int format)
+{
+    const int sign = code >> 7;
+    double mag;
+    if (format == 0) {
+        const int e = (code >> 3) & 0xf, m = code & 0x7;
+        if (e == 15 && m == 7)
+            return NAN;
+        mag = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10); /* (1 + m/8) 2^(e-7) */
+    } else {
+        const int e = (code >> 2) & 0x1f, m = code & 0x3;
+        if (e == 31)
+            return m ? NAN : (sign ? -INFINITY : INFINITY);
+        mag = e == 0 ? ldexp((double)m, -16) : ldexp((double)(4 + m), e - 17); /* (1 + m/4) 2^(e-15) */
+    }
+    return sign ? -mag : mag;
+}
+
+/* UE8M0 scale code -> 2^(e - 127); 255 is NaN. */
+double oracle_ue8m0_to_f64(uint8_t e)
+{
+    return e == 255 ? NAN : ldexp(1.0, (int)e - 127);
+}
+
+/*
+ * double -> bfloat16 bits, round to nearest, ties to even (one rounding).
+ * bfloat16 has 8 significant bits and fp32's exponent range: for |x| in
+ * [2^e, 2^(e+1)), e >= -126, the quantum is 2^(e-7); below 2^-126 it is
+ * 2^-133.  A value that rounds to 2^128 or above becomes inf.
+ */
+uint16_t oracle_f64_to_bf16_rne(double x)
+{
+    if (isnan(x))
+        return 0x7fc0u;
+    const uint16_t sign = signbit(x) ? 0x8000u : 0;
+    const double a = fabs(x);
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7f80u);
+    if (a == 0.0)
+        return sign;
+    int e2;
+    (void)frexp(a, &e2);
+    int e = e2 - 1; /* a in [2^e, 2^(e+1)) */
+    const int subnormal = e < -126;
+    const int qexp = subnormal ? -133 : e - 7;
+    const double q = ldexp(a, -qexp); /* exact: a scaling by a power of two */
+    double qi = floor(q);
+    const double r = q - qi;
+    if (r > 0.5 || (r == 0.5 && fmod(qi, 2.0) != 0.0))
+        qi += 1.0;
+    long qn = (long)qi;
+    if (subnormal) {
+        if (qn == 128) /* rounds up to the smallest normal, 2^-126 */
+            return (uint16_t)(sign | (1u << 7));
+        return (uint16_t)(sign | (uint16_t)qn);
+    }
+    if (qn == 256) {
+        qn = 128;
+        e += 1;
+    }
+    if (e > 127)
+        return (uint16_t)(sign | 0x7f80u);
+    return (uint16_t)(sign | (uint16_t)((e + 127) << 7) | (uint16_t)(qn - 128));
+}
+
+/*
+ * Grouped, block-scaled GEMM over G groups that share N and K:
+ *
+ *   C[r*N + j] = bf16_rne( [relu]( sum_{k<K} a(r,k) sa(r,k/32) * b_g(j,k) sb_g(j,k/32) ) )
+ *
+ * for the rows r = row_offset[g] .. row_offset[g] + m_sizes[g] - 1 of group g:
+ *   a(r,k)   = fp8(A[r*K + k], a_format)            A: stacked rows x K codes
+ *   sa(r,s)  = ue8m0(SFA[r*(K/32) + s])             plain row-major scales
+ *   b_g(j,k) = fp8(B[(g*N + j)*K + k], b_format)    B: G x N x K codes
+ *   sb_g(j,s)= ue8m0(SFB[(g*N + j)*(K/32) + s])
+ * K must be a multiple of 32.  Rows of C outside every group are not
+ * written.  The sum for one output is taken in k order in double.  Returns
+ * 0, or -1 on bad arguments.
+ */
+int oracle_gemm_mxf8_grouped(const uint8_t *A, const uint8_t *SFA, const uint8_t *B, const uint8_t *SFB,
+                             uint16_t *C, const int64_t *row_offset, const int64_t *m_sizes, int G, int64_t N,
+                             int64_t K, int a_format, int b_format, int relu, int nthreads)
+{
+    if (K % 32 != 0 || N < 0 || G < 0)
+        return -1;
+    const int64_t S = K / 32;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#else
+    (void)nthreads;
+#endif
+    for (int g = 0; g < G; ++g) {
+        const int64_t r0 = row_offset[g], mg = m_sizes[g];
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+        for (int64_t i = 0; i < mg; ++i) {
+            const int64_t r = r0 + i;
+            for (int64_t j = 0; j < N; ++j) {
+                const int64_t brow = (int64_t)g * N + j;
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    const double av = oracle_fp8_to_f64(A[r * K + k], a_format) * oracle_ue8m0_to_f64(SFA[r * S + k / 32]);
+                    const double bv = oracle_fp8_to_f64(B[brow * K + k], b_format) * oracle_ue8m0_to_f64(SFB[brow * S + k / 32]);
+                    acc += av * bv;
+                }
+                const double y = relu ? (acc > 0.0 ? acc : 0.0) : acc;
+                C[r * N + j] = oracle_f64_to_bf16_rne(y);
+            }
+        }
+    }
+    return 0;
+}
+
 /* Number of threads OpenMP would use by default (1 without OpenMP). */
 int oracle_max_threads(void)
 {

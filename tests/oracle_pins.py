@@ -10,7 +10,12 @@ AssertionError when the oracle disagrees with:
     summation,
   * closed forms (identity, all-ones, zero operands, overflow),
   * the hand-worked examples of the matmul_relu quick-start kernel
-    ("TileLang" wiki page, "Programming model").
+    ("TileLang" wiki page, "Programming model"),
+  * for the MXFP8 grouped GEMM: torch's own float8_e4m3fn / float8_e5m2 /
+    float8_e8m0fnu decoders and float32 -> bfloat16 rounding (independent
+    implementations), hand-derived bfloat16 edge values, exact rational
+    sums rounded to bfloat16 by search over all bfloat16 values, and
+    closed forms (identity A, scale invariance, group separation).
 """
 from __future__ import annotations
 
@@ -355,6 +360,225 @@ def check_ex_bias_closed_form(lib):
     assert np.array_equal(_bits(got), np.tile(_bits(want), (M, 1)))
 
 
+# --------------------------------------------------------------------------
+# MXFP8 grouped GEMM
+# --------------------------------------------------------------------------
+
+def _torch_fp8(codes, fmt):
+    import torch
+    t = torch.from_numpy(np.asarray(codes, np.uint8).copy())
+    return t.view(torch.float8_e4m3fn if fmt == 0 else torch.float8_e5m2).to(torch.float64).numpy()
+
+
+def _same_values(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    num = ~np.isnan(b)
+    return bool(np.array_equal(np.isnan(a), np.isnan(b)) and np.array_equal(a[num], b[num])
+                and np.array_equal(np.signbit(a[num]), np.signbit(b[num])))
+
+
+def check_fp8_decode_all_codes(lib):
+    """All 256 codes of E4M3 and E5M2 against torch's float8 dtypes (values, NaNs and signs of zero)."""
+    codes = np.arange(256, dtype=np.uint8)
+    for fmt in (0, 1):
+        assert _same_values(oracle.fp8_to_f64(codes, fmt, lib=lib), _torch_fp8(codes, fmt)), fmt
+    # Facts of the formats: E4M3 max 448 and no infinities; E5M2 max 57344 and +-inf.
+    assert oracle.fp8_to_f64([0x7E], 0, lib=lib)[0] == 448.0
+    assert oracle.fp8_to_f64([0x7C], 1, lib=lib)[0] == math.inf
+
+
+def check_ue8m0_decode_all_codes(lib):
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes.copy()).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    assert _same_values(oracle.ue8m0_to_f64(codes, lib=lib), want)
+    assert oracle.ue8m0_to_f64([127], lib=lib)[0] == 1.0
+
+
+def _bf16_value(bits):
+    import torch
+    t = torch.from_numpy(np.asarray(bits, np.uint16).astype(np.int16))
+    return t.view(torch.bfloat16).to(torch.float64).numpy()
+
+
+def check_bf16_rne_vs_torch(lib, n=1 << 15, seed=77):
+    """float32-representable doubles: torch's float32 -> bfloat16 (RNE) is a single rounding there."""
+    import torch
+    rng = np.random.default_rng(seed)
+    bits = rng.integers(0, 1 << 32, size=n, dtype=np.uint64).astype(np.uint32)
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    want = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.f64_to_bf16_bits(f.astype(np.float64), lib=lib)
+    nan = np.isnan(f)
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+def check_bf16_rne_edges(lib):
+    """Hand-derived bfloat16 facts (8 significant bits, fp32's exponent range)."""
+    cases = [
+        (1.0, 0x3F80), (-2.0, 0xC000), (0.0, 0x0000), (-0.0, 0x8000),
+        (1 + 2 ** -8, 0x3F80),            # tie between 1 and 1 + 2^-7: to even (1)
+        (1 + 3 * 2 ** -8, 0x3F82),        # tie between 1 + 2^-7 and 1 + 2^-6: to even
+        (1 + 2 ** -8 + 2 ** -40, 0x3F81), # just above the tie: up (a double-only input)
+        ((2 - 2 ** -7) * 2.0 ** 127, 0x7F7F),   # largest finite
+        ((2 - 2 ** -8) * 2.0 ** 127, 0x7F80),   # halfway to 2^128: ties to even overflow to inf
+        (2.0 ** -133, 0x0001), (2.0 ** -134, 0x0000), (3 * 2.0 ** -134, 0x0002),
+        (2.0 ** -126, 0x0080), ((1 - 2 ** -9) * 2.0 ** -126, 0x0080),
+        (1.5 * 2.0 ** 128, 0x7F80), (-(2.0 ** 200), 0xFF80),   # doubles beyond bfloat16's range
+        (math.inf, 0x7F80), (-math.inf, 0xFF80),
+    ]
+    got = oracle.f64_to_bf16_bits([c[0] for c in cases], lib=lib)
+    for (x, want), g in zip(cases, got):
+        assert int(g) == want, (x, hex(int(g)), hex(want))
+
+
+def _mx_problem(m_sizes, N, K, seed, int_values=True, scale_range=(124, 130)):
+    """Codes, scales and row offsets for a grouped problem (rows padded to 128 per group)."""
+    rng = np.random.default_rng(seed)
+    offs = np.concatenate([[0], np.cumsum([(m + 127) // 128 * 128 for m in m_sizes])[:-1]]).astype(np.int64)
+    rows = int(sum((m + 127) // 128 * 128 for m in m_sizes))
+    G = len(m_sizes)
+    if int_values:
+        # E4M3 codes of the integers -3..3: 0, 1 (0x38), 2 (0x40), 3 (0x44) and their negatives.
+        table = np.array([0xC4, 0xC0, 0xB8, 0x00, 0x38, 0x40, 0x44], np.uint8)
+        A = table[rng.integers(0, 7, size=(rows, K))]
+        B = table[rng.integers(0, 7, size=(G, N, K))]
+    else:
+        A = rng.integers(0, 256, size=(rows, K)).astype(np.uint8)
+        B = rng.integers(0, 256, size=(G, N, K)).astype(np.uint8)
+        A[(A & 0x7F) == 0x7F] = 0x30   # no NaN codes
+        B[(B & 0x7F) == 0x7F] = 0x30
+    SFA = rng.integers(scale_range[0], scale_range[1], size=(rows, K // 32)).astype(np.uint8)
+    SFB = rng.integers(scale_range[0], scale_range[1], size=(G, N, K // 32)).astype(np.uint8)
+    return A, SFA, B, SFB, offs
+
+
+def _nearest_bf16(frac_values):
+    """Exact rationals -> bfloat16 bits by search over every finite bfloat16 (ties to even pattern)."""
+    allbits = np.arange(1 << 16, dtype=np.uint32)
+    vals = _bf16_value(allbits.astype(np.uint16))
+    fin = np.isfinite(vals) & ~((allbits == 0x8000))
+    cand_bits, cand_vals = allbits[fin], vals[fin]
+    order = np.argsort(cand_vals, kind="stable")
+    cand_bits, cand_vals = cand_bits[order], cand_vals[order]
+    out = []
+    for q in frac_values:
+        x = float(q)
+        i = int(np.searchsorted(cand_vals, x))
+        best = None
+        for j in (i - 1, i, i + 1):
+            if 0 <= j < cand_vals.size:
+                d = abs(Fraction(cand_vals[j]) - q)
+                key = (d, int(cand_bits[j]) & 1)
+                if best is None or key < best[0]:
+                    best = (key, int(cand_bits[j]))
+        out.append(best[1])
+    return np.array(out, np.uint16)
+
+
+def check_mxf8_exact_rational_tiny(lib):
+    """Brute force: exact rational sums of torch-decoded scaled values, rounded by search."""
+    m_sizes, N, K = [3, 2], 5, 64
+    for fmt in (0, 1):
+        A, SFA, B, SFB, offs = _mx_problem(m_sizes, N, K, seed=fmt + 1, int_values=False, scale_range=(120, 134))
+        if fmt == 1:
+            A[(A & 0x7C) == 0x7C] = 0x3C  # no E5M2 inf/NaN codes
+            B[(B & 0x7C) == 0x7C] = 0x3C
+        got = oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, fmt, fmt, lib=lib)
+        av, bv = _torch_fp8(A, fmt), _torch_fp8(B, fmt)
+        for g, (m, o) in enumerate(zip(m_sizes, offs)):
+            for i in range(m):
+                r = o + i
+                q = []
+                for j in range(N):
+                    tot = Fraction(0)
+                    for k in range(K):
+                        tot += (Fraction(av[r, k]) * Fraction(2) ** (int(SFA[r, k // 32]) - 127)
+                                * Fraction(bv[g, j, k]) * Fraction(2) ** (int(SFB[g, j, k // 32]) - 127))
+                    q.append(tot)
+                assert np.array_equal(got[r], _nearest_bf16(q)), (fmt, g, i)
+
+
+def check_mxf8_integer_exact(lib):
+    """Integer values with unit scales: the sums are exact integers below 2^24; torch rounds them to bf16."""
+    import torch
+    m_sizes, N, K = [130, 1, 64], 24, 96
+    A, SFA, B, SFB, offs = _mx_problem(m_sizes, N, K, seed=5, scale_range=(127, 128))
+    av, bv = _torch_fp8(A, 0).astype(np.int64), _torch_fp8(B, 0).astype(np.int64)
+    got = oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, lib=lib, relu=True)
+    for g, (m, o) in enumerate(zip(m_sizes, offs)):
+        S = np.maximum(av[o:o + m] @ bv[g].T, 0).astype(np.float32)
+        want = torch.from_numpy(S).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got[o:o + m], want), g
+
+
+def check_mxf8_identity_and_groups(lib):
+    """A = identity (code 0x38 = 1.0, unit scales): group g's rows are rows of B_g^T, i.e.
+    C[o_g + i, j] = b_g(j, i); rows between groups are left untouched."""
+    m_sizes, N, K = [40, 7, 64], 48, 64
+    G = len(m_sizes)
+    A, SFA, B, SFB, offs = _mx_problem(m_sizes, N, K, seed=9, int_values=False, scale_range=(127, 128))
+    A[:] = 0
+    for o, m in zip(offs, m_sizes):
+        A[o + np.arange(m), np.arange(m)] = 0x38
+    guard = np.full(A.shape[0] * N, 0x7E55, np.uint16)
+    got = oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, C=guard, lib=lib)
+    bv = _torch_fp8(B, 0)
+    covered = np.zeros(A.shape[0], bool)
+    for g, (o, m) in enumerate(zip(offs, m_sizes)):
+        want = _bf16_bits_exact(bv[g, :, :m].T + 0.0)      # a sum that starts at +0 is never -0
+        assert np.array_equal(got[o:o + m], want), g
+        covered[o:o + m] = True
+    assert np.all(got[~covered] == 0x7E55)
+
+
+def _bf16_bits_exact(x):
+    """bfloat16 bits of values known to be exactly representable in bfloat16 (fp8 values are)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def check_mxf8_scale_invariance(lib):
+    """Moving a power of two between an element block and its scale changes nothing: doubling
+    every E4M3 value of A's block (r, s) (exponent field + 1) and lowering its scale by one
+    gives the same C; raising one of B's scales by one doubles that block's contribution."""
+    m_sizes, N, K = [5], 16, 96
+    A, SFA, B, SFB, offs = _mx_problem(m_sizes, N, K, seed=13, scale_range=(126, 129))
+    base = oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, lib=lib)
+    A2, SFA2 = A.copy(), SFA.copy()
+    blk = A2[2, 32:64]
+    nz = (blk & 0x7F) != 0
+    blk[nz] = blk[nz] + 0x08                 # exponent + 1 (values are normal and small)
+    SFA2[2, 1] -= 1
+    got = oracle.gemm_mxf8_grouped(A2, SFA2, B, SFB, m_sizes, offs, N, K, lib=lib)
+    assert np.array_equal(got, base)
+    # Only B's block 2 nonzero: raising its scale doubles every output exactly.
+    B3 = B.copy()
+    B3[:, :, :64] = 0
+    c1 = _bf16_value(oracle.gemm_mxf8_grouped(A, SFA, B3, SFB, m_sizes, offs, N, K, lib=lib))
+    SFB3 = SFB.copy()
+    SFB3[:, :, 2] += 1
+    c2 = _bf16_value(oracle.gemm_mxf8_grouped(A, SFA, B3, SFB3, m_sizes, offs, N, K, lib=lib))
+    assert np.array_equal(c2, 2 * c1)
+
+
+def check_mxf8_relu_and_nan(lib):
+    """Without ReLU negative sums stay negative; with it they are +0.  A NaN scale (255) makes
+    its rows NaN without ReLU and +0 with it."""
+    m_sizes, N, K = [9], 12, 32
+    A, SFA, B, SFB, offs = _mx_problem(m_sizes, N, K, seed=17, scale_range=(127, 128))
+    plain = oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, lib=lib)
+    relu = oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, relu=True, lib=lib)
+    pv = _bf16_value(plain[:9])
+    assert (pv < 0).any()
+    assert np.array_equal(relu[:9], np.where(pv > 0, plain[:9], 0).astype(np.uint16))
+    SFA[4, 0] = 255
+    nanrow = _bf16_value(oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, lib=lib)[4])
+    assert np.all(np.isnan(nanrow))
+    assert np.all(oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, relu=True, lib=lib)[4] == 0)
+
+
 ALL_CHECKS = [
     check_f16_to_f32_all_patterns,
     check_f32_to_f16_golden,
@@ -376,4 +600,13 @@ ALL_CHECKS = [
     check_ex_strides,
     check_ex_bias_exact,
     check_ex_bias_closed_form,
+    check_fp8_decode_all_codes,
+    check_ue8m0_decode_all_codes,
+    check_bf16_rne_vs_torch,
+    check_bf16_rne_edges,
+    check_mxf8_exact_rational_tiny,
+    check_mxf8_integer_exact,
+    check_mxf8_identity_and_groups,
+    check_mxf8_scale_invariance,
+    check_mxf8_relu_and_nan,
 ]

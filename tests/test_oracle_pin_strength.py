@@ -27,6 +27,17 @@ MUTANTS = [
      "const float v = (acc[j] > 0.0f ? acc[j] : 0.0f) + (bias ? oracle_f16_to_f32(bias[j]) : 0.0f);"),
     ("ex_transposed_a_ignored", "a_km ? A[k * lda + i] : A[i * lda + k]", "A[i * lda + k]"),
     ("ex_ldc_ignored", "C[i * ldc + j] = oracle_f32_to_f16_rne(v);", "C[i * N + j] = oracle_f32_to_f16_rne(v);"),
+    ("e4m3_nan_as_number", "if (e == 15 && m == 7)", "if (0)"),
+    ("e4m3_wrong_bias", "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 9)"),
+    ("e5m2_wrong_subnormal", "ldexp((double)m, -16)", "ldexp((double)m, -15)"),
+    ("ue8m0_wrong_bias", "ldexp(1.0, (int)e - 127)", "ldexp(1.0, (int)e - 128)"),
+    ("bf16_wrong_quantum", "subnormal ? -133 : e - 7", "subnormal ? -133 : e - 8"),
+    ("bf16_no_overflow", "if (e > 127)", "if (e > 128)"),
+    ("mx_block_index_ignored", "SFA[r * S + k / 32]", "SFA[r * S]"),
+    ("mx_b_not_transposed", "B[brow * K + k]", "B[(int64_t)g * N * K + k * N + j]"),
+    ("mx_group_ignored", "const int64_t brow = (int64_t)g * N + j;", "const int64_t brow = j;"),
+    ("mx_relu_ignored", "relu ? (acc > 0.0 ? acc : 0.0) : acc", "acc"),
+    ("mx_scale_b_dropped", "* oracle_ue8m0_to_f64(SFB[brow * S + k / 32])", ""),
     ("fp64_accumulator", "float *acc = (float *)malloc((size_t)N * sizeof(float));",
      "double *acc = (double *)malloc((size_t)N * sizeof(double));"),
 ]
