@@ -43,7 +43,9 @@ KERNEL_SOURCES = {
     "tc_pair": [_CSRC + "gemm_tc.cuh", _CSRC + "gemm_tc_pair.cuh", _CSRC + "ptx.cuh"],
     "tc_pair512": [_CSRC + "gemm_tc.cuh", _CSRC + "gemm_tc_pair.cuh", _CSRC + "ptx.cuh"],
     "skinny": [_CSRC + "gemm_skinny.cuh", _CSRC + "ptx.cuh"],
+    "mxf8": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
 }
+MX_METRIC = "MXFP8 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP8 tensor peak"
 PROFILES = os.path.join(ROOT, "profiles")
 L2_BYTES = 126 * 1024 * 1024
 
@@ -55,7 +57,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="square8192",
-                    help="square8192 (the metric's workload), square4096, square256, skinny:<M>, ragged:<i>")
+                    help="square8192 (the metric's workload), square4096, square256, skinny:<M>, ragged:<i>, "
+                         "linear8192, mxf8_moe, mxf8_8192")
     ap.add_argument("--path", default="auto", help="force a kernel path: auto, tc, tc_edge, skinny, tc_pair, tc_pair512")
     ap.add_argument("--workspace", choices=["auto", "none"], default="auto",
                     help="auto: give the library the scratch bytes it asks for (repack path for "
@@ -299,6 +302,8 @@ def rank_seed(workload_seed: int, rank: int) -> int:
 # ---------------------------------------------------------------------------
 
 def run_ours(args):
+    if args.workload in inputs.MX_WORKLOADS:
+        return run_ours_mx(args)
     import torch
     import tiled_dense_gemm_fp16_b200 as tg
 
@@ -489,6 +494,155 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(A, B, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _init_ranks(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    return world, rank, dev, dist
+
+
+def mx_flops(m_sizes, N, K) -> int:
+    return 2 * int(sum(m_sizes)) * N * K
+
+
+def cpu_baseline_mx(ops, m_sizes, N, K, target_s: float):
+    """The oracle on the first rows of group 0, grown until one run takes about target_s."""
+    import oracle
+    A, SFA, B, SFB = ops
+    cores = os.cpu_count() or 1
+    rows = 1
+    while True:
+        t0 = time.perf_counter()
+        oracle.gemm_mxf8_grouped(A[:rows], SFA[:rows], B[:1], SFB[:1], [rows], [0], N, K, nthreads=cores)
+        dt = time.perf_counter() - t0
+        if dt >= target_s or rows >= m_sizes[0]:
+            break
+        rows = min(int(m_sizes[0]), max(rows * 2, int(rows * target_s / max(dt, 1e-3) * 0.9)))
+    value = mx_flops([rows], N, K) / dt / 1e12
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"rows 0..{rows - 1} of group 0 ({rows} x {N} x {K}), {dt:.1f} s on {cores} threads",
+            "seconds": dt}
+
+
+def run_ours_mx(args):
+    """The MXFP8 grouped GEMM on one of inputs.MX_WORKLOADS (operands resident in HBM)."""
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    world, rank, dev, dist = _init_ranks(args)
+    m_sizes, N, K, seed = inputs.MX_WORKLOADS[args.workload]
+    m_sizes = list(m_sizes)
+    ops = inputs.mx_operands(m_sizes, N, K, seed if rank == 0 else rank_seed(seed, rank), "normal")
+    A, SFA, B, SFB = ops
+    sfa_b, sfb_b = inputs.mx_scales_blocked(SFA), inputs.mx_scales_blocked(SFB)
+    rows = A.shape[0]
+    Ad, Bd = torch.from_numpy(A).to(dev), torch.from_numpy(B).to(dev)
+    SFAd, SFBd = torch.from_numpy(sfa_b).to(dev), torch.from_numpy(sfb_b).to(dev)
+    Cd = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+    sh = stream.cuda_stream
+    flops = mx_flops(m_sizes, N, K)
+    in_bytes = A.nbytes + B.nbytes + sfa_b.nbytes + sfb_b.nbytes
+    work_bytes = in_bytes + 2 * rows * N
+
+    def call():
+        st = tg.gemm_mxf8_grouped_raw(Ad.data_ptr(), SFAd.data_ptr(), Bd.data_ptr(), SFBd.data_ptr(),
+                                      Cd.data_ptr(), m_sizes, N, K, 0, 0, False, sh)
+        if st != tg.Status.OK:
+            raise tg.TGError(st, "tg_gemm_mxf8_grouped")
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            call()
+    torch.cuda.synchronize(dev)
+    st, word = tg.device_status()
+    if st != tg.Status.OK:
+        raise SystemExit(f"device error after warm-up: {tg.status_string(st)} 0x{word:x}")
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        r0.record(stream)
+        for _ in range(args.steps):
+            call()
+        r1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    step_ms = r0.elapsed_time(r1) / args.steps
+    kern_ms = step_ms
+    if dist is not None:
+        step_ms = max_over_ranks(dist, step_ms, dev)
+    st, word = tg.device_status()
+    if st != tg.Status.OK:
+        raise SystemExit(f"device error in timed region: {tg.status_string(st)} 0x{word:x}")
+    value = aggregate_throughput(world, flops, step_ms)
+
+    hosts = [torch.from_numpy(x).pin_memory() for x in (A, B, sfa_b, sfb_b)]
+    devs = [Ad, Bd, SFAd, SFBd]
+    Ch = torch.empty((rows, N), dtype=torch.bfloat16).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(args.e2e_steps + 1):
+            if i == 1:
+                e0.record(stream)
+            for d_, h_ in zip(devs, hosts):
+                d_.copy_(h_, non_blocking=True)
+            call()
+            Ch.copy_(Cd, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        e2e_ms = max_over_ranks(dist, e2e_ms, dev)
+
+    peaks, peak_src = load_peaks()
+    peak = 2.0 * float(peaks["bf16_tflops"])
+    achieved = flops / (kern_ms * 1e-3) / 1e12
+    line = {
+        "metric": MX_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 x e4m3, ue8m0 scales per 32 (fp32 accumulate, bf16 out)",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "groups": len(m_sizes), "m_sizes": m_sizes, "N": N, "K": K,
+                   "layout": "A stacked rows x K (groups on 128-row boundaries), B groups x N x K, blocked scales",
+                   "values": "N(0,1) rounded to e4m3, scales 2^-3..2^3", "seed": seed, "path": "mxf8_grouped",
+                   "l2": "inputs larger than L2" if work_bytes > 2 * L2_BYTES else "operands partly L2-resident",
+                   "parallelism": f"dp{world} independent problems" if world > 1 else "1 GPU"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": committed_traffic("mxf8", args.workload) if rank == 0 else None,
+                     "peak_source": f"{peak_src} cuBLAS bf16 burst peak x 2 (nominal dense fp8:bf16 ratio)",
+                     "kernel_ms": kern_ms},
+        "e2e": {"value": aggregate_throughput(world, flops, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": 2 * rows * N, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_mx(ops, m_sizes, N, K, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

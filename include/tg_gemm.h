@@ -267,6 +267,55 @@ TG_API const char *tg_path_name(int path);
 /* Library version, major * 10000 + minor * 100 + patch. */
 TG_API int tg_version(void);
 
+/* ---------------------------------------------------------------------------
+ * MXFP8 block-scaled grouped GEMM
+ *
+ * The Blackwell "MXFP8 grouped GEMM with block scaling + transposed B matrix"
+ * (zhichai.net TileLang topic page, "Key Technical Milestones"), with the
+ * number formats of the OCP Microscaling (MX) definitions.  For G groups that
+ * share N and K, group g owning m_sizes[g] rows:
+ *
+ *   C[r*N + j] = bf16( [relu]( sum_{k<K} a(r,k) sa(r,k/32) * b_g(j,k) sb_g(j,k/32) ) )
+ *
+ * A: stacked rows x K fp8 codes, row-major (K-major).  Group g's rows start at
+ *    row o_g = sum_{h<g} roundup(m_sizes[h], 128): every group starts on a
+ *    multiple of 128 rows.  rows = tg_mx_grouped_rows(m_sizes, G).  Rows
+ *    between groups are read but do not affect C.
+ * B: G x N x K fp8 codes; group g's weight is stored N x K (transposed B).
+ * a(r,k), b_g(j,k): E4M3 (TG_FP8_E4M3, OCP "fn": no inf, 0x7F/0xFF NaN) or
+ *    E5M2 (TG_FP8_E5M2) values, chosen per operand.
+ * SFA, SFB: UE8M0 scales (2^(e-127); 255 = NaN), one per 32 elements of a
+ *    row along K, in the 128 x 4 blocked layout: for a matrix of R rows and
+ *    S = K/32 scale columns, padded to R' = roundup(R, 128) and
+ *    S' = roundup(S, 4), scale (r, s) is the byte at
+ *      ((r/128) * (S'/4) + s/4) * 512 + (r%32) * 16 + ((r/32)%4) * 4 + s%4.
+ *    SFA covers A's stacked rows; SFB holds G such arrays back to back, group
+ *    g's for its N rows at offset g * tg_mx_scale_bytes(N, K).  Padding bytes
+ *    are never used for a valid output.
+ * C: stacked rows x N bf16, row-major; only the m_sizes[g] rows of each group
+ *    are written.  relu = 1 maps every value that is not > 0 to +0.
+ * The sum is accumulated in fp32 by the tensor core; the result is rounded to
+ * bf16 (nearest even).
+ *
+ * Requirements (else TG_ERR_INVALID_ARG, nothing enqueued): 0 <= G <= 256,
+ * m_sizes[g] >= 0, K % 32 == 0, N % 8 == 0, 16-byte aligned A, B, SFA, SFB
+ * and C, C not overlapping any input.  m_sizes is a HOST array.  G == 0,
+ * N == 0 or all-empty groups: TG_OK with nothing enqueued; K == 0 writes +0.
+ * Asynchronous on `stream`; no device memory is allocated.
+ * ------------------------------------------------------------------------- */
+enum { TG_FP8_E4M3 = 0, TG_FP8_E5M2 = 1 };
+
+TG_API tg_status tg_gemm_mxf8_grouped(const void *A, const void *SFA, const void *B, const void *SFB, void *C,
+                                      const int64_t *m_sizes, int32_t groups, int64_t N, int64_t K,
+                                      int32_t a_format, int32_t b_format, int32_t relu, void *stream);
+
+/* Stacked rows for these group sizes (each padded to 128), or -1 if invalid. */
+TG_API int64_t tg_mx_grouped_rows(const int64_t *m_sizes, int32_t groups);
+
+/* Bytes of one blocked UE8M0 scale array for `rows` rows and K elements
+ * (roundup(rows, 128) * roundup(K/32, 4)), or -1 if K % 32 != 0. */
+TG_API int64_t tg_mx_scale_bytes(int64_t rows, int64_t K);
+
 #ifdef __cplusplus
 }
 #endif

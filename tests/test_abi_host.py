@@ -195,3 +195,45 @@ def test_extended_options_validation_and_paths():
     assert tg.workspace_size_ex(A0, B0, C0, 304, 512, 512, t) == 0
     # A bias that overlaps C is refused.
     assert tg.gemm_relu_f16_ex_raw(A0, B0, C0, 64, 64, 64, tg.options(bias=C0 + 64)) == Status.INVALID_ARG
+
+
+def test_mx_host_helpers_and_validation():
+    assert tg.mx_grouped_rows([200, 0, 77, 128]) == 256 + 0 + 128 + 128
+    assert tg.mx_grouped_rows([]) == 0
+    assert tg.mx_grouped_rows([-1]) == -1
+    assert tg.mx_grouped_rows([1] * 257) == -1
+    assert tg.mx_scale_bytes(1, 32) == 128 * 4
+    assert tg.mx_scale_bytes(300, 7168) == 384 * 224
+    assert tg.mx_scale_bytes(300, 100) == -1
+    P = 0x40_0000_0000
+    ok = dict(A=P, SFA=P + (1 << 30), B=P + (2 << 30), SFB=P + (3 << 30), C=P + (4 << 30))
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return tg.gemm_mxf8_grouped_raw(a["A"], a["SFA"], a["B"], a["SFB"], a["C"], kw.get("m", [128]),
+                                        kw.get("N", 256), kw.get("K", 256), kw.get("af", 0), kw.get("bf", 0))
+    assert call(K=100) == Status.INVALID_ARG          # K not a multiple of 32
+    assert call(N=100) == Status.INVALID_ARG          # N not a multiple of 8
+    assert call(af=2) == Status.INVALID_ARG
+    assert call(C=P + (4 << 30) + 8) == Status.INVALID_ARG   # C not 16-byte aligned
+    assert call(SFA=0) == Status.INVALID_ARG
+    assert call(C=P + 64) == Status.INVALID_ARG       # C overlaps A
+    assert call(m=[-3]) == Status.INVALID_ARG
+    assert call(m=[0, 0]) == Status.OK                # nothing to do: no launch
+    assert call(N=0) == Status.OK
+
+
+def test_mx_blocked_layout_formula():
+    """The blocked scale layout is a permutation: every (row, block) lands on its own byte, and one
+    128-row x 4-block atom fills 512 consecutive bytes (32 lines of 16)."""
+    import numpy as np
+    from tiled_dense_gemm_fp16_b200 import inputs
+    R, S = 300, 10
+    vals = (np.arange(R * S) % 251 + 1).astype(np.uint8).reshape(R, S)
+    out = inputs.mx_scales_blocked(vals)
+    assert out.size == tg.mx_scale_bytes(R, 32 * S) == 384 * 12
+    assert np.count_nonzero(out) == R * S
+    # Row 37 (line 5, quarter 1), block 6 (atom column 1, byte 2) of the first 128 rows.
+    assert out[(0 * 3 + 1) * 512 + 5 * 16 + 1 * 4 + 2] == vals[37, 6]
+    # Row 200 (second 128-row band): band 1, line 8, quarter 2, block 9 (atom column 2, byte 1).
+    assert out[(1 * 3 + 2) * 512 + 8 * 16 + 2 * 4 + 1] == vals[200, 9]

@@ -11,6 +11,8 @@ from ._binding import (  # noqa: F401
     B_KN,
     B_NK,
     EXPORTS,
+    FP8_E4M3,
+    FP8_E5M2,
     GemmOptions,
     LIB_PATH,
     STATIC_WORKSPACE_BYTES,
@@ -24,8 +26,12 @@ from ._binding import (  # noqa: F401
     gemm_relu_f16_raw,
     gemm_relu_f16_static_ws_raw,
     gemm_relu_f16_ws_raw,
+    gemm_mxf8_grouped_raw,
     linear_relu,
     lib,
+    mx_grouped_rows,
+    mx_scale_bytes,
+    mxf8_grouped,
     options,
     path_name,
     path_supports,

@@ -47,6 +47,7 @@ class TGError(RuntimeError):
 
 A_MK, A_KM = 0, 1
 B_KN, B_NK = 0, 1
+FP8_E4M3, FP8_E5M2 = 0, 1
 
 
 class GemmOptions(ctypes.Structure):
@@ -84,6 +85,9 @@ EXPORTS = (
     "tg_status_string",
     "tg_path_name",
     "tg_version",
+    "tg_gemm_mxf8_grouped",
+    "tg_mx_grouped_rows",
+    "tg_mx_scale_bytes",
 )
 
 _lib = None
@@ -125,6 +129,14 @@ def _bind(lib):
     lib.tg_path_name.restype = ctypes.c_char_p
     lib.tg_version.argtypes = []
     lib.tg_version.restype = i32
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    lib.tg_gemm_mxf8_grouped.argtypes = [vp, vp, vp, vp, vp, i64p, ctypes.c_int32, i64, i64, ctypes.c_int32,
+                                         ctypes.c_int32, ctypes.c_int32, vp]
+    lib.tg_gemm_mxf8_grouped.restype = i32
+    lib.tg_mx_grouped_rows.argtypes = [i64p, ctypes.c_int32]
+    lib.tg_mx_grouped_rows.restype = i64
+    lib.tg_mx_scale_bytes.argtypes = [i64, i64]
+    lib.tg_mx_scale_bytes.restype = i64
     return lib
 
 
@@ -340,4 +352,56 @@ def bmm_relu(A, B, bias=None, out=None, stream=None, workspace="auto"):
     opts = options(bias=bias.data_ptr() if bias is not None else 0, batch=nb, stride_a=M * K, stride_b=K * N,
                    stride_c=M * N)
     _call_ex(A.data_ptr(), B.data_ptr(), out.data_ptr(), M, N, K, opts, A.device, stream, workspace)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# MXFP8 grouped GEMM
+# ---------------------------------------------------------------------------
+
+def _i64_array(values):
+    values = [int(v) for v in values]
+    return (ctypes.c_int64 * max(1, len(values)))(*values), len(values)
+
+
+def mx_grouped_rows(m_sizes) -> int:
+    """Stacked rows of A / C for these group sizes (each group padded to 128 rows); -1 if invalid."""
+    arr, n = _i64_array(m_sizes)
+    return int(lib().tg_mx_grouped_rows(arr, n))
+
+
+def mx_scale_bytes(rows: int, K: int) -> int:
+    """Bytes of one blocked UE8M0 scale array for ``rows`` rows and K elements."""
+    return int(lib().tg_mx_scale_bytes(rows, K))
+
+
+def gemm_mxf8_grouped_raw(A: int, SFA: int, B: int, SFB: int, C: int, m_sizes, N: int, K: int,
+                          a_format: int = FP8_E4M3, b_format: int = FP8_E4M3, relu: bool = False,
+                          stream: int = 0) -> int:
+    arr, n = _i64_array(m_sizes)
+    return int(lib().tg_gemm_mxf8_grouped(A, SFA, B, SFB, C, arr, n, N, K, int(a_format), int(b_format),
+                                          1 if relu else 0, stream))
+
+
+def mxf8_grouped(A, SFA, B, SFB, m_sizes, relu=False, a_format=FP8_E4M3, b_format=FP8_E4M3, out=None,
+                 stream=None):
+    """Grouped MXFP8 GEMM on CUDA tensors (uint8 codes): A (rows, K), B (G, N, K), SFA / SFB in the
+    blocked scale layout; returns C (rows, N) bfloat16 (rows outside the groups untouched)."""
+    import torch
+    if A.dim() != 2 or B.dim() != 3 or A.shape[1] != B.shape[2] or B.shape[0] != len(m_sizes):
+        raise ValueError(f"shape mismatch: A{tuple(A.shape)} B{tuple(B.shape)} groups={len(m_sizes)}")
+    rows, K = A.shape
+    N = B.shape[1]
+    if rows != mx_grouped_rows(m_sizes):
+        raise ValueError("A must have tg_mx_grouped_rows(m_sizes) rows")
+    for t in (A, B, SFA, SFB):
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise TypeError("operands and scales must be contiguous uint8 tensors")
+    if out is None:
+        out = torch.empty((rows, N), dtype=torch.bfloat16, device=A.device)
+    handle = stream.cuda_stream if stream is not None else _stream_handle(A.device)
+    with torch.cuda.device(A.device):
+        st = gemm_mxf8_grouped_raw(A.data_ptr(), SFA.data_ptr(), B.data_ptr(), SFB.data_ptr(), out.data_ptr(),
+                                   m_sizes, N, K, a_format, b_format, relu, handle)
+    _check(st, "tg_gemm_mxf8_grouped")
     return out

@@ -1,0 +1,316 @@
+// gemm_mx.cuh -- MXFP8 block-scaled grouped GEMM on sm_100a tensor cores.
+//
+// The Blackwell MXFP8 grouped GEMM with block scaling and a transposed B
+// ("Key Technical Milestones", zhichai.net TileLang topic page), with the
+// number formats of the OCP Microscaling (MX) definitions:
+//   C[r, j] = bf16( [relu]( sum_k a(r,k) sa(r, k/32) * b_g(j,k) sb_g(j, k/32) ) )
+// for the rows r of group g.  A holds the groups' rows stacked, each group
+// starting on a multiple of 128 rows; B holds one N x K weight per group
+// (rows of length K: the transposed layout); all fp8 operands are K-major.
+//
+// Per CTA (persistent, one per SM): 128 x 256 output tiles, k-stages of 128
+// fp8 elements (one 128-byte swizzled row), 4 stages.  Roles:
+//   warp 0      TMA producer: A box 128 x 128 B, B box 256 x 128 B, plus the
+//               stage's scale factors (512 B for A's 128 rows, 2 x 512 B for
+//               B's 256 rows) with untiled bulk copies;
+//   warp 1      TMEM owner and MMA issuer: per stage, tcgen05.cp moves the
+//               scale factors into TMEM, then four K = 32 MMAs of
+//               kind::mxf8f6f4 with block_scale each read one scale byte;
+//   warps 2-9   epilogue: two warps per TMEM lane quarter, 128 columns each.
+// Scale factors are stored in the 128 x 4 blocked layout that the tensor
+// core reads (512-byte atoms: 32 lines of 16 bytes, line l holding rows
+// l, l+32, l+64, l+96 with four consecutive k-blocks each), so a stage's
+// scales are a contiguous 512 bytes per 128 rows.  The accumulator is single-
+// buffered (256 of 512 TMEM columns; the scale factors use 12 more): the
+// epilogue drains it into registers, frees it, then stores, so the next
+// tile's MMAs overlap the stores.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace tg {
+
+constexpr int kMxMaxGroups = 256;
+
+struct MxParams {
+  const uint8_t* SFA;  // blocked UE8M0 scales of A's stacked rows
+  const uint8_t* SFB;  // blocked UE8M0 scales of B's rows, groups padded to 128 rows
+  __nv_bfloat16* C;    // stacked rows x N
+  int N, K;
+  int k_stages;        // ceil(K / 128): also the number of 512-byte atoms per 128 rows along K
+  int k_blocks;        // K / 32: scale blocks (one MMA each)
+  int n_tiles, m_tiles, num_tiles, group_m;
+  int groups;
+  int n_atoms;         // ceil(N / 128): 128-row scale atoms per group of B
+  int relu;
+  uint32_t idesc;      // formats, shape and scale type; the sf bytes are or-ed in per MMA
+  uint64_t wait_budget_ns;
+  int tile_start[kMxMaxGroups + 1];  // first stacked 128-row tile of each group; [groups] = m_tiles
+  int m_size[kMxMaxGroups];          // rows of each group
+};
+
+struct MxCfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = 256;
+  static constexpr int BK = 128;  // fp8 elements (= bytes) per k-stage
+  static constexpr int STAGES = 4;
+  static constexpr int MMA_WARP = 1;
+  static constexpr int EPI_WARP0 = 2;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
+  static constexpr int A_BYTES = BM * BK;   // 16 KiB
+  static constexpr int B_BYTES = BN * BK;   // 32 KiB
+  static constexpr int SFA_BYTES = 512;
+  static constexpr int SFB_BYTES = 1024;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SFA_COL = 256;       // 4 columns
+  static constexpr int SFB_COL = 264;       // 8 columns
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + BAR_BYTES;
+  static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // 128 columns per epilogue warp
+};
+
+__device__ __forceinline__ void mx_tile_coords(const MxParams& p, int t, int& m_blk, int& n_blk) {
+  const int group_tiles = p.group_m * p.n_tiles;
+  const int g = t / group_tiles;
+  const int first_m = g * p.group_m;
+  const int gm = min(p.m_tiles - first_m, p.group_m);
+  const int local = t - g * group_tiles;
+  m_blk = first_m + local % gm;
+  n_blk = local / gm;
+}
+
+// Group that owns stacked tile row m_blk: the last g with tile_start[g] <= m_blk.
+__device__ __forceinline__ int mx_group_of(const MxParams& p, int m_blk) {
+  int lo = 0, hi = p.groups - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.tile_start[mid] <= m_blk)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float x0, float x1, bool relu) {
+  if (relu) {
+    x0 = x0 > 0.0f ? x0 : 0.0f;
+    x1 = x1 > 0.0f ? x1 : 0.0f;
+  }
+  const __nv_bfloat162 v = __floats2bfloat162_rn(x0, x1);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(MxCfg::THREADS, 1)
+    gemm_mxf8_grouped_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                             const __grid_constant__ MxParams p) {
+  using Cfg = MxCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* a_smem = smem;
+  uint8_t* b_smem = a_smem + Cfg::STAGES * Cfg::A_BYTES;
+  uint8_t* sfa_smem = b_smem + Cfg::STAGES * Cfg::B_BYTES;
+  uint8_t* sfb_smem = sfa_smem + Cfg::STAGES * Cfg::SFA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sfb_smem + Cfg::STAGES * Cfg::SFB_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + Cfg::STAGES;
+  uint64_t* acc_full_bar = bars + 2 * Cfg::STAGES;
+  uint64_t* acc_empty_bar = acc_full_bar + 1;
+  uint64_t* mma_done_bar = acc_empty_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(acc_full_bar, 1);
+    mbar_init(acc_empty_bar, Cfg::EPI_WARPS);
+    mbar_init(mma_done_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    if (p.k_stages > 0) {  // with K = 0 the tensor maps are not encoded
+      tma_prefetch_desc(&tmap_a);
+      tma_prefetch_desc(&tmap_b);
+    }
+  }
+  if (warp == Cfg::MMA_WARP) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_alloc_permit();
+  }
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  tcgen05_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------
+    // Producer
+    // ------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[Cfg::STAGES];
+#pragma unroll
+      for (int s = 0; s < Cfg::STAGES; ++s) last_parity[s] = -1;
+      bool ok = true;
+      const uint64_t pol_b = l2_policy_evict_last();
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        int m_blk, n_blk;
+        mx_tile_coords(p, t, m_blk, n_blk);
+        const int g = mx_group_of(p, m_blk);
+        const int n0 = n_blk * Cfg::BN;
+        const int b_row0 = g * p.N + n0;
+        const int atom_b = g * p.n_atoms + n0 / 128;
+        const bool second_b = n0 / 128 + 1 < p.n_atoms;
+        const uint32_t bytes =
+            Cfg::A_BYTES + Cfg::B_BYTES + Cfg::SFA_BYTES + (second_b ? 2 : 1) * (Cfg::SFB_BYTES / 2);
+        for (int ks = 0; ks < p.k_stages; ++ks) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 41)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          const int k0 = ks * Cfg::BK;
+          tma_load_2d(a_smem + stage * Cfg::A_BYTES, &tmap_a, &full_bar[stage], k0, m_blk * Cfg::BM);
+          tma_load_2d_hint(b_smem + stage * Cfg::B_BYTES, &tmap_b, &full_bar[stage], k0, b_row0, pol_b);
+          bulk_load_g2s(sfa_smem + stage * Cfg::SFA_BYTES,
+                        p.SFA + (static_cast<int64_t>(m_blk) * p.k_stages + ks) * 512, 512, &full_bar[stage]);
+          bulk_load_g2s(sfb_smem + stage * Cfg::SFB_BYTES,
+                        p.SFB + (static_cast<int64_t>(atom_b) * p.k_stages + ks) * 512, 512, &full_bar[stage]);
+          if (second_b)
+            bulk_load_g2s(sfb_smem + stage * Cfg::SFB_BYTES + 512,
+                          p.SFB + (static_cast<int64_t>(atom_b + 1) * p.k_stages + ks) * 512, 512,
+                          &full_bar[stage]);
+          last_parity[stage] = static_cast<int>(phase);
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Every copy issued has landed before the CTA may exit.
+#pragma unroll 1
+      for (int s = 0; s < Cfg::STAGES; ++s) {
+        if (last_parity[s] >= 0) {
+          volatile int no_abort = 0;
+          mbar_wait(&full_bar[s], static_cast<uint32_t>(last_parity[s]), &no_abort, p.wait_budget_ns, 42);
+        }
+      }
+    }
+  } else if (warp == Cfg::MMA_WARP) {
+    // ------------------------------------------------------------------
+    // Scale-factor copies and MMAs
+    // ------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      const uint32_t sfa_tmem = tmem_base + Cfg::SFA_COL;
+      const uint32_t sfb_tmem = tmem_base + Cfg::SFB_COL;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+        if (!mbar_wait(acc_empty_bar, (local & 1) ^ 1u, abort_flag, p.wait_budget_ns, 43)) break;
+        tcgen05_fence_after_sync();
+        for (int ks = 0; ks < p.k_stages; ++ks) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 44)) {
+            ok = false;
+            break;
+          }
+          tcgen05_fence_after_sync();
+          const uint32_t sa = smem_u32(sfa_smem + stage * Cfg::SFA_BYTES);
+          const uint32_t sb = smem_u32(sfb_smem + stage * Cfg::SFB_BYTES);
+          // Copies and MMAs issued by this thread run in issue order, so the
+          // previous stage's MMAs read their scales before these overwrite them.
+          tmem_cp_32x128b_warpx4(sfa_tmem, make_plain_desc(sa, 16, 128));
+          tmem_cp_32x128b_warpx4(sfb_tmem, make_plain_desc(sb, 16, 128));
+          tmem_cp_32x128b_warpx4(sfb_tmem + 4, make_plain_desc(sb + 512, 16, 128));
+          const uint32_t a_addr = smem_u32(a_smem + stage * Cfg::A_BYTES);
+          const uint32_t b_addr = smem_u32(b_smem + stage * Cfg::B_BYTES);
+          const int nk = min(4, p.k_blocks - ks * 4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (k < nk) {
+              const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+              const uint64_t bdesc = make_sw128_desc(b_addr + k * 32, 16, 1024);
+              const uint32_t idesc = p.idesc | (static_cast<uint32_t>(k) << 29) | (static_cast<uint32_t>(k) << 4);
+              const uint32_t byte_sel = static_cast<uint32_t>(k) << 30;
+              umma_mxf8_ss(tmem_base, adesc, bdesc, idesc, sfa_tmem | byte_sel, sfb_tmem | byte_sel,
+                           (ks | k) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(acc_full_bar);
+      }
+      umma_commit(mma_done_bar);
+      volatile int no_abort = 0;
+      mbar_wait(mma_done_bar, 0, &no_abort, p.wait_budget_ns, 45);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------
+    // Epilogue: TMEM -> registers (ReLU, bf16) -> free the accumulator -> C
+    // ------------------------------------------------------------------
+    const int e = warp - Cfg::EPI_WARP0;
+    const int quad = warp & 3;               // TMEM lanes 32*quad .. +31
+    const int half = e >> 2;                 // column half of the tile
+    const bool relu = p.relu != 0;
+    const bool have_k = p.k_blocks > 0;
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      int m_blk, n_blk;
+      mx_tile_coords(p, t, m_blk, n_blk);
+      const int g = mx_group_of(p, m_blk);
+      const bool ready = mbar_wait(acc_full_bar, local & 1, abort_flag, p.wait_budget_ns, 46);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tcgen05_fence_after_sync();
+      uint32_t h[Cfg::EPI_COLS / 2];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + half * Cfg::EPI_COLS;
+#pragma unroll
+      for (int c = 0; c < Cfg::EPI_COLS / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + c * 16, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          h[c * 8 + q] = have_k ? pack_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]), relu) : 0u;
+      }
+      tcgen05_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty_bar);
+      const int local_row = (m_blk - p.tile_start[g]) * Cfg::BM + quad * 32 + lane;
+      if (local_row < p.m_size[g]) {
+        const int row = m_blk * Cfg::BM + quad * 32 + lane;
+        const int col0 = n_blk * Cfg::BN + half * Cfg::EPI_COLS;
+        uint4* dst = reinterpret_cast<uint4*>(p.C + static_cast<int64_t>(row) * p.N + col0);
+#pragma unroll
+        for (int q = 0; q < Cfg::EPI_COLS / 8; ++q)
+          if (col0 + q * 8 < p.N) dst[q] = make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+      }
+    }
+  }
+
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  if (warp == Cfg::MMA_WARP) {
+    tcgen05_fence_after_sync();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace tg

@@ -405,4 +405,60 @@ __host__ __device__ constexpr uint32_t make_idesc_f16_f32(int M, int N, bool a_m
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------------------
+// Block-scaled MMA (kind::mxf8f6f4) and the copies that feed its scale factors
+// ---------------------------------------------------------------------------
+
+// Untiled bulk copy global -> shared of `bytes` (multiple of 16, both
+// addresses 16-byte aligned), completing on `bar` (no multicast).
+__device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled (interleaved) K-major operand:
+// core matrices of 8 rows x 16 bytes, `sbo_bytes` apart along the rows.
+__device__ __forceinline__ uint64_t make_plain_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;  // layout bits 61-63 = 0: no swizzle
+}
+
+// Copy 32 rows x 16 bytes of shared memory (descriptor `sdesc`) into TMEM
+// lanes 0-31 of columns taddr .. taddr+3, replicated into all four 32-lane
+// quarters.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= (A * SFA) . (B * SFB)^T with fp8 A/B and UE8M0 block scales in
+// TMEM; the scale-factor byte used is selected by the descriptor's sf ids.
+__device__ __forceinline__ void umma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor for kind::mxf8f6f4 with fp32 D and UE8M0 scales:
+//   bits 4-5 B scale-factor byte; bits 7-9 / 10-12 A / B format (0 = E4M3,
+//   1 = E5M2); bits 15 / 16 A / B major-ness (0 = K-major); bits 17-22 N >> 3;
+//   bit 23 scale format (1 = UE8M0); bits 24-28 M >> 4; bits 29-30 A
+//   scale-factor byte.
+__host__ __device__ constexpr uint32_t make_idesc_mxf8(int M, int N, int a_fmt, int b_fmt, uint32_t a_sf_byte,
+                                                      uint32_t b_sf_byte) {
+  return ((b_sf_byte & 3u) << 4) | (static_cast<uint32_t>(a_fmt & 7) << 7) |
+         (static_cast<uint32_t>(b_fmt & 7) << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | ((a_sf_byte & 3u) << 29);
+}
+
 }  // namespace tg

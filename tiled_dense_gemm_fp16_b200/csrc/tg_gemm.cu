@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "tg_gemm.h"
+#include "gemm_mx.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc_pair.cuh"
@@ -43,6 +44,7 @@ struct DeviceInfo {
   bool tc_edge_attr = false;
   bool skinny_attr = false;
   unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
+  bool mx_attr = false;
   void* static_ws = nullptr;  // device address of g_static_workspace on this device
 };
 
@@ -732,10 +734,146 @@ bool problem_from_options(const void* A, const void* B, void* C, int64_t M, int6
   return true;
 }
 
+// ---------------------------------------------------------------------------
+// MXFP8 grouped GEMM
+// ---------------------------------------------------------------------------
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Stacked rows of A / C for these group sizes (each group padded to 128
+// rows), or -1 if a size is negative or there are too many groups.
+int64_t mx_rows(const int64_t* m_sizes, int32_t groups) {
+  if (groups < 0 || groups > kMxMaxGroups || (groups > 0 && m_sizes == nullptr)) return -1;
+  int64_t rows = 0;
+  for (int32_t g = 0; g < groups; ++g) {
+    if (m_sizes[g] < 0 || m_sizes[g] > INT_MAX) return -1;
+    rows += round_up(m_sizes[g], 128);
+    if (rows > INT_MAX) return -1;
+  }
+  return rows;
+}
+
+// Bytes of a blocked UE8M0 scale array for `rows` rows and K elements.
+int64_t mx_scale_bytes(int64_t rows, int64_t K) { return round_up(rows, 128) * round_up(K / 32, 4); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool encode_2d_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
+                           const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, int32_t a_format,
+                           int32_t b_format, int32_t relu, void* stream) {
+  const int64_t rows = mx_rows(m_sizes, groups);
+  if (rows < 0 || N < 0 || K < 0 || K % 32 != 0 || N % 8 != 0 || K > INT_MAX) return TG_ERR_INVALID_ARG;
+  if ((a_format != TG_FP8_E4M3 && a_format != TG_FP8_E5M2) || (b_format != TG_FP8_E4M3 && b_format != TG_FP8_E5M2) ||
+      (relu != 0 && relu != 1))
+    return TG_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(groups) * N > INT_MAX - 256) return TG_ERR_INVALID_ARG;
+  if (rows == 0 || N == 0) return TG_OK;
+  if (C == nullptr || !aligned16(C)) return TG_ERR_INVALID_ARG;
+  const int64_t c_bytes = rows * N * 2;
+  if (K > 0) {
+    if (!A || !B || !SFA || !SFB || !aligned16(A) || !aligned16(B) || !aligned16(SFA) || !aligned16(SFB))
+      return TG_ERR_INVALID_ARG;
+    const int64_t a_bytes = rows * K, b_bytes = static_cast<int64_t>(groups) * N * K;
+    const int64_t sfa_bytes = mx_scale_bytes(rows, K), sfb_bytes = groups * mx_scale_bytes(N, K);
+    if (ranges_overlap(C, c_bytes, A, a_bytes) || ranges_overlap(C, c_bytes, B, b_bytes) ||
+        ranges_overlap(C, c_bytes, SFA, sfa_bytes) || ranges_overlap(C, c_bytes, SFB, sfb_bytes))
+      return TG_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  DeviceInfo* info = nullptr;
+  tg_status st = current_device(dev, info);
+  if (st != TG_OK) return st;
+  using Cfg = MxCfg;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!info->mx_attr) {
+      if (cudaFuncSetAttribute(gemm_mxf8_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::SMEM_BYTES) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      info->mx_attr = true;
+    }
+  }
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof ta);
+  std::memset(&tb, 0, sizeof tb);
+  MxParams p;
+  std::memset(&p, 0, sizeof p);
+  if (K > 0) {
+    if (!encode_2d_u8(&ta, A, rows, K, Cfg::BK, Cfg::BM)) return TG_ERR_LAUNCH;
+    if (!encode_2d_u8(&tb, B, static_cast<int64_t>(groups) * N, K, Cfg::BK, Cfg::BN)) return TG_ERR_LAUNCH;
+  }
+  p.SFA = static_cast<const uint8_t*>(SFA);
+  p.SFB = static_cast<const uint8_t*>(SFB);
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.k_stages = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
+  p.k_blocks = static_cast<int>(K / 32);
+  p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
+  p.m_tiles = static_cast<int>(rows / Cfg::BM);
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 8);
+  if (p.group_m < 1) p.group_m = 1;
+  p.groups = groups;
+  p.n_atoms = static_cast<int>((N + 127) / 128);
+  p.relu = relu;
+  p.idesc = make_idesc_mxf8(Cfg::BM, Cfg::BN, a_format, b_format, 0, 0);
+  p.wait_budget_ns = wait_budget(p.k_stages * 2);
+  int tile = 0;
+  for (int32_t g = 0; g < groups; ++g) {
+    p.tile_start[g] = tile;
+    p.m_size[g] = static_cast<int>(m_sizes[g]);
+    tile += static_cast<int>(round_up(m_sizes[g], 128) / 128);
+  }
+  p.tile_start[groups] = tile;
+  const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::SMEM_BYTES);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  LaunchAttrs la;
+  la.fill(cfg, 1);
+  if (cudaLaunchKernelEx(&cfg, gemm_mxf8_grouped_kernel, ta, tb, p) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
+}
+
 }  // namespace
 }  // namespace tg
 
 extern "C" {
+
+tg_status tg_gemm_mxf8_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
+                               const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, int32_t a_format,
+                               int32_t b_format, int32_t relu, void* stream) {
+  return tg::run_mxf8_grouped(A, SFA, B, SFB, C, m_sizes, groups, N, K, a_format, b_format, relu, stream);
+}
+
+int64_t tg_mx_grouped_rows(const int64_t* m_sizes, int32_t groups) { return tg::mx_rows(m_sizes, groups); }
+
+int64_t tg_mx_scale_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K < 0 || K % 32 != 0) return -1;
+  return tg::mx_scale_bytes(rows, K);
+}
 
 tg_status tg_gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream) {
   return tg::run(tg::dense_problem(A, B, C, M, N, K), stream, TG_PATH_AUTO, nullptr, 0);

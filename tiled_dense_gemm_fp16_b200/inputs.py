@@ -54,6 +54,73 @@ def linear_operands(M: int, N: int, K: int, seed: int = 5, dist: str = "uniform"
     return x, W, b
 
 
+# E4M3 codes of the integers -2..2 (values exact in every fp8 format step used here).
+_E4M3_INT_CODES = np.array([0xC0, 0xB8, 0x00, 0x38, 0x40], np.uint8)
+_E5M2_INT_CODES = np.array([0xC0, 0xBC, 0x00, 0x3C, 0x40], np.uint8)
+
+
+def mx_group_offsets(m_sizes):
+    """First stacked row of each group: groups start on multiples of 128 rows."""
+    offs, r = [], 0
+    for m in m_sizes:
+        offs.append(r)
+        r += (int(m) + 127) // 128 * 128
+    return np.array(offs, np.int64), r
+
+
+def _fp8_codes(values: np.ndarray, fmt: int) -> np.ndarray:
+    import torch
+    dt = torch.float8_e4m3fn if fmt == 0 else torch.float8_e5m2
+    return torch.from_numpy(np.ascontiguousarray(values, np.float32)).to(dt).view(torch.uint8).numpy()
+
+
+def mx_operands(m_sizes, N: int, K: int, seed: int, dist: str = "normal", a_format: int = 0, b_format: int = 0,
+                scale_lo: int = 124, scale_hi: int = 131):
+    """Grouped MXFP8 operands: A codes (stacked rows x K, padding rows drawn too), plain row-major
+    scales SFA (rows x K/32), B codes (G x N x K) and SFB (G x N x K/32), in that order from
+    ``default_rng(seed)``.
+
+    ``dist``: "int" draws the integers -2..2 with unit scales (code 127); "normal" draws N(0,1)
+    values rounded to the format by torch (nearest even, saturating formats clamp) and scales
+    uniform in [scale_lo, scale_hi).
+    """
+    rng = np.random.default_rng(seed)
+    G = len(m_sizes)
+    _, rows = mx_group_offsets(m_sizes)
+    S = K // 32
+    if dist == "int":
+        ta = _E4M3_INT_CODES if a_format == 0 else _E5M2_INT_CODES
+        tb = _E4M3_INT_CODES if b_format == 0 else _E5M2_INT_CODES
+        A = ta[rng.integers(0, 5, size=(rows, K))]
+        SFA = np.full((rows, S), 127, np.uint8)
+        B = tb[rng.integers(0, 5, size=(G, N, K))]
+        SFB = np.full((G, N, S), 127, np.uint8)
+        return A, SFA, B, SFB
+    if dist != "normal":
+        raise ValueError(f"unknown distribution {dist!r}")
+    A = _fp8_codes(rng.standard_normal(size=(rows, K)), a_format)
+    SFA = rng.integers(scale_lo, scale_hi, size=(rows, S)).astype(np.uint8)
+    B = _fp8_codes(rng.standard_normal(size=(G, N, K)), b_format)
+    SFB = rng.integers(scale_lo, scale_hi, size=(G, N, S)).astype(np.uint8)
+    return A, SFA, B, SFB
+
+
+def mx_scales_blocked(sf: np.ndarray) -> np.ndarray:
+    """Plain row-major scales (R x S) rearranged into the C ABI's 128 x 4 blocked byte layout:
+    scale (r, s) goes to ((r//128)*(S'/4) + s//4)*512 + (r%32)*16 + ((r//32)%4)*4 + s%4, with
+    S' = roundup(S, 4); padding bytes are 0.  A G x N x S array gives G blocked arrays back to back."""
+    if sf.ndim == 3:
+        parts = [mx_scales_blocked(sf[g]) for g in range(sf.shape[0])]
+        return np.concatenate(parts) if parts else np.zeros(0, np.uint8)
+    R, S = sf.shape
+    Rp, Sp = (R + 127) // 128 * 128, (S + 3) // 4 * 4
+    out = np.zeros(Rp * Sp, np.uint8)
+    r = np.arange(R)[:, None]
+    s = np.arange(S)[None, :]
+    out[((r // 128) * (Sp // 4) + s // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + s % 4] = sf
+    return out
+
+
 @dataclass(frozen=True)
 class Workload:
     name: str
@@ -86,6 +153,13 @@ WORKLOADS = {
     # Beyond the five: a linear layer relu(x W^T + b) with the weight stored N x K.
     "linear8192": Workload("linear8192", ((8192, 8192, 8192),), "uniform", 5,
                            "x (M x K), weight stored N x K, fp16 bias; drawn by linear_operands"),
+}
+
+# MXFP8 grouped workloads: (group sizes, N, K, seed).  "mxf8_moe" is a mixture-of-experts
+# layer shape: 8 experts with ragged token counts (16384 tokens in all), N = 4096, K = 7168.
+MX_WORKLOADS = {
+    "mxf8_moe": ((2304, 1792, 2048, 2560, 1536, 2048, 2176, 1920), 4096, 7168, 6),
+    "mxf8_8192": ((8192,), 8192, 8192, 7),
 }
 
 
