@@ -88,6 +88,13 @@ def _bind(lib):
     lib.oracle_gemm_mxf8_grouped.argtypes = [u8p, u8p, u8p, u8p, u16p, i64p, i64p, ctypes.c_int, i64, i64,
                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     lib.oracle_gemm_mxf8_grouped.restype = ctypes.c_int
+    lib.oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_e2m1_to_f64.restype = ctypes.c_double
+    lib.oracle_ue4m3_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_ue4m3_to_f64.restype = ctypes.c_double
+    lib.oracle_gemm_nvf4_grouped.argtypes = [u8p, u8p, u8p, u8p, u16p, i64p, i64p, ctypes.c_int, i64, i64,
+                                             ctypes.c_double, ctypes.c_int, ctypes.c_int]
+    lib.oracle_gemm_nvf4_grouped.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -236,6 +243,48 @@ def gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, row_offsets, N: int, K: int, a_fo
                                       _ptr(SFB, ctypes.c_uint8), _ptr(C, ctypes.c_uint16), _ptr(row_offsets, ctypes.c_int64),
                                       _ptr(m_sizes, ctypes.c_int64), G, N, K, int(a_format), int(b_format),
                                       1 if relu else 0, int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return C.reshape(rows, N) if N else C
+
+
+def e2m1_to_f64(codes, lib=None) -> np.ndarray:
+    lib = lib or load_library()
+    codes = np.asarray(codes, dtype=np.uint8).reshape(-1)
+    return np.array([lib.oracle_e2m1_to_f64(int(c)) for c in codes], dtype=np.float64)
+
+
+def ue4m3_to_f64(codes, lib=None) -> np.ndarray:
+    lib = lib or load_library()
+    codes = np.asarray(codes, dtype=np.uint8).reshape(-1)
+    return np.array([lib.oracle_ue4m3_to_f64(int(c)) for c in codes], dtype=np.float64)
+
+
+def gemm_nvf4_grouped(A, SFA, B, SFB, m_sizes, row_offsets, N: int, K: int, alpha: float = 1.0, relu: bool = False,
+                      C=None, nthreads: int = 0, lib=None) -> np.ndarray:
+    """Grouped NVF4 GEMM: A (rows x K/2 packed E2M1 bytes), SFA (rows x K/16 UE4M3), B (G x N x K/2),
+    SFB (G x N x K/16); returns bf16 bit patterns (rows x N); rows outside every group keep C's
+    initial contents (zero by default)."""
+    lib = lib or load_library()
+    A = np.ascontiguousarray(np.asarray(A, dtype=np.uint8))
+    SFA = np.ascontiguousarray(np.asarray(SFA, dtype=np.uint8))
+    B = np.ascontiguousarray(np.asarray(B, dtype=np.uint8))
+    SFB = np.ascontiguousarray(np.asarray(SFB, dtype=np.uint8))
+    m_sizes = np.ascontiguousarray(np.asarray(m_sizes, dtype=np.int64))
+    row_offsets = np.ascontiguousarray(np.asarray(row_offsets, dtype=np.int64))
+    G = int(m_sizes.size)
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    rows = A.size // (K // 2) if K else 0
+    if row_offsets.size != G or (G and int((row_offsets + m_sizes).max()) > rows):
+        raise ValueError("groups do not fit in A")
+    if B.size < G * N * (K // 2) or SFB.size < G * N * (K // 16) or SFA.size < rows * (K // 16):
+        raise ValueError("operand too small")
+    C = np.zeros(rows * N, np.uint16) if C is None else np.ascontiguousarray(np.asarray(C, np.uint16)).reshape(-1).copy()
+    rc = lib.oracle_gemm_nvf4_grouped(_ptr(A, ctypes.c_uint8), _ptr(SFA, ctypes.c_uint8), _ptr(B, ctypes.c_uint8),
+                                      _ptr(SFB, ctypes.c_uint8), _ptr(C, ctypes.c_uint16), _ptr(row_offsets, ctypes.c_int64),
+                                      _ptr(m_sizes, ctypes.c_int64), G, N, K, float(alpha), 1 if relu else 0,
+                                      int(nthreads))
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return C.reshape(rows, N) if N else C

@@ -407,6 +407,87 @@ int oracle_gemm_mxf8_grouped(const uint8_t *A, const uint8_t *SFA, const uint8_t
     return 0;
 }
 
+/* ------------------------------------------------------------------------
+ * NVF4 block-scaled grouped GEMM (the NVF4 block-scaled MMA path whose
+ * 8192^3 throughput the tilelang-ai project page quotes, "Three backends
+ * under one language dialect").  The page names the operation only; the
+ * reading taken is NVIDIA's NVFP4 format:
+ *   - elements are FP4 E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa
+ *     bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives), two per byte,
+ *     element 2i in the low nibble and element 2i+1 in the high nibble;
+ *   - every 16 consecutive elements along K share one scale, an FP8 E4M3
+ *     value with its sign bit clear (UE4M3);
+ *   - one fp32 factor alpha multiplies the whole sum (the per-tensor scale);
+ *   - sum in double, optional ReLU, one RNE rounding to bfloat16, as above.
+ * ------------------------------------------------------------------------ */
+
+/* E2M1 code (low 4 bits of `code`) -> value. */
+double oracle_e2m1_to_f64(uint8_t code)
+{
+    const int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -mag : mag;
+}
+
+/* UE4M3 scale code -> value: the E4M3 value of a code with the sign bit
+ * clear; a set sign bit is not a valid scale (NaN here). */
+double oracle_ue4m3_to_f64(uint8_t code)
+{
+    return (code & 0x80) ? NAN : oracle_fp8_to_f64(code, 0);
+}
+
+/*
+ *   C[r*N + j] = bf16_rne( [relu]( alpha * sum_{k<K} a(r,k) sa(r,k/16) * b_g(j,k) sb_g(j,k/16) ) )
+ *
+ * for the rows r = row_offset[g] .. + m_sizes[g] - 1 of group g, with
+ *   a(r,k)    = e2m1(nibble k of row r of A)   A: stacked rows x K/2 bytes
+ *   sa(r,s)   = ue4m3(SFA[r*(K/16) + s])
+ *   b_g(j,k)  = e2m1(nibble k of row g*N + j of B)   B: G x N x K/2 bytes
+ *   sb_g(j,s) = ue4m3(SFB[(g*N + j)*(K/16) + s])
+ * where nibble k of a row is the low half of byte k/2 for even k and the
+ * high half for odd k.  K must be a multiple of 16.  Returns 0, or -1 on bad
+ * arguments.
+ */
+int oracle_gemm_nvf4_grouped(const uint8_t *A, const uint8_t *SFA, const uint8_t *B, const uint8_t *SFB, uint16_t *C,
+                             const int64_t *row_offset, const int64_t *m_sizes, int G, int64_t N, int64_t K,
+                             double alpha, int relu, int nthreads)
+{
+    if (K % 16 != 0 || N < 0 || G < 0)
+        return -1;
+    const int64_t S = K / 16, KB = K / 2;
+#ifdef _OPENMP
+    if (nthreads <= 0)
+        nthreads = omp_get_max_threads();
+#else
+    (void)nthreads;
+#endif
+    for (int g = 0; g < G; ++g) {
+        const int64_t r0 = row_offset[g], mg = m_sizes[g];
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+        for (int64_t i = 0; i < mg; ++i) {
+            const int64_t r = r0 + i;
+            for (int64_t j = 0; j < N; ++j) {
+                const int64_t brow = (int64_t)g * N + j;
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k) {
+                    const int hi = (int)(k & 1);
+                    const uint8_t abyte = A[r * KB + k / 2], bbyte = B[brow * KB + k / 2];
+                    const double av = oracle_e2m1_to_f64(hi ? (uint8_t)(abyte >> 4) : (uint8_t)(abyte & 0xf)) *
+                                      oracle_ue4m3_to_f64(SFA[r * S + k / 16]);
+                    const double bv = oracle_e2m1_to_f64(hi ? (uint8_t)(bbyte >> 4) : (uint8_t)(bbyte & 0xf)) *
+                                      oracle_ue4m3_to_f64(SFB[brow * S + k / 16]);
+                    acc += av * bv;
+                }
+                const double y = alpha * acc;
+                C[r * N + j] = oracle_f64_to_bf16_rne(relu ? (y > 0.0 ? y : 0.0) : y);
+            }
+        }
+    }
+    return 0;
+}
+
 /* Number of threads OpenMP would use by default (1 without OpenMP). */
 int oracle_max_threads(void)
 {

@@ -579,6 +579,128 @@ def check_mxf8_relu_and_nan(lib):
     assert np.all(oracle.gemm_mxf8_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, relu=True, lib=lib)[4] == 0)
 
 
+# --------------------------------------------------------------------------
+# NVF4 grouped GEMM
+# --------------------------------------------------------------------------
+
+def _golden_e2m1():
+    rows = []
+    with open(os.path.join(GOLDEN, "e2m1_values.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                code, val = line.split()[:2]
+                rows.append((int(code, 16), float(val)))
+    return rows
+
+
+def check_e2m1_decode_golden(lib):
+    rows = _golden_e2m1()
+    assert len(rows) == 16
+    got = oracle.e2m1_to_f64([c for c, _ in rows], lib=lib)
+    want = np.array([v for _, v in rows])
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
+    # Only the low nibble is a code: the high nibble of the byte is ignored.
+    assert np.array_equal(oracle.e2m1_to_f64([0xF7, 0x35], lib=lib), [6.0, 3.0])
+
+
+def check_ue4m3_decode(lib):
+    """Scale codes with a clear sign bit are E4M3 values (torch's decoder); a set sign bit is invalid."""
+    codes = np.arange(128, dtype=np.uint8)
+    assert _same_values(oracle.ue4m3_to_f64(codes, lib=lib), _torch_fp8(codes, 0))
+    assert np.all(np.isnan(oracle.ue4m3_to_f64(np.arange(128, 256, dtype=np.uint8), lib=lib)))
+
+
+# E2M1 codes of the integers -4..4 that E2M1 holds: 0, +-1, +-2, +-3, +-4.
+_E2M1_INT = {0: 0x0, 1: 0x2, 2: 0x4, 3: 0x5, 4: 0x6, -1: 0xA, -2: 0xC, -3: 0xD, -4: 0xE}
+
+
+def _pack_nibbles(codes):
+    """Codes (..., K) -> bytes (..., K/2), element 2i in the low nibble."""
+    codes = np.asarray(codes, np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def _nvf4_problem(m_sizes, N, K, seed, int_values=True, scale_codes=(0x38,)):
+    rng = np.random.default_rng(seed)
+    offs, rows = inputs.mx_group_offsets(m_sizes)
+    G = len(m_sizes)
+    if int_values:
+        keys = np.array(sorted(_E2M1_INT))
+        av = keys[rng.integers(0, len(keys), size=(rows, K))]
+        bv = keys[rng.integers(0, len(keys), size=(G, N, K))]
+        ac = np.vectorize(_E2M1_INT.get)(av).astype(np.uint8)
+        bc = np.vectorize(_E2M1_INT.get)(bv).astype(np.uint8)
+    else:
+        ac = rng.integers(0, 16, size=(rows, K)).astype(np.uint8)
+        bc = rng.integers(0, 16, size=(G, N, K)).astype(np.uint8)
+        av = bv = None
+    sc = np.asarray(scale_codes, np.uint8)
+    SFA = sc[rng.integers(0, sc.size, size=(rows, K // 16))]
+    SFB = sc[rng.integers(0, sc.size, size=(G, N, K // 16))]
+    return _pack_nibbles(ac), SFA, _pack_nibbles(bc), SFB, offs, (ac, bc, av, bv)
+
+
+def check_nvf4_integer_exact(lib):
+    """Integer E2M1 values with unit scales (0x38 = 1.0): exact int64 products, rounded by torch."""
+    import torch
+    m_sizes, N, K = [130, 3], 24, 128
+    A, SFA, B, SFB, offs, (_, _, av, bv) = _nvf4_problem(m_sizes, N, K, seed=2)
+    got = oracle.gemm_nvf4_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, lib=lib)
+    for g, (o, m) in enumerate(zip(offs, m_sizes)):
+        S = (av[o:o + m].astype(np.int64) @ bv[g].astype(np.int64).T).astype(np.float32)
+        want = torch.from_numpy(S).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got[o:o + m], want), g
+
+
+def check_nvf4_identity_nibble_order(lib):
+    """A = identity in E2M1 (code 0x2 = 1.0): row i of group g is column i of B_g's stored rows, so the
+    element order inside each packed byte (low nibble first) decides every output."""
+    m_sizes, N, K = [20], 16, 32
+    A, SFA, B, SFB, offs, (_, bc, _, _) = _nvf4_problem(m_sizes, N, K, seed=4, int_values=False)
+    ac = np.zeros((A.shape[0], K), np.uint8)
+    ac[np.arange(20), np.arange(20)] = 0x2
+    SFA[:] = 0x38
+    SFB[:] = 0x38
+    got = oracle.gemm_nvf4_grouped(_pack_nibbles(ac), SFA, B, SFB, m_sizes, offs, N, K, lib=lib)
+    table = dict(_golden_e2m1())
+    want = np.array([[table[int(bc[0, j, i])] for j in range(N)] for i in range(20)], np.float32) + 0.0
+    assert np.array_equal(got[:20], _bf16_bits_exact(want))
+
+
+def check_nvf4_exact_rational_tiny(lib):
+    """Brute force with golden element values, torch-decoded scales, exact sums and alpha."""
+    m_sizes, N, K = [2, 3], 4, 48
+    alpha = 0.3  # not a power of two: the product alpha * sum is rounded once, to bf16
+    A, SFA, B, SFB, offs, (ac, bc, _, _) = _nvf4_problem(m_sizes, N, K, seed=6, int_values=False,
+                                                          scale_codes=(0x20, 0x30, 0x38, 0x41, 0x4C, 0x57))
+    got = oracle.gemm_nvf4_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, alpha=alpha, lib=lib)
+    table = {c: Fraction(v) for c, v in _golden_e2m1()}
+    sc = {int(c): Fraction(float(v)) for c, v in zip(range(127), _torch_fp8(np.arange(127, dtype=np.uint8), 0))}
+    for g, (o, m) in enumerate(zip(offs, m_sizes)):
+        for i in range(m):
+            r = o + i
+            q = []
+            for j in range(N):
+                tot = sum(table[int(ac[r, k])] * sc[int(SFA[r, k // 16])] * table[int(bc[g, j, k])]
+                          * sc[int(SFB[g, j, k // 16])] for k in range(K))
+                q.append(Fraction(alpha) * tot)
+            assert np.array_equal(got[r], _nearest_bf16(q)), (g, i)
+
+
+def check_nvf4_alpha_relu(lib):
+    """alpha = 2^-3 scales every output exactly; ReLU maps the non-positive ones to +0."""
+    m_sizes, N, K = [7], 10, 64
+    A, SFA, B, SFB, offs, _ = _nvf4_problem(m_sizes, N, K, seed=8)
+    base = _bf16_value(oracle.gemm_nvf4_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, lib=lib)[:7])
+    scaled = _bf16_value(oracle.gemm_nvf4_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, alpha=0.125, lib=lib)[:7])
+    assert np.array_equal(scaled, base / 8)
+    assert (base < 0).any()
+    relu = _bf16_value(oracle.gemm_nvf4_grouped(A, SFA, B, SFB, m_sizes, offs, N, K, alpha=0.125, relu=True,
+                                                lib=lib)[:7])
+    assert np.array_equal(relu, np.where(base > 0, base / 8, 0.0))
+
+
 ALL_CHECKS = [
     check_f16_to_f32_all_patterns,
     check_f32_to_f16_golden,
@@ -609,4 +731,10 @@ ALL_CHECKS = [
     check_mxf8_identity_and_groups,
     check_mxf8_scale_invariance,
     check_mxf8_relu_and_nan,
+    check_e2m1_decode_golden,
+    check_ue4m3_decode,
+    check_nvf4_integer_exact,
+    check_nvf4_identity_nibble_order,
+    check_nvf4_exact_rational_tiny,
+    check_nvf4_alpha_relu,
 ]

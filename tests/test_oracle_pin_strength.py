@@ -38,6 +38,15 @@ MUTANTS = [
     ("mx_group_ignored", "const int64_t brow = (int64_t)g * N + j;", "const int64_t brow = j;"),
     ("mx_relu_ignored", "relu ? (acc > 0.0 ? acc : 0.0) : acc", "acc"),
     ("mx_scale_b_dropped", "* oracle_ue8m0_to_f64(SFB[brow * S + k / 32])", ""),
+    ("e2m1_wrong_bias", "ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e - 2)"),
+    ("e2m1_no_subnormal_half", "e == 0 ? 0.5 * m :", "e == 0 ? 1.0 * m :"),
+    ("nvf4_nibbles_swapped", "hi ? (uint8_t)(abyte >> 4) : (uint8_t)(abyte & 0xf)",
+     "hi ? (uint8_t)(abyte & 0xf) : (uint8_t)(abyte >> 4)"),
+    ("nvf4_block_32", "oracle_ue4m3_to_f64(SFA[r * S + k / 16])", "oracle_ue4m3_to_f64(SFA[r * S + k / 32])"),
+    ("nvf4_alpha_ignored", "const double y = alpha * acc;", "const double y = acc;"),
+    ("nvf4_scale_b_dropped", "oracle_ue4m3_to_f64(SFB[brow * S + k / 16])", "1.0"),
+    ("nvf4_group_ignored", "const int64_t brow = (int64_t)g * N + j;\n                double acc = 0.0;\n                for (int64_t k = 0; k < K; ++k) {\n                    const int hi",
+     "const int64_t brow = j;\n                double acc = 0.0;\n                for (int64_t k = 0; k < K; ++k) {\n                    const int hi"),
     ("fp64_accumulator", "float *acc = (float *)malloc((size_t)N * sizeof(float));",
      "double *acc = (double *)malloc((size_t)N * sizeof(double));"),
 ]
