@@ -44,8 +44,10 @@ KERNEL_SOURCES = {
     "tc_pair512": [_CSRC + "gemm_tc.cuh", _CSRC + "gemm_tc_pair.cuh", _CSRC + "ptx.cuh"],
     "skinny": [_CSRC + "gemm_skinny.cuh", _CSRC + "ptx.cuh"],
     "mxf8": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
+    "nvf4": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
 }
 MX_METRIC = "MXFP8 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP8 tensor peak"
+NVF4_METRIC = "NVF4 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP4 tensor peak"
 PROFILES = os.path.join(ROOT, "profiles")
 L2_BYTES = 126 * 1024 * 1024
 
@@ -58,7 +60,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="square8192",
                     help="square8192 (the metric's workload), square4096, square256, skinny:<M>, ragged:<i>, "
-                         "linear8192, mxf8_moe, mxf8_8192")
+                         "linear8192, mxf8_moe, mxf8_8192, nvf4_8192, nvf4_moe")
     ap.add_argument("--path", default="auto", help="force a kernel path: auto, tc, tc_edge, skinny, tc_pair, tc_pair512")
     ap.add_argument("--workspace", choices=["auto", "none"], default="auto",
                     help="auto: give the library the scratch bytes it asks for (repack path for "
@@ -302,7 +304,7 @@ def rank_seed(workload_seed: int, rank: int) -> int:
 # ---------------------------------------------------------------------------
 
 def run_ours(args):
-    if args.workload in inputs.MX_WORKLOADS:
+    if args.workload in inputs.MX_WORKLOADS or args.workload in inputs.NVF4_WORKLOADS:
         return run_ours_mx(args)
     import torch
     import tiled_dense_gemm_fp16_b200 as tg
@@ -525,15 +527,16 @@ def mx_flops(m_sizes, N, K) -> int:
     return 2 * int(sum(m_sizes)) * N * K
 
 
-def cpu_baseline_mx(ops, m_sizes, N, K, target_s: float):
+def cpu_baseline_mx(kind, ops, m_sizes, N, K, target_s: float):
     """The oracle on the first rows of group 0, grown until one run takes about target_s."""
     import oracle
     A, SFA, B, SFB = ops
+    fn = oracle.gemm_mxf8_grouped if kind == "mxf8" else oracle.gemm_nvf4_grouped
     cores = os.cpu_count() or 1
     rows = 1
     while True:
         t0 = time.perf_counter()
-        oracle.gemm_mxf8_grouped(A[:rows], SFA[:rows], B[:1], SFB[:1], [rows], [0], N, K, nthreads=cores)
+        fn(A[:rows], SFA[:rows], B[:1], SFB[:1], [rows], [0], N, K, nthreads=cores)
         dt = time.perf_counter() - t0
         if dt >= target_s or rows >= m_sizes[0]:
             break
@@ -545,13 +548,18 @@ def cpu_baseline_mx(ops, m_sizes, N, K, target_s: float):
 
 
 def run_ours_mx(args):
-    """The MXFP8 grouped GEMM on one of inputs.MX_WORKLOADS (operands resident in HBM)."""
+    """A block-scaled grouped GEMM (MXFP8 or NVF4) on one of its workloads, operands resident in HBM."""
     import torch
     import tiled_dense_gemm_fp16_b200 as tg
     world, rank, dev, dist = _init_ranks(args)
-    m_sizes, N, K, seed = inputs.MX_WORKLOADS[args.workload]
+    kind = "mxf8" if args.workload in inputs.MX_WORKLOADS else "nvf4"
+    m_sizes, N, K, seed = (inputs.MX_WORKLOADS if kind == "mxf8" else inputs.NVF4_WORKLOADS)[args.workload]
     m_sizes = list(m_sizes)
-    ops = inputs.mx_operands(m_sizes, N, K, seed if rank == 0 else rank_seed(seed, rank), "normal")
+    wseed = seed if rank == 0 else rank_seed(seed, rank)
+    if kind == "mxf8":
+        ops = inputs.mx_operands(m_sizes, N, K, wseed, "normal")
+    else:
+        ops = inputs.nvf4_operands(m_sizes, N, K, wseed, "codes")
     A, SFA, B, SFB = ops
     sfa_b, sfb_b = inputs.mx_scales_blocked(SFA), inputs.mx_scales_blocked(SFB)
     rows = A.shape[0]
@@ -565,10 +573,14 @@ def run_ours_mx(args):
     work_bytes = in_bytes + 2 * rows * N
 
     def call():
-        st = tg.gemm_mxf8_grouped_raw(Ad.data_ptr(), SFAd.data_ptr(), Bd.data_ptr(), SFBd.data_ptr(),
-                                      Cd.data_ptr(), m_sizes, N, K, 0, 0, False, sh)
+        if kind == "mxf8":
+            st = tg.gemm_mxf8_grouped_raw(Ad.data_ptr(), SFAd.data_ptr(), Bd.data_ptr(), SFBd.data_ptr(),
+                                          Cd.data_ptr(), m_sizes, N, K, 0, 0, False, sh)
+        else:
+            st = tg.gemm_nvf4_grouped_raw(Ad.data_ptr(), SFAd.data_ptr(), Bd.data_ptr(), SFBd.data_ptr(),
+                                          Cd.data_ptr(), m_sizes, N, K, 1.0, False, sh)
         if st != tg.Status.OK:
-            raise tg.TGError(st, "tg_gemm_mxf8_grouped")
+            raise tg.TGError(st, f"tg_gemm_{kind}_grouped")
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -620,21 +632,27 @@ def run_ours_mx(args):
         e2e_ms = max_over_ranks(dist, e2e_ms, dev)
 
     peaks, peak_src = load_peaks()
-    peak = 2.0 * float(peaks["bf16_tflops"])
+    ratio = 2.0 if kind == "mxf8" else 4.0
+    peak = ratio * float(peaks["bf16_tflops"])
     achieved = flops / (kern_ms * 1e-3) / 1e12
+    if kind == "mxf8":
+        dtype = "e4m3 x e4m3, ue8m0 scales per 32 (fp32 accumulate, bf16 out)"
+        values = "N(0,1) rounded to e4m3, scales 2^-3..2^3"
+    else:
+        dtype = "e2m1 x e2m1, ue4m3 scales per 16, alpha 1 (fp32 accumulate, bf16 out)"
+        values = "uniform E2M1 codes, UE4M3 scale codes 0x28..0x48 (2^-2..2^2)"
     line = {
-        "metric": MX_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3 x e4m3, ue8m0 scales per 32 (fp32 accumulate, bf16 out)",
-        "data": "synthetic",
+        "metric": MX_METRIC if kind == "mxf8" else NVF4_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
         "config": {"workload": args.workload, "groups": len(m_sizes), "m_sizes": m_sizes, "N": N, "K": K,
                    "layout": "A stacked rows x K (groups on 128-row boundaries), B groups x N x K, blocked scales",
-                   "values": "N(0,1) rounded to e4m3, scales 2^-3..2^3", "seed": seed, "path": "mxf8_grouped",
+                   "values": values, "seed": seed, "path": f"{kind}_grouped",
                    "l2": "inputs larger than L2" if work_bytes > 2 * L2_BYTES else "operands partly L2-resident",
                    "parallelism": f"dp{world} independent problems" if world > 1 else "1 GPU"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": committed_traffic("mxf8", args.workload) if rank == 0 else None,
-                     "peak_source": f"{peak_src} cuBLAS bf16 burst peak x 2 (nominal dense fp8:bf16 ratio)",
+                     "frac": achieved / peak, "traffic": committed_traffic(kind, args.workload) if rank == 0 else None,
+                     "peak_source": f"{peak_src} cuBLAS bf16 burst peak x {ratio:g} (nominal dense ratio to bf16)",
                      "kernel_ms": kern_ms},
         "e2e": {"value": aggregate_throughput(world, flops, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": 2 * rows * N, "ms_per_step": e2e_ms},
@@ -642,7 +660,7 @@ def run_ours_mx(args):
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_mx(ops, m_sizes, N, K, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline_mx(kind, ops, m_sizes, N, K, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -316,6 +316,35 @@ TG_API int64_t tg_mx_grouped_rows(const int64_t *m_sizes, int32_t groups);
  * (roundup(rows, 128) * roundup(K/32, 4)), or -1 if K % 32 != 0. */
 TG_API int64_t tg_mx_scale_bytes(int64_t rows, int64_t K);
 
+/* ---------------------------------------------------------------------------
+ * NVF4 block-scaled grouped GEMM
+ *
+ * The NVF4 block-scaled MMA path (tilelang-ai project page, "Three backends
+ * under one language dialect", quoted there at 8192^3), read as NVIDIA's
+ * NVFP4 format, with the grouping and row layout of tg_gemm_mxf8_grouped:
+ *
+ *   C[r*N + j] = bf16( [relu]( alpha * sum_{k<K} a(r,k) sa(r,k/16) * b_g(j,k) sb_g(j,k/16) ) )
+ *
+ * A: stacked rows x K/2 bytes, B: G x N x K/2 bytes; each byte packs two FP4
+ *    E2M1 elements (0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives), element 2i in
+ *    the low nibble.  Group g's rows start at o_g = sum_{h<g} roundup(m_h, 128).
+ * SFA, SFB: one UE4M3 scale (an FP8 E4M3 code with the sign bit clear) per 16
+ *    elements along K, in the 128 x 4 blocked layout described above with
+ *    S = K/16 scale columns; group g's SFB at g * tg_nvf4_scale_bytes(N, K).
+ * alpha: a finite fp32 factor applied to the fp32 accumulator (the per-tensor
+ *    scale of NVFP4).
+ * C: stacked rows x N bf16; only the rows of the groups are written.
+ * Requirements (else TG_ERR_INVALID_ARG, nothing enqueued): K % 64 == 0, the
+ * rest as tg_gemm_mxf8_grouped.  m_sizes is a HOST array.
+ * ------------------------------------------------------------------------- */
+TG_API tg_status tg_gemm_nvf4_grouped(const void *A, const void *SFA, const void *B, const void *SFB, void *C,
+                                      const int64_t *m_sizes, int32_t groups, int64_t N, int64_t K, float alpha,
+                                      int32_t relu, void *stream);
+
+/* Bytes of one blocked UE4M3 scale array for `rows` rows and K elements
+ * (roundup(rows, 128) * roundup(K/16, 4)), or -1 if K % 16 != 0. */
+TG_API int64_t tg_nvf4_scale_bytes(int64_t rows, int64_t K);
+
 #ifdef __cplusplus
 }
 #endif

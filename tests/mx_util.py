@@ -31,3 +31,27 @@ def abs_dot(A, SFA, B, SFB, g, rows, N, K, a_format, b_format):
     av = np.abs(dec_a[A[rows]] * np.repeat(sc[SFA[rows]], 32, axis=1))
     bv = np.abs(dec_b[B[g]] * np.repeat(sc[SFB[g]], 32, axis=1))
     return av @ bv.T
+
+
+def unpack_fp4(packed: np.ndarray) -> np.ndarray:
+    """Bytes (..., K/2) -> 4-bit codes (..., K), element 2i from the low nibble."""
+    packed = np.asarray(packed, np.uint8)
+    out = np.empty(packed.shape[:-1] + (2 * packed.shape[-1],), np.uint8)
+    out[..., 0::2] = packed & 0xF
+    out[..., 1::2] = packed >> 4
+    return out
+
+
+def nvf4_oracle_rows(A, SFA, B, SFB, g, rows, N, K, alpha, relu):
+    rows = np.asarray(rows, np.int64)
+    return oracle.gemm_nvf4_grouped(np.ascontiguousarray(A[rows]), np.ascontiguousarray(SFA[rows]), B[g:g + 1],
+                                    SFB[g:g + 1], [len(rows)], [0], N, K, alpha=alpha, relu=relu)
+
+
+def nvf4_abs_dot(A, SFA, B, SFB, g, rows, N, K):
+    dec = oracle.e2m1_to_f64(np.arange(16, dtype=np.uint8))
+    sc = oracle.ue4m3_to_f64(np.arange(128, dtype=np.uint8))
+    rows = np.asarray(rows, np.int64)
+    av = np.abs(dec[unpack_fp4(A[rows])] * np.repeat(sc[SFA[rows]], 16, axis=1))
+    bv = np.abs(dec[unpack_fp4(B[g])] * np.repeat(sc[SFB[g]], 16, axis=1))
+    return av @ bv.T

@@ -237,3 +237,18 @@ def test_mx_blocked_layout_formula():
     assert out[(0 * 3 + 1) * 512 + 5 * 16 + 1 * 4 + 2] == vals[37, 6]
     # Row 200 (second 128-row band): band 1, line 8, quarter 2, block 9 (atom column 2, byte 1).
     assert out[(1 * 3 + 2) * 512 + 8 * 16 + 2 * 4 + 1] == vals[200, 9]
+
+
+def test_nvf4_host_validation():
+    assert tg.nvf4_scale_bytes(300, 7168) == 384 * 448
+    assert tg.nvf4_scale_bytes(1, 40) == -1
+    P = 0x40_0000_0000
+
+    def call(K=256, N=256, alpha=1.0, m=(128,), C=P + (4 << 30)):
+        return tg.gemm_nvf4_grouped_raw(P, P + (1 << 30), P + (2 << 30), P + (3 << 30), C, list(m), N, K, alpha)
+    assert call(K=96) == Status.INVALID_ARG           # K not a multiple of 64
+    assert call(N=12) == Status.INVALID_ARG
+    assert call(alpha=float("nan")) == Status.INVALID_ARG
+    assert call(alpha=float("inf")) == Status.INVALID_ARG
+    assert call(C=P + 32) == Status.INVALID_ARG       # C overlaps A
+    assert call(m=(0,)) == Status.OK

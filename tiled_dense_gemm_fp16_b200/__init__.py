@@ -27,11 +27,14 @@ from ._binding import (  # noqa: F401
     gemm_relu_f16_static_ws_raw,
     gemm_relu_f16_ws_raw,
     gemm_mxf8_grouped_raw,
+    gemm_nvf4_grouped_raw,
     linear_relu,
     lib,
     mx_grouped_rows,
     mx_scale_bytes,
     mxf8_grouped,
+    nvf4_grouped,
+    nvf4_scale_bytes,
     options,
     path_name,
     path_supports,

@@ -88,6 +88,8 @@ EXPORTS = (
     "tg_gemm_mxf8_grouped",
     "tg_mx_grouped_rows",
     "tg_mx_scale_bytes",
+    "tg_gemm_nvf4_grouped",
+    "tg_nvf4_scale_bytes",
 )
 
 _lib = None
@@ -137,6 +139,11 @@ def _bind(lib):
     lib.tg_mx_grouped_rows.restype = i64
     lib.tg_mx_scale_bytes.argtypes = [i64, i64]
     lib.tg_mx_scale_bytes.restype = i64
+    lib.tg_gemm_nvf4_grouped.argtypes = [vp, vp, vp, vp, vp, i64p, ctypes.c_int32, i64, i64, ctypes.c_float,
+                                         ctypes.c_int32, vp]
+    lib.tg_gemm_nvf4_grouped.restype = i32
+    lib.tg_nvf4_scale_bytes.argtypes = [i64, i64]
+    lib.tg_nvf4_scale_bytes.restype = i64
     return lib
 
 
@@ -404,4 +411,42 @@ def mxf8_grouped(A, SFA, B, SFB, m_sizes, relu=False, a_format=FP8_E4M3, b_forma
         st = gemm_mxf8_grouped_raw(A.data_ptr(), SFA.data_ptr(), B.data_ptr(), SFB.data_ptr(), out.data_ptr(),
                                    m_sizes, N, K, a_format, b_format, relu, handle)
     _check(st, "tg_gemm_mxf8_grouped")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# NVF4 grouped GEMM
+# ---------------------------------------------------------------------------
+
+def nvf4_scale_bytes(rows: int, K: int) -> int:
+    """Bytes of one blocked UE4M3 scale array for ``rows`` rows and K elements."""
+    return int(lib().tg_nvf4_scale_bytes(rows, K))
+
+
+def gemm_nvf4_grouped_raw(A: int, SFA: int, B: int, SFB: int, C: int, m_sizes, N: int, K: int, alpha: float = 1.0,
+                          relu: bool = False, stream: int = 0) -> int:
+    arr, n = _i64_array(m_sizes)
+    return int(lib().tg_gemm_nvf4_grouped(A, SFA, B, SFB, C, arr, n, N, K, float(alpha), 1 if relu else 0, stream))
+
+
+def nvf4_grouped(A, SFA, B, SFB, m_sizes, alpha=1.0, relu=False, out=None, stream=None):
+    """Grouped NVF4 GEMM on CUDA uint8 tensors: A (rows, K/2) and B (G, N, K/2) packed E2M1, SFA / SFB
+    blocked UE4M3 scales; returns C (rows, N) bfloat16 (rows outside the groups untouched)."""
+    import torch
+    if A.dim() != 2 or B.dim() != 3 or A.shape[1] != B.shape[2] or B.shape[0] != len(m_sizes):
+        raise ValueError(f"shape mismatch: A{tuple(A.shape)} B{tuple(B.shape)} groups={len(m_sizes)}")
+    rows, K = A.shape[0], 2 * A.shape[1]
+    N = B.shape[1]
+    if rows != mx_grouped_rows(m_sizes):
+        raise ValueError("A must have tg_mx_grouped_rows(m_sizes) rows")
+    for t in (A, B, SFA, SFB):
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise TypeError("operands and scales must be contiguous uint8 tensors")
+    if out is None:
+        out = torch.empty((rows, N), dtype=torch.bfloat16, device=A.device)
+    handle = stream.cuda_stream if stream is not None else _stream_handle(A.device)
+    with torch.cuda.device(A.device):
+        st = gemm_nvf4_grouped_raw(A.data_ptr(), SFA.data_ptr(), B.data_ptr(), SFB.data_ptr(), out.data_ptr(),
+                                   m_sizes, N, K, alpha, relu, handle)
+    _check(st, "tg_gemm_nvf4_grouped")
     return out

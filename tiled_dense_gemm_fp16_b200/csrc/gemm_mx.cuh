@@ -1,4 +1,5 @@
-// gemm_mx.cuh -- MXFP8 block-scaled grouped GEMM on sm_100a tensor cores.
+// gemm_mx.cuh -- block-scaled grouped GEMMs (MXFP8 and NVF4) on sm_100a
+// tensor cores.
 //
 // The Blackwell MXFP8 grouped GEMM with block scaling and a transposed B
 // ("Key Technical Milestones", zhichai.net TileLang topic page), with the
@@ -24,6 +25,14 @@
 // buffered (256 of 512 TMEM columns; the scale factors use 12 more): the
 // epilogue drains it into registers, frees it, then stores, so the next
 // tile's MMAs overlap the stores.
+//
+// The NVF4 variant (the NVF4 block-scaled MMA path of the tilelang-ai project
+// page, "Three backends under one language dialect", read as NVIDIA's NVFP4)
+// runs the same pipeline with kind::mxf4nvf4: E2M1 elements packed two per
+// byte, so a 128-byte k-stage holds 256 elements; one UE4M3 scale per 16
+// elements, so each K = 64 MMA reads a whole 4-byte scale word per row and a
+// stage carries four 512-byte atoms per 128 rows; an fp32 alpha multiplies
+// the accumulator in the epilogue.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -34,13 +43,17 @@ namespace tg {
 
 constexpr int kMxMaxGroups = 256;
 
+enum { kKindMxf8 = 0, kKindNvf4 = 1 };
+
 struct MxParams {
-  const uint8_t* SFA;  // blocked UE8M0 scales of A's stacked rows
-  const uint8_t* SFB;  // blocked UE8M0 scales of B's rows, groups padded to 128 rows
+  const uint8_t* SFA;  // blocked scales of A's stacked rows
+  const uint8_t* SFB;  // blocked scales of B's rows, groups padded to 128 rows
   __nv_bfloat16* C;    // stacked rows x N
   int N, K;
-  int k_stages;        // ceil(K / 128): also the number of 512-byte atoms per 128 rows along K
-  int k_blocks;        // K / 32: scale blocks (one MMA each)
+  int k_stages;        // k-stages of 128 bytes per row
+  int k_mmas;          // MMAs along K: K / 32 (MXFP8) or K / 64 (NVF4)
+  int atoms_k;         // 512-byte scale atoms per 128 rows along K
+  float alpha;         // multiplies the accumulator (1 for MXFP8)
   int n_tiles, m_tiles, num_tiles, group_m;
   int groups;
   int n_atoms;         // ceil(N / 128): 128-row scale atoms per group of B
@@ -51,22 +64,24 @@ struct MxParams {
   int m_size[kMxMaxGroups];          // rows of each group
 };
 
+template <int KIND>
 struct MxCfg {
   static constexpr int BM = 128;
   static constexpr int BN = 256;
-  static constexpr int BK = 128;  // fp8 elements (= bytes) per k-stage
+  static constexpr int BK = 128;  // bytes of a row per k-stage: 128 fp8 or 256 fp4 elements
   static constexpr int STAGES = 4;
+  static constexpr int ATOMS = KIND == kKindNvf4 ? 4 : 1;  // scale atoms per 128 rows per stage
   static constexpr int MMA_WARP = 1;
   static constexpr int EPI_WARP0 = 2;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
   static constexpr int A_BYTES = BM * BK;   // 16 KiB
   static constexpr int B_BYTES = BN * BK;   // 32 KiB
-  static constexpr int SFA_BYTES = 512;
-  static constexpr int SFB_BYTES = 1024;
+  static constexpr int SFA_BYTES = 512 * ATOMS;
+  static constexpr int SFB_BYTES = 1024 * ATOMS;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SFA_COL = 256;       // 4 columns
-  static constexpr int SFB_COL = 264;       // 8 columns
+  static constexpr int SFA_COL = 256;       // 4 columns per atom
+  static constexpr int SFB_COL = 288;       // 8 columns per atom pair (two 128-row bands)
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + BAR_BYTES;
   static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // 128 columns per epilogue warp
@@ -104,10 +119,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float x0, float x1, bool relu) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(MxCfg::THREADS, 1)
-    gemm_mxf8_grouped_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                             const __grid_constant__ MxParams p) {
-  using Cfg = MxCfg;
+template <int KIND>
+__global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
+    gemm_blockscaled_grouped_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                                    const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ MxParams p) {
+  using Cfg = MxCfg<KIND>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_smem = smem;
@@ -170,26 +186,29 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
         const int g = mx_group_of(p, m_blk);
         const int n0 = n_blk * Cfg::BN;
         const int b_row0 = g * p.N + n0;
-        const int atom_b = g * p.n_atoms + n0 / 128;
+        const int band_b = g * p.n_atoms + n0 / 128;  // first 128-row scale band of this B tile
         const bool second_b = n0 / 128 + 1 < p.n_atoms;
-        const uint32_t bytes =
-            Cfg::A_BYTES + Cfg::B_BYTES + Cfg::SFA_BYTES + (second_b ? 2 : 1) * (Cfg::SFB_BYTES / 2);
         for (int ks = 0; ks < p.k_stages; ++ks) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 41)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full_bar[stage], bytes);
+          const int atom0 = ks * Cfg::ATOMS;
+          const int natoms = min(Cfg::ATOMS, p.atoms_k - atom0);
+          const uint32_t sf_bytes = static_cast<uint32_t>(natoms) * 512u * (second_b ? 3u : 2u);
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::A_BYTES + Cfg::B_BYTES + sf_bytes);
           const int k0 = ks * Cfg::BK;
           tma_load_2d(a_smem + stage * Cfg::A_BYTES, &tmap_a, &full_bar[stage], k0, m_blk * Cfg::BM);
           tma_load_2d_hint(b_smem + stage * Cfg::B_BYTES, &tmap_b, &full_bar[stage], k0, b_row0, pol_b);
+          // A stage's atoms of one 128-row band are contiguous in the blocked layout.
+          const uint32_t span = static_cast<uint32_t>(natoms) * 512u;
           bulk_load_g2s(sfa_smem + stage * Cfg::SFA_BYTES,
-                        p.SFA + (static_cast<int64_t>(m_blk) * p.k_stages + ks) * 512, 512, &full_bar[stage]);
+                        p.SFA + (static_cast<int64_t>(m_blk) * p.atoms_k + atom0) * 512, span, &full_bar[stage]);
           bulk_load_g2s(sfb_smem + stage * Cfg::SFB_BYTES,
-                        p.SFB + (static_cast<int64_t>(atom_b) * p.k_stages + ks) * 512, 512, &full_bar[stage]);
+                        p.SFB + (static_cast<int64_t>(band_b) * p.atoms_k + atom0) * 512, span, &full_bar[stage]);
           if (second_b)
-            bulk_load_g2s(sfb_smem + stage * Cfg::SFB_BYTES + 512,
-                          p.SFB + (static_cast<int64_t>(atom_b + 1) * p.k_stages + ks) * 512, 512,
+            bulk_load_g2s(sfb_smem + stage * Cfg::SFB_BYTES + Cfg::SFB_BYTES / 2,
+                          p.SFB + (static_cast<int64_t>(band_b + 1) * p.atoms_k + atom0) * 512, span,
                           &full_bar[stage]);
           last_parity[stage] = static_cast<int>(phase);
           if (++stage == Cfg::STAGES) {
@@ -231,21 +250,34 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
           const uint32_t sb = smem_u32(sfb_smem + stage * Cfg::SFB_BYTES);
           // Copies and MMAs issued by this thread run in issue order, so the
           // previous stage's MMAs read their scales before these overwrite them.
-          tmem_cp_32x128b_warpx4(sfa_tmem, make_plain_desc(sa, 16, 128));
-          tmem_cp_32x128b_warpx4(sfb_tmem, make_plain_desc(sb, 16, 128));
-          tmem_cp_32x128b_warpx4(sfb_tmem + 4, make_plain_desc(sb + 512, 16, 128));
+          const int natoms = min(Cfg::ATOMS, p.atoms_k - ks * Cfg::ATOMS);
+#pragma unroll
+          for (int a = 0; a < Cfg::ATOMS; ++a) {
+            if (a < natoms) {
+              tmem_cp_32x128b_warpx4(sfa_tmem + 4 * a, make_plain_desc(sa + 512 * a, 16, 128));
+              tmem_cp_32x128b_warpx4(sfb_tmem + 8 * a, make_plain_desc(sb + 512 * a, 16, 128));
+              tmem_cp_32x128b_warpx4(sfb_tmem + 8 * a + 4, make_plain_desc(sb + Cfg::SFB_BYTES / 2 + 512 * a, 16, 128));
+            }
+          }
           const uint32_t a_addr = smem_u32(a_smem + stage * Cfg::A_BYTES);
           const uint32_t b_addr = smem_u32(b_smem + stage * Cfg::B_BYTES);
-          const int nk = min(4, p.k_blocks - ks * 4);
+          const int nk = min(4, p.k_mmas - ks * 4);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             if (k < nk) {
+              // Each MMA consumes 32 bytes of every row (32 fp8 or 64 fp4 elements).
               const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
               const uint64_t bdesc = make_sw128_desc(b_addr + k * 32, 16, 1024);
-              const uint32_t idesc = p.idesc | (static_cast<uint32_t>(k) << 29) | (static_cast<uint32_t>(k) << 4);
-              const uint32_t byte_sel = static_cast<uint32_t>(k) << 30;
-              umma_mxf8_ss(tmem_base, adesc, bdesc, idesc, sfa_tmem | byte_sel, sfb_tmem | byte_sel,
-                           (ks | k) != 0 ? 1u : 0u);
+              const uint32_t accumulate = (ks | k) != 0 ? 1u : 0u;
+              if (KIND == kKindMxf8) {
+                // One scale per 32 elements: MMA k reads byte k of the stage's atom.
+                const uint32_t sel = static_cast<uint32_t>(k);
+                umma_mxf8_ss(tmem_base, adesc, bdesc, p.idesc | (sel << 29) | (sel << 4), sfa_tmem | (sel << 30),
+                             sfb_tmem | (sel << 30), accumulate);
+              } else {
+                // Four scales per 64 elements: MMA k reads the whole words of atom k.
+                umma_nvf4_ss(tmem_base, adesc, bdesc, p.idesc, sfa_tmem + 4 * k, sfb_tmem + 8 * k, accumulate);
+              }
             }
           }
           umma_commit(&empty_bar[stage]);
@@ -270,7 +302,8 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
     const int quad = warp & 3;               // TMEM lanes 32*quad .. +31
     const int half = e >> 2;                 // column half of the tile
     const bool relu = p.relu != 0;
-    const bool have_k = p.k_blocks > 0;
+    const bool have_k = p.k_mmas > 0;
+    const float alpha = p.alpha;
     int local = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
       int m_blk, n_blk;
@@ -288,7 +321,9 @@ __global__ void __launch_bounds__(MxCfg::THREADS, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          h[c * 8 + q] = have_k ? pack_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]), relu) : 0u;
+          h[c * 8 + q] = have_k ? pack_bf16x2(alpha * __uint_as_float(r[2 * q]),
+                                              alpha * __uint_as_float(r[2 * q + 1]), relu)
+                                : 0u;
       }
       tcgen05_fence_before_sync();
       __syncwarp();

@@ -449,6 +449,26 @@ __device__ __forceinline__ void umma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, u
       : "memory");
 }
 
+// D[tmem] (+)= (A * SFA) . (B * SFB)^T with packed E2M1 A/B and one UE4M3
+// scale per 16 elements: each K = 64 MMA reads four scale bytes (one 32-bit
+// TMEM word) per row.
+__device__ __forceinline__ void umma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor for kind::mxf4nvf4 with E2M1 A/B (format 1), fp32 D
+// and UE4M3 scales (bit 23 = 0), K-major operands, K = 64.
+__host__ __device__ constexpr uint32_t make_idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Instruction descriptor for kind::mxf8f6f4 with fp32 D and UE8M0 scales:
 //   bits 4-5 B scale-factor byte; bits 7-9 / 10-12 A / B format (0 = E4M3,
 //   1 = E5M2); bits 15 / 16 A / B major-ness (0 = K-major); bits 17-22 N >> 3;

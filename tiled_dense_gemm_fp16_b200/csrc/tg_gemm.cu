@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include <climits>
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -44,7 +45,7 @@ struct DeviceInfo {
   bool tc_edge_attr = false;
   bool skinny_attr = false;
   unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
-  bool mx_attr = false;
+  bool mx_attr[2] = {false, false};  // per block-scaled kind
   void* static_ws = nullptr;  // device address of g_static_workspace on this device
 };
 
@@ -771,23 +772,33 @@ bool encode_2d_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
   return r == CUDA_SUCCESS;
 }
 
-tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
-                           const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, int32_t a_format,
-                           int32_t b_format, int32_t relu, void* stream) {
+// Bytes of a blocked scale array for `rows` rows and `scales` scale columns.
+int64_t blocked_scale_bytes(int64_t rows, int64_t scales) { return round_up(rows, 128) * round_up(scales, 4); }
+
+// Shared launcher of the block-scaled grouped kernels.  elem_bits: 8 (MXFP8)
+// or 4 (NVF4); block: elements per scale (32 or 16).
+template <int KIND>
+tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
+                                  const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, uint32_t idesc,
+                                  float alpha, int32_t relu, void* stream) {
+  using Cfg = MxCfg<KIND>;
+  constexpr int kBlock = KIND == kKindNvf4 ? 16 : 32;
+  constexpr int kMmaK = KIND == kKindNvf4 ? 64 : 32;
+  constexpr int kElemsPerByte = KIND == kKindNvf4 ? 2 : 1;
   const int64_t rows = mx_rows(m_sizes, groups);
-  if (rows < 0 || N < 0 || K < 0 || K % 32 != 0 || N % 8 != 0 || K > INT_MAX) return TG_ERR_INVALID_ARG;
-  if ((a_format != TG_FP8_E4M3 && a_format != TG_FP8_E5M2) || (b_format != TG_FP8_E4M3 && b_format != TG_FP8_E5M2) ||
-      (relu != 0 && relu != 1))
+  if (rows < 0 || N < 0 || K < 0 || K % kMmaK != 0 || N % 8 != 0 || K > INT_MAX || (relu != 0 && relu != 1))
     return TG_ERR_INVALID_ARG;
   if (static_cast<int64_t>(groups) * N > INT_MAX - 256) return TG_ERR_INVALID_ARG;
   if (rows == 0 || N == 0) return TG_OK;
   if (C == nullptr || !aligned16(C)) return TG_ERR_INVALID_ARG;
   const int64_t c_bytes = rows * N * 2;
+  const int64_t row_bytes = K / kElemsPerByte;
   if (K > 0) {
     if (!A || !B || !SFA || !SFB || !aligned16(A) || !aligned16(B) || !aligned16(SFA) || !aligned16(SFB))
       return TG_ERR_INVALID_ARG;
-    const int64_t a_bytes = rows * K, b_bytes = static_cast<int64_t>(groups) * N * K;
-    const int64_t sfa_bytes = mx_scale_bytes(rows, K), sfb_bytes = groups * mx_scale_bytes(N, K);
+    const int64_t a_bytes = rows * row_bytes, b_bytes = static_cast<int64_t>(groups) * N * row_bytes;
+    const int64_t sfa_bytes = blocked_scale_bytes(rows, K / kBlock);
+    const int64_t sfb_bytes = groups * blocked_scale_bytes(N, K / kBlock);
     if (ranges_overlap(C, c_bytes, A, a_bytes) || ranges_overlap(C, c_bytes, B, b_bytes) ||
         ranges_overlap(C, c_bytes, SFA, sfa_bytes) || ranges_overlap(C, c_bytes, SFB, sfb_bytes))
       return TG_ERR_INVALID_ARG;
@@ -796,16 +807,16 @@ tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const 
   DeviceInfo* info = nullptr;
   tg_status st = current_device(dev, info);
   if (st != TG_OK) return st;
-  using Cfg = MxCfg;
+  auto kernel = gemm_blockscaled_grouped_kernel<KIND>;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!info->mx_attr) {
-      if (cudaFuncSetAttribute(gemm_mxf8_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg::SMEM_BYTES) != cudaSuccess) {
+    if (!info->mx_attr[KIND]) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
+          cudaSuccess) {
         cudaGetLastError();
         return TG_ERR_LAUNCH;
       }
-      info->mx_attr = true;
+      info->mx_attr[KIND] = true;
     }
   }
   CUtensorMap ta, tb;
@@ -814,16 +825,18 @@ tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const 
   MxParams p;
   std::memset(&p, 0, sizeof p);
   if (K > 0) {
-    if (!encode_2d_u8(&ta, A, rows, K, Cfg::BK, Cfg::BM)) return TG_ERR_LAUNCH;
-    if (!encode_2d_u8(&tb, B, static_cast<int64_t>(groups) * N, K, Cfg::BK, Cfg::BN)) return TG_ERR_LAUNCH;
+    if (!encode_2d_u8(&ta, A, rows, row_bytes, Cfg::BK, Cfg::BM)) return TG_ERR_LAUNCH;
+    if (!encode_2d_u8(&tb, B, static_cast<int64_t>(groups) * N, row_bytes, Cfg::BK, Cfg::BN)) return TG_ERR_LAUNCH;
   }
   p.SFA = static_cast<const uint8_t*>(SFA);
   p.SFB = static_cast<const uint8_t*>(SFB);
   p.C = static_cast<__nv_bfloat16*>(C);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.k_stages = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
-  p.k_blocks = static_cast<int>(K / 32);
+  p.k_stages = static_cast<int>((row_bytes + Cfg::BK - 1) / Cfg::BK);
+  p.k_mmas = static_cast<int>(K / kMmaK);
+  p.atoms_k = static_cast<int>(round_up(K / kBlock, 4) / 4);
+  p.alpha = alpha;
   p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
   p.m_tiles = static_cast<int>(rows / Cfg::BM);
   p.num_tiles = p.m_tiles * p.n_tiles;
@@ -832,7 +845,7 @@ tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const 
   p.groups = groups;
   p.n_atoms = static_cast<int>((N + 127) / 128);
   p.relu = relu;
-  p.idesc = make_idesc_mxf8(Cfg::BM, Cfg::BN, a_format, b_format, 0, 0);
+  p.idesc = idesc;
   p.wait_budget_ns = wait_budget(p.k_stages * 2);
   int tile = 0;
   for (int32_t g = 0; g < groups; ++g) {
@@ -850,11 +863,28 @@ tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const 
   cfg.stream = static_cast<cudaStream_t>(stream);
   LaunchAttrs la;
   la.fill(cfg, 1);
-  if (cudaLaunchKernelEx(&cfg, gemm_mxf8_grouped_kernel, ta, tb, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
     cudaGetLastError();
     return TG_ERR_LAUNCH;
   }
   return TG_OK;
+}
+
+tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
+                           const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, int32_t a_format,
+                           int32_t b_format, int32_t relu, void* stream) {
+  if ((a_format != TG_FP8_E4M3 && a_format != TG_FP8_E5M2) || (b_format != TG_FP8_E4M3 && b_format != TG_FP8_E5M2))
+    return TG_ERR_INVALID_ARG;
+  return run_blockscaled_grouped<kKindMxf8>(A, SFA, B, SFB, C, m_sizes, groups, N, K,
+                                            make_idesc_mxf8(128, 256, a_format, b_format, 0, 0), 1.0f, relu, stream);
+}
+
+tg_status run_nvf4_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
+                           const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, float alpha, int32_t relu,
+                           void* stream) {
+  if (!std::isfinite(alpha)) return TG_ERR_INVALID_ARG;
+  return run_blockscaled_grouped<kKindNvf4>(A, SFA, B, SFB, C, m_sizes, groups, N, K, make_idesc_nvf4(128, 256),
+                                            alpha, relu, stream);
 }
 
 }  // namespace
@@ -873,6 +903,17 @@ int64_t tg_mx_grouped_rows(const int64_t* m_sizes, int32_t groups) { return tg::
 int64_t tg_mx_scale_bytes(int64_t rows, int64_t K) {
   if (rows < 0 || K < 0 || K % 32 != 0) return -1;
   return tg::mx_scale_bytes(rows, K);
+}
+
+tg_status tg_gemm_nvf4_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
+                               const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, float alpha,
+                               int32_t relu, void* stream) {
+  return tg::run_nvf4_grouped(A, SFA, B, SFB, C, m_sizes, groups, N, K, alpha, relu, stream);
+}
+
+int64_t tg_nvf4_scale_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K < 0 || K % 16 != 0) return -1;
+  return tg::blocked_scale_bytes(rows, K / 16);
 }
 
 tg_status tg_gemm_relu_f16(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* stream) {

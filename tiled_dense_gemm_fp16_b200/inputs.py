@@ -105,6 +105,44 @@ def mx_operands(m_sizes, N: int, K: int, seed: int, dist: str = "normal", a_form
     return A, SFA, B, SFB
 
 
+# E2M1 codes of the integers -4..4 that the format holds (0, +-1, +-2, +-3, +-4).
+_E2M1_INT_CODES = np.array([0xE, 0xD, 0xC, 0xA, 0x0, 0x2, 0x4, 0x5, 0x6], np.uint8)
+
+
+def pack_fp4(codes: np.ndarray) -> np.ndarray:
+    """4-bit codes (..., K) -> bytes (..., K/2), element 2i in the low nibble."""
+    codes = np.asarray(codes, np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def nvf4_operands(m_sizes, N: int, K: int, seed: int, dist: str = "codes", scale_lo: int = 0x28,
+                  scale_hi: int = 0x49):
+    """Grouped NVF4 operands: packed A (stacked rows x K/2), plain scales SFA (rows x K/16), packed B
+    (G x N x K/2) and SFB (G x N x K/16), drawn in that order from ``default_rng(seed)``.
+
+    ``dist``: "int" draws the E2M1 integers -4..4 with unit scales (UE4M3 code 0x38 = 1.0);
+    "codes" draws every E2M1 code uniformly and scale codes uniform in [scale_lo, scale_hi)
+    (0x28..0x48: 2^-2 .. 2^2 with all mantissas).
+    """
+    rng = np.random.default_rng(seed)
+    G = len(m_sizes)
+    _, rows = mx_group_offsets(m_sizes)
+    S = K // 16
+    if dist == "int":
+        A = _E2M1_INT_CODES[rng.integers(0, 9, size=(rows, K))]
+        SFA = np.full((rows, S), 0x38, np.uint8)
+        B = _E2M1_INT_CODES[rng.integers(0, 9, size=(G, N, K))]
+        SFB = np.full((G, N, S), 0x38, np.uint8)
+    elif dist == "codes":
+        A = rng.integers(0, 16, size=(rows, K)).astype(np.uint8)
+        SFA = rng.integers(scale_lo, scale_hi, size=(rows, S)).astype(np.uint8)
+        B = rng.integers(0, 16, size=(G, N, K)).astype(np.uint8)
+        SFB = rng.integers(scale_lo, scale_hi, size=(G, N, S)).astype(np.uint8)
+    else:
+        raise ValueError(f"unknown distribution {dist!r}")
+    return pack_fp4(A), SFA, pack_fp4(B), SFB
+
+
 def mx_scales_blocked(sf: np.ndarray) -> np.ndarray:
     """Plain row-major scales (R x S) rearranged into the C ABI's 128 x 4 blocked byte layout:
     scale (r, s) goes to ((r//128)*(S'/4) + s//4)*512 + (r%32)*16 + ((r//32)%4)*4 + s%4, with
@@ -160,6 +198,12 @@ WORKLOADS = {
 MX_WORKLOADS = {
     "mxf8_moe": ((2304, 1792, 2048, 2560, 1536, 2048, 2176, 1920), 4096, 7168, 6),
     "mxf8_8192": ((8192,), 8192, 8192, 7),
+}
+
+# NVF4 workloads: the 8192^3 problem the NVF4 path is quoted on, and the MoE layer shape.
+NVF4_WORKLOADS = {
+    "nvf4_8192": ((8192,), 8192, 8192, 8),
+    "nvf4_moe": ((2304, 1792, 2048, 2560, 1536, 2048, 2176, 1920), 4096, 7168, 9),
 }
 
 
