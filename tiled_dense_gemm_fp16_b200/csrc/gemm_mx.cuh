@@ -14,15 +14,21 @@
 //   warp 0      TMA producer: A box 128 x 128 B, B box 256 x 128 B, plus the
 //               stage's scale factors (512 B for A's 128 rows, 2 x 512 B for
 //               B's 256 rows) with untiled bulk copies;
-//   warp 1      TMEM owner and MMA issuer: per stage, tcgen05.cp moves the
-//               scale factors into TMEM, then four K = 32 MMAs of
-//               kind::mxf8f6f4 with block_scale each read one scale byte;
-//   warps 2-9   epilogue: two warps per TMEM lane quarter, 128 columns each.
+//   warp 1      TMEM owner and MMA issuer: per stage, four K = 32 MMAs of
+//               kind::mxf8f6f4 with block_scale, each reading one scale byte;
+//   warps 2-5   scale stagers, one per TMEM lane quarter: per stage they read
+//               the scale atoms from shared memory and write them into that
+//               stage's TMEM scale buffer with tcgen05.st, every quarter
+//               holding the same 32 lines (the layout the MMA reads);
+//   warps 6-13  epilogue: two warps per TMEM lane quarter, 128 columns each.
+// Staging the scales with tcgen05.st keeps them off the tensor pipe, where
+// tcgen05.cp copies would run in order with the MMAs.
 // Scale factors are stored in the 128 x 4 blocked layout that the tensor
 // core reads (512-byte atoms: 32 lines of 16 bytes, line l holding rows
 // l, l+32, l+64, l+96 with four consecutive k-blocks each), so a stage's
 // scales are a contiguous 512 bytes per 128 rows.  The accumulator is single-
-// buffered (256 of 512 TMEM columns; the scale factors use 12 more): the
+// buffered (256 of 512 TMEM columns; the scale factors use one small buffer
+// per pipeline stage in the rest): the
 // epilogue drains it into registers, frees it, then stores, so the next
 // tile's MMAs overlap the stores.
 //
@@ -72,7 +78,9 @@ struct MxCfg {
   static constexpr int STAGES = 4;
   static constexpr int ATOMS = KIND == kKindNvf4 ? 4 : 1;  // scale atoms per 128 rows per stage
   static constexpr int MMA_WARP = 1;
-  static constexpr int EPI_WARP0 = 2;
+  static constexpr int SF_WARP0 = 2;
+  static constexpr int SF_WARPS = 4;
+  static constexpr int EPI_WARP0 = SF_WARP0 + SF_WARPS;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
   static constexpr int A_BYTES = BM * BK;   // 16 KiB
@@ -80,11 +88,17 @@ struct MxCfg {
   static constexpr int SFA_BYTES = 512 * ATOMS;
   static constexpr int SFB_BYTES = 1024 * ATOMS;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SFA_COL = 256;       // 4 columns per atom
-  static constexpr int SFB_COL = 288;       // 8 columns per atom pair (two 128-row bands)
-  static constexpr int BAR_BYTES = 256;
+  // Scale factors in TMEM, one buffer per pipeline stage so that a stage's
+  // copies do not overwrite scales that earlier MMAs may still be reading:
+  // per stage 4 columns of A scales and 8 of B scales per atom.
+  static constexpr int SF_COL0 = 256;
+  static constexpr int SF_STAGE_COLS = 12 * ATOMS <= 16 ? 16 : 12 * ATOMS;
+  static constexpr int SFB_OFF = 4 * ATOMS;
+  static constexpr int BAR_BYTES = 256;  // 3 x STAGES + 3 barriers, the TMEM slot and the abort flag
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + BAR_BYTES;
   static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // 128 columns per epilogue warp
+  static_assert(SF_COL0 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "scale buffers exceed the TMEM allocation");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA exceeded");
 };
 
 __device__ __forceinline__ void mx_tile_coords(const MxParams& p, int t, int& m_blk, int& n_blk) {
@@ -133,7 +147,8 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sfb_smem + Cfg::STAGES * Cfg::SFB_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + Cfg::STAGES;
-  uint64_t* acc_full_bar = bars + 2 * Cfg::STAGES;
+  uint64_t* sf_full_bar = bars + 2 * Cfg::STAGES;
+  uint64_t* acc_full_bar = bars + 3 * Cfg::STAGES;
   uint64_t* acc_empty_bar = acc_full_bar + 1;
   uint64_t* mma_done_bar = acc_empty_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done_bar + 1);
@@ -146,6 +161,7 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
     for (int s = 0; s < Cfg::STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&sf_full_bar[s], Cfg::SF_WARPS);
     }
     mbar_init(acc_full_bar, 1);
     mbar_init(acc_empty_bar, Cfg::EPI_WARPS);
@@ -235,8 +251,6 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      const uint32_t sfa_tmem = tmem_base + Cfg::SFA_COL;
-      const uint32_t sfb_tmem = tmem_base + Cfg::SFB_COL;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
         if (!mbar_wait(acc_empty_bar, (local & 1) ^ 1u, abort_flag, p.wait_budget_ns, 43)) break;
         tcgen05_fence_after_sync();
@@ -245,20 +259,13 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
             ok = false;
             break;
           }
-          tcgen05_fence_after_sync();
-          const uint32_t sa = smem_u32(sfa_smem + stage * Cfg::SFA_BYTES);
-          const uint32_t sb = smem_u32(sfb_smem + stage * Cfg::SFB_BYTES);
-          // Copies and MMAs issued by this thread run in issue order, so the
-          // previous stage's MMAs read their scales before these overwrite them.
-          const int natoms = min(Cfg::ATOMS, p.atoms_k - ks * Cfg::ATOMS);
-#pragma unroll
-          for (int a = 0; a < Cfg::ATOMS; ++a) {
-            if (a < natoms) {
-              tmem_cp_32x128b_warpx4(sfa_tmem + 4 * a, make_plain_desc(sa + 512 * a, 16, 128));
-              tmem_cp_32x128b_warpx4(sfb_tmem + 8 * a, make_plain_desc(sb + 512 * a, 16, 128));
-              tmem_cp_32x128b_warpx4(sfb_tmem + 8 * a + 4, make_plain_desc(sb + Cfg::SFB_BYTES / 2 + 512 * a, 16, 128));
-            }
+          if (!mbar_wait(&sf_full_bar[stage], phase, abort_flag, p.wait_budget_ns, 47)) {
+            ok = false;
+            break;
           }
+          tcgen05_fence_after_sync();
+          const uint32_t sfa_tmem = tmem_base + Cfg::SF_COL0 + stage * Cfg::SF_STAGE_COLS;
+          const uint32_t sfb_tmem = sfa_tmem + Cfg::SFB_OFF;
           const uint32_t a_addr = smem_u32(a_smem + stage * Cfg::A_BYTES);
           const uint32_t b_addr = smem_u32(b_smem + stage * Cfg::B_BYTES);
           const int nk = min(4, p.k_mmas - ks * 4);
@@ -294,6 +301,48 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
       mbar_wait(mma_done_bar, 0, &no_abort, p.wait_budget_ns, 45);
     }
     __syncwarp();
+  } else if (warp < Cfg::EPI_WARP0) {
+    // ------------------------------------------------------------------
+    // Scale stagers: shared memory -> this warp's TMEM lane quarter
+    // ------------------------------------------------------------------
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int ks = 0; ks < p.k_stages; ++ks) {
+        const bool ready = mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 48);
+        if (!__all_sync(0xffffffffu, ready)) {
+          ok = false;
+          break;
+        }
+        const int natoms = min(Cfg::ATOMS, p.atoms_k - ks * Cfg::ATOMS);
+        const uint32_t sfa_tmem = tmem_base + lane_base + Cfg::SF_COL0 + stage * Cfg::SF_STAGE_COLS;
+        const uint32_t sfb_tmem = sfa_tmem + Cfg::SFB_OFF;
+        const uint4* sa = reinterpret_cast<const uint4*>(sfa_smem + stage * Cfg::SFA_BYTES) + lane;
+        const uint4* sb = reinterpret_cast<const uint4*>(sfb_smem + stage * Cfg::SFB_BYTES) + lane;
+#pragma unroll
+        for (int a = 0; a < Cfg::ATOMS; ++a) {
+          if (a < natoms) {
+            // Line `lane` of each 512-byte atom: 16 bytes = 4 TMEM columns.
+            const uint4 va = sa[a * 32];
+            const uint4 vb0 = sb[a * 32];
+            const uint4 vb1 = sb[Cfg::SFB_BYTES / 32 + a * 32];
+            tmem_st_32x32b_x4(sfa_tmem + 4 * a, va);
+            tmem_st_32x32b_x4(sfb_tmem + 8 * a, vb0);
+            tmem_st_32x32b_x4(sfb_tmem + 8 * a + 4, vb1);
+          }
+        }
+        tmem_st_wait();
+        tcgen05_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full_bar[stage]);
+        if (++stage == Cfg::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------------
     // Epilogue: TMEM -> registers (ReLU, bf16) -> free the accumulator -> C

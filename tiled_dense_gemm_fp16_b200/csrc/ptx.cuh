@@ -419,23 +419,16 @@ __device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gmem_s
       : "memory");
 }
 
-// Shared-memory descriptor of an unswizzled (interleaved) K-major operand:
-// core matrices of 8 rows x 16 bytes, `sbo_bytes` apart along the rows.
-__device__ __forceinline__ uint64_t make_plain_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  return d;  // layout bits 61-63 = 0: no swizzle
+// Warp-collective: lane i writes 4 consecutive 32-bit TMEM columns of TMEM
+// lane (taddr.lane + i); the warp may only address its own 32-lane quarter.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint4& v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
-// Copy 32 rows x 16 bytes of shared memory (descriptor `sdesc`) into TMEM
-// lanes 0-31 of columns taddr .. taddr+3, replicated into all four 32-lane
-// quarters.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
+// Wait until this thread's tcgen05.st writes have completed.
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // D[tmem] (+)= (A * SFA) . (B * SFB)^T with fp8 A/B and UE8M0 block scales in
 // TMEM; the scale-factor byte used is selected by the descriptor's sf ids.
