@@ -95,6 +95,8 @@ def _bind(lib):
     lib.oracle_gemm_nvf4_grouped.argtypes = [u8p, u8p, u8p, u8p, u16p, i64p, i64p, ctypes.c_int, i64, i64,
                                              ctypes.c_double, ctypes.c_int, ctypes.c_int]
     lib.oracle_gemm_nvf4_grouped.restype = ctypes.c_int
+    lib.oracle_dequant_w4_f16.argtypes = [u8p, u16p, u16p, i64, i64, i64]
+    lib.oracle_dequant_w4_f16.restype = ctypes.c_int
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
@@ -288,6 +290,31 @@ def gemm_nvf4_grouped(A, SFA, B, SFB, m_sizes, row_offsets, N: int, K: int, alph
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return C.reshape(rows, N) if N else C
+
+
+def dequant_w4_f16(Wq, S, N: int, K: int, group: int, lib=None) -> np.ndarray:
+    """The N x K fp16 weight (float16 array) of 4-bit codes Wq (N x K/2 bytes) and fp16 scales
+    S (N x K/group): f16_rne((q - 8) * s)."""
+    lib = lib or load_library()
+    Wq = np.ascontiguousarray(np.asarray(Wq, dtype=np.uint8))
+    S = _u16(np.asarray(S))
+    if Wq.size < N * (K // 2) or S.size < N * (K // group if group else 0):
+        raise ValueError("operand too small")
+    W = np.empty(N * K, np.uint16)
+    if lib.oracle_dequant_w4_f16(_ptr(Wq, ctypes.c_uint8), _ptr(S, ctypes.c_uint16), _ptr(W, ctypes.c_uint16),
+                                 N, K, group) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return W.view(np.float16).reshape(N, K)
+
+
+def gemm_relu_w4a16(A, Wq, S, group: int, nthreads: int = 0, lib=None) -> np.ndarray:
+    """C = f16_rne(relu(A . dequant(W)^T)) for fp16 A (M x K): the dequantized weight, then the
+    general-layout oracle with the weight stored N x K."""
+    A = np.asarray(A)
+    M, K = A.shape
+    N = np.asarray(Wq).shape[0]
+    W = dequant_w4_f16(Wq, S, N, K, group, lib=lib)
+    return gemm_relu_f16_ex(A, W, M, N, K, K, K, N, b_nk=True, nthreads=nthreads, lib=lib).reshape(M, N)
 
 
 def max_threads(lib=None) -> int:

@@ -488,6 +488,47 @@ int oracle_gemm_nvf4_grouped(const uint8_t *A, const uint8_t *SFA, const uint8_t
     return 0;
 }
 
+/* ------------------------------------------------------------------------
+ * Dequantized (low-bit weight) GEMM: the dequantize_gemm workload that the
+ * TileLang pages name among the kernels the language targets (aiwiki.ai
+ * "TileLang", opening paragraph; the BitBLAS dequantized-GEMM comparisons
+ * under "Ecosystem").  The pages name the operation only; the reading taken
+ * is the common 4-bit weight-only scheme (W4A16):
+ *   - the weight W is N x K, stored as 4-bit codes q in 0..15, two per byte,
+ *     element 2i of a row in the low nibble (as for NVF4 above);
+ *   - each run of `group` consecutive elements of a weight row along K shares
+ *     one fp16 scale s; the zero point is the fixed code 8, so a weight is
+ *     (q - 8) * s;
+ *   - the dequantized weight is rounded to fp16 (the type the fp16 GEMM
+ *     consumes): w = f16_rne((q - 8) * s), the exact product rounded once;
+ *   - the GEMM is then the base operation with the weight in the linear-layer
+ *     layout: C = ReLU(A . W^T), fp32 accumulation, fp16 output
+ *     (oracle_gemm_relu_f16_ex with b_nk = 1).
+ * ------------------------------------------------------------------------ */
+
+/*
+ * W[n*K + k] = f16_rne( (q(n,k) - 8) * f32(S[n*(K/group) + k/group]) ) for the
+ * N x K weight, with q(n,k) nibble k of row n of Wq (rows of K/2 bytes).  The
+ * product of an integer in -8..7 and an fp16 value is exact in fp32, so one
+ * rounding happens.  K must be a multiple of `group` and of 2.  Returns 0, or
+ * -1 on bad arguments.
+ */
+int oracle_dequant_w4_f16(const uint8_t *Wq, const uint16_t *S, uint16_t *W, int64_t N, int64_t K, int64_t group)
+{
+    if (N < 0 || K < 0 || group <= 0 || K % group != 0 || K % 2 != 0)
+        return -1;
+    const int64_t G = K / group;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            const uint8_t byte = Wq[n * (K / 2) + k / 2];
+            const int q = (k & 1) ? (byte >> 4) : (byte & 0xf);
+            const float scale = oracle_f16_to_f32(S[n * G + k / group]);
+            W[n * K + k] = oracle_f32_to_f16_rne((float)(q - 8) * scale);
+        }
+    }
+    return 0;
+}
+
 /* Number of threads OpenMP would use by default (1 without OpenMP). */
 int oracle_max_threads(void)
 {

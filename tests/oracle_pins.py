@@ -701,6 +701,59 @@ def check_nvf4_alpha_relu(lib):
     assert np.array_equal(relu, np.where(base > 0, base / 8, 0.0))
 
 
+# --------------------------------------------------------------------------
+# Dequantized (W4A16) GEMM
+# --------------------------------------------------------------------------
+
+def _pack4(codes):
+    codes = np.asarray(codes, np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def check_dequant_all_codes_all_scales(lib):
+    """Every code 0..15 against every finite fp16 scale: numpy's float32 product (exact) rounded by
+    numpy's float16 conversion (an independent implementation)."""
+    scales = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    scales = scales[np.isfinite(scales)]
+    N, K = scales.size, 16
+    codes = np.tile(np.arange(16, dtype=np.uint8), (N, 1))
+    S = scales.reshape(N, 1)
+    got = oracle.dequant_w4_f16(_pack4(codes), S, N, K, 16, lib=lib)
+    with np.errstate(over="ignore"):  # large scales times 8 overflow to inf, as they should
+        want = ((np.arange(16, dtype=np.float32) - 8)[None, :] * scales.astype(np.float32)[:, None]).astype(np.float16)
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+
+
+def check_dequant_groups_and_nibbles(lib):
+    """Hand-checkable structure: code k % 16 at column k, scale 2^g for group g, group size 32:
+    W[n, k] = (k % 16 - 8) * 2^(k // 32) exactly (small integers times powers of two)."""
+    N, K, group = 3, 128, 32
+    codes = np.tile(np.arange(K) % 16, (N, 1)).astype(np.uint8)
+    S = np.tile(np.array([1.0, 2.0, 4.0, 8.0], np.float16), (N, 1))
+    got = oracle.dequant_w4_f16(_pack4(codes), S, N, K, group, lib=lib).astype(np.float64)
+    k = np.arange(K)
+    want = np.tile((k % 16 - 8) * 2.0 ** (k // 32), (N, 1))
+    assert np.array_equal(got, want)
+    # Row-specific scales: row n uses its own scale row.
+    S2 = np.array([[1.0] * 4, [0.5] * 4, [-3.0] * 4], np.float16)
+    got2 = oracle.dequant_w4_f16(_pack4(codes), S2, N, K, group, lib=lib).astype(np.float64)
+    assert np.array_equal(got2, (k % 16 - 8)[None, :] * np.array([1.0, 0.5, -3.0])[:, None])
+
+
+def check_w4a16_gemm_integer_exact(lib):
+    """Unit scales make W the integers q - 8; with integer A the product is exact (int64 matmul)."""
+    import torch
+    rng = np.random.default_rng(31)
+    M, N, K, group = 7, 20, 256, 64
+    A = rng.integers(-2, 3, size=(M, K)).astype(np.float16)
+    codes = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    S = np.ones((N, K // group), np.float16)
+    got = oracle.gemm_relu_w4a16(A, _pack4(codes), S, group, lib=lib)
+    exact = np.maximum(A.astype(np.int64) @ (codes.astype(np.int64) - 8).T, 0).astype(np.float32)
+    want = torch.from_numpy(exact).to(torch.float16).numpy()
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+
+
 ALL_CHECKS = [
     check_f16_to_f32_all_patterns,
     check_f32_to_f16_golden,
@@ -737,4 +790,7 @@ ALL_CHECKS = [
     check_nvf4_identity_nibble_order,
     check_nvf4_exact_rational_tiny,
     check_nvf4_alpha_relu,
+    check_dequant_all_codes_all_scales,
+    check_dequant_groups_and_nibbles,
+    check_w4a16_gemm_integer_exact,
 ]

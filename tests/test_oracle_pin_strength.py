@@ -47,6 +47,11 @@ MUTANTS = [
     ("nvf4_scale_b_dropped", "oracle_ue4m3_to_f64(SFB[brow * S + k / 16])", "1.0"),
     ("nvf4_group_ignored", "const int64_t brow = (int64_t)g * N + j;\n                double acc = 0.0;\n                for (int64_t k = 0; k < K; ++k) {\n                    const int hi",
      "const int64_t brow = j;\n                double acc = 0.0;\n                for (int64_t k = 0; k < K; ++k) {\n                    const int hi"),
+    ("w4_zero_point_7", "(float)(q - 8) * scale", "(float)(q - 7) * scale"),
+    ("w4_nibbles_swapped", "const int q = (k & 1) ? (byte >> 4) : (byte & 0xf);",
+     "const int q = (k & 1) ? (byte & 0xf) : (byte >> 4);"),
+    ("w4_group_index", "S[n * G + k / group]", "S[n * G + k / (2 * group)]"),
+    ("w4_scale_row_ignored", "S[n * G + k / group]", "S[k / group]"),
     ("fp64_accumulator", "float *acc = (float *)malloc((size_t)N * sizeof(float));",
      "double *acc = (double *)malloc((size_t)N * sizeof(double));"),
 ]
