@@ -291,7 +291,7 @@ TG_API int tg_version(void);
  *      ((r/128) * (S'/4) + s/4) * 512 + (r%32) * 16 + ((r/32)%4) * 4 + s%4.
  *    SFA covers A's stacked rows; SFB holds G such arrays back to back, group
  *    g's for its N rows at offset g * tg_mx_scale_bytes(N, K).  Padding bytes
- *    are never used for a valid output.
+ *    never affect a stored output (any byte is a valid UE8M0 code).
  * C: stacked rows x N bf16, row-major; only the m_sizes[g] rows of each group
  *    are written.  relu = 1 maps every value that is not > 0 to +0.
  * The sum is accumulated in fp32 by the tensor core; the result is rounded to
@@ -331,6 +331,9 @@ TG_API int64_t tg_mx_scale_bytes(int64_t rows, int64_t K);
  * SFA, SFB: one UE4M3 scale (an FP8 E4M3 code with the sign bit clear) per 16
  *    elements along K, in the 128 x 4 blocked layout described above with
  *    S = K/16 scale columns; group g's SFB at g * tg_nvf4_scale_bytes(N, K).
+ *    Every byte of both arrays, padding included, must be a finite UE4M3
+ *    code (0x00 .. 0x7E): the tensor core reads the padding rows' scales too
+ *    (their outputs are discarded), and other codes are not valid scales.
  * alpha: a finite fp32 factor applied to the fp32 accumulator (the per-tensor
  *    scale of NVFP4).
  * C: stacked rows x N bf16; only the rows of the groups are written.

@@ -66,7 +66,9 @@ struct MxParams {
   int relu;
   uint32_t idesc;      // formats, shape and scale type; the sf bytes are or-ed in per MMA
   uint64_t wait_budget_ns;
+  int pair_tiles;      // 256-row pair tiles (pair kernel): ceil(tiles / 2) per group
   int tile_start[kMxMaxGroups + 1];  // first stacked 128-row tile of each group; [groups] = m_tiles
+  int pair_start[kMxMaxGroups + 1];  // first pair tile of each group; [groups] = pair_tiles
   int m_size[kMxMaxGroups];          // rows of each group
 };
 
@@ -310,6 +312,12 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      // The second 128-row band of B's scales is not loaded for a tile that
+      // ends within the first band: its columns are never stored, and zero
+      // scales stand in for the stale shared memory.
+      int m_blk, n_blk;
+      mx_tile_coords(p, t, m_blk, n_blk);
+      const bool second_b = n_blk * 2 + 1 < p.n_atoms;
       for (int ks = 0; ks < p.k_stages; ++ks) {
         const bool ready = mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 48);
         if (!__all_sync(0xffffffffu, ready)) {
@@ -327,7 +335,7 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
             // Line `lane` of each 512-byte atom: 16 bytes = 4 TMEM columns.
             const uint4 va = sa[a * 32];
             const uint4 vb0 = sb[a * 32];
-            const uint4 vb1 = sb[Cfg::SFB_BYTES / 32 + a * 32];
+            const uint4 vb1 = second_b ? sb[Cfg::SFB_BYTES / 32 + a * 32] : make_uint4(0, 0, 0, 0);
             tmem_st_32x32b_x4(sfa_tmem + 4 * a, va);
             tmem_st_32x32b_x4(sfb_tmem + 8 * a, vb0);
             tmem_st_32x32b_x4(sfb_tmem + 8 * a + 4, vb1);

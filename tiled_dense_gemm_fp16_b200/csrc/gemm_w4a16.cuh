@@ -1,0 +1,350 @@
+// gemm_w4a16.cuh -- 4-bit weight-only GEMM: C = ReLU(A . W^T) with fp16 A
+// (M x K), W (N x K) stored as 4-bit codes with one fp16 scale per group of
+// K elements, w = fp16((q - 8) * s); fp32 accumulation, fp16 C (M x N).
+//
+// The dequantize_gemm workload of the TileLang pages ("TileLang" wiki page,
+// opening paragraph), read as the common W4A16 scheme.  Two kernels:
+//   * dequant_w4_kernel: W -> fp16 (N x K) in HBM, bandwidth-bound; a large-M
+//     call dequantizes into the caller's workspace and then runs the fp16
+//     tensor-core GEMM with the weight in the N x K layout;
+//   * gemm_relu_w4a16_skinny_kernel: for M <= 256, one kernel that streams
+//     the packed weight once.  It is the small-M kernel's swap-AB split-K
+//     scheme (C^T = W . A^T, the weight's 128-row panel is the MMA's M side,
+//     a cluster of S CTAs splits K and reduces through distributed shared
+//     memory) with a dequantization stage in front of the MMA:
+//       - warp 0 loads, per 64-deep k-block, the panel's packed codes (128
+//         rows x 32 bytes) and the activations (m_pad rows x 64) into a deep
+//         ring;
+//       - warps 6-13 turn each packed tile into the fp16 tile the MMA reads
+//         (128-byte swizzled, K-major) in a small second ring: a nibble is
+//         placed in the mantissa of 1024.0 (exponent bits 0x6400), 1032 is
+//         subtracted (exact: q - 8), and the fp16 multiply by the group's
+//         scale rounds once to nearest even;
+//       - warp 1 issues 128 x m_pad x 16 MMAs; warps 2-5 move the fp32
+//         partial to shared memory for the cluster reduction.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace tg {
+
+// ---------------------------------------------------------------------------
+// Stand-alone dequantization
+// ---------------------------------------------------------------------------
+
+struct DequantParams {
+  const uint8_t* Wq;  // N x K/2 bytes
+  const __half* S;    // N x K/group scales
+  __half* W;          // N x K output
+  int64_t N, K;
+  int group;
+  int64_t chunks;     // N * K / 8: 8 codes (4 bytes) -> 8 fp16 (16 bytes) each
+};
+
+// Eight 4-bit codes (a 32-bit word, element 2i in the low nibble of byte i)
+// as eight fp16 values (q - 8) * s, packed two per word, low element first.
+__device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2) {
+  const uint32_t magic = 0x64006400u;  // fp16 1024.0 in both halves
+  const uint32_t p01 = (w & 0xFu) | ((w << 12) & 0xF0000u) | magic;
+  const uint32_t p23 = ((w >> 8) & 0xFu) | ((w << 4) & 0xF0000u) | magic;
+  const uint32_t p45 = ((w >> 16) & 0xFu) | ((w >> 4) & 0xF0000u) | magic;
+  const uint32_t p67 = ((w >> 24) & 0xFu) | ((w >> 12) & 0xF0000u) | magic;
+  const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
+  uint32_t out[4];
+  const uint32_t in[4] = {p01, p23, p45, p67};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&in[i]), bias);  // q - 8, exact
+    const __half2 r = __hmul2(v, s2);                                             // one RNE rounding
+    out[i] = *reinterpret_cast<const uint32_t*>(&r);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+__global__ void __launch_bounds__(256) dequant_w4_kernel(const DequantParams p) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const int64_t per_row = p.K / 8;
+  const int64_t groups_per_row = p.K / p.group;
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < p.chunks;
+       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = c / per_row;
+    const int64_t k = (c - n * per_row) * 8;
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.Wq + n * (p.K / 2) + k / 2));
+    const __half s = p.S[n * groups_per_row + k / p.group];
+    reinterpret_cast<uint4*>(p.W + n * p.K)[k / 8] = dequant8(w, __halves2half2(s, s));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused small-M kernel
+// ---------------------------------------------------------------------------
+
+struct W4Params {
+  __half* C;
+  const __half* S;        // N x K/group scales
+  int M, N, K;
+  int group;
+  int m_pad;              // MMA N: M rounded up to a multiple of 16 (16..256)
+  int k_blocks;           // K / 64
+  int splits;             // CTAs per cluster along K
+  int stages;             // depth of the packed ring (<= 16)
+  uint32_t a_stage_bytes; // m_pad * 128
+  uint32_t tmem_cols;
+  uint32_t idesc;
+  int c_aligned;          // rows of C start on 8-byte boundaries
+  uint64_t wait_budget_ns;
+};
+
+struct W4Cfg {
+  static constexpr int BK = 64;
+  static constexpr int PANEL = 128;
+  static constexpr int PACKED_BYTES = PANEL * BK / 2;  // 4 KiB of codes per k-block
+  static constexpr int WDQ_BYTES = PANEL * BK * 2;     // 16 KiB fp16 tile
+  static constexpr int WDQ_SLOTS = 3;
+  static constexpr int EPI_WARP0 = 2;
+  static constexpr int DQ_WARP0 = 6;
+  static constexpr int DQ_WARPS = 8;
+  static constexpr int THREADS = (DQ_WARP0 + DQ_WARPS) * 32;
+  static constexpr int MAX_STAGES = 16;
+  static constexpr int BAR_BYTES = 512;
+
+  static int ring_stage_bytes(int m_pad) { return PACKED_BYTES + m_pad * 128; }
+  static int smem_bytes(int m_pad, int stages) {
+    return 1024 + WDQ_SLOTS * WDQ_BYTES + stages * ring_stage_bytes(m_pad) + BAR_BYTES;
+  }
+};
+
+__global__ void __launch_bounds__(W4Cfg::THREADS, 1)
+    gemm_relu_w4a16_skinny_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
+                                  const W4Params p) {
+  using Cfg = W4Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* wdq_smem = smem;                                               // WDQ_SLOTS x 16 KiB (1024-aligned)
+  uint8_t* a_smem = wdq_smem + Cfg::WDQ_SLOTS * Cfg::WDQ_BYTES;           // stages x a_stage_bytes (1024-aligned)
+  uint8_t* packed_smem = a_smem + p.stages * p.a_stage_bytes;             // stages x 4 KiB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(packed_smem + p.stages * Cfg::PACKED_BYTES);
+  uint64_t* full_bar = bars;                                // [MAX_STAGES]: codes + activations landed
+  uint64_t* empty_bar = bars + Cfg::MAX_STAGES;             // [MAX_STAGES]: the MMAs read the activations
+  uint64_t* wdq_full_bar = bars + 2 * Cfg::MAX_STAGES;      // [WDQ_SLOTS]: fp16 tile written
+  uint64_t* wdq_empty_bar = wdq_full_bar + Cfg::WDQ_SLOTS;  // [WDQ_SLOTS]: the MMAs read the fp16 tile
+  uint64_t* acc_full_bar = wdq_empty_bar + Cfg::WDQ_SLOTS;
+  uint64_t* mma_done_bar = acc_full_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* partial = reinterpret_cast<float*>(smem);          // [m_pad][128], reuses the rings
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int n0 = blockIdx.y * Cfg::PANEL;
+  const int kb_lo = static_cast<int>((static_cast<int64_t>(p.k_blocks) * rank) / p.splits);
+  const int kb_hi = static_cast<int>((static_cast<int64_t>(p.k_blocks) * (rank + 1)) / p.splits);
+  const int my_blocks = kb_hi - kb_lo;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int s = 0; s < Cfg::WDQ_SLOTS; ++s) {
+      mbar_init(&wdq_full_bar[s], Cfg::DQ_WARPS);
+      mbar_init(&wdq_empty_bar[s], 1);
+    }
+    mbar_init(acc_full_bar, 1);
+    mbar_init(mma_done_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish_alloc_permit();
+  }
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  tcgen05_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  if (warp == 0) {
+    // Producer: packed codes of the panel and the activations, per k-block.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[Cfg::MAX_STAGES];
+#pragma unroll
+      for (int s = 0; s < Cfg::MAX_STAGES; ++s) last_parity[s] = -1;
+      const uint32_t tx = Cfg::PACKED_BYTES + p.a_stage_bytes;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 0x61)) break;
+        mbar_arrive_expect_tx(&full_bar[stage], tx);
+        tma_load_2d(packed_smem + stage * Cfg::PACKED_BYTES, &tmap_w, &full_bar[stage], kb * (Cfg::BK / 2), n0);
+        tma_load_2d(a_smem + stage * p.a_stage_bytes, &tmap_a, &full_bar[stage], kb * Cfg::BK, 0);
+        last_parity[stage] = static_cast<int>(phase);
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      for (int s = 0; s < p.stages; ++s) {
+        if (last_parity[s] >= 0) {
+          volatile int no_abort = 0;
+          mbar_wait(&full_bar[s], static_cast<uint32_t>(last_parity[s]), &no_abort, p.wait_budget_ns, 0x62);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // MMA issuer: dequantized weight (K-major, MMA A) x activations (K-major, MMA B).
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int i = 0; i < my_blocks; ++i) {
+        const int slot = i % Cfg::WDQ_SLOTS;
+        const uint32_t slot_phase = static_cast<uint32_t>((i / Cfg::WDQ_SLOTS) & 1);
+        if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 0x63) ||
+            !mbar_wait(&wdq_full_bar[slot], slot_phase, abort_flag, p.wait_budget_ns, 0x64)) {
+          ok = false;
+          break;
+        }
+        tcgen05_fence_after_sync();
+        const uint32_t w_addr = smem_u32(wdq_smem + slot * Cfg::WDQ_BYTES);
+        const uint32_t a_addr = smem_u32(a_smem + stage * p.a_stage_bytes);
+#pragma unroll
+        for (int k = 0; k < Cfg::BK / 16; ++k) {
+          const uint64_t adesc = make_sw128_desc(w_addr + k * 32, 16, 1024);
+          const uint64_t bdesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+          umma_f16_ss(tmem_base, adesc, bdesc, p.idesc, (i | k) != 0 ? 1u : 0u);
+        }
+        umma_commit(&empty_bar[stage]);
+        umma_commit(&wdq_empty_bar[slot]);
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok && my_blocks > 0) umma_commit(acc_full_bar);
+      umma_commit(mma_done_bar);
+      volatile int no_abort = 0;
+      mbar_wait(mma_done_bar, 0, &no_abort, p.wait_budget_ns, 0x65);
+    }
+    __syncwarp();
+  } else if (warp >= Cfg::DQ_WARP0) {
+    // Dequantization: thread t owns row t/2 of the panel and 32 of its 64
+    // codes per k-block (4 chunks of 8).
+    const int t = threadIdx.x - Cfg::DQ_WARP0 * 32;  // 0..255
+    const int r = t >> 1;
+    const int half = t & 1;
+    const bool row_ok = n0 + r < p.N;
+    const int groups_per_row = p.K / p.group;
+    const __half* srow = p.S + static_cast<int64_t>(row_ok ? n0 + r : 0) * groups_per_row;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int i = 0; i < my_blocks; ++i) {
+      const int kb = kb_lo + i;
+      const int slot = i % Cfg::WDQ_SLOTS;
+      const uint32_t slot_phase = static_cast<uint32_t>((i / Cfg::WDQ_SLOTS) & 1);
+      const bool ready = mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 0x66) &&
+                         mbar_wait(&wdq_empty_bar[slot], slot_phase ^ 1u, abort_flag, p.wait_budget_ns, 0x67);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      // Rows past N were zero-filled by TMA; a zero scale keeps them finite.
+      const __half s = row_ok ? srow[(kb * Cfg::BK + half * 32) / p.group] : __float2half(0.0f);
+      const __half2 s2 = __halves2half2(s, s);
+      const uint4 codes = *reinterpret_cast<const uint4*>(packed_smem + stage * Cfg::PACKED_BYTES + r * 32 + half * 16);
+      uint8_t* dst = wdq_smem + slot * Cfg::WDQ_BYTES + r * 128;
+      const uint32_t words[4] = {codes.x, codes.y, codes.z, codes.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int chunk = half * 4 + j;  // 8 fp16 values = 16 bytes
+        *reinterpret_cast<uint4*>(dst + ((chunk ^ (r & 7)) << 4)) = dequant8(words[j], s2);
+      }
+      fence_proxy_async_smem();  // the generic-proxy writes become visible to the MMA's reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&wdq_full_bar[slot]);
+      if (++stage == p.stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  } else {
+    // Epilogue warps: TMEM partial -> shared memory [m][n] (fp32).
+    const int quad = warp & 3;
+    const int n_local = quad * 32 + lane;
+    bool ready = true;
+    if (my_blocks > 0) ready = mbar_wait(acc_full_bar, 0, abort_flag, p.wait_budget_ns, 0x68);
+    ready = __all_sync(0xffffffffu, ready);
+    if (ready) {
+      tcgen05_fence_after_sync();
+      for (int c = 0; c < p.m_pad / 16; ++c) {
+        uint32_t rr[16];
+        if (my_blocks > 0) {
+          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c * 16, rr);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) rr[e] = 0u;
+        }
+        // The rings are free once the last MMA has completed (acc_full).
+#pragma unroll
+        for (int e = 0; e < 16; ++e) partial[(c * 16 + e) * Cfg::PANEL + n_local] = __uint_as_float(rr[e]);
+      }
+    }
+    tcgen05_fence_before_sync();
+  }
+
+  __syncthreads();
+  cluster_sync();  // every partial of the cluster is in shared memory
+
+  if (warp >= Cfg::EPI_WARP0 && warp < Cfg::DQ_WARP0 && !*abort_flag) {
+    // Reduction over the S partials in rank order; items are (m, 4-column group).
+    const int e = threadIdx.x - Cfg::EPI_WARP0 * 32;  // 0..127
+    const int items = p.M * (Cfg::PANEL / 4);
+    const int lo = static_cast<int>((static_cast<int64_t>(items) * rank) / p.splits);
+    const int hi = static_cast<int>((static_cast<int64_t>(items) * (rank + 1)) / p.splits);
+    const uint32_t part_addr = smem_u32(partial);
+    for (int it = lo + e; it < hi; it += 128) {
+      const int m = it / (Cfg::PANEL / 4);
+      const int j = it - m * (Cfg::PANEL / 4);
+      const int n = n0 + 4 * j;
+      if (n >= p.N) continue;
+      const uint32_t off = static_cast<uint32_t>((m * Cfg::PANEL + 4 * j) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < p.splits; ++q) {
+        const float4 v = ld_shared_cluster_f4(mapa_shared(part_addr + off, static_cast<uint32_t>(q)));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const __half2 h01 = __floats2half2_rn(acc.x > 0.f ? acc.x : 0.f, acc.y > 0.f ? acc.y : 0.f);
+      const __half2 h23 = __floats2half2_rn(acc.z > 0.f ? acc.z : 0.f, acc.w > 0.f ? acc.w : 0.f);
+      uint2 packed;
+      packed.x = *reinterpret_cast<const uint32_t*>(&h01);
+      packed.y = *reinterpret_cast<const uint32_t*>(&h23);
+      __half* dst = p.C + static_cast<int64_t>(m) * p.N + n;
+      if (p.c_aligned) {
+        *reinterpret_cast<uint2*>(dst) = packed;
+      } else {
+        unsigned short* d16 = reinterpret_cast<unsigned short*>(dst);
+        const uint32_t w[2] = {packed.x, packed.y};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (n + q < p.N) d16[q] = static_cast<unsigned short>(w[q >> 1] >> ((q & 1) * 16));
+      }
+    }
+  }
+
+  cluster_sync();  // peers are done reading this CTA's partial
+  if (warp == 1) {
+    tcgen05_fence_after_sync();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace tg

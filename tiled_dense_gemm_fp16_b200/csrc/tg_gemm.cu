@@ -16,6 +16,7 @@
 
 #include "tg_gemm.h"
 #include "gemm_mx.cuh"
+#include "gemm_mx_pair.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc_pair.cuh"
@@ -45,7 +46,8 @@ struct DeviceInfo {
   bool tc_edge_attr = false;
   bool skinny_attr = false;
   unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
-  bool mx_attr[2] = {false, false};  // per block-scaled kind
+  bool mx_attr[2] = {false, false};       // per block-scaled kind
+  bool mx_pair_attr[2] = {false, false};
   void* static_ws = nullptr;  // device address of g_static_workspace on this device
 };
 
@@ -775,13 +777,20 @@ bool encode_2d_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
 // Bytes of a blocked scale array for `rows` rows and `scales` scale columns.
 int64_t blocked_scale_bytes(int64_t rows, int64_t scales) { return round_up(rows, 128) * round_up(scales, 4); }
 
-// Shared launcher of the block-scaled grouped kernels.  elem_bits: 8 (MXFP8)
-// or 4 (NVF4); block: elements per scale (32 or 16).
+// Instruction descriptor of a block-scaled MMA of M x 256.
+template <int KIND>
+uint32_t blockscaled_idesc(int M, int a_format, int b_format) {
+  return KIND == kKindNvf4 ? make_idesc_nvf4(M, 256) : make_idesc_mxf8(M, 256, a_format, b_format, 0, 0);
+}
+
+// Shared launcher of the block-scaled grouped kernels (one kind each): the
+// 1-SM kernel or the CTA-pair kernel, whichever needs fewer tile waves.
 template <int KIND>
 tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
-                                  const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, uint32_t idesc,
-                                  float alpha, int32_t relu, void* stream) {
+                                  const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, int a_format,
+                                  int b_format, float alpha, int32_t relu, void* stream) {
   using Cfg = MxCfg<KIND>;
+  using PairCfg = MxPairCfg<KIND>;
   constexpr int kBlock = KIND == kKindNvf4 ? 16 : 32;
   constexpr int kMmaK = KIND == kKindNvf4 ? 64 : 32;
   constexpr int kElemsPerByte = KIND == kKindNvf4 ? 2 : 1;
@@ -807,6 +816,88 @@ tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B,
   DeviceInfo* info = nullptr;
   tg_status st = current_device(dev, info);
   if (st != TG_OK) return st;
+
+  MxParams p;
+  std::memset(&p, 0, sizeof p);
+  p.SFA = static_cast<const uint8_t*>(SFA);
+  p.SFB = static_cast<const uint8_t*>(SFB);
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.k_stages = static_cast<int>((row_bytes + Cfg::BK - 1) / Cfg::BK);
+  p.k_mmas = static_cast<int>(K / kMmaK);
+  p.atoms_k = static_cast<int>(round_up(K / kBlock, 4) / 4);
+  p.alpha = alpha;
+  p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
+  p.m_tiles = static_cast<int>(rows / Cfg::BM);
+  p.groups = groups;
+  p.n_atoms = static_cast<int>((N + 127) / 128);
+  p.relu = relu;
+  p.wait_budget_ns = wait_budget(p.k_stages * 2);
+  int tile = 0, pair = 0;
+  for (int32_t g = 0; g < groups; ++g) {
+    const int tiles_g = static_cast<int>(round_up(m_sizes[g], 128) / 128);
+    p.tile_start[g] = tile;
+    p.pair_start[g] = pair;
+    p.m_size[g] = static_cast<int>(m_sizes[g]);
+    tile += tiles_g;
+    pair += (tiles_g + 1) / 2;
+  }
+  p.tile_start[groups] = tile;
+  p.pair_start[groups] = pair;
+  p.pair_tiles = pair;
+
+  // The CTA-pair kernel computes the same result but measured 1.76x slower
+  // per SM than the 1-SM kernel on B200 for both kinds, so it runs only when
+  // asked for (TG_TUNE_MX_PAIR=1).
+  const int64_t single_tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  const int64_t pair_tiles = static_cast<int64_t>(p.pair_tiles) * p.n_tiles;
+  const int sms = info->sm_count, pairs = info->sm_count / 2;
+  const bool use_pair = tune_int("TG_TUNE_MX_PAIR", 0) == 1 && pairs >= 1;
+
+  CUtensorMap ta, tb;
+  std::memset(&ta, 0, sizeof ta);
+  std::memset(&tb, 0, sizeof tb);
+  if (K > 0) {
+    if (!encode_2d_u8(&ta, A, rows, row_bytes, Cfg::BK, Cfg::BM)) return TG_ERR_LAUNCH;
+    if (!encode_2d_u8(&tb, B, static_cast<int64_t>(groups) * N, row_bytes, Cfg::BK,
+                      use_pair ? PairCfg::B_ROWS : Cfg::BN))
+      return TG_ERR_LAUNCH;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  LaunchAttrs la;
+  if (use_pair) {
+    auto kernel = gemm_blockscaled_pair_kernel<KIND>;
+    {
+      std::lock_guard<std::mutex> lock(g_mutex);
+      if (!info->mx_pair_attr[KIND]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES) !=
+            cudaSuccess) {
+          cudaGetLastError();
+          return TG_ERR_LAUNCH;
+        }
+        info->mx_pair_attr[KIND] = true;
+      }
+    }
+    p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 8);
+    if (p.group_m < 1) p.group_m = 1;
+    p.num_tiles = static_cast<int>(pair_tiles);
+    p.idesc = blockscaled_idesc<KIND>(PairCfg::PAIR_M, a_format, b_format);
+    int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
+    const int max_clusters = tune_int("TG_TUNE_MX_CLUSTERS", 0);
+    if (max_clusters > 0 && max_clusters < clusters) clusters = max_clusters;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+    cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(PairCfg::SMEM_BYTES);
+    la.fill(cfg, 2);
+    if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
+      cudaGetLastError();
+      return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
+  }
   auto kernel = gemm_blockscaled_grouped_kernel<KIND>;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -819,49 +910,14 @@ tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B,
       info->mx_attr[KIND] = true;
     }
   }
-  CUtensorMap ta, tb;
-  std::memset(&ta, 0, sizeof ta);
-  std::memset(&tb, 0, sizeof tb);
-  MxParams p;
-  std::memset(&p, 0, sizeof p);
-  if (K > 0) {
-    if (!encode_2d_u8(&ta, A, rows, row_bytes, Cfg::BK, Cfg::BM)) return TG_ERR_LAUNCH;
-    if (!encode_2d_u8(&tb, B, static_cast<int64_t>(groups) * N, row_bytes, Cfg::BK, Cfg::BN)) return TG_ERR_LAUNCH;
-  }
-  p.SFA = static_cast<const uint8_t*>(SFA);
-  p.SFB = static_cast<const uint8_t*>(SFB);
-  p.C = static_cast<__nv_bfloat16*>(C);
-  p.N = static_cast<int>(N);
-  p.K = static_cast<int>(K);
-  p.k_stages = static_cast<int>((row_bytes + Cfg::BK - 1) / Cfg::BK);
-  p.k_mmas = static_cast<int>(K / kMmaK);
-  p.atoms_k = static_cast<int>(round_up(K / kBlock, 4) / 4);
-  p.alpha = alpha;
-  p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
-  p.m_tiles = static_cast<int>(rows / Cfg::BM);
-  p.num_tiles = p.m_tiles * p.n_tiles;
   p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 8);
   if (p.group_m < 1) p.group_m = 1;
-  p.groups = groups;
-  p.n_atoms = static_cast<int>((N + 127) / 128);
-  p.relu = relu;
-  p.idesc = idesc;
-  p.wait_budget_ns = wait_budget(p.k_stages * 2);
-  int tile = 0;
-  for (int32_t g = 0; g < groups; ++g) {
-    p.tile_start[g] = tile;
-    p.m_size[g] = static_cast<int>(m_sizes[g]);
-    tile += static_cast<int>(round_up(m_sizes[g], 128) / 128);
-  }
-  p.tile_start[groups] = tile;
-  const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof cfg);
+  p.num_tiles = static_cast<int>(single_tiles);
+  p.idesc = blockscaled_idesc<KIND>(Cfg::BM, a_format, b_format);
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::SMEM_BYTES);
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  LaunchAttrs la;
   la.fill(cfg, 1);
   if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
     cudaGetLastError();
@@ -875,16 +931,15 @@ tg_status run_mxf8_grouped(const void* A, const void* SFA, const void* B, const 
                            int32_t b_format, int32_t relu, void* stream) {
   if ((a_format != TG_FP8_E4M3 && a_format != TG_FP8_E5M2) || (b_format != TG_FP8_E4M3 && b_format != TG_FP8_E5M2))
     return TG_ERR_INVALID_ARG;
-  return run_blockscaled_grouped<kKindMxf8>(A, SFA, B, SFB, C, m_sizes, groups, N, K,
-                                            make_idesc_mxf8(128, 256, a_format, b_format, 0, 0), 1.0f, relu, stream);
+  return run_blockscaled_grouped<kKindMxf8>(A, SFA, B, SFB, C, m_sizes, groups, N, K, a_format, b_format, 1.0f, relu,
+                                            stream);
 }
 
 tg_status run_nvf4_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
                            const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, float alpha, int32_t relu,
                            void* stream) {
   if (!std::isfinite(alpha)) return TG_ERR_INVALID_ARG;
-  return run_blockscaled_grouped<kKindNvf4>(A, SFA, B, SFB, C, m_sizes, groups, N, K, make_idesc_nvf4(128, 256),
-                                            alpha, relu, stream);
+  return run_blockscaled_grouped<kKindNvf4>(A, SFA, B, SFB, C, m_sizes, groups, N, K, 0, 0, alpha, relu, stream);
 }
 
 }  // namespace
