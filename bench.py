@@ -45,9 +45,11 @@ KERNEL_SOURCES = {
     "skinny": [_CSRC + "gemm_skinny.cuh", _CSRC + "ptx.cuh"],
     "mxf8": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
     "nvf4": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
+    "w4a16": [_CSRC + "gemm_w4a16.cuh", _CSRC + "ptx.cuh"],
 }
 MX_METRIC = "MXFP8 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP8 tensor peak"
 NVF4_METRIC = "NVF4 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP4 tensor peak"
+W4_METRIC = "W4A16 GEMM+ReLU TFLOP/s (1×B200) and % of its roofline (HBM for decode, tensor for large M)"
 PROFILES = os.path.join(ROOT, "profiles")
 L2_BYTES = 126 * 1024 * 1024
 
@@ -60,7 +62,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="square8192",
                     help="square8192 (the metric's workload), square4096, square256, skinny:<M>, ragged:<i>, "
-                         "linear8192, mxf8_moe, mxf8_8192, nvf4_8192, nvf4_moe")
+                         "linear8192, mxf8_moe, mxf8_8192, nvf4_8192, nvf4_moe, w4a16_decode, w4a16_8192")
     ap.add_argument("--path", default="auto", help="force a kernel path: auto, tc, tc_edge, skinny, tc_pair, tc_pair512")
     ap.add_argument("--workspace", choices=["auto", "none"], default="auto",
                     help="auto: give the library the scratch bytes it asks for (repack path for "
@@ -306,6 +308,8 @@ def rank_seed(workload_seed: int, rank: int) -> int:
 def run_ours(args):
     if args.workload in inputs.MX_WORKLOADS or args.workload in inputs.NVF4_WORKLOADS:
         return run_ours_mx(args)
+    if args.workload in inputs.W4_WORKLOADS:
+        return run_ours_w4(args)
     import torch
     import tiled_dense_gemm_fp16_b200 as tg
 
@@ -661,6 +665,142 @@ def run_ours_mx(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_mx(kind, ops, m_sizes, N, K, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def w4_min_bytes(M, N, K, group) -> int:
+    """Compulsory HBM bytes of one W4A16 GEMM: packed codes, scales, A and C once each."""
+    return N * K // 2 + 2 * N * (K // group) + 2 * M * K + 2 * M * N
+
+
+def run_ours_w4(args):
+    """The 4-bit weight-only GEMM on one of inputs.W4_WORKLOADS (operands resident in HBM)."""
+    import torch
+    import tiled_dense_gemm_fp16_b200 as tg
+    world, rank, dev, dist = _init_ranks(args)
+    M, N, K, group, seed = inputs.W4_WORKLOADS[args.workload]
+    A, Wq, S = inputs.w4_operands(M, N, K, group, seed if rank == 0 else rank_seed(seed, rank), "uniform")
+    stream = torch.cuda.Stream(dev)
+    sh = stream.cuda_stream
+    need = tg.w4a16_workspace_size(M, N, K, group)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    flops = inputs.flops(M, N, K)
+    nbytes = w4_min_bytes(M, N, K, group)
+    # Rotate operand copies when one set fits in L2 (the decode case), so each step reads cold data.
+    sets = []
+    reps = max(1, -(-3 * L2_BYTES // nbytes)) if nbytes <= 2 * L2_BYTES else 1
+    for _ in range(min(reps, 16)):
+        sets.append((torch.from_numpy(A).to(dev), torch.from_numpy(Wq).to(dev), torch.from_numpy(S).to(dev),
+                     torch.empty((M, N), dtype=torch.float16, device=dev)))
+    cur = [0]
+
+    def call(a, w, s_, c):
+        st = tg.gemm_relu_w4a16_raw(a.data_ptr(), w.data_ptr(), s_.data_ptr(), c.data_ptr(), M, N, K, group, sh,
+                                    ws.data_ptr(), need)
+        if st != tg.Status.OK:
+            raise tg.TGError(st, "tg_gemm_relu_w4a16")
+
+    def step():
+        call(*sets[cur[0] % len(sets)])
+        cur[0] += 1
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+    st, word = tg.device_status()
+    if st != tg.Status.OK:
+        raise SystemExit(f"device error after warm-up: {tg.status_string(st)} 0x{word:x}")
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        r0.record(stream)
+        for _ in range(args.steps):
+            step()
+        r1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    step_ms = r0.elapsed_time(r1) / args.steps
+    kern_ms = step_ms
+    if dist is not None:
+        step_ms = max_over_ranks(dist, step_ms, dev)
+    st, word = tg.device_status()
+    if st != tg.Status.OK:
+        raise SystemExit(f"device error in timed region: {tg.status_string(st)} 0x{word:x}")
+    value = aggregate_throughput(world, flops, step_ms)
+
+    Ah, Wh, Sh = (torch.from_numpy(x).pin_memory() for x in (A, Wq, S))
+    Ch = torch.empty((M, N), dtype=torch.float16).pin_memory()
+    a, w, s_, c = sets[0]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for i in range(args.e2e_steps + 1):
+            if i == 1:
+                e0.record(stream)
+            a.copy_(Ah, non_blocking=True)
+            w.copy_(Wh, non_blocking=True)
+            s_.copy_(Sh, non_blocking=True)
+            call(a, w, s_, c)
+            Ch.copy_(c, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist is not None:
+        e2e_ms = max_over_ranks(dist, e2e_ms, dev)
+
+    peaks, peak_src = load_peaks()
+    fused = need == 0
+    if fused:
+        roof = {"bound": "hbm", "achieved": nbytes / (kern_ms * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
+                "unit": "GB/s", "peak_source": f"{peak_src} STREAM-copy HBM bandwidth"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / (kern_ms * 1e-3) / 1e12, "peak": float(peaks["bf16_tflops"]),
+                "unit": "TFLOP/s", "peak_source": f"{peak_src} cuBLAS bf16 burst peak (fp16 runs at the bf16 rate)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = committed_traffic("w4a16", args.workload) if rank == 0 else None
+    roof["kernel_ms"] = kern_ms
+    line = {
+        "metric": W4_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 activations x 4-bit weights (fp16 scales per group), fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "M": M, "N": N, "K": K, "group": group, "seed": seed,
+                   "path": "w4a16 fused" if fused else "dequantize + tc (fp16 GEMM)",
+                   "workspace_bytes": need, "min_bytes": nbytes,
+                   "l2": (f"rotating {len(sets)} operand copies" if len(sets) > 1 else "inputs larger than L2"),
+                   "parallelism": f"dp{world} independent problems" if world > 1 else "1 GPU"},
+        "roofline": roof,
+        "e2e": {"value": aggregate_throughput(world, flops, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": A.nbytes + Wq.nbytes + S.nbytes, "d2h_bytes_per_step": 2 * M * N,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * (1 if fused else 2),
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        cores = os.cpu_count() or 1
+        rows = 1
+        while True:
+            t0 = time.perf_counter()
+            oracle.gemm_relu_w4a16(A[:rows], Wq, S, group, nthreads=cores)
+            dt = time.perf_counter() - t0
+            if dt >= args.cpu_seconds or rows >= M:
+                break
+            rows = min(M, max(rows * 2, int(rows * args.cpu_seconds / max(dt, 1e-3) * 0.9)))
+        line["cpu_baseline"] = {"value": inputs.flops(rows, N, K) / dt / 1e12, "unit": UNIT, "cores": cores,
+                                "kind": "oracle", "seconds": dt,
+                                "sample": f"rows 0..{rows - 1} ({rows} x {N} x {K}), {dt:.1f} s on {cores} threads"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -348,6 +348,39 @@ TG_API tg_status tg_gemm_nvf4_grouped(const void *A, const void *SFA, const void
  * (roundup(rows, 128) * roundup(K/16, 4)), or -1 if K % 16 != 0. */
 TG_API int64_t tg_nvf4_scale_bytes(int64_t rows, int64_t K);
 
+/* ---------------------------------------------------------------------------
+ * 4-bit weight-only GEMM (W4A16)
+ *
+ * The dequantize_gemm workload of the TileLang pages ("TileLang" wiki page,
+ * opening paragraph), read as the common W4A16 scheme:
+ *
+ *   w(n,k)  = fp16( (q(n,k) - 8) * s(n, k/group) )      (exact product, one RNE rounding)
+ *   C[m*N + n] = fp16( max( sum_k A[m*K + k] * w(n,k), 0 ) )   (fp32 accumulation)
+ *
+ * A: M x K fp16, row-major.  Wq: the N x K weight as 4-bit codes q, rows of
+ * K/2 bytes, element 2i of a row in the low nibble of byte i.  scales: N x
+ * (K/group) fp16, row-major.  C: M x N fp16, row-major.  group is a multiple
+ * of 32 that divides K; K % 64 == 0.
+ * M <= 256 runs one fused kernel that streams the packed weight once.  Larger
+ * M dequantizes the weight into `workspace` (tg_w4a16_workspace_size bytes,
+ * 16-byte aligned, 2*N*K rounded up) and runs the fp16 tensor-core GEMM.
+ * Errors (TG_ERR_INVALID_ARG, nothing enqueued): bad sizes or group, A or Wq
+ * not 16-byte aligned, scales or C not 2-byte aligned, C overlapping an
+ * input, too small a workspace.  K == 0 writes +0.  Asynchronous on `stream`.
+ * ------------------------------------------------------------------------- */
+TG_API tg_status tg_gemm_relu_w4a16(const void *A, const void *Wq, const void *scales, void *C, int64_t M,
+                                    int64_t N, int64_t K, int32_t group, void *stream, void *workspace,
+                                    int64_t workspace_bytes);
+
+/* Workspace bytes tg_gemm_relu_w4a16 needs for these sizes (0 for M <= 256),
+ * or -1 if the sizes are invalid. */
+TG_API int64_t tg_w4a16_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group);
+
+/* The dequantized weight alone: W (N x K fp16, 16-byte aligned) = w(n,k) as
+ * above.  Same requirements on Wq, scales, K and group. */
+TG_API tg_status tg_dequant_w4_f16(const void *Wq, const void *scales, void *W, int64_t N, int64_t K,
+                                   int32_t group, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

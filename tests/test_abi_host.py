@@ -252,3 +252,22 @@ def test_nvf4_host_validation():
     assert call(alpha=float("inf")) == Status.INVALID_ARG
     assert call(C=P + 32) == Status.INVALID_ARG       # C overlaps A
     assert call(m=(0,)) == Status.OK
+
+
+def test_w4a16_host_validation():
+    assert tg.w4a16_workspace_size(16, 8192, 8192, 128) == 0
+    assert tg.w4a16_workspace_size(300, 256, 512, 128) == 2 * 256 * 512
+    assert tg.w4a16_workspace_size(300, 256, 500, 128) == -1      # K % 64
+    assert tg.w4a16_workspace_size(300, 256, 512, 48) == -1       # group not a multiple of 32
+    assert tg.w4a16_workspace_size(300, 256, 512, 384) == -1      # group does not divide K
+    P = 0x40_0000_0000
+
+    def call(M=16, N=256, K=512, g=128, A=P, W=P + (1 << 30), S=P + (2 << 30), C=P + (3 << 30)):
+        return tg.gemm_relu_w4a16_raw(A, W, S, C, M, N, K, g)
+    assert call(K=96) == Status.INVALID_ARG
+    assert call(g=16) == Status.INVALID_ARG
+    assert call(A=P + 8) == Status.INVALID_ARG                    # A not 16-byte aligned
+    assert call(S=P + (2 << 30) + 1) == Status.INVALID_ARG        # scales not 2-byte aligned
+    assert call(C=P + 64) == Status.INVALID_ARG                   # C overlaps A
+    assert call(M=0) == Status.OK
+    assert tg.dequant_w4_f16_raw(P, P + (1 << 30), P + 32, 16, 256, 64) == Status.INVALID_ARG  # W overlaps Wq

@@ -90,6 +90,9 @@ EXPORTS = (
     "tg_mx_scale_bytes",
     "tg_gemm_nvf4_grouped",
     "tg_nvf4_scale_bytes",
+    "tg_gemm_relu_w4a16",
+    "tg_w4a16_workspace_size",
+    "tg_dequant_w4_f16",
 )
 
 _lib = None
@@ -144,6 +147,12 @@ def _bind(lib):
     lib.tg_gemm_nvf4_grouped.restype = i32
     lib.tg_nvf4_scale_bytes.argtypes = [i64, i64]
     lib.tg_nvf4_scale_bytes.restype = i64
+    lib.tg_gemm_relu_w4a16.argtypes = [vp, vp, vp, vp, i64, i64, i64, ctypes.c_int32, vp, vp, i64]
+    lib.tg_gemm_relu_w4a16.restype = i32
+    lib.tg_w4a16_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int32]
+    lib.tg_w4a16_workspace_size.restype = i64
+    lib.tg_dequant_w4_f16.argtypes = [vp, vp, vp, i64, i64, ctypes.c_int32, vp]
+    lib.tg_dequant_w4_f16.restype = i32
     return lib
 
 
@@ -449,4 +458,51 @@ def nvf4_grouped(A, SFA, B, SFB, m_sizes, alpha=1.0, relu=False, out=None, strea
         st = gemm_nvf4_grouped_raw(A.data_ptr(), SFA.data_ptr(), B.data_ptr(), SFB.data_ptr(), out.data_ptr(),
                                    m_sizes, N, K, alpha, relu, handle)
     _check(st, "tg_gemm_nvf4_grouped")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# 4-bit weight-only GEMM (W4A16)
+# ---------------------------------------------------------------------------
+
+def w4a16_workspace_size(M: int, N: int, K: int, group: int) -> int:
+    return int(lib().tg_w4a16_workspace_size(M, N, K, group))
+
+
+def gemm_relu_w4a16_raw(A: int, Wq: int, S: int, C: int, M: int, N: int, K: int, group: int, stream: int = 0,
+                        workspace: int = 0, workspace_bytes: int = 0) -> int:
+    return int(lib().tg_gemm_relu_w4a16(A, Wq, S, C, M, N, K, group, stream, workspace, workspace_bytes))
+
+
+def dequant_w4_f16_raw(Wq: int, S: int, W: int, N: int, K: int, group: int, stream: int = 0) -> int:
+    return int(lib().tg_dequant_w4_f16(Wq, S, W, N, K, group, stream))
+
+
+def gemm_relu_w4a16(A, Wq, S, group, out=None, stream=None, workspace="auto"):
+    """ReLU(A @ dequant(W)^T) for CUDA tensors: A (M, K) float16, Wq (N, K/2) uint8 packed codes,
+    S (N, K/group) float16 scales; returns C (M, N) float16."""
+    import torch
+    if A.dim() != 2 or Wq.dim() != 2 or S.dim() != 2 or Wq.shape[1] * 2 != A.shape[1] or S.shape[0] != Wq.shape[0]:
+        raise ValueError(f"shape mismatch: A{tuple(A.shape)} Wq{tuple(Wq.shape)} S{tuple(S.shape)}")
+    if A.dtype != torch.float16 or S.dtype != torch.float16 or Wq.dtype != torch.uint8:
+        raise TypeError("A and S must be float16, Wq uint8")
+    if not (A.is_contiguous() and Wq.is_contiguous() and S.is_contiguous()):
+        raise ValueError("A, Wq and S must be contiguous")
+    M, K = A.shape
+    N = Wq.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    handle = stream.cuda_stream if stream is not None else _stream_handle(A.device)
+    with torch.cuda.device(A.device):
+        need = w4a16_workspace_size(M, N, K, group)
+        if need < 0:
+            raise TGError(Status.INVALID_ARG, "tg_w4a16_workspace_size")
+        ws_ptr, ws_bytes = 0, 0
+        if need > 0 and workspace is not None:
+            if isinstance(workspace, str):
+                workspace = torch.empty(need, dtype=torch.uint8, device=A.device)
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        st = gemm_relu_w4a16_raw(A.data_ptr(), Wq.data_ptr(), S.data_ptr(), out.data_ptr(), M, N, K, group, handle,
+                                 ws_ptr, ws_bytes)
+    _check(st, "tg_gemm_relu_w4a16")
     return out

@@ -13,8 +13,9 @@
 //     a cluster of S CTAs splits K and reduces through distributed shared
 //     memory) with a dequantization stage in front of the MMA:
 //       - warp 0 loads, per 64-deep k-block, the panel's packed codes (128
-//         rows x 32 bytes) and the activations (m_pad rows x 64) into a deep
-//         ring;
+//         rows x 32 bytes), a 16-byte box of each row's scales (8 groups
+//         around the k-block) and the activations (m_pad rows x 64) into a
+//         deep ring, so no scale load sits on the dequantization's path;
 //       - warps 6-13 turn each packed tile into the fp16 tile the MMA reads
 //         (128-byte swizzled, K-major) in a small second ring: a nibble is
 //         placed in the mantissa of 1024.0 (exponent bits 0x6400), 1032 is
@@ -95,6 +96,7 @@ struct W4Params {
   uint32_t tmem_cols;
   uint32_t idesc;
   int c_aligned;          // rows of C start on 8-byte boundaries
+  int scale_tma;          // 1: scales arrive with the ring (rows of K/group fp16 are 16-byte multiples)
   uint64_t wait_budget_ns;
 };
 
@@ -103,7 +105,8 @@ struct W4Cfg {
   static constexpr int PANEL = 128;
   static constexpr int PACKED_BYTES = PANEL * BK / 2;  // 4 KiB of codes per k-block
   static constexpr int WDQ_BYTES = PANEL * BK * 2;     // 16 KiB fp16 tile
-  static constexpr int WDQ_SLOTS = 3;
+  static constexpr int WDQ_SLOTS = 6;
+  static constexpr int SCALE_BYTES = PANEL * 16;        // 128 rows x 8 scales
   static constexpr int EPI_WARP0 = 2;
   static constexpr int DQ_WARP0 = 6;
   static constexpr int DQ_WARPS = 8;
@@ -111,7 +114,7 @@ struct W4Cfg {
   static constexpr int MAX_STAGES = 16;
   static constexpr int BAR_BYTES = 512;
 
-  static int ring_stage_bytes(int m_pad) { return PACKED_BYTES + m_pad * 128; }
+  static int ring_stage_bytes(int m_pad) { return PACKED_BYTES + SCALE_BYTES + m_pad * 128; }
   static int smem_bytes(int m_pad, int stages) {
     return 1024 + WDQ_SLOTS * WDQ_BYTES + stages * ring_stage_bytes(m_pad) + BAR_BYTES;
   }
@@ -119,14 +122,15 @@ struct W4Cfg {
 
 __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     gemm_relu_w4a16_skinny_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
-                                  const W4Params p) {
+                                  const __grid_constant__ CUtensorMap tmap_s, const W4Params p) {
   using Cfg = W4Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* wdq_smem = smem;                                               // WDQ_SLOTS x 16 KiB (1024-aligned)
   uint8_t* a_smem = wdq_smem + Cfg::WDQ_SLOTS * Cfg::WDQ_BYTES;           // stages x a_stage_bytes (1024-aligned)
   uint8_t* packed_smem = a_smem + p.stages * p.a_stage_bytes;             // stages x 4 KiB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(packed_smem + p.stages * Cfg::PACKED_BYTES);
+  uint8_t* scale_smem = packed_smem + p.stages * Cfg::PACKED_BYTES;       // stages x 2 KiB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scale_smem + p.stages * Cfg::SCALE_BYTES);
   uint64_t* full_bar = bars;                                // [MAX_STAGES]: codes + activations landed
   uint64_t* empty_bar = bars + Cfg::MAX_STAGES;             // [MAX_STAGES]: the MMAs read the activations
   uint64_t* wdq_full_bar = bars + 2 * Cfg::MAX_STAGES;      // [WDQ_SLOTS]: fp16 tile written
@@ -160,6 +164,7 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     fence_mbarrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_w);
+    if (p.scale_tma) tma_prefetch_desc(&tmap_s);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, p.tmem_cols);
@@ -180,11 +185,14 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
       int last_parity[Cfg::MAX_STAGES];
 #pragma unroll
       for (int s = 0; s < Cfg::MAX_STAGES; ++s) last_parity[s] = -1;
-      const uint32_t tx = Cfg::PACKED_BYTES + p.a_stage_bytes;
+      const uint32_t tx = Cfg::PACKED_BYTES + p.a_stage_bytes + (p.scale_tma ? Cfg::SCALE_BYTES : 0u);
       for (int kb = kb_lo; kb < kb_hi; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 0x61)) break;
         mbar_arrive_expect_tx(&full_bar[stage], tx);
         tma_load_2d(packed_smem + stage * Cfg::PACKED_BYTES, &tmap_w, &full_bar[stage], kb * (Cfg::BK / 2), n0);
+        if (p.scale_tma)  // the 8 groups that start at the k-block's group rounded down to a multiple of 8
+          tma_load_2d(scale_smem + stage * Cfg::SCALE_BYTES, &tmap_s, &full_bar[stage],
+                      (kb * Cfg::BK / p.group) & ~7, n0);
         tma_load_2d(a_smem + stage * p.a_stage_bytes, &tmap_a, &full_bar[stage], kb * Cfg::BK, 0);
         last_parity[stage] = static_cast<int>(phase);
         if (++stage == p.stages) {
@@ -254,7 +262,12 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
                          mbar_wait(&wdq_empty_bar[slot], slot_phase ^ 1u, abort_flag, p.wait_budget_ns, 0x67);
       if (!__all_sync(0xffffffffu, ready)) break;
       // Rows past N were zero-filled by TMA; a zero scale keeps them finite.
-      const __half s = row_ok ? srow[(kb * Cfg::BK + half * 32) / p.group] : __float2half(0.0f);
+      const int g = (kb * Cfg::BK + half * 32) / p.group;
+      __half s = __float2half(0.0f);
+      if (row_ok) {
+        s = p.scale_tma ? reinterpret_cast<const __half*>(scale_smem + stage * Cfg::SCALE_BYTES + r * 16)[g & 7]
+                        : srow[g];
+      }
       const __half2 s2 = __halves2half2(s, s);
       const uint4 codes = *reinterpret_cast<const uint4*>(packed_smem + stage * Cfg::PACKED_BYTES + r * 32 + half * 16);
       uint8_t* dst = wdq_smem + slot * Cfg::WDQ_BYTES + r * 128;

@@ -20,6 +20,7 @@
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc_pair.cuh"
+#include "gemm_w4a16.cuh"
 #include "ptx.cuh"
 #include "repack.cuh"
 
@@ -48,6 +49,7 @@ struct DeviceInfo {
   unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
   bool mx_attr[2] = {false, false};       // per block-scaled kind
   bool mx_pair_attr[2] = {false, false};
+  bool w4_attr = false;
   void* static_ws = nullptr;  // device address of g_static_workspace on this device
 };
 
@@ -316,6 +318,20 @@ bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, i
   cuuint32_t estride[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estride,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// fp16 matrix (rows x cols, row stride cols) with an unswizzled box.
+bool encode_2d_f16_plain(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -761,7 +777,8 @@ int64_t mx_scale_bytes(int64_t rows, int64_t K) { return round_up(rows, 128) * r
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool encode_2d_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+bool encode_2d_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows,
+                  bool swizzle128 = true) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -769,8 +786,8 @@ bool encode_2d_u8(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estride[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -942,6 +959,147 @@ tg_status run_nvf4_grouped(const void* A, const void* SFA, const void* B, const 
   return run_blockscaled_grouped<kKindNvf4>(A, SFA, B, SFB, C, m_sizes, groups, N, K, 0, 0, alpha, relu, stream);
 }
 
+// ---------------------------------------------------------------------------
+// 4-bit weight-only GEMM (W4A16)
+// ---------------------------------------------------------------------------
+
+constexpr int64_t kW4FusedMaxM = 256;
+
+bool w4_args_valid(const void* A, const void* Wq, const void* S, const void* C, int64_t M, int64_t N, int64_t K,
+                   int32_t group) {
+  if (M < 0 || N < 0 || K < 0 || M > INT_MAX || N > INT_MAX || K > INT_MAX) return false;
+  if (group < 32 || group % 32 != 0 || K % 64 != 0 || (K > 0 && K % group != 0)) return false;
+  if (M == 0 || N == 0) return true;
+  if (!C || (reinterpret_cast<uintptr_t>(C) & 1u)) return false;
+  if (K == 0) return true;
+  if (!A || !Wq || !S || !aligned16(A) || !aligned16(Wq) || (reinterpret_cast<uintptr_t>(S) & 1u)) return false;
+  const int64_t c_bytes = 2 * M * N;
+  return !(ranges_overlap(C, c_bytes, A, 2 * M * K) || ranges_overlap(C, c_bytes, Wq, N * K / 2) ||
+           ranges_overlap(C, c_bytes, S, 2 * N * (K / group)));
+}
+
+int64_t w4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return (M > kW4FusedMaxM && N > 0 && K > 0) ? round_up(2 * N * K, 256) : 0;
+}
+
+tg_status launch_dequant_w4(const void* Wq, const void* S, void* W, int64_t N, int64_t K, int32_t group,
+                            cudaStream_t stream, DeviceInfo* info) {
+  DequantParams dp;
+  dp.Wq = static_cast<const uint8_t*>(Wq);
+  dp.S = static_cast<const __half*>(S);
+  dp.W = static_cast<__half*>(W);
+  dp.N = N;
+  dp.K = K;
+  dp.group = group;
+  dp.chunks = N * K / 8;
+  return launch_simple(dequant_w4_kernel, dp, dp.chunks, 4, stream, info);
+}
+
+tg_status launch_w4a16_fused(const void* A, const void* Wq, const void* S, void* C, int64_t M, int64_t N, int64_t K,
+                             int32_t group, cudaStream_t stream, DeviceInfo* info) {
+  using Cfg = W4Cfg;
+  constexpr int kMaxSmem = 227 * 1024;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!info->w4_attr) {
+      if (cudaFuncSetAttribute(gemm_relu_w4a16_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kMaxSmem) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      info->w4_attr = true;
+    }
+  }
+  W4Params p;
+  std::memset(&p, 0, sizeof p);
+  p.C = static_cast<__half*>(C);
+  p.S = static_cast<const __half*>(S);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.group = group;
+  p.m_pad = static_cast<int>((M + 15) / 16 * 16);
+  p.k_blocks = static_cast<int>(K / Cfg::BK);
+  p.a_stage_bytes = static_cast<uint32_t>(p.m_pad * 128);
+  const int ring = Cfg::ring_stage_bytes(p.m_pad);
+  int stages = (kMaxSmem - 1024 - Cfg::WDQ_SLOTS * Cfg::WDQ_BYTES - Cfg::BAR_BYTES) / ring;
+  const int cap = tune_int("TG_TUNE_W4_STAGES", Cfg::MAX_STAGES);
+  if (stages > cap) stages = cap;
+  if (stages > Cfg::MAX_STAGES) stages = Cfg::MAX_STAGES;
+  if (stages < 2) return TG_ERR_INTERNAL;
+  // The fp32 partial [M_pad][128] reuses the rings after the main loop.
+  if (Cfg::WDQ_SLOTS * Cfg::WDQ_BYTES + stages * ring < p.m_pad * Cfg::PANEL * 4) return TG_ERR_INTERNAL;
+  p.stages = stages;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(p.m_pad)) cols <<= 1;
+  p.tmem_cols = cols;
+  p.idesc = make_idesc_f16_f32(Cfg::PANEL, p.m_pad, false, false);
+  p.c_aligned = ((reinterpret_cast<uintptr_t>(C) & 7u) == 0 && N % 4 == 0) ? 1 : 0;
+  p.wait_budget_ns = wait_budget(p.k_blocks);
+  const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);
+  if (panels > 65535) return TG_ERR_INVALID_ARG;
+  int splits = tune_int("TG_TUNE_W4_SPLITS", info->sm_count / panels);
+  splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
+  if (splits > p.k_blocks) splits = p.k_blocks;
+  p.splits = splits;
+
+  CUtensorMap ta, tw, ts;
+  std::memset(&ts, 0, sizeof ts);
+  if (!encode_2d(&ta, A, M, K, K, 64, p.m_pad)) return TG_ERR_LAUNCH;
+  if (!encode_2d_u8(&tw, Wq, N, K / 2, Cfg::BK / 2, Cfg::PANEL, false)) return TG_ERR_LAUNCH;
+  // Scales by TMA when a row of them is a multiple of 16 bytes (and the base
+  // is 16-byte aligned); otherwise the dequantizing threads read them.
+  const int64_t groups_per_row = K / group;
+  p.scale_tma = (groups_per_row % 8 == 0 && aligned16(S) && tune_int("TG_TUNE_W4_SCALE_TMA", 1)) ? 1 : 0;
+  if (p.scale_tma && !encode_2d_f16_plain(&ts, S, N, groups_per_row, 8, Cfg::PANEL)) return TG_ERR_LAUNCH;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(panels), 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::smem_bytes(p.m_pad, stages));
+  cfg.stream = stream;
+  LaunchAttrs la;
+  la.fill(cfg, static_cast<unsigned>(splits));
+  if (cudaLaunchKernelEx(&cfg, gemm_relu_w4a16_skinny_kernel, ta, tw, ts, p) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
+}
+
+tg_status run_w4a16(const void* A, const void* Wq, const void* S, void* C, int64_t M, int64_t N, int64_t K,
+                    int32_t group, void* stream_ptr, void* ws, int64_t ws_bytes) {
+  if (!w4_args_valid(A, Wq, S, C, M, N, K, group)) return TG_ERR_INVALID_ARG;
+  if (ws_bytes < 0 || (ws_bytes > 0 && ws == nullptr)) return TG_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return TG_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  int dev = 0;
+  DeviceInfo* info = nullptr;
+  tg_status st = current_device(dev, info);
+  if (st != TG_OK) return st;
+  if (K == 0) {
+    if (cudaMemsetAsync(C, 0, static_cast<size_t>(2 * M * N), stream) != cudaSuccess) {
+      cudaGetLastError();
+      return TG_ERR_LAUNCH;
+    }
+    return TG_OK;
+  }
+  if (M <= kW4FusedMaxM) return launch_w4a16_fused(A, Wq, S, C, M, N, K, group, stream, info);
+  // Large M: dequantize into the workspace, then the fp16 tensor-core GEMM
+  // with the weight in the N x K layout.
+  const int64_t need = w4_workspace_bytes(M, N, K);
+  if (ws_bytes < need || !aligned16(ws) || ranges_overlap(ws, need, A, 2 * M * K) ||
+      ranges_overlap(ws, need, C, 2 * M * N) || ranges_overlap(ws, need, Wq, N * K / 2) ||
+      ranges_overlap(ws, need, S, 2 * N * (K / group)))
+    return TG_ERR_INVALID_ARG;
+  st = launch_dequant_w4(Wq, S, ws, N, K, group, stream, info);
+  if (st != TG_OK) return st;
+  Problem p = dense_problem(A, ws, C, M, N, K);
+  p.b_nk = true;
+  p.ldb = K;
+  return run(p, stream_ptr, TG_PATH_AUTO, nullptr, 0);
+}
+
 }  // namespace
 }  // namespace tg
 
@@ -964,6 +1122,33 @@ tg_status tg_gemm_nvf4_grouped(const void* A, const void* SFA, const void* B, co
                                const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, float alpha,
                                int32_t relu, void* stream) {
   return tg::run_nvf4_grouped(A, SFA, B, SFB, C, m_sizes, groups, N, K, alpha, relu, stream);
+}
+
+tg_status tg_gemm_relu_w4a16(const void* A, const void* Wq, const void* scales, void* C, int64_t M, int64_t N,
+                              int64_t K, int32_t group, void* stream, void* workspace, int64_t workspace_bytes) {
+  return tg::run_w4a16(A, Wq, scales, C, M, N, K, group, stream, workspace, workspace_bytes);
+}
+
+int64_t tg_w4a16_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group) {
+  if (M < 0 || N < 0 || K < 0 || group < 32 || group % 32 != 0 || K % 64 != 0 || (K > 0 && K % group != 0))
+    return -1;
+  return tg::w4_workspace_bytes(M, N, K);
+}
+
+tg_status tg_dequant_w4_f16(const void* Wq, const void* scales, void* W, int64_t N, int64_t K, int32_t group,
+                            void* stream) {
+  if (N < 0 || K < 0 || group < 32 || group % 32 != 0 || K % 64 != 0 || (K > 0 && K % group != 0))
+    return TG_ERR_INVALID_ARG;
+  if (N == 0 || K == 0) return TG_OK;
+  if (!Wq || !scales || !W || !tg::aligned16(Wq) || !tg::aligned16(W) ||
+      (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+      tg::ranges_overlap(W, 2 * N * K, Wq, N * K / 2) || tg::ranges_overlap(W, 2 * N * K, scales, 2 * N * (K / group)))
+    return TG_ERR_INVALID_ARG;
+  int dev = 0;
+  tg::DeviceInfo* info = nullptr;
+  tg_status st = tg::current_device(dev, info);
+  if (st != TG_OK) return st;
+  return tg::launch_dequant_w4(Wq, scales, W, N, K, group, static_cast<cudaStream_t>(stream), info);
 }
 
 int64_t tg_nvf4_scale_bytes(int64_t rows, int64_t K) {

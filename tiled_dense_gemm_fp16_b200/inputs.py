@@ -143,6 +143,29 @@ def nvf4_operands(m_sizes, N: int, K: int, seed: int, dist: str = "codes", scale
     return pack_fp4(A), SFA, pack_fp4(B), SFB
 
 
+def w4_operands(M: int, N: int, K: int, group: int, seed: int, dist: str = "uniform"):
+    """4-bit weight-only operands, drawn in this order from ``default_rng(seed)``: A (M x K fp16),
+    the weight's codes (N x K, 0..15) packed two per byte (N x K/2), and fp16 scales (N x K/group).
+
+    ``dist``: "int" draws A from the integers -2..2 and scales from {0.5, 1, 2} (every product
+    and sum exact); "uniform" draws A from U[-1,1] and scales from U[0.002, 0.02] (the magnitude of
+    a trained layer's weight step).
+    """
+    rng = np.random.default_rng(seed)
+    if dist == "int":
+        A = rng.integers(-2, 3, size=(M, K)).astype(np.float16)
+    elif dist == "uniform":
+        A = rng.uniform(-1.0, 1.0, size=(M, K)).astype(np.float16)
+    else:
+        raise ValueError(f"unknown distribution {dist!r}")
+    codes = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    if dist == "int":
+        S = np.array([0.5, 1.0, 2.0], np.float16)[rng.integers(0, 3, size=(N, K // group))]
+    else:
+        S = rng.uniform(0.002, 0.02, size=(N, K // group)).astype(np.float16)
+    return A, pack_fp4(codes), S
+
+
 def mx_scales_blocked(sf: np.ndarray) -> np.ndarray:
     """Plain row-major scales (R x S) rearranged into the C ABI's 128 x 4 blocked byte layout:
     scale (r, s) goes to ((r//128)*(S'/4) + s//4)*512 + (r%32)*16 + ((r//32)%4)*4 + s%4, with
@@ -198,6 +221,14 @@ WORKLOADS = {
 MX_WORKLOADS = {
     "mxf8_moe": ((2304, 1792, 2048, 2560, 1536, 2048, 2176, 1920), 4096, 7168, 6),
     "mxf8_8192": ((8192,), 8192, 8192, 7),
+}
+
+# 4-bit weight-only workloads: (M, N, K, group, seed).  "w4a16_decode" is a decode step of a
+# 8192-wide layer (16 tokens), bound by streaming the packed weight; "w4a16_8192" is the
+# large-M case (dequantize, then the fp16 tensor-core GEMM).
+W4_WORKLOADS = {
+    "w4a16_decode": (16, 8192, 8192, 128, 10),
+    "w4a16_8192": (8192, 8192, 8192, 128, 11),
 }
 
 # NVF4 workloads: the 8192^3 problem the NVF4 path is quoted on, and the MoE layer shape.
