@@ -359,8 +359,8 @@ TG_API int64_t tg_nvf4_scale_bytes(int64_t rows, int64_t K);
  *
  * A: M x K fp16, row-major.  Wq: the N x K weight as 4-bit codes q, rows of
  * K/2 bytes, element 2i of a row in the low nibble of byte i.  scales: N x
- * (K/group) fp16, row-major.  C: M x N fp16, row-major.  group is a multiple
- * of 32 that divides K; K % 64 == 0.
+ * (K/group) fp16, row-major.  C: M x N fp16, row-major.  group is a power of
+ * two >= 32 that divides K; K % 64 == 0.
  * M <= 256 runs one fused kernel that streams the packed weight once.  Larger
  * M dequantizes the weight into `workspace` (tg_w4a16_workspace_size bytes,
  * 16-byte aligned, 2*N*K rounded up) and runs the fp16 tensor-core GEMM.

@@ -259,6 +259,7 @@ def test_w4a16_host_validation():
     assert tg.w4a16_workspace_size(300, 256, 512, 128) == 2 * 256 * 512
     assert tg.w4a16_workspace_size(300, 256, 500, 128) == -1      # K % 64
     assert tg.w4a16_workspace_size(300, 256, 512, 48) == -1       # group not a multiple of 32
+    assert tg.w4a16_workspace_size(300, 256, 768, 96) == -1       # group not a power of two
     assert tg.w4a16_workspace_size(300, 256, 512, 384) == -1      # group does not divide K
     P = 0x40_0000_0000
 

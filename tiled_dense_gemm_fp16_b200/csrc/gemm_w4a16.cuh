@@ -46,22 +46,22 @@ struct DequantParams {
 
 // Eight 4-bit codes (a 32-bit word, element 2i in the low nibble of byte i)
 // as eight fp16 values (q - 8) * s, packed two per word, low element first.
+// Masking the word with 0x000F000F pairs elements i and i + 4 in the two
+// halves; each half becomes 1024 + q (the code in the mantissa of 1024.0),
+// 1032 is subtracted exactly, the multiply rounds once, and byte permutes
+// restore the element order.
 __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2) {
-  const uint32_t magic = 0x64006400u;  // fp16 1024.0 in both halves
-  const uint32_t p01 = (w & 0xFu) | ((w << 12) & 0xF0000u) | magic;
-  const uint32_t p23 = ((w >> 8) & 0xFu) | ((w << 4) & 0xF0000u) | magic;
-  const uint32_t p45 = ((w >> 16) & 0xFu) | ((w >> 4) & 0xF0000u) | magic;
-  const uint32_t p67 = ((w >> 24) & 0xFu) | ((w >> 12) & 0xF0000u) | magic;
+  const uint32_t mask = 0x000F000Fu, magic = 0x64006400u;  // fp16 1024.0 in both halves
+  uint32_t v[4] = {(w & mask) | magic, ((w >> 4) & mask) | magic, ((w >> 8) & mask) | magic,
+                   ((w >> 12) & mask) | magic};  // (e0,e4), (e1,e5), (e2,e6), (e3,e7)
   const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
-  uint32_t out[4];
-  const uint32_t in[4] = {p01, p23, p45, p67};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const __half2 v = __hsub2(*reinterpret_cast<const __half2*>(&in[i]), bias);  // q - 8, exact
-    const __half2 r = __hmul2(v, s2);                                             // one RNE rounding
-    out[i] = *reinterpret_cast<const uint32_t*>(&r);
+    const __half2 x = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v[i]), bias), s2);
+    v[i] = *reinterpret_cast<const uint32_t*>(&x);
   }
-  return make_uint4(out[0], out[1], out[2], out[3]);
+  return make_uint4(__byte_perm(v[0], v[1], 0x5410), __byte_perm(v[2], v[3], 0x5410),
+                    __byte_perm(v[0], v[1], 0x7632), __byte_perm(v[2], v[3], 0x7632));
 }
 
 __global__ void __launch_bounds__(256) dequant_w4_kernel(const DequantParams p) {
@@ -96,6 +96,7 @@ struct W4Params {
   uint32_t tmem_cols;
   uint32_t idesc;
   int c_aligned;          // rows of C start on 8-byte boundaries
+  int wdq_slots;          // fp16 tiles in flight (<= MAX_WDQ_SLOTS)
   int scale_tma;          // 1: scales arrive with the ring (rows of K/group fp16 are 16-byte multiples)
   uint64_t wait_budget_ns;
 };
@@ -105,7 +106,7 @@ struct W4Cfg {
   static constexpr int PANEL = 128;
   static constexpr int PACKED_BYTES = PANEL * BK / 2;  // 4 KiB of codes per k-block
   static constexpr int WDQ_BYTES = PANEL * BK * 2;     // 16 KiB fp16 tile
-  static constexpr int WDQ_SLOTS = 6;
+  static constexpr int MAX_WDQ_SLOTS = 6;
   static constexpr int SCALE_BYTES = PANEL * 16;        // 128 rows x 8 scales
   static constexpr int EPI_WARP0 = 2;
   static constexpr int DQ_WARP0 = 6;
@@ -115,27 +116,27 @@ struct W4Cfg {
   static constexpr int BAR_BYTES = 512;
 
   static int ring_stage_bytes(int m_pad) { return PACKED_BYTES + SCALE_BYTES + m_pad * 128; }
-  static int smem_bytes(int m_pad, int stages) {
-    return 1024 + WDQ_SLOTS * WDQ_BYTES + stages * ring_stage_bytes(m_pad) + BAR_BYTES;
+  static int smem_bytes(int m_pad, int stages, int wdq_slots) {
+    return 1024 + wdq_slots * WDQ_BYTES + stages * ring_stage_bytes(m_pad) + BAR_BYTES;
   }
 };
 
-__global__ void __launch_bounds__(W4Cfg::THREADS, 1)
+__global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     gemm_relu_w4a16_skinny_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
                                   const __grid_constant__ CUtensorMap tmap_s, const W4Params p) {
   using Cfg = W4Cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* wdq_smem = smem;                                               // WDQ_SLOTS x 16 KiB (1024-aligned)
-  uint8_t* a_smem = wdq_smem + Cfg::WDQ_SLOTS * Cfg::WDQ_BYTES;           // stages x a_stage_bytes (1024-aligned)
+  uint8_t* wdq_smem = smem;                                               // wdq_slots x 16 KiB (1024-aligned)
+  uint8_t* a_smem = wdq_smem + p.wdq_slots * Cfg::WDQ_BYTES;              // stages x a_stage_bytes (1024-aligned)
   uint8_t* packed_smem = a_smem + p.stages * p.a_stage_bytes;             // stages x 4 KiB
   uint8_t* scale_smem = packed_smem + p.stages * Cfg::PACKED_BYTES;       // stages x 2 KiB
   uint64_t* bars = reinterpret_cast<uint64_t*>(scale_smem + p.stages * Cfg::SCALE_BYTES);
   uint64_t* full_bar = bars;                                // [MAX_STAGES]: codes + activations landed
   uint64_t* empty_bar = bars + Cfg::MAX_STAGES;             // [MAX_STAGES]: the MMAs read the activations
-  uint64_t* wdq_full_bar = bars + 2 * Cfg::MAX_STAGES;      // [WDQ_SLOTS]: fp16 tile written
-  uint64_t* wdq_empty_bar = wdq_full_bar + Cfg::WDQ_SLOTS;  // [WDQ_SLOTS]: the MMAs read the fp16 tile
-  uint64_t* acc_full_bar = wdq_empty_bar + Cfg::WDQ_SLOTS;
+  uint64_t* wdq_full_bar = bars + 2 * Cfg::MAX_STAGES;          // [MAX_WDQ_SLOTS]: fp16 tile written
+  uint64_t* wdq_empty_bar = wdq_full_bar + Cfg::MAX_WDQ_SLOTS;  // [MAX_WDQ_SLOTS]: the MMAs read the fp16 tile
+  uint64_t* acc_full_bar = wdq_empty_bar + Cfg::MAX_WDQ_SLOTS;
   uint64_t* mma_done_bar = acc_full_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -154,7 +155,7 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int s = 0; s < Cfg::WDQ_SLOTS; ++s) {
+    for (int s = 0; s < p.wdq_slots; ++s) {
       mbar_init(&wdq_full_bar[s], Cfg::DQ_WARPS);
       mbar_init(&wdq_empty_bar[s], 1);
     }
@@ -214,8 +215,8 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int i = 0; i < my_blocks; ++i) {
-        const int slot = i % Cfg::WDQ_SLOTS;
-        const uint32_t slot_phase = static_cast<uint32_t>((i / Cfg::WDQ_SLOTS) & 1);
+        const int slot = i % p.wdq_slots;
+        const uint32_t slot_phase = static_cast<uint32_t>((i / p.wdq_slots) & 1);
         if (!mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 0x63) ||
             !mbar_wait(&wdq_full_bar[slot], slot_phase, abort_flag, p.wait_budget_ns, 0x64)) {
           ok = false;
@@ -256,8 +257,8 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     uint32_t phase = 0;
     for (int i = 0; i < my_blocks; ++i) {
       const int kb = kb_lo + i;
-      const int slot = i % Cfg::WDQ_SLOTS;
-      const uint32_t slot_phase = static_cast<uint32_t>((i / Cfg::WDQ_SLOTS) & 1);
+      const int slot = i % p.wdq_slots;
+      const uint32_t slot_phase = static_cast<uint32_t>((i / p.wdq_slots) & 1);
       const bool ready = mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 0x66) &&
                          mbar_wait(&wdq_empty_bar[slot], slot_phase ^ 1u, abort_flag, p.wait_budget_ns, 0x67);
       if (!__all_sync(0xffffffffu, ready)) break;

@@ -968,7 +968,7 @@ constexpr int64_t kW4FusedMaxM = 256;
 bool w4_args_valid(const void* A, const void* Wq, const void* S, const void* C, int64_t M, int64_t N, int64_t K,
                    int32_t group) {
   if (M < 0 || N < 0 || K < 0 || M > INT_MAX || N > INT_MAX || K > INT_MAX) return false;
-  if (group < 32 || group % 32 != 0 || K % 64 != 0 || (K > 0 && K % group != 0)) return false;
+  if (group < 32 || (group & (group - 1)) != 0 || K % 64 != 0 || (K > 0 && K % group != 0)) return false;
   if (M == 0 || N == 0) return true;
   if (!C || (reinterpret_cast<uintptr_t>(C) & 1u)) return false;
   if (K == 0) return true;
@@ -1022,13 +1022,19 @@ tg_status launch_w4a16_fused(const void* A, const void* Wq, const void* S, void*
   p.k_blocks = static_cast<int>(K / Cfg::BK);
   p.a_stage_bytes = static_cast<uint32_t>(p.m_pad * 128);
   const int ring = Cfg::ring_stage_bytes(p.m_pad);
-  int stages = (kMaxSmem - 1024 - Cfg::WDQ_SLOTS * Cfg::WDQ_BYTES - Cfg::BAR_BYTES) / ring;
+  // Two CTAs per SM for small M (each within half the shared memory), one
+  // with a deeper ring otherwise.
+  const bool two_per_sm = tune_int("TG_TUNE_W4_TWO_PER_SM", p.m_pad <= 32 ? 1 : 0) != 0;
+  p.wdq_slots = tune_int("TG_TUNE_W4_WDQ", two_per_sm ? 3 : Cfg::MAX_WDQ_SLOTS);
+  if (p.wdq_slots < 2 || p.wdq_slots > Cfg::MAX_WDQ_SLOTS) return TG_ERR_INVALID_ARG;
+  const int budget = two_per_sm ? 113 * 1024 : kMaxSmem;
+  int stages = (budget - Cfg::smem_bytes(p.m_pad, 0, p.wdq_slots)) / ring;
   const int cap = tune_int("TG_TUNE_W4_STAGES", Cfg::MAX_STAGES);
   if (stages > cap) stages = cap;
   if (stages > Cfg::MAX_STAGES) stages = Cfg::MAX_STAGES;
   if (stages < 2) return TG_ERR_INTERNAL;
   // The fp32 partial [M_pad][128] reuses the rings after the main loop.
-  if (Cfg::WDQ_SLOTS * Cfg::WDQ_BYTES + stages * ring < p.m_pad * Cfg::PANEL * 4) return TG_ERR_INTERNAL;
+  if (p.wdq_slots * Cfg::WDQ_BYTES + stages * ring < p.m_pad * Cfg::PANEL * 4) return TG_ERR_INTERNAL;
   p.stages = stages;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(p.m_pad)) cols <<= 1;
@@ -1038,7 +1044,7 @@ tg_status launch_w4a16_fused(const void* A, const void* Wq, const void* S, void*
   p.wait_budget_ns = wait_budget(p.k_blocks);
   const int panels = static_cast<int>((N + Cfg::PANEL - 1) / Cfg::PANEL);
   if (panels > 65535) return TG_ERR_INVALID_ARG;
-  int splits = tune_int("TG_TUNE_W4_SPLITS", info->sm_count / panels);
+  int splits = tune_int("TG_TUNE_W4_SPLITS", (two_per_sm ? 2 : 1) * info->sm_count / panels);
   splits = splits < 1 ? 1 : (splits > 8 ? 8 : splits);
   if (splits > p.k_blocks) splits = p.k_blocks;
   p.splits = splits;
@@ -1056,7 +1062,7 @@ tg_status launch_w4a16_fused(const void* A, const void* Wq, const void* S, void*
   std::memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(panels), 1);
   cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::smem_bytes(p.m_pad, stages));
+  cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::smem_bytes(p.m_pad, stages, p.wdq_slots));
   cfg.stream = stream;
   LaunchAttrs la;
   la.fill(cfg, static_cast<unsigned>(splits));
@@ -1130,14 +1136,14 @@ tg_status tg_gemm_relu_w4a16(const void* A, const void* Wq, const void* scales, 
 }
 
 int64_t tg_w4a16_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group) {
-  if (M < 0 || N < 0 || K < 0 || group < 32 || group % 32 != 0 || K % 64 != 0 || (K > 0 && K % group != 0))
+  if (M < 0 || N < 0 || K < 0 || group < 32 || (group & (group - 1)) != 0 || K % 64 != 0 || (K > 0 && K % group != 0))
     return -1;
   return tg::w4_workspace_bytes(M, N, K);
 }
 
 tg_status tg_dequant_w4_f16(const void* Wq, const void* scales, void* W, int64_t N, int64_t K, int32_t group,
                             void* stream) {
-  if (N < 0 || K < 0 || group < 32 || group % 32 != 0 || K % 64 != 0 || (K > 0 && K % group != 0))
+  if (N < 0 || K < 0 || group < 32 || (group & (group - 1)) != 0 || K % 64 != 0 || (K > 0 && K % group != 0))
     return TG_ERR_INVALID_ARG;
   if (N == 0 || K == 0) return TG_OK;
   if (!Wq || !scales || !W || !tg::aligned16(Wq) || !tg::aligned16(W) ||
