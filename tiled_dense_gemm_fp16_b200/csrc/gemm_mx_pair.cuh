@@ -292,10 +292,10 @@ __global__ void __launch_bounds__(MxPairCfg<KIND>::THREADS, 1)
             tmem_st_32x32b_x4(sfb_tmem + 8 * a + 4, vb1);
           }
         }
-        tmem_st_wait();
+        tmem_st_wait();  // the stores are complete before the signal
         tcgen05_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full_bar[stage]), 0));
+        if (lane == 0) mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(&sf_full_bar[stage]), 0));
         if (++stage == Cfg::STAGES) {
           stage = 0;
           phase ^= 1u;

@@ -372,6 +372,15 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 
+// As mbar_arrive_cluster without release semantics, for signals that order
+// only tcgen05 work: the arriving thread has completed it (tcgen05.wait::st)
+// and fenced it (tcgen05.fence::before_thread_sync), and the waiter fences
+// with tcgen05.fence::after_thread_sync.  A cluster-scope release here costs
+// each arrival a fence that measured about 1 us.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // Thread-block clusters and distributed shared memory
 // ----------------------------------------------------------------------------
