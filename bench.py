@@ -245,10 +245,68 @@ def cpu_baseline(A, B, target_s: float):
 # Reference arm: the oracle on host cores, per step a bounded row sample
 # ---------------------------------------------------------------------------
 
+def run_reference_variant(args):
+    """The oracle on a bounded sample of a block-scaled or W4A16 workload (rank 0 only)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    if args.workload in inputs.W4_WORKLOADS:
+        M, N, K, group, seed = inputs.W4_WORKLOADS[args.workload]
+        A, Wq, S = inputs.w4_operands(M, N, K, group, seed, "uniform")
+        metric, shape = W4_METRIC, (M, N, K)
+        run = lambda rows: oracle.gemm_relu_w4a16(A[:rows], Wq, S, group, nthreads=cores)
+        limit = M
+        config = {"workload": args.workload, "M": M, "N": N, "K": K, "group": group, "seed": seed}
+    else:
+        kind = "mxf8" if args.workload in inputs.MX_WORKLOADS else "nvf4"
+        m_sizes, N, K, seed = (inputs.MX_WORKLOADS if kind == "mxf8" else inputs.NVF4_WORKLOADS)[args.workload]
+        ops = (inputs.mx_operands(list(m_sizes), N, K, seed, "normal") if kind == "mxf8"
+               else inputs.nvf4_operands(list(m_sizes), N, K, seed, "codes"))
+        A, SFA, B, SFB = ops
+        fn = oracle.gemm_mxf8_grouped if kind == "mxf8" else oracle.gemm_nvf4_grouped
+        metric, shape = (MX_METRIC if kind == "mxf8" else NVF4_METRIC), (sum(m_sizes), N, K)
+        run = lambda rows: fn(A[:rows], SFA[:rows], B[:1], SFB[:1], [rows], [0], N, K, nthreads=cores)
+        limit = m_sizes[0]
+        config = {"workload": args.workload, "groups": len(m_sizes), "m_sizes": list(m_sizes), "N": N, "K": K,
+                  "seed": seed}
+    rows = 1
+    while True:
+        t0 = time.perf_counter()
+        run(rows)
+        dt = time.perf_counter() - t0
+        if dt >= budget or rows >= limit:
+            break
+        rows = min(limit, max(rows * 2, int(rows * budget / max(dt, 1e-3) * 0.9)))
+    for _ in range(args.warmup):
+        run(rows)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        run(rows)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = inputs.flops(rows, shape[1], shape[2]) * args.steps / total / 1e12
+    sample = f"each step computes {rows} rows of group 0 ({rows} x {shape[1]} x {shape[2]}) with the CPU oracle"
+    line = {
+        "impl": "reference", "metric": metric, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 sum (oracle)",
+        "data": "synthetic", "config": config,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    if (args.workload in inputs.MX_WORKLOADS or args.workload in inputs.NVF4_WORKLOADS
+            or args.workload in inputs.W4_WORKLOADS):
+        return run_reference_variant(args)
     import oracle
     name, M, N, K, A, B = workload_problem(args.workload)
     cores = os.cpu_count() or 1
