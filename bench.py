@@ -47,6 +47,7 @@ KERNEL_SOURCES = {
     "nvf4": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
     "w4a16": [_CSRC + "gemm_w4a16.cuh", _CSRC + "ptx.cuh"],
 }
+E2E_MODE = "every step uploads its inputs and downloads its result; two buffer sets overlap the copies with the GEMM"
 MX_METRIC = "MXFP8 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP8 tensor peak"
 NVF4_METRIC = "NVF4 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP4 tensor peak"
 W4_METRIC = "W4A16 GEMM+ReLU TFLOP/s (1×B200) and % of its roofline (HBM for decode, tensor for large M)"
@@ -67,7 +68,7 @@ def parse_args():
     ap.add_argument("--workspace", choices=["auto", "none"], default="auto",
                     help="auto: give the library the scratch bytes it asks for (repack path for "
                          "operands TMA cannot describe), allocated by torch outside the timed region")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -226,6 +227,46 @@ def _rows_for_budget(oracle, A, B, cores, budget_s):
     if rows >= cores:
         rows = (rows // cores) * cores
     return max(1, min(M, rows))
+
+
+def pipelined_e2e(dev, compute_stream, hosts, make_inputs, out_shape, out_dtype, call, steps):
+    """End-to-end time per step through the library call, with every step's inputs copied from
+    pinned host memory and its result copied back.  Two device buffer sets let step i+1's
+    uploads (copy stream) and step i-1's download (second copy stream) overlap step i's GEMM;
+    events order each set's reuse.  Returns milliseconds per step (steps after one untimed step)."""
+    import torch
+    sets = [make_inputs() for _ in range(2)]
+    outs = [torch.empty(out_shape, dtype=out_dtype, device=dev) for _ in range(2)]
+    houts = [torch.empty(out_shape, dtype=out_dtype).pin_memory() for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    freed = [None, None]          # set k may be overwritten once its GEMM and download are done
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(steps + 1):
+        k = i % 2
+        if i == 1:
+            start.record(up)
+        if freed[k] is not None:
+            up.wait_event(freed[k])
+        with torch.cuda.stream(up):
+            for d_, h_ in zip(sets[k], hosts):
+                d_.copy_(h_, non_blocking=True)
+        loaded = ev()
+        loaded.record(up)
+        compute_stream.wait_event(loaded)
+        with torch.cuda.stream(compute_stream):
+            call(*sets[k], outs[k])
+        done = ev()
+        done.record(compute_stream)
+        down.wait_event(done)
+        with torch.cuda.stream(down):
+            houts[k].copy_(outs[k], non_blocking=True)
+        fin = ev()
+        fin.record(down)
+        freed[k] = fin
+    end.record(down)
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(end) / steps
 
 
 def cpu_baseline(A, B, target_s: float):
@@ -505,24 +546,11 @@ def run_ours(args):
 
     value = aggregate_throughput(world, flops, step_ms)
 
-    # End to end through the C ABI from pinned host buffers: H2D of A and B,
-    # the call, D2H of C, every step.
-    Ah = torch.from_numpy(A).pin_memory()
-    Bh = torch.from_numpy(B).pin_memory()
-    Ch = torch.empty((M, N), dtype=torch.float16).pin_memory()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for i in range(args.e2e_steps + 1):
-            if i == 1:
-                e0.record(stream)
-            Ad.copy_(Ah, non_blocking=True)
-            Bd.copy_(Bh, non_blocking=True)
-            call(Ad, Bd, Cd)
-            Ch.copy_(Cd, non_blocking=True)
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    # End to end through the C ABI from pinned host buffers: every step copies
+    # A and B in and C out, pipelined over two buffer sets (pipelined_e2e).
+    hosts = [torch.from_numpy(A).pin_memory(), torch.from_numpy(B).pin_memory()]
+    e2e_ms = pipelined_e2e(dev, stream, hosts, lambda: [torch.empty_like(Ad), torch.empty_like(Bd)], (M, N),
+                           torch.float16, call, args.e2e_steps)
     if dist is not None:
         e2e_ms = max_over_ranks(dist, e2e_ms, dev)
     e2e_value = aggregate_throughput(world, flops, e2e_ms)
@@ -552,7 +580,7 @@ def run_ours(args):
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
                      "kernel_ms": kern_avg_ms},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * (M * K + K * N),
-                "d2h_bytes_per_step": 2 * M * N, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": 2 * M * N, "ms_per_step": e2e_ms, "mode": E2E_MODE},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": sampler.summary(),
     }
@@ -676,20 +704,16 @@ def run_ours_mx(args):
     value = aggregate_throughput(world, flops, step_ms)
 
     hosts = [torch.from_numpy(x).pin_memory() for x in (A, B, sfa_b, sfb_b)]
-    devs = [Ad, Bd, SFAd, SFBd]
-    Ch = torch.empty((rows, N), dtype=torch.bfloat16).pin_memory()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for i in range(args.e2e_steps + 1):
-            if i == 1:
-                e0.record(stream)
-            for d_, h_ in zip(devs, hosts):
-                d_.copy_(h_, non_blocking=True)
-            call()
-            Ch.copy_(Cd, non_blocking=True)
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+
+    def call_sets(a, b, sa, sb, c):
+        fn = tg.gemm_mxf8_grouped_raw if kind == "mxf8" else tg.gemm_nvf4_grouped_raw
+        extra = (0, 0, False) if kind == "mxf8" else (1.0, False)
+        st = fn(a.data_ptr(), sa.data_ptr(), b.data_ptr(), sb.data_ptr(), c.data_ptr(), m_sizes, N, K, *extra, sh)
+        if st != tg.Status.OK:
+            raise tg.TGError(st, f"tg_gemm_{kind}_grouped")
+
+    e2e_ms = pipelined_e2e(dev, stream, hosts, lambda: [torch.empty_like(x) for x in (Ad, Bd, SFAd, SFBd)],
+                           (rows, N), torch.bfloat16, call_sets, args.e2e_steps)
     if dist is not None:
         e2e_ms = max_over_ranks(dist, e2e_ms, dev)
 
@@ -717,7 +741,7 @@ def run_ours_mx(args):
                      "peak_source": f"{peak_src} cuBLAS bf16 burst peak x {ratio:g} (nominal dense ratio to bf16)",
                      "kernel_ms": kern_ms},
         "e2e": {"value": aggregate_throughput(world, flops, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": 2 * rows * N, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": 2 * rows * N, "ms_per_step": e2e_ms, "mode": E2E_MODE},
         "gpu_launches": args.steps,
         "clocks": sampler.summary(),
     }
@@ -798,22 +822,9 @@ def run_ours_w4(args):
         raise SystemExit(f"device error in timed region: {tg.status_string(st)} 0x{word:x}")
     value = aggregate_throughput(world, flops, step_ms)
 
-    Ah, Wh, Sh = (torch.from_numpy(x).pin_memory() for x in (A, Wq, S))
-    Ch = torch.empty((M, N), dtype=torch.float16).pin_memory()
-    a, w, s_, c = sets[0]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for i in range(args.e2e_steps + 1):
-            if i == 1:
-                e0.record(stream)
-            a.copy_(Ah, non_blocking=True)
-            w.copy_(Wh, non_blocking=True)
-            s_.copy_(Sh, non_blocking=True)
-            call(a, w, s_, c)
-            Ch.copy_(c, non_blocking=True)
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    hosts = [torch.from_numpy(x).pin_memory() for x in (A, Wq, S)]
+    e2e_ms = pipelined_e2e(dev, stream, hosts, lambda: [torch.empty_like(x) for x in sets[0][:3]], (M, N),
+                           torch.float16, call, args.e2e_steps)
     if dist is not None:
         e2e_ms = max_over_ranks(dist, e2e_ms, dev)
 
@@ -841,7 +852,7 @@ def run_ours_w4(args):
         "roofline": roof,
         "e2e": {"value": aggregate_throughput(world, flops, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": A.nbytes + Wq.nbytes + S.nbytes, "d2h_bytes_per_step": 2 * M * N,
-                "ms_per_step": e2e_ms},
+                "ms_per_step": e2e_ms, "mode": E2E_MODE},
         "gpu_launches": args.steps * (1 if fused else 2),
         "clocks": sampler.summary(),
     }
