@@ -71,6 +71,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cublas", action="store_true",
+                    help="also time torch.relu(torch.matmul(A, B)) (cuBLAS) on the same operands, as context")
     return ap.parse_args()
 
 
@@ -584,6 +586,24 @@ def run_ours(args):
         "gpu_launches": args.steps * launches_per_step,
         "clocks": sampler.summary(),
     }
+    if args.cublas and not linear:
+        # Context only (a library GEMM, not this path): the same operand sets,
+        # events around the whole region, as for our kernel.
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                a_, b_, _ = sets[i % len(sets)]
+                torch.relu(torch.matmul(a_, b_))
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            c0.record(stream)
+            for i in range(args.steps):
+                a_, b_, _ = sets[i % len(sets)]
+                torch.relu(torch.matmul(a_, b_))
+            c1.record(stream)
+        torch.cuda.synchronize(dev)
+        cms = c0.elapsed_time(c1) / args.steps
+        line["context_cublas"] = {"op": "torch.relu(torch.matmul(A, B))", "ms_per_step": cms,
+                                  "tflops": flops / (cms * 1e-3) / 1e12}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(A, B, args.cpu_seconds)
     if rank == 0:

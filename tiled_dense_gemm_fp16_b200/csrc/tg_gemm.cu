@@ -898,7 +898,7 @@ tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B,
         info->mx_pair_attr[KIND] = true;
       }
     }
-    p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 8);
+    p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 16);
     if (p.group_m < 1) p.group_m = 1;
     p.num_tiles = static_cast<int>(pair_tiles);
     p.idesc = blockscaled_idesc<KIND>(PairCfg::PAIR_M, a_format, b_format);
@@ -927,7 +927,7 @@ tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B,
       info->mx_attr[KIND] = true;
     }
   }
-  p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 8);
+  p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 16);
   if (p.group_m < 1) p.group_m = 1;
   p.num_tiles = static_cast<int>(single_tiles);
   p.idesc = blockscaled_idesc<KIND>(Cfg::BM, a_format, b_format);
