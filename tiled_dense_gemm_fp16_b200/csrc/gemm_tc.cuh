@@ -109,6 +109,32 @@ __device__ __forceinline__ void load_bias16(const __half* bias, int col, int N, 
     b[e] = (col + e < N) ? __half2float(__ushort_as_half(__ldg(s16 + e))) : 0.0f;
 }
 
+// 8 bias values bias[col .. col + 8) as fp32 (0 past N or without bias): the
+// narrower form of load_bias16 for epilogues short of registers.
+__device__ __forceinline__ void load_bias8(const __half* bias, int col, int N, float (&b)[8]) {
+  if (bias == nullptr) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) b[e] = 0.0f;
+    return;
+  }
+  const __half* src = bias + col;
+  if (col + 8 <= N && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[q]));
+      b[2 * q] = f.x;
+      b[2 * q + 1] = f.y;
+    }
+    return;
+  }
+  const unsigned short* s16 = reinterpret_cast<const unsigned short*>(src);
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    b[e] = (col + e < N) ? __half2float(__ushort_as_half(__ldg(s16 + e))) : 0.0f;
+}
+
 // relu_pack_f16x2 of (a + bias_a, b + bias_b): the bias is added to the fp32
 // accumulator with one fp32 addition before ReLU.
 __device__ __forceinline__ uint32_t relu_pack_f16x2_bias(uint32_t a, uint32_t b, float ba, float bb) {

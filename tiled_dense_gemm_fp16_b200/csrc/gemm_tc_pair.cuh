@@ -22,7 +22,12 @@
 //     on the even CTA's "accumulator empty" barrier;
 //   * per SM, each 64-deep k-block moves 32 KiB from L2 for 128 x 256 x 64
 //     MACs at BN = 256 (two thirds of what the single-CTA 128 x 256 tile
-//     needs) and 48 KiB for 128 x 512 x 64 MACs at BN = 512 (one half).
+//     needs) and 48 KiB for 128 x 512 x 64 MACs at BN = 512 (one half);
+//   * BN = 512 drains the accumulator 32 columns per TMEM round trip into
+//     registers as packed fp16, frees it, then stages C through shared
+//     memory in 32 x 32 boxes that TMA writes out (rows of C 16-byte
+//     aligned), so each warp's stores leave as whole 64-byte row pieces
+//     instead of one 16-byte piece per row and store instruction.
 // Every wait is bounded; a cluster barrier brackets the kernel so that no
 // CTA exits while its peer may still touch its shared memory or barriers.
 #pragma once
@@ -59,21 +64,44 @@ struct TcPairCfg {
   static constexpr int NUM_ACC = (BN == 256) ? 2 : 1;
   static constexpr int TMEM_COLS = 512;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + BAR_BYTES;
+  // C staging of the BN = 512 epilogue: per epilogue warp two 2 KiB buffers,
+  // each one 32-row x 32-column fp16 box of C with the 64-byte swizzle,
+  // written by the warp and stored by TMA while the warp fills the other.
+  static constexpr int C_BOX_COLS = 32;
+  static constexpr int C_BUF_BYTES = 32 * C_BOX_COLS * 2;
+  static constexpr int C_STAGE_BYTES = (BN == 512) ? EPI_WARPS * 2 * C_BUF_BYTES : 0;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + C_STAGE_BYTES + BAR_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA");
   static_assert(BN == 256 || BN == 512, "pair tile width");
   static_assert(NUM_ACC * BN <= TMEM_COLS, "TMEM columns");
 };
 
+// One 16-byte shared-memory store.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// tma_store_2d with an L2 cache policy for the written lines.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, const void* smem_src, int x, int y,
+                                                  uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
 template <int STAGES, int BN>
 __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
     gemm_relu_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                             const TcParams p) {
+                             const __grid_constant__ CUtensorMap tmap_c, const TcParams p) {
   using Cfg = TcPairCfg<STAGES, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* a_smem = smem;
   uint8_t* b_smem = smem + Cfg::STAGES * Cfg::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES));
+  uint8_t* c_stage = smem + Cfg::STAGES * (Cfg::A_BYTES + Cfg::B_BYTES);  // 1 KiB aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(c_stage + Cfg::C_STAGE_BYTES);
   uint64_t* full_bar = bars;                         // used in the even CTA
   uint64_t* empty_bar = bars + Cfg::STAGES;          // per CTA
   uint64_t* acc_full_bar = bars + 2 * Cfg::STAGES;   // per CTA
@@ -103,6 +131,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
     fence_mbarrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
+    if (Cfg::C_STAGE_BYTES > 0 && p.c_aligned) tma_prefetch_desc(&tmap_c);
   }
   if (warp == Cfg::MMA_WARP) {
     tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
@@ -285,30 +314,67 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
         // warp, and only then store, so the stores overlap the next tile's MMAs.
         uint32_t h[Cfg::EPI_COLS / 2];
 #pragma unroll
-        for (int c = 0; c < Cfg::EPI_COLS / 16; ++c) {
-          uint32_t r[16];  // 16 columns at a time keeps the register peak low
-          tmem_ld_32x32b_x16(taddr + c * 16, r);
+        for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
+          uint32_t r[32];  // 32 columns per TMEM round trip
+          tmem_ld_32x32b_x32(taddr + c * 32, r);
           tmem_ld_wait();
           if (p.bias != nullptr) {
-            float bv[16];
-            load_bias16(p.bias, n_blk * Cfg::BN + col_base + c * 16, p.N, bv);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) h[c * 8 + e] = relu_pack_f16x2_bias(r[2 * e], r[2 * e + 1], bv[2 * e], bv[2 * e + 1]);
+            for (int part = 0; part < 4; ++part) {
+              float bv[8];
+              load_bias8(p.bias, n_blk * Cfg::BN + col_base + c * 32 + part * 8, p.N, bv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                h[c * 16 + part * 4 + e] =
+                    relu_pack_f16x2_bias(r[part * 8 + 2 * e], r[part * 8 + 2 * e + 1], bv[2 * e], bv[2 * e + 1]);
+            }
           } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) h[c * 8 + e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
+            for (int e = 0; e < 16; ++e) h[c * 16 + e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
           }
         }
         tcgen05_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
+        if (p.c_aligned) {
+          // Rows of C start on 16-byte boundaries: stage 32 x 32 boxes (lane
+          // = row, 64 bytes each, 16-byte chunks swizzled by bits 1..2 of the
+          // row) and let TMA write them; rows and columns past C are clipped
+          // by the tensor map.  Each buffer is refilled only once the store
+          // issued two boxes earlier has read it.
+          const int y0 = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM + quad * 32;
+          uint8_t* wbuf = c_stage + (warp - Cfg::EPI_WARP0) * 2 * Cfg::C_BUF_BYTES;
+          const uint64_t pol = p.store_streaming ? l2_policy_evict_first() : l2_policy_evict_normal();
+          if (y0 < p.M) {
 #pragma unroll
-        for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
-          const int col0 = n_blk * Cfg::BN + col_base + c * 32;
-          uint32_t hc[16];
+            for (int c = 0; c < Cfg::EPI_COLS / Cfg::C_BOX_COLS; ++c) {
+              const int col0 = n_blk * Cfg::BN + col_base + c * Cfg::C_BOX_COLS;
+              if (col0 >= p.N) break;
+              uint8_t* buf = wbuf + (c & 1) * Cfg::C_BUF_BYTES;
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              const uint32_t row_addr = smem_u32(buf) + lane * 64;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) hc[e] = h[c * 16 + e];
-          if (row_ok && col0 < p.N) store_row_chunk(crow, col0, p.N, hc, p.c_aligned != 0, p.store_streaming != 0);
+              for (int q = 0; q < 4; ++q)
+                st_shared_v4(row_addr + ((q ^ ((lane >> 1) & 3)) << 4), h[c * 16 + 4 * q], h[c * 16 + 4 * q + 1],
+                             h[c * 16 + 4 * q + 2], h[c * 16 + 4 * q + 3]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d_hint(&tmap_c, buf, col0, y0, pol);
+                bulk_commit_group();
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
+            const int col0 = n_blk * Cfg::BN + col_base + c * 32;
+            uint32_t hc[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) hc[e] = h[c * 16 + e];
+            if (row_ok && col0 < p.N) store_row_chunk(crow, col0, p.N, hc, false, p.store_streaming != 0);
+          }
         }
       } else {
         // Double-buffered accumulator: the next tile's MMAs already run in
@@ -339,6 +405,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
     }
   }
 
+  if (Cfg::C_STAGE_BYTES > 0 && warp >= Cfg::EPI_WARP0 && lane == 0) bulk_wait_group<0>();  // C is written
   tcgen05_fence_before_sync();
   __syncthreads();
   cluster_sync();  // the pair is done with each other's shared memory and barriers

@@ -307,9 +307,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Row-major fp16 matrix of rows x cols with a row stride of `ld` elements
 // (ld * 2 a multiple of 16); box = box_cols x box_rows, 128-byte swizzle
-// (box_cols * 2 must be 128).  Columns past `cols` read as zero.
+// (box_cols * 2 must be 128; with the 64-byte swizzle, 64).  Columns past
+// `cols` read as zero, and stores past them are dropped.
 bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_cols,
-               int box_rows) {
+               int box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -317,7 +318,7 @@ bool encode_2d(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, i
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estride[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estride,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -457,8 +458,13 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
       info->tc_pair_attr |= kAttrBit;
     }
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   if (!encode_operands(o, &ta, &tb, Cfg::BM, 128)) return TG_ERR_LAUNCH;
+  // C for the TMA-store epilogue of the 256 x 512 tile: 32 x 32 boxes.
+  std::memset(&tc, 0, sizeof tc);
+  if (Cfg::C_STAGE_BYTES > 0 && o.c_aligned &&
+      !encode_2d(&tc, o.C, o.M, o.N, o.ldc, Cfg::C_BOX_COLS, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return TG_ERR_LAUNCH;
   TcParams p;
   fill_tc_params(p, o);
   p.m_tiles = static_cast<int>((M + Cfg::PAIR_M - 1) / Cfg::PAIR_M);
@@ -482,7 +488,7 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
   cfg.stream = stream;
   LaunchAttrs la;
   la.fill(cfg, 2);
-  if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, tc, p) != cudaSuccess) {
     cudaGetLastError();
     return TG_ERR_LAUNCH;
   }
