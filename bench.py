@@ -850,6 +850,9 @@ def run_ours_w4(args):
 
     peaks, peak_src = load_peaks()
     fused = need == 0
+    kind = tg.w4a16_kernel(M, N, K, group)
+    path_name = {tg.W4Kernel.DECODE: "w4a16 decode (register dequantization, mma.sync, cluster split-K)",
+                 tg.W4Kernel.FUSED: "w4a16 fused (tcgen05)"}.get(kind, "dequantize + tc (fp16 GEMM)")
     if fused:
         roof = {"bound": "hbm", "achieved": nbytes / (kern_ms * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
                 "unit": "GB/s", "peak_source": f"{peak_src} STREAM-copy HBM bandwidth"}
@@ -865,7 +868,7 @@ def run_ours_w4(args):
         "vs_baseline": None, "dtype": "f16 activations x 4-bit weights (fp16 scales per group), fp32 accumulate",
         "data": "synthetic",
         "config": {"workload": args.workload, "M": M, "N": N, "K": K, "group": group, "seed": seed,
-                   "path": "w4a16 fused" if fused else "dequantize + tc (fp16 GEMM)",
+                   "path": path_name,
                    "workspace_bytes": need, "min_bytes": nbytes,
                    "l2": (f"rotating {len(sets)} operand copies" if len(sets) > 1 else "inputs larger than L2"),
                    "parallelism": f"dp{world} independent problems" if world > 1 else "1 GPU"},

@@ -361,7 +361,9 @@ TG_API int64_t tg_nvf4_scale_bytes(int64_t rows, int64_t K);
  * K/2 bytes, element 2i of a row in the low nibble of byte i.  scales: N x
  * (K/group) fp16, row-major.  C: M x N fp16, row-major.  group is a power of
  * two >= 32 that divides K; K % 64 == 0.
- * M <= 256 runs one fused kernel that streams the packed weight once.  Larger
+ * M <= 256 runs one fused kernel that streams the packed weight once (for
+ * M <= 16 and K % 256 == 0, K <= 16384, a decode kernel that dequantizes in
+ * registers; tg_w4a16_kernel tells which).  Larger
  * M dequantizes the weight into `workspace` (tg_w4a16_workspace_size bytes,
  * 16-byte aligned, 2*N*K rounded up) and runs the fp16 tensor-core GEMM.
  * Errors (TG_ERR_INVALID_ARG, nothing enqueued): bad sizes or group, A or Wq
@@ -371,6 +373,20 @@ TG_API int64_t tg_nvf4_scale_bytes(int64_t rows, int64_t K);
 TG_API tg_status tg_gemm_relu_w4a16(const void *A, const void *Wq, const void *scales, void *C, int64_t M,
                                     int64_t N, int64_t K, int32_t group, void *stream, void *workspace,
                                     int64_t workspace_bytes);
+
+/* The kernels tg_gemm_relu_w4a16 runs for these sizes (host logic only). */
+typedef enum tg_w4a16_kernel_kind {
+    TG_W4_INVALID = -1,  /* the sizes or the group are invalid                 */
+    TG_W4_NONE = 0,      /* nothing to compute: M == 0 or N == 0, or K == 0 (C = +0) */
+    TG_W4_DECODE = 1,    /* M <= 16, K % 256 == 0, K <= 16384: dequantization in
+                            registers feeding warp-level MMAs, split-K over a
+                            cluster of up to 8 CTAs reduced in shared memory */
+    TG_W4_FUSED = 2,     /* M <= 256: the tcgen05 kernel with a dequantization
+                            stage in front of the MMA                         */
+    TG_W4_DEQUANT_GEMM = 3 /* larger M: dequantize into the workspace, then
+                            the fp16 tensor-core GEMM                        */
+} tg_w4a16_kernel_kind;
+TG_API int tg_w4a16_kernel(int64_t M, int64_t N, int64_t K, int32_t group);
 
 /* Workspace bytes tg_gemm_relu_w4a16 needs for these sizes (0 for M <= 256),
  * or -1 if the sizes are invalid. */

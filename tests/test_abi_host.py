@@ -142,6 +142,29 @@ def test_workspace_size_and_repack_choice():
     assert tg.select_path_ws(A0, B0, C0, 4096, 4096, 4096, need) == Path.TC_PAIR512
 
 
+def test_w4a16_kernel_choice():
+    K4 = tg.W4Kernel
+    assert tg.w4a16_kernel(16, 8192, 8192, 128) == K4.DECODE      # the decode workload
+    assert tg.w4a16_kernel(1, 1, 256, 32) == K4.DECODE
+    assert tg.w4a16_kernel(1, 1, 384, 32) == K4.FUSED               # K % 256 != 0
+    assert tg.w4a16_kernel(16, 8192, 16384, 128) == K4.DECODE     # K / 8 = 2048: the longest slice
+    assert tg.w4a16_kernel(16, 8192, 32768, 128) == K4.FUSED      # slices would be longer
+    assert tg.w4a16_kernel(16, 8192, 8192 + 128, 128) == K4.FUSED  # K % 256 != 0
+    assert tg.w4a16_kernel(17, 8192, 8192, 128) == K4.FUSED
+    assert tg.w4a16_kernel(256, 8192, 8192, 128) == K4.FUSED
+    assert tg.w4a16_kernel(257, 8192, 8192, 128) == K4.DEQUANT_GEMM
+    assert tg.w4a16_kernel(0, 8192, 8192, 128) == K4.NONE
+    assert tg.w4a16_kernel(4, 8, 0, 32) == K4.NONE
+    assert tg.w4a16_kernel(4, 8, 128, 48) == K4.INVALID          # group not a power of two
+    assert tg.w4a16_kernel(4, 8, 96, 32) == K4.INVALID           # K % 64 != 0
+    assert tg.w4a16_kernel(-1, 8, 128, 32) == K4.INVALID
+
+
+def test_w4a16_decode_switch(monkeypatch):
+    monkeypatch.setenv("TG_TUNE_W4_DECODE", "0")
+    assert tg.w4a16_kernel(16, 8192, 8192, 128) == tg.W4Kernel.FUSED
+
+
 def test_workspace_argument_checks():
     M, N, K = 300, 301, 299
     need = tg.workspace_size(A0, B0, C0, M, N, K)

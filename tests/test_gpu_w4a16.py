@@ -108,3 +108,44 @@ def test_workloads_sampled_rows(name):
     rows = sample_rows(M, n=16, seed=seed) if M > 16 else np.arange(M)
     want = oracle.gemm_relu_w4a16(np.ascontiguousarray(A[rows]), Wq, S, group)
     assert_close(C[torch.from_numpy(np.asarray(rows)).cuda()].cpu().numpy(), want, f"{name} rows")
+
+
+# ---------------------------------------------------------------------------
+# M <= 16 with K % 256 == 0 takes the decode kernel (register dequantization,
+# warp-level MMAs, cluster split-K); the shapes below cover its splits of K
+# (8 down to 1), ragged N, every scale group from 32 to K, and K that it does
+# not take (K % 256 != 0, or slices longer than it holds), which falls back
+# to the tcgen05 kernel.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M", [1, 3, 16])
+@pytest.mark.parametrize("N,K,group", [(130, 256, 32), (1000, 768, 128), (257, 3072, 1024), (640, 16384, 64),
+                                       (520, 1280, 256), (130, 384, 128), (384, 32768, 256)])
+def test_decode_integer_bitexact(M, N, K, group):
+    import tiled_dense_gemm_fp16_b200 as tg
+    want = tg.W4Kernel.DECODE if (K % 256 == 0 and K <= 16384) else tg.W4Kernel.FUSED
+    assert tg.w4a16_kernel(M, N, K, group) == want
+    got, (A, Wq, S) = run_w4(M, N, K, group, "int", seed=3 * M + N + K)
+    assert_bitexact(got, oracle.gemm_relu_w4a16(A, Wq, S, group), f"W4A16 decode {(M, N, K, group)}")
+
+
+@pytest.mark.parametrize("M,N,K,group", [(16, 8192, 1024, 128), (7, 1536, 8192, 32)])
+def test_decode_float(M, N, K, group):
+    got, (A, Wq, S) = run_w4(M, N, K, group, "uniform", seed=M + 5 * K)
+    assert_close(got, oracle.gemm_relu_w4a16(A, Wq, S, group), f"W4A16 decode float {(M, N, K, group)}")
+
+
+@pytest.mark.parametrize("M,N,K,group", [(1, 520, 1024, 32), (16, 1000, 512, 128), (9, 4096, 4096, 128)])
+def test_tcgen05_kernel_still_serves_small_m(monkeypatch, M, N, K, group):
+    # With the decode kernel switched off, the tcgen05 fused kernel takes these shapes.
+    import tiled_dense_gemm_fp16_b200 as tg
+    monkeypatch.setenv("TG_TUNE_W4_DECODE", "0")
+    assert tg.w4a16_kernel(M, N, K, group) == tg.W4Kernel.FUSED
+    got, (A, Wq, S) = run_w4(M, N, K, group, "int", seed=M * 11 + K)
+    assert_bitexact(got, oracle.gemm_relu_w4a16(A, Wq, S, group), f"W4A16 tcgen05 {(M, N, K, group)}")
+
+
+def test_decode_deterministic():
+    a, _ = run_w4(16, 2048, 8192, 128, "uniform", seed=77)
+    b, _ = run_w4(16, 2048, 8192, 128, "uniform", seed=77)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))

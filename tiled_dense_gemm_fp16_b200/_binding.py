@@ -92,6 +92,7 @@ EXPORTS = (
     "tg_nvf4_scale_bytes",
     "tg_gemm_relu_w4a16",
     "tg_w4a16_workspace_size",
+    "tg_w4a16_kernel",
     "tg_dequant_w4_f16",
 )
 
@@ -151,6 +152,8 @@ def _bind(lib):
     lib.tg_gemm_relu_w4a16.restype = i32
     lib.tg_w4a16_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int32]
     lib.tg_w4a16_workspace_size.restype = i64
+    lib.tg_w4a16_kernel.argtypes = [i64, i64, i64, ctypes.c_int32]
+    lib.tg_w4a16_kernel.restype = ctypes.c_int
     lib.tg_dequant_w4_f16.argtypes = [vp, vp, vp, i64, i64, ctypes.c_int32, vp]
     lib.tg_dequant_w4_f16.restype = i32
     return lib
@@ -467,6 +470,19 @@ def nvf4_grouped(A, SFA, B, SFB, m_sizes, alpha=1.0, relu=False, out=None, strea
 
 def w4a16_workspace_size(M: int, N: int, K: int, group: int) -> int:
     return int(lib().tg_w4a16_workspace_size(M, N, K, group))
+
+
+class W4Kernel(enum.IntEnum):
+    INVALID = -1
+    NONE = 0
+    DECODE = 1
+    FUSED = 2
+    DEQUANT_GEMM = 3
+
+
+def w4a16_kernel(M: int, N: int, K: int, group: int) -> "W4Kernel":
+    """The kernels tg_gemm_relu_w4a16 runs for these sizes (host logic only)."""
+    return W4Kernel(int(lib().tg_w4a16_kernel(M, N, K, group)))
 
 
 def gemm_relu_w4a16_raw(A: int, Wq: int, S: int, C: int, M: int, N: int, K: int, group: int, stream: int = 0,

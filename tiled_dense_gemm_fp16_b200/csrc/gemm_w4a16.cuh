@@ -45,21 +45,29 @@ struct DequantParams {
 };
 
 // Eight 4-bit codes (a 32-bit word, element 2i in the low nibble of byte i)
-// as eight fp16 values (q - 8) * s, packed two per word, low element first.
-// Masking the word with 0x000F000F pairs elements i and i + 4 in the two
-// halves; each half becomes 1024 + q (the code in the mantissa of 1024.0),
-// 1032 is subtracted exactly, the multiply rounds once, and byte permutes
-// restore the element order.
-__device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2) {
+// as eight fp16 values (q - 8) * s, in the pairs the arithmetic yields:
+// v[i] = (e_i, e_{i+4}), low half first.  Masking the word with 0x000F000F
+// pairs elements i and i + 4 in the two halves; each half becomes 1024 + q
+// (the code in the mantissa of 1024.0), 1032 is subtracted exactly, and the
+// multiply by the scale rounds once to nearest even.
+__device__ __forceinline__ void dequant8_pairs(uint32_t w, __half2 s2, uint32_t (&v)[4]) {
   const uint32_t mask = 0x000F000Fu, magic = 0x64006400u;  // fp16 1024.0 in both halves
-  uint32_t v[4] = {(w & mask) | magic, ((w >> 4) & mask) | magic, ((w >> 8) & mask) | magic,
-                   ((w >> 12) & mask) | magic};  // (e0,e4), (e1,e5), (e2,e6), (e3,e7)
+  v[0] = (w & mask) | magic;
+  v[1] = ((w >> 4) & mask) | magic;
+  v[2] = ((w >> 8) & mask) | magic;
+  v[3] = ((w >> 12) & mask) | magic;
   const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const __half2 x = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v[i]), bias), s2);
     v[i] = *reinterpret_cast<const uint32_t*>(&x);
   }
+}
+
+// The same eight values in element order, packed two per word.
+__device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2) {
+  uint32_t v[4];
+  dequant8_pairs(w, s2, v);
   return make_uint4(__byte_perm(v[0], v[1], 0x5410), __byte_perm(v[2], v[3], 0x5410),
                     __byte_perm(v[0], v[1], 0x7632), __byte_perm(v[2], v[3], 0x7632));
 }
@@ -359,6 +367,224 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     tcgen05_fence_after_sync();
     tmem_dealloc(tmem_base, p.tmem_cols);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Decode kernel (M <= 16): dequantization in registers, warp-level MMAs
+// ---------------------------------------------------------------------------
+// A decode step is bound by streaming the packed weight from HBM, so this
+// kernel keeps every step of a warp's work in its own registers: no shared
+// memory round trip for the dequantized weight and no hand-off to an MMA
+// thread.  A warp owns 32 weight rows (4 groups of 8, the n side of
+// mma.sync.m16n8k16); per 256-deep step of K the 4 lanes that share a row
+// load its 128 bytes (256 codes) as two 64-byte halves, 16 bytes per lane
+// per half, so every load instruction reads whole 32-byte sectors.  The codes are dequantized with the arithmetic of dequant8_pairs and
+// fed straight into the MMA (fp16 operands, fp32 accumulation) as the B
+// fragment.  The pairs come out as (e_i, e_{i+4}); instead of reordering
+// them, the k order of the MMA is permuted the same way on the activation
+// side, where byte permutes build the A fragments from the CTA's slice of
+// the activations (rows 0..15, zero past M), copied once into shared memory
+// by cp.async in row order with the 16-byte chunks of each 128-byte line
+// XOR-swizzled so that the fragment reads are conflict-free.  A sum over k
+// is the same sum in any order, so only the fp32 rounding order changes.
+//
+// Grid (S, N/128): a cluster of S CTAs along K shares a 128-column panel;
+// each CTA (4 warps) streams its K/S slice with two steps of codes and
+// scales in flight per warp, then the cluster adds its S fp32 partials
+// through distributed shared memory in rank order (deterministic) and
+// writes ReLU(sum) rounded to fp16.
+struct W4DecodeParams {
+  const __half* A;    // M x K
+  const uint8_t* Wq;  // N x K/2
+  const __half* S;    // N x K/group
+  __half* C;          // M x N
+  int M, N, K;
+  int group_shift;    // log2(group)
+  int k_split;        // K per CTA: a multiple of kW4DecodeStepK, at most kW4DecodeMaxSplit
+};
+
+constexpr int kW4DecodeThreads = 128;
+constexpr int kW4DecodePanel = 128;      // columns per CTA: 4 warps x 32
+constexpr int kW4DecodeStepK = 256;      // K per main-loop step: 128 bytes of each weight row
+constexpr int kW4DecodeMaxSplit = 2048;  // K per CTA (its A fragments take k_split * 32 bytes)
+
+__host__ __device__ constexpr int w4_decode_smem_bytes(int k_split) { return k_split * 32 + 16 * kW4DecodePanel * 4; }
+
+// Byte offset of the 16-byte chunk kc (8 activations) of row r in the CTA's
+// activation slice: rows of k_split * 2 bytes, and inside each 128-byte line
+// the chunk position XOR (2 (line mod 2) + (r mod 2)).  The lanes of a
+// quarter warp read rows g, g + 1 at chunks 4t + q (+ a multiple of 16):
+// positions q and q + 4 of two consecutive lines, which the XOR spreads over
+// the eight 16-byte bank groups.
+__device__ __forceinline__ uint32_t w4_act_offset(int r, int kc, int k_split) {
+  const int line = kc >> 3;
+  const int pos = (kc & 7) ^ (((line & 1) << 1) | (r & 1));
+  return static_cast<uint32_t>(r * k_split * 2 + line * 128 + pos * 16);
+}
+
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void mma_m16n8k16_f16_f32(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+
+// Codes and scales of one step for one lane: per row group, 8 words (64
+// codes: k = 128 u + 32 t + 8 q + i of the step) and the scales of its
+// halves u = 0, 1 (low and high half).
+struct W4DecodeStep {
+  uint4 w[4][2];
+  __half2 s[4];
+};
+
+__global__ void __launch_bounds__(kW4DecodeThreads, 4) gemm_relu_w4a16_decode_kernel(const W4DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const uint32_t act = smem_u32(smem);                            // [16][k_split] fp16, swizzled
+  float* part = reinterpret_cast<float*>(smem + p.k_split * 32);  // [16][128] fp32
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t split = cluster_ctarank();
+  const int splits = static_cast<int>(gridDim.x);
+  const int k0 = static_cast<int>(blockIdx.x) * p.k_split;
+  const int n_panel = static_cast<int>(blockIdx.y) * kW4DecodePanel;
+  const int nsteps = p.k_split / kW4DecodeStepK;
+  const int64_t row_bytes = p.K / 2;
+  const int64_t scales_per_row = p.K >> p.group_shift;
+
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  // The activation slice: every copy in flight at once, no registers held.
+  {
+    const int chunks = p.k_split / 8;
+    for (int idx = threadIdx.x; idx < 16 * chunks; idx += kW4DecodeThreads) {
+      const int r = idx / chunks, kc = idx - r * chunks;
+      const __half* src = p.A + static_cast<int64_t>(r < p.M ? r : 0) * p.K + k0 + 8 * kc;
+      cp_async_16(act + w4_act_offset(r, kc, p.k_split), src, r < p.M ? 16u : 0u);
+    }
+  }
+
+  // This lane's weight rows (one per 8-column group; a row past N reads row
+  // N - 1 instead, whose columns are never stored) and the byte where its
+  // first 32 codes of step 0 start.
+  const int n_lane = n_panel + warp * 32 + g;
+  const uint8_t* wbase = p.Wq + k0 / 2 + 16 * t;
+  auto row_of = [&](int gi) { return static_cast<int64_t>(min(n_lane + gi * 8, p.N - 1)); };
+  // Step c's codes and scales (nothing is read past the slice).
+  auto load = [&](int c, W4DecodeStep& d) {
+    if (c >= nsteps) return;
+    const int kq = k0 + kW4DecodeStepK * c + 32 * t;
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) {
+      const int64_t n = row_of(gi);
+      const uint8_t* src = wbase + n * row_bytes + c * 128;
+      d.w[gi][0] = __ldg(reinterpret_cast<const uint4*>(src));
+      d.w[gi][1] = __ldg(reinterpret_cast<const uint4*>(src + 64));
+      const __half* srow = p.S + n * scales_per_row;
+      d.s[gi] = __halves2half2(__ldg(srow + (kq >> p.group_shift)), __ldg(srow + ((kq + 128) >> p.group_shift)));
+    }
+  };
+  W4DecodeStep cur, nxt;
+  load(0, cur);
+  load(1, nxt);
+
+  cp_async_commit_wait_all();
+  __syncthreads();
+
+  float acc[4][4];
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[gi][e] = 0.0f;
+
+#pragma unroll 1
+  for (int c = 0; c < nsteps; ++c) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        // Word q of each group gives k-steps 2q ((e0,e4), (e1,e5)) and 2q + 1
+        // ((e2,e6), (e3,e7)); the activations of rows g and g + 8 at the same
+        // 8 k build the A fragments of both (words 0/2 from row g, 1/3 from
+        // row g + 8).
+        const int kc = 32 * c + 16 * u + 4 * t + q;
+        const uint4 lo = lds128(act + w4_act_offset(g, kc, p.k_split));
+        const uint4 hi = lds128(act + w4_act_offset(g + 8, kc, p.k_split));
+        const uint4 af0 = make_uint4(__byte_perm(lo.x, lo.z, 0x5410), __byte_perm(hi.x, hi.z, 0x5410),
+                                     __byte_perm(lo.x, lo.z, 0x7632), __byte_perm(hi.x, hi.z, 0x7632));
+        const uint4 af1 = make_uint4(__byte_perm(lo.y, lo.w, 0x5410), __byte_perm(hi.y, hi.w, 0x5410),
+                                     __byte_perm(lo.y, lo.w, 0x7632), __byte_perm(hi.y, hi.w, 0x7632));
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          const uint4& w = cur.w[gi][u];
+          const uint32_t word = q == 0 ? w.x : q == 1 ? w.y : q == 2 ? w.z : w.w;
+          uint32_t bv[4];
+          dequant8_pairs(word, u == 0 ? __low2half2(cur.s[gi]) : __high2half2(cur.s[gi]), bv);
+          mma_m16n8k16_f16_f32(acc[gi], af0, bv[0], bv[1]);
+          mma_m16n8k16_f16_f32(acc[gi], af1, bv[2], bv[3]);
+        }
+      }
+    }
+    cur = nxt;
+    load(c + 2, nxt);
+  }
+
+  // This CTA's fp32 partial: rows g and g + 8, columns 2t, 2t + 1 of each group.
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) {
+    const int col = warp * 32 + gi * 8 + 2 * t;
+    *reinterpret_cast<float2*>(part + g * kW4DecodePanel + col) = make_float2(acc[gi][0], acc[gi][1]);
+    *reinterpret_cast<float2*>(part + (g + 8) * kW4DecodePanel + col) = make_float2(acc[gi][2], acc[gi][3]);
+  }
+  cluster_sync();  // every partial of the cluster is written
+
+  // CTA `split` finishes columns [split * 128 / S, +128 / S): four at a time,
+  // the S partials added in rank order.
+  const int cols = kW4DecodePanel / splits;
+  const int quads = 16 * cols / 4;
+  for (int i = threadIdx.x; i < quads; i += kW4DecodeThreads) {
+    const int r = (i * 4) / cols;
+    const int cl = static_cast<int>(split) * cols + (i * 4) % cols;
+    if (r >= p.M) continue;
+    const uint32_t local = smem_u32(part + r * kW4DecodePanel + cl);
+    float4 v[8];  // all remote reads in flight before the adds (splits <= 8)
+#pragma unroll
+    for (int rk = 0; rk < 8; ++rk)
+      if (rk < splits) v[rk] = ld_shared_cluster_f4(mapa_shared(local, static_cast<uint32_t>(rk)));
+    float4 sum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int rk = 0; rk < 8; ++rk) {
+      if (rk < splits) {
+        sum.x += v[rk].x;
+        sum.y += v[rk].y;
+        sum.z += v[rk].z;
+        sum.w += v[rk].w;
+      }
+    }
+    const float o[4] = {sum.x, sum.y, sum.z, sum.w};
+    __half* crow = p.C + static_cast<int64_t>(r) * p.N;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int n = n_panel + cl + e;
+      if (n < p.N) crow[n] = __float2half_rn(o[e] > 0.0f ? o[e] : 0.0f);
+    }
+  }
+  cluster_sync();  // no CTA leaves while a peer may still read its partial
 }
 
 }  // namespace tg

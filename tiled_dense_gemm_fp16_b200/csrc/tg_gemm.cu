@@ -50,6 +50,7 @@ struct DeviceInfo {
   bool mx_attr[2] = {false, false};       // per block-scaled kind
   bool mx_pair_attr[2] = {false, false};
   bool w4_attr = false;
+  bool w4_decode_attr = false;
   void* static_ws = nullptr;  // device address of g_static_workspace on this device
 };
 
@@ -971,10 +972,14 @@ tg_status run_nvf4_grouped(const void* A, const void* SFA, const void* B, const 
 
 constexpr int64_t kW4FusedMaxM = 256;
 
+bool w4_sizes_valid(int64_t M, int64_t N, int64_t K, int32_t group) {
+  if (M < 0 || N < 0 || K < 0 || M > INT_MAX || N > INT_MAX || K > INT_MAX) return false;
+  return !(group < 32 || (group & (group - 1)) != 0 || K % 64 != 0 || (K > 0 && K % group != 0));
+}
+
 bool w4_args_valid(const void* A, const void* Wq, const void* S, const void* C, int64_t M, int64_t N, int64_t K,
                    int32_t group) {
-  if (M < 0 || N < 0 || K < 0 || M > INT_MAX || N > INT_MAX || K > INT_MAX) return false;
-  if (group < 32 || (group & (group - 1)) != 0 || K % 64 != 0 || (K > 0 && K % group != 0)) return false;
+  if (!w4_sizes_valid(M, N, K, group)) return false;
   if (M == 0 || N == 0) return true;
   if (!C || (reinterpret_cast<uintptr_t>(C) & 1u)) return false;
   if (K == 0) return true;
@@ -1079,6 +1084,60 @@ tg_status launch_w4a16_fused(const void* A, const void* Wq, const void* S, void*
   return TG_OK;
 }
 
+// Splits of K for the decode kernel (M <= 16): the most (up to 8) that keep
+// each CTA's slice a multiple of kW4DecodeStepK and at most
+// kW4DecodeMaxSplit; 0 when the shape does not suit it (K % 256 != 0, K too
+// long, or turned off).
+int w4_decode_splits(int64_t M, int64_t N, int64_t K) {
+  if (M > 16 || K <= 0 || K % kW4DecodeStepK != 0 || (N + kW4DecodePanel - 1) / kW4DecodePanel > 65535) return 0;
+  if (!tune_int("TG_TUNE_W4_DECODE", 1)) return 0;
+  for (int s = 8; s >= 1; s >>= 1)
+    if (K % (kW4DecodeStepK * s) == 0 && K / s <= kW4DecodeMaxSplit) return s;
+  return 0;
+}
+
+tg_status launch_w4a16_decode(const void* A, const void* Wq, const void* S, void* C, int64_t M, int64_t N,
+                              int64_t K, int32_t group, int splits, cudaStream_t stream, DeviceInfo* info) {
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!info->w4_decode_attr) {
+      if (cudaFuncSetAttribute(gemm_relu_w4a16_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               w4_decode_smem_bytes(kW4DecodeMaxSplit)) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      info->w4_decode_attr = true;
+    }
+  }
+  W4DecodeParams p;
+  std::memset(&p, 0, sizeof p);
+  p.A = static_cast<const __half*>(A);
+  p.Wq = static_cast<const uint8_t*>(Wq);
+  p.S = static_cast<const __half*>(S);
+  p.C = static_cast<__half*>(C);
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  int shift = 0;
+  while ((1 << shift) < group) ++shift;
+  p.group_shift = shift;
+  p.k_split = static_cast<int>(K / splits);
+  const int panels = static_cast<int>((N + kW4DecodePanel - 1) / kW4DecodePanel);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(splits), static_cast<unsigned>(panels), 1);
+  cfg.blockDim = dim3(kW4DecodeThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(w4_decode_smem_bytes(p.k_split));
+  cfg.stream = stream;
+  LaunchAttrs la;
+  la.fill(cfg, static_cast<unsigned>(splits));
+  if (cudaLaunchKernelEx(&cfg, gemm_relu_w4a16_decode_kernel, p) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
+}
+
 tg_status run_w4a16(const void* A, const void* Wq, const void* S, void* C, int64_t M, int64_t N, int64_t K,
                     int32_t group, void* stream_ptr, void* ws, int64_t ws_bytes) {
   if (!w4_args_valid(A, Wq, S, C, M, N, K, group)) return TG_ERR_INVALID_ARG;
@@ -1096,6 +1155,8 @@ tg_status run_w4a16(const void* A, const void* Wq, const void* S, void* C, int64
     }
     return TG_OK;
   }
+  if (const int splits = w4_decode_splits(M, N, K))
+    return launch_w4a16_decode(A, Wq, S, C, M, N, K, group, splits, stream, info);
   if (M <= kW4FusedMaxM) return launch_w4a16_fused(A, Wq, S, C, M, N, K, group, stream, info);
   // Large M: dequantize into the workspace, then the fp16 tensor-core GEMM
   // with the weight in the N x K layout.
@@ -1139,6 +1200,13 @@ tg_status tg_gemm_nvf4_grouped(const void* A, const void* SFA, const void* B, co
 tg_status tg_gemm_relu_w4a16(const void* A, const void* Wq, const void* scales, void* C, int64_t M, int64_t N,
                               int64_t K, int32_t group, void* stream, void* workspace, int64_t workspace_bytes) {
   return tg::run_w4a16(A, Wq, scales, C, M, N, K, group, stream, workspace, workspace_bytes);
+}
+
+int tg_w4a16_kernel(int64_t M, int64_t N, int64_t K, int32_t group) {
+  if (!tg::w4_sizes_valid(M, N, K, group)) return TG_W4_INVALID;
+  if (M == 0 || N == 0 || K == 0) return TG_W4_NONE;
+  if (tg::w4_decode_splits(M, N, K) > 0) return TG_W4_DECODE;
+  return M <= tg::kW4FusedMaxM ? TG_W4_FUSED : TG_W4_DEQUANT_GEMM;
 }
 
 int64_t tg_w4a16_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group) {
