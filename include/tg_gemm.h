@@ -106,12 +106,16 @@ TG_API tg_status tg_gemm_relu_f16_path(const void *A, const void *B, void *C, in
 
 /*
  * C = ReLU(A . B) with a caller-provided device workspace.  Identical to
- * tg_gemm_relu_f16 except when TMA cannot describe A or B (a row stride that
- * is not a multiple of 16 bytes, or a base that is not 16-byte aligned): then,
- * if `workspace_bytes` >= tg_workspace_size(...), those operands are first
- * copied into zero-padded rows in the workspace (path TG_PATH_REPACK) and a
- * TMA kernel runs on the copies, which is several times faster than the edge
- * mode.  With less workspace the call behaves like tg_gemm_relu_f16.
+ * tg_gemm_relu_f16 except in two cases (path TG_PATH_REPACK):
+ *   - TMA cannot describe A or B (a row stride that is not a multiple of 16
+ *     bytes, or a base that is not 16-byte aligned) and the workspace holds
+ *     their copies: they are first copied into zero-padded rows in the
+ *     workspace and a TMA kernel runs on the copies, several times faster
+ *     than the edge mode;
+ *   - the rows of C are not 16-byte aligned, M > 256, and the workspace also
+ *     holds a padded C (tg_workspace_size covers it): the GEMM writes that
+ *     copy with its aligned stores and a realigning copy moves it into C.
+ * With less workspace the call behaves like tg_gemm_relu_f16.
  *   workspace        device pointer, 256-byte aligned, not overlapping A, B
  *                    or C; owned by the caller and free to reuse once the
  *                    call's work on `stream` has finished (may be NULL if
@@ -134,9 +138,11 @@ TG_API tg_status tg_gemm_relu_f16_ws(const void *A, const void *B, void *C, int6
  * device buffer of TG_STATIC_WORKSPACE_BYTES (16 MiB) that the library holds
  * on every GPU where it is loaded, until the process exits.  It calls no
  * allocating routine.  The caller still passes A, B and C.
- *   - Problems whose repack would need more than TG_STATIC_WORKSPACE_BYTES
- *     (tg_workspace_size > 16 MiB) are rejected with TG_ERR_TOO_LARGE and
- *     nothing is enqueued; aligned problems need no scratch and always run.
+ *   - Problems whose copies of A and B would need more than
+ *     TG_STATIC_WORKSPACE_BYTES are rejected with TG_ERR_TOO_LARGE and
+ *     nothing is enqueued; problems whose A and B TMA can describe need no
+ *     scratch and always run.  The padded C of tg_gemm_relu_f16_ws is used
+ *     only when it fits in the buffer beside those copies.
  *   - The first call on a device looks up the buffer's device address for
  *     that device (with that device current); make that first call before
  *     any stream capture.
@@ -217,9 +223,12 @@ TG_API int tg_select_path_ex(const void *A, const void *B, const void *C, int64_
                              const tg_gemm_options *options, int64_t workspace_bytes);
 
 /*
- * Workspace bytes tg_gemm_relu_f16_ws needs to take the repack path for these
- * arguments: 0 when no repacking is needed, -1 for invalid arguments.  Host
- * logic only.
+ * Workspace bytes tg_gemm_relu_f16_ws needs for its fastest path with these
+ * arguments: copies of A and B when TMA cannot describe them, plus, when the
+ * rows of C are not 16-byte aligned and a tensor-core kernel runs (M > 256),
+ * a padded C that the GEMM writes and a realigning copy moves into C.  Less
+ * workspace still takes the repack path as long as the A and B copies fit.
+ * 0 when neither applies, -1 for invalid arguments.  Host logic only.
  */
 TG_API int64_t tg_workspace_size(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K);
 

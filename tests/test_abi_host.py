@@ -124,21 +124,29 @@ def test_no_device_is_reported_not_faked():
 
 
 def test_workspace_size_and_repack_choice():
-    # TMA-describable operands need no workspace, whatever C's alignment.
-    assert tg.workspace_size(A0, B0, C0, 8192, 8192, 8192) == 0
-    assert tg.workspace_size(A0, B0, C0 + 2, 512, 512, 512) == 0
-    assert tg.select_path(A0, B0, C0 + 2, 512, 512, 512) != Path.TC_EDGE
-    # Odd K pads A to K rounded up to 8; odd N pads B; each copy 256-byte aligned.
     up = lambda x: (x + 255) // 256 * 256
+    # TMA-describable operands and 16-byte aligned rows of C need no workspace.
+    assert tg.workspace_size(A0, B0, C0, 8192, 8192, 8192) == 0
+    # C's rows not 16-byte aligned: the fastest path writes a padded C
+    # (M x N rounded up to 8) in the workspace; without one it still runs.
+    assert tg.workspace_size(A0, B0, C0 + 2, 512, 512, 512) == up(2 * 512 * 512)
+    assert tg.select_path(A0, B0, C0 + 2, 512, 512, 512) == Path.TC_PAIR
+    assert tg.select_path_ws(A0, B0, C0 + 2, 512, 512, 512, up(2 * 512 * 512)) == Path.REPACK
+    assert tg.select_path_ws(A0, B0, C0 + 2, 512, 512, 512, up(2 * 512 * 512) - 1) == Path.TC_PAIR
+    assert tg.workspace_size(A0, B0, C0, 512, 509, 512) == 2 * up(2 * 512 * 512)    # odd N: B copy and C copy
+    assert tg.workspace_size(A0, B0, C0 + 2, 64, 512, 512) == 0                      # the small-M kernel
+    # Odd K pads A to K rounded up to 8; odd N pads B, and C (odd N) too; each copy 256-byte aligned.
     M, N, K = 3001, 5003, 1021
-    assert tg.workspace_size(A0, B0, C0, M, N, K) == up(2 * M * 1024) + up(2 * K * 5008)
-    assert tg.workspace_size(A0, B0, C0, 8191, 129, 8193) == up(2 * 8191 * 8200) + up(2 * 8193 * 136)
-    assert tg.workspace_size(A0, B0, C0, 64, 64, 100) == up(2 * 64 * 104)          # only A
+    ab = up(2 * M * 1024) + up(2 * K * 5008)
+    assert tg.workspace_size(A0, B0, C0, M, N, K) == ab + up(2 * M * 5008)
+    assert tg.workspace_size(A0, B0, C0, 8191, 129, 8193) == up(2 * 8191 * 8200) + up(2 * 8193 * 136) + up(2 * 8191 * 136)
+    assert tg.workspace_size(A0, B0, C0, 64, 64, 100) == up(2 * 64 * 104)          # only A (small M: no C copy)
     assert tg.workspace_size(A0 + 2, B0, C0, 64, 64, 64) == up(2 * 64 * 64)        # misaligned A base
     assert tg.workspace_size(A0, B0, C0, -1, 4, 4) == -1
     need = tg.workspace_size(A0, B0, C0, M, N, K)
     assert tg.select_path_ws(A0, B0, C0, M, N, K, need) == Path.REPACK
-    assert tg.select_path_ws(A0, B0, C0, M, N, K, need - 1) == Path.TC_EDGE
+    assert tg.select_path_ws(A0, B0, C0, M, N, K, ab) == Path.REPACK                # A and B copies only
+    assert tg.select_path_ws(A0, B0, C0, M, N, K, ab - 1) == Path.TC_EDGE
     assert tg.select_path_ws(A0, B0, C0, 4096, 4096, 4096, need) == Path.TC_PAIR512
 
 

@@ -144,7 +144,8 @@ def test_repack_integer_bitexact(M, N, K):
 
 @pytest.mark.parametrize("offsets", [(1, 0, 0), (0, 3, 0), (0, 0, 5), (7, 2, 1), (0, 0, 4)])
 def test_unaligned_bases(offsets):
-    """Misaligned A or B go through the repack path; a misaligned C alone keeps the TMA kernels."""
+    """Misaligned A or B go through the repack path; a misaligned C alone keeps the TMA kernels without a
+    workspace and, with one, has the GEMM write a padded C that a realigning copy moves into place."""
     for (M, N, K) in [(300, 264, 136), (64, 520, 72)]:
         A, B = inputs.operands(M, N, K, "int", seed=sum(offsets) + M)
         ref = oracle.gemm_relu_f16(A, B)
@@ -152,6 +153,21 @@ def test_unaligned_bases(offsets):
             got, guards = run_gpu(A, B, offsets=offsets, workspace=ws)
             assert guards, (offsets, M, N, K, ws)
             assert_bitexact(got, ref, f"offsets {offsets} {(M, N, K)} ws={ws}")
+
+
+@pytest.mark.parametrize("c_off", [1, 2, 3, 7])
+@pytest.mark.parametrize("M,N,K", [(520, 1032, 264), (777, 1001, 136), (300, 8, 64), (1100, 2053, 512)])
+def test_padded_c_copy_back(M, N, K, c_off):
+    """C's rows not 16-byte aligned, with a workspace: the GEMM writes a padded C and the realigning copy
+    writes every element of C (interior 16-byte blocks and the ragged ends of each row) and nothing else."""
+    import tiled_dense_gemm_fp16_b200 as tg
+    A, B = inputs.operands(M, N, K, "int", seed=M + N + c_off)
+    # K % 8 == 0 keeps A and B TMA-describable when N % 8 == 0, so only C is copied.
+    if K % 8 == 0 and N % 8 == 0:
+        assert tg.select_path_ws(16, 1 << 40, (1 << 41) + 2 * c_off, M, N, K, 1 << 40) == Path.REPACK
+    got, guards = run_gpu(A, B, offsets=(0, 0, c_off), workspace=True)
+    assert guards, (M, N, K, c_off)
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"padded C {(M, N, K)} offset {c_off}")
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 301, 299), (1000, 1001, 1003)])

@@ -1,6 +1,7 @@
 // repack.cuh -- copy a row-major fp16 matrix whose rows are not 16-byte
 // aligned into a row-major copy with rows padded to a multiple of 8 elements
-// (16 bytes), zero in the padding, so that TMA can describe it.
+// (16 bytes), zero in the padding, so that TMA can describe it; and the
+// reverse copy for C (unpad_rows_kernel below).
 //
 // Used by the workspace path of C = ReLU(A . B) for operands whose leading
 // dimension (K for A, N for B) is not a multiple of 8 or whose base address
@@ -63,6 +64,53 @@ __global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
       const uint4 v = plan[u].fast ? edge_realign(lo[u], hi[u], plan[u].shift)
                                    : load_chunk_pred(p.src, p.src_ld, row[u], p.rows, col[u], p.cols);
       *reinterpret_cast<uint4*>(p.dst + static_cast<int64_t>(row[u]) * p.cols_pad + col[u]) = v;
+    }
+  }
+}
+
+// The reverse copy, for C: the GEMM writes a padded copy (rows of cols_pad
+// elements, 16-byte aligned) and this kernel moves it into C, whose rows may
+// start on any 2-byte boundary.  Each thread writes one 16-byte-aligned block
+// of a destination row: its 8 values are read with two aligned 16-byte loads
+// of the padded copy and shifted into place, so every interior store is a
+// whole aligned 16 bytes; the partial blocks at either end of a row are
+// written element by element.  Nothing outside [0, cols) of a row is written,
+// and nothing outside the padded copy is read.
+struct UnpadParams {
+  const __half* src;  // rows x cols_pad, 16-byte aligned
+  __half* dst;        // rows of `cols` elements, row stride dst_ld, 2-byte aligned
+  int64_t dst_ld;
+  int rows, cols, cols_pad;
+  int blocks_per_row;  // cols / 8 + 2: enough 16-byte blocks for any alignment of a row
+  int64_t blocks;      // rows * blocks_per_row
+};
+
+__global__ void __launch_bounds__(256) unpad_rows_kernel(const UnpadParams p) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const __half* src_end = p.src + static_cast<int64_t>(p.rows) * p.cols_pad;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < p.blocks; i += stride) {
+    const int r = static_cast<int>(i / p.blocks_per_row);
+    const int j = static_cast<int>(i - static_cast<int64_t>(r) * p.blocks_per_row);
+    __half* drow = p.dst + static_cast<int64_t>(r) * p.dst_ld;
+    const int a = static_cast<int>((reinterpret_cast<uintptr_t>(drow) & 15u) >> 1);  // elements before the row's first aligned block
+    const int e0 = 8 * j - a;                                                         // first row element of block j
+    if (e0 >= p.cols) continue;
+    const __half* srow = p.src + static_cast<int64_t>(r) * p.cols_pad;
+    if (e0 >= 0 && e0 + 8 <= p.cols) {
+      const uintptr_t s = reinterpret_cast<uintptr_t>(srow + e0);
+      const uintptr_t s0 = s & ~uintptr_t(15);
+      if (s0 + 32 <= reinterpret_cast<uintptr_t>(src_end) || s == s0) {
+        const uint4 lo = __ldg(reinterpret_cast<const uint4*>(s0));
+        const uint4 hi = s == s0 ? lo : __ldg(reinterpret_cast<const uint4*>(s0) + 1);
+        *reinterpret_cast<uint4*>(drow + e0) = edge_realign(lo, hi, static_cast<uint32_t>(s - s0));
+        continue;
+      }
+    }
+    for (int k = 0; k < 8; ++k) {
+      const int e = e0 + k;
+      if (e >= 0 && e < p.cols) drow[e] = srow[e];
     }
   }
 }

@@ -172,34 +172,59 @@ bool c_rows_aligned(const Problem& p) {
   return (reinterpret_cast<uintptr_t>(p.C) & 15u) == 0 && p.ldc % 8 == 0 && (p.batch == 1 || p.sc % 8 == 0);
 }
 
+// The tensor-core kernels store C fastest when its rows start on 16-byte
+// boundaries (whole 16-byte pieces, or TMA boxes); the small-M kernel writes
+// C element by element either way.
+bool c_pad_useful(const Problem& p) {
+  return !c_rows_aligned(p) && !(p.M <= kSkinnyMaxM && !p.a_km);
+}
+
 // Workspace of the repack path: zero-padded copies (rows rounded up to 8
 // elements) of one batch entry of whichever of A and B TMA cannot describe,
-// each 256-byte aligned; batch entries reuse it in stream order.
+// and, with `with_c`, a padded C (M x N rounded up to 8) that the GEMM writes
+// and a realigning copy then moves into C when C's rows are not 16-byte
+// aligned; each 256-byte aligned; batch entries reuse it in stream order.
 struct RepackPlan {
-  bool pad_a = false, pad_b = false;
+  bool pad_a = false, pad_b = false, pad_c = false;
   int64_t kp = 0, np = 0, mp = 0;
-  int64_t off_a = 0, off_b = 0, bytes = 0;
+  int64_t off_a = 0, off_b = 0, off_c = 0, bytes = 0;
 };
 
-RepackPlan repack_plan(const Problem& p) {
+RepackPlan repack_plan(const Problem& p, bool with_c) {
   RepackPlan r;
   r.kp = (p.K + 7) / 8 * 8;
   r.np = (p.N + 7) / 8 * 8;
   r.mp = (p.M + 7) / 8 * 8;
   r.pad_a = !tma_ok_a(p);
   r.pad_b = !tma_ok_b(p);
+  r.pad_c = with_c && c_pad_useful(p);
   auto up256 = [](int64_t x) { return (x + 255) / 256 * 256; };
   const int64_t bytes_a = r.pad_a ? up256(p.a_km ? 2 * p.K * r.mp : 2 * p.M * r.kp) : 0;
   const int64_t bytes_b = r.pad_b ? up256(p.b_nk ? 2 * p.N * r.kp : 2 * p.K * r.np) : 0;
+  const int64_t bytes_c = r.pad_c ? up256(2 * p.M * r.np) : 0;
   r.off_a = 0;
   r.off_b = bytes_a;
-  r.bytes = bytes_a + bytes_b;
+  r.off_c = bytes_a + bytes_b;
+  r.bytes = bytes_a + bytes_b + bytes_c;
   return r;
 }
 
-int64_t workspace_bytes_needed(const Problem& p) {
+// Workspace the call needs at the least (the A and B copies when TMA cannot
+// describe them) and for its fastest path (plus the padded C).
+int64_t repack_bytes_needed(const Problem& p) {
   if (p.M == 0 || p.N == 0 || p.K == 0 || tma_ok(p)) return 0;
-  return repack_plan(p).bytes;
+  return repack_plan(p, false).bytes;
+}
+int64_t workspace_bytes_needed(const Problem& p) {
+  if (p.M == 0 || p.N == 0 || p.K == 0) return 0;
+  return repack_plan(p, true).bytes;
+}
+
+// The repack plan a call with `ws_bytes` of workspace takes: with the padded
+// C when it fits.
+RepackPlan chosen_plan(const Problem& p, int64_t ws_bytes) {
+  const RepackPlan full = repack_plan(p, true);
+  return ws_bytes >= full.bytes ? full : repack_plan(p, false);
 }
 
 bool path_supports(int path, const Problem& p) {
@@ -218,7 +243,7 @@ bool path_supports(int path, const Problem& p) {
     case TG_PATH_SKINNY:
       return tma_ok(p) && p.M <= kSkinnyMaxM && !p.a_km;
     case TG_PATH_REPACK:
-      return !tma_ok(p);
+      return !tma_ok(p) || c_pad_useful(p);
     default:
       return false;
   }
@@ -246,8 +271,9 @@ int pick_tc_kernel(int64_t M, int64_t N, int64_t K, bool c_aligned) {
 }
 
 // The tensor-core kernel that runs on TMA-describable (possibly repacked) operands.
-int inner_path(const Problem& p) {
-  return (p.M <= kSkinnyMaxM && !p.a_km) ? TG_PATH_SKINNY : pick_tc_kernel(p.M, p.N, p.K, c_rows_aligned(p));
+int inner_path(const Problem& p, bool c_padded = false) {
+  return (p.M <= kSkinnyMaxM && !p.a_km) ? TG_PATH_SKINNY
+                                         : pick_tc_kernel(p.M, p.N, p.K, c_padded || c_rows_aligned(p));
 }
 
 // The path a call takes with `ws_bytes` of workspace (-2: invalid arguments).
@@ -259,9 +285,12 @@ int select_path(const Problem& p, int64_t ws_bytes) {
   if (p.M == 0 || p.N == 0) return TG_PATH_NONE;
   if (p.K == 0) return TG_PATH_ZERO;
   if (!tma_ok(p)) {
-    if (ws_bytes >= repack_plan(p).bytes || p.b_nk || p.a_km) return TG_PATH_REPACK;
+    if (ws_bytes >= repack_plan(p, false).bytes || p.b_nk || p.a_km) return TG_PATH_REPACK;
     return TG_PATH_TC_EDGE;
   }
+  // Operands TMA can read, but C's rows are not 16-byte aligned: the GEMM
+  // writes a padded C in the workspace when there is room for it.
+  if (c_pad_useful(p) && ws_bytes >= repack_plan(p, true).bytes) return TG_PATH_REPACK;
   return inner_path(p);
 }
 
@@ -652,6 +681,20 @@ tg_status launch_pad(const void* src, int64_t src_ld, void* dst, int64_t rows, i
   return launch_simple(pad_rows_kernel, rp, rp.chunks, 4, stream, info);
 }
 
+tg_status launch_unpad(const void* src, int64_t cols_pad, void* dst, int64_t dst_ld, int64_t rows, int64_t cols,
+                       cudaStream_t stream, DeviceInfo* info) {
+  UnpadParams up;
+  up.src = static_cast<const __half*>(src);
+  up.dst = static_cast<__half*>(dst);
+  up.dst_ld = dst_ld;
+  up.rows = static_cast<int>(rows);
+  up.cols = static_cast<int>(cols);
+  up.cols_pad = static_cast<int>(cols_pad);
+  up.blocks_per_row = static_cast<int>(cols / 8 + 2);
+  up.blocks = rows * up.blocks_per_row;
+  return launch_simple(unpad_rows_kernel, up, up.blocks, 4, stream, info);
+}
+
 // K == 0: C = ReLU(bias), or +0 without a bias (the empty sum).
 tg_status launch_k_zero(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   if (o.bias == nullptr) {
@@ -682,8 +725,8 @@ tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws
   if (path == TG_PATH_NONE) return TG_OK;
   RepackPlan plan;
   if (path == TG_PATH_REPACK) {
-    plan = repack_plan(p);
-    if (ws == nullptr || ws_bytes < plan.bytes || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    plan = chosen_plan(p, ws ? ws_bytes : 0);
+    if (ws == nullptr || ws_bytes < plan.bytes || plan.bytes == 0 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
       return TG_ERR_INVALID_ARG;
     if (ranges_overlap(ws, plan.bytes, p.A, span_a(p)) || ranges_overlap(ws, plan.bytes, p.B, span_b(p)) ||
         ranges_overlap(ws, plan.bytes, p.C, span_c(p)) || (p.bias && ranges_overlap(ws, plan.bytes, p.bias, 2 * p.N)))
@@ -694,7 +737,7 @@ tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws
   tg_status st = current_device(dev, info);
   if (st != TG_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  const int inner = (path == TG_PATH_REPACK) ? inner_path(p) : path;
+  const int inner = (path == TG_PATH_REPACK) ? inner_path(p, plan.pad_c) : path;
   for (int64_t e = 0; e < p.batch; ++e) {
     Operands o{static_cast<const uint8_t*>(p.A) + 2 * e * p.sa,
                p.lda,
@@ -727,7 +770,18 @@ tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws
         o.B = base + plan.off_b;
         o.ldb = cols_pad;
       }
-      st = launch_path(inner, o, stream, info);
+      if (plan.pad_c) {
+        // The GEMM writes the padded C; the realigning copy moves it into C.
+        void* c_final = o.C;
+        o.C = base + plan.off_c;
+        o.ldc = plan.np;
+        o.c_aligned = true;
+        st = launch_path(inner, o, stream, info);
+        if (st != TG_OK) return st;
+        st = launch_unpad(base + plan.off_c, plan.np, c_final, p.ldc, p.M, p.N, stream, info);
+      } else {
+        st = launch_path(inner, o, stream, info);
+      }
     } else {
       st = launch_path(path, o, stream, info);
     }
@@ -1282,7 +1336,8 @@ tg_status tg_gemm_relu_f16_static_ws(const void* A, const void* B, void* C, int6
                                      void* stream) {
   const tg::Problem p = tg::dense_problem(A, B, C, M, N, K);
   if (!tg::problem_valid(p)) return TG_ERR_INVALID_ARG;
-  const int64_t need = tg::workspace_bytes_needed(p);
+  // Only the copies of A and B are required; a padded C is used when it fits too.
+  const int64_t need = tg::repack_bytes_needed(p);
   if (need > TG_STATIC_WORKSPACE_BYTES) return TG_ERR_TOO_LARGE;
   if (M == 0 || N == 0) return TG_OK;  // empty C: nothing to do
   int dev = 0;
