@@ -64,12 +64,12 @@ struct TcPairCfg {
   static constexpr int NUM_ACC = (BN == 256) ? 2 : 1;
   static constexpr int TMEM_COLS = 512;
   static constexpr int BAR_BYTES = 256;
-  // C staging of the BN = 512 epilogue: per epilogue warp two 2 KiB buffers,
-  // each one 32-row x 32-column fp16 box of C with the 64-byte swizzle,
-  // written by the warp and stored by TMA while the warp fills the other.
+  // C staging of the epilogue: per epilogue warp two 2 KiB buffers, each one
+  // 32-row x 32-column fp16 box of C with the 64-byte swizzle, written by the
+  // warp and stored by TMA while the warp fills the other.
   static constexpr int C_BOX_COLS = 32;
   static constexpr int C_BUF_BYTES = 32 * C_BOX_COLS * 2;
-  static constexpr int C_STAGE_BYTES = (BN == 512) ? EPI_WARPS * 2 * C_BUF_BYTES : 0;
+  static constexpr int C_STAGE_BYTES = EPI_WARPS * 2 * C_BUF_BYTES;
   static constexpr int SMEM_BYTES = 1024 + STAGES * (A_BYTES + B_BYTES) + C_STAGE_BYTES + BAR_BYTES;
   static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA");
   static_assert(BN == 256 || BN == 512, "pair tile width");
@@ -378,14 +378,46 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
         }
       } else {
         // Double-buffered accumulator: the next tile's MMAs already run in
-        // the other buffer; drain 32 columns at a time.
+        // the other buffer; drain 32 columns at a time.  With 16-byte aligned
+        // rows of C each 32 x 32 piece goes out through a swizzled staging
+        // box and a TMA store, as in the single-accumulator epilogue.
+        const int y0 = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM + quad * 32;
+        uint8_t* wbuf = c_stage + (warp - Cfg::EPI_WARP0) * 2 * Cfg::C_BUF_BYTES;
+        const uint64_t pol = p.store_streaming ? l2_policy_evict_first() : l2_policy_evict_normal();
 #pragma unroll 1
         for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(taddr + c * 32, r);
           tmem_ld_wait();
           const int col0 = n_blk * Cfg::BN + col_base + c * 32;
-          if (row_ok && col0 < p.N) {
+          if (p.c_aligned) {
+            if (y0 < p.M && col0 < p.N) {
+              float b0[16], b1[16];
+              load_bias16(p.bias, col0, p.N, b0);
+              load_bias16(p.bias, col0 + 16, p.N, b1);
+              uint32_t hc[16];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                hc[e] = relu_pack_f16x2_bias(r[2 * e], r[2 * e + 1], b0[2 * e], b0[2 * e + 1]);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                hc[8 + e] = relu_pack_f16x2_bias(r[16 + 2 * e], r[16 + 2 * e + 1], b1[2 * e], b1[2 * e + 1]);
+              uint8_t* buf = wbuf + (c & 1) * Cfg::C_BUF_BYTES;
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              const uint32_t row_addr = smem_u32(buf) + lane * 64;
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                st_shared_v4(row_addr + ((q ^ ((lane >> 1) & 3)) << 4), hc[4 * q], hc[4 * q + 1], hc[4 * q + 2],
+                             hc[4 * q + 3]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d_hint(&tmap_c, buf, col0, y0, pol);
+                bulk_commit_group();
+              }
+            }
+          } else if (row_ok && col0 < p.N) {
             float b0[16], b1[16];
             load_bias16(p.bias, col0, p.N, b0);
             load_bias16(p.bias, col0 + 16, p.N, b1);
@@ -395,7 +427,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               hc[8 + e] = relu_pack_f16x2_bias(r[16 + 2 * e], r[16 + 2 * e + 1], b1[2 * e], b1[2 * e + 1]);
-            store_row_chunk(crow, col0, p.N, hc, p.c_aligned != 0, p.store_streaming != 0);
+            store_row_chunk(crow, col0, p.N, hc, false, p.store_streaming != 0);
           }
         }
         tcgen05_fence_before_sync();
@@ -405,7 +437,7 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
     }
   }
 
-  if (Cfg::C_STAGE_BYTES > 0 && warp >= Cfg::EPI_WARP0 && lane == 0) bulk_wait_group<0>();  // C is written
+  if (warp >= Cfg::EPI_WARP0 && lane == 0) bulk_wait_group<0>();  // C is written
   tcgen05_fence_before_sync();
   __syncthreads();
   cluster_sync();  // the pair is done with each other's shared memory and barriers

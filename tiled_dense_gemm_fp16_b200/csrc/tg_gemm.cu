@@ -490,7 +490,7 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
   }
   CUtensorMap ta, tb, tc;
   if (!encode_operands(o, &ta, &tb, Cfg::BM, 128)) return TG_ERR_LAUNCH;
-  // C for the TMA-store epilogue of the 256 x 512 tile: 32 x 32 boxes.
+  // C for the TMA-store epilogue: 32 x 32 boxes.
   std::memset(&tc, 0, sizeof tc);
   if (Cfg::C_STAGE_BYTES > 0 && o.c_aligned &&
       !encode_2d(&tc, o.C, o.M, o.N, o.ldc, Cfg::C_BOX_COLS, 32, CU_TENSOR_MAP_SWIZZLE_64B))
@@ -534,7 +534,6 @@ tg_status launch_tc_pair(const Operands& o, cudaStream_t stream, DeviceInfo* inf
   }
   switch (tune_int("TG_TUNE_PAIR_STAGES", 6)) {
     case 5: return launch_tc_pair_cfg<5, 256>(o, stream, info);
-    case 7: return launch_tc_pair_cfg<7, 256>(o, stream, info);
     default: return launch_tc_pair_cfg<6, 256>(o, stream, info);
   }
 }
