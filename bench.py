@@ -473,10 +473,13 @@ def run_ours(args):
     if ws_bytes > 0:
         chosen = tg.select_path_ws(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, ws_bytes)
 
-    # Kernels per step: one GEMM, plus one row-padding copy per repacked operand.
+    # Kernels per step: one GEMM, plus one row-padding copy per repacked operand
+    # and, when the GEMM writes a padded C (rows of C not 16-byte aligned,
+    # M > 256), the copy that moves it into C.
     launches_per_step = 1
     if chosen == tg.Path.REPACK:
         launches_per_step += int(K % 8 != 0 or Ad.data_ptr() % 16 != 0) + int(N % 8 != 0 or Bd.data_ptr() % 16 != 0)
+        launches_per_step += int((N % 8 != 0 or Cd.data_ptr() % 16 != 0) and M > 256)
 
     lin_opts = tg.options(b_layout=tg.B_NK, bias=bias_d.data_ptr()) if linear else None
     if linear:
