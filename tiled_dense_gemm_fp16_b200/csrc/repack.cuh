@@ -86,31 +86,52 @@ struct UnpadParams {
 };
 
 __global__ void __launch_bounds__(256) unpad_rows_kernel(const UnpadParams p) {
+  constexpr int kUnroll = 4;  // four blocks' loads in flight per thread before any store
   grid_dependency_wait();
   grid_launch_dependents();
-  const __half* src_end = p.src + static_cast<int64_t>(p.rows) * p.cols_pad;
+  const uintptr_t src_end = reinterpret_cast<uintptr_t>(p.src + static_cast<int64_t>(p.rows) * p.cols_pad);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < p.blocks; i += stride) {
-    const int r = static_cast<int>(i / p.blocks_per_row);
-    const int j = static_cast<int>(i - static_cast<int64_t>(r) * p.blocks_per_row);
-    __half* drow = p.dst + static_cast<int64_t>(r) * p.dst_ld;
-    const int a = static_cast<int>((reinterpret_cast<uintptr_t>(drow) & 15u) >> 1);  // elements before the row's first aligned block
-    const int e0 = 8 * j - a;                                                         // first row element of block j
-    if (e0 >= p.cols) continue;
-    const __half* srow = p.src + static_cast<int64_t>(r) * p.cols_pad;
-    if (e0 >= 0 && e0 + 8 <= p.cols) {
-      const uintptr_t s = reinterpret_cast<uintptr_t>(srow + e0);
-      const uintptr_t s0 = s & ~uintptr_t(15);
-      if (s0 + 32 <= reinterpret_cast<uintptr_t>(src_end) || s == s0) {
-        const uint4 lo = __ldg(reinterpret_cast<const uint4*>(s0));
-        const uint4 hi = s == s0 ? lo : __ldg(reinterpret_cast<const uint4*>(s0) + 1);
-        *reinterpret_cast<uint4*>(drow + e0) = edge_realign(lo, hi, static_cast<uint32_t>(s - s0));
-        continue;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < p.blocks;
+       base += stride * kUnroll) {
+    __half* drow[kUnroll];
+    const __half* srow[kUnroll];
+    int e0[kUnroll];
+    uintptr_t s[kUnroll], s0[kUnroll];
+    bool fast[kUnroll], live[kUnroll];
+    uint4 lo[kUnroll], hi[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = base + u * stride;
+      live[u] = i < p.blocks;
+      const int r = live[u] ? static_cast<int>(i / p.blocks_per_row) : 0;
+      const int j = live[u] ? static_cast<int>(i - static_cast<int64_t>(r) * p.blocks_per_row) : 0;
+      drow[u] = p.dst + static_cast<int64_t>(r) * p.dst_ld;
+      srow[u] = p.src + static_cast<int64_t>(r) * p.cols_pad;
+      // Elements before the row's first aligned block, then block j's first element.
+      const int a = static_cast<int>((reinterpret_cast<uintptr_t>(drow[u]) & 15u) >> 1);
+      e0[u] = 8 * j - a;
+      live[u] = live[u] && e0[u] < p.cols;
+      s[u] = reinterpret_cast<uintptr_t>(srow[u] + e0[u]);
+      s0[u] = s[u] & ~uintptr_t(15);
+      fast[u] = live[u] && e0[u] >= 0 && e0[u] + 8 <= p.cols && (s0[u] + 32 <= src_end || s[u] == s0[u]);
+      lo[u] = make_uint4(0u, 0u, 0u, 0u);
+      hi[u] = lo[u];
+      if (fast[u]) {
+        lo[u] = __ldg(reinterpret_cast<const uint4*>(s0[u]));
+        if (s[u] != s0[u]) hi[u] = __ldg(reinterpret_cast<const uint4*>(s0[u]) + 1);
       }
     }
-    for (int k = 0; k < 8; ++k) {
-      const int e = e0 + k;
-      if (e >= 0 && e < p.cols) drow[e] = srow[e];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (!live[u]) continue;
+      if (fast[u]) {
+        *reinterpret_cast<uint4*>(drow[u] + e0[u]) = edge_realign(lo[u], hi[u], static_cast<uint32_t>(s[u] - s0[u]));
+      } else {
+        for (int k = 0; k < 8; ++k) {
+          const int e = e0[u] + k;
+          if (e >= 0 && e < p.cols) drow[u][e] = srow[u][e];
+        }
+      }
     }
   }
 }
