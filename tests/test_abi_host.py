@@ -173,6 +173,27 @@ def test_w4a16_decode_switch(monkeypatch):
     assert tg.w4a16_kernel(16, 8192, 8192, 128) == tg.W4Kernel.FUSED
 
 
+def test_padded_c_with_general_layouts():
+    up = lambda x: (x + 255) // 256 * 256
+    M, N, K = 1000, 1001, 512      # A and B describable by TMA in every layout below; C rows of 2002 bytes
+    for opts, b_copy in [(tg.options(), up(2 * K * 1008)),                     # B K x N: row of 1001 -> padded
+                         (tg.options(b_layout=tg.B_NK), 0),                     # B N x K: rows of K, aligned
+                         (tg.options(a_layout=tg.A_KM, ldb=1008), 0)]:          # A K x M (M % 8 == 0), B padded ld
+        need = tg.workspace_size_ex(A0, B0, C0, M, N, K, opts)
+        assert need == b_copy + up(2 * M * 1008), (opts.b_layout, opts.a_layout)
+        assert tg.select_path_ex(A0, B0, C0, M, N, K, opts, need) == Path.REPACK
+        # Without room for the padded C, describable operands keep the tensor-core kernels.
+        if b_copy == 0:
+            assert tg.select_path_ex(A0, B0, C0, M, N, K, opts, need - 1) in (Path.TC, Path.TC_PAIR, Path.TC_PAIR512)
+    # 16-byte aligned rows of C (ldc a multiple of 8) need no copy of C.
+    assert tg.workspace_size_ex(A0, B0, C0, M, N, K, tg.options(b_layout=tg.B_NK, ldc=1008)) == 0
+    # Strided batches: one padded C serves every entry in turn.
+    o = tg.options(b_layout=tg.B_NK, batch=3, stride_a=M * K, stride_b=N * K, stride_c=M * N + 3)
+    assert tg.workspace_size_ex(A0, B0, C0, M, N, K, o) == up(2 * M * 1008)
+    # Small M keeps the small-M kernel, which writes C element by element anyway.
+    assert tg.workspace_size_ex(A0, B0, C0, 200, N, K, tg.options(b_layout=tg.B_NK)) == 0
+
+
 def test_workspace_argument_checks():
     M, N, K = 300, 301, 299
     need = tg.workspace_size(A0, B0, C0, M, N, K)
