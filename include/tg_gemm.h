@@ -17,10 +17,16 @@
  *
  * Layout: A, B and C are dense and row-major (leading dimensions K, N and N
  * elements), fp16 (IEEE binary16), in device memory of the current CUDA
- * device.  The caller owns all three buffers; the library never allocates,
- * frees or retains device memory and keeps no pointer after a call returns;
- * the one call that uses scratch memory (tg_gemm_relu_f16_ws) takes it from
- * the caller.
+ * device.  The caller owns all three buffers and the library keeps no
+ * pointer to them after a call returns.  No call allocates or frees device
+ * memory at run time.  Scratch memory comes from two places:
+ *   - the caller: tg_gemm_relu_f16_ws, tg_gemm_relu_f16_ex and
+ *     tg_gemm_relu_w4a16 take an optional (or, for some layouts, required)
+ *     workspace pointer and size;
+ *   - one fixed module buffer of TG_STATIC_WORKSPACE_BYTES (16 MiB) that the
+ *     library holds on every GPU where it is loaded, until the process
+ *     exits; only tg_gemm_relu_f16_static_ws uses it.
+ * tg_gemm_relu_f16 itself needs no scratch.
  *
  * Threading and streams: calls are asynchronous on `stream` (a cudaStream_t
  * passed as void*; NULL is the legacy default stream).  On TG_OK the work is

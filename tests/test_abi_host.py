@@ -168,9 +168,10 @@ def test_w4a16_kernel_choice():
     assert tg.w4a16_kernel(-1, 8, 128, 32) == K4.INVALID
 
 
-def test_w4a16_decode_switch(monkeypatch):
+def test_environment_cannot_change_the_shipped_kernel_choice(monkeypatch):
+    # Tuning knobs exist only in a -DTG_TUNING build; the shipped library ignores them.
     monkeypatch.setenv("TG_TUNE_W4_DECODE", "0")
-    assert tg.w4a16_kernel(16, 8192, 8192, 128) == tg.W4Kernel.FUSED
+    assert tg.w4a16_kernel(16, 8192, 8192, 128) == tg.W4Kernel.DECODE
 
 
 def test_padded_c_with_general_layouts():

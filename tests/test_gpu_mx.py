@@ -142,24 +142,20 @@ def test_workloads_sampled_rows(name):
     check_rows(got, ops, m_sizes, N, K, sample=6)
 
 
-@pytest.mark.parametrize("kernel", ["single", "pair"])
 @pytest.mark.parametrize("m_sizes,N,K", [
     ((128,), 256, 128),
     ((200, 0, 77, 128), 512, 256),
     ((1, 129, 255, 384), 264, 160),
     ((64,) * 11 + (3,), 384, 384),
 ], ids=["one_tile", "ragged_groups", "odd_tile_counts", "twelve_groups"])
-def test_forced_kernel_integer_bitexact(m_sizes, N, K, kernel, monkeypatch):
-    """Both the 1-SM and the CTA-pair kernel, including groups with an odd number of 128-row tiles
-    (the pair kernel's half pairs) and a last group that ends the stacked rows."""
-    monkeypatch.setenv("TG_TUNE_MX_PAIR", "1" if kernel == "pair" else "0")
+def test_kernel_integer_bitexact(m_sizes, N, K):
+    """Groups with an odd number of 128-row tiles, an empty group, and a last group that ends the
+    stacked rows."""
     got, ops = run_mx(m_sizes, N, K, dist="int", seed=len(m_sizes) + 2 * N, relu=True)
     check_rows(got, ops, m_sizes, N, K, relu=True, exact=True)
 
 
-@pytest.mark.parametrize("kernel", ["single", "pair"])
-def test_forced_kernel_normal_values(kernel, monkeypatch):
-    monkeypatch.setenv("TG_TUNE_MX_PAIR", "1" if kernel == "pair" else "0")
+def test_kernel_normal_values():
     m_sizes, N, K = (333, 128, 45), 520, 1024
     got, ops = run_mx(m_sizes, N, K, dist="normal", seed=31, a_format=1, b_format=0)
     check_rows(got, ops, m_sizes, N, K, a_format=1, b_format=0)

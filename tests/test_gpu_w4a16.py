@@ -135,11 +135,11 @@ def test_decode_float(M, N, K, group):
     assert_close(got, oracle.gemm_relu_w4a16(A, Wq, S, group), f"W4A16 decode float {(M, N, K, group)}")
 
 
-@pytest.mark.parametrize("M,N,K,group", [(1, 520, 1024, 32), (16, 1000, 512, 128), (9, 4096, 4096, 128)])
-def test_tcgen05_kernel_still_serves_small_m(monkeypatch, M, N, K, group):
-    # With the decode kernel switched off, the tcgen05 fused kernel takes these shapes.
+@pytest.mark.parametrize("M,N,K,group", [(1, 520, 1088, 64), (16, 1000, 576, 64), (9, 4096, 4160, 64),
+                                         (4, 512, 16640, 128)])
+def test_tcgen05_kernel_still_serves_small_m(M, N, K, group):
+    # K not a multiple of 256, or K beyond the decode kernel's 16384: the tcgen05 fused kernel.
     import tiled_dense_gemm_fp16_b200 as tg
-    monkeypatch.setenv("TG_TUNE_W4_DECODE", "0")
     assert tg.w4a16_kernel(M, N, K, group) == tg.W4Kernel.FUSED
     got, (A, Wq, S) = run_w4(M, N, K, group, "int", seed=M * 11 + K)
     assert_bitexact(got, oracle.gemm_relu_w4a16(A, Wq, S, group), f"W4A16 tcgen05 {(M, N, K, group)}")

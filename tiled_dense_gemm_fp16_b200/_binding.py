@@ -281,7 +281,7 @@ def gemm_relu(A, B, out=None, path: int = Path.AUTO, stream=None, workspace="aut
     ``workspace``: "auto" lets torch allocate the scratch bytes the repack path
     needs when TMA cannot describe A or B (odd row lengths, unaligned bases);
     None never uses a workspace (edge mode instead); a uint8 CUDA tensor is
-    used as given.  The library itself never allocates.
+    used as given.  The library itself allocates nothing at run time.
     """
     import torch
     if A.dtype != torch.float16 or B.dtype != torch.float16:

@@ -66,9 +66,7 @@ struct MxParams {
   int relu;
   uint32_t idesc;      // formats, shape and scale type; the sf bytes are or-ed in per MMA
   uint64_t wait_budget_ns;
-  int pair_tiles;      // 256-row pair tiles (pair kernel): ceil(tiles / 2) per group
   int tile_start[kMxMaxGroups + 1];  // first stacked 128-row tile of each group; [groups] = m_tiles
-  int pair_start[kMxMaxGroups + 1];  // first pair tile of each group; [groups] = pair_tiles
   int m_size[kMxMaxGroups];          // rows of each group
 };
 

@@ -497,31 +497,6 @@ __device__ __forceinline__ void umma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, u
       : "memory");
 }
 
-// Pair forms (cta_group::2, issued by the even CTA of a 2-CTA cluster): each
-// CTA supplies half of A's rows and half of B's rows from its own shared
-// memory and holds half of D's rows, its A scales and all of B's scales in its
-// own TMEM at the same addresses.
-__device__ __forceinline__ void umma_mxf8_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_nvf4_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
 // Instruction descriptor for kind::mxf4nvf4 with E2M1 A/B (format 1), fp32 D
 // and UE4M3 scales (bit 23 = 0), K-major operands, K = 64.
 __host__ __device__ constexpr uint32_t make_idesc_nvf4(int M, int N) {

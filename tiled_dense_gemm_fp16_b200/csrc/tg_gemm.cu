@@ -16,7 +16,6 @@
 
 #include "tg_gemm.h"
 #include "gemm_mx.cuh"
-#include "gemm_mx_pair.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc_pair.cuh"
@@ -48,7 +47,6 @@ struct DeviceInfo {
   bool skinny_attr = false;
   unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
   bool mx_attr[2] = {false, false};       // per block-scaled kind
-  bool mx_pair_attr[2] = {false, false};
   bool w4_attr = false;
   bool w4_decode_attr = false;
   void* static_ws = nullptr;  // device address of g_static_workspace on this device
@@ -62,12 +60,32 @@ DeviceInfo g_devices[kMaxDevices];
 // from cudaGetSymbolAddress with the device current.
 __device__ __align__(256) uint8_t g_static_workspace[TG_STATIC_WORKSPACE_BYTES];
 
-// Tuning knobs for experiments (environment, read on each launch); the
-// defaults are the tuned values.
+// Tuning knobs.  The shipped library always uses the tuned defaults: the
+// environment cannot change a kernel configuration, and no launch pays for
+// a lookup.  A build with -DTG_TUNING reads TG_TUNE_* variables instead,
+// each once per process (for sweeps).
+#ifdef TG_TUNING
 int tune_int(const char* name, int dflt) {
+  static std::mutex m;
+  static const char* names[64];
+  static int values[64];
+  static bool present[64];
+  static int count = 0;
+  std::lock_guard<std::mutex> lock(m);
+  for (int i = 0; i < count; ++i)
+    if (std::strcmp(names[i], name) == 0) return present[i] ? values[i] : dflt;
   const char* v = std::getenv(name);
+  if (count < 64) {
+    names[count] = name;
+    present[count] = v && *v;
+    values[count] = present[count] ? std::atoi(v) : 0;
+    ++count;
+  }
   return (v && *v) ? std::atoi(v) : dflt;
 }
+#else
+constexpr int tune_int(const char*, int dflt) { return dflt; }
+#endif
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 bool g_encode_probed = false;
 
@@ -860,14 +878,13 @@ uint32_t blockscaled_idesc(int M, int a_format, int b_format) {
   return KIND == kKindNvf4 ? make_idesc_nvf4(M, 256) : make_idesc_mxf8(M, 256, a_format, b_format, 0, 0);
 }
 
-// Shared launcher of the block-scaled grouped kernels (one kind each): the
-// 1-SM kernel or the CTA-pair kernel, whichever needs fewer tile waves.
+// Shared launcher of the block-scaled grouped kernels (one kind each):
+// persistent 128 x 256 tiles over the stacked rows of all groups.
 template <int KIND>
 tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B, const void* SFB, void* C,
                                   const int64_t* m_sizes, int32_t groups, int64_t N, int64_t K, int a_format,
                                   int b_format, float alpha, int32_t relu, void* stream) {
   using Cfg = MxCfg<KIND>;
-  using PairCfg = MxPairCfg<KIND>;
   constexpr int kBlock = KIND == kKindNvf4 ? 16 : 32;
   constexpr int kMmaK = KIND == kKindNvf4 ? 64 : 32;
   constexpr int kElemsPerByte = KIND == kKindNvf4 ? 2 : 1;
@@ -911,69 +928,20 @@ tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B,
   p.n_atoms = static_cast<int>((N + 127) / 128);
   p.relu = relu;
   p.wait_budget_ns = wait_budget(p.k_stages * 2);
-  int tile = 0, pair = 0;
+  int tile = 0;
   for (int32_t g = 0; g < groups; ++g) {
-    const int tiles_g = static_cast<int>(round_up(m_sizes[g], 128) / 128);
     p.tile_start[g] = tile;
-    p.pair_start[g] = pair;
     p.m_size[g] = static_cast<int>(m_sizes[g]);
-    tile += tiles_g;
-    pair += (tiles_g + 1) / 2;
+    tile += static_cast<int>(round_up(m_sizes[g], 128) / 128);
   }
   p.tile_start[groups] = tile;
-  p.pair_start[groups] = pair;
-  p.pair_tiles = pair;
-
-  // The CTA-pair kernel computes the same result and measured level with the
-  // 1-SM kernel on B200 (within 2 %), so the simpler 1-SM kernel runs unless
-  // the pair kernel is asked for (TG_TUNE_MX_PAIR=1).
-  const int64_t single_tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
-  const int64_t pair_tiles = static_cast<int64_t>(p.pair_tiles) * p.n_tiles;
-  const int sms = info->sm_count, pairs = info->sm_count / 2;
-  const bool use_pair = tune_int("TG_TUNE_MX_PAIR", 0) == 1 && pairs >= 1;
 
   CUtensorMap ta, tb;
   std::memset(&ta, 0, sizeof ta);
   std::memset(&tb, 0, sizeof tb);
   if (K > 0) {
     if (!encode_2d_u8(&ta, A, rows, row_bytes, Cfg::BK, Cfg::BM)) return TG_ERR_LAUNCH;
-    if (!encode_2d_u8(&tb, B, static_cast<int64_t>(groups) * N, row_bytes, Cfg::BK,
-                      use_pair ? PairCfg::B_ROWS : Cfg::BN))
-      return TG_ERR_LAUNCH;
-  }
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof cfg);
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  LaunchAttrs la;
-  if (use_pair) {
-    auto kernel = gemm_blockscaled_pair_kernel<KIND>;
-    {
-      std::lock_guard<std::mutex> lock(g_mutex);
-      if (!info->mx_pair_attr[KIND]) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES) !=
-            cudaSuccess) {
-          cudaGetLastError();
-          return TG_ERR_LAUNCH;
-        }
-        info->mx_pair_attr[KIND] = true;
-      }
-    }
-    p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 16);
-    if (p.group_m < 1) p.group_m = 1;
-    p.num_tiles = static_cast<int>(pair_tiles);
-    p.idesc = blockscaled_idesc<KIND>(PairCfg::PAIR_M, a_format, b_format);
-    int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
-    const int max_clusters = tune_int("TG_TUNE_MX_CLUSTERS", 0);
-    if (max_clusters > 0 && max_clusters < clusters) clusters = max_clusters;
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-    cfg.blockDim = dim3(PairCfg::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(PairCfg::SMEM_BYTES);
-    la.fill(cfg, 2);
-    if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
-      cudaGetLastError();
-      return TG_ERR_LAUNCH;
-    }
-    return TG_OK;
+    if (!encode_2d_u8(&tb, B, static_cast<int64_t>(groups) * N, row_bytes, Cfg::BK, Cfg::BN)) return TG_ERR_LAUNCH;
   }
   auto kernel = gemm_blockscaled_grouped_kernel<KIND>;
   {
@@ -989,12 +957,16 @@ tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B,
   }
   p.group_m = tune_int("TG_TUNE_MX_GROUP_M", 16);
   if (p.group_m < 1) p.group_m = 1;
-  p.num_tiles = static_cast<int>(single_tiles);
+  p.num_tiles = static_cast<int>(static_cast<int64_t>(p.m_tiles) * p.n_tiles);
   p.idesc = blockscaled_idesc<KIND>(Cfg::BM, a_format, b_format);
-  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.stream = static_cast<cudaStream_t>(stream);
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(Cfg::SMEM_BYTES);
+  LaunchAttrs la;
   la.fill(cfg, 1);
   if (cudaLaunchKernelEx(&cfg, kernel, ta, tb, p) != cudaSuccess) {
     cudaGetLastError();
