@@ -7,9 +7,17 @@ resident in HBM.  Prints ONE JSON line (rank 0).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload square8192]
     python bench.py --impl reference ...     # the CPU oracle, timed on host cores
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own
-independent problem (weak scaling, no data-path collective); the timed region
-is bracketed by barriers and the slowest rank's time is reported.
+At N=1 the line also carries one record per other configuration of the
+metric's workloads ("configs"), a back-to-back "sustained" run of the headline
+kernel, and the measured host-link rates beside the end-to-end number.
+
+Multi-GPU (torchrun, one process per GPU): by default one problem's M rows are
+split over the ranks, rank r taking rows [floor(rM/G), floor((r+1)M/G)) with B
+replicated, each rank running the unchanged kernel on its row block (strong
+scaling, no collective in the timed step; C is stitched afterwards by an NCCL
+all-gather, which --gather-c also times).  --parallel replicas gives every
+rank its own independent problem instead (weak scaling).  The timed region is
+bracketed by barriers and the slowest rank's time is reported.
 """
 from __future__ import annotations
 
@@ -71,6 +79,19 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", choices=["all", "none"], default="all",
+                    help="all: at N=1 also measure every other configuration of the metric's workloads "
+                         "(square256 float and integer, square4096, skinny M=1/16/64, the three ragged shapes "
+                         "with and without a workspace), one record each in the line's 'configs'")
+    ap.add_argument("--config-cpu-seconds", type=float, default=1.0,
+                    help="target CPU work of each configuration's oracle sample")
+    ap.add_argument("--sustained-seconds", type=float, default=2.0,
+                    help="at N=1, also run the headline kernel back to back this long (0: skip)")
+    ap.add_argument("--parallel", choices=["rows", "replicas"], default="rows",
+                    help="N>1: rows = split one problem's M rows over the ranks with B replicated "
+                         "(strong scaling); replicas = every rank runs its own problem (weak scaling)")
+    ap.add_argument("--gather-c", action="store_true",
+                    help="rows mode: also time the NCCL all-gather that stitches C on every rank")
     ap.add_argument("--cublas", action="store_true",
                     help="also time torch.relu(torch.matmul(A, B)) (cuBLAS) on the same operands, as context")
     return ap.parse_args()
@@ -132,7 +153,7 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.period = period_s
         self.samples = []
         self.reasons = 0
@@ -153,8 +174,10 @@ class ClockSampler:
         nv = self.nvml
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
-                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((mhz, reasons))
+                self.reasons |= reasons & ~self.REASONS["gpu_idle"]
             except Exception:
                 pass
             self._stop.wait(self.period)
@@ -173,8 +196,10 @@ class ClockSampler:
         if self.nvml is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
         names = [k for k, bit in self.REASONS.items() if self.reasons & bit and k != "gpu_idle"]
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+        busy = [mhz for mhz, r in self.samples if not (r & self.REASONS["gpu_idle"])]
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                "samples_under_load": len(busy), "period_ms": self.period * 1e3}
 
 
 # ---------------------------------------------------------------------------
@@ -406,6 +431,294 @@ def rank_seed(workload_seed: int, rank: int) -> int:
 # Our arm
 # ---------------------------------------------------------------------------
 
+# ---------------------------------------------------------------------------
+# Row partition of one problem over ranks (also exercised by CPU gloo tests)
+# ---------------------------------------------------------------------------
+
+def row_range(M: int, world: int, rank: int):
+    """Rows [r0, r1) of C (and of A) that rank `rank` of `world` computes: floor(r*M/G) .. floor((r+1)*M/G)."""
+    return (rank * M) // world, ((rank + 1) * M) // world
+
+
+def gather_rows(dist, block, M: int, world: int, rank: int):
+    """All-gather every rank's row block of C into the full M x N C (row-major, rank order).
+
+    Blocks differ by at most one row; each is padded to the largest so that the
+    collective moves equal sizes, and the padding is dropped when stitching.
+    Works on CPU tensors (gloo) and CUDA tensors (NCCL)."""
+    import torch
+    rows = [row_range(M, world, r) for r in range(world)]
+    most = max(r1 - r0 for r0, r1 in rows)
+    N = block.shape[1]
+    padded = torch.zeros((most, N), dtype=block.dtype, device=block.device)
+    padded[: block.shape[0]].copy_(block)
+    parts = [torch.empty_like(padded) for _ in range(world)]
+    dist.all_gather(parts, padded)
+    return torch.cat([parts[r][: r1 - r0] for r, (r0, r1) in enumerate(rows)], dim=0)
+
+
+# ---------------------------------------------------------------------------
+# Roofline, host link, L2 hygiene
+# ---------------------------------------------------------------------------
+
+def roofline_for(M, N, K, kernel_ms, peaks, peak_src, sustained=False):
+    """Roofline record of one fp16 GEMM: the bound is whichever roof its arithmetic
+    intensity (2MNK flops over the compulsory 2(MK+KN+MN) bytes) meets first."""
+    flops = inputs.flops(M, N, K)
+    nbytes = inputs.min_bytes(M, N, K)
+    tkey = "bf16_tflops_sustained" if sustained and "bf16_tflops_sustained" in peaks else "bf16_tflops"
+    t_peak, h_peak = float(peaks[tkey]), float(peaks["hbm_gbs"])
+    ridge = t_peak * 1e12 / (h_peak * 1e9)
+    intensity = flops / nbytes
+    if intensity >= ridge:
+        achieved = flops / (kernel_ms * 1e-3) / 1e12
+        rec = {"bound": "tensor", "achieved": achieved, "peak": t_peak, "unit": "TFLOP/s",
+               "peak_source": f"{peak_src} cuBLAS bf16 {'sustained' if 'sustained' in tkey else 'burst'} peak "
+                              f"(fp16 kind::f16 runs at the bf16 rate)"}
+    else:
+        achieved = nbytes / (kernel_ms * 1e-3) / 1e9
+        rec = {"bound": "hbm", "achieved": achieved, "peak": h_peak, "unit": "GB/s",
+               "peak_source": f"{peak_src} STREAM-copy HBM bandwidth"}
+    rec["frac"] = rec["achieved"] / rec["peak"]
+    rec["intensity_flop_per_byte"] = intensity
+    rec["ridge_flop_per_byte"] = ridge
+    rec["kernel_ms"] = kernel_ms
+    return rec
+
+
+def host_link(dev, h2d_bytes: int, d2h_bytes: int, reps: int = 3):
+    """Measured pinned-host <-> device copy bandwidth (GB/s) for copies of the e2e leg's sizes."""
+    import torch
+    out = {}
+    for name, nbytes in (("h2d", h2d_bytes), ("d2h", d2h_bytes)):
+        n = max(1, nbytes)
+        host = torch.empty(n, dtype=torch.uint8).pin_memory()
+        devb = torch.empty(n, dtype=torch.uint8, device=dev)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        best = None
+        for _ in range(reps):
+            torch.cuda.synchronize(dev)
+            ev0.record()
+            if name == "h2d":
+                devb.copy_(host, non_blocking=True)
+            else:
+                host.copy_(devb, non_blocking=True)
+            ev1.record()
+            torch.cuda.synchronize(dev)
+            ms = ev0.elapsed_time(ev1)
+            best = ms if best is None else min(best, ms)
+        out[name + "_gbs"] = n / (best * 1e-3) / 1e9
+        del host, devb
+    return out
+
+
+def operand_sets(torch, dev, tensors, work_bytes: int):
+    """Device operand sets for timing: operands well beyond L2 are used as they are; mid-size ones
+    rotate over R identical copies (R x working set >= 3 x L2) so every step reads cold operands;
+    tiny ones get an L2 flush buffer (a write of twice the L2 size between timed steps)."""
+    sets = [tuple(tensors)]
+    flush = None
+    if work_bytes <= 2 * L2_BYTES:
+        R = -(-3 * L2_BYTES // max(1, work_bytes))
+        if R <= 64:
+            for _ in range(R - 1):
+                sets.append(tuple(t.clone() for t in tensors))
+        else:
+            flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+    note = ("inputs larger than L2" if work_bytes > 2 * L2_BYTES else
+            f"rotating {len(sets)} operand copies ({len(sets) * work_bytes / 2**20:.0f} MiB > 3x L2)"
+            if flush is None else "L2 flushed between timed steps")
+    return sets, flush, note
+
+
+def repack_launches(tg, M, N, K, a_ptr, b_ptr, c_ptr, chosen) -> int:
+    """Kernels one call launches: the GEMM, plus on the repack path one row-padding copy per operand TMA
+    cannot describe and, when the GEMM writes a padded C (rows of C not 16-byte aligned, M > 256), the
+    copy that moves it into C."""
+    n = 1
+    if chosen == tg.Path.REPACK:
+        n += int(K % 8 != 0 or a_ptr % 16 != 0) + int(N % 8 != 0 or b_ptr % 16 != 0)
+        n += int((N % 8 != 0 or c_ptr % 16 != 0) and M > 256)
+    return n
+
+
+def timed_region(torch, dev, stream, step, steps, flush, dist=None, clock_period_s=0.001):
+    """Mean device time per step (ms) of `steps` calls of step() on `stream`, bracketed by a barrier and a
+    synchronize on both sides, with NVML clocks sampled during the region.  With an L2 flush buffer, each
+    step gets its own event pair so the flush stays outside the timed steps; otherwise one pair around
+    the region (tiny kernels are not charged for event records)."""
+    per_step = flush is not None
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps if per_step else 0)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps if per_step else 0)]
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0, clock_period_s)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        r0.record(stream)
+        for i in range(steps):
+            if per_step:
+                flush.fill_(1)
+                starts[i].record(stream)
+            step()
+            if per_step:
+                ends[i].record(stream)
+        r1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    if dist is not None:
+        dist.barrier()
+    if per_step:
+        ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / steps
+    else:
+        ms = r0.elapsed_time(r1) / steps
+    return ms, sampler.summary()
+
+
+class Fp16Case:
+    """One fp16 GEMM+ReLU problem resident in HBM, called through the C ABI.
+
+    mode "auto": tg_gemm_relu_f16_ws with the scratch bytes the library asks for (allocated by torch
+    outside the timed region); "none": tg_gemm_relu_f16, no workspace; "linear": tg_gemm_relu_f16_ex with
+    the weight stored N x K and a bias."""
+
+    def __init__(self, tg, torch, dev, stream, M, N, K, A, B, mode="auto", path=None, bias=None):
+        self.tg, self.torch, self.dev, self.stream = tg, torch, dev, stream
+        self.M, self.N, self.K, self.mode = M, N, K, mode
+        self.A_host, self.B_host = A, B
+        Ad, Bd = torch.from_numpy(A).to(dev), torch.from_numpy(B).to(dev)
+        Cd = torch.empty((M, N), dtype=torch.float16, device=dev)
+        self.bias_d = torch.from_numpy(bias).to(dev) if bias is not None else None
+        self.sets, self.flush, self.l2_note = operand_sets(torch, dev, (Ad, Bd, Cd), inputs.min_bytes(M, N, K))
+        self.path = tg.Path.AUTO if path is None else path
+        self.ws_bytes = 0
+        if mode == "auto" and self.path == tg.Path.AUTO:
+            self.ws_bytes = max(tg.workspace_size(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K)
+                                for a, b, c in self.sets)
+        self.ws = torch.empty(max(self.ws_bytes, 1), dtype=torch.uint8, device=dev)
+        self.opts = (tg.options(b_layout=tg.B_NK, bias=self.bias_d.data_ptr()) if mode == "linear" else None)
+        a, b, c = self.sets[0]
+        if mode == "linear":
+            self.chosen = tg.select_path_ex(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, self.opts, 0)
+        elif self.path != tg.Path.AUTO:
+            self.chosen = self.path
+        else:
+            self.chosen = tg.select_path_ws(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, self.ws_bytes)
+        self.launches_per_step = repack_launches(tg, M, N, K, a.data_ptr(), b.data_ptr(), c.data_ptr(), self.chosen)
+        self.cur = 0
+
+    def call(self, a, b, c):
+        tg, sh = self.tg, self.stream.cuda_stream
+        M, N, K = self.M, self.N, self.K
+        if self.mode == "linear":
+            st = tg.gemm_relu_f16_ex_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, self.opts, sh)
+        elif self.ws_bytes > 0:
+            st = tg.gemm_relu_f16_ws_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, sh,
+                                         self.ws.data_ptr(), self.ws_bytes)
+        else:
+            st = tg.gemm_relu_f16_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, sh, self.path)
+        if st != tg.Status.OK:
+            raise tg.TGError(st, "tg_gemm_relu_f16")
+
+    def step(self):
+        self.call(*self.sets[self.cur % len(self.sets)])
+        self.cur += 1
+
+    def warm(self, warmup):
+        torch, tg = self.torch, self.tg
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                if self.flush is not None:
+                    self.flush.fill_(1)
+                self.step()
+        torch.cuda.synchronize(self.dev)
+        st, word = tg.device_status()
+        if st != tg.Status.OK:
+            raise SystemExit(f"device error after warm-up: {tg.status_string(st)} 0x{word:x}")
+
+    def time(self, steps, dist=None):
+        ms, clocks = timed_region(self.torch, self.dev, self.stream, self.step, steps, self.flush, dist)
+        st, word = self.tg.device_status()
+        if st != self.tg.Status.OK:
+            raise SystemExit(f"device error in timed region: {self.tg.status_string(st)} 0x{word:x}")
+        return ms, clocks
+
+    def release(self):
+        self.sets = self.ws = self.flush = None
+
+
+def sustained_record(case, seconds, peaks, peak_src):
+    """The headline kernel back to back for about `seconds` (one event pair around the loop, clocks
+    sampled every millisecond), against the sustained (power-capped) tensor peak."""
+    # Estimate the step time from a short burst, then size the loop.
+    ms, _ = case.time(5)
+    est_ms = max(ms, 1e-3)
+    steps = max(10, int(seconds * 1e3 / est_ms))
+    ms, clocks = case.time(steps)
+    rec = roofline_for(case.M, case.N, case.K, ms, peaks, peak_src, sustained=True)
+    rec.update({"steps": steps, "seconds": steps * ms * 1e-3, "ms_per_step": ms, "clocks": clocks})
+    if clocks.get("sm_mhz"):
+        rec["ms_x_sm_mhz"] = ms * clocks["sm_mhz"]
+    return rec
+
+
+# The configurations the metric's workloads are quoted on (besides the headline square8192), each
+# measured as its own record: (label, workload, sub-index, value distribution or None, workspace mode).
+CONFIG_RECORDS = [
+    ("square256", "square256", None, None, "auto"),
+    ("square256_int", "square256", None, "int", "auto"),
+    ("square4096", "square4096", None, None, "auto"),
+    ("skinny_m1", "skinny", 0, None, "auto"),
+    ("skinny_m16", "skinny", 1, None, "auto"),
+    ("skinny_m64", "skinny", 2, None, "auto"),
+    ("ragged0_no_ws", "ragged", 0, None, "none"),
+    ("ragged0_ws", "ragged", 0, None, "auto"),
+    ("ragged1_no_ws", "ragged", 1, None, "none"),
+    ("ragged1_ws", "ragged", 1, None, "auto"),
+    ("ragged2_no_ws", "ragged", 2, None, "none"),
+    ("ragged2_ws", "ragged", 2, None, "auto"),
+]
+
+
+def config_problem(workload, idx, dist):
+    """(M, N, K, A, B) of one shape of a workload, exactly as the workload draws it (the generator is
+    advanced over the workload's earlier shapes); `dist` overrides the value distribution."""
+    wl = inputs.WORKLOADS[workload]
+    for i, ((m, n, k), A, B) in enumerate(wl.problems(dist)):
+        if i == (idx or 0):
+            return m, n, k, A, B
+    raise KeyError((workload, idx))
+
+
+def measure_configs(tg, torch, dev, stream, args, peaks, peak_src):
+    """One record per configuration: time, roofline against the roof its intensity meets, clocks, and the
+    oracle timed on a short row sample on the host cores."""
+    records = []
+    for label, workload, idx, dist, mode in CONFIG_RECORDS:
+        M, N, K, A, B = config_problem(workload, idx, dist)
+        case = Fp16Case(tg, torch, dev, stream, M, N, K, A, B, mode=mode)
+        case.warm(args.warmup)
+        ms, clocks = case.time(args.steps)
+        rec = {"config": label, "workload": workload + (f":{idx}" if idx is not None else ""),
+               "M": M, "N": N, "K": K, "values": dist or inputs.WORKLOADS[workload].dist,
+               "seed": inputs.WORKLOADS[workload].seed,
+               "entry_point": "tg_gemm_relu_f16" if case.ws_bytes == 0 else "tg_gemm_relu_f16_ws",
+               "path": tg.path_name(case.chosen), "workspace_bytes": case.ws_bytes, "l2": case.l2_note,
+               "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+               "value": inputs.flops(M, N, K) / (ms * 1e-3) / 1e12, "unit": UNIT,
+               "roofline": roofline_for(M, N, K, ms, peaks, peak_src),
+               "gpu_launches": args.steps * case.launches_per_step, "clocks": clocks}
+        rec["roofline"]["traffic"] = committed_traffic(tg.path_name(case.chosen), label)
+        if not args.no_cpu_baseline:
+            rec["cpu_baseline"] = cpu_baseline(A, B, args.config_cpu_seconds)
+        case.release()
+        del A, B
+        records.append(rec)
+    return records
+
+
 def run_ours(args):
     if args.workload in inputs.MX_WORKLOADS or args.workload in inputs.NVF4_WORKLOADS:
         return run_ours_mx(args)
@@ -414,201 +727,111 @@ def run_ours(args):
     import torch
     import tiled_dense_gemm_fp16_b200 as tg
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-
+    world, rank, dev, dist = _init_ranks(args)
     path = {"auto": tg.Path.AUTO, "tc": tg.Path.TC, "tc_edge": tg.Path.TC_EDGE, "skinny": tg.Path.SKINNY,
             "tc_pair": tg.Path.TC_PAIR, "tc_pair512": tg.Path.TC_PAIR512}[args.path]
-    name, M, N, K, A, B = workload_problem(args.workload, rank)
-    flops = inputs.flops(M, N, K)
+    rows_mode = world > 1 and args.parallel == "rows"
+    # Row partition: every rank draws the workload itself (same seed) and keeps its rows of A; B is
+    # replicated.  Replicas: every rank runs its own independent problem.
+    name, M, N, K, A, B = workload_problem(args.workload, 0 if rows_mode else rank)
     linear = name == "linear8192"
-    bias_d = None
+    bias = None
     if linear:
         B, bias = B
-        bias_d = torch.from_numpy(bias).to(dev)
-
-    Ad = torch.from_numpy(A).to(dev)
-    Bd = torch.from_numpy(B).to(dev)
-    Cd = torch.empty((M, N), dtype=torch.float16, device=dev)
+    r0, r1 = row_range(M, world, rank) if rows_mode else (0, M)
+    Mr = r1 - r0
+    A_r = np.ascontiguousarray(A[r0:r1])
     stream = torch.cuda.Stream(dev)
-    sh = stream.cuda_stream
-    chosen = tg.select_path(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K) if path == tg.Path.AUTO else path
-    ws = 2 * (M * K + K * N + M * N)
-    # Keep L2 from serving a step with the previous step's operands.  Operands
-    # well beyond L2 need nothing.  Mid-size ones rotate over R identical copies
-    # (R x working set >= 3 x L2), so every step reads clean, cold operands.
-    # Tiny ones get an L2 flush (a write of twice the L2 size) between timed
-    # steps, outside the per-step events.
-    sets = [(Ad, Bd, Cd)]
-    flush = None
-    if ws <= 2 * L2_BYTES:
-        R = -(-3 * L2_BYTES // ws)
-        if R <= 64:
-            for _ in range(R - 1):
-                sets.append((Ad.clone(), Bd.clone(), torch.empty_like(Cd)))
-        else:
-            flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
-    l2_note = ("inputs larger than L2" if ws > 2 * L2_BYTES else
-               f"rotating {len(sets)} operand copies ({len(sets) * ws / 2**20:.0f} MiB > 3x L2)" if flush is None else
-               "L2 flushed between timed steps")
-    cur = [0]
+    mode = "linear" if linear else ("none" if args.workspace == "none" else "auto")
+    case = Fp16Case(tg, torch, dev, stream, Mr, N, K, A_r, B, mode=mode,
+                    path=None if path == tg.Path.AUTO else path, bias=bias)
+    case.warm(args.warmup)
+    kern_ms, clocks = case.time(args.steps, dist)
+    step_ms = max_over_ranks(dist, kern_ms, dev) if dist is not None else kern_ms
+    flops_rank = inputs.flops(Mr, N, K)
+    flops_total = inputs.flops(M, N, K) if rows_mode else world * flops_rank
+    value = flops_total / (step_ms * 1e-3) / 1e12
 
-    ws_bytes = 0
-    if args.workspace == "auto" and path == tg.Path.AUTO:
-        ws_bytes = max(tg.workspace_size(s_[0].data_ptr(), s_[1].data_ptr(), s_[2].data_ptr(), M, N, K)
-                       for s_ in sets)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    if ws_bytes > 0:
-        chosen = tg.select_path_ws(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, ws_bytes)
+    gather = None
+    if rows_mode:
+        # Stitch C once (outside the timed region) so every rank holds the full result; with
+        # --gather-c the all-gather is also timed on its own over the same steps.
+        c_block = case.sets[0][2]
+        full = gather_rows(dist, c_block, M, world, rank)
+        assert full.shape == (M, N)
+        gather = {"stitched": True}
+        if args.gather_c:
+            with torch.cuda.stream(stream):
+                gather_rows(dist, c_block, M, world, rank)
+            g_ms, _ = timed_region(torch, dev, stream, lambda: gather_rows(dist, c_block, M, world, rank),
+                                   args.steps, None, dist)
+            gather["all_gather_ms"] = max_over_ranks(dist, g_ms, dev)
+            gather["step_ms_with_gather"] = step_ms + gather["all_gather_ms"]
+        del full
 
-    # Kernels per step: one GEMM, plus one row-padding copy per repacked operand
-    # and, when the GEMM writes a padded C (rows of C not 16-byte aligned,
-    # M > 256), the copy that moves it into C.
-    launches_per_step = 1
-    if chosen == tg.Path.REPACK:
-        launches_per_step += int(K % 8 != 0 or Ad.data_ptr() % 16 != 0) + int(N % 8 != 0 or Bd.data_ptr() % 16 != 0)
-        launches_per_step += int((N % 8 != 0 or Cd.data_ptr() % 16 != 0) and M > 256)
-
-    lin_opts = tg.options(b_layout=tg.B_NK, bias=bias_d.data_ptr()) if linear else None
-    if linear:
-        chosen = tg.select_path_ex(Ad.data_ptr(), Bd.data_ptr(), Cd.data_ptr(), M, N, K, lin_opts, 0)
-
-    def call(a, b, c):
-        if linear:
-            st = tg.gemm_relu_f16_ex_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, lin_opts, sh)
-        elif ws_bytes > 0:
-            st = tg.gemm_relu_f16_ws_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, sh, ws.data_ptr(), ws_bytes)
-        else:
-            st = tg.gemm_relu_f16_raw(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, sh, path)
-        if st != tg.Status.OK:
-            raise tg.TGError(st, "tg_gemm_relu_f16")
-
-    def step():
-        call(*sets[cur[0] % len(sets)])
-        cur[0] += 1
-
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            if flush is not None:
-                flush.fill_(1)
-            step()
-    torch.cuda.synchronize(dev)
-    st, word = tg.device_status()
-    if st != tg.Status.OK:
-        raise SystemExit(f"device error after warm-up: {tg.status_string(st)} 0x{word:x}")
-
-    # Per-step event pairs only when an L2 flush runs between steps (they
-    # bracket the steps and leave the flushes out); otherwise one pair around
-    # the whole region, so tiny kernels are not charged for event records.
-    per_step = flush is not None
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps if per_step else 0)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps if per_step else 0)]
-    region0 = torch.cuda.Event(enable_timing=True)
-    region1 = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    sampler.start()
-    with torch.cuda.stream(stream):
-        region0.record(stream)
-        for i in range(args.steps):
-            if per_step:
-                flush.fill_(1)
-                starts[i].record(stream)
-            step()
-            if per_step:
-                ends[i].record(stream)
-        region1.record(stream)
-    torch.cuda.synchronize(dev)
-    sampler.stop()
-    if dist is not None:
-        dist.barrier()
-    region_ms = region0.elapsed_time(region1)
-    if per_step:
-        step_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.steps
-    else:
-        step_ms = region_ms / args.steps
-    kern_avg_ms = step_ms
-    if dist is not None:
-        step_ms = max_over_ranks(dist, step_ms, dev)
-        kern_avg_ms = step_ms
-    st, word = tg.device_status()
-    if st != tg.Status.OK:
-        raise SystemExit(f"device error in timed region: {tg.status_string(st)} 0x{word:x}")
-
-    value = aggregate_throughput(world, flops, step_ms)
-
-    # End to end through the C ABI from pinned host buffers: every step copies
-    # A and B in and C out, pipelined over two buffer sets (pipelined_e2e).
-    hosts = [torch.from_numpy(A).pin_memory(), torch.from_numpy(B).pin_memory()]
-    e2e_ms = pipelined_e2e(dev, stream, hosts, lambda: [torch.empty_like(Ad), torch.empty_like(Bd)], (M, N),
-                           torch.float16, call, args.e2e_steps)
+    # End to end through the C ABI from pinned host buffers: every step copies A and B in and C out,
+    # pipelined over two buffer sets (pipelined_e2e).
+    Ad0, Bd0 = case.sets[0][0], case.sets[0][1]
+    hosts = [torch.from_numpy(A_r).pin_memory(), torch.from_numpy(B).pin_memory()]
+    e2e_ms = pipelined_e2e(dev, stream, hosts, lambda: [torch.empty_like(Ad0), torch.empty_like(Bd0)], (Mr, N),
+                           torch.float16, case.call, args.e2e_steps)
     if dist is not None:
         e2e_ms = max_over_ranks(dist, e2e_ms, dev)
-    e2e_value = aggregate_throughput(world, flops, e2e_ms)
+    h2d, d2h = 2 * (Mr * K + K * N), 2 * Mr * N
+    link = host_link(dev, h2d, d2h)
+    floor_ms = max(h2d / (link["h2d_gbs"] * 1e9), d2h / (link["d2h_gbs"] * 1e9)) * 1e3
 
     peaks, peak_src = load_peaks()
-    if chosen in (tg.Path.TC, tg.Path.TC_EDGE, tg.Path.TC_PAIR, tg.Path.TC_PAIR512) and (
-            name.startswith("square") or linear):
-        bound, unit_r = "tensor", "TFLOP/s"
-        achieved = flops / (kern_avg_ms * 1e-3) / 1e12
-        peak = float(peaks["bf16_tflops"])
-        peak_note = f"{peak_src} cuBLAS bf16 burst peak (fp16 kind::f16 runs at the bf16 rate)"
+    roof = roofline_for(Mr, N, K, kern_ms, peaks, peak_src)
+    roof["traffic"] = committed_traffic(tg.path_name(case.chosen), name) if rank == 0 else None
+    if rows_mode:
+        parallelism = (f"rows{world}: rank r computes rows [floor(rM/{world}), floor((r+1)M/{world})) of one "
+                       f"{M}x{N}x{K} problem with B replicated; C stitched by an NCCL all-gather")
+    elif world > 1:
+        parallelism = f"dp{world} independent problems"
     else:
-        bound, unit_r = "hbm", "GB/s"
-        achieved = inputs.min_bytes(M, N, K) / (kern_avg_ms * 1e-3) / 1e9
-        peak = float(peaks["hbm_gbs"])
-        peak_note = f"{peak_src} STREAM-copy HBM bandwidth"
-    traffic = committed_traffic(tg.path_name(chosen), name) if rank == 0 else None
-
+        parallelism = "1 GPU"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "strong" if rows_mode else "weak",
         "vs_baseline": None, "dtype": "f16 (fp32 accumulate)", "data": "synthetic",
-        "config": {**describe(name, M, N, K), "path": tg.path_name(chosen), "workspace_bytes": ws_bytes,
-                   "l2": l2_note,
-                   "parallelism": f"dp{world} independent problems" if world > 1 else "1 GPU"},
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit_r,
-                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_note,
-                     "kernel_ms": kern_avg_ms},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 2 * (M * K + K * N),
-                "d2h_bytes_per_step": 2 * M * N, "ms_per_step": e2e_ms, "mode": E2E_MODE},
-        "gpu_launches": args.steps * launches_per_step,
-        "clocks": sampler.summary(),
+        "config": {**describe(name, M, N, K), "path": tg.path_name(case.chosen), "workspace_bytes": case.ws_bytes,
+                   "l2": case.l2_note, "parallelism": parallelism,
+                   **({"rows_per_rank": [row_range(M, world, r)[1] - row_range(M, world, r)[0]
+                                         for r in range(world)]} if rows_mode else {})},
+        "roofline": roof,
+        "e2e": {"value": flops_total / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "mode": E2E_MODE,
+                "host_link": {**link, "copy_floor_ms": floor_ms, "e2e_over_floor": e2e_ms / floor_ms,
+                              "note": "floor = the larger of the upload and the download at the measured "
+                                      "pinned-copy rates (they run on separate copy engines)"}},
+        "gpu_launches": args.steps * case.launches_per_step,
+        "clocks": clocks,
     }
+    if gather is not None:
+        line["gather"] = gather
+    if rank == 0 and world == 1 and args.sustained_seconds > 0:
+        line["sustained"] = sustained_record(case, args.sustained_seconds, peaks, peak_src)
     if args.cublas and not linear:
-        # Context only (a library GEMM, not this path): the same operand sets,
-        # events around the whole region, as for our kernel.
+        # Context only (a library GEMM, not this path): the same operand sets, events around the region.
+        def cublas_step():
+            a_, b_, _ = case.sets[case.cur % len(case.sets)]
+            case.cur += 1
+            torch.relu(torch.matmul(a_, b_))
         with torch.cuda.stream(stream):
-            for i in range(args.warmup):
-                a_, b_, _ = sets[i % len(sets)]
-                torch.relu(torch.matmul(a_, b_))
-            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize(dev)
-            c0.record(stream)
-            for i in range(args.steps):
-                a_, b_, _ = sets[i % len(sets)]
-                torch.relu(torch.matmul(a_, b_))
-            c1.record(stream)
-        torch.cuda.synchronize(dev)
-        cms = c0.elapsed_time(c1) / args.steps
+            for _ in range(args.warmup):
+                cublas_step()
+        cms, _ = timed_region(torch, dev, stream, cublas_step, args.steps, case.flush)
         line["context_cublas"] = {"op": "torch.relu(torch.matmul(A, B))", "ms_per_step": cms,
-                                  "tflops": flops / (cms * 1e-3) / 1e12}
+                                  "tflops": flops_rank / (cms * 1e-3) / 1e12}
+    case.release()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(A, B, args.cpu_seconds)
+    if rank == 0 and world == 1 and args.configs == "all" and not linear:
+        del A, B, A_r, hosts
+        line["configs"] = measure_configs(tg, torch, dev, stream, args, peaks, peak_src)
+        line["gpu_launches"] += sum(r["gpu_launches"] for r in line["configs"])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -70,3 +70,63 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     args = type("Args", (), {"workload": "square8192", "steps": 1, "warmup": 3, "gpus": 2})()
     assert bench.run_reference(args) == 0               # returns at once: no oracle run
+
+
+def test_row_ranges_tile_m_exactly():
+    import bench
+    for M in (1, 2, 7, 37, 256, 3001, 8191, 8192):
+        for world in (1, 2, 3, 4, 8):
+            ranges = [bench.row_range(M, world, r) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == M
+            assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+            sizes = [r1 - r0 for r0, r1 in ranges]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 0
+
+
+def _rows_worker(rank, world, port, out):
+    import datetime
+    import sys
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import oracle
+    from tiled_dense_gemm_fp16_b200 import inputs
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        M, N, K = 37, 24, 40                               # odd M: the blocks differ by one row
+        A, B = inputs.operands(M, N, K, "int", seed=11)    # every rank draws the same problem
+        r0, r1 = bench.row_range(M, world, rank)
+        # Stand-in for the rank's GPU kernel (this test only): the oracle on the rank's rows.
+        block = oracle.gemm_relu_f16(np.ascontiguousarray(A[r0:r1]), B)
+        full = bench.gather_rows(dist, torch.from_numpy(block), M, world, rank)
+        out.put((rank, r0, r1, full.numpy().view(np.uint16).copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_rows_and_stitch_c():
+    import numpy as np
+
+    import oracle
+    from tiled_dense_gemm_fp16_b200 import inputs
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rows_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted((out.get(timeout=120) for _ in procs), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    A, B = inputs.operands(37, 24, 40, "int", seed=11)
+    want = oracle.gemm_relu_f16(A, B).view(np.uint16)
+    assert [(r0, r1) for _, r0, r1, _ in results] == [(0, 18), (18, 37)]
+    for _, _, _, full in results:                          # every rank holds the whole, stitched C
+        assert full.shape == (37, 24)
+        assert np.array_equal(full, want)
