@@ -72,17 +72,19 @@ def parse_args():
     ap.add_argument("--workload", default="square8192",
                     help="square8192 (the metric's workload), square4096, square256, skinny:<M>, ragged:<i>, "
                          "linear8192, mxf8_moe, mxf8_8192, nvf4_8192, nvf4_moe, w4a16_decode, w4a16_8192")
-    ap.add_argument("--path", default="auto", help="force a kernel path: auto, tc, tc_edge, skinny, tc_pair, tc_pair512")
+    ap.add_argument("--path", default="auto",
+                    help="force a kernel path: auto, tc, tc_edge, skinny, tc_pair, tc_pair512, rc")
     ap.add_argument("--workspace", choices=["auto", "none"], default="auto",
                     help="auto: give the library the scratch bytes it asks for (repack path for "
                          "operands TMA cannot describe), allocated by torch outside the timed region")
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--configs", choices=["all", "none"], default="all",
+    ap.add_argument("--configs", default="all",
                     help="all: at N=1 also measure every other configuration of the metric's workloads "
                          "(square256 float and integer, square4096, skinny M=1/16/64, the three ragged shapes "
-                         "with and without a workspace), one record each in the line's 'configs'")
+                         "with and without a workspace), one record each in the line's 'configs'; none: skip; "
+                         "or a comma-separated list of their labels")
     ap.add_argument("--config-cpu-seconds", type=float, default=1.0,
                     help="target CPU work of each configuration's oracle sample")
     ap.add_argument("--sustained-seconds", type=float, default=2.0,
@@ -696,7 +698,10 @@ def measure_configs(tg, torch, dev, stream, args, peaks, peak_src):
     """One record per configuration: time, roofline against the roof its intensity meets, clocks, and the
     oracle timed on a short row sample on the host cores."""
     records = []
+    wanted = None if args.configs == "all" else set(args.configs.split(","))
     for label, workload, idx, dist, mode in CONFIG_RECORDS:
+        if wanted is not None and label not in wanted:
+            continue
         M, N, K, A, B = config_problem(workload, idx, dist)
         case = Fp16Case(tg, torch, dev, stream, M, N, K, A, B, mode=mode)
         case.warm(args.warmup)
@@ -729,7 +734,7 @@ def run_ours(args):
 
     world, rank, dev, dist = _init_ranks(args)
     path = {"auto": tg.Path.AUTO, "tc": tg.Path.TC, "tc_edge": tg.Path.TC_EDGE, "skinny": tg.Path.SKINNY,
-            "tc_pair": tg.Path.TC_PAIR, "tc_pair512": tg.Path.TC_PAIR512}[args.path]
+            "tc_pair": tg.Path.TC_PAIR, "tc_pair512": tg.Path.TC_PAIR512, "rc": tg.Path.RC}[args.path]
     rows_mode = world > 1 and args.parallel == "rows"
     # Row partition: every rank draws the workload itself (same seed) and keeps its rows of A; B is
     # replicated.  Replicas: every rank runs its own independent problem.
@@ -828,7 +833,7 @@ def run_ours(args):
     case.release()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(A, B, args.cpu_seconds)
-    if rank == 0 and world == 1 and args.configs == "all" and not linear:
+    if rank == 0 and world == 1 and args.configs != "none" and not linear:
         del A, B, A_r, hosts
         line["configs"] = measure_configs(tg, torch, dev, stream, args, peaks, peak_src)
         line["gpu_launches"] += sum(r["gpu_launches"] for r in line["configs"])

@@ -79,9 +79,15 @@ typedef enum tg_path {
                             (cta_group::2), 256x256 tiles; same alignment
                             needs as TC                                     */
     TG_PATH_TC_PAIR512 = 7, /* as TC_PAIR with 256x512 tiles                */
-    TG_PATH_REPACK = 8   /* operands TMA cannot describe are first copied
+    TG_PATH_REPACK = 8,  /* operands TMA cannot describe are first copied
                             into zero-padded rows in the caller's workspace,
                             then a TMA kernel runs (tg_gemm_relu_f16_ws)    */
+    TG_PATH_RC = 9       /* no scratch, any 2-byte alignment of A, B and C:
+                            A's rows are loaded by TMA in residue classes
+                            (row mod 8, rows sharing one 16-byte offset),
+                            B's k-rows shifted to match; B realigned in
+                            shared memory when TMA cannot describe it (then
+                            K >= 8); A stored M x K, B stored K x N only    */
 } tg_path;
 
 /*

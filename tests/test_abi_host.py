@@ -87,12 +87,12 @@ def test_path_selection():
     for M in (1, 16, 64, 256):
         assert tg.select_path(A0, B0, C0, M, 8192, 8192) == Path.SKINNY
     assert tg.select_path(A0, B0, C0, 257, 8192, 8192) == Path.TC_PAIR
-    assert tg.select_path(A0, B0, C0, 64, 8191, 8192) == Path.TC_EDGE
+    assert tg.select_path(A0, B0, C0, 64, 8191, 8192) == Path.RC
     # Row strides that are not 16-byte multiples, or misaligned bases, need the edge mode.
-    assert tg.select_path(A0, B0, C0, 3001, 5003, 1021) == Path.TC_EDGE
-    assert tg.select_path(A0, B0, C0, 777, 12289, 4095) == Path.TC_EDGE
-    assert tg.select_path(A0, B0, C0, 8191, 129, 8193) == Path.TC_EDGE
-    assert tg.select_path(A0 + 2, B0, C0, 256, 256, 256) == Path.TC_EDGE
+    assert tg.select_path(A0, B0, C0, 3001, 5003, 1021) == Path.RC
+    assert tg.select_path(A0, B0, C0, 777, 12289, 4095) == Path.RC
+    assert tg.select_path(A0, B0, C0, 8191, 129, 8193) == Path.RC
+    assert tg.select_path(A0 + 2, B0, C0, 256, 256, 256) == Path.RC
 
 
 def test_forced_path_requirements():
@@ -146,7 +146,7 @@ def test_workspace_size_and_repack_choice():
     need = tg.workspace_size(A0, B0, C0, M, N, K)
     assert tg.select_path_ws(A0, B0, C0, M, N, K, need) == Path.REPACK
     assert tg.select_path_ws(A0, B0, C0, M, N, K, ab) == Path.REPACK                # A and B copies only
-    assert tg.select_path_ws(A0, B0, C0, M, N, K, ab - 1) == Path.TC_EDGE
+    assert tg.select_path_ws(A0, B0, C0, M, N, K, ab - 1) == Path.RC
     assert tg.select_path_ws(A0, B0, C0, 4096, 4096, 4096, need) == Path.TC_PAIR512
 
 
@@ -221,9 +221,9 @@ def test_extended_options_validation_and_paths():
                                                                  stride_c=64 * 128)) == Path.SKINNY
     # Padded strides that are multiples of 8 keep TMA; others need the repack path.
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=520, ldb=528, ldc=536)) == Path.TC_PAIR
-    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513)) == Path.TC_EDGE
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513)) == Path.RC
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513), 1 << 30) == Path.REPACK
-    # B stored N x K with an odd K: only the repack path (the edge mode reads K x N).
+    # B stored N x K with an odd K: only the repack path (the no-scratch kernels read B stored K x N).
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 511, tg.options(b_layout=tg.B_NK)) == Path.REPACK
     up = lambda x: (x + 255) // 256 * 256
     assert tg.workspace_size_ex(A0, B0, C0, 300, 200, 511, tg.options(b_layout=tg.B_NK)) == up(2 * 300 * 512) + up(2 * 200 * 512)

@@ -37,6 +37,7 @@ class Path(enum.IntEnum):
     TC_PAIR = 6
     TC_PAIR512 = 7
     REPACK = 8
+    RC = 9
 
 
 class TGError(RuntimeError):

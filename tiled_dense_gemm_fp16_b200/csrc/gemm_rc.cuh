@@ -1,0 +1,614 @@
+// gemm_rc.cuh -- C = ReLU(A . B) when TMA cannot describe A (or B) as they
+// are: row strides that are not a multiple of 16 bytes, or bases that are not
+// 16-byte aligned.  No scratch memory: every operand is read in place.
+//
+// The tile model is the quick-start kernel's ("TileLang" wiki page,
+// "Programming model": a ceildiv grid of output tiles, A and B tiles staged
+// in shared memory through a pipelined K loop, a cleared fp32 accumulator,
+// tile MMAs, max(acc, 0), fp16 output).  What changes is how the tiles are
+// staged when the rows are misaligned.
+//
+// Residue classes of A's rows.  With A's row stride lda (elements), the rows
+// r and r + 8 start 16*lda bytes apart, a multiple of 16.  So the rows of one
+// class {r : r mod 8 = s} form a matrix with a 16-byte row stride whose rows
+// all start e_s elements (0..7) past a 16-byte boundary.  One tensor map per
+// class (base rounded down to 16 bytes, inner extent K + e_s) then loads a
+// class's rows with 128-byte swizzle straight into the MMA's K-major layout,
+// each row shifted by the same e_s elements: map column x holds A[r][x - e_s].
+// Every output tile takes its 128 rows from one class, and the k-block kb
+// loads map columns [64 kb, 64 kb + 64), that is A[r][64 kb - e_s + j].  The
+// shift is undone on the other operand: the B tile of the same k-block holds
+// the k-rows 64 kb - e_s + j, which is a row offset of B, and TMA takes any
+// row offset (negative rows read as zero).  The first k-block's A columns
+// with k < 0 (the previous row's tail, or bytes just before A) are cleared in
+// shared memory before its MMAs; columns k >= K read as zero.  Output row
+// 8 q + s of C is row q of class s (lda a multiple of 8: one class).
+//
+// B as it is, when TMA can describe it: 64-column boxes with 128-byte
+// swizzle at row offset 64 kb - e_s (the MN-major operand).  Otherwise B's
+// k-rows fall into residue classes the same way (k mod 8), one tensor map per
+// class loads each class's rows unswizzled, with 8 spare columns, into a
+// staging buffer, and four realigning warps shift every row into the swizzled
+// operand tile: two aligned 16-byte shared-memory reads and a funnel shift per
+// 16-byte chunk.  Their lane order keeps both the reads and the swizzled
+// writes free of bank conflicts.
+//
+// C is written with aligned 16-byte stores: each epilogue thread owns one row
+// of the tile and shifts its values into the 16-byte blocks of that row
+// (RowWriter); only the partial blocks at the two ends of a row's piece are
+// written element by element.
+//
+// Shapes with few tiles (one narrow column of tiles, N <= 240 say) split K
+// over a cluster of CTAs: each keeps its fp32 partial in shared memory and,
+// after a cluster barrier, sums a share of the tile's rows over the
+// cluster's partials in rank order (distributed shared memory), the small-M
+// path's reduction turned on its side.  Every wait is bounded.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace tg {
+
+constexpr int kRcClasses = 8;
+
+// Tensor maps of one call: A per residue class of rows; B either one map of
+// the whole matrix (direct mode, b[0]) or one per residue class of k-rows.
+struct RcMaps {
+  CUtensorMap a[kRcClasses];
+  CUtensorMap b[kRcClasses];
+};
+
+struct RcParams {
+  __half* C;
+  const __half* bias;      // optional fp16[N] added before ReLU; nullptr = none
+  int64_t ldc;             // row stride of C (elements)
+  int M, N, K;
+  int a_classes;           // 8, or 1 when A's row stride is a multiple of 8 elements
+  int b_classes;           // staging mode: 8, or 1 when B's row stride is a multiple of 8
+  int a_shift[kRcClasses]; // e_s: elements between the class map's column 0 and A[r][0]
+  int b_shift[kRcClasses]; // f_t: the same for B's classes (staging mode)
+  int rows_in_class[kRcClasses];
+  int tile_start[kRcClasses + 1];  // first 128-row tile of each class; [a_classes] = m_tiles
+  int m_tiles, n_tiles, num_tiles, group_m;
+  int bn;                  // tile width: 256, or N rounded up to 16 when N <= 240
+  int panels;              // 64-column panels of the B tile: ceil(bn / 64)
+  int halves;              // staging: column halves of the B tile (2 when bn > 240)
+  int hw;                  // staging: columns per half
+  int bw;                  // staging: box width, hw + 8
+  int ring_stages, stg_slots;
+  int ring_stage_bytes;    // 16 KiB of A + panels x 8 KiB of B
+  int stg_bytes;           // halves x 64 x bw x 2
+  int splits;              // CTAs per cluster along K (split mode)
+  int c_stride;            // split mode: bytes per row of the fp32 partial (bn * 4 + 16)
+  uint32_t idesc;
+  uint64_t wait_budget_ns;
+};
+
+template <bool STAGE_B>
+struct RcCfg {
+  static constexpr int BM = 128;
+  static constexpr int BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;   // 16 KiB
+  static constexpr int PANEL_BYTES = BK * 64 * 2;  // 8 KiB: 64 k-rows x 64 columns
+  static constexpr int MMA_WARP = 1;
+  static constexpr int EPI_WARP0 = 2;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int REAL_WARP0 = EPI_WARP0 + EPI_WARPS;
+  static constexpr int REAL_WARPS = STAGE_B ? 4 : 0;
+  static constexpr int THREADS = (REAL_WARP0 + REAL_WARPS) * 32;
+  static constexpr int MAX_RING = 8;
+  static constexpr int MAX_STG = 4;
+  static constexpr int BAR_BYTES = 512;
+};
+
+// Writes one piece of a row of C, columns [c0, c0 + count), from values that
+// arrive 32 at a time as 16 packed fp16 pairs in column order (the first
+// chunk starting at c0).  The row piece starts g elements (0..7) past a
+// 16-byte boundary; block b covers the elements [8 b - g, 8 b - g + 8) of the
+// piece.  Blocks wholly inside the piece leave as one 16-byte store; the
+// partial blocks at either end are written element by element, so nothing
+// outside the piece is touched.
+struct RowWriter {
+  unsigned short* blk0;  // 16-byte aligned: element 0 of block 0
+  int lo, hi;            // element indices (from blk0) inside the piece: [g, g + count)
+  uint32_t g;
+  int next;              // next block to write
+  uint4 carry;           // the previous chunk's last 8 values
+};
+
+__device__ __forceinline__ void rw_init(RowWriter& w, __half* piece, int count) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(piece);
+  w.g = static_cast<uint32_t>((a >> 1) & 7u);
+  w.blk0 = reinterpret_cast<unsigned short*>(a - 2u * w.g);
+  w.lo = static_cast<int>(w.g);
+  w.hi = static_cast<int>(w.g) + count;
+  w.next = 0;
+  w.carry = make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ void rw_emit(RowWriter& w, const uint4& v) {
+  const int s = 8 * w.next;
+  ++w.next;
+  if (s >= w.hi || s + 8 <= w.lo) return;
+  if (s >= w.lo && s + 8 <= w.hi) {
+    __stcs(reinterpret_cast<int4*>(w.blk0 + s), *reinterpret_cast<const int4*>(&v));
+    return;
+  }
+  const uint32_t words[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int idx = s + e;
+    if (idx >= w.lo && idx < w.hi) w.blk0[idx] = static_cast<unsigned short>(words[e >> 1] >> ((e & 1) * 16));
+  }
+}
+
+__device__ __forceinline__ void rw_push(RowWriter& w, const uint32_t (&h)[16]) {
+  const uint4 q0 = make_uint4(h[0], h[1], h[2], h[3]);
+  const uint4 q1 = make_uint4(h[4], h[5], h[6], h[7]);
+  const uint4 q2 = make_uint4(h[8], h[9], h[10], h[11]);
+  const uint4 q3 = make_uint4(h[12], h[13], h[14], h[15]);
+  if (w.g == 0) {
+    rw_emit(w, q0);
+    rw_emit(w, q1);
+    rw_emit(w, q2);
+    rw_emit(w, q3);
+    return;
+  }
+  // Block b starts (8 - g) elements into the pair (previous 8 values, next 8).
+  const uint32_t sh = 16u - 2u * w.g;
+  rw_emit(w, edge_realign(w.carry, q0, sh));
+  rw_emit(w, edge_realign(q0, q1, sh));
+  rw_emit(w, edge_realign(q1, q2, sh));
+  rw_emit(w, edge_realign(q2, q3, sh));
+  w.carry = q3;
+}
+
+// The block holding the piece's last g values (nothing when g == 0).
+__device__ __forceinline__ void rw_finish(RowWriter& w) {
+  if (w.g != 0) rw_emit(w, edge_realign(w.carry, make_uint4(0u, 0u, 0u, 0u), 16u - 2u * w.g));
+}
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint4& v) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+}
+
+__device__ __forceinline__ void st_shared_u4(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// One output tile: class s, rows q0 .. q0 + 127 of the class, columns
+// n0 .. n0 + bn - 1, and this CTA's k-blocks [kb_lo, kb_hi) of the class's
+// ceil((K + e) / 64).
+struct RcTile {
+  int s, q0, n0, e, kb_lo, kb_hi;
+};
+
+__device__ __forceinline__ RcTile rc_tile(const RcParams& p, int t, int rank, int splits) {
+  const int group_tiles = p.group_m * p.n_tiles;
+  const int g = t / group_tiles;
+  const int first = g * p.group_m;
+  const int gm = min(p.m_tiles - first, p.group_m);
+  const int local = t - g * group_tiles;
+  const int mt = first + local % gm;
+  RcTile r;
+  r.n0 = (local / gm) * p.bn;
+  int s = 0;
+#pragma unroll
+  for (int c = 1; c < kRcClasses; ++c)
+    if (c < p.a_classes && p.tile_start[c] <= mt) s = c;
+  r.s = s;
+  r.q0 = (mt - p.tile_start[s]) * 128;
+  r.e = p.a_shift[s];
+  const int kb_total = (p.K + r.e + 63) / 64;
+  r.kb_lo = static_cast<int>((static_cast<int64_t>(kb_total) * rank) / splits);
+  r.kb_hi = static_cast<int>((static_cast<int64_t>(kb_total) * (rank + 1)) / splits);
+  return r;
+}
+
+template <bool STAGE_B, bool SPLIT>
+__global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
+    gemm_relu_rc_kernel(const __grid_constant__ RcMaps maps, const RcParams p) {
+  using Cfg = RcCfg<STAGE_B>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint8_t* stg = smem + p.ring_stages * p.ring_stage_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (STAGE_B ? p.stg_slots * p.stg_bytes : 0));
+  uint64_t* full_bar = bars;                       // [ring] TMA bytes landed
+  uint64_t* empty_bar = bars + Cfg::MAX_RING;      // [ring] MMAs done with the slot
+  uint64_t* bfull_bar = bars + 2 * Cfg::MAX_RING;  // [ring] realigned B written (staging mode)
+  uint64_t* stg_full = bars + 3 * Cfg::MAX_RING;   // [stg]
+  uint64_t* stg_empty = stg_full + Cfg::MAX_STG;   // [stg]
+  uint64_t* acc_full = stg_empty + Cfg::MAX_STG;   // [2]
+  uint64_t* acc_empty = acc_full + 2;              // [2]
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = SPLIT ? static_cast<int>(cluster_ctarank()) : 0;
+  const int splits = SPLIT ? p.splits : 1;
+  const int t_first = SPLIT ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
+  const int t_step = SPLIT ? p.num_tiles : static_cast<int>(gridDim.x);
+  constexpr uint32_t kTmemCols = SPLIT ? 256 : 512;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.ring_stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      mbar_init(&bfull_bar[s], Cfg::REAL_WARPS > 0 ? Cfg::REAL_WARPS : 1);
+    }
+    for (int s = 0; s < p.stg_slots; ++s) {
+      mbar_init(&stg_full[s], 1);
+      mbar_init(&stg_empty[s], Cfg::REAL_WARPS);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], Cfg::EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == Cfg::MMA_WARP) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  tcgen05_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------
+    // Producer: A's class boxes into the ring; B into the ring (direct) or
+    // its class boxes into the staging buffers.
+    // ------------------------------------------------------------------
+    if (lane == 0) {
+      int r = 0, q = 0;
+      uint32_t rph = 0, qph = 0;
+      int last_full[Cfg::MAX_RING], last_stg[Cfg::MAX_STG];
+      for (int i = 0; i < Cfg::MAX_RING; ++i) last_full[i] = -1;
+      for (int i = 0; i < Cfg::MAX_STG; ++i) last_stg[i] = -1;
+      const int cb = p.b_classes;
+      const int box_rows = 64 / cb;
+      bool ok = true;
+      for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
+        const RcTile T = rc_tile(p, t, rank, splits);
+        for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
+          if (!mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x61)) {
+            ok = false;
+            break;
+          }
+          uint8_t* slot = ring + r * p.ring_stage_bytes;
+          const int k_lo = kb * 64 - T.e;  // B's first k-row of this block
+          mbar_arrive_expect_tx(&full_bar[r], STAGE_B ? Cfg::A_BYTES : Cfg::A_BYTES + p.panels * Cfg::PANEL_BYTES);
+          tma_load_2d(slot, &maps.a[T.s], &full_bar[r], kb * 64, T.q0);
+          if (!STAGE_B) {
+            for (int c = 0; c < p.panels; ++c)
+              tma_load_2d(slot + Cfg::A_BYTES + c * Cfg::PANEL_BYTES, &maps.b[0], &full_bar[r], T.n0 + 64 * c, k_lo);
+          } else {
+            if (!mbar_wait(&stg_empty[q], qph ^ 1u, abort_flag, p.wait_budget_ns, 0x62)) {
+              ok = false;
+              last_full[r] = static_cast<int>(rph);  // A's box is in flight
+              break;
+            }
+            mbar_arrive_expect_tx(&stg_full[q], static_cast<uint32_t>(p.stg_bytes));
+            uint8_t* sbuf = stg + q * p.stg_bytes;
+            for (int h = 0; h < p.halves; ++h) {
+              for (int tc = 0; tc < cb; ++tc) {
+                // First k-row of class tc at or after k_lo, and its row in the class map.
+                const int kt = k_lo + (((tc - k_lo) % cb) + cb) % cb;
+                const int y = (kt - tc) / cb;
+                tma_load_2d(sbuf + (h * 64 + tc * box_rows) * p.bw * 2, &maps.b[tc], &stg_full[q],
+                            T.n0 + h * p.hw, y);
+              }
+            }
+            last_stg[q] = static_cast<int>(qph);
+            if (++q == p.stg_slots) {
+              q = 0;
+              qph ^= 1u;
+            }
+          }
+          last_full[r] = static_cast<int>(rph);
+          if (++r == p.ring_stages) {
+            r = 0;
+            rph ^= 1u;
+          }
+        }
+      }
+      // Every load issued has landed before the CTA may exit.
+      volatile int no_abort = 0;
+      for (int i = 0; i < p.stg_slots; ++i)
+        if (last_stg[i] >= 0) mbar_wait(&stg_full[i], static_cast<uint32_t>(last_stg[i]), &no_abort, p.wait_budget_ns, 0x63);
+      for (int i = 0; i < p.ring_stages; ++i)
+        if (last_full[i] >= 0)
+          mbar_wait(&full_bar[i], static_cast<uint32_t>(last_full[i]), &no_abort, p.wait_budget_ns, 0x64);
+    }
+  } else if (warp == Cfg::MMA_WARP) {
+    // ------------------------------------------------------------------
+    // MMA issuer (lane 0), with the whole warp clearing the first k-block's
+    // A columns that lie before k = 0.
+    // ------------------------------------------------------------------
+    int r = 0, local = 0;
+    uint32_t rph = 0;
+    bool ok = true;
+    for (int t = t_first; t < p.num_tiles && ok; t += t_step, ++local) {
+      const RcTile T = rc_tile(p, t, rank, splits);
+      const int acc = SPLIT ? 0 : (local & 1);
+      const uint32_t acc_phase = SPLIT ? 0u : static_cast<uint32_t>((local >> 1) & 1);
+      if (!SPLIT) {
+        const bool free_acc = mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, p.wait_budget_ns, 0x65);
+        if (!__all_sync(0xffffffffu, free_acc)) break;
+      }
+      tcgen05_fence_after_sync();
+      const uint32_t d_tmem = tmem_base + acc * 256;
+      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
+        bool landed = mbar_wait(&full_bar[r], rph, abort_flag, p.wait_budget_ns, 0x66);
+        if (STAGE_B) landed = landed && mbar_wait(&bfull_bar[r], rph, abort_flag, p.wait_budget_ns, 0x6C);
+        if (!__all_sync(0xffffffffu, landed)) {
+          ok = false;
+          break;
+        }
+        tcgen05_fence_after_sync();
+        uint8_t* slot = ring + r * p.ring_stage_bytes;
+        if (kb == 0 && T.e > 0) {
+          // Columns j < e of k-block 0 are k < 0: clear them (chunk 0 of
+          // each swizzled 128-byte row sits at (row & 7) * 16).
+          const uint32_t keep_from = static_cast<uint32_t>(T.e);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int row = lane + 32 * i;
+            const uint32_t addr = smem_u32(slot) + row * 128 + ((row & 7) << 4);
+            uint4 v;
+            ld_shared_v4(addr, v);
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (static_cast<uint32_t>(e) < keep_from) w[e >> 1] &= (e & 1) ? 0x0000ffffu : 0xffff0000u;
+            st_shared_u4(addr, make_uint4(w[0], w[1], w[2], w[3]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(slot);
+          const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
+            const uint64_t bdesc = make_sw128_desc(b_addr + k * 2048, Cfg::PANEL_BYTES, 1024);
+            umma_f16_ss(d_tmem, adesc, bdesc, p.idesc, (kb != T.kb_lo || k != 0) ? 1u : 0u);
+          }
+          umma_commit(&empty_bar[r]);
+        }
+        __syncwarp();
+        if (++r == p.ring_stages) {
+          r = 0;
+          rph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0 && T.kb_hi > T.kb_lo) umma_commit(&acc_full[acc]);
+      __syncwarp();
+    }
+    if (lane == 0) {
+      umma_commit(mma_done);
+      volatile int no_abort = 0;
+      mbar_wait(mma_done, 0, &no_abort, p.wait_budget_ns, 0x67);
+    }
+    __syncwarp();
+  } else if (warp < Cfg::REAL_WARP0) {
+    // ------------------------------------------------------------------
+    // Epilogue: TMEM -> registers -> (bias) ReLU -> fp16 -> C rows, or, in
+    // split mode, the fp32 partial into shared memory.
+    // ------------------------------------------------------------------
+    const int quad = warp & 3;
+    const int i = quad * 32 + lane;  // row of the tile = TMEM lane
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    if (!SPLIT) {
+      int local = 0;
+      for (int t = t_first; t < p.num_tiles; t += t_step, ++local) {
+        const RcTile T = rc_tile(p, t, rank, splits);
+        const int acc = local & 1;
+        const uint32_t acc_phase = static_cast<uint32_t>((local >> 1) & 1);
+        const bool ready = mbar_wait(&acc_full[acc], acc_phase, abort_flag, p.wait_budget_ns, 0x68);
+        if (!__all_sync(0xffffffffu, ready)) break;
+        tcgen05_fence_after_sync();
+        const int qrow = T.q0 + i;
+        const bool valid = qrow < p.rows_in_class[T.s];
+        const int64_t row = static_cast<int64_t>(qrow) * p.a_classes + T.s;
+        const int ncols = min(p.bn, p.N - T.n0);
+        RowWriter w;
+        if (valid) rw_init(w, p.C + row * p.ldc + T.n0, ncols);
+        for (int c = 0; c * 32 < ncols; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(lane_base + acc * 256 + c * 32, v);
+          tmem_ld_wait();
+          const int col0 = T.n0 + c * 32;
+          float b0[16], b1[16];
+          load_bias16(p.bias, col0, p.N, b0);
+          load_bias16(p.bias, col0 + 16, p.N, b1);
+          uint32_t h[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) h[e] = relu_pack_f16x2_bias(v[2 * e], v[2 * e + 1], b0[2 * e], b0[2 * e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            h[8 + e] = relu_pack_f16x2_bias(v[16 + 2 * e], v[17 + 2 * e], b1[2 * e], b1[2 * e + 1]);
+          if (valid) rw_push(w, h);
+        }
+        if (valid) rw_finish(w);
+        tcgen05_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
+    } else {
+      const RcTile T = rc_tile(p, t_first, rank, splits);
+      const bool has_k = T.kb_hi > T.kb_lo;
+      bool ready = true;
+      if (has_k) ready = mbar_wait(&acc_full[0], 0, abort_flag, p.wait_budget_ns, 0x69);
+      ready = __all_sync(0xffffffffu, ready);
+      if (ready) {
+        tcgen05_fence_after_sync();
+        const uint32_t prow = smem_u32(ring) + static_cast<uint32_t>(i * p.c_stride);
+        for (int c = 0; c * 16 < p.bn; ++c) {
+          uint32_t v[16];
+          if (has_k) {
+            tmem_ld_32x32b_x16(lane_base + c * 16, v);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0u;  // empty K share: the partial is zero
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            st_shared_u4(prow + c * 64 + e * 16, make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
+        }
+      }
+      tcgen05_fence_before_sync();
+    }
+  } else if (STAGE_B) {
+    // ------------------------------------------------------------------
+    // Realigning warps: staged class rows of B -> swizzled MN-major tile.
+    // Unit U = (lambda, d, seg): k-row j = 8 lambda + ((lambda + d) & 7)
+    // and its 64-column segment seg.  The 8 lanes of each shared-memory
+    // phase differ in lambda, so their reads hit 8 different 16-byte bank
+    // groups (staging rows are an odd number of 16-byte units long) and
+    // their swizzled writes too (j & 7 differs).
+    // ------------------------------------------------------------------
+    const int tid = threadIdx.x - Cfg::REAL_WARP0 * 32;
+    const int segs_per_half = (p.hw + 63) / 64;
+    const int units = 64 * p.panels;
+    int r = 0, q = 0;
+    uint32_t rph = 0, qph = 0;
+    bool ok = true;
+    for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
+      const RcTile T = rc_tile(p, t, rank, splits);
+      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
+        bool got = mbar_wait(&stg_full[q], qph, abort_flag, p.wait_budget_ns, 0x6A);
+        got = got && mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        const int k_lo = kb * 64 - T.e;
+        const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
+        const uint32_t bbase = smem_u32(ring + r * p.ring_stage_bytes) + Cfg::A_BYTES;
+        for (int U = tid; U < units; U += Cfg::REAL_WARPS * 32) {
+          const int lam = U & 7, d = (U >> 3) & 7, seg = U >> 6;
+          const int j = 8 * lam + ((lam + d) & 7);
+          int srow, f;
+          if (p.b_classes == 8) {
+            const int tc = (j + k_lo) & 7;
+            srow = 8 * tc + (j >> 3);
+            f = p.b_shift[tc];
+          } else {
+            srow = j;
+            f = p.b_shift[0];
+          }
+          const int h = seg / segs_per_half;
+          const int cih = 64 * (seg - h * segs_per_half);
+          const int nch = min(8, (p.hw - cih) >> 3);
+          const uint32_t src = sbase + static_cast<uint32_t>(((h * 64 + srow) * p.bw + cih) * 2);
+          uint4 blk[9];
+#pragma unroll
+          for (int c = 0; c < 9; ++c) {
+            blk[c] = make_uint4(0u, 0u, 0u, 0u);
+            if (c <= nch) ld_shared_v4(src + c * 16, blk[c]);
+          }
+          const uint32_t dst = bbase + static_cast<uint32_t>(seg * Cfg::PANEL_BYTES + j * 128);
+          const uint32_t sh = 2u * static_cast<uint32_t>(f);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), edge_realign(blk[c], blk[c + 1], sh));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bfull_bar[r]);
+          mbar_arrive(&stg_empty[q]);
+        }
+        if (++r == p.ring_stages) {
+          r = 0;
+          rph ^= 1u;
+        }
+        if (++q == p.stg_slots) {
+          q = 0;
+          qph ^= 1u;
+        }
+      }
+    }
+  }
+
+  if (SPLIT) {
+    // Sum this CTA's share of the tile's rows over the cluster's partials.
+    __syncthreads();
+    cluster_sync();
+    if (warp >= Cfg::EPI_WARP0 && warp < Cfg::REAL_WARP0 && !*abort_flag) {
+      const RcTile T = rc_tile(p, t_first, rank, splits);
+      const int tid = threadIdx.x - Cfg::EPI_WARP0 * 32;
+      const int r_lo = (128 * rank) / splits, r_hi = (128 * (rank + 1)) / splits;
+      const int nrows = r_hi - r_lo;
+      const int ncols = min(p.bn, p.N - T.n0);
+      const int segs = (ncols + 63) / 64;
+      const uint32_t part = smem_u32(ring);
+      for (int it = tid; it < nrows * segs; it += Cfg::EPI_WARPS * 32) {
+        const int i = r_lo + it % nrows;
+        const int seg = it / nrows;
+        const int qrow = T.q0 + i;
+        if (qrow >= p.rows_in_class[T.s]) continue;
+        const int64_t row = static_cast<int64_t>(qrow) * p.a_classes + T.s;
+        const int c0 = 64 * seg, c1 = min(c0 + 64, ncols);
+        RowWriter w;
+        rw_init(w, p.C + row * p.ldc + T.n0 + c0, c1 - c0);
+        for (int cc = c0; cc < c1; cc += 32) {
+          float acc[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
+          const uint32_t off = static_cast<uint32_t>(i * p.c_stride + cc * 4);
+          for (int qr = 0; qr < splits; ++qr) {
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4) {
+              const float4 x = ld_shared_cluster_f4(mapa_shared(part + off + v4 * 16, static_cast<uint32_t>(qr)));
+              acc[4 * v4] += x.x;
+              acc[4 * v4 + 1] += x.y;
+              acc[4 * v4 + 2] += x.z;
+              acc[4 * v4 + 3] += x.w;
+            }
+          }
+          float b0[16], b1[16];
+          load_bias16(p.bias, T.n0 + cc, p.N, b0);
+          load_bias16(p.bias, T.n0 + cc + 16, p.N, b1);
+          uint32_t h[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            h[e] = relu_pack_f16x2_bias(__float_as_uint(acc[2 * e]), __float_as_uint(acc[2 * e + 1]), b0[2 * e],
+                                        b0[2 * e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            h[8 + e] = relu_pack_f16x2_bias(__float_as_uint(acc[16 + 2 * e]), __float_as_uint(acc[17 + 2 * e]),
+                                            b1[2 * e], b1[2 * e + 1]);
+          rw_push(w, h);
+        }
+        rw_finish(w);
+      }
+    }
+    cluster_sync();  // peers are done reading this CTA's partial
+  }
+
+  tcgen05_fence_before_sync();
+  __syncthreads();
+  if (warp == Cfg::MMA_WARP) {
+    tcgen05_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace tg

@@ -16,6 +16,7 @@
 
 #include "tg_gemm.h"
 #include "gemm_mx.cuh"
+#include "gemm_rc.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc_pair.cuh"
@@ -47,6 +48,7 @@ struct DeviceInfo {
   bool skinny_attr = false;
   unsigned tc_pair_attr = 0;  // one bit per (stages, tile width) instance with its attribute set
   bool mx_attr[2] = {false, false};       // per block-scaled kind
+  unsigned rc_attr = 0;       // one bit per residue-class kernel instance with its attribute set
   bool w4_attr = false;
   bool w4_decode_attr = false;
   void* static_ws = nullptr;  // device address of g_static_workspace on this device
@@ -245,6 +247,11 @@ RepackPlan chosen_plan(const Problem& p, int64_t ws_bytes) {
   return ws_bytes >= full.bytes ? full : repack_plan(p, false);
 }
 
+// The residue-class kernel reads A stored M x K and B stored K x N; when it
+// realigns B's rows in shared memory, each of B's eight row classes needs a
+// row (K >= 8).
+bool rc_ok(const Problem& p) { return !p.a_km && !p.b_nk && (tma_ok_b(p) || p.K >= 8); }
+
 bool path_supports(int path, const Problem& p) {
   if (!problem_valid(p)) return false;
   if (p.M == 0 || p.N == 0) return path == TG_PATH_NONE || path == TG_PATH_AUTO;
@@ -262,6 +269,8 @@ bool path_supports(int path, const Problem& p) {
       return tma_ok(p) && p.M <= kSkinnyMaxM && !p.a_km;
     case TG_PATH_REPACK:
       return !tma_ok(p) || c_pad_useful(p);
+    case TG_PATH_RC:
+      return rc_ok(p);
     default:
       return false;
   }
@@ -304,7 +313,7 @@ int select_path(const Problem& p, int64_t ws_bytes) {
   if (p.K == 0) return TG_PATH_ZERO;
   if (!tma_ok(p)) {
     if (ws_bytes >= repack_plan(p, false).bytes || p.b_nk || p.a_km) return TG_PATH_REPACK;
-    return TG_PATH_TC_EDGE;
+    return rc_ok(p) ? TG_PATH_RC : TG_PATH_TC_EDGE;
   }
   // Operands TMA can read, but C's rows are not 16-byte aligned: the GEMM
   // writes a padded C in the workspace when there is room for it.
@@ -631,6 +640,160 @@ tg_status launch_skinny(const Operands& o, cudaStream_t stream, DeviceInfo* info
   return TG_OK;
 }
 
+
+// Tensor map of a row-major fp16 matrix given by a 16-byte aligned base, its
+// inner extent (elements), row count and row stride in bytes.
+bool encode_2d_raw(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int64_t stride_bytes,
+                   int box_inner, int box_rows, CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Residue classes of a row-major matrix's rows: `classes` maps, class c
+// holding rows c, c + classes, ...  Each map starts at the 16-byte boundary at
+// or below its first row and is `shift[c]` elements wider than the rows
+// (column x of the map is element x - shift[c] of a row).  Classes without a
+// row get no map (rows[c] = 0).
+bool encode_classes(CUtensorMap* maps, const void* base, int64_t rows, int64_t cols, int64_t ld, int classes,
+                    int box_inner, int box_rows, CUtensorMapSwizzle swizzle, int* shift, int* class_rows) {
+  for (int c = 0; c < classes; ++c) {
+    const int64_t n = rows > c ? (rows - c + classes - 1) / classes : 0;
+    class_rows[c] = static_cast<int>(n);
+    shift[c] = 0;
+    if (n == 0) continue;
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(base) + static_cast<uintptr_t>(2 * c * ld);
+    const uintptr_t aligned = addr & ~uintptr_t(15);
+    shift[c] = static_cast<int>((addr - aligned) / 2);
+    if (!encode_2d_raw(&maps[c], reinterpret_cast<const void*>(aligned), cols + shift[c], n, 2 * classes * ld,
+                       box_inner, box_rows, swizzle))
+      return false;
+  }
+  return true;
+}
+
+template <bool STAGE_B, bool SPLIT>
+tg_status launch_rc_cfg(const RcMaps& maps, const RcParams& p, int smem, int grid_x, int grid_y,
+                        cudaStream_t stream, DeviceInfo* info) {
+  auto kernel = gemm_relu_rc_kernel<STAGE_B, SPLIT>;
+  constexpr unsigned kBit = 1u << ((STAGE_B ? 1 : 0) + (SPLIT ? 2 : 0));
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!(info->rc_attr & kBit)) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess) {
+        cudaGetLastError();
+        return TG_ERR_LAUNCH;
+      }
+      info->rc_attr |= kBit;
+    }
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(grid_x), static_cast<unsigned>(grid_y), 1);
+  cfg.blockDim = dim3(RcCfg<STAGE_B>::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  LaunchAttrs la;
+  la.fill(cfg, SPLIT ? static_cast<unsigned>(p.splits) : 1u);
+  if (cudaLaunchKernelEx(&cfg, kernel, maps, p) != cudaSuccess) {
+    cudaGetLastError();
+    return TG_ERR_LAUNCH;
+  }
+  return TG_OK;
+}
+
+// Residue-class path: see gemm_rc.cuh.
+tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
+  const int64_t M = o.M, N = o.N, K = o.K;
+  RcMaps maps;
+  std::memset(&maps, 0, sizeof maps);
+  RcParams p;
+  std::memset(&p, 0, sizeof p);
+  p.C = static_cast<__half*>(o.C);
+  p.bias = static_cast<const __half*>(o.bias);
+  p.ldc = o.ldc;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  // One class when the row stride is a multiple of 8 elements and covers the
+  // widened rows; else the eight residue classes of the rows.
+  const int e0 = static_cast<int>((reinterpret_cast<uintptr_t>(o.A) & 15u) / 2);
+  p.a_classes = (o.lda % 8 == 0 && o.lda >= K + e0) ? 1 : kRcClasses;
+  if (!encode_classes(maps.a, o.A, M, K, o.lda, p.a_classes, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, p.a_shift,
+                      p.rows_in_class))
+    return TG_ERR_LAUNCH;
+  int mt = 0, kb_max = 0;
+  for (int c = 0; c < p.a_classes; ++c) {
+    p.tile_start[c] = mt;
+    mt += (p.rows_in_class[c] + 127) / 128;
+    const int kb = static_cast<int>((K + p.a_shift[c] + 63) / 64);
+    kb_max = kb > kb_max ? kb : kb_max;
+  }
+  p.tile_start[p.a_classes] = mt;
+  p.m_tiles = mt;
+  p.bn = N <= 240 ? static_cast<int>((N + 15) / 16 * 16) : 256;
+  p.n_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
+  p.num_tiles = p.m_tiles * p.n_tiles;
+  p.panels = (p.bn + 63) / 64;
+  p.group_m = tune_int("TG_TUNE_RC_GROUP_M", 8);
+  if (p.group_m < 1) p.group_m = 1;
+  const bool stage_b = !((reinterpret_cast<uintptr_t>(o.B) & 15u) == 0 && o.ldb % 8 == 0);
+  if (stage_b) {
+    if (K < kRcClasses) return TG_ERR_INVALID_ARG;
+    const int f0 = static_cast<int>((reinterpret_cast<uintptr_t>(o.B) & 15u) / 2);
+    p.b_classes = (o.ldb % 8 == 0 && o.ldb >= N + f0) ? 1 : kRcClasses;
+    p.halves = p.bn > 240 ? 2 : 1;
+    p.hw = p.bn / p.halves;
+    p.bw = p.hw + 8;
+    int b_rows[kRcClasses];
+    if (!encode_classes(maps.b, o.B, K, N, o.ldb, p.b_classes, p.bw, 64 / p.b_classes, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        p.b_shift, b_rows))
+      return TG_ERR_LAUNCH;
+    p.stg_bytes = p.halves * 64 * p.bw * 2;
+    p.stg_slots = 2;
+  } else if (!encode_2d(&maps.b[0], o.B, K, N, o.ldb, 64, 64)) {
+    return TG_ERR_LAUNCH;
+  }
+  p.ring_stage_bytes = RcCfg<false>::A_BYTES + p.panels * RcCfg<false>::PANEL_BYTES;
+  constexpr int kSmemMax = 232448, kFixed = 1024 + 512;
+  int ring = (kSmemMax - kFixed - p.stg_slots * p.stg_bytes) / p.ring_stage_bytes;
+  ring = ring > RcCfg<false>::MAX_RING ? RcCfg<false>::MAX_RING : ring;
+  if (ring < 2) return TG_ERR_INTERNAL;
+  p.ring_stages = ring;
+  p.c_stride = p.bn * 4 + 16;
+  p.idesc = make_idesc_f16_f32(128, p.bn, false, true);
+  p.wait_budget_ns = wait_budget(kb_max);
+  const int smem = kFixed + ring * p.ring_stage_bytes + p.stg_slots * p.stg_bytes;
+  // Few tiles: split K over a cluster (each CTA keeps at least 4 k-blocks),
+  // when the fp32 partial fits in the ring.
+  const int sms = info->sm_count;
+  int splits = 1;
+  if (2 * p.num_tiles <= sms && 128 * p.c_stride <= ring * p.ring_stage_bytes) {
+    splits = sms / p.num_tiles;
+    const int kb_min = static_cast<int>((K + 63) / 64);
+    splits = splits > 8 ? 8 : splits;
+    while (splits > 1 && kb_min / splits < 4) --splits;
+    splits = tune_int("TG_TUNE_RC_SPLITS", splits);
+    if (splits > 8) splits = 8;
+  }
+  p.splits = splits;
+  if (splits > 1) {
+    if (p.num_tiles > 65535) return TG_ERR_INVALID_ARG;
+    return stage_b ? launch_rc_cfg<true, true>(maps, p, smem, splits, p.num_tiles, stream, info)
+                   : launch_rc_cfg<false, true>(maps, p, smem, splits, p.num_tiles, stream, info);
+  }
+  const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  return stage_b ? launch_rc_cfg<true, false>(maps, p, smem, grid, 1, stream, info)
+                 : launch_rc_cfg<false, false>(maps, p, smem, grid, 1, stream, info);
+}
+
 __global__ void wait_timeout_selftest_kernel(uint64_t budget_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -659,6 +822,8 @@ tg_status launch_path(int path, const Operands& o, cudaStream_t stream, DeviceIn
       return launch_tc_pair(o, stream, info, 256);
     case TG_PATH_TC_PAIR512:
       return launch_tc_pair(o, stream, info, 512);
+    case TG_PATH_RC:
+      return launch_rc(o, stream, info);
     default:
       return TG_ERR_INTERNAL;
   }
@@ -1407,6 +1572,7 @@ const char* tg_path_name(int path) {
     case TG_PATH_TC_PAIR: return "tc_pair";
     case TG_PATH_TC_PAIR512: return "tc_pair512";
     case TG_PATH_REPACK: return "repack";
+    case TG_PATH_RC: return "rc";
     default: return "invalid";
   }
 }
