@@ -120,7 +120,7 @@ def test_rc_infinities_do_not_leak_into_the_next_row(M, N, K, a_off):
 def test_rc_strides_bias_batches(M, N, K, strides, bias):
     from test_gpu_layouts import STRIDES, run_ex
     lda, ldb, ldc = STRIDES[strides](M, N, K, False)
-    got, ref, guards = run_ex(M, N, K, lda=lda, ldb=ldb, ldc=ldc, b_nk=False, bias=bias, batch=2, gap=3,
+    got, ref, guards = run_ex(M, N, K, lda=lda, ldb=ldb, ldc=ldc, b_nk=False, bias=bias, batch=2, gap=40,
                               seed=M + K, path=RC, workspace=False)
     assert guards
     for e, (g, r) in enumerate(zip(got, ref)):
