@@ -86,8 +86,8 @@ typedef enum tg_path {
                             A's rows are loaded by TMA in residue classes
                             (row mod 8, rows sharing one 16-byte offset),
                             B's k-rows shifted to match; B realigned in
-                            shared memory when TMA cannot describe it (then
-                            K >= 8); A stored M x K, B stored K x N only    */
+                            shared memory when TMA cannot describe it;
+                            A stored M x K, B stored K x N only             */
 } tg_path;
 
 /*

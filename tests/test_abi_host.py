@@ -133,17 +133,25 @@ def test_workspace_size_and_repack_choice():
     assert tg.select_path(A0, B0, C0 + 2, 512, 512, 512) == Path.TC_PAIR
     assert tg.select_path_ws(A0, B0, C0 + 2, 512, 512, 512, up(2 * 512 * 512)) == Path.REPACK
     assert tg.select_path_ws(A0, B0, C0 + 2, 512, 512, 512, up(2 * 512 * 512) - 1) == Path.TC_PAIR
-    assert tg.workspace_size(A0, B0, C0, 512, 509, 512) == 2 * up(2 * 512 * 512)    # odd N: B copy and C copy
+    # Operands TMA cannot describe.  When 1/N + 1/K > 1/2400 the residue-class kernel takes
+    # them, needing at most a padded copy of B (rows rounded up to 8 elements, 256-byte aligned).
+    assert tg.workspace_size(A0, B0, C0, 512, 509, 512) == up(2 * 512 * 512)        # odd N: B copy only
+    assert tg.select_path_ws(A0, B0, C0, 512, 509, 512, up(2 * 512 * 512)) == Path.RC
     assert tg.workspace_size(A0, B0, C0 + 2, 64, 512, 512) == 0                      # the small-M kernel
-    # Odd K pads A to K rounded up to 8; odd N pads B, and C (odd N) too; each copy 256-byte aligned.
     M, N, K = 3001, 5003, 1021
-    ab = up(2 * M * 1024) + up(2 * K * 5008)
-    assert tg.workspace_size(A0, B0, C0, M, N, K) == ab + up(2 * M * 5008)
-    assert tg.workspace_size(A0, B0, C0, 8191, 129, 8193) == up(2 * 8191 * 8200) + up(2 * 8193 * 136) + up(2 * 8191 * 136)
-    assert tg.workspace_size(A0, B0, C0, 64, 64, 100) == up(2 * 64 * 104)          # only A (small M: no C copy)
-    assert tg.workspace_size(A0 + 2, B0, C0, 64, 64, 64) == up(2 * 64 * 64)        # misaligned A base
+    assert tg.workspace_size(A0, B0, C0, M, N, K) == up(2 * K * 5008)
+    assert tg.workspace_size(A0, B0, C0, 8191, 129, 8193) == up(2 * 8193 * 136)
+    assert tg.workspace_size(A0, B0, C0, 64, 64, 100) == 0                          # odd K: only A, read in place
+    assert tg.workspace_size(A0 + 2, B0, C0, 64, 64, 64) == 0                       # misaligned A base
     assert tg.workspace_size(A0, B0, C0, -1, 4, 4) == -1
+    for ws in (0, up(2 * K * 5008)):
+        assert tg.select_path_ws(A0, B0, C0, M, N, K, ws) == Path.RC
+    # Large N and K: the repack path (copies of A, B and C around the CTA-pair kernel) when the
+    # workspace holds its copies, the residue-class kernel otherwise.
+    M, N, K = 777, 12289, 4095
+    ab = up(2 * M * 4096) + up(2 * K * 12296)
     need = tg.workspace_size(A0, B0, C0, M, N, K)
+    assert need == ab + up(2 * M * 12296)
     assert tg.select_path_ws(A0, B0, C0, M, N, K, need) == Path.REPACK
     assert tg.select_path_ws(A0, B0, C0, M, N, K, ab) == Path.REPACK                # A and B copies only
     assert tg.select_path_ws(A0, B0, C0, M, N, K, ab - 1) == Path.RC
@@ -177,8 +185,11 @@ def test_environment_cannot_change_the_shipped_kernel_choice(monkeypatch):
 def test_padded_c_with_general_layouts():
     up = lambda x: (x + 255) // 256 * 256
     M, N, K = 1000, 1001, 512      # A and B describable by TMA in every layout below; C rows of 2002 bytes
-    for opts, b_copy in [(tg.options(), up(2 * K * 1008)),                     # B K x N: row of 1001 -> padded
-                         (tg.options(b_layout=tg.B_NK), 0),                     # B N x K: rows of K, aligned
+    # B K x N with rows of 1001: the residue-class kernel on a padded copy of B, writing C itself.
+    need = tg.workspace_size_ex(A0, B0, C0, M, N, K, tg.options())
+    assert need == up(2 * K * 1008)
+    assert tg.select_path_ex(A0, B0, C0, M, N, K, tg.options(), need) == Path.RC
+    for opts, b_copy in [(tg.options(b_layout=tg.B_NK), 0),                     # B N x K: rows of K, aligned
                          (tg.options(a_layout=tg.A_KM, ldb=1008), 0)]:          # A K x M (M % 8 == 0), B padded ld
         need = tg.workspace_size_ex(A0, B0, C0, M, N, K, opts)
         assert need == b_copy + up(2 * M * 1008), (opts.b_layout, opts.a_layout)
@@ -222,7 +233,7 @@ def test_extended_options_validation_and_paths():
     # Padded strides that are multiples of 8 keep TMA; others need the repack path.
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=520, ldb=528, ldc=536)) == Path.TC_PAIR
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513)) == Path.RC
-    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513), 1 << 30) == Path.REPACK
+    assert tg.select_path_ex(A0, B0, C0, 512, 512, 512, tg.options(lda=513), 1 << 30) == Path.RC
     # B stored N x K with an odd K: only the repack path (the no-scratch kernels read B stored K x N).
     assert tg.select_path_ex(A0, B0, C0, 512, 512, 511, tg.options(b_layout=tg.B_NK)) == Path.REPACK
     up = lambda x: (x + 255) // 256 * 256

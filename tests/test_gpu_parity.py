@@ -130,16 +130,22 @@ def test_misaligned_base_pointers_use_edge_mode(offset, M, N, K):
 # ---------------------------------------------------------------------------
 
 REPACK_SHAPES = [(1, 9, 7), (15, 17, 9), (129, 257, 65), (255, 129, 127), (300, 301, 299),
-                 (640, 520, 75), (1000, 1001, 1003), (16, 8191, 517), (257, 777, 1021)]
+                 (640, 520, 75), (1000, 1001, 1003), (16, 8191, 517), (257, 777, 1021),
+                 (200, 6001, 6001), (300, 8191, 5003), (129, 4999, 8193)]
 
 
 @pytest.mark.parametrize("M,N,K", REPACK_SHAPES)
 def test_repack_integer_bitexact(M, N, K):
-    """Odd row lengths: A and/or B copied into zero-padded rows, then a TMA kernel; C stored unaligned."""
+    """Odd row lengths with a workspace: the residue-class kernel on a padded copy of B, or, for large N
+    and K (1/N + 1/K <= 1/2400), A and B copied into zero-padded rows around the CTA-pair kernel with a
+    padded C copied back."""
+    import tiled_dense_gemm_fp16_b200 as tg
     A, B = inputs.operands(M, N, K, "int", seed=M + 3 * N + 5 * K)
+    want = Path.REPACK if 2400 * (N + K) <= N * K else Path.RC
+    assert tg.select_path_ws(1 << 12, 1 << 40, 1 << 41, M, N, K, 1 << 40) == want
     got, guards = run_gpu(A, B, workspace=True)
     assert guards, (M, N, K)
-    assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"repack {(M, N, K)}")
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"workspace route {(M, N, K)}")
 
 
 @pytest.mark.parametrize("offsets", [(1, 0, 0), (0, 3, 0), (0, 0, 5), (7, 2, 1), (0, 0, 4)])
@@ -183,12 +189,12 @@ def test_torch_api_allocates_workspace_itself():
     import tiled_dense_gemm_fp16_b200 as tg
     A, B = inputs.operands(257, 259, 261, "int", seed=4)
     Ad, Bd = torch.from_numpy(A).cuda(), torch.from_numpy(B).cuda()
-    C1 = tg.gemm_relu(Ad, Bd)                  # repack path, torch-allocated workspace
-    C2 = tg.gemm_relu(Ad, Bd, workspace=None)  # edge mode
+    C1 = tg.gemm_relu(Ad, Bd)                  # B copied into a torch-allocated workspace
+    C2 = tg.gemm_relu(Ad, Bd, workspace=None)  # no workspace
     torch.cuda.synchronize()
     ref = oracle.gemm_relu_f16(A, B)
-    assert_bitexact(C1.cpu().numpy(), ref, "torch api repack")
-    assert_bitexact(C2.cpu().numpy(), ref, "torch api edge")
+    assert_bitexact(C1.cpu().numpy(), ref, "torch api with workspace")
+    assert_bitexact(C2.cpu().numpy(), ref, "torch api without workspace")
 
 
 def test_random_shapes_fuzz():

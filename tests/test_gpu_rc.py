@@ -36,9 +36,9 @@ def test_rc_integer_bitexact(M, N, K):
     assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"rc {(M, N, K)}")
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 16, 3), (5, 64, 1), (100, 8, 7), (33, 520, 5)])
-def test_rc_short_k_with_describable_b(M, N, K):
-    """K < 8 needs B's rows describable by TMA (N % 8 == 0, aligned base): only A is misaligned."""
+@pytest.mark.parametrize("M,N,K", [(1, 16, 3), (5, 64, 1), (100, 8, 7), (33, 520, 5), (40, 9, 3), (300, 257, 1)])
+def test_rc_short_k(M, N, K):
+    """K < 8: fewer k-rows than row classes, with B describable by TMA or realigned."""
     A, B = inputs.operands(M, N, K, "int", seed=K + N)
     got, guards = run_gpu(A, B, RC)
     assert guards
@@ -130,6 +130,5 @@ def test_rc_strides_bias_batches(M, N, K, strides, bias):
 def test_rc_is_the_no_workspace_route_for_unaligned_rows():
     import tiled_dense_gemm_fp16_b200 as tg
     A0, B0, C0 = 0x10_0000_0000, 0x20_0000_0000, 0x30_0000_0000   # never dereferenced
-    for (M, N, K) in [(3001, 5003, 1021), (777, 12289, 4095), (8191, 129, 8193), (100, 8, 7)]:
+    for (M, N, K) in [(3001, 5003, 1021), (777, 12289, 4095), (8191, 129, 8193), (100, 8, 7), (100, 9, 7)]:
         assert tg.select_path(A0, B0, C0, M, N, K) == RC
-    assert tg.select_path(A0, B0, C0, 100, 9, 7) == Path.TC_EDGE   # K < 8 with unaligned B rows

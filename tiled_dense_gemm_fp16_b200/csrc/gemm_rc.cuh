@@ -54,33 +54,31 @@ namespace tg {
 
 constexpr int kRcClasses = 8;
 
-// Tensor maps of one call: A per residue class of rows; B either one map of
-// the whole matrix (direct mode, b[0]) or one per residue class of k-rows.
+// Tensor maps of one call: A per residue class of rows, and B as a whole
+// (direct mode only).
 struct RcMaps {
   CUtensorMap a[kRcClasses];
-  CUtensorMap b[kRcClasses];
+  CUtensorMap b;
 };
 
 struct RcParams {
   __half* C;
+  const __half* B;         // staging mode: B read in place by the realigning warps
   const __half* bias;      // optional fp16[N] added before ReLU; nullptr = none
+  int64_t ldb;             // row stride of B (elements)
   int64_t ldc;             // row stride of C (elements)
   int M, N, K;
   int a_classes;           // 8, or 1 when A's row stride is a multiple of 8 elements
-  int b_classes;           // staging mode: 8, or 1 when B's row stride is a multiple of 8
   int a_shift[kRcClasses]; // e_s: elements between the class map's column 0 and A[r][0]
-  int b_shift[kRcClasses]; // f_t: the same for B's classes (staging mode)
   int rows_in_class[kRcClasses];
   int tile_start[kRcClasses + 1];  // first 128-row tile of each class; [a_classes] = m_tiles
   int m_tiles, n_tiles, num_tiles, group_m;
   int bn;                  // tile width: 256, or N rounded up to 16 when N <= 240
   int panels;              // 64-column panels of the B tile: ceil(bn / 64)
-  int halves;              // staging: column halves of the B tile (2 when bn > 240)
-  int hw;                  // staging: columns per half
-  int bw;                  // staging: box width, hw + 8
+  int stg_blocks;          // staging: 16-byte blocks per B row piece, bn / 8 + 1
   int ring_stages, stg_slots;
   int ring_stage_bytes;    // 16 KiB of A + panels x 8 KiB of B
-  int stg_bytes;           // halves x 64 x bw x 2
+  int stg_bytes;           // 64 x stg_blocks x 16
   int splits;              // CTAs per cluster along K (split mode)
   int c_stride;            // split mode: bytes per row of the fp32 partial (bn * 4 + 16)
   uint32_t idesc;
@@ -180,6 +178,33 @@ __device__ __forceinline__ void st_shared_u4(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only); both addresses
+// 16-byte aligned.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed;
+// the arrival counts toward the barrier's expected count.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier among `threads` threads (whole warps) on barrier `id`, returning
+// whether `v` holds for all of them.
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t threads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
 // One output tile: class s, rows q0 .. q0 + 127 of the class, columns
 // n0 .. n0 + bn - 1, and this CTA's k-blocks [kb_lo, kb_hi) of the class's
 // ceil((K + e) / 64).
@@ -221,9 +246,8 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
   uint64_t* full_bar = bars;                       // [ring] TMA bytes landed
   uint64_t* empty_bar = bars + Cfg::MAX_RING;      // [ring] MMAs done with the slot
   uint64_t* bfull_bar = bars + 2 * Cfg::MAX_RING;  // [ring] realigned B written (staging mode)
-  uint64_t* stg_full = bars + 3 * Cfg::MAX_RING;   // [stg]
-  uint64_t* stg_empty = stg_full + Cfg::MAX_STG;   // [stg]
-  uint64_t* acc_full = stg_empty + Cfg::MAX_STG;   // [2]
+  uint64_t* stg_full = bars + 3 * Cfg::MAX_RING;   // [stg] a staging slot's copies landed
+  uint64_t* acc_full = stg_full + Cfg::MAX_STG;    // [2]
   uint64_t* acc_empty = acc_full + 2;              // [2]
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -243,10 +267,7 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       mbar_init(&empty_bar[s], 1);
       mbar_init(&bfull_bar[s], Cfg::REAL_WARPS > 0 ? Cfg::REAL_WARPS : 1);
     }
-    for (int s = 0; s < p.stg_slots; ++s) {
-      mbar_init(&stg_full[s], 1);
-      mbar_init(&stg_empty[s], Cfg::REAL_WARPS);
-    }
+    for (int s = 0; s < p.stg_slots; ++s) mbar_init(&stg_full[s], Cfg::REAL_WARPS * 32);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], Cfg::EPI_WARPS);
@@ -268,17 +289,14 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------
-    // Producer: A's class boxes into the ring; B into the ring (direct) or
-    // its class boxes into the staging buffers.
+    // Producer: A's class boxes into the ring, and B's boxes too in direct
+    // mode (in staging mode the realigning warps fetch B).
     // ------------------------------------------------------------------
     if (lane == 0) {
-      int r = 0, q = 0;
-      uint32_t rph = 0, qph = 0;
-      int last_full[Cfg::MAX_RING], last_stg[Cfg::MAX_STG];
+      int r = 0;
+      uint32_t rph = 0;
+      int last_full[Cfg::MAX_RING];
       for (int i = 0; i < Cfg::MAX_RING; ++i) last_full[i] = -1;
-      for (int i = 0; i < Cfg::MAX_STG; ++i) last_stg[i] = -1;
-      const int cb = p.b_classes;
-      const int box_rows = 64 / cb;
       bool ok = true;
       for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
         const RcTile T = rc_tile(p, t, rank, splits);
@@ -293,29 +311,7 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
           tma_load_2d(slot, &maps.a[T.s], &full_bar[r], kb * 64, T.q0);
           if (!STAGE_B) {
             for (int c = 0; c < p.panels; ++c)
-              tma_load_2d(slot + Cfg::A_BYTES + c * Cfg::PANEL_BYTES, &maps.b[0], &full_bar[r], T.n0 + 64 * c, k_lo);
-          } else {
-            if (!mbar_wait(&stg_empty[q], qph ^ 1u, abort_flag, p.wait_budget_ns, 0x62)) {
-              ok = false;
-              last_full[r] = static_cast<int>(rph);  // A's box is in flight
-              break;
-            }
-            mbar_arrive_expect_tx(&stg_full[q], static_cast<uint32_t>(p.stg_bytes));
-            uint8_t* sbuf = stg + q * p.stg_bytes;
-            for (int h = 0; h < p.halves; ++h) {
-              for (int tc = 0; tc < cb; ++tc) {
-                // First k-row of class tc at or after k_lo, and its row in the class map.
-                const int kt = k_lo + (((tc - k_lo) % cb) + cb) % cb;
-                const int y = (kt - tc) / cb;
-                tma_load_2d(sbuf + (h * 64 + tc * box_rows) * p.bw * 2, &maps.b[tc], &stg_full[q],
-                            T.n0 + h * p.hw, y);
-              }
-            }
-            last_stg[q] = static_cast<int>(qph);
-            if (++q == p.stg_slots) {
-              q = 0;
-              qph ^= 1u;
-            }
+              tma_load_2d(slot + Cfg::A_BYTES + c * Cfg::PANEL_BYTES, &maps.b, &full_bar[r], T.n0 + 64 * c, k_lo);
           }
           last_full[r] = static_cast<int>(rph);
           if (++r == p.ring_stages) {
@@ -326,8 +322,6 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       }
       // Every load issued has landed before the CTA may exit.
       volatile int no_abort = 0;
-      for (int i = 0; i < p.stg_slots; ++i)
-        if (last_stg[i] >= 0) mbar_wait(&stg_full[i], static_cast<uint32_t>(last_stg[i]), &no_abort, p.wait_budget_ns, 0x63);
       for (int i = 0; i < p.ring_stages; ++i)
         if (last_full[i] >= 0)
           mbar_wait(&full_bar[i], static_cast<uint32_t>(last_full[i]), &no_abort, p.wait_budget_ns, 0x64);
@@ -476,75 +470,122 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
     }
   } else if (STAGE_B) {
     // ------------------------------------------------------------------
-    // Realigning warps: staged class rows of B -> swizzled MN-major tile.
-    // Unit U = (lambda, d, seg): k-row j = 8 lambda + ((lambda + d) & 7)
-    // and its 64-column segment seg.  The 8 lanes of each shared-memory
-    // phase differ in lambda, so their reads hit 8 different 16-byte bank
-    // groups (staging rows are an odd number of 16-byte units long) and
-    // their swizzled writes too (j & 7 differs).
+    // Realigning warps.  Per k-block, once the current k-block's rows have
+    // landed, fetch B's rows for the k-block (stg_slots - 1) ahead: each warp copies whole row pieces, the 16-byte
+    // aligned blocks that cover B[k][n0 .. n0 + bn), lane l taking blocks l
+    // and l + 32, so one instruction moves whole cache lines; rows outside
+    // [0, K) and blocks that start past a row's end are not fetched.  Then
+    // shift the current k-block's rows into the swizzled MN-major tile.  A
+    // block that ends past a row's end reads at most 14 bytes beyond it, in
+    // the same 16-byte block (so never another page); those values only
+    // reach output columns past N, which are not stored.
+    // Unit U = (lambda, d, seg): k-row j = 8 lambda + ((lambda + d) & 7),
+    // 64-column segment seg; the 8 lanes of a shared-memory phase differ in
+    // lambda, so their reads (staging rows are an odd number of 16-byte
+    // blocks) and their swizzled writes (j & 7 differs) hit 8 different
+    // bank groups.  Rows outside [0, K) are written as zeros.
     // ------------------------------------------------------------------
     const int tid = threadIdx.x - Cfg::REAL_WARP0 * 32;
-    const int segs_per_half = (p.hw + 63) / 64;
+    const int rwarp = tid >> 5;
     const int units = 64 * p.panels;
-    int r = 0, q = 0;
-    uint32_t rph = 0, qph = 0;
+    const int S = p.stg_slots;
+    const uint32_t pitch = static_cast<uint32_t>(p.stg_blocks * 16);
+    // Load cursor: the (tile, k-block) whose rows are fetched next.
+    int lt = t_first, lkb = 0, lcount = 0;
+    RcTile LT;
+    bool lmore = lt < p.num_tiles;
+    if (lmore) {
+      LT = rc_tile(p, lt, rank, splits);
+      lkb = LT.kb_lo;
+    }
+    auto fetch = [&]() {
+      // Advance past tiles without k-blocks, then fetch one k-block.
+      while (lmore && lkb >= LT.kb_hi) {
+        lt += t_step;
+        lmore = lt < p.num_tiles;
+        if (lmore) {
+          LT = rc_tile(p, lt, rank, splits);
+          lkb = LT.kb_lo;
+        }
+      }
+      if (!lmore) return;
+      const int slot = lcount % S;
+      const uint32_t sbase = smem_u32(stg + slot * p.stg_bytes);
+      const int k_lo = lkb * 64 - LT.e;
+      const uintptr_t bbytes = reinterpret_cast<uintptr_t>(p.B);
+      for (int j = rwarp; j < 64; j += Cfg::REAL_WARPS) {
+        const int k = k_lo + j;
+        if (k < 0 || k >= p.K) continue;
+        const uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k) * p.ldb);
+        const uintptr_t row_end = row + 2u * static_cast<uintptr_t>(p.N);
+        const uintptr_t a0 = (row + 2u * static_cast<uintptr_t>(LT.n0)) & ~uintptr_t(15);
+        for (int b = lane; b < p.stg_blocks; b += 32) {
+          const uintptr_t g = a0 + 16u * static_cast<uintptr_t>(b);
+          if (g < row_end) cp_async_16(sbase + j * pitch + b * 16, reinterpret_cast<const void*>(g));
+        }
+      }
+      cp_async_mbar_arrive(&stg_full[slot]);
+      ++lkb;
+      ++lcount;
+    };
+    for (int i = 0; i < S - 1; ++i) fetch();
+    int r = 0, cnt = 0;
+    uint32_t rph = 0;
     bool ok = true;
     for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
       const RcTile T = rc_tile(p, t, rank, splits);
-      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
-        bool got = mbar_wait(&stg_full[q], qph, abort_flag, p.wait_budget_ns, 0x6A);
+      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb, ++cnt) {
+        const int q = cnt % S;
+        bool got = mbar_wait(&stg_full[q], static_cast<uint32_t>((cnt / S) & 1), abort_flag, p.wait_budget_ns, 0x6A);
         got = got && mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
-        if (!__all_sync(0xffffffffu, got)) {
+        // One decision for all realigning warps; passing it also means every
+        // one of them is done with the previous k-block's slot, which the
+        // fetch below refills.
+        if (!named_barrier_and(1, Cfg::REAL_WARPS * 32, got)) {
           ok = false;
           break;
         }
+        fetch();
         const int k_lo = kb * 64 - T.e;
         const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
         const uint32_t bbase = smem_u32(ring + r * p.ring_stage_bytes) + Cfg::A_BYTES;
         for (int U = tid; U < units; U += Cfg::REAL_WARPS * 32) {
           const int lam = U & 7, d = (U >> 3) & 7, seg = U >> 6;
           const int j = 8 * lam + ((lam + d) & 7);
-          int srow, f;
-          if (p.b_classes == 8) {
-            const int tc = (j + k_lo) & 7;
-            srow = 8 * tc + (j >> 3);
-            f = p.b_shift[tc];
-          } else {
-            srow = j;
-            f = p.b_shift[0];
+          const int k = k_lo + j;
+          const int nch = min(8, (p.bn - 64 * seg) >> 3);
+          const uint32_t dst = bbase + static_cast<uint32_t>(seg * Cfg::PANEL_BYTES + j * 128);
+          if (k < 0 || k >= p.K) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), make_uint4(0u, 0u, 0u, 0u));
+            continue;
           }
-          const int h = seg / segs_per_half;
-          const int cih = 64 * (seg - h * segs_per_half);
-          const int nch = min(8, (p.hw - cih) >> 3);
-          const uint32_t src = sbase + static_cast<uint32_t>(((h * 64 + srow) * p.bw + cih) * 2);
+          // This row piece starts f elements past its first aligned block.
+          const uint32_t f = static_cast<uint32_t>(
+              ((reinterpret_cast<uintptr_t>(p.B) + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k) * p.ldb + T.n0)) >> 1) & 7u);
+          const uint32_t src = sbase + j * pitch + seg * 128;
           uint4 blk[9];
 #pragma unroll
           for (int c = 0; c < 9; ++c) {
             blk[c] = make_uint4(0u, 0u, 0u, 0u);
             if (c <= nch) ld_shared_v4(src + c * 16, blk[c]);
           }
-          const uint32_t dst = bbase + static_cast<uint32_t>(seg * Cfg::PANEL_BYTES + j * 128);
-          const uint32_t sh = 2u * static_cast<uint32_t>(f);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), edge_realign(blk[c], blk[c + 1], sh));
+            if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), edge_realign(blk[c], blk[c + 1], 2u * f));
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bfull_bar[r]);
-          mbar_arrive(&stg_empty[q]);
-        }
+        if (lane == 0) mbar_arrive(&bfull_bar[r]);
         if (++r == p.ring_stages) {
           r = 0;
           rph ^= 1u;
         }
-        if (++q == p.stg_slots) {
-          q = 0;
-          qph ^= 1u;
-        }
       }
     }
+    // Every copy issued has landed before the CTA may exit.
+    asm volatile("cp.async.wait_all;" ::: "memory");
   }
 
   if (SPLIT) {

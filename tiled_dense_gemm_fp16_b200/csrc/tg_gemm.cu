@@ -187,6 +187,28 @@ bool tma_ok_b(const Problem& p) {
 }
 bool tma_ok(const Problem& p) { return tma_ok_a(p) && tma_ok_b(p); }
 
+// The residue-class kernel reads A stored M x K and B stored K x N.
+bool rc_ok(const Problem& p) { return !p.a_km && !p.b_nk; }
+
+// Operands TMA cannot describe, with a workspace: the residue-class kernel
+// (on a padded copy of B when B needs one) or the repack path (padded copies
+// of A, B and C around the faster CTA-pair kernel).  The repack path moves
+// about 2 (MK + MN) more bytes twice; its kernel saves about a fifth of the
+// main loop's time on 2 MNK flops.  With copies at about 5 TB/s and the loop
+// at about 1.2 PFLOP/s, the residue-class kernel wins when
+// 1/N + 1/K > 1/2400 (measured at (3001, 5003, 1021) and (8191, 129, 8193),
+// and the other way at (777, 12289, 4095)).
+bool rc_preferred(const Problem& p) {
+  return rc_ok(p) && 2400.0 * static_cast<double>(p.N + p.K) > static_cast<double>(p.N) * static_cast<double>(p.K);
+}
+
+// Bytes of the padded copy of B (rows rounded up to 8 elements) that the
+// residue-class kernel reads when TMA cannot describe B, else 0.
+int64_t rc_b_copy_bytes(const Problem& p) {
+  if (p.K <= 0 || p.N <= 0 || tma_ok_b(p)) return 0;
+  return (2 * p.K * ((p.N + 7) / 8 * 8) + 255) / 256 * 256;
+}
+
 // Every row of C, in every batch entry, starts on a 16-byte boundary.
 bool c_rows_aligned(const Problem& p) {
   return (reinterpret_cast<uintptr_t>(p.C) & 15u) == 0 && p.ldc % 8 == 0 && (p.batch == 1 || p.sc % 8 == 0);
@@ -233,10 +255,11 @@ RepackPlan repack_plan(const Problem& p, bool with_c) {
 // describe them) and for its fastest path (plus the padded C).
 int64_t repack_bytes_needed(const Problem& p) {
   if (p.M == 0 || p.N == 0 || p.K == 0 || tma_ok(p)) return 0;
-  return repack_plan(p, false).bytes;
+  return rc_preferred(p) ? rc_b_copy_bytes(p) : repack_plan(p, false).bytes;
 }
 int64_t workspace_bytes_needed(const Problem& p) {
   if (p.M == 0 || p.N == 0 || p.K == 0) return 0;
+  if (!tma_ok(p) && rc_preferred(p)) return rc_b_copy_bytes(p);
   return repack_plan(p, true).bytes;
 }
 
@@ -246,11 +269,6 @@ RepackPlan chosen_plan(const Problem& p, int64_t ws_bytes) {
   const RepackPlan full = repack_plan(p, true);
   return ws_bytes >= full.bytes ? full : repack_plan(p, false);
 }
-
-// The residue-class kernel reads A stored M x K and B stored K x N; when it
-// realigns B's rows in shared memory, each of B's eight row classes needs a
-// row (K >= 8).
-bool rc_ok(const Problem& p) { return !p.a_km && !p.b_nk && (tma_ok_b(p) || p.K >= 8); }
 
 bool path_supports(int path, const Problem& p) {
   if (!problem_valid(p)) return false;
@@ -312,6 +330,8 @@ int select_path(const Problem& p, int64_t ws_bytes) {
   if (p.M == 0 || p.N == 0) return TG_PATH_NONE;
   if (p.K == 0) return TG_PATH_ZERO;
   if (!tma_ok(p)) {
+    // rc_preferred: with a workspace holding B's copy, run() pads B first.
+    if (rc_preferred(p)) return TG_PATH_RC;
     if (ws_bytes >= repack_plan(p, false).bytes || p.b_nk || p.a_km) return TG_PATH_REPACK;
     return rc_ok(p) ? TG_PATH_RC : TG_PATH_TC_EDGE;
   }
@@ -709,7 +729,8 @@ tg_status launch_rc_cfg(const RcMaps& maps, const RcParams& p, int smem, int gri
   return TG_OK;
 }
 
-// Residue-class path: see gemm_rc.cuh.
+// Residue-class path: see gemm_rc.cuh.  B's rows are realigned in shared
+// memory (staging mode) when TMA cannot describe B.
 tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   const int64_t M = o.M, N = o.N, K = o.K;
   RcMaps maps;
@@ -745,20 +766,14 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   p.group_m = tune_int("TG_TUNE_RC_GROUP_M", 8);
   if (p.group_m < 1) p.group_m = 1;
   const bool stage_b = !((reinterpret_cast<uintptr_t>(o.B) & 15u) == 0 && o.ldb % 8 == 0);
+  p.B = static_cast<const __half*>(o.B);
+  p.ldb = o.ldb;
   if (stage_b) {
-    if (K < kRcClasses) return TG_ERR_INVALID_ARG;
-    const int f0 = static_cast<int>((reinterpret_cast<uintptr_t>(o.B) & 15u) / 2);
-    p.b_classes = (o.ldb % 8 == 0 && o.ldb >= N + f0) ? 1 : kRcClasses;
-    p.halves = p.bn > 240 ? 2 : 1;
-    p.hw = p.bn / p.halves;
-    p.bw = p.hw + 8;
-    int b_rows[kRcClasses];
-    if (!encode_classes(maps.b, o.B, K, N, o.ldb, p.b_classes, p.bw, 64 / p.b_classes, CU_TENSOR_MAP_SWIZZLE_NONE,
-                        p.b_shift, b_rows))
-      return TG_ERR_LAUNCH;
-    p.stg_bytes = p.halves * 64 * p.bw * 2;
-    p.stg_slots = 2;
-  } else if (!encode_2d(&maps.b[0], o.B, K, N, o.ldb, 64, 64)) {
+    p.stg_blocks = p.bn / 8 + 1;
+    p.stg_bytes = 64 * p.stg_blocks * 16;
+    p.stg_slots = tune_int("TG_TUNE_RC_STG", 3);
+    if (p.stg_slots < 2 || p.stg_slots > RcCfg<true>::MAX_STG) return TG_ERR_INVALID_ARG;
+  } else if (!encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
     return TG_ERR_LAUNCH;
   }
   p.ring_stage_bytes = RcCfg<false>::A_BYTES + p.panels * RcCfg<false>::PANEL_BYTES;
@@ -914,6 +929,18 @@ tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws
         ranges_overlap(ws, plan.bytes, p.C, span_c(p)) || (p.bias && ranges_overlap(ws, plan.bytes, p.bias, 2 * p.N)))
       return TG_ERR_INVALID_ARG;
   }
+  // The residue-class kernel reads a padded copy of B when the workspace holds one.
+  int64_t rc_b_bytes = 0;
+  if (path == TG_PATH_RC && ws != nullptr) {
+    const int64_t need = rc_b_copy_bytes(p);
+    if (need > 0 && ws_bytes >= need) {
+      if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ranges_overlap(ws, need, p.A, span_a(p)) ||
+          ranges_overlap(ws, need, p.B, span_b(p)) || ranges_overlap(ws, need, p.C, span_c(p)) ||
+          (p.bias && ranges_overlap(ws, need, p.bias, 2 * p.N)))
+        return TG_ERR_INVALID_ARG;
+      rc_b_bytes = need;
+    }
+  }
   int dev = 0;
   DeviceInfo* info = nullptr;
   tg_status st = current_device(dev, info);
@@ -936,6 +963,14 @@ tg_status run(const Problem& p, void* stream_ptr, int path, void* ws, int64_t ws
                c_rows_aligned(p)};
     if (path == TG_PATH_ZERO) {
       st = launch_k_zero(o, stream, info);
+    } else if (path == TG_PATH_RC && rc_b_bytes > 0) {
+      // B padded into the workspace, so TMA loads it as it is.
+      const int64_t np = (p.N + 7) / 8 * 8;
+      st = launch_pad(o.B, o.ldb, ws, p.K, p.N, np, stream, info);
+      if (st != TG_OK) return st;
+      o.B = ws;
+      o.ldb = np;
+      st = launch_path(path, o, stream, info);
     } else if (path == TG_PATH_REPACK) {
       uint8_t* base = static_cast<uint8_t*>(ws);
       if (plan.pad_a) {
@@ -1472,7 +1507,9 @@ tg_status tg_gemm_relu_f16_static_ws(const void* A, const void* B, void* C, int6
                                      void* stream) {
   const tg::Problem p = tg::dense_problem(A, B, C, M, N, K);
   if (!tg::problem_valid(p)) return TG_ERR_INVALID_ARG;
-  // Only the copies of A and B are required; a padded C is used when it fits too.
+  // Only the copies of the operands are required (B's alone on the
+  // residue-class route; A's and B's on the repack route, with a padded C
+  // when it fits too).
   const int64_t need = tg::repack_bytes_needed(p);
   if (need > TG_STATIC_WORKSPACE_BYTES) return TG_ERR_TOO_LARGE;
   if (M == 0 || N == 0) return TG_OK;  // empty C: nothing to do
