@@ -54,6 +54,10 @@ KERNEL_SOURCES = {
     "mxf8": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
     "nvf4": [_CSRC + "gemm_mx.cuh", _CSRC + "ptx.cuh"],
     "w4a16": [_CSRC + "gemm_w4a16.cuh", _CSRC + "ptx.cuh"],
+    "rc": [_CSRC + "gemm_rc.cuh", _CSRC + "gemm_tc.cuh", _CSRC + "ptx.cuh"],
+    "rc_ws": [_CSRC + "gemm_rc.cuh", _CSRC + "gemm_tc.cuh", _CSRC + "repack.cuh", _CSRC + "ptx.cuh"],
+    "repack": [_CSRC + "repack.cuh", _CSRC + "gemm_tc.cuh", _CSRC + "gemm_tc_pair.cuh", _CSRC + "gemm_skinny.cuh",
+               _CSRC + "ptx.cuh"],
 }
 E2E_MODE = "every step uploads its inputs and downloads its result; two buffer sets overlap the copies with the GEMM"
 MX_METRIC = "MXFP8 block-scaled grouped GEMM TFLOP/s (1×B200) and % of dense FP8 tensor peak"
@@ -706,7 +710,8 @@ def measure_configs(tg, torch, dev, stream, args, peaks, peak_src):
         case = Fp16Case(tg, torch, dev, stream, M, N, K, A, B, mode=mode)
         case.warm(args.warmup)
         ms, clocks = case.time(args.steps)
-        rec = {"config": label, "workload": workload + (f":{idx}" if idx is not None else ""),
+        spec = f"skinny:{M}" if workload == "skinny" else workload + (f":{idx}" if idx is not None else "")
+        rec = {"config": label, "workload": spec,
                "M": M, "N": N, "K": K, "values": dist or inputs.WORKLOADS[workload].dist,
                "seed": inputs.WORKLOADS[workload].seed,
                "entry_point": "tg_gemm_relu_f16" if case.ws_bytes == 0 else "tg_gemm_relu_f16_ws",
@@ -715,7 +720,9 @@ def measure_configs(tg, torch, dev, stream, args, peaks, peak_src):
                "value": inputs.flops(M, N, K) / (ms * 1e-3) / 1e12, "unit": UNIT,
                "roofline": roofline_for(M, N, K, ms, peaks, peak_src),
                "gpu_launches": args.steps * case.launches_per_step, "clocks": clocks}
-        rec["roofline"]["traffic"] = committed_traffic(tg.path_name(case.chosen), label)
+        # A profile is keyed by path, and by "_ws" when a workspace changes what the path runs.
+        key = tg.path_name(case.chosen) + ("_ws" if case.ws_bytes > 0 and case.chosen == tg.Path.RC else "")
+        rec["roofline"]["traffic"] = committed_traffic(key, spec)
         if not args.no_cpu_baseline:
             rec["cpu_baseline"] = cpu_baseline(A, B, args.config_cpu_seconds)
         case.release()
@@ -817,7 +824,13 @@ def run_ours(args):
     if gather is not None:
         line["gather"] = gather
     if rank == 0 and world == 1 and args.sustained_seconds > 0:
-        line["sustained"] = sustained_record(case, args.sustained_seconds, peaks, peak_src)
+        sus = sustained_record(case, args.sustained_seconds, peaks, peak_src)
+        line["sustained"] = sus
+        if sus.get("ms_x_sm_mhz"):
+            # The kernel is clock-bound (tensor pipe), so time x clock is about constant: the
+            # sustained run's product over the headline's time estimates the clock the headline
+            # steps actually ran at, which NVML's sampled clock need not show for a short burst.
+            line["clocks"]["effective_sm_mhz_estimate"] = sus["ms_x_sm_mhz"] / step_ms
     if args.cublas and not linear:
         # Context only (a library GEMM, not this path): the same operand sets, events around the region.
         def cublas_step():

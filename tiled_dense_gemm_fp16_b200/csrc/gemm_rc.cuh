@@ -96,7 +96,8 @@ struct RcCfg {
   static constexpr int EPI_WARPS = 4;
   static constexpr int REAL_WARP0 = EPI_WARP0 + EPI_WARPS;
   static constexpr int REAL_WARPS = STAGE_B ? 4 : 0;
-  static constexpr int THREADS = (REAL_WARP0 + REAL_WARPS) * 32;
+  static constexpr int FETCH_WARP = REAL_WARP0 + REAL_WARPS;  // staging mode: copies B's rows
+  static constexpr int THREADS = (REAL_WARP0 + REAL_WARPS + (STAGE_B ? 1 : 0)) * 32;
   static constexpr int MAX_RING = 8;
   static constexpr int MAX_STG = 4;
   static constexpr int BAR_BYTES = 512;
@@ -190,21 +191,6 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Barrier among `threads` threads (whole warps) on barrier `id`, returning
-// whether `v` holds for all of them.
-__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t threads, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(threads)
-      : "memory");
-  return r != 0;
-}
-
 // One output tile: class s, rows q0 .. q0 + 127 of the class, columns
 // n0 .. n0 + bn - 1, and this CTA's k-blocks [kb_lo, kb_hi) of the class's
 // ceil((K + e) / 64).
@@ -247,7 +233,8 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
   uint64_t* empty_bar = bars + Cfg::MAX_RING;      // [ring] MMAs done with the slot
   uint64_t* bfull_bar = bars + 2 * Cfg::MAX_RING;  // [ring] realigned B written (staging mode)
   uint64_t* stg_full = bars + 3 * Cfg::MAX_RING;   // [stg] a staging slot's copies landed
-  uint64_t* acc_full = stg_full + Cfg::MAX_STG;    // [2]
+  uint64_t* stg_empty = stg_full + Cfg::MAX_STG;   // [stg] a staging slot's rows realigned
+  uint64_t* acc_full = stg_empty + Cfg::MAX_STG;   // [2]
   uint64_t* acc_empty = acc_full + 2;              // [2]
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -267,7 +254,10 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       mbar_init(&empty_bar[s], 1);
       mbar_init(&bfull_bar[s], Cfg::REAL_WARPS > 0 ? Cfg::REAL_WARPS : 1);
     }
-    for (int s = 0; s < p.stg_slots; ++s) mbar_init(&stg_full[s], Cfg::REAL_WARPS * 32);
+    for (int s = 0; s < p.stg_slots; ++s) {
+      mbar_init(&stg_full[s], 32);  // the fetch warp's lanes, as their copies land
+      mbar_init(&stg_empty[s], Cfg::REAL_WARPS);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], Cfg::EPI_WARPS);
@@ -468,84 +458,33 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       }
       tcgen05_fence_before_sync();
     }
-  } else if (STAGE_B) {
+  } else if (STAGE_B && warp < Cfg::FETCH_WARP) {
     // ------------------------------------------------------------------
-    // Realigning warps.  Per k-block, once the current k-block's rows have
-    // landed, fetch B's rows for the k-block (stg_slots - 1) ahead: each warp copies whole row pieces, the 16-byte
-    // aligned blocks that cover B[k][n0 .. n0 + bn), lane l taking blocks l
-    // and l + 32, so one instruction moves whole cache lines; rows outside
-    // [0, K) and blocks that start past a row's end are not fetched.  Then
-    // shift the current k-block's rows into the swizzled MN-major tile.  A
-    // block that ends past a row's end reads at most 14 bytes beyond it, in
-    // the same 16-byte block (so never another page); those values only
-    // reach output columns past N, which are not stored.
-    // Unit U = (lambda, d, seg): k-row j = 8 lambda + ((lambda + d) & 7),
-    // 64-column segment seg; the 8 lanes of a shared-memory phase differ in
-    // lambda, so their reads (staging rows are an odd number of 16-byte
-    // blocks) and their swizzled writes (j & 7 differs) hit 8 different
-    // bank groups.  Rows outside [0, K) are written as zeros.
+    // Realigning warps: shift each staged row of B into the swizzled
+    // MN-major operand tile.  Unit U = (lambda, d, seg): k-row
+    // j = 8 lambda + ((lambda + d) & 7), 64-column segment seg; the 8 lanes
+    // of a shared-memory phase differ in lambda, so their reads (staging
+    // rows are an odd number of 16-byte blocks long) and their swizzled
+    // writes (j & 7 differs) hit 8 different bank groups.  Rows outside
+    // [0, K) are written as zeros.  These warps issue no asynchronous
+    // copies of their own, so their proxy fence has nothing in flight to
+    // wait for.
     // ------------------------------------------------------------------
     const int tid = threadIdx.x - Cfg::REAL_WARP0 * 32;
-    const int rwarp = tid >> 5;
     const int units = 64 * p.panels;
-    const int S = p.stg_slots;
     const uint32_t pitch = static_cast<uint32_t>(p.stg_blocks * 16);
-    // Load cursor: the (tile, k-block) whose rows are fetched next.
-    int lt = t_first, lkb = 0, lcount = 0;
-    RcTile LT;
-    bool lmore = lt < p.num_tiles;
-    if (lmore) {
-      LT = rc_tile(p, lt, rank, splits);
-      lkb = LT.kb_lo;
-    }
-    auto fetch = [&]() {
-      // Advance past tiles without k-blocks, then fetch one k-block.
-      while (lmore && lkb >= LT.kb_hi) {
-        lt += t_step;
-        lmore = lt < p.num_tiles;
-        if (lmore) {
-          LT = rc_tile(p, lt, rank, splits);
-          lkb = LT.kb_lo;
-        }
-      }
-      if (!lmore) return;
-      const int slot = lcount % S;
-      const uint32_t sbase = smem_u32(stg + slot * p.stg_bytes);
-      const int k_lo = lkb * 64 - LT.e;
-      const uintptr_t bbytes = reinterpret_cast<uintptr_t>(p.B);
-      for (int j = rwarp; j < 64; j += Cfg::REAL_WARPS) {
-        const int k = k_lo + j;
-        if (k < 0 || k >= p.K) continue;
-        const uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k) * p.ldb);
-        const uintptr_t row_end = row + 2u * static_cast<uintptr_t>(p.N);
-        const uintptr_t a0 = (row + 2u * static_cast<uintptr_t>(LT.n0)) & ~uintptr_t(15);
-        for (int b = lane; b < p.stg_blocks; b += 32) {
-          const uintptr_t g = a0 + 16u * static_cast<uintptr_t>(b);
-          if (g < row_end) cp_async_16(sbase + j * pitch + b * 16, reinterpret_cast<const void*>(g));
-        }
-      }
-      cp_async_mbar_arrive(&stg_full[slot]);
-      ++lkb;
-      ++lcount;
-    };
-    for (int i = 0; i < S - 1; ++i) fetch();
-    int r = 0, cnt = 0;
-    uint32_t rph = 0;
+    int r = 0, q = 0;
+    uint32_t rph = 0, qph = 0;
     bool ok = true;
     for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
       const RcTile T = rc_tile(p, t, rank, splits);
-      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb, ++cnt) {
-        const int q = cnt % S;
-        bool got = mbar_wait(&stg_full[q], static_cast<uint32_t>((cnt / S) & 1), abort_flag, p.wait_budget_ns, 0x6A);
+      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
+        bool got = mbar_wait(&stg_full[q], qph, abort_flag, p.wait_budget_ns, 0x6A);
         got = got && mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
-        // One decision for all realigning warps; passing it also means every
-        // one of them is done with the previous k-block's slot, which the
-        // fetch below refills.
-        if (!named_barrier_and(1, Cfg::REAL_WARPS * 32, got)) {
+        if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
-        fetch();
         const int k_lo = kb * 64 - T.e;
         const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
         const uint32_t bbase = smem_u32(ring + r * p.ring_stage_bytes) + Cfg::A_BYTES;
@@ -577,10 +516,65 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bfull_bar[r]);
+        if (lane == 0) {
+          mbar_arrive(&bfull_bar[r]);
+          mbar_arrive(&stg_empty[q]);
+        }
         if (++r == p.ring_stages) {
           r = 0;
           rph ^= 1u;
+        }
+        if (++q == p.stg_slots) {
+          q = 0;
+          qph ^= 1u;
+        }
+      }
+    }
+  } else if (STAGE_B) {
+    // ------------------------------------------------------------------
+    // Fetch warp: for each k-block, once its staging slot is free, copy the
+    // 16-byte aligned blocks that cover B[k][n0 .. n0 + bn) of each of the
+    // 64 k-rows (lane l takes blocks l and l + 32, so each instruction moves
+    // whole cache lines); rows outside [0, K) and blocks that start past a
+    // row's end are not fetched.  A block that ends past a row's end reads
+    // at most 14 bytes beyond it, in the same 16-byte block (so never
+    // another page); those values only reach output columns past N, which
+    // are not stored.  The slot's barrier completes as the copies land.
+    // ------------------------------------------------------------------
+    const uint32_t pitch = static_cast<uint32_t>(p.stg_blocks * 16);
+    const uintptr_t bbytes = reinterpret_cast<uintptr_t>(p.B);
+    int q = 0;
+    uint32_t qph = 0;
+    bool ok = true;
+    for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
+      const RcTile T = rc_tile(p, t, rank, splits);
+      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
+        const bool free_slot = mbar_wait(&stg_empty[q], qph ^ 1u, abort_flag, p.wait_budget_ns, 0x6D);
+        if (!__all_sync(0xffffffffu, free_slot)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
+        const int k_lo = kb * 64 - T.e;
+        const int j_lo = k_lo < 0 ? -k_lo : 0;              // rows inside [0, K)
+        const int j_hi = min(64, p.K - k_lo);
+        const uintptr_t row_step = 2u * static_cast<uintptr_t>(p.ldb);
+        uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k_lo + j_lo) * p.ldb);
+        const uintptr_t n0_bytes = 2u * static_cast<uintptr_t>(T.n0), n_bytes = 2u * static_cast<uintptr_t>(p.N);
+        const uintptr_t off0 = 16u * static_cast<uintptr_t>(lane), off1 = off0 + 512u;
+        const bool second = lane + 32 < p.stg_blocks;
+#pragma unroll 4
+        for (int j = j_lo; j < j_hi; ++j, row += row_step) {
+          const uintptr_t a0 = (row + n0_bytes) & ~uintptr_t(15);
+          const uintptr_t row_end = row + n_bytes;
+          const uint32_t dst = sbase + j * pitch + lane * 16;
+          if (a0 + off0 < row_end) cp_async_16(dst, reinterpret_cast<const void*>(a0 + off0));
+          if (second && a0 + off1 < row_end) cp_async_16(dst + 512, reinterpret_cast<const void*>(a0 + off1));
+        }
+        cp_async_mbar_arrive(&stg_full[q]);
+        if (++q == p.stg_slots) {
+          q = 0;
+          qph ^= 1u;
         }
       }
     }
