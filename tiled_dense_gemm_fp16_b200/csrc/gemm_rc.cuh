@@ -79,6 +79,7 @@ struct RcParams {
   int ring_stages, stg_slots;
   int ring_stage_bytes;    // 16 KiB of A + panels x 8 KiB of B
   int stg_bytes;           // 64 x stg_blocks x 16
+  int bulk_fetch;          // staging: 1 = one bulk copy per row piece, 0 = 16-byte cp.async per block
   int splits;              // CTAs per cluster along K (split mode)
   int c_stride;            // split mode: bytes per row of the fp32 partial (bn * 4 + 16)
   uint32_t idesc;
@@ -255,7 +256,9 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       mbar_init(&bfull_bar[s], Cfg::REAL_WARPS > 0 ? Cfg::REAL_WARPS : 1);
     }
     for (int s = 0; s < p.stg_slots; ++s) {
-      mbar_init(&stg_full[s], 32);  // the fetch warp's lanes, as their copies land
+      // Bulk copies: one arrival with the slot's byte count; 16-byte copies:
+      // the fetch warp's 32 lanes, as their copies land.
+      mbar_init(&stg_full[s], p.bulk_fetch ? 1 : 32);
       mbar_init(&stg_empty[s], Cfg::REAL_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
@@ -545,6 +548,8 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
     const uintptr_t bbytes = reinterpret_cast<uintptr_t>(p.B);
     int q = 0;
     uint32_t qph = 0;
+    int last_fill[Cfg::MAX_STG];
+    for (int i = 0; i < Cfg::MAX_STG; ++i) last_fill[i] = -1;
     bool ok = true;
     for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
       const RcTile T = rc_tile(p, t, rank, splits);
@@ -556,6 +561,43 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
         }
         const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
         const int k_lo = kb * 64 - T.e;
+        if (p.bulk_fetch) {
+          // Lane l copies rows l and l + 32, each as one bulk copy of the
+          // 16-byte blocks from the one holding B[k][n0] to the one holding
+          // the piece's last element (or the row's, past N).
+          uint32_t bytes[2] = {0u, 0u};
+          uintptr_t src[2] = {0u, 0u};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = lane + 32 * h;
+            const int k = k_lo + j;
+            if (k >= 0 && k < p.K) {
+              const uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k) * p.ldb);
+              const uintptr_t a0 = (row + 2u * static_cast<uintptr_t>(T.n0)) & ~uintptr_t(15);
+              const uintptr_t end = (row + 2u * static_cast<uintptr_t>(p.N) + 15u) & ~uintptr_t(15);
+              const uintptr_t span = end - a0;
+              const uintptr_t cap = 16u * static_cast<uintptr_t>(p.stg_blocks);
+              bytes[h] = static_cast<uint32_t>(span < cap ? span : cap);
+              src[h] = a0;
+            }
+          }
+          uint32_t total = bytes[0] + bytes[1];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+          if (lane == 0) mbar_arrive_expect_tx(&stg_full[q], total);
+          __syncwarp();
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (bytes[h] > 0)
+              bulk_load_g2s(stg + q * p.stg_bytes + (lane + 32 * h) * pitch, reinterpret_cast<const void*>(src[h]),
+                            bytes[h], &stg_full[q]);
+          last_fill[q] = static_cast<int>(qph);
+          if (++q == p.stg_slots) {
+            q = 0;
+            qph ^= 1u;
+          }
+          continue;
+        }
         const int j_lo = k_lo < 0 ? -k_lo : 0;              // rows inside [0, K)
         const int j_hi = min(64, p.K - k_lo);
         const uintptr_t row_step = 2u * static_cast<uintptr_t>(p.ldb);
@@ -580,6 +622,12 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
     }
     // Every copy issued has landed before the CTA may exit.
     asm volatile("cp.async.wait_all;" ::: "memory");
+    if (p.bulk_fetch && lane == 0) {
+      // The bulk copies of each slot's last fill have landed.
+      volatile int no_abort = 0;
+      for (int i = 0; i < p.stg_slots; ++i)
+        if (last_fill[i] >= 0) mbar_wait(&stg_full[i], static_cast<uint32_t>(last_fill[i]), &no_abort, p.wait_budget_ns, 0x6E);
+    }
   }
 
   if (SPLIT) {
