@@ -370,35 +370,3 @@ def test_more_than_2_31_elements(K):
     assert_bitexact(ones_row, ref_ones, "all-ones row")
     del Ad, Bd, C
     torch.cuda.empty_cache()
-
-
-# ---------------------------------------------------------------------------
-# 256 x 512 pair tiles with a quarter-tile tail: the last, partial wave of
-# tiles runs as 256 x 128 quarters spread over every SM pair
-# ---------------------------------------------------------------------------
-
-@pytest.mark.parametrize("M,N,K", [(2304, 4608, 256), (4096, 4096, 512), (2560, 4100, 200), (2304, 4616, 72)])
-def test_pair512_quarter_tail_integer_bitexact(M, N, K):
-    """Tile counts 81, 128, 90 and 90 on 74 pairs: 7, 54, 16 and 16 tail tiles become quarters (N past
-    the last whole 512 columns included)."""
-    A, B = inputs.operands(M, N, K, "int", seed=M + N + K)
-    got, guards = run_gpu(A, B, WIDE)
-    assert guards
-    assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"pair512 quarter tail {(M, N, K)}")
-
-
-@pytest.mark.parametrize("c_off", [0, 3])
-def test_pair512_quarter_tail_unaligned_c_and_floats(c_off):
-    M, N, K = 2304, 4608, 136
-    A, B = inputs.operands(M, N, K, "uniform", seed=9 + c_off)
-    got, guards = run_gpu(A, B, WIDE, offsets=(0, 0, c_off))
-    assert guards
-    assert_close(got, oracle.gemm_relu_f16(A, B), f"pair512 quarter tail, C offset {c_off}")
-
-
-def test_pair512_quarter_tail_weight_layout_and_bias():
-    from test_gpu_layouts import run_ex
-    M, N, K = 2304, 4608, 264
-    got, ref, guards = run_ex(M, N, K, lda=K, ldb=K, ldc=N, b_nk=True, bias=True, path=WIDE, seed=31)
-    assert guards
-    assert_bitexact(got[0], ref[0], "pair512 quarter tail, N x K weight, bias")

@@ -48,9 +48,6 @@ struct TcParams {
   int l2_hints;          // bit 0: A loads evict-last; bit 1: B loads evict-last; bit 2: B loads evict-first
   int prefetch_kb;       // > 0: also prefetch into L2 the boxes this many k-blocks ahead
   int c_aligned;         // 1: every row of C starts on a 16-byte boundary (C aligned, N % 8 == 0)
-  int full_tiles;        // pair kernel, BN = 512: tiles [0, full_tiles) are whole; each later index is a
-                         // quarter (256 x 128) of one of the last (num_tiles - full_tiles) / 4 tiles
-  uint32_t idesc_q;      // pair kernel: instruction descriptor of the 256 x 128 quarter MMA
   uint64_t wait_budget_ns;
 };
 

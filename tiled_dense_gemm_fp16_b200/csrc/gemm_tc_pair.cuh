@@ -91,22 +91,7 @@ __device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, const 
       : "memory");
 }
 
-// Work item t of the pair kernel: a whole tile (quarter = -1), or, past
-// full_tiles, quarter (t - full_tiles) % 4 of tile full_tiles + (t -
-// full_tiles) / 4, i.e. its columns [128 quarter, 128 quarter + 128).  The
-// quarters of the last, partial wave of tiles spread over every pair.
-__device__ __forceinline__ void pair_work(const TcParams& p, int t, int& m_blk, int& n_blk, int& quarter) {
-  if (t < p.full_tiles) {
-    tile_coords(p, t, m_blk, n_blk);
-    quarter = -1;
-    return;
-  }
-  const int qt = t - p.full_tiles;
-  tile_coords(p, p.full_tiles + (qt >> 2), m_blk, n_blk);
-  quarter = qt & 3;
-}
-
-template <int STAGES, int BN, bool QUARTERS>
+template <int STAGES, int BN>
 __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
     gemm_relu_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                              const __grid_constant__ CUtensorMap tmap_c, const TcParams p) {
@@ -178,26 +163,18 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
                              : (p.l2_hints & 4) ? l2_policy_evict_first()
                                                 : l2_policy_evict_normal();
       for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters) {
-        int m_blk, n_blk, quarter = -1;
-        if (QUARTERS)
-          pair_work(p, t, m_blk, n_blk, quarter);
-        else
-          tile_coords(p, t, m_blk, n_blk);
+        int m_blk, n_blk;
+        tile_coords(p, t, m_blk, n_blk);
         const int m0 = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM;
-        // This CTA's 128 columns of slab j start at n0 + 256 j + 128 r; of a
-        // quarter, its 64 columns start at n0 + 128 quarter + 64 r.
-        const int nb = quarter < 0 ? n_blk * Cfg::BN + static_cast<int>(rank) * 128
-                                   : n_blk * Cfg::BN + quarter * 128 + static_cast<int>(rank) * 64;
-        // A quarter's B box: 64 columns x 64 k (K x N), or the 128-row box of the N x K map.
-        const uint32_t tx = quarter < 0 ? 2 * (Cfg::A_BYTES + Cfg::B_BYTES)
-                                        : 2 * (Cfg::A_BYTES + (p.b_kmajor ? Cfg::B_SLAB_BYTES : Cfg::B_CHUNK_BYTES));
+        // This CTA's 128 columns of slab j start at n0 + 256 j + 128 r.
+        const int nb = n_blk * Cfg::BN + static_cast<int>(rank) * 128;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, p.wait_budget_ns, 0x41)) {
             ok = false;
             break;
           }
           const uint32_t full_even = mapa_shared(smem_u32(&full_bar[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
+          if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
           const int k0 = kb * Cfg::BK;
           uint8_t* bdst = b_smem + stage * Cfg::B_BYTES;
           if (p.a_mnmajor) {
@@ -208,25 +185,18 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           } else {
             tma_load_2d_pair_hint(a_smem + stage * Cfg::A_BYTES, &tmap_a, full_even, k0, m0, pol_a);
           }
-          if (quarter >= 0) {
-            if (p.b_kmajor)
-              tma_load_2d_pair_hint(bdst, &tmap_b, full_even, k0, nb, pol_b);
-            else
-              tma_load_2d_pair_hint(bdst, &tmap_b, full_even, nb, k0, pol_b);
-          } else {
 #pragma unroll
-            for (int j = 0; j < Cfg::SLABS; ++j) {
-              if (p.b_kmajor) {
-                // B stored N x K: this CTA's 128 n-rows x 64 k of slab j, K-major.
-                tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, k0, nb + 256 * j, pol_b);
-              } else {
-                tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, nb + 256 * j, k0, pol_b);
-                tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES + Cfg::B_CHUNK_BYTES, &tmap_b, full_even,
-                                      nb + 256 * j + 64, k0, pol_b);
-              }
+          for (int j = 0; j < Cfg::SLABS; ++j) {
+            if (p.b_kmajor) {
+              // B stored N x K: this CTA's 128 n-rows x 64 k of slab j, K-major.
+              tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, k0, nb + 256 * j, pol_b);
+            } else {
+              tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES, &tmap_b, full_even, nb + 256 * j, k0, pol_b);
+              tma_load_2d_pair_hint(bdst + j * Cfg::B_SLAB_BYTES + Cfg::B_CHUNK_BYTES, &tmap_b, full_even,
+                                    nb + 256 * j + 64, k0, pol_b);
             }
           }
-          if (quarter < 0 && p.prefetch_kb > 0 && kb + p.prefetch_kb < p.k_blocks) {
+          if (p.prefetch_kb > 0 && kb + p.prefetch_kb < p.k_blocks) {
             // Warm L2 with the boxes a few k-blocks ahead, so the ring's
             // loads find them there instead of waiting on HBM.
             const int kp = (kb + p.prefetch_kb) * Cfg::BK;
@@ -276,7 +246,6 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
       bool ok = true;
       const uint32_t idesc = make_idesc_f16_f32(Cfg::PAIR_M, 256, p.a_mnmajor != 0, p.b_kmajor == 0);
       for (int t = cluster_id; t < p.num_tiles && ok; t += num_clusters, ++local) {
-        const bool quarter = QUARTERS && t >= p.full_tiles;
         const int acc = local % Cfg::NUM_ACC;
         const uint32_t acc_phase = (local / Cfg::NUM_ACC) & 1;
         if (!mbar_wait(&acc_empty_bar[acc], acc_phase ^ 1u, abort_flag, p.wait_budget_ns, 0x43)) break;
@@ -294,21 +263,14 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           for (int k = 0; k < Cfg::BK / 16; ++k) {
             const uint64_t adesc = p.a_mnmajor ? make_sw128_desc(a_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024)
                                                : make_sw128_desc(a_addr + k * 32, 16, 1024);
-            if (quarter) {
-              // 256 x 128: this CTA's 64 columns (one panel, or 64 K-major rows).
-              const uint64_t bdesc = p.b_kmajor ? make_sw128_desc(b_addr + k * 32, 16, 1024)
-                                                : make_sw128_desc(b_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
-              umma_f16_ss_pair(d_tmem, adesc, bdesc, p.idesc_q, (kb | k) != 0 ? 1u : 0u);
-            } else {
 #pragma unroll
-              for (int j = 0; j < Cfg::SLABS; ++j) {
-                // Slab j: as K x N, this CTA's two 64-column panels, 8 KiB apart;
-                // as N x K, 128 K-major rows like A.
-                const uint32_t slab_addr = b_addr + j * Cfg::B_SLAB_BYTES;
-                const uint64_t bdesc = p.b_kmajor ? make_sw128_desc(slab_addr + k * 32, 16, 1024)
-                                                  : make_sw128_desc(slab_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
-                umma_f16_ss_pair(d_tmem + 256 * j, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
-              }
+            for (int j = 0; j < Cfg::SLABS; ++j) {
+              // Slab j: as K x N, this CTA's two 64-column panels, 8 KiB apart;
+              // as N x K, 128 K-major rows like A.
+              const uint32_t slab_addr = b_addr + j * Cfg::B_SLAB_BYTES;
+              const uint64_t bdesc = p.b_kmajor ? make_sw128_desc(slab_addr + k * 32, 16, 1024)
+                                                : make_sw128_desc(slab_addr + k * 2048, Cfg::B_CHUNK_BYTES, 1024);
+              umma_f16_ss_pair(d_tmem + 256 * j, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
             }
           }
           umma_commit_pair_mc(&empty_bar[stage], 0x3);  // both CTAs may refill this stage
@@ -335,11 +297,8 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
     const int col_base = ((warp - Cfg::EPI_WARP0) >> 2) * Cfg::EPI_COLS;
     int local = 0;
     for (int t = cluster_id; t < p.num_tiles; t += num_clusters, ++local) {
-      int m_blk, n_blk, quarter = -1;
-      if (QUARTERS)
-        pair_work(p, t, m_blk, n_blk, quarter);
-      else
-        tile_coords(p, t, m_blk, n_blk);
+      int m_blk, n_blk;
+      tile_coords(p, t, m_blk, n_blk);
       const int acc = local % Cfg::NUM_ACC;
       const uint32_t acc_phase = (local / Cfg::NUM_ACC) & 1;
       const bool ready = mbar_wait(&acc_full_bar[acc], acc_phase, abort_flag, p.wait_budget_ns, 0x46);
@@ -354,68 +313,8 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
         // registers as ReLU'd fp16 pairs, release the accumulator to the MMA
         // warp, and only then store, so the stores overlap the next tile's MMAs.
         uint32_t h[Cfg::EPI_COLS / 2];
-        if (QUARTERS && quarter >= 0) {
-          // A quarter tile: accumulator columns 0..127, written by the four
-          // warps of slab 0 (32 columns per TMEM round trip, then stores as
-          // below); the other four only release the accumulator.
-          const int n_base = n_blk * Cfg::BN + quarter * 128;  // first column of C of this quarter
-          if (col_base == 0) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(taddr + c * 32, r);
-              tmem_ld_wait();
-#pragma unroll
-              for (int part = 0; part < 4; ++part) {
-                float bv[8];
-                load_bias8(p.bias, n_base + c * 32 + part * 8, p.N, bv);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  h[c * 16 + part * 4 + e] =
-                      relu_pack_f16x2_bias(r[part * 8 + 2 * e], r[part * 8 + 2 * e + 1], bv[2 * e], bv[2 * e + 1]);
-              }
-            }
-          }
-          tcgen05_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty_bar[acc]), 0));
-          if (col_base == 0) {
-            const int y0 = m_blk * Cfg::PAIR_M + static_cast<int>(rank) * Cfg::BM + quad * 32;
-            uint8_t* wbuf = c_stage + (warp - Cfg::EPI_WARP0) * 2 * Cfg::C_BUF_BYTES;
-            const uint64_t pol = p.store_streaming ? l2_policy_evict_first() : l2_policy_evict_normal();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int col0 = n_base + c * 32;
-              if (col0 >= p.N) break;
-              if (p.c_aligned) {
-                if (y0 >= p.M) break;
-                uint8_t* buf = wbuf + (c & 1) * Cfg::C_BUF_BYTES;
-                if (lane == 0) bulk_wait_group_read<1>();
-                __syncwarp();
-                const uint32_t row_addr = smem_u32(buf) + lane * 64;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  st_shared_v4(row_addr + ((q ^ ((lane >> 1) & 3)) << 4), h[c * 16 + 4 * q], h[c * 16 + 4 * q + 1],
-                               h[c * 16 + 4 * q + 2], h[c * 16 + 4 * q + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                  tma_store_2d_hint(&tmap_c, buf, col0, y0, pol);
-                  bulk_commit_group();
-                }
-              } else if (row_ok) {
-                uint32_t hc[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) hc[e] = h[c * 16 + e];
-                store_row_chunk(crow, col0, p.N, hc, false, p.store_streaming != 0);
-              }
-            }
-          }
-          continue;
-        }
 #pragma unroll
         for (int c = 0; c < Cfg::EPI_COLS / 32; ++c) {
-          {
           uint32_t r[32];  // 32 columns per TMEM round trip
           tmem_ld_32x32b_x32(taddr + c * 32, r);
           tmem_ld_wait();
@@ -432,7 +331,6 @@ __global__ void __launch_bounds__(TcPairCfg<STAGES, BN>::THREADS, 1)
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) h[c * 16 + e] = relu_pack_f16x2(r[2 * e], r[2 * e + 1]);
-          }
           }
         }
         tcgen05_fence_before_sync();

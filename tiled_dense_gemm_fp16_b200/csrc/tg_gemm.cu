@@ -294,16 +294,6 @@ bool path_supports(int path, const Problem& p) {
   }
 }
 
-// Tiles of the 256 x 512 pair kernel's last, partial wave that run as
-// quarters (256 x 128 each, four work items per tile): all of them when
-// their quarters take fewer than four quarter-waves on `pairs` SM pairs,
-// else none.
-int pair_quarter_tail(int64_t tiles, int64_t pairs, int bn) {
-  if (bn != 512 || pairs <= 0 || tiles <= pairs || tune_int("TG_TUNE_QUARTERS", 1) == 0) return 0;
-  const int64_t r = tiles % pairs;
-  return (r > 0 && (4 * r + pairs - 1) / pairs < 4) ? static_cast<int>(r) : 0;
-}
-
 // Estimated relative time of the three tensor-core kernels on a 148-SM
 // device: waves of tiles x per-SM work of one tile.  The main loop of a tile
 // costs its per-SM MACs over the kernel's measured relative efficiency
@@ -320,12 +310,7 @@ int pick_tc_kernel(int64_t M, int64_t N, int64_t K, bool c_aligned) {
   const double area1 = 128.0 * 256.0, area3 = 128.0 * 512.0;
   const double t1 = waves(((M + 127) / 128) * ((N + 255) / 256), kSms) * area1 * k / 0.85 + area1 * kepi;
   const double t2 = waves(((M + 255) / 256) * ((N + 255) / 256), kPairs) * area1 * k / 0.88 + area1 * kepi;
-  // The 256 x 512 tile's partial last wave may run as quarters (at about
-  // the 1-SM kernel's efficiency).
-  const int64_t tiles3 = ((M + 255) / 256) * ((N + 511) / 512);
-  const int64_t tail3 = pair_quarter_tail(tiles3, kPairs, 512);
-  const double t3 = waves(tiles3 - tail3, kPairs) * area3 * (k + kepi) +
-                    (tail3 > 0 ? waves(4 * tail3, kPairs) * 0.25 * area3 * (k / 0.85 + kepi) : 0.0);
+  const double t3 = waves(((M + 255) / 256) * ((N + 511) / 512), kPairs) * area3 * (k + kepi);
   if (t3 <= t2 && t3 <= t1) return TG_PATH_TC_PAIR512;
   return t2 <= t1 ? TG_PATH_TC_PAIR : TG_PATH_TC;
 }
@@ -533,12 +518,12 @@ tg_status launch_tc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
 }
 
 // 2-CTA path: 256 x 256 tiles on SM pairs, clusters of 2 along x.
-template <int STAGES, int BN, bool QUARTERS>
+template <int STAGES, int BN>
 tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   using Cfg = TcPairCfg<STAGES, BN>;
   const int64_t M = o.M, N = o.N, K = o.K;
-  auto kernel = gemm_relu_tc_pair_kernel<STAGES, BN, QUARTERS>;
-  constexpr unsigned kAttrBit = 1u << (STAGES + (BN == 512 ? 16 : 0) + (QUARTERS ? 8 : 0));
+  auto kernel = gemm_relu_tc_pair_kernel<STAGES, BN>;
+  constexpr unsigned kAttrBit = 1u << (STAGES + (BN == 512 ? 16 : 0));
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!(info->tc_pair_attr & kAttrBit)) {
@@ -561,15 +546,7 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
   fill_tc_params(p, o);
   p.m_tiles = static_cast<int>((M + Cfg::PAIR_M - 1) / Cfg::PAIR_M);
   p.n_tiles = static_cast<int>((N + Cfg::BN - 1) / Cfg::BN);
-  const int pairs = info->sm_count / 2;
-  const int tiles = p.m_tiles * p.n_tiles;
-  // 256 x 512 tiles: the last, partial wave runs as quarters (256 x 128)
-  // spread over every pair when that takes fewer quarter-waves than a whole
-  // tile's time.
-  const int tail = QUARTERS ? pair_quarter_tail(tiles, pairs, BN) : 0;
-  p.full_tiles = tiles - tail;
-  p.num_tiles = p.full_tiles + 4 * tail;
-  p.idesc_q = make_idesc_f16_f32(Cfg::PAIR_M, 128, o.a_km, !o.b_nk);
+  p.num_tiles = p.m_tiles * p.n_tiles;
   p.k_blocks = static_cast<int>((K + Cfg::BK - 1) / Cfg::BK);
   p.group_m = tune_int("TG_TUNE_GROUP_M", BN == 512 ? 16 : 12);
   if (p.group_m < 1) p.group_m = 1;
@@ -577,6 +554,7 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
   p.l2_hints = tune_int("TG_TUNE_L2_HINTS", BN == 512 ? 2 : 5);
   p.prefetch_kb = tune_int("TG_TUNE_PREFETCH_KB", 0);
   p.wait_budget_ns = wait_budget(p.k_blocks);
+  const int pairs = info->sm_count / 2;
   const int clusters = p.num_tiles < pairs ? p.num_tiles : pairs;
 
   cudaLaunchConfig_t cfg;
@@ -596,17 +574,14 @@ tg_status launch_tc_pair_cfg(const Operands& o, cudaStream_t stream, DeviceInfo*
 
 tg_status launch_tc_pair(const Operands& o, cudaStream_t stream, DeviceInfo* info, int bn) {
   if (bn == 512) {
-    // The instance with a quarter-tile tail only where the tiles leave one.
-    const int64_t tiles = ((o.M + 255) / 256) * ((o.N + 511) / 512);
-    if (pair_quarter_tail(tiles, info->sm_count / 2, 512) > 0) return launch_tc_pair_cfg<4, 512, true>(o, stream, info);
     switch (tune_int("TG_TUNE_PAIR_STAGES", 4)) {
-      case 3: return launch_tc_pair_cfg<3, 512, false>(o, stream, info);
-      default: return launch_tc_pair_cfg<4, 512, false>(o, stream, info);
+      case 3: return launch_tc_pair_cfg<3, 512>(o, stream, info);
+      default: return launch_tc_pair_cfg<4, 512>(o, stream, info);
     }
   }
   switch (tune_int("TG_TUNE_PAIR_STAGES", 6)) {
-    case 5: return launch_tc_pair_cfg<5, 256, false>(o, stream, info);
-    default: return launch_tc_pair_cfg<6, 256, false>(o, stream, info);
+    case 5: return launch_tc_pair_cfg<5, 256>(o, stream, info);
+    default: return launch_tc_pair_cfg<6, 256>(o, stream, info);
   }
 }
 
