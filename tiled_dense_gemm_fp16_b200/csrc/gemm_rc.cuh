@@ -171,6 +171,35 @@ __device__ __forceinline__ void rw_finish(RowWriter& w) {
   if (w.g != 0) rw_emit(w, edge_realign(w.carry, make_uint4(0u, 0u, 0u, 0u), 16u - 2u * w.g));
 }
 
+// The 8 chunks of 8 values that start f elements (0..7) into 9 aligned
+// 16-byte blocks: chunk c = elements [8 c + f, 8 c + f + 8).  The shift is the
+// same for the whole row, so it is resolved once: a word offset f / 2 (one
+// of four unrolled copies) and a 0- or 16-bit funnel shift per word.
+__device__ __forceinline__ void realign_row8(const uint4 (&blk)[9], uint32_t f, uint4 (&out)[8]) {
+  uint32_t w[36];
+#pragma unroll
+  for (int b = 0; b < 9; ++b) {
+    w[4 * b] = blk[b].x;
+    w[4 * b + 1] = blk[b].y;
+    w[4 * b + 2] = blk[b].z;
+    w[4 * b + 3] = blk[b].w;
+  }
+  const uint32_t bits = (f & 1u) * 16u;
+#define TG_REALIGN_CASE(WO)                                                                          \
+  _Pragma("unroll") for (int c = 0; c < 8; ++c) out[c] =                                             \
+      make_uint4(__funnelshift_r(w[4 * c + (WO)], w[4 * c + (WO) + 1], bits),                        \
+                 __funnelshift_r(w[4 * c + (WO) + 1], w[4 * c + (WO) + 2], bits),                    \
+                 __funnelshift_r(w[4 * c + (WO) + 2], w[4 * c + (WO) + 3], bits),                    \
+                 __funnelshift_r(w[4 * c + (WO) + 3], w[4 * c + (WO) + 4], bits));
+  switch (f >> 1) {
+    case 0: TG_REALIGN_CASE(0) break;
+    case 1: TG_REALIGN_CASE(1) break;
+    case 2: TG_REALIGN_CASE(2) break;
+    default: TG_REALIGN_CASE(3) break;
+  }
+#undef TG_REALIGN_CASE
+}
+
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint4& v) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
 }
@@ -513,9 +542,11 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
             blk[c] = make_uint4(0u, 0u, 0u, 0u);
             if (c <= nch) ld_shared_v4(src + c * 16, blk[c]);
           }
+          uint4 out[8];
+          realign_row8(blk, f, out);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), edge_realign(blk[c], blk[c + 1], 2u * f));
+            if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), out[c]);
         }
         fence_proxy_async_smem();
         __syncwarp();
