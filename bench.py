@@ -537,14 +537,18 @@ def operand_sets(torch, dev, tensors, work_bytes: int):
     return sets, flush, note
 
 
-def repack_launches(tg, M, N, K, a_ptr, b_ptr, c_ptr, chosen) -> int:
+def repack_launches(tg, M, N, K, a_ptr, b_ptr, c_ptr, chosen, ws_bytes=0) -> int:
     """Kernels one call launches: the GEMM, plus on the repack path one row-padding copy per operand TMA
     cannot describe and, when the GEMM writes a padded C (rows of C not 16-byte aligned, M > 256), the
-    copy that moves it into C."""
+    copy that moves it into C; on the residue-class path with a workspace, the copy of B when TMA cannot
+    describe B."""
     n = 1
+    b_unaligned = N % 8 != 0 or b_ptr % 16 != 0
     if chosen == tg.Path.REPACK:
-        n += int(K % 8 != 0 or a_ptr % 16 != 0) + int(N % 8 != 0 or b_ptr % 16 != 0)
+        n += int(K % 8 != 0 or a_ptr % 16 != 0) + int(b_unaligned)
         n += int((N % 8 != 0 or c_ptr % 16 != 0) and M > 256)
+    elif chosen == tg.Path.RC and ws_bytes > 0:
+        n += int(b_unaligned)
     return n
 
 
@@ -612,7 +616,8 @@ class Fp16Case:
             self.chosen = self.path
         else:
             self.chosen = tg.select_path_ws(a.data_ptr(), b.data_ptr(), c.data_ptr(), M, N, K, self.ws_bytes)
-        self.launches_per_step = repack_launches(tg, M, N, K, a.data_ptr(), b.data_ptr(), c.data_ptr(), self.chosen)
+        self.launches_per_step = repack_launches(tg, M, N, K, a.data_ptr(), b.data_ptr(), c.data_ptr(), self.chosen,
+                                                 self.ws_bytes)
         self.cur = 0
 
     def call(self, a, b, c):

@@ -316,56 +316,34 @@ __global__ void __launch_bounds__(MxCfg<KIND>::THREADS, 1)
       int m_blk, n_blk;
       mx_tile_coords(p, t, m_blk, n_blk);
       const bool second_b = n_blk * 2 + 1 < p.n_atoms;
-      // Two stages per round: both stages' scales are stored, then one
-      // tcgen05.wait::st and two arrivals, which halves the stores' round
-      // trips on this role (it otherwise trails the MMAs).
-      for (int ks = 0; ks < p.k_stages; ks += 2) {
-        const int nst = min(2, p.k_stages - ks);
-        int stage2 = stage + 1;
-        uint32_t phase2 = phase;
-        if (stage2 == Cfg::STAGES) {
-          stage2 = 0;
-          phase2 ^= 1u;
-        }
-        bool ready = mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 48);
-        if (nst == 2) ready = ready && mbar_wait(&full_bar[stage2], phase2, abort_flag, p.wait_budget_ns, 49);
+      for (int ks = 0; ks < p.k_stages; ++ks) {
+        const bool ready = mbar_wait(&full_bar[stage], phase, abort_flag, p.wait_budget_ns, 48);
         if (!__all_sync(0xffffffffu, ready)) {
           ok = false;
           break;
         }
+        const int natoms = min(Cfg::ATOMS, p.atoms_k - ks * Cfg::ATOMS);
+        const uint32_t sfa_tmem = tmem_base + lane_base + Cfg::SF_COL0 + stage * Cfg::SF_STAGE_COLS;
+        const uint32_t sfb_tmem = sfa_tmem + Cfg::SFB_OFF;
+        const uint4* sa = reinterpret_cast<const uint4*>(sfa_smem + stage * Cfg::SFA_BYTES) + lane;
+        const uint4* sb = reinterpret_cast<const uint4*>(sfb_smem + stage * Cfg::SFB_BYTES) + lane;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (u < nst) {
-            const int st = u ? stage2 : stage;
-            const int natoms = min(Cfg::ATOMS, p.atoms_k - (ks + u) * Cfg::ATOMS);
-            const uint32_t sfa_tmem = tmem_base + lane_base + Cfg::SF_COL0 + st * Cfg::SF_STAGE_COLS;
-            const uint32_t sfb_tmem = sfa_tmem + Cfg::SFB_OFF;
-            const uint4* sa = reinterpret_cast<const uint4*>(sfa_smem + st * Cfg::SFA_BYTES) + lane;
-            const uint4* sb = reinterpret_cast<const uint4*>(sfb_smem + st * Cfg::SFB_BYTES) + lane;
-#pragma unroll
-            for (int a = 0; a < Cfg::ATOMS; ++a) {
-              if (a < natoms) {
-                // Line `lane` of each 512-byte atom: 16 bytes = 4 TMEM columns.
-                const uint4 va = sa[a * 32];
-                const uint4 vb0 = sb[a * 32];
-                const uint4 vb1 = second_b ? sb[Cfg::SFB_BYTES / 32 + a * 32] : make_uint4(0, 0, 0, 0);
-                tmem_st_32x32b_x4(sfa_tmem + 4 * a, va);
-                tmem_st_32x32b_x4(sfb_tmem + 8 * a, vb0);
-                tmem_st_32x32b_x4(sfb_tmem + 8 * a + 4, vb1);
-              }
-            }
+        for (int a = 0; a < Cfg::ATOMS; ++a) {
+          if (a < natoms) {
+            // Line `lane` of each 512-byte atom: 16 bytes = 4 TMEM columns.
+            const uint4 va = sa[a * 32];
+            const uint4 vb0 = sb[a * 32];
+            const uint4 vb1 = second_b ? sb[Cfg::SFB_BYTES / 32 + a * 32] : make_uint4(0, 0, 0, 0);
+            tmem_st_32x32b_x4(sfa_tmem + 4 * a, va);
+            tmem_st_32x32b_x4(sfb_tmem + 8 * a, vb0);
+            tmem_st_32x32b_x4(sfb_tmem + 8 * a + 4, vb1);
           }
         }
         tmem_st_wait();
         tcgen05_fence_before_sync();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&sf_full_bar[stage]);
-          if (nst == 2) mbar_arrive(&sf_full_bar[stage2]);
-        }
-        stage = stage2;
-        phase = phase2;
-        if (nst == 2 && ++stage == Cfg::STAGES) {
+        if (lane == 0) mbar_arrive(&sf_full_bar[stage]);
+        if (++stage == Cfg::STAGES) {
           stage = 0;
           phase ^= 1u;
         }

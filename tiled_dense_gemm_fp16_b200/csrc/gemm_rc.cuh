@@ -79,7 +79,6 @@ struct RcParams {
   int ring_stages, stg_slots;
   int ring_stage_bytes;    // 16 KiB of A + panels x 8 KiB of B
   int stg_bytes;           // 64 x stg_blocks x 16
-  int bulk_fetch;          // staging: 1 = one bulk copy per row piece, 0 = 16-byte cp.async per block
   int splits;              // CTAs per cluster along K (split mode)
   int c_stride;            // split mode: bytes per row of the fp32 partial (bn * 4 + 16)
   uint32_t idesc;
@@ -97,8 +96,9 @@ struct RcCfg {
   static constexpr int EPI_WARPS = 4;
   static constexpr int REAL_WARP0 = EPI_WARP0 + EPI_WARPS;
   static constexpr int REAL_WARPS = STAGE_B ? 4 : 0;
-  static constexpr int FETCH_WARP = REAL_WARP0 + REAL_WARPS;  // staging mode: copies B's rows
-  static constexpr int THREADS = (REAL_WARP0 + REAL_WARPS + (STAGE_B ? 1 : 0)) * 32;
+  static constexpr int FETCH_WARP0 = REAL_WARP0 + REAL_WARPS;  // staging mode: copy B's rows
+  static constexpr int FETCH_WARPS = STAGE_B ? 4 : 0;
+  static constexpr int THREADS = (FETCH_WARP0 + FETCH_WARPS) * 32;
   static constexpr int MAX_RING = 8;
   static constexpr int MAX_STG = 4;
   static constexpr int BAR_BYTES = 512;
@@ -164,6 +164,21 @@ __device__ __forceinline__ void rw_push(RowWriter& w, const uint32_t (&h)[16]) {
   rw_emit(w, edge_realign(q1, q2, sh));
   rw_emit(w, edge_realign(q2, q3, sh));
   w.carry = q3;
+}
+
+// As rw_push for 16 values (8 packed pairs).
+__device__ __forceinline__ void rw_push8(RowWriter& w, const uint32_t (&h)[8]) {
+  const uint4 q0 = make_uint4(h[0], h[1], h[2], h[3]);
+  const uint4 q1 = make_uint4(h[4], h[5], h[6], h[7]);
+  if (w.g == 0) {
+    rw_emit(w, q0);
+    rw_emit(w, q1);
+    return;
+  }
+  const uint32_t sh = 16u - 2u * w.g;
+  rw_emit(w, edge_realign(w.carry, q0, sh));
+  rw_emit(w, edge_realign(q0, q1, sh));
+  w.carry = q1;
 }
 
 // The block holding the piece's last g values (nothing when g == 0).
@@ -285,9 +300,7 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       mbar_init(&bfull_bar[s], Cfg::REAL_WARPS > 0 ? Cfg::REAL_WARPS : 1);
     }
     for (int s = 0; s < p.stg_slots; ++s) {
-      // Bulk copies: one arrival with the slot's byte count; 16-byte copies:
-      // the fetch warp's 32 lanes, as their copies land.
-      mbar_init(&stg_full[s], p.bulk_fetch ? 1 : 32);
+      mbar_init(&stg_full[s], Cfg::FETCH_WARPS * 32);  // every fetching lane, as its copies land
       mbar_init(&stg_empty[s], Cfg::REAL_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
@@ -490,7 +503,7 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       }
       tcgen05_fence_before_sync();
     }
-  } else if (STAGE_B && warp < Cfg::FETCH_WARP) {
+  } else if (STAGE_B && warp < Cfg::FETCH_WARP0) {
     // ------------------------------------------------------------------
     // Realigning warps: shift each staged row of B into the swizzled
     // MN-major operand tile.  Unit U = (lambda, d, seg): k-row
@@ -566,24 +579,30 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
     }
   } else if (STAGE_B) {
     // ------------------------------------------------------------------
-    // Fetch warp: for each k-block, once its staging slot is free, copy the
-    // 16-byte aligned blocks that cover B[k][n0 .. n0 + bn) of each of the
-    // 64 k-rows (lane l takes blocks l and l + 32, so each instruction moves
-    // whole cache lines); rows outside [0, K) and blocks that start past a
-    // row's end are not fetched.  A block that ends past a row's end reads
-    // at most 14 bytes beyond it, in the same 16-byte block (so never
-    // another page); those values only reach output columns past N, which
-    // are not stored.  The slot's barrier completes as the copies land.
+    // Fetch warps: for each k-block, once its staging slot is free, copy the
+    // 16-byte aligned blocks that cover B[k][n0 .. n0 + bn) of the k-rows
+    // this warp owns (every FETCH_WARPS-th of the 64; lane l takes blocks l
+    // and l + 32, so each instruction moves whole cache lines); rows outside
+    // [0, K) and blocks that start past a row's end are not fetched.  A block
+    // that ends past a row's end reads at most 14 bytes beyond it, in the same
+    // 16-byte block (so never another page); those values only reach output
+    // columns past N, which are not stored.  The slot's barrier completes as
+    // every lane's copies land.  One warp alone issues too slowly (its
+    // dependent address arithmetic, about 2 us per k-block), hence four.
     // ------------------------------------------------------------------
+    const int fw = warp - Cfg::FETCH_WARP0;
     const uint32_t pitch = static_cast<uint32_t>(p.stg_blocks * 16);
     const uintptr_t bbytes = reinterpret_cast<uintptr_t>(p.B);
+    const uintptr_t n_bytes = 2u * static_cast<uintptr_t>(p.N);
+    const uintptr_t row_step = 2u * Cfg::FETCH_WARPS * static_cast<uintptr_t>(p.ldb);
+    const uintptr_t off0 = 16u * static_cast<uintptr_t>(lane), off1 = off0 + 512u;
+    const bool second = lane + 32 < p.stg_blocks;
     int q = 0;
     uint32_t qph = 0;
-    int last_fill[Cfg::MAX_STG];
-    for (int i = 0; i < Cfg::MAX_STG; ++i) last_fill[i] = -1;
     bool ok = true;
     for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
       const RcTile T = rc_tile(p, t, rank, splits);
+      const uintptr_t n0_bytes = 2u * static_cast<uintptr_t>(T.n0);
       for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
         const bool free_slot = mbar_wait(&stg_empty[q], qph ^ 1u, abort_flag, p.wait_budget_ns, 0x6D);
         if (!__all_sync(0xffffffffu, free_slot)) {
@@ -592,52 +611,13 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
         }
         const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
         const int k_lo = kb * 64 - T.e;
-        if (p.bulk_fetch) {
-          // Lane l copies rows l and l + 32, each as one bulk copy of the
-          // 16-byte blocks from the one holding B[k][n0] to the one holding
-          // the piece's last element (or the row's, past N).
-          uint32_t bytes[2] = {0u, 0u};
-          uintptr_t src[2] = {0u, 0u};
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int j = lane + 32 * h;
-            const int k = k_lo + j;
-            if (k >= 0 && k < p.K) {
-              const uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k) * p.ldb);
-              const uintptr_t a0 = (row + 2u * static_cast<uintptr_t>(T.n0)) & ~uintptr_t(15);
-              const uintptr_t end = (row + 2u * static_cast<uintptr_t>(p.N) + 15u) & ~uintptr_t(15);
-              const uintptr_t span = end - a0;
-              const uintptr_t cap = 16u * static_cast<uintptr_t>(p.stg_blocks);
-              bytes[h] = static_cast<uint32_t>(span < cap ? span : cap);
-              src[h] = a0;
-            }
-          }
-          uint32_t total = bytes[0] + bytes[1];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-          if (lane == 0) mbar_arrive_expect_tx(&stg_full[q], total);
-          __syncwarp();
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            if (bytes[h] > 0)
-              bulk_load_g2s(stg + q * p.stg_bytes + (lane + 32 * h) * pitch, reinterpret_cast<const void*>(src[h]),
-                            bytes[h], &stg_full[q]);
-          last_fill[q] = static_cast<int>(qph);
-          if (++q == p.stg_slots) {
-            q = 0;
-            qph ^= 1u;
-          }
-          continue;
-        }
-        const int j_lo = k_lo < 0 ? -k_lo : 0;              // rows inside [0, K)
+        // This warp's first row inside [0, K), and the rows' end.
+        int j = fw;
+        if (k_lo + j < 0) j += ((-(k_lo + j) + Cfg::FETCH_WARPS - 1) / Cfg::FETCH_WARPS) * Cfg::FETCH_WARPS;
         const int j_hi = min(64, p.K - k_lo);
-        const uintptr_t row_step = 2u * static_cast<uintptr_t>(p.ldb);
-        uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k_lo + j_lo) * p.ldb);
-        const uintptr_t n0_bytes = 2u * static_cast<uintptr_t>(T.n0), n_bytes = 2u * static_cast<uintptr_t>(p.N);
-        const uintptr_t off0 = 16u * static_cast<uintptr_t>(lane), off1 = off0 + 512u;
-        const bool second = lane + 32 < p.stg_blocks;
+        uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k_lo + j) * p.ldb);
 #pragma unroll 4
-        for (int j = j_lo; j < j_hi; ++j, row += row_step) {
+        for (; j < j_hi; j += Cfg::FETCH_WARPS, row += row_step) {
           const uintptr_t a0 = (row + n0_bytes) & ~uintptr_t(15);
           const uintptr_t row_end = row + n_bytes;
           const uint32_t dst = sbase + j * pitch + lane * 16;
@@ -653,12 +633,6 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
     }
     // Every copy issued has landed before the CTA may exit.
     asm volatile("cp.async.wait_all;" ::: "memory");
-    if (p.bulk_fetch && lane == 0) {
-      // The bulk copies of each slot's last fill have landed.
-      volatile int no_abort = 0;
-      for (int i = 0; i < p.stg_slots; ++i)
-        if (last_fill[i] >= 0) mbar_wait(&stg_full[i], static_cast<uint32_t>(last_fill[i]), &no_abort, p.wait_budget_ns, 0x6E);
-    }
   }
 
   if (SPLIT) {
@@ -682,14 +656,14 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
         const int c0 = 64 * seg, c1 = min(c0 + 64, ncols);
         RowWriter w;
         rw_init(w, p.C + row * p.ldc + T.n0 + c0, c1 - c0);
-        for (int cc = c0; cc < c1; cc += 32) {
-          float acc[32];
+        for (int cc = c0; cc < c1; cc += 16) {
+          float acc[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
+          for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
           const uint32_t off = static_cast<uint32_t>(i * p.c_stride + cc * 4);
           for (int qr = 0; qr < splits; ++qr) {
 #pragma unroll
-            for (int v4 = 0; v4 < 8; ++v4) {
+            for (int v4 = 0; v4 < 4; ++v4) {
               const float4 x = ld_shared_cluster_f4(mapa_shared(part + off + v4 * 16, static_cast<uint32_t>(qr)));
               acc[4 * v4] += x.x;
               acc[4 * v4 + 1] += x.y;
@@ -697,19 +671,14 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
               acc[4 * v4 + 3] += x.w;
             }
           }
-          float b0[16], b1[16];
+          float b0[16];
           load_bias16(p.bias, T.n0 + cc, p.N, b0);
-          load_bias16(p.bias, T.n0 + cc + 16, p.N, b1);
-          uint32_t h[16];
+          uint32_t h[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             h[e] = relu_pack_f16x2_bias(__float_as_uint(acc[2 * e]), __float_as_uint(acc[2 * e + 1]), b0[2 * e],
                                         b0[2 * e + 1]);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            h[8 + e] = relu_pack_f16x2_bias(__float_as_uint(acc[16 + 2 * e]), __float_as_uint(acc[17 + 2 * e]),
-                                            b1[2 * e], b1[2 * e + 1]);
-          rw_push(w, h);
+          rw_push8(w, h);
         }
         rw_finish(w);
       }

@@ -772,7 +772,6 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
     p.stg_blocks = p.bn / 8 + 1;
     p.stg_bytes = 64 * p.stg_blocks * 16;
     p.stg_slots = tune_int("TG_TUNE_RC_STG", 3);
-    p.bulk_fetch = tune_int("TG_TUNE_RC_BULK", 1);
     if (p.stg_slots < 2 || p.stg_slots > RcCfg<true>::MAX_STG) return TG_ERR_INVALID_ARG;
   } else if (!encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
     return TG_ERR_LAUNCH;
