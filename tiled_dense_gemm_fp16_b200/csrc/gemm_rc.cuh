@@ -590,11 +590,12 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
     // every lane's copies land.  One warp alone issues too slowly (its
     // dependent address arithmetic, about 2 us per k-block), hence four.
     // ------------------------------------------------------------------
+    constexpr int kFw = Cfg::FETCH_WARPS > 0 ? Cfg::FETCH_WARPS : 1;  // (this branch runs in staging mode only)
     const int fw = warp - Cfg::FETCH_WARP0;
     const uint32_t pitch = static_cast<uint32_t>(p.stg_blocks * 16);
     const uintptr_t bbytes = reinterpret_cast<uintptr_t>(p.B);
     const uintptr_t n_bytes = 2u * static_cast<uintptr_t>(p.N);
-    const uintptr_t row_step = 2u * Cfg::FETCH_WARPS * static_cast<uintptr_t>(p.ldb);
+    const uintptr_t row_step = 2u * kFw * static_cast<uintptr_t>(p.ldb);
     const uintptr_t off0 = 16u * static_cast<uintptr_t>(lane), off1 = off0 + 512u;
     const bool second = lane + 32 < p.stg_blocks;
     int q = 0;
@@ -613,11 +614,11 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
         const int k_lo = kb * 64 - T.e;
         // This warp's first row inside [0, K), and the rows' end.
         int j = fw;
-        if (k_lo + j < 0) j += ((-(k_lo + j) + Cfg::FETCH_WARPS - 1) / Cfg::FETCH_WARPS) * Cfg::FETCH_WARPS;
+        if (k_lo + j < 0) j += ((-(k_lo + j) + kFw - 1) / kFw) * kFw;
         const int j_hi = min(64, p.K - k_lo);
         uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k_lo + j) * p.ldb);
 #pragma unroll 4
-        for (; j < j_hi; j += Cfg::FETCH_WARPS, row += row_step) {
+        for (; j < j_hi; j += kFw, row += row_step) {
           const uintptr_t a0 = (row + n0_bytes) & ~uintptr_t(15);
           const uintptr_t row_end = row + n_bytes;
           const uint32_t dst = sbase + j * pitch + lane * 16;
