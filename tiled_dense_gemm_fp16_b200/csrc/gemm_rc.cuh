@@ -80,7 +80,6 @@ struct RcParams {
   int ring_stage_bytes;    // 16 KiB of A + panels x 8 KiB of B
   int stg_bytes;           // 64 x stg_blocks x 16
   int splits;              // CTAs per cluster along K (split mode)
-  int prefetch_kb;         // > 0: also prefetch A's boxes into L2 this many k-blocks ahead
   int c_stride;            // split mode: bytes per row of the fp32 partial (bn * 4 + 16)
   uint32_t idesc;
   uint64_t wait_budget_ns;
@@ -345,10 +344,6 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
           const int k_lo = kb * 64 - T.e;  // B's first k-row of this block
           mbar_arrive_expect_tx(&full_bar[r], STAGE_B ? Cfg::A_BYTES : Cfg::A_BYTES + p.panels * Cfg::PANEL_BYTES);
           tma_load_2d(slot, &maps.a[T.s], &full_bar[r], kb * 64, T.q0);
-          // A narrow tile streams A from HBM: warm L2 a few k-blocks ahead so
-          // the ring's loads wait on L2, not on HBM.
-          if (p.prefetch_kb > 0 && kb + p.prefetch_kb < T.kb_hi)
-            tma_prefetch_l2_2d(&maps.a[T.s], (kb + p.prefetch_kb) * 64, T.q0);
           if (!STAGE_B) {
             for (int c = 0; c < p.panels; ++c)
               tma_load_2d(slot + Cfg::A_BYTES + c * Cfg::PANEL_BYTES, &maps.b, &full_bar[r], T.n0 + 64 * c, k_lo);

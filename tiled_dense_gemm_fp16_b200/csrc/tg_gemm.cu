@@ -783,7 +783,6 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   if (ring < 2) return TG_ERR_INTERNAL;
   p.ring_stages = ring;
   p.c_stride = p.bn * 4 + 16;
-  p.prefetch_kb = tune_int("TG_TUNE_RC_PREFETCH_KB", p.n_tiles == 1 ? 8 : 0);
   p.idesc = make_idesc_f16_f32(128, p.bn, false, true);
   p.wait_budget_ns = wait_budget(kb_max);
   const int smem = kFixed + ring * p.ring_stage_bytes + p.stg_slots * p.stg_bytes;
