@@ -25,13 +25,13 @@
 // 8 q + s of C is row q of class s (lda a multiple of 8: one class).
 //
 // B as it is, when TMA can describe it: 64-column boxes with 128-byte
-// swizzle at row offset 64 kb - e_s (the MN-major operand).  Otherwise B's
-// k-rows fall into residue classes the same way (k mod 8), one tensor map per
-// class loads each class's rows unswizzled, with 8 spare columns, into a
-// staging buffer, and four realigning warps shift every row into the swizzled
-// operand tile: two aligned 16-byte shared-memory reads and a funnel shift per
-// 16-byte chunk.  Their lane order keeps both the reads and the swizzled
-// writes free of bank conflicts.
+// swizzle at row offset 64 kb - e_s (the MN-major operand).  Otherwise eight
+// realigning warps read B's k-rows in place: one coalesced 16-byte load per
+// lane and row, the neighbouring block from the next lane by a shuffle, a
+// funnel shift by the row's offset (the same across the warp), and a store
+// into the swizzled operand tile that keeps each shared-memory phase free of
+// bank conflicts.  The next k-block's rows are loaded into registers while
+// this one's are shifted.
 //
 // C is written with aligned 16-byte stores: each epilogue thread owns one row
 // of the tile and shifts its values into the 16-byte blocks of that row
@@ -63,7 +63,7 @@ struct RcMaps {
 
 struct RcParams {
   __half* C;
-  const __half* B;         // staging mode: B read in place by the realigning warps
+  const __half* B;         // realigning mode: B read in place by the realigning warps
   const __half* bias;      // optional fp16[N] added before ReLU; nullptr = none
   int64_t ldb;             // row stride of B (elements)
   int64_t ldc;             // row stride of C (elements)
@@ -75,17 +75,15 @@ struct RcParams {
   int m_tiles, n_tiles, num_tiles, group_m;
   int bn;                  // tile width: 256, or N rounded up to 16 when N <= 240
   int panels;              // 64-column panels of the B tile: ceil(bn / 64)
-  int stg_blocks;          // staging: 16-byte blocks per B row piece, bn / 8 + 1
-  int ring_stages, stg_slots;
+  int ring_stages;
   int ring_stage_bytes;    // 16 KiB of A + panels x 8 KiB of B
-  int stg_bytes;           // 64 x stg_blocks x 16
   int splits;              // CTAs per cluster along K (split mode)
   int c_stride;            // split mode: bytes per row of the fp32 partial (bn * 4 + 16)
   uint32_t idesc;
   uint64_t wait_budget_ns;
 };
 
-template <bool STAGE_B>
+template <bool REALIGN_B>
 struct RcCfg {
   static constexpr int BM = 128;
   static constexpr int BK = 64;
@@ -95,12 +93,9 @@ struct RcCfg {
   static constexpr int EPI_WARP0 = 2;
   static constexpr int EPI_WARPS = 4;
   static constexpr int REAL_WARP0 = EPI_WARP0 + EPI_WARPS;
-  static constexpr int REAL_WARPS = STAGE_B ? 4 : 0;
-  static constexpr int FETCH_WARP0 = REAL_WARP0 + REAL_WARPS;  // staging mode: copy B's rows
-  static constexpr int FETCH_WARPS = STAGE_B ? 4 : 0;
-  static constexpr int THREADS = (FETCH_WARP0 + FETCH_WARPS) * 32;
+  static constexpr int REAL_WARPS = REALIGN_B ? 8 : 0;  // realigning warps (B read in place)
+  static constexpr int THREADS = (REAL_WARP0 + REAL_WARPS) * 32;
   static constexpr int MAX_RING = 8;
-  static constexpr int MAX_STG = 4;
   static constexpr int BAR_BYTES = 512;
 };
 
@@ -186,33 +181,13 @@ __device__ __forceinline__ void rw_finish(RowWriter& w) {
   if (w.g != 0) rw_emit(w, edge_realign(w.carry, make_uint4(0u, 0u, 0u, 0u), 16u - 2u * w.g));
 }
 
-// The 8 chunks of 8 values that start f elements (0..7) into 9 aligned
-// 16-byte blocks: chunk c = elements [8 c + f, 8 c + f + 8).  The shift is the
-// same for the whole row, so it is resolved once: a word offset f / 2 (one
-// of four unrolled copies) and a 0- or 16-bit funnel shift per word.
-__device__ __forceinline__ void realign_row8(const uint4 (&blk)[9], uint32_t f, uint4 (&out)[8]) {
-  uint32_t w[36];
-#pragma unroll
-  for (int b = 0; b < 9; ++b) {
-    w[4 * b] = blk[b].x;
-    w[4 * b + 1] = blk[b].y;
-    w[4 * b + 2] = blk[b].z;
-    w[4 * b + 3] = blk[b].w;
-  }
-  const uint32_t bits = (f & 1u) * 16u;
-#define TG_REALIGN_CASE(WO)                                                                          \
-  _Pragma("unroll") for (int c = 0; c < 8; ++c) out[c] =                                             \
-      make_uint4(__funnelshift_r(w[4 * c + (WO)], w[4 * c + (WO) + 1], bits),                        \
-                 __funnelshift_r(w[4 * c + (WO) + 1], w[4 * c + (WO) + 2], bits),                    \
-                 __funnelshift_r(w[4 * c + (WO) + 2], w[4 * c + (WO) + 3], bits),                    \
-                 __funnelshift_r(w[4 * c + (WO) + 3], w[4 * c + (WO) + 4], bits));
-  switch (f >> 1) {
-    case 0: TG_REALIGN_CASE(0) break;
-    case 1: TG_REALIGN_CASE(1) break;
-    case 2: TG_REALIGN_CASE(2) break;
-    default: TG_REALIGN_CASE(3) break;
-  }
-#undef TG_REALIGN_CASE
+__device__ __forceinline__ void st_shared_u4_pred(uint32_t addr, const uint4& v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "@p st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n\t}" ::"r"(addr),
+      "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(static_cast<uint32_t>(pred))
+      : "memory");
 }
 
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint4& v) {
@@ -224,16 +199,26 @@ __device__ __forceinline__ void st_shared_u4(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
-// 16-byte asynchronous copy global -> shared (L2 only); both addresses
-// 16-byte aligned.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-// Arrive on `bar` once every cp.async this thread issued so far has landed;
-// the arrival counts toward the barrier's expected count.
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Realigning step for 8 k-rows whose pieces start WO words plus bits / 16
+// elements past their first aligned block: lane l holds block l of each row
+// (lane 31 also block 32, in ext), takes block l + 1 from lane l + 1, and
+// stores output chunk l at dst + 1024 m (row 8 m of the panel layout).
+template <int WO, int R>
+__device__ __forceinline__ void rc_shift_rows(const uint4 (&cur)[R], const uint4 (&ext)[R], uint32_t bits, uint32_t dst,
+                                              bool stores, bool last_lane) {
+#pragma unroll
+  for (int m = 0; m < R; ++m) {
+    uint32_t w[8] = {cur[m].x, cur[m].y, cur[m].z, cur[m].w, 0u, 0u, 0u, 0u};
+    const uint32_t e[4] = {ext[m].x, ext[m].y, ext[m].z, ext[m].w};
+#pragma unroll
+    for (int i = 0; i <= WO; ++i) {
+      const uint32_t v = __shfl_down_sync(0xffffffffu, w[i], 1);
+      w[4 + i] = last_lane ? e[i] : v;
+    }
+    const uint4 out = make_uint4(__funnelshift_r(w[WO], w[WO + 1], bits), __funnelshift_r(w[WO + 1], w[WO + 2], bits),
+                                 __funnelshift_r(w[WO + 2], w[WO + 3], bits), __funnelshift_r(w[WO + 3], w[WO + 4], bits));
+    st_shared_u4_pred(dst + 1024u * m, out, stores);
+  }
 }
 
 // One output tile: class s, rows q0 .. q0 + 127 of the class, columns
@@ -265,21 +250,18 @@ __device__ __forceinline__ RcTile rc_tile(const RcParams& p, int t, int rank, in
   return r;
 }
 
-template <bool STAGE_B, bool SPLIT>
-__global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
+template <bool REALIGN_B, bool SPLIT>
+__global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
     gemm_relu_rc_kernel(const __grid_constant__ RcMaps maps, const RcParams p) {
-  using Cfg = RcCfg<STAGE_B>;
+  using Cfg = RcCfg<REALIGN_B>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint8_t* stg = smem + p.ring_stages * p.ring_stage_bytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stg + (STAGE_B ? p.stg_slots * p.stg_bytes : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.ring_stages * p.ring_stage_bytes);
   uint64_t* full_bar = bars;                       // [ring] TMA bytes landed
   uint64_t* empty_bar = bars + Cfg::MAX_RING;      // [ring] MMAs done with the slot
-  uint64_t* bfull_bar = bars + 2 * Cfg::MAX_RING;  // [ring] realigned B written (staging mode)
-  uint64_t* stg_full = bars + 3 * Cfg::MAX_RING;   // [stg] a staging slot's copies landed
-  uint64_t* stg_empty = stg_full + Cfg::MAX_STG;   // [stg] a staging slot's rows realigned
-  uint64_t* acc_full = stg_empty + Cfg::MAX_STG;   // [2]
+  uint64_t* bfull_bar = bars + 2 * Cfg::MAX_RING;  // [ring] realigned B written (realigning mode)
+  uint64_t* acc_full = bars + 3 * Cfg::MAX_RING;   // [2]
   uint64_t* acc_empty = acc_full + 2;              // [2]
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -298,10 +280,6 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
       mbar_init(&bfull_bar[s], Cfg::REAL_WARPS > 0 ? Cfg::REAL_WARPS : 1);
-    }
-    for (int s = 0; s < p.stg_slots; ++s) {
-      mbar_init(&stg_full[s], Cfg::FETCH_WARPS * 32);  // every fetching lane, as its copies land
-      mbar_init(&stg_empty[s], Cfg::REAL_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -325,7 +303,7 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------
     // Producer: A's class boxes into the ring, and B's boxes too in direct
-    // mode (in staging mode the realigning warps fetch B).
+    // mode (otherwise the realigning warps bring B).
     // ------------------------------------------------------------------
     if (lane == 0) {
       int r = 0;
@@ -342,9 +320,9 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
           }
           uint8_t* slot = ring + r * p.ring_stage_bytes;
           const int k_lo = kb * 64 - T.e;  // B's first k-row of this block
-          mbar_arrive_expect_tx(&full_bar[r], STAGE_B ? Cfg::A_BYTES : Cfg::A_BYTES + p.panels * Cfg::PANEL_BYTES);
+          mbar_arrive_expect_tx(&full_bar[r], REALIGN_B ? Cfg::A_BYTES : Cfg::A_BYTES + p.panels * Cfg::PANEL_BYTES);
           tma_load_2d(slot, &maps.a[T.s], &full_bar[r], kb * 64, T.q0);
-          if (!STAGE_B) {
+          if (!REALIGN_B) {
             for (int c = 0; c < p.panels; ++c)
               tma_load_2d(slot + Cfg::A_BYTES + c * Cfg::PANEL_BYTES, &maps.b, &full_bar[r], T.n0 + 64 * c, k_lo);
           }
@@ -381,7 +359,7 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       const uint32_t d_tmem = tmem_base + acc * 256;
       for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
         bool landed = mbar_wait(&full_bar[r], rph, abort_flag, p.wait_budget_ns, 0x66);
-        if (STAGE_B) landed = landed && mbar_wait(&bfull_bar[r], rph, abort_flag, p.wait_budget_ns, 0x6C);
+        if (REALIGN_B) landed = landed && mbar_wait(&bfull_bar[r], rph, abort_flag, p.wait_budget_ns, 0x6C);
         if (!__all_sync(0xffffffffu, landed)) {
           ok = false;
           break;
@@ -503,137 +481,115 @@ __global__ void __launch_bounds__(RcCfg<STAGE_B>::THREADS, 1)
       }
       tcgen05_fence_before_sync();
     }
-  } else if (STAGE_B && warp < Cfg::FETCH_WARP0) {
+  } else if (REALIGN_B) {
     // ------------------------------------------------------------------
-    // Realigning warps: shift each staged row of B into the swizzled
-    // MN-major operand tile.  Unit U = (lambda, d, seg): k-row
-    // j = 8 lambda + ((lambda + d) & 7), 64-column segment seg; the 8 lanes
-    // of a shared-memory phase differ in lambda, so their reads (staging
-    // rows are an odd number of 16-byte blocks long) and their swizzled
-    // writes (j & 7 differs) hit 8 different bank groups.  Rows outside
-    // [0, K) are written as zeros.  These warps issue no asynchronous
-    // copies of their own, so their proxy fence has nothing in flight to
-    // wait for.
+    // Realigning warps: B's k-rows straight from global memory into the
+    // swizzled MN-major operand tile, no staging buffer.  Warp w owns the
+    // k-rows j = 8 m + w of a block.  For one row, lane l loads the 16-byte
+    // aligned block l of the row piece (one coalesced load per row; lane 31
+    // also loads block 32), takes block l + 1 from lane l + 1 by a shuffle,
+    // shifts the pair by the piece's offset f and stores output chunk l to
+    // panel l / 8, position (l mod 8) xor (j mod 8): the 8 lanes of a
+    // shared-memory phase hit 8 different bank groups.  Rows 8 apart start
+    // 16 ldb bytes apart, so a warp's eight rows share f for the whole tile:
+    // one uniform branch per k-block picks the word offset and the rows'
+    // steps interleave.  The next k-block's rows are loaded into registers
+    // while this block's are shifted.  Blocks that start past a row's end are
+    // not loaded; a block that ends past it reads at most 14 bytes beyond, in
+    // the same 16-byte block (never another page), and those values reach
+    // only output columns that are not stored.  Rows outside [0, K) are
+    // written as zeros.
     // ------------------------------------------------------------------
-    const int tid = threadIdx.x - Cfg::REAL_WARP0 * 32;
-    const int units = 64 * p.panels;
-    const uint32_t pitch = static_cast<uint32_t>(p.stg_blocks * 16);
-    int r = 0, q = 0;
-    uint32_t rph = 0, qph = 0;
-    bool ok = true;
-    for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
-      const RcTile T = rc_tile(p, t, rank, splits);
-      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
-        bool got = mbar_wait(&stg_full[q], qph, abort_flag, p.wait_budget_ns, 0x6A);
-        got = got && mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
-        if (!__all_sync(0xffffffffu, got)) {
-          ok = false;
-          break;
-        }
-        const int k_lo = kb * 64 - T.e;
-        const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
-        const uint32_t bbase = smem_u32(ring + r * p.ring_stage_bytes) + Cfg::A_BYTES;
-        for (int U = tid; U < units; U += Cfg::REAL_WARPS * 32) {
-          const int lam = U & 7, d = (U >> 3) & 7, seg = U >> 6;
-          const int j = 8 * lam + ((lam + d) & 7);
-          const int k = k_lo + j;
-          const int nch = min(8, (p.bn - 64 * seg) >> 3);
-          const uint32_t dst = bbase + static_cast<uint32_t>(seg * Cfg::PANEL_BYTES + j * 128);
-          if (k < 0 || k >= p.K) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), make_uint4(0u, 0u, 0u, 0u));
-            continue;
-          }
-          // This row piece starts f elements past its first aligned block.
-          const uint32_t f = static_cast<uint32_t>(
-              ((reinterpret_cast<uintptr_t>(p.B) + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k) * p.ldb + T.n0)) >> 1) & 7u);
-          const uint32_t src = sbase + j * pitch + seg * 128;
-          uint4 blk[9];
-#pragma unroll
-          for (int c = 0; c < 9; ++c) {
-            blk[c] = make_uint4(0u, 0u, 0u, 0u);
-            if (c <= nch) ld_shared_v4(src + c * 16, blk[c]);
-          }
-          uint4 out[8];
-          realign_row8(blk, f, out);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            if (c < nch) st_shared_u4(dst + ((c ^ (j & 7)) << 4), out[c]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bfull_bar[r]);
-          mbar_arrive(&stg_empty[q]);
-        }
-        if (++r == p.ring_stages) {
-          r = 0;
-          rph ^= 1u;
-        }
-        if (++q == p.stg_slots) {
-          q = 0;
-          qph ^= 1u;
-        }
-      }
-    }
-  } else if (STAGE_B) {
-    // ------------------------------------------------------------------
-    // Fetch warps: for each k-block, once its staging slot is free, copy the
-    // 16-byte aligned blocks that cover B[k][n0 .. n0 + bn) of the k-rows
-    // this warp owns (every FETCH_WARPS-th of the 64; lane l takes blocks l
-    // and l + 32, so each instruction moves whole cache lines); rows outside
-    // [0, K) and blocks that start past a row's end are not fetched.  A block
-    // that ends past a row's end reads at most 14 bytes beyond it, in the same
-    // 16-byte block (so never another page); those values only reach output
-    // columns past N, which are not stored.  The slot's barrier completes as
-    // every lane's copies land.  One warp alone issues too slowly (its
-    // dependent address arithmetic, about 2 us per k-block), hence four.
-    // ------------------------------------------------------------------
-    constexpr int kFw = Cfg::FETCH_WARPS > 0 ? Cfg::FETCH_WARPS : 1;  // (this branch runs in staging mode only)
-    const int fw = warp - Cfg::FETCH_WARP0;
-    const uint32_t pitch = static_cast<uint32_t>(p.stg_blocks * 16);
+    static_assert(!REALIGN_B || Cfg::REAL_WARPS == 8, "k-rows j = 8 m + warp: row j mod 8 is the warp's");
+    constexpr int kRows = 8;
+    const int rw = warp - Cfg::REAL_WARP0;
     const uintptr_t bbytes = reinterpret_cast<uintptr_t>(p.B);
     const uintptr_t n_bytes = 2u * static_cast<uintptr_t>(p.N);
-    const uintptr_t row_step = 2u * kFw * static_cast<uintptr_t>(p.ldb);
-    const uintptr_t off0 = 16u * static_cast<uintptr_t>(lane), off1 = off0 + 512u;
-    const bool second = lane + 32 < p.stg_blocks;
-    int q = 0;
-    uint32_t qph = 0;
-    bool ok = true;
-    for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
-      const RcTile T = rc_tile(p, t, rank, splits);
-      const uintptr_t n0_bytes = 2u * static_cast<uintptr_t>(T.n0);
-      for (int kb = T.kb_lo; kb < T.kb_hi; ++kb) {
-        const bool free_slot = mbar_wait(&stg_empty[q], qph ^ 1u, abort_flag, p.wait_budget_ns, 0x6D);
-        if (!__all_sync(0xffffffffu, free_slot)) {
-          ok = false;
-          break;
-        }
-        const uint32_t sbase = smem_u32(stg + q * p.stg_bytes);
-        const int k_lo = kb * 64 - T.e;
-        // This warp's first row inside [0, K), and the rows' end.
-        int j = fw;
-        if (k_lo + j < 0) j += ((-(k_lo + j) + kFw - 1) / kFw) * kFw;
-        const int j_hi = min(64, p.K - k_lo);
-        uintptr_t row = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k_lo + j) * p.ldb);
-#pragma unroll 4
-        for (; j < j_hi; j += kFw, row += row_step) {
-          const uintptr_t a0 = (row + n0_bytes) & ~uintptr_t(15);
-          const uintptr_t row_end = row + n_bytes;
-          const uint32_t dst = sbase + j * pitch + lane * 16;
-          if (a0 + off0 < row_end) cp_async_16(dst, reinterpret_cast<const void*>(a0 + off0));
-          if (second && a0 + off1 < row_end) cp_async_16(dst + 512, reinterpret_cast<const void*>(a0 + off1));
-        }
-        cp_async_mbar_arrive(&stg_full[q]);
-        if (++q == p.stg_slots) {
-          q = 0;
-          qph ^= 1u;
-        }
+    const uintptr_t stride = 16u * static_cast<uintptr_t>(p.ldb);  // 8 k-rows, in bytes
+    const int chunks = p.bn >> 3;  // 16-byte chunks per operand row, <= 32
+    // Chunk `lane` of row j = 8 m + rw sits in panel lane / 8 at row j,
+    // position (lane mod 8) xor (j mod 8), and j mod 8 = rw.
+    const uint32_t dst_off = static_cast<uint32_t>((lane >> 3) * Cfg::PANEL_BYTES + rw * 128 +
+                                                   (((lane & 7) ^ (rw & 7)) << 4));
+    const bool stores = lane < chunks;
+    const bool extra = lane == 31 && chunks == 32;  // block 32 of the piece
+    uint4 cur[kRows], ext[kRows];
+    uint32_t f_cur = 0, f_next = 0;  // the rows' offset past their first aligned block
+    // The k-blocks this CTA walks, in the order every role walks them.
+    int t = t_first, kb = 0;
+    RcTile T{};
+    bool valid = false;
+    for (; t < p.num_tiles; t += t_step) {
+      T = rc_tile(p, t, rank, splits);
+      if (T.kb_hi > T.kb_lo) {
+        kb = T.kb_lo;
+        valid = true;
+        break;
       }
     }
-    // Every copy issued has landed before the CTA may exit.
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // Rows k0 + 8 m: their pieces start at the same offset f past a 16-byte
+    // boundary (8 rows are 16 ldb bytes apart), so one address and one
+    // bounds test serve all eight.
+    auto load_rows = [&](const RcTile& U, int kbu) {
+      const int k0 = kbu * 64 - U.e + rw;
+      const uintptr_t row0 = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k0) * p.ldb);
+      const uintptr_t start = row0 + 2u * static_cast<uintptr_t>(U.n0);
+      const uintptr_t a0 = start & ~uintptr_t(15);
+      const uintptr_t blk = a0 + 16u * static_cast<uintptr_t>(lane);
+      const bool lane_ok = lane <= chunks && blk < row0 + n_bytes;
+      const bool ext_ok = extra && a0 + 512u < row0 + n_bytes;
+      f_next = static_cast<uint32_t>((start >> 1) & 7u);
+#pragma unroll
+      for (int m = 0; m < kRows; ++m) {
+        const bool in = static_cast<unsigned>(k0 + 8 * m) < static_cast<unsigned>(p.K);
+        cur[m] = make_uint4(0u, 0u, 0u, 0u);
+        ext[m] = make_uint4(0u, 0u, 0u, 0u);
+        ld_nc_v4_pred(cur[m], reinterpret_cast<const void*>(blk + m * stride), in && lane_ok);
+        ld_nc_v4_pred(ext[m], reinterpret_cast<const void*>(a0 + 512u + m * stride), in && ext_ok);
+      }
+    };
+    if (valid) load_rows(T, kb);
+    int r = 0;
+    uint32_t rph = 0;
+    while (valid) {
+      // The next k-block in the walk.
+      int t2 = t, kb2 = kb + 1;
+      RcTile T2 = T;
+      bool valid2 = true;
+      while (kb2 >= T2.kb_hi) {
+        t2 += t_step;
+        if (t2 >= p.num_tiles) {
+          valid2 = false;
+          break;
+        }
+        T2 = rc_tile(p, t2, rank, splits);
+        kb2 = T2.kb_lo;
+      }
+      f_cur = f_next;
+      const bool got = mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
+      if (!__all_sync(0xffffffffu, got)) break;
+      // Rows outside [0, K) were loaded as zeros and shift to zeros.
+      const uint32_t dst = smem_u32(ring + r * p.ring_stage_bytes) + Cfg::A_BYTES + dst_off;
+      const uint32_t bits = (f_cur & 1u) * 16u;
+      switch (f_cur >> 1) {
+        case 0: rc_shift_rows<0>(cur, ext, bits, dst, stores, lane == 31); break;
+        case 1: rc_shift_rows<1>(cur, ext, bits, dst, stores, lane == 31); break;
+        case 2: rc_shift_rows<2>(cur, ext, bits, dst, stores, lane == 31); break;
+        default: rc_shift_rows<3>(cur, ext, bits, dst, stores, lane == 31); break;
+      }
+      if (valid2) load_rows(T2, kb2);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bfull_bar[r]);
+      if (++r == p.ring_stages) {
+        r = 0;
+        rph ^= 1u;
+      }
+      t = t2;
+      kb = kb2;
+      T = T2;
+      valid = valid2;
+    }
   }
 
   if (SPLIT) {

@@ -768,24 +768,19 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   const bool stage_b = !((reinterpret_cast<uintptr_t>(o.B) & 15u) == 0 && o.ldb % 8 == 0);
   p.B = static_cast<const __half*>(o.B);
   p.ldb = o.ldb;
-  if (stage_b) {
-    p.stg_blocks = p.bn / 8 + 1;
-    p.stg_bytes = 64 * p.stg_blocks * 16;
-    p.stg_slots = tune_int("TG_TUNE_RC_STG", 3);
-    if (p.stg_slots < 2 || p.stg_slots > RcCfg<true>::MAX_STG) return TG_ERR_INVALID_ARG;
-  } else if (!encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
+  if (!stage_b && !encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
     return TG_ERR_LAUNCH;
   }
   p.ring_stage_bytes = RcCfg<false>::A_BYTES + p.panels * RcCfg<false>::PANEL_BYTES;
   constexpr int kSmemMax = 232448, kFixed = 1024 + 512;
-  int ring = (kSmemMax - kFixed - p.stg_slots * p.stg_bytes) / p.ring_stage_bytes;
+  int ring = (kSmemMax - kFixed) / p.ring_stage_bytes;
   ring = ring > RcCfg<false>::MAX_RING ? RcCfg<false>::MAX_RING : ring;
   if (ring < 2) return TG_ERR_INTERNAL;
   p.ring_stages = ring;
   p.c_stride = p.bn * 4 + 16;
   p.idesc = make_idesc_f16_f32(128, p.bn, false, true);
   p.wait_budget_ns = wait_budget(kb_max);
-  const int smem = kFixed + ring * p.ring_stage_bytes + p.stg_slots * p.stg_bytes;
+  const int smem = kFixed + ring * p.ring_stage_bytes;
   // Few tiles: split K over a cluster (each CTA keeps at least 4 k-blocks),
   // when the fp32 partial fits in the ring.
   const int sms = info->sm_count;
