@@ -190,6 +190,12 @@ __device__ __forceinline__ void st_shared_u4_pred(uint32_t addr, const uint4& v,
       : "memory");
 }
 
+// 16-byte store to a shared::cluster address (this CTA's or a peer's).
+__device__ __forceinline__ void st_shared_cluster_u4(uint32_t addr, const uint4& v) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint4& v) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
 }
@@ -457,28 +463,11 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
       }
     } else {
+      // The partial stays in TMEM until every CTA of the cluster is done
+      // with its ring (below).  A failed wait has set the abort flag.
       const RcTile T = rc_tile(p, t_first, rank, splits);
-      const bool has_k = T.kb_hi > T.kb_lo;
-      bool ready = true;
-      if (has_k) ready = mbar_wait(&acc_full[0], 0, abort_flag, p.wait_budget_ns, 0x69);
-      ready = __all_sync(0xffffffffu, ready);
-      if (ready) {
-        tcgen05_fence_after_sync();
-        const uint32_t prow = smem_u32(ring) + static_cast<uint32_t>(i * p.c_stride);
-        for (int c = 0; c * 16 < p.bn; ++c) {
-          uint32_t v[16];
-          if (has_k) {
-            tmem_ld_32x32b_x16(lane_base + c * 16, v);
-            tmem_ld_wait();
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = 0u;  // empty K share: the partial is zero
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            st_shared_u4(prow + c * 64 + e * 16, make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
-        }
-      }
+      if (T.kb_hi > T.kb_lo) mbar_wait(&acc_full[0], 0, abort_flag, p.wait_budget_ns, 0x69);
+      __syncwarp();
       tcgen05_fence_before_sync();
     }
   } else if (REALIGN_B) {
@@ -593,21 +582,53 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
   }
 
   if (SPLIT) {
-    // Sum this CTA's share of the tile's rows over the cluster's partials.
+    // Rank q owns the tile's rows [128 q / S, 128 (q + 1) / S).  Once every
+    // CTA of the cluster is done with its ring, each epilogue thread pushes
+    // its row of the fp32 partial into the owner's shared memory, slot
+    // `rank` (remote stores, nothing waits on a round trip); after a second
+    // cluster barrier each owner sums its rows over the slots in rank order,
+    // from its own shared memory, and writes them to C.
+    const RcTile T = rc_tile(p, t_first, rank, splits);
+    const int rpo = (128 + splits - 1) / splits;  // slot rows
+    const uint32_t part = smem_u32(ring);
+    tcgen05_fence_before_sync();
     __syncthreads();
     cluster_sync();
-    if (warp >= Cfg::EPI_WARP0 && warp < Cfg::REAL_WARP0 && !*abort_flag) {
-      const RcTile T = rc_tile(p, t_first, rank, splits);
-      const int tid = threadIdx.x - Cfg::EPI_WARP0 * 32;
+    if (warp >= Cfg::EPI_WARP0 && warp < Cfg::EPI_WARP0 + Cfg::EPI_WARPS && !*abort_flag) {
+      tcgen05_fence_after_sync();
+      const int quad = warp & 3;
+      const int i = quad * 32 + lane;  // row of the tile = TMEM lane
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+      int q = (i * splits) / 128;
+      if ((128 * (q + 1)) / splits <= i) ++q;
+      const int il = i - (128 * q) / splits;
+      const uint32_t dst =
+          mapa_shared(part + static_cast<uint32_t>((rank * rpo + il) * p.c_stride), static_cast<uint32_t>(q));
+      const bool has_k = T.kb_hi > T.kb_lo;
+      for (int c = 0; c * 16 < p.bn; ++c) {
+        uint32_t v[16];
+        if (has_k) {
+          tmem_ld_32x32b_x16(lane_base + c * 16, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = 0u;  // empty K share: the partial is zero
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          st_shared_cluster_u4(dst + c * 64 + e * 16, make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
+      }
+    }
+    cluster_sync();
+    if (!*abort_flag) {
       const int r_lo = (128 * rank) / splits, r_hi = (128 * (rank + 1)) / splits;
       const int nrows = r_hi - r_lo;
       const int ncols = min(p.bn, p.N - T.n0);
       const int segs = (ncols + 63) / 64;
-      const uint32_t part = smem_u32(ring);
-      for (int it = tid; it < nrows * segs; it += Cfg::EPI_WARPS * 32) {
-        const int i = r_lo + it % nrows;
+      for (int it = threadIdx.x; it < nrows * segs; it += Cfg::THREADS) {
+        const int il = it % nrows;
         const int seg = it / nrows;
-        const int qrow = T.q0 + i;
+        const int qrow = T.q0 + r_lo + il;
         if (qrow >= p.rows_in_class[T.s]) continue;
         const int64_t row = static_cast<int64_t>(qrow) * p.a_classes + T.s;
         const int c0 = 64 * seg, c1 = min(c0 + 64, ncols);
@@ -617,15 +638,16 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
           float acc[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
-          const uint32_t off = static_cast<uint32_t>(i * p.c_stride + cc * 4);
           for (int qr = 0; qr < splits; ++qr) {
+            const uint32_t off = part + static_cast<uint32_t>((qr * rpo + il) * p.c_stride + cc * 4);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
-              const float4 x = ld_shared_cluster_f4(mapa_shared(part + off + v4 * 16, static_cast<uint32_t>(qr)));
-              acc[4 * v4] += x.x;
-              acc[4 * v4 + 1] += x.y;
-              acc[4 * v4 + 2] += x.z;
-              acc[4 * v4 + 3] += x.w;
+              uint4 x;
+              ld_shared_v4(off + v4 * 16, x);
+              acc[4 * v4] += __uint_as_float(x.x);
+              acc[4 * v4 + 1] += __uint_as_float(x.y);
+              acc[4 * v4 + 2] += __uint_as_float(x.z);
+              acc[4 * v4 + 3] += __uint_as_float(x.w);
             }
           }
           float b0[16];
@@ -640,7 +662,6 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
         rw_finish(w);
       }
     }
-    cluster_sync();  // peers are done reading this CTA's partial
   }
 
   tcgen05_fence_before_sync();

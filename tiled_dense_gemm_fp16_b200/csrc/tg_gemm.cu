@@ -782,16 +782,18 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   p.wait_budget_ns = wait_budget(kb_max);
   const int smem = kFixed + ring * p.ring_stage_bytes;
   // Few tiles: split K over a cluster (each CTA keeps at least 4 k-blocks),
-  // when the fp32 partial fits in the ring.
+  // when the cluster's partials of one CTA's rows (S slots of ceil(128 / S)
+  // rows) fit in the ring.
   const int sms = info->sm_count;
   int splits = 1;
-  if (2 * p.num_tiles <= sms && 128 * p.c_stride <= ring * p.ring_stage_bytes) {
+  if (2 * p.num_tiles <= sms) {
     splits = sms / p.num_tiles;
     const int kb_min = static_cast<int>((K + 63) / 64);
     splits = splits > 8 ? 8 : splits;
     while (splits > 1 && kb_min / splits < 4) --splits;
     splits = tune_int("TG_TUNE_RC_SPLITS", splits);
     if (splits > 8) splits = 8;
+    while (splits > 1 && splits * ((128 + splits - 1) / splits) * p.c_stride > ring * p.ring_stage_bytes) --splits;
   }
   p.splits = splits;
   if (splits > 1) {
