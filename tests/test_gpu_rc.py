@@ -56,9 +56,10 @@ def test_rc_unaligned_bases(offsets, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1000, 129, 4099), (8191, 129, 1027), (300, 16, 5000), (50, 240, 3001),
-                                   (2000, 200, 777), (129, 72, 20000)])
+                                   (2000, 200, 777), (129, 72, 20000), (2000, 72, 3001), (3000, 16, 4000)])
 def test_rc_split_k_cluster(M, N, K):
-    """One column of tiles and few rows of tiles: K split over a cluster, partials summed over DSMEM."""
+    """One column of tiles and few rows of tiles: K split over a cluster, partials summed over DSMEM.
+    (8191, 129, 1027), (2000, 72, 3001) and (3000, 16, 4000) take 256-row tiles (two accumulators)."""
     A, B = inputs.operands(M, N, K, "int", seed=M + N + K)
     got, guards = run_gpu(A, B, RC)
     assert guards

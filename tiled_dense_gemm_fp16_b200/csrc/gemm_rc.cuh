@@ -71,14 +71,15 @@ struct RcParams {
   int a_classes;           // 8, or 1 when A's row stride is a multiple of 8 elements
   int a_shift[kRcClasses]; // e_s: elements between the class map's column 0 and A[r][0]
   int rows_in_class[kRcClasses];
-  int tile_start[kRcClasses + 1];  // first 128-row tile of each class; [a_classes] = m_tiles
+  int tile_start[kRcClasses + 1];  // first tile of each class; [a_classes] = m_tiles
   int m_tiles, n_tiles, num_tiles, group_m;
   int bn;                  // tile width: 256, or N rounded up to 16 when N <= 240
   int panels;              // 64-column panels of the B tile: ceil(bn / 64)
   int ring_stages;
-  int ring_stage_bytes;    // 16 KiB of A + panels x 8 KiB of B
+  int msub;                // 128-row sub-tiles per tile: 1, or 2 in split mode (one tile per CTA,
+                           // two accumulators sharing each B stage)
+  int ring_stage_bytes;    // msub x 16 KiB of A + panels x 8 KiB of B
   int splits;              // CTAs per cluster along K (split mode)
-  int c_stride;            // split mode: bytes per row of the fp32 partial (bn * 4 + 16)
   uint32_t idesc;
   uint64_t wait_budget_ns;
 };
@@ -248,7 +249,7 @@ __device__ __forceinline__ RcTile rc_tile(const RcParams& p, int t, int rank, in
   for (int c = 1; c < kRcClasses; ++c)
     if (c < p.a_classes && p.tile_start[c] <= mt) s = c;
   r.s = s;
-  r.q0 = (mt - p.tile_start[s]) * 128;
+  r.q0 = (mt - p.tile_start[s]) * 128 * p.msub;
   r.e = p.a_shift[s];
   const int kb_total = (p.K + r.e + 63) / 64;
   r.kb_lo = static_cast<int>((static_cast<int64_t>(kb_total) * rank) / splits);
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
   const int splits = SPLIT ? p.splits : 1;
   const int t_first = SPLIT ? static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.x);
   const int t_step = SPLIT ? p.num_tiles : static_cast<int>(gridDim.x);
-  constexpr uint32_t kTmemCols = SPLIT ? 256 : 512;
+  constexpr uint32_t kTmemCols = 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ring_stages; ++s) {
@@ -326,11 +327,12 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
           }
           uint8_t* slot = ring + r * p.ring_stage_bytes;
           const int k_lo = kb * 64 - T.e;  // B's first k-row of this block
-          mbar_arrive_expect_tx(&full_bar[r], REALIGN_B ? Cfg::A_BYTES : Cfg::A_BYTES + p.panels * Cfg::PANEL_BYTES);
+          const int a_bytes = p.msub * Cfg::A_BYTES;
+          mbar_arrive_expect_tx(&full_bar[r], REALIGN_B ? a_bytes : a_bytes + p.panels * Cfg::PANEL_BYTES);
           tma_load_2d(slot, &maps.a[T.s], &full_bar[r], kb * 64, T.q0);
           if (!REALIGN_B) {
             for (int c = 0; c < p.panels; ++c)
-              tma_load_2d(slot + Cfg::A_BYTES + c * Cfg::PANEL_BYTES, &maps.b, &full_bar[r], T.n0 + 64 * c, k_lo);
+              tma_load_2d(slot + a_bytes + c * Cfg::PANEL_BYTES, &maps.b, &full_bar[r], T.n0 + 64 * c, k_lo);
           }
           last_full[r] = static_cast<int>(rph);
           if (++r == p.ring_stages) {
@@ -377,28 +379,32 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
           // each swizzled 128-byte row sits at (row & 7) * 16).
           const uint32_t keep_from = static_cast<uint32_t>(T.e);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 8; ++i) {
             const int row = lane + 32 * i;
-            const uint32_t addr = smem_u32(slot) + row * 128 + ((row & 7) << 4);
-            uint4 v;
-            ld_shared_v4(addr, v);
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            if (i < 4 * p.msub) {
+              const uint32_t addr = smem_u32(slot) + row * 128 + ((row & 7) << 4);
+              uint4 v;
+              ld_shared_v4(addr, v);
+              uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if (static_cast<uint32_t>(e) < keep_from) w[e >> 1] &= (e & 1) ? 0x0000ffffu : 0xffff0000u;
-            st_shared_u4(addr, make_uint4(w[0], w[1], w[2], w[3]));
+              for (int e = 0; e < 8; ++e)
+                if (static_cast<uint32_t>(e) < keep_from) w[e >> 1] &= (e & 1) ? 0x0000ffffu : 0xffff0000u;
+              st_shared_u4(addr, make_uint4(w[0], w[1], w[2], w[3]));
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
         }
         if (lane == 0) {
           const uint32_t a_addr = smem_u32(slot);
-          const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+          const uint32_t b_addr = a_addr + p.msub * Cfg::A_BYTES;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t adesc = make_sw128_desc(a_addr + k * 32, 16, 1024);
             const uint64_t bdesc = make_sw128_desc(b_addr + k * 2048, Cfg::PANEL_BYTES, 1024);
-            umma_f16_ss(d_tmem, adesc, bdesc, p.idesc, (kb != T.kb_lo || k != 0) ? 1u : 0u);
+            for (int u = 0; u < p.msub; ++u) {
+              const uint64_t adesc = make_sw128_desc(a_addr + u * Cfg::A_BYTES + k * 32, 16, 1024);
+              umma_f16_ss(d_tmem + u * 256, adesc, bdesc, p.idesc, (kb != T.kb_lo || k != 0) ? 1u : 0u);
+            }
           }
           umma_commit(&empty_bar[r]);
         }
@@ -558,7 +564,7 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
       const bool got = mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
       if (!__all_sync(0xffffffffu, got)) break;
       // Rows outside [0, K) were loaded as zeros and shift to zeros.
-      const uint32_t dst = smem_u32(ring + r * p.ring_stage_bytes) + Cfg::A_BYTES + dst_off;
+      const uint32_t dst = smem_u32(ring + r * p.ring_stage_bytes) + p.msub * Cfg::A_BYTES + dst_off;
       const uint32_t bits = (f_cur & 1u) * 16u;
       switch (f_cur >> 1) {
         case 0: rc_shift_rows<0>(cur, ext, bits, dst, stores, lane == 31); break;
@@ -582,14 +588,19 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
   }
 
   if (SPLIT) {
-    // Rank q owns the tile's rows [128 q / S, 128 (q + 1) / S).  Once every
-    // CTA of the cluster is done with its ring, each epilogue thread pushes
-    // its row of the fp32 partial into the owner's shared memory, slot
-    // `rank` (remote stores, nothing waits on a round trip); after a second
-    // cluster barrier each owner sums its rows over the slots in rank order,
-    // from its own shared memory, and writes them to C.
+    // The tile has R = 128 msub rows; rank q owns rows [R q / S, R (q + 1) / S).
+    // Once every CTA of the cluster is done with its ring, each epilogue
+    // thread pushes its row of the fp32 partial into the owner's shared
+    // memory, slot `rank` (remote stores, nothing waits on a round trip).  A
+    // slot is laid out by 16-byte column chunk, then row (chunk c4 of slot
+    // row il at (c4 rpo + il) x 16 bytes), so a warp's 32 rows store one
+    // contiguous 512-byte block.  After a second cluster barrier each owner
+    // sums its rows over the slots in rank order, from its own shared
+    // memory, and writes them to C.
     const RcTile T = rc_tile(p, t_first, rank, splits);
-    const int rpo = (128 + splits - 1) / splits;  // slot rows
+    const int R = 128 * p.msub;
+    const int rpo = (R + splits - 1) / splits;  // slot rows
+    const uint32_t slot_bytes = static_cast<uint32_t>(rpo * p.bn * 4);
     const uint32_t part = smem_u32(ring);
     tcgen05_fence_before_sync();
     __syncthreads();
@@ -599,29 +610,32 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
       const int quad = warp & 3;
       const int i = quad * 32 + lane;  // row of the tile = TMEM lane
       const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-      int q = (i * splits) / 128;
-      if ((128 * (q + 1)) / splits <= i) ++q;
-      const int il = i - (128 * q) / splits;
-      const uint32_t dst =
-          mapa_shared(part + static_cast<uint32_t>((rank * rpo + il) * p.c_stride), static_cast<uint32_t>(q));
       const bool has_k = T.kb_hi > T.kb_lo;
-      for (int c = 0; c * 16 < p.bn; ++c) {
-        uint32_t v[16];
-        if (has_k) {
-          tmem_ld_32x32b_x16(lane_base + c * 16, v);
-          tmem_ld_wait();
-        } else {
+      for (int u = 0; u < p.msub; ++u) {
+        const int row = u * 128 + i;  // sub-tile u sits in TMEM columns [256 u, 256 u + bn)
+        int q = (row * splits) / R;
+        if ((R * (q + 1)) / splits <= row) ++q;
+        const int il = row - (R * q) / splits;
+        const uint32_t dst = mapa_shared(part + rank * slot_bytes + static_cast<uint32_t>(il * 16), static_cast<uint32_t>(q));
+        for (int c = 0; c * 16 < p.bn; ++c) {
+          uint32_t v[16];
+          if (has_k) {
+            tmem_ld_32x32b_x16(lane_base + u * 256 + c * 16, v);
+            tmem_ld_wait();
+          } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = 0u;  // empty K share: the partial is zero
+            for (int e = 0; e < 16; ++e) v[e] = 0u;  // empty K share: the partial is zero
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            st_shared_cluster_u4(dst + static_cast<uint32_t>((4 * c + e) * rpo * 16),
+                                 make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          st_shared_cluster_u4(dst + c * 64 + e * 16, make_uint4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
       }
     }
     cluster_sync();
     if (!*abort_flag) {
-      const int r_lo = (128 * rank) / splits, r_hi = (128 * (rank + 1)) / splits;
+      const int r_lo = (R * rank) / splits, r_hi = (R * (rank + 1)) / splits;
       const int nrows = r_hi - r_lo;
       const int ncols = min(p.bn, p.N - T.n0);
       const int segs = (ncols + 63) / 64;
@@ -639,11 +653,11 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
           for (int qr = 0; qr < splits; ++qr) {
-            const uint32_t off = part + static_cast<uint32_t>((qr * rpo + il) * p.c_stride + cc * 4);
+            const uint32_t off = part + qr * slot_bytes + static_cast<uint32_t>(((cc >> 2) * rpo + il) * 16);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
               uint4 x;
-              ld_shared_v4(off + v4 * 16, x);
+              ld_shared_v4(off + static_cast<uint32_t>(v4 * rpo * 16), x);
               acc[4 * v4] += __uint_as_float(x.x);
               acc[4 * v4 + 1] += __uint_as_float(x.y);
               acc[4 * v4 + 2] += __uint_as_float(x.z);

@@ -747,22 +747,66 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   // widened rows; else the eight residue classes of the rows.
   const int e0 = static_cast<int>((reinterpret_cast<uintptr_t>(o.A) & 15u) / 2);
   p.a_classes = (o.lda % 8 == 0 && o.lda >= K + e0) ? 1 : kRcClasses;
-  if (!encode_classes(maps.a, o.A, M, K, o.lda, p.a_classes, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, p.a_shift,
+  const int sms = info->sm_count;
+  const int kb_min = static_cast<int>((K + 63) / 64);
+  p.bn = N <= 240 ? static_cast<int>((N + 15) / 16 * 16) : 256;
+  p.n_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
+  p.panels = (p.bn + 63) / 64;
+  auto tiles_for = [&](int rows) {
+    int t = 0;
+    for (int c = 0; c < p.a_classes; ++c) {
+      const int64_t n = M > c ? (M - c + p.a_classes - 1) / p.a_classes : 0;
+      t += static_cast<int>((n + rows - 1) / rows);
+    }
+    return t * p.n_tiles;
+  };
+  constexpr int kSmemMax = 232448, kFixed = 1024 + 512;
+  auto ring_for = [&](int msub, int* stages, int* stage_bytes) {
+    *stage_bytes = msub * RcCfg<false>::A_BYTES + p.panels * RcCfg<false>::PANEL_BYTES;
+    int r = (kSmemMax - kFixed) / *stage_bytes;
+    *stages = r > RcCfg<false>::MAX_RING ? RcCfg<false>::MAX_RING : r;
+  };
+  // Few tiles: split K over a cluster of S CTAs (each keeps at least 4
+  // k-blocks), when the cluster's partials of one tile's rows (S slots of
+  // ceil(R / S) rows) fit in the ring.  For one column of narrow tiles (A
+  // streams from memory) a tile takes 2 x 128 class rows, two accumulators
+  // sharing each B stage, when that still splits.
+  auto splits_for = [&](int tiles, int msub) {
+    int st, sb;
+    ring_for(msub, &st, &sb);
+    if (st < 2 || 2 * tiles > sms) return 1;
+    int s = sms / tiles;
+    s = s > 8 ? 8 : s;
+    while (s > 1 && kb_min / s < 4) --s;
+    s = tune_int("TG_TUNE_RC_SPLITS", s);
+    if (s > 8) s = 8;
+    const int R = 128 * msub;
+    while (s > 1 && s * ((R + s - 1) / s) * p.bn * 4 > st * sb) --s;
+    return s;
+  };
+  int msub = 1;
+  int splits = splits_for(tiles_for(128), 1);
+  if (splits > 1 && p.bn <= 240 && tiles_for(256) < tiles_for(128) && tune_int("TG_TUNE_RC_MSUB2", 1)) {
+    const int s2 = splits_for(tiles_for(256), 2);
+    if (s2 > 1) {
+      msub = 2;
+      splits = s2;
+    }
+  }
+  p.msub = msub;
+  if (!encode_classes(maps.a, o.A, M, K, o.lda, p.a_classes, 64, 128 * msub, CU_TENSOR_MAP_SWIZZLE_128B, p.a_shift,
                       p.rows_in_class))
     return TG_ERR_LAUNCH;
   int mt = 0, kb_max = 0;
   for (int c = 0; c < p.a_classes; ++c) {
     p.tile_start[c] = mt;
-    mt += (p.rows_in_class[c] + 127) / 128;
+    mt += (p.rows_in_class[c] + 128 * msub - 1) / (128 * msub);
     const int kb = static_cast<int>((K + p.a_shift[c] + 63) / 64);
     kb_max = kb > kb_max ? kb : kb_max;
   }
   p.tile_start[p.a_classes] = mt;
   p.m_tiles = mt;
-  p.bn = N <= 240 ? static_cast<int>((N + 15) / 16 * 16) : 256;
-  p.n_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
   p.num_tiles = p.m_tiles * p.n_tiles;
-  p.panels = (p.bn + 63) / 64;
   p.group_m = tune_int("TG_TUNE_RC_GROUP_M", 8);
   if (p.group_m < 1) p.group_m = 1;
   const bool stage_b = !((reinterpret_cast<uintptr_t>(o.B) & 15u) == 0 && o.ldb % 8 == 0);
@@ -771,30 +815,13 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   if (!stage_b && !encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
     return TG_ERR_LAUNCH;
   }
-  p.ring_stage_bytes = RcCfg<false>::A_BYTES + p.panels * RcCfg<false>::PANEL_BYTES;
-  constexpr int kSmemMax = 232448, kFixed = 1024 + 512;
-  int ring = (kSmemMax - kFixed) / p.ring_stage_bytes;
-  ring = ring > RcCfg<false>::MAX_RING ? RcCfg<false>::MAX_RING : ring;
+  int ring = 0;
+  ring_for(msub, &ring, &p.ring_stage_bytes);
   if (ring < 2) return TG_ERR_INTERNAL;
   p.ring_stages = ring;
-  p.c_stride = p.bn * 4 + 16;
   p.idesc = make_idesc_f16_f32(128, p.bn, false, true);
   p.wait_budget_ns = wait_budget(kb_max);
   const int smem = kFixed + ring * p.ring_stage_bytes;
-  // Few tiles: split K over a cluster (each CTA keeps at least 4 k-blocks),
-  // when the cluster's partials of one CTA's rows (S slots of ceil(128 / S)
-  // rows) fit in the ring.
-  const int sms = info->sm_count;
-  int splits = 1;
-  if (2 * p.num_tiles <= sms) {
-    splits = sms / p.num_tiles;
-    const int kb_min = static_cast<int>((K + 63) / 64);
-    splits = splits > 8 ? 8 : splits;
-    while (splits > 1 && kb_min / splits < 4) --splits;
-    splits = tune_int("TG_TUNE_RC_SPLITS", splits);
-    if (splits > 8) splits = 8;
-    while (splits > 1 && splits * ((128 + splits - 1) / splits) * p.c_stride > ring * p.ring_stage_bytes) --splits;
-  }
   p.splits = splits;
   if (splits > 1) {
     if (p.num_tiles > 65535) return TG_ERR_INVALID_ARG;
