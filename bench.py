@@ -713,18 +713,24 @@ def measure_configs(tg, torch, dev, stream, args, peaks, peak_src):
             continue
         M, N, K, A, B = config_problem(workload, idx, dist)
         case = Fp16Case(tg, torch, dev, stream, M, N, K, A, B, mode=mode)
+        # Short kernels get more steps than the headline: at least 20 ms of
+        # warm-up (clocks settle after the set-up between records) and 10 ms
+        # of timed steps, so a record is not one launch's jitter.
         case.warm(args.warmup)
-        ms, clocks = case.time(args.steps)
+        est_ms, _ = case.time(max(3, args.warmup))
+        steps = min(4000, max(args.steps, math.ceil(10.0 / max(est_ms, 1e-3))))
+        case.warm(min(4000, max(args.warmup, math.ceil(20.0 / max(est_ms, 1e-3)))))
+        ms, clocks = case.time(steps)
         spec = f"skinny:{M}" if workload == "skinny" else workload + (f":{idx}" if idx is not None else "")
         rec = {"config": label, "workload": spec,
                "M": M, "N": N, "K": K, "values": dist or inputs.WORKLOADS[workload].dist,
                "seed": inputs.WORKLOADS[workload].seed,
                "entry_point": "tg_gemm_relu_f16" if case.ws_bytes == 0 else "tg_gemm_relu_f16_ws",
                "path": tg.path_name(case.chosen), "workspace_bytes": case.ws_bytes, "l2": case.l2_note,
-               "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+               "steps": steps, "warmup": args.warmup, "ms_per_step": ms,
                "value": inputs.flops(M, N, K) / (ms * 1e-3) / 1e12, "unit": UNIT,
                "roofline": roofline_for(M, N, K, ms, peaks, peak_src),
-               "gpu_launches": args.steps * case.launches_per_step, "clocks": clocks}
+               "gpu_launches": steps * case.launches_per_step, "clocks": clocks}
         # A profile is keyed by path, and by "_ws" when a workspace changes what the path runs.
         key = tg.path_name(case.chosen) + ("_ws" if case.ws_bytes > 0 and case.chosen == tg.Path.RC else "")
         rec["roofline"]["traffic"] = committed_traffic(key, spec)
