@@ -81,7 +81,7 @@ def parse_args():
     ap.add_argument("--workspace", choices=["auto", "none"], default="auto",
                     help="auto: give the library the scratch bytes it asks for (repack path for "
                          "operands TMA cannot describe), allocated by torch outside the timed region")
-    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--configs", default="all",
@@ -515,6 +515,33 @@ def host_link(dev, h2d_bytes: int, d2h_bytes: int, reps: int = 3):
             best = ms if best is None else min(best, ms)
         out[name + "_gbs"] = n / (best * 1e-3) / 1e9
         del host, devb
+    # Both directions at once, as an e2e step runs them (upload on one copy
+    # engine, download on the other): their shared link can be slower than
+    # either alone.
+    hin = torch.empty(max(1, h2d_bytes), dtype=torch.uint8).pin_memory()
+    hout = torch.empty(max(1, d2h_bytes), dtype=torch.uint8).pin_memory()
+    din = torch.empty(max(1, h2d_bytes), dtype=torch.uint8, device=dev)
+    dout = torch.empty(max(1, d2h_bytes), dtype=torch.uint8, device=dev)
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    best = None
+    for _ in range(reps):
+        torch.cuda.synchronize(dev)
+        ev0 = torch.cuda.Event(enable_timing=True)
+        e_up, e_down = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        s_up.wait_event(ev0)
+        s_down.wait_event(ev0)
+        with torch.cuda.stream(s_up):
+            din.copy_(hin, non_blocking=True)
+            e_up.record(s_up)
+        with torch.cuda.stream(s_down):
+            hout.copy_(dout, non_blocking=True)
+            e_down.record(s_down)
+        torch.cuda.synchronize(dev)
+        ms = max(ev0.elapsed_time(e_up), ev0.elapsed_time(e_down))
+        best = ms if best is None else min(best, ms)
+    out["both_ms"] = best
+    del hin, hout, din, dout
     return out
 
 
@@ -802,7 +829,7 @@ def run_ours(args):
         e2e_ms = max_over_ranks(dist, e2e_ms, dev)
     h2d, d2h = 2 * (Mr * K + K * N), 2 * Mr * N
     link = host_link(dev, h2d, d2h)
-    floor_ms = max(h2d / (link["h2d_gbs"] * 1e9), d2h / (link["d2h_gbs"] * 1e9)) * 1e3
+    floor_ms = max(h2d / (link["h2d_gbs"] * 1e9) * 1e3, d2h / (link["d2h_gbs"] * 1e9) * 1e3, link["both_ms"])
 
     peaks, peak_src = load_peaks()
     roof = roofline_for(Mr, N, K, kern_ms, peaks, peak_src)
@@ -827,8 +854,9 @@ def run_ours(args):
         "e2e": {"value": flops_total / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "mode": E2E_MODE,
                 "host_link": {**link, "copy_floor_ms": floor_ms, "e2e_over_floor": e2e_ms / floor_ms,
-                              "note": "floor = the larger of the upload and the download at the measured "
-                                      "pinned-copy rates (they run on separate copy engines)"}},
+                              "note": "floor = the longest of the upload alone, the download alone and both "
+                                      "at once on two streams (separate copy engines sharing the link), "
+                                      "measured with pinned host buffers of the step's sizes"}},
         "gpu_launches": args.steps * case.launches_per_step,
         "clocks": clocks,
     }
