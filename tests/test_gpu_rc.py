@@ -46,9 +46,10 @@ def test_rc_short_k(M, N, K):
 
 
 @pytest.mark.parametrize("offsets", [(1, 0, 0), (0, 3, 0), (0, 0, 5), (7, 6, 1), (2, 4, 6), (3, 3, 3)])
-@pytest.mark.parametrize("M,N,K", [(131, 264, 200), (300, 257, 129), (77, 136, 1000)])
+@pytest.mark.parametrize("M,N,K", [(131, 264, 200), (300, 257, 129), (77, 136, 1000), (2000, 72, 2048)])
 def test_rc_unaligned_bases(offsets, M, N, K):
-    """Bases 2, 4, ..., 14 bytes past a 16-byte boundary, per operand: every class shift of A and B."""
+    """Bases 2, 4, ..., 14 bytes past a 16-byte boundary, per operand: every class shift of A and B.
+    (2000, 72, 2048) takes 256-row tiles with K split over a cluster."""
     A, B = inputs.operands(M, N, K, "int", seed=sum(offsets) + M)
     got, guards = run_gpu(A, B, RC, offsets=offsets)
     assert guards
@@ -83,7 +84,7 @@ def test_rc_on_aligned_operands(M, N, K):
     assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"rc aligned {(M, N, K)}")
 
 
-@pytest.mark.parametrize("M,N,K,a_off", [(64, 136, 77, 3), (200, 129, 1021, 1), (1000, 16, 5003, 7)])
+@pytest.mark.parametrize("M,N,K,a_off", [(64, 136, 77, 3), (200, 129, 1021, 1), (1000, 16, 5003, 7), (2000, 129, 1021, 5)])
 def test_rc_infinities_do_not_leak_into_the_next_row(M, N, K, a_off):
     """The first k-block of a class holds, before k = 0, the previous row's last values (or the bytes
     just before A).  Those sit next to infinities here and NaN patterns fill the bytes before A; the
@@ -117,7 +118,7 @@ def test_rc_infinities_do_not_leak_into_the_next_row(M, N, K, a_off):
 
 @pytest.mark.parametrize("bias", [False, True], ids=["nobias", "bias"])
 @pytest.mark.parametrize("strides", ["odd", "padded8"])
-@pytest.mark.parametrize("M,N,K", [(300, 264, 136), (517, 1000, 333), (1000, 129, 2000)])
+@pytest.mark.parametrize("M,N,K", [(300, 264, 136), (517, 1000, 333), (1000, 129, 2000), (2000, 136, 2000)])
 def test_rc_strides_bias_batches(M, N, K, strides, bias):
     from test_gpu_layouts import STRIDES, run_ex
     lda, ldb, ldc = STRIDES[strides](M, N, K, False)
