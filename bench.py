@@ -15,8 +15,11 @@ Multi-GPU (torchrun, one process per GPU): by default one problem's M rows are
 split over the ranks, rank r taking rows [floor(rM/G), floor((r+1)M/G)) with B
 replicated, each rank running the unchanged kernel on its row block (strong
 scaling, no collective in the timed step; C is stitched afterwards by an NCCL
-all-gather, which --gather-c also times).  --parallel replicas gives every
-rank its own independent problem instead (weak scaling).  The timed region is
+all-gather, which --gather-c also times).  --parallel cols splits N instead:
+rank r keeps the column block [c_r, c_{r+1}) of B (boundaries floor(rN/G)
+rounded down to a multiple of 8) with A replicated, and C's column blocks are
+stitched the same way.  --parallel replicas gives every rank its own
+independent problem instead (weak scaling).  The timed region is
 bracketed by barriers and the slowest rank's time is reported.
 """
 from __future__ import annotations
@@ -93,11 +96,12 @@ def parse_args():
                     help="target CPU work of each configuration's oracle sample")
     ap.add_argument("--sustained-seconds", type=float, default=2.0,
                     help="at N=1, also run the headline kernel back to back this long (0: skip)")
-    ap.add_argument("--parallel", choices=["rows", "replicas"], default="rows",
+    ap.add_argument("--parallel", choices=["rows", "cols", "replicas"], default="rows",
                     help="N>1: rows = split one problem's M rows over the ranks with B replicated "
-                         "(strong scaling); replicas = every rank runs its own problem (weak scaling)")
+                         "(strong scaling); cols = split its N columns with A replicated (strong scaling); "
+                         "replicas = every rank runs its own problem (weak scaling)")
     ap.add_argument("--gather-c", action="store_true",
-                    help="rows mode: also time the NCCL all-gather that stitches C on every rank")
+                    help="rows or cols mode: also time the NCCL all-gather that stitches C on every rank")
     ap.add_argument("--cublas", action="store_true",
                     help="also time torch.relu(torch.matmul(A, B)) (cuBLAS) on the same operands, as context")
     return ap.parse_args()
@@ -446,6 +450,30 @@ def row_range(M: int, world: int, rank: int):
     return (rank * M) // world, ((rank + 1) * M) // world
 
 
+def col_range(N: int, world: int, rank: int):
+    """Columns [c0, c1) of C (and of B) that rank `rank` of `world` computes: the boundaries
+    floor(r*N/G) rounded down to a multiple of 8 (so every block of a row-major B or C starts on a
+    16-byte boundary), the last one N."""
+    def bound(r):
+        return N if r >= world else ((r * N // world) // 8) * 8
+    return bound(rank), bound(rank + 1)
+
+
+def gather_cols(dist, block, N: int, world: int, rank: int):
+    """All-gather every rank's column block of C (M x (c1 - c0), row-major) into the full M x N C.
+    Blocks are padded to the widest so the collective moves equal sizes; the padding is dropped
+    when stitching.  Works on CPU tensors (gloo) and CUDA tensors (NCCL)."""
+    import torch
+    cols = [col_range(N, world, r) for r in range(world)]
+    widest = max(c1 - c0 for c0, c1 in cols)
+    M = block.shape[0]
+    padded = torch.zeros((M, widest), dtype=block.dtype, device=block.device)
+    padded[:, : block.shape[1]].copy_(block)
+    parts = [torch.empty_like(padded) for _ in range(world)]
+    dist.all_gather(parts, padded)
+    return torch.cat([parts[r][:, : c1 - c0] for r, (c0, c1) in enumerate(cols)], dim=1)
+
+
 def gather_rows(dist, block, M: int, world: int, rank: int):
     """All-gather every rank's row block of C into the full M x N C (row-major, rank order).
 
@@ -781,16 +809,24 @@ def run_ours(args):
     path = {"auto": tg.Path.AUTO, "tc": tg.Path.TC, "tc_edge": tg.Path.TC_EDGE, "skinny": tg.Path.SKINNY,
             "tc_pair": tg.Path.TC_PAIR, "tc_pair512": tg.Path.TC_PAIR512, "rc": tg.Path.RC}[args.path]
     rows_mode = world > 1 and args.parallel == "rows"
+    cols_mode = world > 1 and args.parallel == "cols"
+    split = rows_mode or cols_mode
     # Row partition: every rank draws the workload itself (same seed) and keeps its rows of A; B is
-    # replicated.  Replicas: every rank runs its own independent problem.
-    name, M, N, K, A, B = workload_problem(args.workload, 0 if rows_mode else rank)
+    # replicated.  Column partition: it keeps its column block of B; A is replicated.  Replicas:
+    # every rank runs its own independent problem.
+    name, M, N_full, K, A, B = workload_problem(args.workload, 0 if split else rank)
     linear = name == "linear8192"
     bias = None
     if linear:
         B, bias = B
+        if cols_mode:
+            raise SystemExit("--parallel cols: the linear workload stores its weight N x K; split rows instead")
     r0, r1 = row_range(M, world, rank) if rows_mode else (0, M)
-    Mr = r1 - r0
+    c0, c1 = col_range(N_full, world, rank) if cols_mode else (0, N_full)
+    Mr, N = r1 - r0, c1 - c0
     A_r = np.ascontiguousarray(A[r0:r1])
+    if cols_mode:
+        B = np.ascontiguousarray(B[:, c0:c1])
     stream = torch.cuda.Stream(dev)
     mode = "linear" if linear else ("none" if args.workspace == "none" else "auto")
     case = Fp16Case(tg, torch, dev, stream, Mr, N, K, A_r, B, mode=mode,
@@ -799,22 +835,23 @@ def run_ours(args):
     kern_ms, clocks = case.time(args.steps, dist)
     step_ms = max_over_ranks(dist, kern_ms, dev) if dist is not None else kern_ms
     flops_rank = inputs.flops(Mr, N, K)
-    flops_total = inputs.flops(M, N, K) if rows_mode else world * flops_rank
+    flops_total = inputs.flops(M, N_full, K) if split else world * flops_rank
     value = flops_total / (step_ms * 1e-3) / 1e12
 
     gather = None
-    if rows_mode:
+    if split:
         # Stitch C once (outside the timed region) so every rank holds the full result; with
         # --gather-c the all-gather is also timed on its own over the same steps.
         c_block = case.sets[0][2]
-        full = gather_rows(dist, c_block, M, world, rank)
-        assert full.shape == (M, N)
+        stitch = ((lambda: gather_rows(dist, c_block, M, world, rank)) if rows_mode else
+                  (lambda: gather_cols(dist, c_block, N_full, world, rank)))
+        full = stitch()
+        assert full.shape == (M, N_full)
         gather = {"stitched": True}
         if args.gather_c:
             with torch.cuda.stream(stream):
-                gather_rows(dist, c_block, M, world, rank)
-            g_ms, _ = timed_region(torch, dev, stream, lambda: gather_rows(dist, c_block, M, world, rank),
-                                   args.steps, None, dist)
+                stitch()
+            g_ms, _ = timed_region(torch, dev, stream, stitch, args.steps, None, dist)
             gather["all_gather_ms"] = max_over_ranks(dist, g_ms, dev)
             gather["step_ms_with_gather"] = step_ms + gather["all_gather_ms"]
         del full
@@ -837,6 +874,10 @@ def run_ours(args):
     if rows_mode:
         parallelism = (f"rows{world}: rank r computes rows [floor(rM/{world}), floor((r+1)M/{world})) of one "
                        f"{M}x{N}x{K} problem with B replicated; C stitched by an NCCL all-gather")
+    elif cols_mode:
+        parallelism = (f"cols{world}: rank r computes the columns [8 floor(floor(rN/{world})/8), ...) of one "
+                       f"{M}x{N_full}x{K} problem, holding only its column block of B, with A replicated; "
+                       f"C stitched by an NCCL all-gather")
     elif world > 1:
         parallelism = f"dp{world} independent problems"
     else:
@@ -844,12 +885,14 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-        "scaling": "strong" if rows_mode else "weak",
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None, "dtype": "f16 (fp32 accumulate)", "data": "synthetic",
-        "config": {**describe(name, M, N, K), "path": tg.path_name(case.chosen), "workspace_bytes": case.ws_bytes,
-                   "l2": case.l2_note, "parallelism": parallelism,
+        "config": {**describe(name, M, N_full, K), "path": tg.path_name(case.chosen),
+                   "workspace_bytes": case.ws_bytes, "l2": case.l2_note, "parallelism": parallelism,
                    **({"rows_per_rank": [row_range(M, world, r)[1] - row_range(M, world, r)[0]
-                                         for r in range(world)]} if rows_mode else {})},
+                                         for r in range(world)]} if rows_mode else {}),
+                   **({"cols_per_rank": [col_range(N_full, world, r)[1] - col_range(N_full, world, r)[0]
+                                         for r in range(world)]} if cols_mode else {})},
         "roofline": roof,
         "e2e": {"value": flops_total / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "mode": E2E_MODE,

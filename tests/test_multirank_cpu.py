@@ -1,8 +1,12 @@
 """The multi-rank plumbing of bench.py, on CPU with the gloo backend (world size 2).
 
-With N GPUs every rank runs its own independent problem (weak scaling, no
-data-path collective); the only collectives are the barriers around the timed
-region and the max-reduction of the per-rank step times.
+bench.py --gpus N splits one problem over the ranks: by rows of A (B
+replicated, the default) or by column blocks of B (A replicated), and stitches
+C with an all-gather; --parallel replicas gives every rank its own problem.
+These tests check the partitions tile the problem exactly, that the stitched C
+equals the oracle's full result (each rank computes its block with the oracle
+as a stand-in for its GPU kernel, in the test only), the max-reduction of the
+per-rank step times, and the per-rank seeds of the replicas.
 """
 import os
 import socket
@@ -129,4 +133,63 @@ def test_two_gloo_ranks_split_rows_and_stitch_c():
     assert [(r0, r1) for _, r0, r1, _ in results] == [(0, 18), (18, 37)]
     for _, _, _, full in results:                          # every rank holds the whole, stitched C
         assert full.shape == (37, 24)
+        assert np.array_equal(full, want)
+
+
+def test_col_ranges_tile_n_exactly_on_16_byte_boundaries():
+    import bench
+    for N in (1, 8, 9, 24, 43, 129, 5003, 8192, 12289):
+        for world in (1, 2, 3, 4, 8):
+            ranges = [bench.col_range(N, world, r) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == N
+            assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+            assert all(c0 % 8 == 0 and c1 >= c0 for c0, c1 in ranges)
+
+
+def _cols_worker(rank, world, port, out):
+    import datetime
+    import sys
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import oracle
+    from tiled_dense_gemm_fp16_b200 import inputs
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        M, N, K = 37, 43, 40                               # odd N: blocks of 16 and 27 columns
+        A, B = inputs.operands(M, N, K, "int", seed=12)    # every rank draws the same problem
+        c0, c1 = bench.col_range(N, world, rank)
+        # Stand-in for the rank's GPU kernel (this test only): the oracle on the rank's columns of B.
+        block = oracle.gemm_relu_f16(A, np.ascontiguousarray(B[:, c0:c1]))
+        full = bench.gather_cols(dist, torch.from_numpy(block), N, world, rank)
+        out.put((rank, c0, c1, full.numpy().view(np.uint16).copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_columns_and_stitch_c():
+    import numpy as np
+
+    import oracle
+    from tiled_dense_gemm_fp16_b200 import inputs
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cols_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted((out.get(timeout=120) for _ in procs), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    A, B = inputs.operands(37, 43, 40, "int", seed=12)
+    want = oracle.gemm_relu_f16(A, B).view(np.uint16)
+    assert [(c0, c1) for _, c0, c1, _ in results] == [(0, 16), (16, 43)]
+    for _, _, _, full in results:                          # every rank holds the whole, stitched C
+        assert full.shape == (37, 43)
         assert np.array_equal(full, want)
