@@ -25,6 +25,7 @@ SHAPES = [
     (1, 1, 8), (1, 8, 1), (3, 9, 8), (7, 17, 9), (8, 8, 8), (9, 129, 63), (15, 240, 64), (16, 241, 65),
     (17, 256, 127), (63, 257, 128), (127, 513, 199), (128, 255, 8), (129, 16, 1021), (200, 136, 72),
     (257, 777, 300), (300, 301, 299), (640, 520, 75), (1000, 1001, 1003), (1025, 129, 2049),
+    (2000, 3000, 300),  # enough tiles for a full wave: 176-wide tiles (the width is chosen per wave count)
 ]
 
 

@@ -750,6 +750,30 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   const int sms = info->sm_count;
   const int kb_min = static_cast<int>((K + 63) / 64);
   p.bn = N <= 240 ? static_cast<int>((N + 15) / 16 * 16) : 256;
+  {
+    // The persistent CTAs take the tiles in waves.  When 256-wide tiles fill
+    // at least one wave, pick the width w (a multiple of 16, 128..256) with
+    // the least waves x bytes per k-block (16 KiB of A and 128 w of B: the
+    // kernel moves operands rather than multiplies), so that the last wave is
+    // not mostly idle; ties go to the wider tile.
+    int64_t m128 = 0;
+    for (int c = 0; c < p.a_classes; ++c) {
+      const int64_t n = M > c ? (M - c + p.a_classes - 1) / p.a_classes : 0;
+      m128 += (n + 127) / 128;
+    }
+    if (N > 240 && m128 * ((N + 255) / 256) >= sms) {
+      int64_t best = -1;
+      for (int w = 256; w >= 128; w -= 16) {
+        const int64_t cost = (m128 * ((N + w - 1) / w) + sms - 1) / sms * (16384 + 128 * w);
+        if (best < 0 || cost < best) {
+          best = cost;
+          p.bn = w;
+        }
+      }
+    }
+    p.bn = tune_int("TG_TUNE_RC_BN", p.bn);
+    if (p.bn < 16 || p.bn > 256 || p.bn % 16 != 0) return TG_ERR_INVALID_ARG;
+  }
   p.n_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
   p.panels = (p.bn + 63) / 64;
   auto tiles_for = [&](int rows) {
