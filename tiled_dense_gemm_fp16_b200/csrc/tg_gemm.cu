@@ -699,11 +699,11 @@ bool encode_classes(CUtensorMap* maps, const void* base, int64_t rows, int64_t c
   return true;
 }
 
-template <bool STAGE_B, bool SPLIT>
+template <bool REALIGN_B, bool SPLIT>
 tg_status launch_rc_cfg(const RcMaps& maps, const RcParams& p, int smem, int grid_x, int grid_y,
                         cudaStream_t stream, DeviceInfo* info) {
-  auto kernel = gemm_relu_rc_kernel<STAGE_B, SPLIT>;
-  constexpr unsigned kBit = 1u << ((STAGE_B ? 1 : 0) + (SPLIT ? 2 : 0));
+  auto kernel = gemm_relu_rc_kernel<REALIGN_B, SPLIT>;
+  constexpr unsigned kBit = 1u << ((REALIGN_B ? 1 : 0) + (SPLIT ? 2 : 0));
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!(info->rc_attr & kBit)) {
@@ -717,7 +717,7 @@ tg_status launch_rc_cfg(const RcMaps& maps, const RcParams& p, int smem, int gri
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   cfg.gridDim = dim3(static_cast<unsigned>(grid_x), static_cast<unsigned>(grid_y), 1);
-  cfg.blockDim = dim3(RcCfg<STAGE_B>::THREADS, 1, 1);
+  cfg.blockDim = dim3(RcCfg<REALIGN_B>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   LaunchAttrs la;
@@ -729,8 +729,8 @@ tg_status launch_rc_cfg(const RcMaps& maps, const RcParams& p, int smem, int gri
   return TG_OK;
 }
 
-// Residue-class path: see gemm_rc.cuh.  B's rows are realigned in shared
-// memory (staging mode) when TMA cannot describe B.
+// Residue-class path: see gemm_rc.cuh.  When TMA cannot describe B, the
+// kernel's realigning warps read B's rows in place.
 tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   const int64_t M = o.M, N = o.N, K = o.K;
   RcMaps maps;
@@ -833,10 +833,10 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.group_m = tune_int("TG_TUNE_RC_GROUP_M", 8);
   if (p.group_m < 1) p.group_m = 1;
-  const bool stage_b = !((reinterpret_cast<uintptr_t>(o.B) & 15u) == 0 && o.ldb % 8 == 0);
+  const bool realign_b = !((reinterpret_cast<uintptr_t>(o.B) & 15u) == 0 && o.ldb % 8 == 0);
   p.B = static_cast<const __half*>(o.B);
   p.ldb = o.ldb;
-  if (!stage_b && !encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
+  if (!realign_b && !encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
     return TG_ERR_LAUNCH;
   }
   int ring = 0;
@@ -849,11 +849,11 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   p.splits = splits;
   if (splits > 1) {
     if (p.num_tiles > 65535) return TG_ERR_INVALID_ARG;
-    return stage_b ? launch_rc_cfg<true, true>(maps, p, smem, splits, p.num_tiles, stream, info)
+    return realign_b ? launch_rc_cfg<true, true>(maps, p, smem, splits, p.num_tiles, stream, info)
                    : launch_rc_cfg<false, true>(maps, p, smem, splits, p.num_tiles, stream, info);
   }
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  return stage_b ? launch_rc_cfg<true, false>(maps, p, smem, grid, 1, stream, info)
+  return realign_b ? launch_rc_cfg<true, false>(maps, p, smem, grid, 1, stream, info)
                  : launch_rc_cfg<false, false>(maps, p, smem, grid, 1, stream, info);
 }
 
