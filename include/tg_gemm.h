@@ -85,9 +85,10 @@ typedef enum tg_path {
     TG_PATH_RC = 9       /* no scratch, any 2-byte alignment of A, B and C:
                             A's rows are loaded by TMA in residue classes
                             (row mod 8, rows sharing one 16-byte offset),
-                            B's k-rows shifted to match; B realigned in
-                            shared memory when TMA cannot describe it;
-                            A stored M x K, B stored K x N only             */
+                            B's k-rows shifted to match; B's rows read in
+                            place and realigned into the operand tile when
+                            TMA cannot describe them; A stored M x K,
+                            B stored K x N only                              */
 } tg_path;
 
 /*
