@@ -253,7 +253,8 @@ TG_API int tg_select_path_ws(const void *A, const void *B, const void *C, int64_
  * The path tg_gemm_relu_f16 would take for these arguments (a tg_path value;
  * TG_PATH_NONE for an empty C), or -2 when the arguments are invalid.  Host
  * logic only: makes no CUDA call and needs no GPU.  Rules: K == 0 -> ZERO;
- * A or B rows not 16-byte aligned -> TC_EDGE; M <= 256 -> SKINNY; otherwise the
+ * A or B rows not TMA-describable (strides or bases off 16 bytes) -> RC;
+ * M <= 128, or M <= 256 with N * K >= 2^23 -> SKINNY; otherwise the
  * tensor-core kernel (TC, TC_PAIR or TC_PAIR512) with the least estimated
  * time from its tile count in waves of a 148-SM device.
  */

@@ -83,9 +83,13 @@ def test_path_selection():
     assert tg.select_path(A0, B0, C0, 300, 264, 64) == Path.TC_PAIR       # 4 pair tiles vs 2 wide ones
     assert tg.select_path(A0, B0, C0, 20000, 256, 64) == Path.TC_PAIR
     assert tg.select_path(A0, B0, C0, 384, 10240, 64) == Path.TC          # 120 CTA tiles fit one wave
-    # Small M with aligned rows: the split-K small-M kernel.
+    # Small M with aligned rows: the split-K small-M kernel; above M = 128 only for a large B.
     for M in (1, 16, 64, 256):
         assert tg.select_path(A0, B0, C0, M, 8192, 8192) == Path.SKINNY
+    assert tg.select_path(A0, B0, C0, 128, 256, 256) == Path.SKINNY
+    assert tg.select_path(A0, B0, C0, 256, 4096, 4096) == Path.SKINNY
+    assert tg.select_path(A0, B0, C0, 256, 256, 256) == Path.TC_PAIR
+    assert tg.select_path(A0, B0, C0, 256, 2048, 2048) == Path.TC_PAIR
     assert tg.select_path(A0, B0, C0, 257, 8192, 8192) == Path.TC_PAIR
     assert tg.select_path(A0, B0, C0, 64, 8191, 8192) == Path.RC
     # Row strides that are not 16-byte multiples, or misaligned bases, need the edge mode.
@@ -202,8 +206,10 @@ def test_padded_c_with_general_layouts():
     # Strided batches: one padded C serves every entry in turn.
     o = tg.options(b_layout=tg.B_NK, batch=3, stride_a=M * K, stride_b=N * K, stride_c=M * N + 3)
     assert tg.workspace_size_ex(A0, B0, C0, M, N, K, o) == up(2 * M * 1008)
-    # Small M keeps the small-M kernel, which writes C element by element anyway.
-    assert tg.workspace_size_ex(A0, B0, C0, 200, N, K, tg.options(b_layout=tg.B_NK)) == 0
+    # Small M keeps the small-M kernel, which writes C element by element anyway; M = 200 with this
+    # small B takes the tile kernels, which ask for the padded C.
+    assert tg.workspace_size_ex(A0, B0, C0, 100, N, K, tg.options(b_layout=tg.B_NK)) == 0
+    assert tg.workspace_size_ex(A0, B0, C0, 200, N, K, tg.options(b_layout=tg.B_NK)) == up(2 * 200 * 1008)
 
 
 def test_workspace_argument_checks():

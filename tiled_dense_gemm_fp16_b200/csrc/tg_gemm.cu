@@ -214,11 +214,22 @@ bool c_rows_aligned(const Problem& p) {
   return (reinterpret_cast<uintptr_t>(p.C) & 15u) == 0 && p.ldc % 8 == 0 && (p.batch == 1 || p.sc % 8 == 0);
 }
 
+// The small-M kernel (A stored M x K) for M <= 128, where two CTAs share an
+// SM and the split-K partials are small; for 128 < M <= 256 only when B is
+// large (N x K >= 2^23), since the partials (M x 128 fp32 per CTA) then cost
+// less than the tile kernels' few waves.  Measured, µs (small-M vs best tile
+// kernel): 256 x 256 x 256 10.5 / 7.2, 256 x 2048 x 2048 23.8 / 16.9,
+// 256 x 4096 x 4096 18.4 / 27.4; at M <= 128 the small-M kernel wins down to
+// 64 x 512 x 512 (6.1 / 7.5).
+bool skinny_route(const Problem& p) {
+  return p.M <= kSkinnyMaxM && !p.a_km && (p.M <= 128 || p.N * p.K >= (int64_t(1) << 23));
+}
+
 // The tensor-core kernels store C fastest when its rows start on 16-byte
 // boundaries (whole 16-byte pieces, or TMA boxes); the small-M kernel writes
 // C element by element either way.
 bool c_pad_useful(const Problem& p) {
-  return !c_rows_aligned(p) && !(p.M <= kSkinnyMaxM && !p.a_km);
+  return !c_rows_aligned(p) && !skinny_route(p);
 }
 
 // Workspace of the repack path: zero-padded copies (rows rounded up to 8
@@ -317,8 +328,7 @@ int pick_tc_kernel(int64_t M, int64_t N, int64_t K, bool c_aligned) {
 
 // The tensor-core kernel that runs on TMA-describable (possibly repacked) operands.
 int inner_path(const Problem& p, bool c_padded = false) {
-  return (p.M <= kSkinnyMaxM && !p.a_km) ? TG_PATH_SKINNY
-                                         : pick_tc_kernel(p.M, p.N, p.K, c_padded || c_rows_aligned(p));
+  return skinny_route(p) ? TG_PATH_SKINNY : pick_tc_kernel(p.M, p.N, p.K, c_padded || c_rows_aligned(p));
 }
 
 // The path a call takes with `ws_bytes` of workspace (-2: invalid arguments).
