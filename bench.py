@@ -216,11 +216,19 @@ class ClockSampler:
 # ncu traffic figure (committed summary), valid only for unchanged sources
 # ---------------------------------------------------------------------------
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines, so that a comment edit leaves the hash alone."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", line).rstrip() for line in text.splitlines())
+    return "\n".join(line for line in lines if line.strip())
+
+
 def kernel_source_sha(path_name: str):
+    """Hash of the code (comments and blank lines dropped) of the sources a path's kernels come from."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES.get(path_name, []):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -15,7 +15,8 @@
 // class (base rounded down to 16 bytes, inner extent K + e_s) then loads a
 // class's rows with 128-byte swizzle straight into the MMA's K-major layout,
 // each row shifted by the same e_s elements: map column x holds A[r][x - e_s].
-// Every output tile takes its 128 rows from one class, and the k-block kb
+// Every output tile takes its rows (128, or 256 in split mode) from one
+// class, and the k-block kb
 // loads map columns [64 kb, 64 kb + 64), that is A[r][64 kb - e_s + j].  The
 // shift is undone on the other operand: the B tile of the same k-block holds
 // the k-rows 64 kb - e_s + j, which is a row offset of B, and TMA takes any
@@ -39,9 +40,11 @@
 // written element by element.
 //
 // Shapes with few tiles (one narrow column of tiles, N <= 240 say) split K
-// over a cluster of CTAs: each keeps its fp32 partial in shared memory and,
-// after a cluster barrier, sums a share of the tile's rows over the
-// cluster's partials in rank order (distributed shared memory), the small-M
+// over a cluster of CTAs, one tile per CTA; when a class spans more than one
+// 128-row tile, a tile takes 2 x 128 of its rows (two accumulators sharing
+// each B stage).  After a cluster barrier each CTA pushes its fp32 partial
+// rows from TMEM into the shared memory of the rank that owns them, and each
+// owner sums its rows over the cluster's partials in rank order: the small-M
 // path's reduction turned on its side.  Every wait is bounded.
 #pragma once
 
