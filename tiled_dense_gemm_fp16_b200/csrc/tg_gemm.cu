@@ -1217,7 +1217,9 @@ tg_status run_blockscaled_grouped(const void* A, const void* SFA, const void* B,
   if (p.group_m < 1) p.group_m = 1;
   p.num_tiles = static_cast<int>(static_cast<int64_t>(p.m_tiles) * p.n_tiles);
   p.idesc = blockscaled_idesc<KIND>(Cfg::BM, a_format, b_format);
-  const int grid = p.num_tiles < info->sm_count ? p.num_tiles : info->sm_count;
+  const int ctas = tune_int("TG_TUNE_MX_CTAS", info->sm_count);
+  if (ctas < 1) return TG_ERR_INVALID_ARG;
+  const int grid = p.num_tiles < ctas ? p.num_tiles : ctas;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof cfg);
   cfg.stream = static_cast<cudaStream_t>(stream);
