@@ -18,9 +18,9 @@
 //         deep ring, so no scale load sits on the dequantization's path;
 //       - warps 6-13 turn each packed tile into the fp16 tile the MMA reads
 //         (128-byte swizzled, K-major) in a small second ring: a nibble is
-//         placed in the mantissa of 1024.0 (exponent bits 0x6400), 1032 is
-//         subtracted (exact: q - 8), and the fp16 multiply by the group's
-//         scale rounds once to nearest even;
+//         masked into the mantissa of 1024.0 or of 64.0 (where its bits have
+//         unit weight), 1032 or 72 is subtracted (exact: q - 8), and the fp16
+//         multiply by the group's scale rounds once to nearest even;
 //       - warp 1 issues 128 x m_pad x 16 MMAs; warps 2-5 move the fp32
 //         partial to shared memory for the cluster reduction.
 #pragma once
@@ -46,20 +46,22 @@ struct DequantParams {
 
 // Eight 4-bit codes (a 32-bit word, element 2i in the low nibble of byte i)
 // as eight fp16 values (q - 8) * s, in the pairs the arithmetic yields:
-// v[i] = (e_i, e_{i+4}), low half first.  Masking the word with 0x000F000F
-// pairs elements i and i + 4 in the two halves; each half becomes 1024 + q
-// (the code in the mantissa of 1024.0), 1032 is subtracted exactly, and the
-// multiply by the scale rounds once to nearest even.
+// v[i] = (e_i, e_{i+4}), low half first.  Masking the word (or the word
+// shifted by 8) with 0x000F000F puts elements i and i + 4 in the low mantissa
+// bits of 1024.0 (1024 + q, 1032 subtracted exactly); masking with 0x00F000F0
+// puts the odd elements in mantissa bits 4..7, which have unit weight in
+// 64.0 (64 + q, 72 subtracted exactly).  One mask per pair, one shift per
+// word; the multiply by the scale then rounds once to nearest even.
 __device__ __forceinline__ void dequant8_pairs(uint32_t w, __half2 s2, uint32_t (&v)[4]) {
-  const uint32_t mask = 0x000F000Fu, magic = 0x64006400u;  // fp16 1024.0 in both halves
-  v[0] = (w & mask) | magic;
-  v[1] = ((w >> 4) & mask) | magic;
-  v[2] = ((w >> 8) & mask) | magic;
-  v[3] = ((w >> 12) & mask) | magic;
-  const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
+  const uint32_t w8 = w >> 8;
+  v[0] = (w & 0x000F000Fu) | 0x64006400u;   // 1024 + q
+  v[1] = (w & 0x00F000F0u) | 0x54005400u;   // 64 + q
+  v[2] = (w8 & 0x000F000Fu) | 0x64006400u;
+  v[3] = (w8 & 0x00F000F0u) | 0x54005400u;
+  const __half2 even_bias = __floats2half2_rn(1032.0f, 1032.0f), odd_bias = __floats2half2_rn(72.0f, 72.0f);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const __half2 x = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v[i]), bias), s2);
+    const __half2 x = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v[i]), (i & 1) ? odd_bias : even_bias), s2);
     v[i] = *reinterpret_cast<const uint32_t*>(&x);
   }
 }
