@@ -144,7 +144,12 @@ def test_workspace_size_and_repack_choice():
     assert tg.workspace_size(A0, B0, C0 + 2, 64, 512, 512) == 0                      # the small-M kernel
     M, N, K = 3001, 5003, 1021
     assert tg.workspace_size(A0, B0, C0, M, N, K) == up(2 * K * 5008)
-    assert tg.workspace_size(A0, B0, C0, 8191, 129, 8193) == up(2 * 8193 * 136)
+    # One column of 144-wide tiles with 256 rows and 32+ k-blocks per CTA: B is realigned in
+    # place with two k-blocks in flight, faster than copying it first, so no workspace.
+    assert tg.workspace_size(A0, B0, C0, 8191, 129, 8193) == 0
+    assert tg.select_path_ws(A0, B0, C0, 8191, 129, 8193, up(2 * 8193 * 136)) == Path.RC
+    # Short K walks (17 k-blocks) keep the copy: (8191, 129, 1027).
+    assert tg.workspace_size(A0, B0, C0, 8191, 129, 1027) == up(2 * 1027 * 136)
     assert tg.workspace_size(A0, B0, C0, 64, 64, 100) == 0                          # odd K: only A, read in place
     assert tg.workspace_size(A0 + 2, B0, C0, 64, 64, 64) == 0                       # misaligned A base
     assert tg.workspace_size(A0, B0, C0, -1, 4, 4) == -1

@@ -68,6 +68,22 @@ def test_rc_split_k_cluster(M, N, K):
     assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"rc split {(M, N, K)}")
 
 
+@pytest.mark.parametrize("M,N,K,offsets", [
+    (2000, 129, 16385, (0, 0, 0)),  # 256-row tiles, K split over a cluster, 32+ k-blocks per CTA
+    (2000, 129, 16385, (5, 1, 3)),
+    (8000, 601, 2100, (0, 0, 0)),   # a wave of 160-column tiles, 33 k-blocks each
+    (8000, 601, 2100, (0, 3, 0)),
+    (8191, 129, 8193, (0, 0, 0)),   # the small-N workload at full size
+])
+def test_rc_realign_two_blocks_in_flight(M, N, K, offsets):
+    """B realigned in place with two k-blocks in flight: tiles narrower than 256 columns and K walks
+    of 32 or more k-blocks per CTA."""
+    A, B = inputs.operands(M, N, K, "int", seed=M + N + K + sum(offsets))
+    got, guards = run_gpu(A, B, RC, offsets=offsets)
+    assert guards
+    assert_bitexact(got, oracle.gemm_relu_f16(A, B), f"rc two-deep {(M, N, K)} {offsets}")
+
+
 @pytest.mark.parametrize("M,N,K", [(129, 257, 65), (1000, 1001, 1003), (2000, 129, 4099)])
 def test_rc_uniform(M, N, K):
     A, B = inputs.operands(M, N, K, "uniform", seed=7 + K)

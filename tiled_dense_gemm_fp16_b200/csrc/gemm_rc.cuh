@@ -260,7 +260,9 @@ __device__ __forceinline__ RcTile rc_tile(const RcParams& p, int t, int rank, in
   return r;
 }
 
-template <bool REALIGN_B, bool SPLIT>
+// B_DEEP (realigning mode, tiles narrower than 256 columns): the realigning
+// warps keep two k-blocks of B in flight instead of one.
+template <bool REALIGN_B, bool SPLIT, bool B_DEEP = false>
 __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
     gemm_relu_rc_kernel(const __grid_constant__ RcMaps maps, const RcParams p) {
   using Cfg = RcCfg<REALIGN_B>;
@@ -510,83 +512,185 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
     const uint32_t dst_off = static_cast<uint32_t>((lane >> 3) * Cfg::PANEL_BYTES + rw * 128 +
                                                    (((lane & 7) ^ (rw & 7)) << 4));
     const bool stores = lane < chunks;
-    const bool extra = lane == 31 && chunks == 32;  // block 32 of the piece
-    uint4 cur[kRows], ext[kRows];
-    uint32_t f_cur = 0, f_next = 0;  // the rows' offset past their first aligned block
-    // The k-blocks this CTA walks, in the order every role walks them.
-    int t = t_first, kb = 0;
-    RcTile T{};
-    bool valid = false;
-    for (; t < p.num_tiles; t += t_step) {
-      T = rc_tile(p, t, rank, splits);
-      if (T.kb_hi > T.kb_lo) {
-        kb = T.kb_lo;
-        valid = true;
-        break;
-      }
-    }
-    // Rows k0 + 8 m: their pieces start at the same offset f past a 16-byte
-    // boundary (8 rows are 16 ldb bytes apart), so one address and one
-    // bounds test serve all eight.
-    auto load_rows = [&](const RcTile& U, int kbu) {
-      const int k0 = kbu * 64 - U.e + rw;
-      const uintptr_t row0 = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k0) * p.ldb);
-      const uintptr_t start = row0 + 2u * static_cast<uintptr_t>(U.n0);
-      const uintptr_t a0 = start & ~uintptr_t(15);
-      const uintptr_t blk = a0 + 16u * static_cast<uintptr_t>(lane);
-      const bool lane_ok = lane <= chunks && blk < row0 + n_bytes;
-      const bool ext_ok = extra && a0 + 512u < row0 + n_bytes;
-      f_next = static_cast<uint32_t>((start >> 1) & 7u);
-#pragma unroll
-      for (int m = 0; m < kRows; ++m) {
-        const bool in = static_cast<unsigned>(k0 + 8 * m) < static_cast<unsigned>(p.K);
-        cur[m] = make_uint4(0u, 0u, 0u, 0u);
-        ext[m] = make_uint4(0u, 0u, 0u, 0u);
-        ld_nc_v4_pred(cur[m], reinterpret_cast<const void*>(blk + m * stride), in && lane_ok);
-        ld_nc_v4_pred(ext[m], reinterpret_cast<const void*>(a0 + 512u + m * stride), in && ext_ok);
-      }
-    };
-    if (valid) load_rows(T, kb);
-    int r = 0;
-    uint32_t rph = 0;
-    while (valid) {
-      // The next k-block in the walk.
-      int t2 = t, kb2 = kb + 1;
-      RcTile T2 = T;
-      bool valid2 = true;
-      while (kb2 >= T2.kb_hi) {
-        t2 += t_step;
-        if (t2 >= p.num_tiles) {
-          valid2 = false;
+    if constexpr (B_DEEP) {
+      // Two k-blocks in flight: two register sets of 8 rows (tiles
+      // narrower than 256 columns, so lane 31 never needs a 33rd block).
+      const bool extra = !B_DEEP && lane == 31 && chunks == 32;  // block 32 of the piece
+      // Row registers: one k-block plus lane 31's 33rd blocks, or (B_DEEP,
+      // at most 31 chunks, so block 32 is never needed) two k-blocks.
+      constexpr int kSets = B_DEEP ? 2 : 1;
+      uint4 rows[kSets][kRows], ext[kRows];
+      uint32_t f_row[kSets] = {};  // the rows' offset past their first aligned block
+      // The k-blocks this CTA walks, in the order every role walks them: `ld`
+      // is the next one to load, `pr` the next one to realign.
+      struct Walk {
+        int t, kb;
+        RcTile T;
+        bool valid;
+      };
+      Walk ld{t_first, 0, RcTile{}, false};
+      for (; ld.t < p.num_tiles; ld.t += t_step) {
+        ld.T = rc_tile(p, ld.t, rank, splits);
+        if (ld.T.kb_hi > ld.T.kb_lo) {
+          ld.kb = ld.T.kb_lo;
+          ld.valid = true;
           break;
         }
-        T2 = rc_tile(p, t2, rank, splits);
-        kb2 = T2.kb_lo;
       }
-      f_cur = f_next;
-      const bool got = mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
-      if (!__all_sync(0xffffffffu, got)) break;
-      // Rows outside [0, K) were loaded as zeros and shift to zeros.
-      const uint32_t dst = smem_u32(ring + r * p.ring_stage_bytes) + p.msub * Cfg::A_BYTES + dst_off;
-      const uint32_t bits = (f_cur & 1u) * 16u;
-      switch (f_cur >> 1) {
-        case 0: rc_shift_rows<0>(cur, ext, bits, dst, stores, lane == 31); break;
-        case 1: rc_shift_rows<1>(cur, ext, bits, dst, stores, lane == 31); break;
-        case 2: rc_shift_rows<2>(cur, ext, bits, dst, stores, lane == 31); break;
-        default: rc_shift_rows<3>(cur, ext, bits, dst, stores, lane == 31); break;
+      auto advance = [&](Walk& w) {
+        ++w.kb;
+        while (w.kb >= w.T.kb_hi) {
+          w.t += t_step;
+          if (w.t >= p.num_tiles) {
+            w.valid = false;
+            return;
+          }
+          w.T = rc_tile(p, w.t, rank, splits);
+          w.kb = w.T.kb_lo;
+        }
+      };
+      Walk pr = ld;
+      // Rows k0 + 8 m: their pieces start at the same offset f past a 16-byte
+      // boundary (8 rows are 16 ldb bytes apart), so one address and one
+      // bounds test serve all eight.
+      auto load_rows = [&](uint4 (&cur)[kRows], uint32_t& f) {
+        const int k0 = ld.kb * 64 - ld.T.e + rw;
+        const uintptr_t row0 = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k0) * p.ldb);
+        const uintptr_t start = row0 + 2u * static_cast<uintptr_t>(ld.T.n0);
+        const uintptr_t a0 = start & ~uintptr_t(15);
+        const uintptr_t blk = a0 + 16u * static_cast<uintptr_t>(lane);
+        const bool lane_ok = lane <= chunks && blk < row0 + n_bytes;
+        const bool ext_ok = extra && a0 + 512u < row0 + n_bytes;
+        f = static_cast<uint32_t>((start >> 1) & 7u);
+  #pragma unroll
+        for (int m = 0; m < kRows; ++m) {
+          const bool in = static_cast<unsigned>(k0 + 8 * m) < static_cast<unsigned>(p.K);
+          cur[m] = make_uint4(0u, 0u, 0u, 0u);
+          ld_nc_v4_pred(cur[m], reinterpret_cast<const void*>(blk + m * stride), in && lane_ok);
+          if (!B_DEEP) {
+            ext[m] = make_uint4(0u, 0u, 0u, 0u);
+            ld_nc_v4_pred(ext[m], reinterpret_cast<const void*>(a0 + 512u + m * stride), in && ext_ok);
+          }
+        }
+        advance(ld);
+      };
+  #pragma unroll
+      for (int i = 0; i < kSets; ++i)
+        if (ld.valid) load_rows(rows[i], f_row[i]);
+      int r = 0;
+      uint32_t rph = 0;
+      bool ok = true;
+      // Realign k-block `pr` from one register set, then refill that set with
+      // the next k-block still to load.
+      auto step = [&](uint4 (&cur)[kRows], uint32_t& f) {
+        if (!mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B)) ok = false;
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          return;
+        }
+        // Rows outside [0, K) were loaded as zeros and shift to zeros.
+        const uint32_t dst = smem_u32(ring + r * p.ring_stage_bytes) + p.msub * Cfg::A_BYTES + dst_off;
+        const uint32_t bits = (f & 1u) * 16u;
+        const uint4 (&e)[kRows] = B_DEEP ? cur : ext;  // lane 31's block 32 only when !B_DEEP
+        switch (f >> 1) {
+          case 0: rc_shift_rows<0>(cur, e, bits, dst, stores, extra); break;
+          case 1: rc_shift_rows<1>(cur, e, bits, dst, stores, extra); break;
+          case 2: rc_shift_rows<2>(cur, e, bits, dst, stores, extra); break;
+          default: rc_shift_rows<3>(cur, e, bits, dst, stores, extra); break;
+        }
+        if (ld.valid) load_rows(cur, f);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bfull_bar[r]);
+        if (++r == p.ring_stages) {
+          r = 0;
+          rph ^= 1u;
+        }
+        advance(pr);
+      };
+      while (pr.valid && ok) {
+        step(rows[0], f_row[0]);
+        if (B_DEEP && pr.valid && ok) step(rows[kSets - 1], f_row[kSets - 1]);
       }
-      if (valid2) load_rows(T2, kb2);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bfull_bar[r]);
-      if (++r == p.ring_stages) {
-        r = 0;
-        rph ^= 1u;
+    } else {
+      const bool extra = lane == 31 && chunks == 32;  // block 32 of the piece
+      uint4 cur[kRows], ext[kRows];
+      uint32_t f_cur = 0, f_next = 0;  // the rows' offset past their first aligned block
+      // The k-blocks this CTA walks, in the order every role walks them.
+      int t = t_first, kb = 0;
+      RcTile T{};
+      bool valid = false;
+      for (; t < p.num_tiles; t += t_step) {
+        T = rc_tile(p, t, rank, splits);
+        if (T.kb_hi > T.kb_lo) {
+          kb = T.kb_lo;
+          valid = true;
+          break;
+        }
       }
-      t = t2;
-      kb = kb2;
-      T = T2;
-      valid = valid2;
+      // Rows k0 + 8 m: their pieces start at the same offset f past a 16-byte
+      // boundary (8 rows are 16 ldb bytes apart), so one address and one
+      // bounds test serve all eight.
+      auto load_rows = [&](const RcTile& U, int kbu) {
+        const int k0 = kbu * 64 - U.e + rw;
+        const uintptr_t row0 = bbytes + 2u * static_cast<uintptr_t>(static_cast<int64_t>(k0) * p.ldb);
+        const uintptr_t start = row0 + 2u * static_cast<uintptr_t>(U.n0);
+        const uintptr_t a0 = start & ~uintptr_t(15);
+        const uintptr_t blk = a0 + 16u * static_cast<uintptr_t>(lane);
+        const bool lane_ok = lane <= chunks && blk < row0 + n_bytes;
+        const bool ext_ok = extra && a0 + 512u < row0 + n_bytes;
+        f_next = static_cast<uint32_t>((start >> 1) & 7u);
+  #pragma unroll
+        for (int m = 0; m < kRows; ++m) {
+          const bool in = static_cast<unsigned>(k0 + 8 * m) < static_cast<unsigned>(p.K);
+          cur[m] = make_uint4(0u, 0u, 0u, 0u);
+          ext[m] = make_uint4(0u, 0u, 0u, 0u);
+          ld_nc_v4_pred(cur[m], reinterpret_cast<const void*>(blk + m * stride), in && lane_ok);
+          ld_nc_v4_pred(ext[m], reinterpret_cast<const void*>(a0 + 512u + m * stride), in && ext_ok);
+        }
+      };
+      if (valid) load_rows(T, kb);
+      int r = 0;
+      uint32_t rph = 0;
+      while (valid) {
+        // The next k-block in the walk.
+        int t2 = t, kb2 = kb + 1;
+        RcTile T2 = T;
+        bool valid2 = true;
+        while (kb2 >= T2.kb_hi) {
+          t2 += t_step;
+          if (t2 >= p.num_tiles) {
+            valid2 = false;
+            break;
+          }
+          T2 = rc_tile(p, t2, rank, splits);
+          kb2 = T2.kb_lo;
+        }
+        f_cur = f_next;
+        const bool got = mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B);
+        if (!__all_sync(0xffffffffu, got)) break;
+        // Rows outside [0, K) were loaded as zeros and shift to zeros.
+        const uint32_t dst = smem_u32(ring + r * p.ring_stage_bytes) + p.msub * Cfg::A_BYTES + dst_off;
+        const uint32_t bits = (f_cur & 1u) * 16u;
+        switch (f_cur >> 1) {
+          case 0: rc_shift_rows<0>(cur, ext, bits, dst, stores, lane == 31); break;
+          case 1: rc_shift_rows<1>(cur, ext, bits, dst, stores, lane == 31); break;
+          case 2: rc_shift_rows<2>(cur, ext, bits, dst, stores, lane == 31); break;
+          default: rc_shift_rows<3>(cur, ext, bits, dst, stores, lane == 31); break;
+        }
+        if (valid2) load_rows(T2, kb2);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bfull_bar[r]);
+        if (++r == p.ring_stages) {
+          r = 0;
+          rph ^= 1u;
+        }
+        t = t2;
+        kb = kb2;
+        T = T2;
+        valid = valid2;
+      }
     }
   }
 

@@ -202,10 +202,117 @@ bool rc_preferred(const Problem& p) {
   return rc_ok(p) && 2400.0 * static_cast<double>(p.N + p.K) > static_cast<double>(p.N) * static_cast<double>(p.K);
 }
 
+// Tile plan of the residue-class kernel (host logic only): tile width, rows
+// per tile, K split and ring, for a device of `sms` SMs.
+struct RcPlan {
+  int bn = 0, n_tiles = 0, panels = 0, msub = 1, splits = 1, ring = 0, ring_bytes = 0;
+  int kb_per_cta = 0;    // k-blocks a CTA walks per tile (upper bound over the classes)
+  bool b_deep = false;   // B realigned in place keeps two k-blocks in flight
+};
+constexpr int kRcSmemMax = 232448, kRcFixed = 1024 + 512;
+constexpr int kRcPlanSms = 148;  // SMs assumed by the host-only queries
+
+// One class when A's row stride is a multiple of 8 elements and covers the
+// widened rows; else the eight residue classes of the rows.
+int rc_a_classes(const void* A, int64_t lda, int64_t K) {
+  const int64_t e0 = static_cast<int64_t>((reinterpret_cast<uintptr_t>(A) & 15u) / 2);
+  return (lda % 8 == 0 && lda >= K + e0) ? 1 : kRcClasses;
+}
+
+bool rc_plan(int64_t M, int64_t N, int64_t K, int a_classes, int sms, RcPlan* out) {
+  RcPlan pl;
+  const int kb_min = static_cast<int>((K + 63) / 64);
+  pl.bn = N <= 240 ? static_cast<int>((N + 15) / 16 * 16) : 256;
+  int64_t m128 = 0;
+  for (int c = 0; c < a_classes; ++c) {
+    const int64_t n = M > c ? (M - c + a_classes - 1) / a_classes : 0;
+    m128 += (n + 127) / 128;
+  }
+  // The persistent CTAs take the tiles in waves.  When 256-wide tiles fill
+  // at least one wave, pick the width w (a multiple of 16, 128..256) with
+  // the least waves x bytes per k-block (16 KiB of A and 128 w of B: the
+  // kernel moves operands rather than multiplies), so that the last wave is
+  // not mostly idle; ties go to the wider tile.
+  if (N > 240 && m128 * ((N + 255) / 256) >= sms) {
+    int64_t best = -1;
+    for (int w = 256; w >= 128; w -= 16) {
+      const int64_t cost = (m128 * ((N + w - 1) / w) + sms - 1) / sms * (16384 + 128 * w);
+      if (best < 0 || cost < best) {
+        best = cost;
+        pl.bn = w;
+      }
+    }
+  }
+  pl.bn = tune_int("TG_TUNE_RC_BN", pl.bn);
+  if (pl.bn < 16 || pl.bn > 256 || pl.bn % 16 != 0) return false;
+  pl.n_tiles = static_cast<int>((N + pl.bn - 1) / pl.bn);
+  pl.panels = (pl.bn + 63) / 64;
+  auto tiles_for = [&](int rows) {
+    int t = 0;
+    for (int c = 0; c < a_classes; ++c) {
+      const int64_t n = M > c ? (M - c + a_classes - 1) / a_classes : 0;
+      t += static_cast<int>((n + rows - 1) / rows);
+    }
+    return t * pl.n_tiles;
+  };
+  auto ring_for = [&](int msub, int* stages, int* stage_bytes) {
+    *stage_bytes = msub * RcCfg<false>::A_BYTES + pl.panels * RcCfg<false>::PANEL_BYTES;
+    int r = (kRcSmemMax - kRcFixed) / *stage_bytes;
+    *stages = r > RcCfg<false>::MAX_RING ? RcCfg<false>::MAX_RING : r;
+  };
+  // Few tiles: split K over a cluster of S CTAs (each keeps at least 4
+  // k-blocks), when the cluster's partials of one tile's rows (S slots of
+  // ceil(R / S) rows) fit in the ring.  For one column of narrow tiles (A
+  // streams from memory) a tile takes 2 x 128 class rows, two accumulators
+  // sharing each B stage, when that still splits.
+  auto splits_for = [&](int tiles, int msub) {
+    int st, sb;
+    ring_for(msub, &st, &sb);
+    if (st < 2 || 2 * tiles > sms) return 1;
+    int s = sms / tiles;
+    s = s > 8 ? 8 : s;
+    while (s > 1 && kb_min / s < 4) --s;
+    s = tune_int("TG_TUNE_RC_SPLITS", s);
+    if (s > 8) s = 8;
+    const int R = 128 * msub;
+    while (s > 1 && s * ((R + s - 1) / s) * pl.bn * 4 > st * sb) --s;
+    return s;
+  };
+  pl.splits = splits_for(tiles_for(128), 1);
+  if (pl.splits > 1 && pl.bn <= 240 && tiles_for(256) < tiles_for(128) && tune_int("TG_TUNE_RC_MSUB2", 1)) {
+    const int s2 = splits_for(tiles_for(256), 2);
+    if (s2 > 1) {
+      pl.msub = 2;
+      pl.splits = s2;
+    }
+  }
+  ring_for(pl.msub, &pl.ring, &pl.ring_bytes);
+  if (pl.ring < 2) return false;
+  // B realigned in place keeps two k-blocks in flight with tiles narrower
+  // than 256 columns (at most 31 chunks per row, so no lane needs a 33rd
+  // block) and long K walks (32 or more k-blocks per CTA and tile).
+  // Measured without a workspace: (8191, 129, 8193) 47.0 -> 44.5 us, (777,
+  // 12289, 4095) 192.8 -> 179.6 us; with 16 k-blocks, (3001, 5003, 1021) went
+  // from 72.5 to 75-76 us, so short walks keep one.
+  const int kb_walk = static_cast<int>((K + 7 + 63) / 64);
+  pl.kb_per_cta = (kb_walk + pl.splits - 1) / pl.splits;
+  pl.b_deep = pl.bn < 256 && pl.kb_per_cta >= 32 && tune_int("TG_TUNE_RC_B_DEEP", 1);
+  *out = pl;
+  return true;
+}
+
 // Bytes of the padded copy of B (rows rounded up to 8 elements) that the
-// residue-class kernel reads when TMA cannot describe B, else 0.
+// residue-class kernel reads when TMA cannot describe B, else 0.  No copy
+// either where realigning B in place is the faster route: two k-blocks in
+// flight and a B tile no wider than the tile's rows of A (bn <= 128 msub), so
+// that B is the smaller stream.  Measured at (8191, 129, 8193): 44.5 us in
+// place against 49.7 us with the copy (a dependent kernel between GEMMs).
 int64_t rc_b_copy_bytes(const Problem& p) {
   if (p.K <= 0 || p.N <= 0 || tma_ok_b(p)) return 0;
+  RcPlan pl;
+  if (!p.a_km && rc_plan(p.M, p.N, p.K, rc_a_classes(p.A, p.lda, p.K), kRcPlanSms, &pl) && pl.b_deep &&
+      pl.bn <= 128 * pl.msub)
+    return 0;
   return (2 * p.K * ((p.N + 7) / 8 * 8) + 255) / 256 * 256;
 }
 
@@ -709,11 +816,11 @@ bool encode_classes(CUtensorMap* maps, const void* base, int64_t rows, int64_t c
   return true;
 }
 
-template <bool REALIGN_B, bool SPLIT>
+template <bool REALIGN_B, bool SPLIT, bool B_DEEP = false>
 tg_status launch_rc_cfg(const RcMaps& maps, const RcParams& p, int smem, int grid_x, int grid_y,
                         cudaStream_t stream, DeviceInfo* info) {
-  auto kernel = gemm_relu_rc_kernel<REALIGN_B, SPLIT>;
-  constexpr unsigned kBit = 1u << ((REALIGN_B ? 1 : 0) + (SPLIT ? 2 : 0));
+  auto kernel = gemm_relu_rc_kernel<REALIGN_B, SPLIT, B_DEEP>;
+  constexpr unsigned kBit = 1u << ((REALIGN_B ? 1 : 0) + (SPLIT ? 2 : 0) + (B_DEEP ? 4 : 0));
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!(info->rc_attr & kBit)) {
@@ -753,80 +860,14 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  // One class when the row stride is a multiple of 8 elements and covers the
-  // widened rows; else the eight residue classes of the rows.
-  const int e0 = static_cast<int>((reinterpret_cast<uintptr_t>(o.A) & 15u) / 2);
-  p.a_classes = (o.lda % 8 == 0 && o.lda >= K + e0) ? 1 : kRcClasses;
+  p.a_classes = rc_a_classes(o.A, o.lda, K);
   const int sms = info->sm_count;
-  const int kb_min = static_cast<int>((K + 63) / 64);
-  p.bn = N <= 240 ? static_cast<int>((N + 15) / 16 * 16) : 256;
-  {
-    // The persistent CTAs take the tiles in waves.  When 256-wide tiles fill
-    // at least one wave, pick the width w (a multiple of 16, 128..256) with
-    // the least waves x bytes per k-block (16 KiB of A and 128 w of B: the
-    // kernel moves operands rather than multiplies), so that the last wave is
-    // not mostly idle; ties go to the wider tile.
-    int64_t m128 = 0;
-    for (int c = 0; c < p.a_classes; ++c) {
-      const int64_t n = M > c ? (M - c + p.a_classes - 1) / p.a_classes : 0;
-      m128 += (n + 127) / 128;
-    }
-    if (N > 240 && m128 * ((N + 255) / 256) >= sms) {
-      int64_t best = -1;
-      for (int w = 256; w >= 128; w -= 16) {
-        const int64_t cost = (m128 * ((N + w - 1) / w) + sms - 1) / sms * (16384 + 128 * w);
-        if (best < 0 || cost < best) {
-          best = cost;
-          p.bn = w;
-        }
-      }
-    }
-    p.bn = tune_int("TG_TUNE_RC_BN", p.bn);
-    if (p.bn < 16 || p.bn > 256 || p.bn % 16 != 0) return TG_ERR_INVALID_ARG;
-  }
-  p.n_tiles = static_cast<int>((N + p.bn - 1) / p.bn);
-  p.panels = (p.bn + 63) / 64;
-  auto tiles_for = [&](int rows) {
-    int t = 0;
-    for (int c = 0; c < p.a_classes; ++c) {
-      const int64_t n = M > c ? (M - c + p.a_classes - 1) / p.a_classes : 0;
-      t += static_cast<int>((n + rows - 1) / rows);
-    }
-    return t * p.n_tiles;
-  };
-  constexpr int kSmemMax = 232448, kFixed = 1024 + 512;
-  auto ring_for = [&](int msub, int* stages, int* stage_bytes) {
-    *stage_bytes = msub * RcCfg<false>::A_BYTES + p.panels * RcCfg<false>::PANEL_BYTES;
-    int r = (kSmemMax - kFixed) / *stage_bytes;
-    *stages = r > RcCfg<false>::MAX_RING ? RcCfg<false>::MAX_RING : r;
-  };
-  // Few tiles: split K over a cluster of S CTAs (each keeps at least 4
-  // k-blocks), when the cluster's partials of one tile's rows (S slots of
-  // ceil(R / S) rows) fit in the ring.  For one column of narrow tiles (A
-  // streams from memory) a tile takes 2 x 128 class rows, two accumulators
-  // sharing each B stage, when that still splits.
-  auto splits_for = [&](int tiles, int msub) {
-    int st, sb;
-    ring_for(msub, &st, &sb);
-    if (st < 2 || 2 * tiles > sms) return 1;
-    int s = sms / tiles;
-    s = s > 8 ? 8 : s;
-    while (s > 1 && kb_min / s < 4) --s;
-    s = tune_int("TG_TUNE_RC_SPLITS", s);
-    if (s > 8) s = 8;
-    const int R = 128 * msub;
-    while (s > 1 && s * ((R + s - 1) / s) * p.bn * 4 > st * sb) --s;
-    return s;
-  };
-  int msub = 1;
-  int splits = splits_for(tiles_for(128), 1);
-  if (splits > 1 && p.bn <= 240 && tiles_for(256) < tiles_for(128) && tune_int("TG_TUNE_RC_MSUB2", 1)) {
-    const int s2 = splits_for(tiles_for(256), 2);
-    if (s2 > 1) {
-      msub = 2;
-      splits = s2;
-    }
-  }
+  RcPlan pl;
+  if (!rc_plan(M, N, K, p.a_classes, sms, &pl)) return TG_ERR_INTERNAL;  // a bad tuning width, or no room for two stages
+  p.bn = pl.bn;
+  p.n_tiles = pl.n_tiles;
+  p.panels = pl.panels;
+  const int msub = pl.msub, splits = pl.splits;
   p.msub = msub;
   if (!encode_classes(maps.a, o.A, M, K, o.lda, p.a_classes, 64, 128 * msub, CU_TENSOR_MAP_SWIZZLE_128B, p.a_shift,
                       p.rows_in_class))
@@ -849,22 +890,24 @@ tg_status launch_rc(const Operands& o, cudaStream_t stream, DeviceInfo* info) {
   if (!realign_b && !encode_2d(&maps.b, o.B, K, N, o.ldb, 64, 64)) {
     return TG_ERR_LAUNCH;
   }
-  int ring = 0;
-  ring_for(msub, &ring, &p.ring_stage_bytes);
-  if (ring < 2) return TG_ERR_INTERNAL;
+  const int ring = pl.ring;
+  p.ring_stage_bytes = pl.ring_bytes;
   p.ring_stages = ring;
   p.idesc = make_idesc_f16_f32(128, p.bn, false, true);
   p.wait_budget_ns = wait_budget(kb_max);
-  const int smem = kFixed + ring * p.ring_stage_bytes;
+  const int smem = kRcFixed + ring * p.ring_stage_bytes;
   p.splits = splits;
+  const bool b_deep = realign_b && pl.b_deep;
   if (splits > 1) {
     if (p.num_tiles > 65535) return TG_ERR_INVALID_ARG;
-    return realign_b ? launch_rc_cfg<true, true>(maps, p, smem, splits, p.num_tiles, stream, info)
-                   : launch_rc_cfg<false, true>(maps, p, smem, splits, p.num_tiles, stream, info);
+    if (!realign_b) return launch_rc_cfg<false, true>(maps, p, smem, splits, p.num_tiles, stream, info);
+    return b_deep ? launch_rc_cfg<true, true, true>(maps, p, smem, splits, p.num_tiles, stream, info)
+                  : launch_rc_cfg<true, true>(maps, p, smem, splits, p.num_tiles, stream, info);
   }
   const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-  return realign_b ? launch_rc_cfg<true, false>(maps, p, smem, grid, 1, stream, info)
-                 : launch_rc_cfg<false, false>(maps, p, smem, grid, 1, stream, info);
+  if (!realign_b) return launch_rc_cfg<false, false>(maps, p, smem, grid, 1, stream, info);
+  return b_deep ? launch_rc_cfg<true, false, true>(maps, p, smem, grid, 1, stream, info)
+                : launch_rc_cfg<true, false>(maps, p, smem, grid, 1, stream, info);
 }
 
 __global__ void wait_timeout_selftest_kernel(uint64_t budget_ns) {
