@@ -119,12 +119,16 @@ TG_API tg_status tg_gemm_relu_f16_path(const void *A, const void *B, void *C, in
 
 /*
  * C = ReLU(A . B) with a caller-provided device workspace.  Identical to
- * tg_gemm_relu_f16 except in two cases (path TG_PATH_REPACK):
+ * tg_gemm_relu_f16 except where the workspace lets a faster route run:
  *   - TMA cannot describe A or B (a row stride that is not a multiple of 16
- *     bytes, or a base that is not 16-byte aligned) and the workspace holds
- *     their copies: they are first copied into zero-padded rows in the
- *     workspace and a TMA kernel runs on the copies, several times faster
- *     than the edge mode;
+ *     bytes, or a base that is not 16-byte aligned).  Where the residue-class
+ *     kernel takes them (1/N + 1/K > 1/2400, TG_PATH_RC), B alone is first
+ *     copied into zero-padded rows in the workspace and loaded by TMA, except
+ *     where realigning B in place is the faster route (tiles narrower than
+ *     256 columns, 32 or more k-blocks per CTA, B's tile no wider than the
+ *     tile's rows of A): then nothing is copied.  Elsewhere (TG_PATH_REPACK)
+ *     A and B are copied into zero-padded rows and a TMA kernel runs on the
+ *     copies;
  *   - the rows of C are not 16-byte aligned, M > 256, and the workspace also
  *     holds a padded C (tg_workspace_size covers it): the GEMM writes that
  *     copy with its aligned stores and a realigning copy moves it into C.
@@ -212,10 +216,11 @@ typedef struct tg_gemm_options {
 /*
  * C = ReLU(A . B + bias) with the layouts and batching of `options`.
  * Operands TMA cannot describe (row or batch strides that are not multiples
- * of 8 elements, bases that are not 16-byte aligned) go through the repack
- * path when `workspace_bytes` >= tg_workspace_size_ex(...); without enough
- * workspace, A stored M x K with B stored K x N uses the edge mode and the
- * other layouts are refused (TG_ERR_INVALID_ARG).  A stored K x M runs on the
+ * of 8 elements, bases that are not 16-byte aligned) take, for A stored M x K
+ * with B stored K x N, the residue-class kernel (with B's padded copy when
+ * the workspace holds it and the rule of tg_gemm_relu_f16_ws asks for it) or
+ * the repack path; the other layouts need the repack path's workspace
+ * (tg_workspace_size_ex) and are refused without it (TG_ERR_INVALID_ARG).  A stored K x M runs on the
  * 128- and 256-row tensor-core kernels (not the small-M kernel).  Batch entries run in order on `stream` and share the
  * workspace.  Errors as tg_gemm_relu_f16_ws, plus TG_ERR_INVALID_ARG for
  * strides below the row lengths, overlapping C entries, an unknown b_layout
@@ -237,11 +242,14 @@ TG_API int tg_select_path_ex(const void *A, const void *B, const void *C, int64_
 
 /*
  * Workspace bytes tg_gemm_relu_f16_ws needs for its fastest path with these
- * arguments: copies of A and B when TMA cannot describe them, plus, when the
- * rows of C are not 16-byte aligned and a tensor-core kernel runs (M > 256),
- * a padded C that the GEMM writes and a realigning copy moves into C.  Less
- * workspace still takes the repack path as long as the A and B copies fit.
- * 0 when neither applies, -1 for invalid arguments.  Host logic only.
+ * arguments: when TMA cannot describe A or B, B's padded copy on the
+ * residue-class route (or nothing, where B is realigned in place; see
+ * tg_gemm_relu_f16_ws), else copies of A and B, plus, when the rows of C are
+ * not 16-byte aligned and a tensor-core kernel runs (M > 256), a padded C
+ * that the GEMM writes and a realigning copy moves into C.  Less workspace
+ * still takes the repack path as long as the A and B copies fit.  0 when
+ * none applies, -1 for invalid arguments.  Host logic only (it assumes the
+ * 148 SMs of a B200 where the choice depends on the SM count).
  */
 TG_API int64_t tg_workspace_size(const void *A, const void *B, const void *C, int64_t M, int64_t N, int64_t K);
 
