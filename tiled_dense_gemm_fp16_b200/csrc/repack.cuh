@@ -30,24 +30,27 @@ struct RepackParams {
   int64_t chunks;            // rows * cols_pad / 8
 };
 
-__global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
+// Index: the type of the chunk arithmetic.  32-bit when the copy has fewer
+// than 2^31 chunks (a 32-bit division per chunk instead of a 64-bit one,
+// which is a long software routine on the GPU), else 64-bit.
+template <typename Index>
+__device__ __forceinline__ void pad_rows_body(const RepackParams& p) {
   constexpr int kUnroll = 4;
-  grid_dependency_wait();
-  grid_launch_dependents();
-  const int chunks_per_row = p.cols_pad >> 3;
+  const Index chunks_per_row = static_cast<Index>(p.cols_pad >> 3);
+  const Index chunks = static_cast<Index>(p.chunks);
   const __half* src_end = p.src + static_cast<int64_t>(p.rows - 1) * p.src_ld + p.cols;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < p.chunks;
+  const Index stride = static_cast<Index>(gridDim.x) * blockDim.x;
+  for (Index base = static_cast<Index>(blockIdx.x) * blockDim.x + threadIdx.x; base < chunks;
        base += stride * kUnroll) {
     EdgeChunk plan[kUnroll];
     int row[kUnroll], col[kUnroll];
     bool live[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t c = base + u * stride;
-      live[u] = c < p.chunks;
+      const Index c = base + u * stride;
+      live[u] = c < chunks;
       row[u] = live[u] ? static_cast<int>(c / chunks_per_row) : 0;
-      col[u] = live[u] ? static_cast<int>(c - static_cast<int64_t>(row[u]) * chunks_per_row) * 8 : 0;
+      col[u] = live[u] ? static_cast<int>(c - static_cast<Index>(row[u]) * chunks_per_row) * 8 : 0;
       plan[u] = edge_chunk_plan(p.src, src_end, p.src_ld, live[u] ? row[u] : p.rows, p.rows, col[u], p.cols);
     }
     uint4 lo[kUnroll], hi[kUnroll];
@@ -68,6 +71,15 @@ __global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
   }
 }
 
+__global__ void __launch_bounds__(256) pad_rows_kernel(const RepackParams p) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (p.chunks < (int64_t(1) << 31))
+    pad_rows_body<uint32_t>(p);
+  else
+    pad_rows_body<int64_t>(p);
+}
+
 // The reverse copy, for C: the GEMM writes a padded copy (rows of cols_pad
 // elements, 16-byte aligned) and this kernel moves it into C, whose rows may
 // start on any 2-byte boundary.  Each thread writes one 16-byte-aligned block
@@ -85,13 +97,15 @@ struct UnpadParams {
   int64_t blocks;      // rows * blocks_per_row
 };
 
-__global__ void __launch_bounds__(256) unpad_rows_kernel(const UnpadParams p) {
+// Index as in pad_rows_body.
+template <typename Index>
+__device__ __forceinline__ void unpad_rows_body(const UnpadParams& p) {
   constexpr int kUnroll = 4;  // four blocks' loads in flight per thread before any store
-  grid_dependency_wait();
-  grid_launch_dependents();
   const uintptr_t src_end = reinterpret_cast<uintptr_t>(p.src + static_cast<int64_t>(p.rows) * p.cols_pad);
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < p.blocks;
+  const Index blocks = static_cast<Index>(p.blocks);
+  const Index blocks_per_row = static_cast<Index>(p.blocks_per_row);
+  const Index stride = static_cast<Index>(gridDim.x) * blockDim.x;
+  for (Index base = static_cast<Index>(blockIdx.x) * blockDim.x + threadIdx.x; base < blocks;
        base += stride * kUnroll) {
     __half* drow[kUnroll];
     const __half* srow[kUnroll];
@@ -101,10 +115,10 @@ __global__ void __launch_bounds__(256) unpad_rows_kernel(const UnpadParams p) {
     uint4 lo[kUnroll], hi[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t i = base + u * stride;
-      live[u] = i < p.blocks;
-      const int r = live[u] ? static_cast<int>(i / p.blocks_per_row) : 0;
-      const int j = live[u] ? static_cast<int>(i - static_cast<int64_t>(r) * p.blocks_per_row) : 0;
+      const Index i = base + u * stride;
+      live[u] = i < blocks;
+      const int r = live[u] ? static_cast<int>(i / blocks_per_row) : 0;
+      const int j = live[u] ? static_cast<int>(i - static_cast<Index>(r) * blocks_per_row) : 0;
       drow[u] = p.dst + static_cast<int64_t>(r) * p.dst_ld;
       srow[u] = p.src + static_cast<int64_t>(r) * p.cols_pad;
       // Elements before the row's first aligned block, then block j's first element.
@@ -134,6 +148,15 @@ __global__ void __launch_bounds__(256) unpad_rows_kernel(const UnpadParams p) {
       }
     }
   }
+}
+
+__global__ void __launch_bounds__(256) unpad_rows_kernel(const UnpadParams p) {
+  grid_dependency_wait();
+  grid_launch_dependents();
+  if (p.blocks < (int64_t(1) << 31))
+    unpad_rows_body<uint32_t>(p);
+  else
+    unpad_rows_body<int64_t>(p);
 }
 
 }  // namespace tg
