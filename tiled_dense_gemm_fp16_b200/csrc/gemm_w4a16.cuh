@@ -74,19 +74,51 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2) {
                     __byte_perm(v[0], v[1], 0x7632), __byte_perm(v[2], v[3], 0x7632));
 }
 
+// Index: the type of the chunk arithmetic, 32-bit below 2^31 chunks (a
+// 64-bit division is a long software routine on the GPU).  Four chunks per
+// thread and round, their code and scale loads issued before any store, so
+// that enough bytes are in flight to cover the memory latency.
+template <typename Index>
+__device__ __forceinline__ void dequant_w4_body(const DequantParams& p) {
+  constexpr int kUnroll = 4;
+  const Index per_row = static_cast<Index>(p.K / 8);
+  const Index chunks = static_cast<Index>(p.chunks);
+  const Index stride = static_cast<Index>(gridDim.x) * blockDim.x;
+  const int gshift = __ffs(p.group) - 1;  // the group is a power of two
+  const int64_t groups_per_row = p.K >> gshift;
+  for (Index base = static_cast<Index>(blockIdx.x) * blockDim.x + threadIdx.x; base < chunks;
+       base += stride * kUnroll) {
+    uint32_t w[kUnroll];
+    __half sc[kUnroll];
+    int64_t n[kUnroll], k[kUnroll];
+    bool live[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const Index c = base + u * stride;
+      live[u] = c < chunks;
+      const Index nr = live[u] ? c / per_row : 0;
+      n[u] = static_cast<int64_t>(nr);
+      k[u] = static_cast<int64_t>(c - nr * per_row) * 8;
+      w[u] = 0u;
+      sc[u] = __float2half(0.0f);
+      if (live[u]) {
+        w[u] = __ldg(reinterpret_cast<const uint32_t*>(p.Wq + n[u] * (p.K / 2) + k[u] / 2));
+        sc[u] = p.S[n[u] * groups_per_row + (k[u] >> gshift)];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (live[u]) reinterpret_cast<uint4*>(p.W + n[u] * p.K)[k[u] / 8] = dequant8(w[u], __halves2half2(sc[u], sc[u]));
+  }
+}
+
 __global__ void __launch_bounds__(256) dequant_w4_kernel(const DequantParams p) {
   grid_dependency_wait();
   grid_launch_dependents();
-  const int64_t per_row = p.K / 8;
-  const int64_t groups_per_row = p.K / p.group;
-  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < p.chunks;
-       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = c / per_row;
-    const int64_t k = (c - n * per_row) * 8;
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p.Wq + n * (p.K / 2) + k / 2));
-    const __half s = p.S[n * groups_per_row + k / p.group];
-    reinterpret_cast<uint4*>(p.W + n * p.K)[k / 8] = dequant8(w, __halves2half2(s, s));
-  }
+  if (p.chunks < (int64_t(1) << 31))
+    dequant_w4_body<uint32_t>(p);
+  else
+    dequant_w4_body<int64_t>(p);
 }
 
 // ---------------------------------------------------------------------------
