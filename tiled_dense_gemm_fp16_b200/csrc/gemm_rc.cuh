@@ -513,14 +513,12 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
                                                    (((lane & 7) ^ (rw & 7)) << 4));
     const bool stores = lane < chunks;
     if constexpr (B_DEEP) {
-      // Two k-blocks in flight: two register sets of 8 rows (tiles
-      // narrower than 256 columns, so lane 31 never needs a 33rd block).
-      const bool extra = !B_DEEP && lane == 31 && chunks == 32;  // block 32 of the piece
-      // Row registers: one k-block plus lane 31's 33rd blocks, or (B_DEEP,
-      // at most 31 chunks, so block 32 is never needed) two k-blocks.
-      constexpr int kSets = B_DEEP ? 2 : 1;
-      uint4 rows[kSets][kRows], ext[kRows];
-      uint32_t f_row[kSets] = {};  // the rows' offset past their first aligned block
+      // Two k-blocks in flight: two register sets of 8 rows.  Tiles are
+      // narrower than 256 columns (at most 31 chunks per row), so no lane
+      // needs a 33rd block and the registers that hold it in the one-block
+      // loop below hold the second set here.
+      uint4 rows[2][kRows];
+      uint32_t f_row[2] = {};  // the rows' offset past their first aligned block
       // The k-blocks this CTA walks, in the order every role walks them: `ld`
       // is the next one to load, `pr` the next one to realign.
       struct Walk {
@@ -560,28 +558,24 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
         const uintptr_t a0 = start & ~uintptr_t(15);
         const uintptr_t blk = a0 + 16u * static_cast<uintptr_t>(lane);
         const bool lane_ok = lane <= chunks && blk < row0 + n_bytes;
-        const bool ext_ok = extra && a0 + 512u < row0 + n_bytes;
         f = static_cast<uint32_t>((start >> 1) & 7u);
-  #pragma unroll
+#pragma unroll
         for (int m = 0; m < kRows; ++m) {
           const bool in = static_cast<unsigned>(k0 + 8 * m) < static_cast<unsigned>(p.K);
           cur[m] = make_uint4(0u, 0u, 0u, 0u);
           ld_nc_v4_pred(cur[m], reinterpret_cast<const void*>(blk + m * stride), in && lane_ok);
-          if (!B_DEEP) {
-            ext[m] = make_uint4(0u, 0u, 0u, 0u);
-            ld_nc_v4_pred(ext[m], reinterpret_cast<const void*>(a0 + 512u + m * stride), in && ext_ok);
-          }
         }
         advance(ld);
       };
-  #pragma unroll
-      for (int i = 0; i < kSets; ++i)
-        if (ld.valid) load_rows(rows[i], f_row[i]);
+      if (ld.valid) load_rows(rows[0], f_row[0]);
+      if (ld.valid) load_rows(rows[1], f_row[1]);
       int r = 0;
       uint32_t rph = 0;
       bool ok = true;
       // Realign k-block `pr` from one register set, then refill that set with
-      // the next k-block still to load.
+      // the next k-block still to load.  Lane 31's output chunk is never
+      // stored (chunks <= 31), so its shuffle partner may be any value: the
+      // set itself stands in for the 33rd block.
       auto step = [&](uint4 (&cur)[kRows], uint32_t& f) {
         if (!mbar_wait(&empty_bar[r], rph ^ 1u, abort_flag, p.wait_budget_ns, 0x6B)) ok = false;
         if (!__all_sync(0xffffffffu, ok)) {
@@ -591,12 +585,11 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
         // Rows outside [0, K) were loaded as zeros and shift to zeros.
         const uint32_t dst = smem_u32(ring + r * p.ring_stage_bytes) + p.msub * Cfg::A_BYTES + dst_off;
         const uint32_t bits = (f & 1u) * 16u;
-        const uint4 (&e)[kRows] = B_DEEP ? cur : ext;  // lane 31's block 32 only when !B_DEEP
         switch (f >> 1) {
-          case 0: rc_shift_rows<0>(cur, e, bits, dst, stores, extra); break;
-          case 1: rc_shift_rows<1>(cur, e, bits, dst, stores, extra); break;
-          case 2: rc_shift_rows<2>(cur, e, bits, dst, stores, extra); break;
-          default: rc_shift_rows<3>(cur, e, bits, dst, stores, extra); break;
+          case 0: rc_shift_rows<0>(cur, cur, bits, dst, stores, false); break;
+          case 1: rc_shift_rows<1>(cur, cur, bits, dst, stores, false); break;
+          case 2: rc_shift_rows<2>(cur, cur, bits, dst, stores, false); break;
+          default: rc_shift_rows<3>(cur, cur, bits, dst, stores, false); break;
         }
         if (ld.valid) load_rows(cur, f);
         fence_proxy_async_smem();
@@ -610,7 +603,7 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
       };
       while (pr.valid && ok) {
         step(rows[0], f_row[0]);
-        if (B_DEEP && pr.valid && ok) step(rows[kSets - 1], f_row[kSets - 1]);
+        if (pr.valid && ok) step(rows[1], f_row[1]);
       }
     } else {
       const bool extra = lane == 31 && chunks == 32;  // block 32 of the piece
@@ -640,7 +633,7 @@ __global__ void __launch_bounds__(RcCfg<REALIGN_B>::THREADS, 1)
         const bool lane_ok = lane <= chunks && blk < row0 + n_bytes;
         const bool ext_ok = extra && a0 + 512u < row0 + n_bytes;
         f_next = static_cast<uint32_t>((start >> 1) & 7u);
-  #pragma unroll
+#pragma unroll
         for (int m = 0; m < kRows; ++m) {
           const bool in = static_cast<unsigned>(k0 + 8 * m) < static_cast<unsigned>(p.K);
           cur[m] = make_uint4(0u, 0u, 0u, 0u);
